@@ -1,0 +1,344 @@
+#!/usr/bin/env python3
+"""Benchmark of the Gated DeltaNet layer on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+
+One step = one chunked prefill of the Qwen3-Next layer workload (B=1, T=8192, 16 QK /
+32 V heads, d=128, bf16 I/O, fp32 state) through the C ABI.  The decode step (256
+sequences, fp32 state, 1 token and a 4-token verify) is measured alongside and
+reported under "decode".  Inputs are seeded synthetic tensors resident in HBM; L2 is
+flushed (a 256 MiB write) between timed steps, outside the timed events.
+
+Multi-GPU: every rank runs an independent replica of the same workload (the layer
+shards by sequence and head with no exchange); value = all ranks' tokens / the
+slowest rank's time ("scaling": "weak").
+
+--impl reference times the fp64 CPU oracle (the only reference this layer has) on a
+bounded sample of the same workload, on this host's cores, and prints the same line
+with "impl": "reference".
+"""
+
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "GDN prefill tokens/s (% BF16 tensor peak); decode tokens/s (% HBM GB/s)"
+UNIT = "tokens/s"
+WORKLOAD = "layer_prefill"
+HK, HV, D, C = 16, 32, 128, 64
+
+# Algorithmic work per token of prefill (GEMM flops of the chunked form) and bytes.
+PREFILL_FLOP_PER_TOKEN = HV * (3 * 2 * C * D + 3 * 2 * D * D) + HK * (2 * 2 * C * D)  # 5,242,880
+PREFILL_BYTES_PER_TOKEN = 2 * HK * D * 2 + HV * D * 2 * 2 + HV * 4 * 2                # 24,832
+STATE_BYTES = HV * D * D * 4                                                          # per sequence
+
+
+def decode_bytes(num_seqs, ntok):
+    """State read + write, q, k, v, out and gates for one decode step."""
+    return num_seqs * (STATE_BYTES * 2 + ntok * PREFILL_BYTES_PER_TOKEN)
+
+
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            p = json.load(f)
+        return dict(hbm_gbs=float(p["hbm_gbs"]), bf16_tflops=float(p["bf16_tflops"]),
+                    bf16_tflops_sustained=float(p.get("bf16_tflops_sustained", p["bf16_tflops"])),
+                    source="measured")
+    except (OSError, KeyError, ValueError):
+        return dict(hbm_gbs=6650.0, bf16_tflops=1590.0, bf16_tflops_sustained=1400.0,
+                    source="fallback")
+
+
+# ---------------------------------------------------------------- clocks sampling
+class ClockSampler:
+    QUERY = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+             "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+             "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index):
+        self.gpu = gpu_index
+        self.proc = None
+        self.path = None
+
+    def __enter__(self):
+        fd, self.path = tempfile.mkstemp(prefix="clocks_", suffix=".csv")
+        os.close(fd)
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.gpu), "--query-gpu=" + self.QUERY,
+                 "--format=csv,noheader,nounits", "-lms", "100"],
+                stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
+            time.sleep(0.3)
+        except OSError:
+            self.proc = None
+        return self
+
+    def __exit__(self, *exc):
+        if self.proc is not None:
+            time.sleep(0.2)
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+
+    def summary(self):
+        if not self.path or not os.path.exists(self.path):
+            return None
+        rows = []
+        for line in open(self.path):
+            parts = [p.strip() for p in line.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                rows.append(dict(sm=float(parts[1]), smax=float(parts[2]),
+                                 hw=parts[5], hwt=parts[6], swt=parts[7], swp=parts[8]))
+            except ValueError:
+                continue
+        os.unlink(self.path)
+        if not rows:
+            return None
+        reasons = set()
+        for r in rows:
+            for key, name in (("hw", "hw_slowdown"), ("hwt", "hw_thermal_slowdown"),
+                              ("swt", "sw_thermal_slowdown"), ("swp", "sw_power_cap")):
+                if r[key].lower() == "active":
+                    reasons.add(name)
+        return {"sm_mhz": statistics.median(r["sm"] for r in rows),
+                "sm_max_mhz": max(r["smax"] for r in rows),
+                "reasons": sorted(reasons), "samples": len(rows)}
+
+
+# ---------------------------------------------------------------- reference arm
+def oracle_tokens_per_s(x, heads_sample, threads=None):
+    """Times the fp64 oracle on `heads_sample` QK heads of workload x and scales to the
+    whole workload's tokens/s (heads are independent, so cost is linear in heads)."""
+    import oracle
+    T = x["q"].shape[0]
+    hk = x["q"].shape[1]
+    t0 = time.perf_counter()
+    oracle.forward_heads(x["q"], x["k"], x["v"], x["g"], x["beta"], x["cu_seqlens"],
+                         list(range(heads_sample)), threads=threads)
+    dt = time.perf_counter() - t0
+    return T / (dt * hk / heads_sample), dt
+
+
+def reference_arm(args, rank, world):
+    if rank != 0:
+        return 0
+    import oracle
+    from linear_attention_layer_gated_b200 import inputs
+    x = inputs.make(inputs.workload(WORKLOAD), device="cpu")
+    cores = oracle.host_threads()
+    heads_sample = HK
+    vals = []
+    for _ in range(max(args.warmup, 0)):
+        oracle_tokens_per_s(x, heads_sample)
+    for _ in range(args.steps):
+        v, dt = oracle_tokens_per_s(x, heads_sample)
+        vals.append(v)
+    value = statistics.mean(vals)
+    T = x["q"].shape[0]
+    sample = ("fp64 oracle (token recurrence, C, %d threads) on the whole T=%d, 16/32-head "
+              "workload, one pass per step" % (cores, T))
+    line = {"impl": "reference", "metric": METRIC, "value": value, "unit": UNIT,
+            "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": T / value * 1e3, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": {"workload": "layer_prefill: B=1, T=8192, 16 QK / 32 V heads, d=128",
+                       "sample": "whole workload"},
+            "cpu_baseline": {"kind": "oracle", "value": value, "unit": UNIT, "cores": cores,
+                             "sample": sample},
+            "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+            "gpu_launches": 0}
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+# ---------------------------------------------------------------- our arm
+def main_ours(args, rank, world, local_rank):
+    import torch
+    import torch.distributed as dist
+    from linear_attention_layer_gated_b200 import build, gdn, inputs
+
+    build.build()
+    torch.cuda.set_device(local_rank)
+    dev = torch.device("cuda", local_rank)
+    peaks = load_peaks()
+    stream = torch.cuda.current_stream(dev)
+    algo = {"auto": gdn.GDN_ALGO_AUTO, "simt": gdn.GDN_ALGO_SIMT,
+            "tensor": gdn.GDN_ALGO_TENSOR}[args.algo]
+
+    w = inputs.workload(WORKLOAD)
+    x = inputs.make(w, device=dev)
+    T = x["q"].shape[0]
+    out = torch.empty_like(x["v"])
+    fin = torch.empty((1, HV, D, D), dtype=torch.float32, device=dev)
+    shape = gdn.prefill_shape(x["q"], x["v"], x["cu_seqlens"], algo)
+    ws = gdn.alloc_workspace(shape, dev)
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+
+    def prefill_once():
+        gdn.gdn_chunk_prefill(x["q"], x["k"], x["v"], x["g"], x["beta"], None, x["cu_seqlens"],
+                              out, fin, workspace=ws, algo=algo, stream=stream)
+
+    def barrier():
+        if world > 1:
+            dist.barrier()
+        torch.cuda.synchronize(dev)
+
+    def timed(fn, steps, warmup, flush_between=True):
+        for _ in range(warmup):
+            fn()
+        ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+              for _ in range(steps)]
+        barrier()
+        for a, b in ev:
+            if flush_between:
+                flush.fill_(1)
+            a.record(stream)
+            fn()
+            b.record(stream)
+        barrier()
+        return [a.elapsed_time(b) for a, b in ev]
+
+    def max_over_ranks(v):
+        if world == 1:
+            return v
+        t = torch.tensor([v], dtype=torch.float64, device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        return float(t.item())
+
+    with ClockSampler(local_rank) as clk:
+        ms = timed(prefill_once, args.steps, args.warmup)
+    clocks = clk.summary()
+    ms_step = max_over_ranks(sum(ms) / len(ms))
+    value = world * T / (ms_step * 1e-3)
+
+    # ---- dominant kernel roofline (the prefill is one launch per step on this path)
+    launches_per_step = gdn_launches_per_prefill(algo, x["q"].dtype)
+    flop = PREFILL_FLOP_PER_TOKEN * T
+    achieved_tflops = flop / (ms_step * 1e-3) / 1e12
+    peak = peaks["bf16_tflops"]
+    roofline = {"bound": "tensor", "achieved": achieved_tflops, "peak": peak, "unit": "TFLOP/s",
+                "frac": achieved_tflops / peak, "traffic": None,
+                "peak_source": peaks["source"] + " bf16 dense (burst)",
+                "kernel": "gdn prefill step (all launches)",
+                "algorithmic_flop_per_launch": flop}
+
+    # ---- end to end through the C ABI with pinned host buffers
+    host = {k2: x[k2].cpu().pin_memory() for k2 in ("q", "k", "v", "g", "beta", "cu_seqlens")}
+    dbuf = {k2: torch.empty_like(x[k2]) for k2 in host}
+    hout = torch.empty(out.shape, dtype=out.dtype).pin_memory()
+
+    def e2e_once():
+        for k2 in host:
+            dbuf[k2].copy_(host[k2], non_blocking=True)
+        gdn.gdn_chunk_prefill(dbuf["q"], dbuf["k"], dbuf["v"], dbuf["g"], dbuf["beta"], None,
+                              dbuf["cu_seqlens"], out, fin, workspace=ws, algo=algo, stream=stream)
+        hout.copy_(out, non_blocking=True)
+
+    e2e_ms = timed(e2e_once, max(3, args.steps // 2), 2)
+    e2e_step = max_over_ranks(sum(e2e_ms) / len(e2e_ms))
+    h2d = sum(t.numel() * t.element_size() for t in host.values())
+    d2h = hout.numel() * hout.element_size()
+
+    # ---- decode: 256 sequences, 1 token and 4-token verify
+    dec = {}
+    for ntok in (1, 4):
+        d = inputs.make_decode(256, ntok, seed=3, device=dev)
+        dout = torch.empty_like(d["v"])
+
+        def dec_once():
+            gdn.gdn_decode_step(d["q"], d["k"], d["v"], d["g"], d["beta"], d["state"], dout,
+                                stream=stream)
+
+        dms = timed(dec_once, max(args.steps, 10), args.warmup)
+        dstep = max_over_ranks(sum(dms) / len(dms))
+        nbytes = decode_bytes(256, ntok)
+        gbs = nbytes / (dstep * 1e-3) / 1e9
+        dec["ntok%d" % ntok] = {
+            "tokens_per_s": world * 256 * ntok / (dstep * 1e-3), "ms_per_step": dstep,
+            "roofline": {"bound": "hbm", "achieved": gbs, "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                         "frac": gbs / peaks["hbm_gbs"], "frac_of_8TBs": gbs / 8000.0,
+                         "traffic": None, "algorithmic_bytes_per_launch": nbytes}}
+
+    # ---- CPU baseline: the oracle on a bounded sample (rank 0, N=1 only)
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        import oracle
+        xs = {k2: (x[k2].cpu() if hasattr(x[k2], "cpu") else x[k2]) for k2 in x}
+        v_cpu, dt = oracle_tokens_per_s(xs, HK)
+        cpu = {"value": v_cpu, "unit": UNIT, "cores": oracle.host_threads(), "kind": "oracle",
+               "sample": "fp64 oracle (token recurrence) on the whole T=8192, 16/32-head "
+                         "workload, one pass, %.1f s" % dt}
+
+    if rank == 0:
+        line = {"metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world,
+                "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_step,
+                "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+                "dtype": "bf16", "data": "synthetic",
+                "config": {"workload": "layer_prefill: B=1, T=8192, 16 QK / 32 V heads, d=128, "
+                                       "bf16 I/O, fp32 state, chunk 64",
+                           "parallelism": "replicas" if world > 1 else "single",
+                           "l2": "flushed between timed steps (256 MiB write)",
+                           "algo": args.algo},
+                "roofline": roofline, "cpu_baseline": cpu,
+                "e2e": {"value": world * T / (e2e_step * 1e-3), "unit": UNIT,
+                        "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
+                "gpu_launches": launches_per_step * args.steps,
+                "decode": dec, "clocks": clocks, "peaks": peaks}
+        print(json.dumps(line), flush=True)
+    return 0
+
+
+def gdn_launches_per_prefill(algo, dtype):
+    """Kernels libgdn.so launches per gdn_chunk_prefill call on the chosen path."""
+    return 1
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--algo", default="auto", choices=["auto", "simt", "tensor"])
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    if args.warmup < 3 and args.impl == "ours":
+        args.warmup = 3
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+    if args.impl == "reference":
+        return reference_arm(args, rank, world)
+    if world > 1:
+        import datetime
+        import torch
+        import torch.distributed as dist
+        torch.cuda.set_device(local_rank)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local_rank))
+    try:
+        return main_ours(args, rank, world, local_rank)
+    finally:
+        if world > 1:
+            import torch.distributed as dist
+            dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    sys.exit(main())

@@ -1,0 +1,159 @@
+/*
+ * gdn.h -- C ABI of libgdn.so, the B200 (sm_100a) Gated DeltaNet layer.
+ *
+ * The layer.  Gated DeltaNet is the linear-attention layer of Qwen3-Next
+ * (Qwen3-Next-80B-A3B model card, "Highlights": Hybrid Attention; "Model Overview":
+ * Gated DeltaNet with 32 linear-attention heads for V and 16 for QK, head dimension
+ * 128; the layout puts it in 36 of the 48 layers).  Per sequence and per V head h it
+ * keeps a fixed-size fp32 state S (d_v x d_k = 128 x 128) and applies the gated delta
+ * rule to every token:
+ *
+ *     S_t = exp(g_t) * S_{t-1} * (I - beta_t k_t k_t^T) + beta_t v_t k_t^T
+ *     o_t = S_t q_t
+ *
+ * where k_t = k / sqrt(|k|^2 + 1e-6), q_t = q / sqrt(|q|^2 + 1e-6) / sqrt(128)
+ * (normalisation and scaling happen inside the library: pass raw q and k), g_t <= 0
+ * and 0 < beta_t < 1 (already activated gates; documented preconditions, not checked
+ * on the device).  V head h reads QK head h / (num_v_heads / num_qk_heads), i.e. V
+ * heads 2j and 2j+1 share QK head j in the 16/32 layout.
+ *
+ * Layouts (all contiguous, row-major, token-major; T = total packed tokens,
+ * N = num_seqs, HK = num_qk_heads, HV = num_v_heads, D = head_dim = 128):
+ *   q, k          [T][HK][D]   io dtype (bf16 or fp32)
+ *   v, out        [T][HV][D]   io dtype
+ *   g, beta       [T][HV]      fp32
+ *   states        [N][HV][D][D] fp32, S[n][h][i][j] with i the d_v (row) index
+ *   cu_seqlens    [N+1] int32, DEVICE memory, cu_seqlens[0] = 0, non-decreasing,
+ *                 cu_seqlens[N] = T; sequence n owns tokens [cu[n], cu[n+1]).
+ * For decode the token axis is [N][num_tokens] flattened (sequence-major).
+ *
+ * Ownership and behaviour common to all entry points:
+ *   - Every pointer except `shape` is a device pointer owned by the caller; the
+ *     library never allocates, frees, synchronises or reads device memory on the
+ *     host inside gdn_chunk_prefill / gdn_decode_step.  Work is enqueued on `stream`
+ *     (a cudaStream_t passed as void*; NULL = legacy default stream).  Both calls are
+ *     therefore stream-ordered and can be captured into CUDA graphs.
+ *   - Device pointers must be 16-byte aligned (GDN_ERR_ALIGN otherwise).
+ *   - The return value reports host-side validation and launch errors only.  Device
+ *     side faults surface through the CUDA runtime (GDN_ERR_CUDA from a later call or
+ *     cudaStreamSynchronize); a bounded device wait that gave up is recorded in the
+ *     workspace and read back by gdn_get_device_error.
+ *   - `out` must not alias any input.  initial_state and final_state may alias each
+ *     other (in-place state carry).
+ */
+#ifndef GDN_H
+#define GDN_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#define GDN_ABI_VERSION 1
+
+typedef enum {
+    GDN_OK = 0,
+    GDN_ERR_NULL = 1,           /* a required pointer is NULL */
+    GDN_ERR_SHAPE = 2,          /* unsupported or inconsistent sizes */
+    GDN_ERR_ALIGN = 3,          /* a device pointer is not 16-byte aligned */
+    GDN_ERR_DTYPE = 4,          /* io_dtype not one of gdn_dtype */
+    GDN_ERR_NUM_TOKENS = 5,     /* decode num_tokens outside [1, 4] */
+    GDN_ERR_WORKSPACE = 6,      /* workspace missing or smaller than required */
+    GDN_ERR_CUDA = 7,           /* the CUDA runtime reported an error */
+    GDN_ERR_DEVICE_TIMEOUT = 8, /* a bounded device-side wait expired */
+    GDN_ERR_UNSUPPORTED = 9     /* requested algorithm not available for these inputs */
+} gdn_status;
+
+typedef enum { GDN_BF16 = 0, GDN_F32 = 1 } gdn_dtype;
+
+/* Prefill algorithm selection (gdn_shape.algo). */
+typedef enum {
+    GDN_ALGO_AUTO = 0,          /* tensor-core path for bf16 I/O, SIMT fp32 path for fp32 I/O */
+    GDN_ALGO_SIMT = 1,          /* chunked form on CUDA cores in fp32 (any io dtype) */
+    GDN_ALGO_TENSOR = 2         /* chunked form on tcgen05 tensor cores (bf16 I/O only) */
+} gdn_algo;
+
+typedef struct {
+    int32_t num_seqs;      /* N >= 0 (prefill: sequences; decode: batch) */
+    int32_t total_tokens;  /* T >= 0 (prefill only; decode ignores it) */
+    int32_t max_seqlen;    /* optional hint, 0 = unknown; if > 0 must be <= total_tokens */
+    int32_t num_qk_heads;  /* HK >= 1 */
+    int32_t num_v_heads;   /* HV, a multiple of HK */
+    int32_t head_dim;      /* must be 128 (d_k = d_v) */
+    int32_t io_dtype;      /* gdn_dtype of q, k, v, out */
+    int32_t algo;          /* gdn_algo (prefill only) */
+} gdn_shape;
+
+/*
+ * Workspace the caller must provide to gdn_chunk_prefill for `shape` (bytes, a
+ * multiple of 256).  It depends on total_tokens, num_seqs, the head counts and the
+ * algorithm.  Returns 0 if the shape is invalid.
+ */
+size_t gdn_prefill_workspace_bytes(const gdn_shape *shape);
+
+/*
+ * Chunked prefill over a packed varlen batch.  The chunked form of the gated delta
+ * rule processes each sequence in chunks of 64 tokens: per chunk it builds the
+ * cumulative-gate-weighted intra-chunk UT representation (the unit lower-triangular
+ * system I + strictly_lower(beta * K K^T * decay)), applies it to the entering state
+ * and carries the fp32 state to the next chunk.  Chunks restart at each sequence
+ * start; the last chunk of a sequence may be partial; empty sequences are allowed
+ * (their final state equals their initial state).
+ *
+ *   q, k, v, g, beta   inputs, layouts above
+ *   initial_state      [N][HV][D][D] fp32, or NULL for zero states
+ *   cu_seqlens         [N+1] int32 device array
+ *   out                [T][HV][D] written for every token
+ *   final_state        [N][HV][D][D] fp32, or NULL (not written); may alias initial_state
+ *   shape              host pointer
+ *   workspace          device scratch of >= gdn_prefill_workspace_bytes(shape) bytes,
+ *                      256-byte aligned; its contents on entry do not matter; it must
+ *                      not be shared by calls that overlap on the device
+ *   stream             cudaStream_t
+ */
+gdn_status gdn_chunk_prefill(const void *q, const void *k, const void *v,
+                             const float *g, const float *beta,
+                             const float *initial_state, const int32_t *cu_seqlens,
+                             void *out, float *final_state, const gdn_shape *shape,
+                             void *workspace, size_t workspace_bytes, void *stream);
+
+/*
+ * Decode / multi-token verify step: advances every sequence's state by num_tokens
+ * (1..4) tokens in place and writes the output of every token.  This is the memory
+ * bound step a speculative-decoding verifier uses (the pages' multi-token prediction
+ * serving, up to 4 draft tokens).
+ *
+ *   q, k            [N][num_tokens][HK][D] io dtype (raw; normalised inside)
+ *   v               [N][num_tokens][HV][D] io dtype
+ *   g, beta         [N][num_tokens][HV] fp32
+ *   state_inout     [N][HV][D][D] fp32, read and overwritten with the state after
+ *                   the last token
+ *   out             [N][num_tokens][HV][D] io dtype
+ *   num_tokens      1..4, the same for every sequence (GDN_ERR_NUM_TOKENS otherwise)
+ *   shape           uses num_seqs, num_qk_heads, num_v_heads, head_dim, io_dtype
+ */
+gdn_status gdn_decode_step(const void *q, const void *k, const void *v,
+                           const float *g, const float *beta, float *state_inout,
+                           void *out, int32_t num_tokens, const gdn_shape *shape,
+                           void *stream);
+
+/*
+ * Reads the device error word of a prefill workspace (synchronises `stream`; meant for
+ * tests and debugging).  Returns GDN_ERR_DEVICE_TIMEOUT if a bounded device wait of a
+ * previous prefill gave up, GDN_ERR_CUDA if the runtime reports an error, else GDN_OK.
+ */
+gdn_status gdn_get_device_error(void *workspace, void *stream);
+
+/* Static, human-readable name of a status code. */
+const char *gdn_status_string(gdn_status status);
+
+/* GDN_ABI_VERSION of the loaded library. */
+int32_t gdn_abi_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* GDN_H */

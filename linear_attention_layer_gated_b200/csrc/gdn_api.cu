@@ -1,0 +1,121 @@
+// gdn_api.cu -- C ABI of libgdn.so: argument validation, workspace sizing and kernel
+// dispatch on the caller's stream.  Declarations and contracts are in include/gdn.h.
+//
+// Nothing here allocates, synchronises or reads device memory inside the prefill and
+// decode entry points, so both are stream-ordered and graph-capturable; the only
+// device-side work besides kernels is a 256-byte memset of the workspace header.
+#include <cstdint>
+#include <cstring>
+
+#include "gdn_internal.cuh"
+
+namespace {
+
+constexpr size_t kHeaderBytes = 256;  // workspace header: device error word + reserved
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+gdn_status check_common(const gdn_shape* s) {
+    if (!s) return GDN_ERR_NULL;
+    if (s->io_dtype != GDN_BF16 && s->io_dtype != GDN_F32) return GDN_ERR_DTYPE;
+    if (s->head_dim != gdn::kD) return GDN_ERR_SHAPE;
+    if (s->num_seqs < 0 || s->num_qk_heads < 1 || s->num_v_heads < 1) return GDN_ERR_SHAPE;
+    if (s->num_v_heads % s->num_qk_heads != 0) return GDN_ERR_SHAPE;
+    if (s->num_v_heads > 4096) return GDN_ERR_SHAPE;
+    return GDN_OK;
+}
+
+gdn_status check_prefill_shape(const gdn_shape* s) {
+    gdn_status st = check_common(s);
+    if (st != GDN_OK) return st;
+    if (s->total_tokens < 0 || s->max_seqlen < 0 || s->max_seqlen > s->total_tokens) return GDN_ERR_SHAPE;
+    if (s->algo != GDN_ALGO_AUTO && s->algo != GDN_ALGO_SIMT && s->algo != GDN_ALGO_TENSOR) return GDN_ERR_SHAPE;
+    if ((int64_t)s->num_seqs * s->num_v_heads * 4 > INT32_MAX) return GDN_ERR_SHAPE;
+    return GDN_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+int32_t gdn_abi_version(void) { return GDN_ABI_VERSION; }
+
+const char* gdn_status_string(gdn_status status) {
+    switch (status) {
+    case GDN_OK: return "GDN_OK";
+    case GDN_ERR_NULL: return "GDN_ERR_NULL: a required pointer is NULL";
+    case GDN_ERR_SHAPE: return "GDN_ERR_SHAPE: unsupported or inconsistent sizes";
+    case GDN_ERR_ALIGN: return "GDN_ERR_ALIGN: device pointer not 16-byte aligned";
+    case GDN_ERR_DTYPE: return "GDN_ERR_DTYPE: io_dtype must be GDN_BF16 or GDN_F32";
+    case GDN_ERR_NUM_TOKENS: return "GDN_ERR_NUM_TOKENS: decode num_tokens must be in [1, 4]";
+    case GDN_ERR_WORKSPACE: return "GDN_ERR_WORKSPACE: workspace missing or too small";
+    case GDN_ERR_CUDA: return "GDN_ERR_CUDA: CUDA runtime error";
+    case GDN_ERR_DEVICE_TIMEOUT: return "GDN_ERR_DEVICE_TIMEOUT: a bounded device wait expired";
+    case GDN_ERR_UNSUPPORTED: return "GDN_ERR_UNSUPPORTED: algorithm not available for these inputs";
+    }
+    return "unknown gdn_status";
+}
+
+size_t gdn_prefill_workspace_bytes(const gdn_shape* shape) {
+    if (check_prefill_shape(shape) != GDN_OK) return 0;
+    return kHeaderBytes;
+}
+
+gdn_status gdn_chunk_prefill(const void* q, const void* k, const void* v, const float* g,
+                             const float* beta, const float* initial_state,
+                             const int32_t* cu_seqlens, void* out, float* final_state,
+                             const gdn_shape* shape, void* workspace, size_t workspace_bytes,
+                             void* stream) {
+    gdn_status st = check_prefill_shape(shape);
+    if (st != GDN_OK) return st;
+    const size_t need = gdn_prefill_workspace_bytes(shape);
+    if (!workspace || workspace_bytes < need) return GDN_ERR_WORKSPACE;
+    if ((reinterpret_cast<uintptr_t>(workspace) & 255u) != 0) return GDN_ERR_ALIGN;
+    if (shape->num_seqs == 0) return GDN_OK;
+    if (!cu_seqlens) return GDN_ERR_NULL;
+    if (shape->total_tokens > 0 && (!q || !k || !v || !g || !beta || !out)) return GDN_ERR_NULL;
+    const void* ptrs[] = {q, k, v, g, beta, initial_state, cu_seqlens, out, final_state};
+    for (const void* p : ptrs)
+        if (p && !aligned16(p)) return GDN_ERR_ALIGN;
+
+    gdn_dtype io = (gdn_dtype)shape->io_dtype;
+    int algo = shape->algo;
+    if (algo == GDN_ALGO_TENSOR) return GDN_ERR_UNSUPPORTED;
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    if (cudaMemsetAsync(workspace, 0, kHeaderBytes, s) != cudaSuccess) return GDN_ERR_CUDA;
+    cudaError_t e = gdn::launch_prefill_simt(q, k, v, g, beta, initial_state, cu_seqlens, out,
+                                             final_state, shape->num_seqs, shape->num_qk_heads,
+                                             shape->num_v_heads, io, s);
+    return e == cudaSuccess ? GDN_OK : GDN_ERR_CUDA;
+}
+
+gdn_status gdn_decode_step(const void* q, const void* k, const void* v, const float* g,
+                           const float* beta, float* state_inout, void* out, int32_t num_tokens,
+                           const gdn_shape* shape, void* stream) {
+    gdn_status st = check_common(shape);
+    if (st != GDN_OK) return st;
+    if (num_tokens < 1 || num_tokens > 4) return GDN_ERR_NUM_TOKENS;
+    if ((int64_t)shape->num_seqs * shape->num_v_heads > INT32_MAX) return GDN_ERR_SHAPE;
+    if (shape->num_seqs == 0) return GDN_OK;
+    if (!q || !k || !v || !g || !beta || !state_inout || !out) return GDN_ERR_NULL;
+    const void* ptrs[] = {q, k, v, g, beta, state_inout, out};
+    for (const void* p : ptrs)
+        if (!aligned16(p)) return GDN_ERR_ALIGN;
+    cudaError_t e = gdn::launch_decode(q, k, v, g, beta, state_inout, out, num_tokens,
+                                       shape->num_seqs, shape->num_qk_heads, shape->num_v_heads,
+                                       (gdn_dtype)shape->io_dtype,
+                                       reinterpret_cast<cudaStream_t>(stream));
+    return e == cudaSuccess ? GDN_OK : GDN_ERR_CUDA;
+}
+
+gdn_status gdn_get_device_error(void* workspace, void* stream) {
+    if (!workspace) return GDN_ERR_NULL;
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    if (cudaStreamSynchronize(s) != cudaSuccess) return GDN_ERR_CUDA;
+    int32_t word = 0;
+    if (cudaMemcpy(&word, workspace, sizeof(word), cudaMemcpyDeviceToHost) != cudaSuccess)
+        return GDN_ERR_CUDA;
+    return word != 0 ? GDN_ERR_DEVICE_TIMEOUT : GDN_OK;
+}
+
+}  // extern "C"

@@ -1,0 +1,58 @@
+// gdn_internal.cuh -- shared device helpers and internal launcher declarations of
+// libgdn.so.  Not part of the public ABI (that is include/gdn.h).
+#pragma once
+
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "../../include/gdn.h"
+
+namespace gdn {
+
+constexpr int kD = 128;       // head dimension (d_k = d_v), Qwen3-Next model card "Model Overview"
+constexpr int kChunk = 64;    // tokens per chunk of the chunked form
+constexpr float kNormEps = 1e-6f;  // x / sqrt(sum(x^2) + eps)
+
+// ---------------------------------------------------------------- conversions
+__device__ __forceinline__ float to_f32(float x) { return x; }
+__device__ __forceinline__ float to_f32(__nv_bfloat16 x) { return __bfloat162float(x); }
+
+template <typename T> __device__ __forceinline__ T from_f32(float x);
+template <> __device__ __forceinline__ float from_f32<float>(float x) { return x; }
+template <> __device__ __forceinline__ __nv_bfloat16 from_f32<__nv_bfloat16>(float x) {
+    return __float2bfloat16_rn(x);
+}
+
+// Loads 4 consecutive elements (16-byte aligned for fp32, 8-byte for bf16) as fp32.
+__device__ __forceinline__ float4 load4(const float* p) { return *reinterpret_cast<const float4*>(p); }
+__device__ __forceinline__ float4 load4(const __nv_bfloat16* p) {
+    uint2 u = *reinterpret_cast<const uint2*>(p);
+    __nv_bfloat162 a = *reinterpret_cast<__nv_bfloat162*>(&u.x);
+    __nv_bfloat162 b = *reinterpret_cast<__nv_bfloat162*>(&u.y);
+    float2 fa = __bfloat1622float2(a), fb = __bfloat1622float2(b);
+    return make_float4(fa.x, fa.y, fb.x, fb.y);
+}
+
+__device__ __forceinline__ void store4(float* p, float4 v) { *reinterpret_cast<float4*>(p) = v; }
+__device__ __forceinline__ void store4(__nv_bfloat16* p, float4 v) {
+    __nv_bfloat162 a = __floats2bfloat162_rn(v.x, v.y);
+    __nv_bfloat162 b = __floats2bfloat162_rn(v.z, v.w);
+    uint2 u;
+    u.x = *reinterpret_cast<uint32_t*>(&a);
+    u.y = *reinterpret_cast<uint32_t*>(&b);
+    *reinterpret_cast<uint2*>(p) = u;
+}
+
+// ---------------------------------------------------------------- launchers
+// Each returns cudaSuccess or the launch error; arguments were validated by the caller.
+cudaError_t launch_decode(const void* q, const void* k, const void* v, const float* g,
+                          const float* beta, float* state, void* out, int num_tokens,
+                          int num_seqs, int hk, int hv, gdn_dtype io, cudaStream_t stream);
+
+cudaError_t launch_prefill_simt(const void* q, const void* k, const void* v, const float* g,
+                                const float* beta, const float* s0, const int32_t* cu,
+                                void* out, float* sT, int num_seqs, int hk, int hv,
+                                gdn_dtype io, cudaStream_t stream);
+
+}  // namespace gdn

@@ -1,0 +1,188 @@
+"""ctypes binding of libgdn.so (C ABI in include/gdn.h) -- argument marshalling only.
+
+The functions carry the C entry points' names.  Tensors are torch CUDA tensors used
+purely as device memory; every step of the layer runs in the library's kernels.
+There is no CPU fallback: if the library is missing or a call fails, these raise.
+"""
+
+from __future__ import annotations
+
+import ctypes
+import os
+import threading
+
+import torch
+
+HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(HERE, "libgdn.so")
+
+GDN_OK = 0
+GDN_BF16, GDN_F32 = 0, 1
+GDN_ALGO_AUTO, GDN_ALGO_SIMT, GDN_ALGO_TENSOR = 0, 1, 2
+STATUS = {0: "GDN_OK", 1: "GDN_ERR_NULL", 2: "GDN_ERR_SHAPE", 3: "GDN_ERR_ALIGN",
+          4: "GDN_ERR_DTYPE", 5: "GDN_ERR_NUM_TOKENS", 6: "GDN_ERR_WORKSPACE",
+          7: "GDN_ERR_CUDA", 8: "GDN_ERR_DEVICE_TIMEOUT", 9: "GDN_ERR_UNSUPPORTED"}
+EXPORTED = ["gdn_prefill_workspace_bytes", "gdn_chunk_prefill", "gdn_decode_step",
+            "gdn_get_device_error", "gdn_status_string", "gdn_abi_version"]
+
+
+class GdnShape(ctypes.Structure):
+    _fields_ = [("num_seqs", ctypes.c_int32), ("total_tokens", ctypes.c_int32),
+                ("max_seqlen", ctypes.c_int32), ("num_qk_heads", ctypes.c_int32),
+                ("num_v_heads", ctypes.c_int32), ("head_dim", ctypes.c_int32),
+                ("io_dtype", ctypes.c_int32), ("algo", ctypes.c_int32)]
+
+
+class GdnError(RuntimeError):
+    def __init__(self, code: int, what: str):
+        super().__init__("%s failed: %s" % (what, gdn_status_string(code)))
+        self.code = code
+
+
+_lock = threading.Lock()
+_lib = None
+
+
+def lib() -> ctypes.CDLL:
+    """Loads libgdn.so (raises if it has not been built)."""
+    global _lib
+    with _lock:
+        if _lib is None:
+            if not os.path.exists(LIB_PATH):
+                raise RuntimeError("libgdn.so is missing at %s; build it with "
+                                   "`python -m linear_attention_layer_gated_b200.build`" % LIB_PATH)
+            L = ctypes.CDLL(LIB_PATH)
+            vp, fp, ip = ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p
+            sp = ctypes.POINTER(GdnShape)
+            L.gdn_prefill_workspace_bytes.restype = ctypes.c_size_t
+            L.gdn_prefill_workspace_bytes.argtypes = [sp]
+            L.gdn_chunk_prefill.restype = ctypes.c_int
+            L.gdn_chunk_prefill.argtypes = [vp, vp, vp, fp, fp, fp, ip, vp, fp, sp, vp,
+                                            ctypes.c_size_t, vp]
+            L.gdn_decode_step.restype = ctypes.c_int
+            L.gdn_decode_step.argtypes = [vp, vp, vp, fp, fp, fp, vp, ctypes.c_int32, sp, vp]
+            L.gdn_get_device_error.restype = ctypes.c_int
+            L.gdn_get_device_error.argtypes = [vp, vp]
+            L.gdn_status_string.restype = ctypes.c_char_p
+            L.gdn_status_string.argtypes = [ctypes.c_int]
+            L.gdn_abi_version.restype = ctypes.c_int32
+            L.gdn_abi_version.argtypes = []
+            _lib = L
+    return _lib
+
+
+def gdn_status_string(code: int) -> str:
+    return lib().gdn_status_string(int(code)).decode()
+
+
+def gdn_abi_version() -> int:
+    return int(lib().gdn_abi_version())
+
+
+def _io_dtype(t: torch.Tensor) -> int:
+    if t.dtype == torch.bfloat16:
+        return GDN_BF16
+    if t.dtype == torch.float32:
+        return GDN_F32
+    raise TypeError("q/k/v/out must be bfloat16 or float32, got %s" % t.dtype)
+
+
+def _ptr(t):
+    if t is None:
+        return None
+    if isinstance(t, int):
+        return t
+    if not t.is_cuda:
+        raise ValueError("expected a CUDA tensor")
+    if not t.is_contiguous():
+        raise ValueError("expected a contiguous tensor")
+    return t.data_ptr()
+
+
+def _stream(stream):
+    if stream is None:
+        return torch.cuda.current_stream().cuda_stream
+    if isinstance(stream, int):
+        return stream
+    return stream.cuda_stream
+
+
+def make_shape(num_seqs, total_tokens, num_qk_heads, num_v_heads, head_dim=128,
+               io_dtype=GDN_BF16, algo=GDN_ALGO_AUTO, max_seqlen=0) -> GdnShape:
+    return GdnShape(int(num_seqs), int(total_tokens), int(max_seqlen), int(num_qk_heads),
+                    int(num_v_heads), int(head_dim), int(io_dtype), int(algo))
+
+
+def gdn_prefill_workspace_bytes(shape: GdnShape) -> int:
+    return int(lib().gdn_prefill_workspace_bytes(ctypes.byref(shape)))
+
+
+def prefill_shape(q, v, cu_seqlens, algo=GDN_ALGO_AUTO, max_seqlen=0) -> GdnShape:
+    T, HK, D = q.shape
+    return make_shape(cu_seqlens.numel() - 1, T, HK, v.shape[1], D, _io_dtype(q), algo, max_seqlen)
+
+
+def alloc_workspace(shape: GdnShape, device) -> torch.Tensor:
+    n = gdn_prefill_workspace_bytes(shape)
+    if n == 0:
+        raise ValueError("invalid prefill shape")
+    return torch.empty(n, dtype=torch.uint8, device=device)
+
+
+def gdn_chunk_prefill(q, k, v, g, beta, initial_state, cu_seqlens, out, final_state,
+                      workspace=None, algo=GDN_ALGO_AUTO, max_seqlen=0, stream=None):
+    """Calls gdn_chunk_prefill.  Shapes: q, k [T, HK, 128]; v, out [T, HV, 128];
+    g, beta [T, HV] fp32; states [N, HV, 128, 128] fp32 or None; cu_seqlens [N+1] int32."""
+    if q.dtype != k.dtype or q.dtype != v.dtype or out.dtype != q.dtype:
+        raise TypeError("q, k, v and out must share one dtype")
+    if cu_seqlens.dtype != torch.int32:
+        raise TypeError("cu_seqlens must be int32")
+    shape = prefill_shape(q, v, cu_seqlens, algo, max_seqlen)
+    if workspace is None:
+        workspace = alloc_workspace(shape, q.device)
+    rc = lib().gdn_chunk_prefill(_ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(beta),
+                                 _ptr(initial_state), _ptr(cu_seqlens), _ptr(out),
+                                 _ptr(final_state), ctypes.byref(shape), _ptr(workspace),
+                                 workspace.numel(), _stream(stream))
+    if rc != GDN_OK:
+        raise GdnError(rc, "gdn_chunk_prefill")
+    return workspace
+
+
+def gdn_decode_step(q, k, v, g, beta, state_inout, out, num_tokens=None, stream=None):
+    """Calls gdn_decode_step.  Shapes: q, k [N, m, HK, 128]; v, out [N, m, HV, 128];
+    g, beta [N, m, HV] fp32; state_inout [N, HV, 128, 128] fp32 (updated in place)."""
+    N, m, HK, D = q.shape
+    if num_tokens is None:
+        num_tokens = m
+    shape = make_shape(N, N * m, HK, v.shape[2], D, _io_dtype(q))
+    rc = lib().gdn_decode_step(_ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(beta), _ptr(state_inout),
+                               _ptr(out), int(num_tokens), ctypes.byref(shape), _stream(stream))
+    if rc != GDN_OK:
+        raise GdnError(rc, "gdn_decode_step")
+
+
+def gdn_get_device_error(workspace, stream=None) -> int:
+    return int(lib().gdn_get_device_error(_ptr(workspace), _stream(stream)))
+
+
+# ------------------------------------------------------------------ conveniences
+def prefill(q, k, v, g, beta, cu_seqlens, initial_state=None, want_final_state=True,
+            algo=GDN_ALGO_AUTO, workspace=None, stream=None):
+    """Allocates out (and final_state) and runs gdn_chunk_prefill."""
+    out = torch.empty_like(v)
+    N = cu_seqlens.numel() - 1
+    fin = None
+    if want_final_state:
+        fin = torch.empty((N, v.shape[1], v.shape[2], v.shape[2]), dtype=torch.float32,
+                          device=v.device)
+    gdn_chunk_prefill(q, k, v, g, beta, initial_state, cu_seqlens, out, fin,
+                      workspace=workspace, algo=algo, stream=stream)
+    return out, fin
+
+
+def decode(q, k, v, g, beta, state_inout, stream=None):
+    """Allocates out and runs gdn_decode_step (state_inout is updated in place)."""
+    out = torch.empty_like(v)
+    gdn_decode_step(q, k, v, g, beta, state_inout, out, stream=stream)
+    return out

@@ -1,0 +1,127 @@
+"""C ABI checks that need no GPU: the library loads, exports every function that
+include/gdn.h declares, and rejects bad arguments on the host before touching the
+device (fake device addresses are never dereferenced on these paths)."""
+
+import ctypes
+import os
+import re
+
+import pytest
+
+from linear_attention_layer_gated_b200 import build, gdn
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "gdn.h")
+
+FAKE = 0x7F0000000000  # 16-byte (and 256-byte) aligned, never dereferenced on these paths
+
+
+def declared_functions():
+    text = open(HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(gdn_[a-z_]+)\s*\(", text)))
+
+
+@pytest.fixture(scope="module")
+def L():
+    build.build()
+    return gdn.lib()
+
+
+def test_exports_every_declared_symbol(L):
+    names = declared_functions()
+    assert set(names) >= set(gdn.EXPORTED)
+    for name in names:
+        assert hasattr(L, name), name
+
+
+def test_abi_version_and_status_strings(L):
+    assert gdn.gdn_abi_version() == 1
+    for code, name in gdn.STATUS.items():
+        assert gdn.gdn_status_string(code).startswith(name)
+
+
+def shape(**kw):
+    base = dict(num_seqs=2, total_tokens=100, num_qk_heads=16, num_v_heads=32, head_dim=128,
+                io_dtype=gdn.GDN_BF16, algo=gdn.GDN_ALGO_AUTO, max_seqlen=0)
+    base.update(kw)
+    return gdn.make_shape(**base)
+
+
+def prefill_call(L, s, ws_bytes=None, **ptrs):
+    p = dict(q=FAKE, k=FAKE, v=FAKE, g=FAKE, beta=FAKE, s0=None, cu=FAKE, out=FAKE, sT=None,
+             ws=FAKE)
+    p.update(ptrs)
+    if ws_bytes is None:
+        ws_bytes = L.gdn_prefill_workspace_bytes(ctypes.byref(s))
+    return L.gdn_chunk_prefill(p["q"], p["k"], p["v"], p["g"], p["beta"], p["s0"], p["cu"],
+                               p["out"], p["sT"], ctypes.byref(s), p["ws"], ws_bytes, None)
+
+
+def test_workspace_size_valid_and_invalid(L):
+    assert L.gdn_prefill_workspace_bytes(ctypes.byref(shape())) % 256 == 0
+    assert L.gdn_prefill_workspace_bytes(ctypes.byref(shape())) > 0
+    assert L.gdn_prefill_workspace_bytes(ctypes.byref(shape(head_dim=64))) == 0
+    assert L.gdn_prefill_workspace_bytes(ctypes.byref(shape(num_v_heads=33))) == 0
+    assert L.gdn_prefill_workspace_bytes(None) == 0
+
+
+@pytest.mark.parametrize("kw,code", [
+    (dict(head_dim=64), "GDN_ERR_SHAPE"),
+    (dict(num_v_heads=24, num_qk_heads=16), "GDN_ERR_SHAPE"),
+    (dict(num_qk_heads=0), "GDN_ERR_SHAPE"),
+    (dict(io_dtype=7), "GDN_ERR_DTYPE"),
+    (dict(total_tokens=-1), "GDN_ERR_SHAPE"),
+    (dict(max_seqlen=101), "GDN_ERR_SHAPE"),
+    (dict(algo=9), "GDN_ERR_SHAPE"),
+])
+def test_prefill_rejects_bad_shapes(L, kw, code):
+    assert gdn.STATUS[prefill_call(L, shape(**kw), ws_bytes=1 << 20)] == code
+
+
+def test_prefill_rejects_null_and_misaligned(L):
+    s = shape()
+    assert gdn.STATUS[prefill_call(L, s, q=None)] == "GDN_ERR_NULL"
+    assert gdn.STATUS[prefill_call(L, s, cu=None)] == "GDN_ERR_NULL"
+    assert gdn.STATUS[prefill_call(L, s, out=None)] == "GDN_ERR_NULL"
+    assert gdn.STATUS[prefill_call(L, s, v=FAKE + 8)] == "GDN_ERR_ALIGN"
+    assert gdn.STATUS[prefill_call(L, s, s0=FAKE + 4)] == "GDN_ERR_ALIGN"
+    assert gdn.STATUS[prefill_call(L, s, ws=FAKE + 16)] == "GDN_ERR_ALIGN"
+    assert gdn.STATUS[prefill_call(L, s, ws=None)] == "GDN_ERR_WORKSPACE"
+    assert gdn.STATUS[prefill_call(L, s, ws_bytes=16)] == "GDN_ERR_WORKSPACE"
+    assert L.gdn_chunk_prefill(FAKE, FAKE, FAKE, FAKE, FAKE, None, FAKE, FAKE, None, None,
+                               FAKE, 1 << 20, None) == 1
+
+
+def decode_call(L, s, ntok=1, **ptrs):
+    p = dict(q=FAKE, k=FAKE, v=FAKE, g=FAKE, beta=FAKE, st=FAKE, out=FAKE)
+    p.update(ptrs)
+    return L.gdn_decode_step(p["q"], p["k"], p["v"], p["g"], p["beta"], p["st"], p["out"], ntok,
+                             ctypes.byref(s), None)
+
+
+@pytest.mark.parametrize("ntok", [0, 5, -1, 100])
+def test_decode_rejects_num_tokens(L, ntok):
+    assert gdn.STATUS[decode_call(L, shape(num_seqs=4), ntok=ntok)] == "GDN_ERR_NUM_TOKENS"
+
+
+def test_decode_rejects_null_misaligned_and_shape(L):
+    s = shape(num_seqs=4)
+    assert gdn.STATUS[decode_call(L, s, st=None)] == "GDN_ERR_NULL"
+    assert gdn.STATUS[decode_call(L, s, out=FAKE + 2)] == "GDN_ERR_ALIGN"
+    assert gdn.STATUS[decode_call(L, shape(head_dim=256))] == "GDN_ERR_SHAPE"
+    assert gdn.STATUS[decode_call(L, shape(io_dtype=3))] == "GDN_ERR_DTYPE"
+
+
+def test_empty_batches_are_no_ops(L):
+    # num_seqs == 0 returns before any device work; no pointer is touched
+    assert prefill_call(L, shape(num_seqs=0, total_tokens=0), q=None, k=None, v=None, g=None,
+                        beta=None, cu=None, out=None) == 0
+    assert decode_call(L, shape(num_seqs=0), q=None) == 0
+
+
+def test_binding_refuses_cpu_tensors():
+    import torch
+    q = torch.zeros(4, 16, 128, dtype=torch.bfloat16)
+    with pytest.raises(ValueError):
+        gdn._ptr(q)

@@ -1,0 +1,249 @@
+"""GPU parity: libgdn.so (through its C ABI) against the fp64 oracle on the same
+seeded inputs.
+
+Tolerances are relative L2 errors over whole flattened tensors, computed separately
+for outputs and states: <= 1e-4 for fp32 I/O (fp32 arithmetic throughout), <= 1e-2 for
+bf16 I/O with fp32 state.  Max-abs error is reported in the assertion message.
+Full-size workloads compare a sample of heads: every (sequence, V head) recurrence is
+independent, so the oracle on a subset of QK heads (and the V heads that read them) is
+an exact sample of the full result.
+"""
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from linear_attention_layer_gated_b200 import gdn, inputs
+
+pytestmark = pytest.mark.gpu
+
+TOL_F32 = 1e-4
+TOL_BF16 = 1e-2
+ALGOS = [gdn.GDN_ALGO_SIMT, gdn.GDN_ALGO_TENSOR]
+
+
+def errs(x, ref):
+    x = x.detach().double().cpu().numpy() if hasattr(x, "detach") else np.asarray(x, np.float64)
+    ref = np.asarray(ref, np.float64)
+    rel = float(np.linalg.norm(x - ref) / max(np.linalg.norm(ref), 1e-300))
+    return rel, float(np.max(np.abs(x - ref))) if x.size else 0.0
+
+
+def assert_close(x, ref, tol, what):
+    rel, mx = errs(x, ref)
+    assert np.isfinite(rel) and rel <= tol, "%s: rel-L2 %.3e (tol %.0e), max-abs %.3e" % (what, rel, tol, mx)
+    return rel, mx
+
+
+def run_prefill(x, algo, want_final=True):
+    try:
+        return gdn.prefill(x["q"], x["k"], x["v"], x["g"], x["beta"], x["cu_seqlens"],
+                           x["initial_state"], want_final, algo=algo)
+    except gdn.GdnError as e:
+        if e.code == 9:
+            pytest.skip("algorithm not available for these inputs")
+        raise
+
+
+def to_dev(x, dev="cuda"):
+    return {k: (v.to(dev) if hasattr(v, "to") else v) for k, v in x.items()}
+
+
+# ------------------------------------------------------------------ decode
+@pytest.mark.parametrize("ntok", [1, 2, 3, 4])
+def test_decode_full_batch_matches_oracle(ntok):
+    w = inputs.workload("decode")
+    x = inputs.make_decode(w.num_seqs, ntok, seed=w.seed, device="cuda")
+    s_ref = x["state"].clone()
+    o_ref, sn_ref = oracle.decode(x["q"], x["k"], x["v"], x["g"], x["beta"], s_ref)
+    st = x["state"].clone()
+    out = gdn.decode(x["q"], x["k"], x["v"], x["g"], x["beta"], st)
+    torch.cuda.synchronize()
+    assert_close(out, o_ref, TOL_BF16, "decode out ntok=%d" % ntok)
+    assert_close(st, sn_ref, TOL_BF16, "decode state ntok=%d" % ntok)
+
+
+def test_decode_fp32_io_tight():
+    x = inputs.make_decode(8, 4, hk=4, hv=8, io_dtype=torch.float32, seed=11, device="cuda")
+    o_ref, sn_ref = oracle.decode(x["q"], x["k"], x["v"], x["g"], x["beta"], x["state"])
+    st = x["state"].clone()
+    out = gdn.decode(x["q"], x["k"], x["v"], x["g"], x["beta"], st)
+    assert_close(out, o_ref, TOL_F32, "decode fp32 out")
+    assert_close(st, sn_ref, TOL_F32, "decode fp32 state")
+
+
+def test_decode_four_tokens_equals_four_single_steps_and_prefill():
+    x = inputs.make_decode(16, 4, hk=4, hv=8, io_dtype=torch.float32, seed=12, device="cuda")
+    s4 = x["state"].clone()
+    o4 = gdn.decode(x["q"], x["k"], x["v"], x["g"], x["beta"], s4)
+    s1 = x["state"].clone()
+    for t in range(4):
+        sl = lambda a: a[:, t:t + 1].contiguous()  # noqa: E731
+        o1 = gdn.decode(sl(x["q"]), sl(x["k"]), sl(x["v"]), sl(x["g"]), sl(x["beta"]), s1)
+        assert_close(o1[:, 0], o4[:, t].double().cpu().numpy(), 1e-5, "decode step %d" % t)
+    assert_close(s1, s4.double().cpu().numpy(), 1e-5, "decode state 4x1 vs 4")
+    N = 16
+    cu = torch.arange(0, 4 * N + 1, 4, dtype=torch.int32, device="cuda")
+    flat = lambda a: a.reshape(N * 4, *a.shape[2:]).contiguous()  # noqa: E731
+    op, sp = gdn.prefill(flat(x["q"]), flat(x["k"]), flat(x["v"]), flat(x["g"]), flat(x["beta"]),
+                         cu, x["state"], algo=gdn.GDN_ALGO_SIMT)
+    assert_close(op.reshape(N, 4, 8, 128), o4.double().cpu().numpy(), 1e-5, "decode vs prefill out")
+    assert_close(sp, s4.double().cpu().numpy(), 1e-5, "decode vs prefill state")
+
+
+# ------------------------------------------------------------------ prefill, small
+def test_prefill_tiny_fp32_matches_oracle():
+    x = inputs.make(inputs.workload("tiny"), device="cuda")
+    o_ref, s_ref = oracle.forward(x["q"], x["k"], x["v"], x["g"], x["beta"], x["cu_seqlens"], None)
+    out, fin = run_prefill(x, gdn.GDN_ALGO_AUTO)
+    torch.cuda.synchronize()
+    assert_close(out, o_ref, TOL_F32, "tiny out")
+    assert_close(fin, s_ref, TOL_F32, "tiny final state")
+
+
+@pytest.mark.parametrize("algo", ALGOS)
+@pytest.mark.parametrize("io", [torch.bfloat16, torch.float32])
+def test_prefill_ragged_varlen_with_states(algo, io):
+    if algo == gdn.GDN_ALGO_TENSOR and io == torch.float32:
+        pytest.skip("tensor-core path is bf16 I/O only")
+    lens = [1, 63, 64, 65, 0, 200, 129, 7]
+    x = inputs.make_prefill(lens, hk=2, hv=4, io_dtype=io, state_std=0.02, seed=21, device="cuda")
+    o_ref, s_ref = oracle.forward(x["q"], x["k"], x["v"], x["g"], x["beta"], x["cu_seqlens"],
+                                  x["initial_state"])
+    out, fin = run_prefill(x, algo)
+    torch.cuda.synchronize()
+    tol = TOL_F32 if io == torch.float32 else TOL_BF16
+    assert_close(out, o_ref, tol, "ragged out")
+    assert_close(fin, s_ref, tol, "ragged final state")
+    # an empty sequence hands its initial state through unchanged
+    torch.testing.assert_close(fin[4], x["initial_state"][4], rtol=0, atol=0)
+
+
+@pytest.mark.parametrize("algo", ALGOS)
+def test_prefill_full_heads_small_T(algo):
+    x = inputs.make_prefill([300], seed=22, device="cuda")
+    o_ref, s_ref = oracle.forward(x["q"], x["k"], x["v"], x["g"], x["beta"], x["cu_seqlens"], None)
+    out, fin = run_prefill(x, algo)
+    assert_close(out, o_ref, TOL_BF16, "16/32 heads out")
+    assert_close(fin, s_ref, TOL_BF16, "16/32 heads state")
+
+
+@pytest.mark.parametrize("algo", ALGOS)
+def test_prefill_in_place_state_carry(algo):
+    x = inputs.make_prefill([70, 130], hk=2, hv=4, state_std=0.02, seed=23, device="cuda")
+    o_ref, s_ref = oracle.forward(x["q"], x["k"], x["v"], x["g"], x["beta"], x["cu_seqlens"],
+                                  x["initial_state"])
+    st = x["initial_state"].clone()
+    out = torch.empty_like(x["v"])
+    try:
+        gdn.gdn_chunk_prefill(x["q"], x["k"], x["v"], x["g"], x["beta"], st, x["cu_seqlens"], out,
+                              st, algo=algo)
+    except gdn.GdnError as e:
+        if e.code == 9:
+            pytest.skip("algorithm not available")
+        raise
+    assert_close(out, o_ref, TOL_BF16, "in-place out")
+    assert_close(st, s_ref, TOL_BF16, "in-place state")
+
+
+@pytest.mark.parametrize("algo", ALGOS)
+def test_prefill_paired_heads_identical(algo):
+    x = inputs.make_prefill([150], hk=2, hv=4, seed=24, device="cuda")
+    for a in ("v", "g", "beta"):
+        x[a][:, 1] = x[a][:, 0]
+    out, fin = run_prefill(x, algo)
+    torch.testing.assert_close(out[:, 1], out[:, 0], rtol=0, atol=0)
+    torch.testing.assert_close(fin[:, 1], fin[:, 0], rtol=0, atol=0)
+
+
+def test_device_error_word_is_clear_after_prefill():
+    x = inputs.make_prefill([100], hk=2, hv=4, seed=25, device="cuda")
+    ws = gdn.alloc_workspace(gdn.prefill_shape(x["q"], x["v"], x["cu_seqlens"]), "cuda")
+    gdn.prefill(x["q"], x["k"], x["v"], x["g"], x["beta"], x["cu_seqlens"], workspace=ws)
+    assert gdn.gdn_get_device_error(ws) == gdn.GDN_OK
+
+
+def test_graph_capture_replays_prefill_and_decode():
+    x = inputs.make_prefill([64, 100], hk=2, hv=4, state_std=0.02, seed=26, device="cuda")
+    out = torch.empty_like(x["v"])
+    fin = torch.empty_like(x["initial_state"])
+    ws = gdn.alloc_workspace(gdn.prefill_shape(x["q"], x["v"], x["cu_seqlens"]), "cuda")
+    d = inputs.make_decode(4, 2, hk=2, hv=4, seed=27, device="cuda")
+    st0 = d["state"].clone()
+    st = d["state"].clone()
+    dout = torch.empty_like(d["v"])
+    s = torch.cuda.Stream()
+    s.wait_stream(torch.cuda.current_stream())
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.stream(s):
+        with torch.cuda.graph(graph, stream=s):
+            gdn.gdn_chunk_prefill(x["q"], x["k"], x["v"], x["g"], x["beta"], x["initial_state"],
+                                  x["cu_seqlens"], out, fin, workspace=ws, stream=s)
+            gdn.gdn_decode_step(d["q"], d["k"], d["v"], d["g"], d["beta"], st, dout, stream=s)
+    st.copy_(st0)
+    graph.replay()
+    torch.cuda.synchronize()
+    o_ref, s_ref = oracle.forward(x["q"], x["k"], x["v"], x["g"], x["beta"], x["cu_seqlens"],
+                                  x["initial_state"])
+    assert_close(out, o_ref, TOL_BF16, "graph prefill out")
+    assert_close(fin, s_ref, TOL_BF16, "graph prefill state")
+    do_ref, ds_ref = oracle.decode(d["q"], d["k"], d["v"], d["g"], d["beta"], st0)
+    assert_close(dout, do_ref, TOL_BF16, "graph decode out")
+    assert_close(st, ds_ref, TOL_BF16, "graph decode state")
+    del graph
+
+
+# ------------------------------------------------------------------ full-size workloads
+@pytest.mark.parametrize("algo", ALGOS)
+def test_layer_prefill_8192_sampled_heads(algo):
+    w = inputs.workload("layer_prefill")
+    x = inputs.make(w, device="cuda")
+    out, fin = run_prefill(x, algo)
+    torch.cuda.synchronize()
+    assert torch.isfinite(out.float()).all() and torch.isfinite(fin).all()
+    heads = [0, 7, 15]
+    o_ref, s_ref, vh = oracle.forward_heads(x["q"], x["k"], x["v"], x["g"], x["beta"],
+                                            x["cu_seqlens"], heads)
+    assert_close(out[:, vh], o_ref, TOL_BF16, "T=8192 out (sampled heads)")
+    assert_close(fin[:, vh], s_ref, TOL_BF16, "T=8192 state (sampled heads)")
+
+
+@pytest.mark.parametrize("algo", ALGOS)
+def test_varlen_8_sequences_sampled_heads(algo):
+    w = inputs.workload("varlen")
+    x = inputs.make(w, device="cuda")
+    out, fin = run_prefill(x, algo)
+    torch.cuda.synchronize()
+    heads = [3, 12]
+    o_ref, s_ref, vh = oracle.forward_heads(x["q"], x["k"], x["v"], x["g"], x["beta"],
+                                            x["cu_seqlens"], heads, x["initial_state"])
+    assert_close(out[:, vh], o_ref, TOL_BF16, "varlen out (sampled heads)")
+    assert_close(fin[:, vh], s_ref, TOL_BF16, "varlen state (sampled heads)")
+
+
+@pytest.mark.parametrize("algo", ALGOS)
+def test_long_context_split_carry_and_sampled_heads(algo):
+    w = inputs.workload("long")
+    x = inputs.make(w, device="cuda")
+    out, fin = run_prefill(x, algo)
+    torch.cuda.synchronize()
+    # 4 segments of 65536 with the state carried in place
+    T = x["q"].shape[0]
+    seg = T // 4
+    st = torch.zeros_like(fin)
+    out_s = torch.empty_like(out)
+    for s in range(4):
+        sl = slice(s * seg, (s + 1) * seg)
+        cu = torch.tensor([0, seg], dtype=torch.int32, device="cuda")
+        gdn.gdn_chunk_prefill(x["q"][sl], x["k"][sl], x["v"][sl], x["g"][sl], x["beta"][sl],
+                              st, cu, out_s[sl], st, algo=algo)
+    torch.cuda.synchronize()
+    # 65536 is a multiple of the chunk size: the split run is the same arithmetic
+    torch.testing.assert_close(out_s, out, rtol=0, atol=0)
+    torch.testing.assert_close(st, fin, rtol=0, atol=0)
+    heads = [5]
+    o_ref, s_ref, vh = oracle.forward_heads(x["q"], x["k"], x["v"], x["g"], x["beta"],
+                                            x["cu_seqlens"], heads)
+    assert_close(out[:, vh], o_ref, TOL_BF16, "T=262144 out (sampled heads)")
+    assert_close(fin[:, vh], s_ref, TOL_BF16, "T=262144 state (sampled heads)")
