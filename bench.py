@@ -305,8 +305,13 @@ def main_ours(args, rank, world, local_rank):
 
 
 def gdn_launches_per_prefill(algo, dtype):
-    """Kernels libgdn.so launches per gdn_chunk_prefill call on the chosen path."""
-    return 1
+    """Kernels libgdn.so launches per gdn_chunk_prefill call on the chosen path:
+    the SIMT path is one kernel; the tensor-core path is chunk table, chunk prep and
+    chunk state (the workspace-header memset is not a kernel of ours)."""
+    from linear_attention_layer_gated_b200 import gdn
+    import torch
+    tensor = algo == gdn.GDN_ALGO_TENSOR or (algo == gdn.GDN_ALGO_AUTO and dtype == torch.bfloat16)
+    return 3 if tensor else 1
 
 
 def main():

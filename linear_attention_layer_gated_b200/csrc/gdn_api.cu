@@ -56,8 +56,18 @@ const char* gdn_status_string(gdn_status status) {
     return "unknown gdn_status";
 }
 
+// Which kernel family serves a (validated) shape: true = tensor cores.
+static bool use_tensor_path(const gdn_shape* s) {
+    if (s->algo == GDN_ALGO_TENSOR) return true;
+    if (s->algo == GDN_ALGO_SIMT) return false;
+    return s->io_dtype == GDN_BF16;
+}
+
 size_t gdn_prefill_workspace_bytes(const gdn_shape* shape) {
     if (check_prefill_shape(shape) != GDN_OK) return 0;
+    if (use_tensor_path(shape) && shape->io_dtype == GDN_BF16)
+        return gdn::tc_workspace_bytes(shape->num_seqs, shape->total_tokens, shape->num_qk_heads,
+                                       shape->num_v_heads);
     return kHeaderBytes;
 }
 
@@ -79,13 +89,19 @@ gdn_status gdn_chunk_prefill(const void* q, const void* k, const void* v, const 
         if (p && !aligned16(p)) return GDN_ERR_ALIGN;
 
     gdn_dtype io = (gdn_dtype)shape->io_dtype;
-    int algo = shape->algo;
-    if (algo == GDN_ALGO_TENSOR) return GDN_ERR_UNSUPPORTED;
+    const bool tensor = use_tensor_path(shape);
+    if (tensor && io != GDN_BF16) return GDN_ERR_UNSUPPORTED;
     cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
     if (cudaMemsetAsync(workspace, 0, kHeaderBytes, s) != cudaSuccess) return GDN_ERR_CUDA;
-    cudaError_t e = gdn::launch_prefill_simt(q, k, v, g, beta, initial_state, cu_seqlens, out,
-                                             final_state, shape->num_seqs, shape->num_qk_heads,
-                                             shape->num_v_heads, io, s);
+    cudaError_t e;
+    if (tensor)
+        e = gdn::launch_prefill_tc(q, k, v, g, beta, initial_state, cu_seqlens, out, final_state,
+                                   shape->num_seqs, shape->total_tokens, shape->num_qk_heads,
+                                   shape->num_v_heads, workspace, s);
+    else
+        e = gdn::launch_prefill_simt(q, k, v, g, beta, initial_state, cu_seqlens, out,
+                                     final_state, shape->num_seqs, shape->num_qk_heads,
+                                     shape->num_v_heads, io, s);
     return e == cudaSuccess ? GDN_OK : GDN_ERR_CUDA;
 }
 

@@ -55,4 +55,11 @@ cudaError_t launch_prefill_simt(const void* q, const void* k, const void* v, con
                                 void* out, float* sT, int num_seqs, int hk, int hv,
                                 gdn_dtype io, cudaStream_t stream);
 
+// Tensor-core prefill (bf16 I/O): total workspace bytes (header included) and launch.
+size_t tc_workspace_bytes(int num_seqs, int total_tokens, int hk, int hv);
+cudaError_t launch_prefill_tc(const void* q, const void* k, const void* v, const float* g,
+                              const float* beta, const float* s0, const int32_t* cu, void* out,
+                              float* sT, int num_seqs, int total_tokens, int hk, int hv,
+                              void* workspace, cudaStream_t stream);
+
 }  // namespace gdn
