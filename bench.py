@@ -41,6 +41,11 @@ HK, HV, D, C = 16, 32, 128, 64
 PREFILL_FLOP_PER_TOKEN = HV * (3 * 2 * C * D + 3 * 2 * D * D) + HK * (2 * 2 * C * D)  # 5,242,880
 PREFILL_BYTES_PER_TOKEN = 2 * HK * D * 2 + HV * D * 2 * 2 + HV * 4 * 2                # 24,832
 STATE_BYTES = HV * D * D * 4                                                          # per sequence
+# Split of the GEMM flops between the two tensor-core phases:
+#   prep  = Gram matrices (per QK head) + W and U (per V head)
+#   state = [W; Q] S^T, P Delta and the state update (per V head)
+PREP_FLOP_PER_TOKEN = HK * (2 * 2 * C * D) + HV * (2 * 2 * C * D)                    # 1,572,864
+STATE_FLOP_PER_TOKEN = HV * (2 * C * D + 3 * 2 * D * D)                               # 3,670,016
 
 
 def decode_bytes(num_seqs, ntok):
@@ -182,6 +187,8 @@ def main_ours(args, rank, world, local_rank):
             "tensor": gdn.GDN_ALGO_TENSOR}[args.algo]
 
     w = inputs.workload(WORKLOAD)
+    if args.tokens:
+        w.seqlens = [args.tokens]
     x = inputs.make(w, device=dev)
     T = x["q"].shape[0]
     out = torch.empty_like(x["v"])
@@ -190,9 +197,24 @@ def main_ours(args, rank, world, local_rank):
     ws = gdn.alloc_workspace(shape, dev)
     flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
 
+    tensor_path = gdn_launches_per_prefill(algo, x["q"].dtype) == 3
+    phase_ev = []
+
     def prefill_once():
         gdn.gdn_chunk_prefill(x["q"], x["k"], x["v"], x["g"], x["beta"], None, x["cu_seqlens"],
                               out, fin, workspace=ws, algo=algo, stream=stream)
+
+    def prefill_phased():
+        # the same two launches gdn_chunk_prefill makes, with events between them
+        e = [torch.cuda.Event(enable_timing=True) for _ in range(3)]
+        e[0].record(stream)
+        gdn.gdn_chunk_prefill_prep(x["q"], x["k"], x["v"], x["g"], x["beta"], x["cu_seqlens"],
+                                   ws, algo=algo, stream=stream)
+        e[1].record(stream)
+        gdn.gdn_chunk_prefill_state(None, x["cu_seqlens"], out, fin, ws, x["q"], algo=algo,
+                                    stream=stream)
+        e[2].record(stream)
+        phase_ev.append(e)
 
     def barrier():
         if world > 1:
@@ -221,22 +243,43 @@ def main_ours(args, rank, world, local_rank):
         dist.all_reduce(t, op=dist.ReduceOp.MAX)
         return float(t.item())
 
+    step_fn = prefill_phased if tensor_path else prefill_once
     with ClockSampler(local_rank) as clk:
-        ms = timed(prefill_once, args.steps, args.warmup)
+        ms = timed(step_fn, args.steps, args.warmup)
     clocks = clk.summary()
     ms_step = max_over_ranks(sum(ms) / len(ms))
     value = world * T / (ms_step * 1e-3)
 
-    # ---- dominant kernel roofline (the prefill is one launch per step on this path)
+    # ---- dominant kernel roofline, from CUDA events on the launching stream
     launches_per_step = gdn_launches_per_prefill(algo, x["q"].dtype)
-    flop = PREFILL_FLOP_PER_TOKEN * T
-    achieved_tflops = flop / (ms_step * 1e-3) / 1e12
     peak = peaks["bf16_tflops"]
-    roofline = {"bound": "tensor", "achieved": achieved_tflops, "peak": peak, "unit": "TFLOP/s",
-                "frac": achieved_tflops / peak, "traffic": None,
-                "peak_source": peaks["source"] + " bf16 dense (burst)",
-                "kernel": "gdn prefill step (all launches)",
-                "algorithmic_flop_per_launch": flop}
+    phases = None
+    if tensor_path:
+        timed_ev = phase_ev[-args.steps:]
+        prep_ms = max_over_ranks(sum(e[0].elapsed_time(e[1]) for e in timed_ev) / args.steps)
+        state_ms = max_over_ranks(sum(e[1].elapsed_time(e[2]) for e in timed_ev) / args.steps)
+        phases = {
+            "prep": {"kernels": "chunk_table_kernel + chunk_prep_kernel", "ms": prep_ms,
+                     "flop": PREP_FLOP_PER_TOKEN * T,
+                     "tflops": PREP_FLOP_PER_TOKEN * T / (prep_ms * 1e-3) / 1e12},
+            "state": {"kernels": "chunk_state_kernel", "ms": state_ms,
+                      "flop": STATE_FLOP_PER_TOKEN * T,
+                      "tflops": STATE_FLOP_PER_TOKEN * T / (state_ms * 1e-3) / 1e12}}
+        dom = max(phases, key=lambda k2: phases[k2]["ms"])
+        achieved = phases[dom]["tflops"]
+        roofline = {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
+                    "frac": achieved / peak, "traffic": None,
+                    "peak_source": peaks["source"] + " bf16 dense (burst)",
+                    "kernel": phases[dom]["kernels"],
+                    "algorithmic_flop_per_launch": phases[dom]["flop"],
+                    "step_frac": PREFILL_FLOP_PER_TOKEN * T / (ms_step * 1e-3) / 1e12 / peak}
+    else:
+        flop = PREFILL_FLOP_PER_TOKEN * T
+        achieved = flop / (ms_step * 1e-3) / 1e12
+        roofline = {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
+                    "frac": achieved / peak, "traffic": None,
+                    "peak_source": peaks["source"] + " bf16 dense (burst)",
+                    "kernel": "prefill_simt_kernel", "algorithmic_flop_per_launch": flop}
 
     # ---- end to end through the C ABI with pinned host buffers
     host = {k2: x[k2].cpu().pin_memory() for k2 in ("q", "k", "v", "g", "beta", "cu_seqlens")}
@@ -250,14 +293,18 @@ def main_ours(args, rank, world, local_rank):
                               dbuf["cu_seqlens"], out, fin, workspace=ws, algo=algo, stream=stream)
         hout.copy_(out, non_blocking=True)
 
-    e2e_ms = timed(e2e_once, max(3, args.steps // 2), 2)
-    e2e_step = max_over_ranks(sum(e2e_ms) / len(e2e_ms))
-    h2d = sum(t.numel() * t.element_size() for t in host.values())
-    d2h = hout.numel() * hout.element_size()
+    e2e = None
+    if not args.no_e2e:
+        e2e_ms = timed(e2e_once, max(3, args.steps // 2), 2)
+        e2e_step = max_over_ranks(sum(e2e_ms) / len(e2e_ms))
+        h2d = sum(t.numel() * t.element_size() for t in host.values())
+        d2h = hout.numel() * hout.element_size()
+        e2e = {"value": world * T / (e2e_step * 1e-3), "unit": UNIT,
+               "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h}
 
     # ---- decode: 256 sequences, 1 token and 4-token verify
     dec = {}
-    for ntok in (1, 4):
+    for ntok in ((1, 4) if args.only != "prefill" else ()):
         d = inputs.make_decode(256, ntok, seed=3, device=dev)
         dout = torch.empty_like(d["v"])
 
@@ -277,7 +324,7 @@ def main_ours(args, rank, world, local_rank):
 
     # ---- CPU baseline: the oracle on a bounded sample (rank 0, N=1 only)
     cpu = None
-    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+    if rank == 0 and world == 1 and not args.no_cpu_baseline and not args.tokens:
         import oracle
         xs = {k2: (x[k2].cpu() if hasattr(x[k2], "cpu") else x[k2]) for k2 in x}
         v_cpu, dt = oracle_tokens_per_s(xs, HK)
@@ -296,9 +343,8 @@ def main_ours(args, rank, world, local_rank):
                            "l2": "flushed between timed steps (256 MiB write)",
                            "algo": args.algo},
                 "roofline": roofline, "cpu_baseline": cpu,
-                "e2e": {"value": world * T / (e2e_step * 1e-3), "unit": UNIT,
-                        "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
-                "gpu_launches": launches_per_step * args.steps,
+                "e2e": e2e,
+                "gpu_launches": launches_per_step * args.steps, "phases": phases,
                 "decode": dec, "clocks": clocks, "peaks": peaks}
         print(json.dumps(line), flush=True)
     return 0
@@ -322,6 +368,11 @@ def main():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--algo", default="auto", choices=["auto", "simt", "tensor"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-e2e", action="store_true", help="skip the host-buffer end-to-end leg")
+    ap.add_argument("--only", default="all", choices=["all", "prefill"],
+                    help="prefill: skip the decode measurements (profiling runs)")
+    ap.add_argument("--tokens", type=int, default=0,
+                    help="override the prefill length (profiling runs; not a bench line)")
     args = ap.parse_args()
     if args.warmup < 3 and args.impl == "ours":
         args.warmup = 3

@@ -120,6 +120,28 @@ gdn_status gdn_chunk_prefill(const void *q, const void *k, const void *v,
                              void *workspace, size_t workspace_bytes, void *stream);
 
 /*
+ * The tensor-core prefill in two phases, for callers that want to schedule or time
+ * them separately (gdn_chunk_prefill is exactly prep followed by state on one stream).
+ *
+ * gdn_chunk_prefill_prep: builds the chunk table from cu_seqlens and, for every chunk
+ *   and head in parallel, the chunk's UT representation (W, U, P, decay factors and the
+ *   normalised keys) into `workspace`.  Reads q, k, v, g, beta, cu_seqlens.
+ * gdn_chunk_prefill_state: carries each sequence's fp32 state across its chunks using
+ *   the workspace written by the prep phase of the same shape, writing out and
+ *   final_state.  Reads initial_state, cu_seqlens.
+ * Both require io_dtype == GDN_BF16 and an algo of GDN_ALGO_AUTO or GDN_ALGO_TENSOR
+ * (GDN_ERR_UNSUPPORTED otherwise); arguments as for gdn_chunk_prefill.  The workspace
+ * header is cleared by the prep phase.
+ */
+gdn_status gdn_chunk_prefill_prep(const void *q, const void *k, const void *v,
+                                  const float *g, const float *beta,
+                                  const int32_t *cu_seqlens, const gdn_shape *shape,
+                                  void *workspace, size_t workspace_bytes, void *stream);
+gdn_status gdn_chunk_prefill_state(const float *initial_state, const int32_t *cu_seqlens,
+                                   void *out, float *final_state, const gdn_shape *shape,
+                                   void *workspace, size_t workspace_bytes, void *stream);
+
+/*
  * Decode / multi-token verify step: advances every sequence's state by num_tokens
  * (1..4) tokens in place and writes the output of every token.  This is the memory
  * bound step a speculative-decoding verifier uses (the pages' multi-token prediction
@@ -145,6 +167,17 @@ gdn_status gdn_decode_step(const void *q, const void *k, const void *v,
  * previous prefill gave up, GDN_ERR_CUDA if the runtime reports an error, else GDN_OK.
  */
 gdn_status gdn_get_device_error(void *workspace, void *stream);
+
+/*
+ * Failure-path self-test.  Clears the workspace header, then launches a kernel that waits
+ * on a barrier nothing completes, using the same bounded wait as the prefill kernels
+ * but with a limit of `limit_us` microseconds (1 .. 2,000,000).  When the limit expires
+ * the kernel records the timeout in the header and returns normally; a following
+ * gdn_get_device_error(workspace, stream) then returns GDN_ERR_DEVICE_TIMEOUT and the
+ * CUDA context remains usable.  `workspace` needs >= 256 bytes, 256-byte aligned.
+ */
+gdn_status gdn_selftest_wait_timeout(void *workspace, size_t workspace_bytes, uint32_t limit_us,
+                                     void *stream);
 
 /* Static, human-readable name of a status code. */
 const char *gdn_status_string(gdn_status status);

@@ -94,14 +94,67 @@ gdn_status gdn_chunk_prefill(const void* q, const void* k, const void* v, const 
     cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
     if (cudaMemsetAsync(workspace, 0, kHeaderBytes, s) != cudaSuccess) return GDN_ERR_CUDA;
     cudaError_t e;
-    if (tensor)
-        e = gdn::launch_prefill_tc(q, k, v, g, beta, initial_state, cu_seqlens, out, final_state,
-                                   shape->num_seqs, shape->total_tokens, shape->num_qk_heads,
-                                   shape->num_v_heads, workspace, s);
-    else
+    if (tensor) {
+        e = gdn::launch_prefill_tc_prep(q, k, v, g, beta, cu_seqlens, shape->num_seqs,
+                                        shape->total_tokens, shape->num_qk_heads,
+                                        shape->num_v_heads, workspace, s);
+        if (e == cudaSuccess)
+            e = gdn::launch_prefill_tc_state(initial_state, cu_seqlens, out, final_state,
+                                             shape->num_seqs, shape->total_tokens,
+                                             shape->num_qk_heads, shape->num_v_heads, workspace, s);
+    } else
         e = gdn::launch_prefill_simt(q, k, v, g, beta, initial_state, cu_seqlens, out,
                                      final_state, shape->num_seqs, shape->num_qk_heads,
                                      shape->num_v_heads, io, s);
+    return e == cudaSuccess ? GDN_OK : GDN_ERR_CUDA;
+}
+
+// Shared validation of the two tensor-core prefill phases.
+static gdn_status check_phase(const gdn_shape* shape, const int32_t* cu_seqlens, void* workspace,
+                              size_t workspace_bytes) {
+    gdn_status st = check_prefill_shape(shape);
+    if (st != GDN_OK) return st;
+    if (shape->io_dtype != GDN_BF16 || !use_tensor_path(shape)) return GDN_ERR_UNSUPPORTED;
+    if (!workspace || workspace_bytes < gdn_prefill_workspace_bytes(shape)) return GDN_ERR_WORKSPACE;
+    if ((reinterpret_cast<uintptr_t>(workspace) & 255u) != 0) return GDN_ERR_ALIGN;
+    if (shape->num_seqs > 0 && !cu_seqlens) return GDN_ERR_NULL;
+    if (cu_seqlens && !aligned16(cu_seqlens)) return GDN_ERR_ALIGN;
+    return GDN_OK;
+}
+
+gdn_status gdn_chunk_prefill_prep(const void* q, const void* k, const void* v, const float* g,
+                                  const float* beta, const int32_t* cu_seqlens,
+                                  const gdn_shape* shape, void* workspace, size_t workspace_bytes,
+                                  void* stream) {
+    gdn_status st = check_phase(shape, cu_seqlens, workspace, workspace_bytes);
+    if (st != GDN_OK) return st;
+    if (shape->num_seqs == 0) return GDN_OK;
+    if (shape->total_tokens > 0 && (!q || !k || !v || !g || !beta)) return GDN_ERR_NULL;
+    const void* ptrs[] = {q, k, v, g, beta};
+    for (const void* p : ptrs)
+        if (p && !aligned16(p)) return GDN_ERR_ALIGN;
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    if (cudaMemsetAsync(workspace, 0, kHeaderBytes, s) != cudaSuccess) return GDN_ERR_CUDA;
+    cudaError_t e = gdn::launch_prefill_tc_prep(q, k, v, g, beta, cu_seqlens, shape->num_seqs,
+                                                shape->total_tokens, shape->num_qk_heads,
+                                                shape->num_v_heads, workspace, s);
+    return e == cudaSuccess ? GDN_OK : GDN_ERR_CUDA;
+}
+
+gdn_status gdn_chunk_prefill_state(const float* initial_state, const int32_t* cu_seqlens,
+                                   void* out, float* final_state, const gdn_shape* shape,
+                                   void* workspace, size_t workspace_bytes, void* stream) {
+    gdn_status st = check_phase(shape, cu_seqlens, workspace, workspace_bytes);
+    if (st != GDN_OK) return st;
+    if (shape->num_seqs == 0) return GDN_OK;
+    if (shape->total_tokens > 0 && !out) return GDN_ERR_NULL;
+    const void* ptrs[] = {initial_state, out, final_state};
+    for (const void* p : ptrs)
+        if (p && !aligned16(p)) return GDN_ERR_ALIGN;
+    cudaError_t e = gdn::launch_prefill_tc_state(initial_state, cu_seqlens, out, final_state,
+                                                 shape->num_seqs, shape->total_tokens,
+                                                 shape->num_qk_heads, shape->num_v_heads,
+                                                 workspace, reinterpret_cast<cudaStream_t>(stream));
     return e == cudaSuccess ? GDN_OK : GDN_ERR_CUDA;
 }
 
@@ -121,6 +174,18 @@ gdn_status gdn_decode_step(const void* q, const void* k, const void* v, const fl
                                        shape->num_seqs, shape->num_qk_heads, shape->num_v_heads,
                                        (gdn_dtype)shape->io_dtype,
                                        reinterpret_cast<cudaStream_t>(stream));
+    return e == cudaSuccess ? GDN_OK : GDN_ERR_CUDA;
+}
+
+gdn_status gdn_selftest_wait_timeout(void* workspace, size_t workspace_bytes, uint32_t limit_us,
+                                      void* stream) {
+    if (!workspace) return GDN_ERR_NULL;
+    if (workspace_bytes < kHeaderBytes) return GDN_ERR_WORKSPACE;
+    if ((reinterpret_cast<uintptr_t>(workspace) & 255u) != 0) return GDN_ERR_ALIGN;
+    if (limit_us < 1 || limit_us > 2000000) return GDN_ERR_SHAPE;
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    if (cudaMemsetAsync(workspace, 0, kHeaderBytes, s) != cudaSuccess) return GDN_ERR_CUDA;
+    cudaError_t e = gdn::launch_wait_timeout_selftest(workspace, (uint64_t)limit_us * 1000u, s);
     return e == cudaSuccess ? GDN_OK : GDN_ERR_CUDA;
 }
 

@@ -57,9 +57,16 @@ cudaError_t launch_prefill_simt(const void* q, const void* k, const void* v, con
 
 // Tensor-core prefill (bf16 I/O): total workspace bytes (header included) and launch.
 size_t tc_workspace_bytes(int num_seqs, int total_tokens, int hk, int hv);
-cudaError_t launch_prefill_tc(const void* q, const void* k, const void* v, const float* g,
-                              const float* beta, const float* s0, const int32_t* cu, void* out,
-                              float* sT, int num_seqs, int total_tokens, int hk, int hv,
-                              void* workspace, cudaStream_t stream);
+// Phase 1 (chunk table + per-chunk UT representation) and phase 2 (state pass).
+cudaError_t launch_prefill_tc_prep(const void* q, const void* k, const void* v, const float* g,
+                                   const float* beta, const int32_t* cu, int num_seqs,
+                                   int total_tokens, int hk, int hv, void* workspace,
+                                   cudaStream_t stream);
+cudaError_t launch_prefill_tc_state(const float* s0, const int32_t* cu, void* out, float* sT,
+                                    int num_seqs, int total_tokens, int hk, int hv,
+                                    void* workspace, cudaStream_t stream);
+
+// Diagnostic: a bounded wait that is guaranteed to expire (failure-path self-test).
+cudaError_t launch_wait_timeout_selftest(void* workspace, uint64_t limit_ns, cudaStream_t stream);
 
 }  // namespace gdn

@@ -649,17 +649,15 @@ size_t tc_workspace_bytes(int num_seqs, int total_tokens, int hk, int hv) {
     return ws_layout(num_seqs, total_tokens, hk, hv).total;
 }
 
-cudaError_t launch_prefill_tc(const void* q, const void* k, const void* v, const float* g,
-                              const float* beta, const float* s0, const int32_t* cu, void* out,
-                              float* sT, int num_seqs, int total_tokens, int hk, int hv,
-                              void* workspace, cudaStream_t stream) {
+cudaError_t launch_prefill_tc_prep(const void* q, const void* k, const void* v, const float* g,
+                                   const float* beta, const int32_t* cu, int num_seqs,
+                                   int total_tokens, int hk, int hv, void* workspace,
+                                   cudaStream_t stream) {
     if (num_seqs == 0) return cudaSuccess;
     unsigned char* ws = static_cast<unsigned char*>(workspace);
     const WsLayout L = ws_layout(num_seqs, total_tokens, hk, hv);
-    cudaError_t e;
-    e = cudaFuncSetAttribute(chunk_prep_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kPrepSmem);
-    if (e != cudaSuccess) return e;
-    e = cudaFuncSetAttribute(chunk_state_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kStateSmem);
+    cudaError_t e = cudaFuncSetAttribute(chunk_prep_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         (int)kPrepSmem);
     if (e != cudaSuccess) return e;
     chunk_table_kernel<<<1, 1024, 0, stream>>>(cu, num_seqs, ws);
     if (L.max_chunks > 0 && total_tokens > 0) {
@@ -667,8 +665,19 @@ cudaError_t launch_prefill_tc(const void* q, const void* k, const void* v, const
             (const __nv_bfloat16*)q, (const __nv_bfloat16*)k, (const __nv_bfloat16*)v, g, beta, ws,
             num_seqs, total_tokens, hk, hv);
     }
+    return cudaGetLastError();
+}
+
+cudaError_t launch_prefill_tc_state(const float* s0, const int32_t* cu, void* out, float* sT,
+                                    int num_seqs, int total_tokens, int hk, int hv,
+                                    void* workspace, cudaStream_t stream) {
+    if (num_seqs == 0) return cudaSuccess;
+    cudaError_t e = cudaFuncSetAttribute(chunk_state_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         (int)kStateSmem);
+    if (e != cudaSuccess) return e;
     chunk_state_kernel<<<(unsigned)num_seqs * hv * 2, kThreads, kStateSmem, stream>>>(
-        s0, cu, (__nv_bfloat16*)out, sT, ws, num_seqs, total_tokens, hk, hv);
+        s0, cu, (__nv_bfloat16*)out, sT, static_cast<unsigned char*>(workspace), num_seqs,
+        total_tokens, hk, hv);
     return cudaGetLastError();
 }
 

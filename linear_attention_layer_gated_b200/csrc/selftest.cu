@@ -1,0 +1,33 @@
+// selftest.cu -- exercises the device-side failure path without faulting the GPU.
+//
+// The kernel arms an mbarrier that nothing will ever complete and waits on it with the
+// same bounded wait the prefill kernels use, but with a caller-chosen limit.  When the
+// wait gives up it records GDN_ERR_DEVICE_TIMEOUT's device word in the workspace header,
+// exactly as a stuck prefill would, and returns normally, so the CUDA context stays
+// usable.  Nothing here traps, spins without a limit or touches invalid memory.
+#include "gdn_internal.cuh"
+#include "sm100.cuh"
+
+namespace gdn {
+namespace {
+
+__global__ void wait_timeout_kernel(int32_t* header, uint64_t limit_ns) {
+    __shared__ uint64_t bar;
+    if (threadIdx.x == 0) {
+        sm100::mbar_init(&bar, 1);
+        sm100::fence_mbar_init();
+    }
+    __syncthreads();
+    // No thread arrives: phase 0 never completes, so the bounded wait must expire.
+    const bool ok = sm100::mbar_wait(&bar, 0, limit_ns);
+    if (!ok && threadIdx.x == 0) atomicOr(header, 1);
+}
+
+}  // namespace
+
+cudaError_t launch_wait_timeout_selftest(void* workspace, uint64_t limit_ns, cudaStream_t stream) {
+    wait_timeout_kernel<<<1, 32, 0, stream>>>(static_cast<int32_t*>(workspace), limit_ns);
+    return cudaGetLastError();
+}
+
+}  // namespace gdn

@@ -22,8 +22,9 @@ GDN_ALGO_AUTO, GDN_ALGO_SIMT, GDN_ALGO_TENSOR = 0, 1, 2
 STATUS = {0: "GDN_OK", 1: "GDN_ERR_NULL", 2: "GDN_ERR_SHAPE", 3: "GDN_ERR_ALIGN",
           4: "GDN_ERR_DTYPE", 5: "GDN_ERR_NUM_TOKENS", 6: "GDN_ERR_WORKSPACE",
           7: "GDN_ERR_CUDA", 8: "GDN_ERR_DEVICE_TIMEOUT", 9: "GDN_ERR_UNSUPPORTED"}
-EXPORTED = ["gdn_prefill_workspace_bytes", "gdn_chunk_prefill", "gdn_decode_step",
-            "gdn_get_device_error", "gdn_status_string", "gdn_abi_version"]
+EXPORTED = ["gdn_prefill_workspace_bytes", "gdn_chunk_prefill", "gdn_chunk_prefill_prep",
+            "gdn_chunk_prefill_state", "gdn_decode_step", "gdn_get_device_error",
+            "gdn_selftest_wait_timeout", "gdn_status_string", "gdn_abi_version"]
 
 
 class GdnShape(ctypes.Structure):
@@ -59,10 +60,16 @@ def lib() -> ctypes.CDLL:
             L.gdn_chunk_prefill.restype = ctypes.c_int
             L.gdn_chunk_prefill.argtypes = [vp, vp, vp, fp, fp, fp, ip, vp, fp, sp, vp,
                                             ctypes.c_size_t, vp]
+            L.gdn_chunk_prefill_prep.restype = ctypes.c_int
+            L.gdn_chunk_prefill_prep.argtypes = [vp, vp, vp, fp, fp, ip, sp, vp, ctypes.c_size_t, vp]
+            L.gdn_chunk_prefill_state.restype = ctypes.c_int
+            L.gdn_chunk_prefill_state.argtypes = [fp, ip, vp, fp, sp, vp, ctypes.c_size_t, vp]
             L.gdn_decode_step.restype = ctypes.c_int
             L.gdn_decode_step.argtypes = [vp, vp, vp, fp, fp, fp, vp, ctypes.c_int32, sp, vp]
             L.gdn_get_device_error.restype = ctypes.c_int
             L.gdn_get_device_error.argtypes = [vp, vp]
+            L.gdn_selftest_wait_timeout.restype = ctypes.c_int
+            L.gdn_selftest_wait_timeout.argtypes = [vp, ctypes.c_size_t, ctypes.c_uint32, vp]
             L.gdn_status_string.restype = ctypes.c_char_p
             L.gdn_status_string.argtypes = [ctypes.c_int]
             L.gdn_abi_version.restype = ctypes.c_int32
@@ -149,6 +156,29 @@ def gdn_chunk_prefill(q, k, v, g, beta, initial_state, cu_seqlens, out, final_st
     return workspace
 
 
+def gdn_chunk_prefill_prep(q, k, v, g, beta, cu_seqlens, workspace, algo=GDN_ALGO_AUTO,
+                           stream=None):
+    """Calls gdn_chunk_prefill_prep (tensor-core path, phase 1)."""
+    shape = prefill_shape(q, v, cu_seqlens, algo)
+    rc = lib().gdn_chunk_prefill_prep(_ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(beta),
+                                      _ptr(cu_seqlens), ctypes.byref(shape), _ptr(workspace),
+                                      workspace.numel(), _stream(stream))
+    if rc != GDN_OK:
+        raise GdnError(rc, "gdn_chunk_prefill_prep")
+
+
+def gdn_chunk_prefill_state(initial_state, cu_seqlens, out, final_state, workspace, q_shape_like,
+                            algo=GDN_ALGO_AUTO, stream=None):
+    """Calls gdn_chunk_prefill_state (tensor-core path, phase 2).  ``q_shape_like`` is the
+    q tensor (or any tensor of q's shape and dtype) the prep phase was given."""
+    shape = prefill_shape(q_shape_like, out, cu_seqlens, algo)
+    rc = lib().gdn_chunk_prefill_state(_ptr(initial_state), _ptr(cu_seqlens), _ptr(out),
+                                       _ptr(final_state), ctypes.byref(shape), _ptr(workspace),
+                                       workspace.numel(), _stream(stream))
+    if rc != GDN_OK:
+        raise GdnError(rc, "gdn_chunk_prefill_state")
+
+
 def gdn_decode_step(q, k, v, g, beta, state_inout, out, num_tokens=None, stream=None):
     """Calls gdn_decode_step.  Shapes: q, k [N, m, HK, 128]; v, out [N, m, HV, 128];
     g, beta [N, m, HV] fp32; state_inout [N, HV, 128, 128] fp32 (updated in place)."""
@@ -160,6 +190,14 @@ def gdn_decode_step(q, k, v, g, beta, state_inout, out, num_tokens=None, stream=
                                _ptr(out), int(num_tokens), ctypes.byref(shape), _stream(stream))
     if rc != GDN_OK:
         raise GdnError(rc, "gdn_decode_step")
+
+
+def gdn_selftest_wait_timeout(workspace, limit_us=20000, stream=None):
+    """Calls gdn_selftest_wait_timeout (a bounded device wait that must expire)."""
+    rc = lib().gdn_selftest_wait_timeout(_ptr(workspace), workspace.numel(), int(limit_us),
+                                         _stream(stream))
+    if rc != GDN_OK:
+        raise GdnError(rc, "gdn_selftest_wait_timeout")
 
 
 def gdn_get_device_error(workspace, stream=None) -> int:

@@ -125,3 +125,10 @@ def test_binding_refuses_cpu_tensors():
     q = torch.zeros(4, 16, 128, dtype=torch.bfloat16)
     with pytest.raises(ValueError):
         gdn._ptr(q)
+
+
+def test_selftest_rejects_bad_arguments(L):
+    assert gdn.STATUS[L.gdn_selftest_wait_timeout(None, 256, 1000, None)] == "GDN_ERR_NULL"
+    assert gdn.STATUS[L.gdn_selftest_wait_timeout(FAKE, 16, 1000, None)] == "GDN_ERR_WORKSPACE"
+    assert gdn.STATUS[L.gdn_selftest_wait_timeout(FAKE + 16, 256, 1000, None)] == "GDN_ERR_ALIGN"
+    assert gdn.STATUS[L.gdn_selftest_wait_timeout(FAKE, 256, 0, None)] == "GDN_ERR_SHAPE"

@@ -247,3 +247,17 @@ def test_long_context_split_carry_and_sampled_heads(algo):
                                             x["cu_seqlens"], heads)
     assert_close(out[:, vh], o_ref, TOL_BF16, "T=262144 out (sampled heads)")
     assert_close(fin[:, vh], s_ref, TOL_BF16, "T=262144 state (sampled heads)")
+
+
+def test_bounded_wait_expiry_is_reported_and_context_survives():
+    """A device wait that nothing completes gives up after its limit, records the
+    timeout in the workspace header and returns; the next calls still work."""
+    ws = torch.zeros(256, dtype=torch.uint8, device="cuda")
+    gdn.gdn_selftest_wait_timeout(ws, limit_us=20000)
+    assert gdn.STATUS[gdn.gdn_get_device_error(ws)] == "GDN_ERR_DEVICE_TIMEOUT"
+    x = inputs.make_prefill([80], hk=2, hv=4, seed=28, device="cuda")
+    ws2 = gdn.alloc_workspace(gdn.prefill_shape(x["q"], x["v"], x["cu_seqlens"]), "cuda")
+    out, fin = gdn.prefill(x["q"], x["k"], x["v"], x["g"], x["beta"], x["cu_seqlens"], workspace=ws2)
+    assert gdn.gdn_get_device_error(ws2) == gdn.GDN_OK
+    o_ref, _ = oracle.forward(x["q"], x["k"], x["v"], x["g"], x["beta"], x["cu_seqlens"], None)
+    assert_close(out, o_ref, TOL_BF16, "prefill after a reported timeout")
