@@ -169,6 +169,34 @@ gdn_status gdn_decode_step(const void *q, const void *k, const void *v,
 gdn_status gdn_get_device_error(void *workspace, void *stream);
 
 /*
+ * Prefill that allocates nothing, for callers that cannot allocate device memory where
+ * they run (for example a plugin whose host framework owns every device allocation and
+ * hands it only fixed input and output buffers, or code that must not block on an
+ * allocation on its hot path).  The paper has no counterpart: this is a library
+ * convenience, not part of the method.
+ *
+ * Same arguments and results as gdn_chunk_prefill on the tensor-core path, minus the
+ * workspace: the scratch is a static device array of GDN_NOALLOC_SCRATCH_BYTES bytes
+ * inside libgdn.so, which every GPU that loads the library holds until exit.
+ *   - Calls no cudaMalloc, cudaFree or other allocating routine.
+ *   - Workloads whose gdn_prefill_workspace_bytes(shape) exceeds the maximum are rejected
+ *     with GDN_ERR_WORKSPACE (about 31 chunks of 64 tokens with 16 QK / 32 V heads, e.g.
+ *     one sequence of up to 1,920 tokens); fp32 I/O or GDN_ALGO_SIMT give
+ *     GDN_ERR_UNSUPPORTED.
+ *   - The first call on each device (with that device current) looks up the array's
+ *     device address once and caches it; make that first call before any stream capture.
+ *   - Every call on a device shares the one array, which keeps the previous call's
+ *     contents; each call clears what must start at zero.  Calls that overlap on the GPU
+ *     (e.g. on unordered streams) race on the array.
+ */
+#define GDN_NOALLOC_SCRATCH_BYTES ((size_t)64 << 20)
+gdn_status gdn_chunk_prefill_noalloc(const void *q, const void *k, const void *v,
+                                     const float *g, const float *beta,
+                                     const float *initial_state, const int32_t *cu_seqlens,
+                                     void *out, float *final_state, const gdn_shape *shape,
+                                     void *stream);
+
+/*
  * Failure-path self-test.  Clears the workspace header, then launches a kernel that waits
  * on a barrier nothing completes, using the same bounded wait as the prefill kernels
  * but with a limit of `limit_us` microseconds (1 .. 2,000,000).  When the limit expires

@@ -24,7 +24,8 @@ STATUS = {0: "GDN_OK", 1: "GDN_ERR_NULL", 2: "GDN_ERR_SHAPE", 3: "GDN_ERR_ALIGN"
           7: "GDN_ERR_CUDA", 8: "GDN_ERR_DEVICE_TIMEOUT", 9: "GDN_ERR_UNSUPPORTED"}
 EXPORTED = ["gdn_prefill_workspace_bytes", "gdn_chunk_prefill", "gdn_chunk_prefill_prep",
             "gdn_chunk_prefill_state", "gdn_decode_step", "gdn_get_device_error",
-            "gdn_selftest_wait_timeout", "gdn_status_string", "gdn_abi_version"]
+            "gdn_selftest_wait_timeout", "gdn_status_string", "gdn_abi_version",
+            "gdn_chunk_prefill_noalloc"]
 
 
 class GdnShape(ctypes.Structure):
@@ -68,6 +69,8 @@ def lib() -> ctypes.CDLL:
             L.gdn_decode_step.argtypes = [vp, vp, vp, fp, fp, fp, vp, ctypes.c_int32, sp, vp]
             L.gdn_get_device_error.restype = ctypes.c_int
             L.gdn_get_device_error.argtypes = [vp, vp]
+            L.gdn_chunk_prefill_noalloc.restype = ctypes.c_int
+            L.gdn_chunk_prefill_noalloc.argtypes = [vp, vp, vp, fp, fp, fp, ip, vp, fp, sp, vp]
             L.gdn_selftest_wait_timeout.restype = ctypes.c_int
             L.gdn_selftest_wait_timeout.argtypes = [vp, ctypes.c_size_t, ctypes.c_uint32, vp]
             L.gdn_status_string.restype = ctypes.c_char_p
@@ -190,6 +193,18 @@ def gdn_decode_step(q, k, v, g, beta, state_inout, out, num_tokens=None, stream=
                                _ptr(out), int(num_tokens), ctypes.byref(shape), _stream(stream))
     if rc != GDN_OK:
         raise GdnError(rc, "gdn_decode_step")
+
+
+def gdn_chunk_prefill_noalloc(q, k, v, g, beta, initial_state, cu_seqlens, out, final_state,
+                              stream=None):
+    """Calls gdn_chunk_prefill_noalloc: the tensor-core prefill with the library's own
+    static scratch instead of a caller workspace, for callers that cannot allocate."""
+    shape = prefill_shape(q, v, cu_seqlens)
+    rc = lib().gdn_chunk_prefill_noalloc(_ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(beta),
+                                         _ptr(initial_state), _ptr(cu_seqlens), _ptr(out),
+                                         _ptr(final_state), ctypes.byref(shape), _stream(stream))
+    if rc != GDN_OK:
+        raise GdnError(rc, "gdn_chunk_prefill_noalloc")
 
 
 def gdn_selftest_wait_timeout(workspace, limit_us=20000, stream=None):
