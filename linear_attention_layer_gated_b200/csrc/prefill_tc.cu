@@ -11,22 +11,31 @@
 // Three kernels, all on the caller's stream:
 //  K0 chunk_table_kernel  cu_seqlens -> per-sequence first chunk id and a (seq, start,
 //                         length) entry per chunk, on the device (no host read).
-//  K1 chunk_prep_kernel   one CTA per (chunk, QK head), all chunks in parallel:
-//                         normalisation, K K^T and Q K^T on tcgen05 (M=128: [K; Q] x K^T),
-//                         decay masks, T by fp32 forward substitution, W^T = K^T (T diag(b gam))^T
-//                         and U^T = V^T (T diag(b))^T on tcgen05, for both V heads of the QK
-//                         head.  Writes bf16 operand images, already in the 128-byte
-//                         swizzled layout the state kernel's MMAs read, to the workspace.
+//  K1 chunk_prep_kernel   one CTA per (chunk, QK head), all chunks in parallel, both V
+//                         heads of the QK head:
+//                         - normalisation; K K^T and Q K^T as one M=128 MMA [K; Q] K^T;
+//                         - decay masks; T = (I + A)^-1 in fp32 by blocks (16x16 diagonal
+//                           inverses by forward substitution, then block products);
+//                         - W and U of both heads as M=128 MMAs [T_0 D_0; T_1 D_1] x (K or V),
+//                           so each thread owns one output row and writes 16-byte chunks;
+//                         - bf16 operand images, already in the 128-byte swizzled layout the
+//                           state kernel's MMAs read, go to the workspace.
 //  K2 chunk_state_kernel  one CTA per (sequence, V head, half of d_v), sequential over the
-//                         sequence's chunks: [X; Y] = [W; diag(gam) Q] S^T (M=128),
-//                         Delta = U - X, O = Y + P Delta (M=128 with a zero upper half),
-//                         S^T <- gam_L S^T + K^T diag(c) Delta; the fp32 state slice lives in
-//                         registers (one d_k row per thread), its bf16 copy in shared memory
-//                         as the next chunk's MMA operand.  Chunk operands stream in with
-//                         double-buffered bulk copies.
-// Every mbarrier wait is bounded (1 s); on expiry the kernel records an error in the
-// workspace header, drains its own copies and MMAs (again bounded), frees Tensor Memory
-// and returns.
+//                         sequence's chunks.  Warp 4 issues the bulk copies (one chunk ahead)
+//                         and the MMAs; warps 0-3 compute.  Per chunk:
+//                           [X; Y] = [W; Q] S^T         (M=128, K=128)
+//                           Delta = U - X, c Delta      (warps 0-1, token rows)
+//                           K^T diag(c) Delta           (M=128: d_k rows)   <- on the chain
+//                           P Delta                     (M=128, zero upper half)
+//                           S^T <- gam_L S^T + K^T diag(c) Delta   (fp32 in registers)
+//                           O = diag(gam) Y + P Delta   (warps 2-3, off the chain)
+//                         Hand-offs between the producer and the compute warps are mbarriers;
+//                         the output accumulators are double-buffered in Tensor Memory so
+//                         the output epilogue stays off the state chain.
+// Every mbarrier wait is bounded (1 s) and, in the state kernel, also gives up as soon as
+// another thread of the CTA has given up; the kernel then records an error in the
+// workspace header, drains its own copies and MMAs (bounded), frees Tensor Memory and
+// returns.
 #include "gdn_internal.cuh"
 #include "sm100.cuh"
 
@@ -39,15 +48,16 @@ constexpr int kThreads = 128;
 constexpr float kInvSqrtD = 0.08838834764831845f;  // 1 / sqrt(128)
 
 // Operand image sizes (bytes)
-constexpr uint32_t kA1Bytes = 32768;   // [W; diag(gam) Q]: 128 rows x 128 (K-major, 2 K-blocks)
-constexpr uint32_t kUBytes = 16384;    // U: 2 halves of d_v, 64 rows x 64 each
-constexpr uint32_t kPBytes = 8192;     // P: 64 rows x 64 (K-major)
-constexpr uint32_t kCvecBytes = 512;   // c_j (64 floats) and gam_L at [64]
+constexpr uint32_t kWBytes = 16384;    // W: 64 token rows x 128 d_k, K-major, [K-block][64 rows]
+constexpr uint32_t kQBytes = 16384;    // normalised Q, same layout (per QK head)
+constexpr uint32_t kUBytes = 16384;    // U: [d_v half][64 rows][64]
+constexpr uint32_t kPBytes = 8192;     // P: 64 rows x 64, K-major
+constexpr uint32_t kCvecBytes = 1024;  // c_j at [0,64), gam_L at [64], gam_r at [128,192)
 constexpr uint32_t kKTBytes = 16384;   // K as an MN-major operand (d_k x chunk)
-constexpr uint32_t kChunkLoadBytes = kA1Bytes + kKTBytes + kPBytes + kUBytes / 2 + kCvecBytes;
+constexpr uint32_t kChunkLoadBytes = kWBytes + kQBytes + kKTBytes + kPBytes + kUBytes / 2 + kCvecBytes;
 
 struct WsLayout {
-    size_t seq_chunk0, table, a1, u, p, cvec, kt, total;
+    size_t seq_chunk0, table, w, u, p, cvec, kt, qn, total;
     long long max_chunks;
 };
 
@@ -61,8 +71,8 @@ __host__ __device__ inline WsLayout ws_layout(int num_seqs, int total_tokens, in
     off = round_up(off + (size_t)(num_seqs + 1) * 4, 1024);
     L.table = off;
     off = round_up(off + (size_t)L.max_chunks * 16, 1024);
-    L.a1 = off;
-    off += (size_t)L.max_chunks * hv * kA1Bytes;
+    L.w = off;
+    off += (size_t)L.max_chunks * hv * kWBytes;
     L.u = off;
     off += (size_t)L.max_chunks * hv * kUBytes;
     L.p = off;
@@ -71,6 +81,8 @@ __host__ __device__ inline WsLayout ws_layout(int num_seqs, int total_tokens, in
     off += (size_t)L.max_chunks * hv * kCvecBytes;
     L.kt = off;
     off += (size_t)L.max_chunks * hk * kKTBytes;
+    L.qn = off;
+    off += (size_t)L.max_chunks * hk * kQBytes;
     L.total = round_up(off, 1024);
     return L;
 }
@@ -133,10 +145,6 @@ __device__ __forceinline__ void unpack8(uint4 u, float* x) {
         x[2 * i + 1] = f.y;
     }
 }
-__device__ __forceinline__ void st_shared_b16(uint32_t addr, float x) {
-    __nv_bfloat16 h = __float2bfloat16_rn(x);
-    asm volatile("st.shared.b16 [%0], %1;" ::"r"(addr), "h"(*reinterpret_cast<uint16_t*>(&h)) : "memory");
-}
 
 __device__ __forceinline__ float sum8(float x) {  // over groups of 8 consecutive lanes
     x += __shfl_xor_sync(0xffffffffu, x, 4);
@@ -154,13 +162,17 @@ __device__ __forceinline__ float warp_inclusive_scan(float x, int lane) {
     return x;
 }
 
+// fp32 64x64 matrix in shared memory, rows of 64 floats; the float4 groups of row R are
+// XOR-permuted by R so that 32 threads writing 32 different rows hit different banks.
+__device__ __forceinline__ int af_idx(int R, int J) { return R * 64 + 4 * ((J >> 2) ^ (R & 15)) + (J & 3); }
+
 // ===================================================================== K1
 // Shared memory map (bytes from a 1024-aligned base):
-constexpr uint32_t kP_GRAM = 0;          // [K; Q] K-major, 32 KB   | later: V images (2 x 16 KB)
-constexpr uint32_t kP_KT = 32768;        // K MN-major, 16 KB
-constexpr uint32_t kP_AF = 49152;        // A fp32, 2 heads x 16 KB | later: W/U staging, head 0
-constexpr uint32_t kP_B = 81920;         // T images: Bw0, Bu0, Bw1, Bu1 (8 KB each) | later: staging, head 1
-constexpr uint32_t kP_SMALL = 114688;    // gates and barriers
+constexpr uint32_t kP_GR = 0;        // [K; Q] K-major (32 KB)  | after the Gram MMA: V images of both heads
+constexpr uint32_t kP_KT = 32768;    // K MN-major (16 KB)
+constexpr uint32_t kP_AF = 49152;    // A / T fp32, 2 heads (32 KB) | then [T0 D0; T1 D1] images for W and U
+constexpr uint32_t kP_XS = 81920;    // block-solve scratch, 2 heads x 3 blocks of 16x16 fp32 (6 KB)
+constexpr uint32_t kP_SMALL = 90112; // gates, barrier, TMEM address
 constexpr uint32_t kPrepSmem = kP_SMALL + 2048 + 1024;
 
 struct PrepSmall {
@@ -171,7 +183,7 @@ struct PrepSmall {
     uint32_t tmem_base;
 };
 
-__global__ void __launch_bounds__(kThreads, 1)
+__global__ void __launch_bounds__(kThreads, 2)
 chunk_prep_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __restrict__ k,
                   const __nv_bfloat16* __restrict__ v, const float* __restrict__ g,
                   const float* __restrict__ beta, unsigned char* ws, int num_seqs,
@@ -180,6 +192,8 @@ chunk_prep_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __re
     unsigned char* sm = reinterpret_cast<unsigned char*>((reinterpret_cast<uintptr_t>(smem_dyn) + 1023) & ~uintptr_t(1023));
     const uint32_t sb = smem_u32(sm);
     PrepSmall& ss = *reinterpret_cast<PrepSmall*>(sm + kP_SMALL);
+    float* af = reinterpret_cast<float*>(sm + kP_AF);   // [head][64][64] (swizzled rows)
+    float* xs = reinterpret_cast<float*>(sm + kP_XS);   // [head][3][16][16]
 
     const WsLayout L = ws_layout(num_seqs, total_tokens, hk, hv);
     int32_t* header = reinterpret_cast<int32_t*>(ws);
@@ -188,12 +202,31 @@ chunk_prep_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __re
     if (cid >= header[1]) return;
     const int4 ent = reinterpret_cast<const int4*>(ws + L.table)[cid];
     const int t0 = ent.y, len = ent.z;
-    const int group = hv / hk;
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    const int h0 = jq * 2;  // the two V heads of this QK head
 
-    // ---- gates of the two V heads, barrier, TMEM
+    // Thread's slice of a row for the row loads: 16 elements = 2 chunks of one 64-wide block.
+    const int sub = tid & 7, kb = sub >> 2, c0 = (sub & 3) * 2;
+    int err = 0;
+    bool ok;
+
+    // ---- 0. issue the q, k row loads (4 passes of 16 rows), gates, TMEM, barrier
+    uint4 kr[4][2], qr[4][2];
+#pragma unroll
+    for (int pass = 0; pass < 4; ++pass) {
+        const int r = pass * 16 + (tid >> 3);
+        if (r < len) {
+            const size_t base = ((size_t)(t0 + r) * hk + jq) * kD + sub * 16;
+            kr[pass][0] = *reinterpret_cast<const uint4*>(k + base);
+            kr[pass][1] = *reinterpret_cast<const uint4*>(k + base + 8);
+            qr[pass][0] = *reinterpret_cast<const uint4*>(q + base);
+            qr[pass][1] = *reinterpret_cast<const uint4*>(q + base + 8);
+        } else {
+            kr[pass][0] = kr[pass][1] = qr[pass][0] = qr[pass][1] = make_uint4(0, 0, 0, 0);
+        }
+    }
     if (warp < 2) {
-        const int h = jq * group + warp;
+        const int h = h0 + warp;
         const float g0 = (lane < len) ? g[(size_t)(t0 + lane) * hv + h] : 0.f;
         const float g1 = (lane + 32 < len) ? g[(size_t)(t0 + lane + 32) * hv + h] : 0.f;
         const float G0 = warp_inclusive_scan(g0, lane);
@@ -217,32 +250,19 @@ chunk_prep_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __re
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = ss.tmem_base;
-    int32_t err = 0;
 
-    unsigned char* a1_base[2];
-    for (int hh = 0; hh < 2; ++hh)
-        a1_base[hh] = ws + L.a1 + ((size_t)cid * hv + jq * group + hh) * kA1Bytes;
-
-    // ---- 1. normalise K and Q rows; K-major [K; Q], MN-major K, diag(gam) Q rows of A1
+    // ---- 1. normalise; [K; Q] K-major and K MN-major in smem; K and Q images to the workspace
     {
-        const int sub = tid & 7;             // 16 consecutive elements of a row
-        const int kb = sub >> 2;             // 64-wide block of the row
-        const int c0 = (sub & 3) * 2;        // first of two 16-byte chunks in the block
+        unsigned char* kt_img = ws + L.kt + ((size_t)cid * hk + jq) * kKTBytes;
+        unsigned char* qn_img = ws + L.qn + ((size_t)cid * hk + jq) * kQBytes;
+#pragma unroll
         for (int pass = 0; pass < 4; ++pass) {
             const int r = pass * 16 + (tid >> 3);
             float kv[16], qv[16];
-            if (r < len) {
-                const size_t base = ((size_t)(t0 + r) * hk + jq) * kD + sub * 16;
-                const uint4* kp = reinterpret_cast<const uint4*>(k + base);
-                const uint4* qp = reinterpret_cast<const uint4*>(q + base);
-                unpack8(kp[0], kv);
-                unpack8(kp[1], kv + 8);
-                unpack8(qp[0], qv);
-                unpack8(qp[1], qv + 8);
-            } else {
-#pragma unroll
-                for (int e = 0; e < 16; ++e) { kv[e] = 0.f; qv[e] = 0.f; }
-            }
+            unpack8(kr[pass][0], kv);
+            unpack8(kr[pass][1], kv + 8);
+            unpack8(qr[pass][0], qv);
+            unpack8(qr[pass][1], qv + 8);
             float ssk = 0.f, ssq = 0.f;
 #pragma unroll
             for (int e = 0; e < 16; ++e) { ssk = fmaf(kv[e], kv[e], ssk); ssq = fmaf(qv[e], qv[e], ssq); }
@@ -254,43 +274,48 @@ chunk_prep_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __re
             for (int cc = 0; cc < 2; ++cc) {
                 const int ch = c0 + cc;
                 const uint4 kp8 = pack8(kv + 8 * cc), qp8 = pack8(qv + 8 * cc);
-                *reinterpret_cast<uint4*>(sm + kP_GRAM + kb * 16384 + sw128(r, ch)) = kp8;
-                *reinterpret_cast<uint4*>(sm + kP_GRAM + kb * 16384 + sw128(64 + r, ch)) = qp8;
+                *reinterpret_cast<uint4*>(sm + kP_GR + kb * 16384 + sw128(r, ch)) = kp8;
+                *reinterpret_cast<uint4*>(sm + kP_GR + kb * 16384 + sw128(64 + r, ch)) = qp8;
                 *reinterpret_cast<uint4*>(sm + kP_KT + kb * 8192 + sw128(r, ch)) = kp8;
-#pragma unroll
-                for (int hh = 0; hh < 2; ++hh) {
-                    const float gm = ss.gam[hh][r];
-                    float t8[8];
-#pragma unroll
-                    for (int e = 0; e < 8; ++e) t8[e] = qv[8 * cc + e] * gm;
-                    *reinterpret_cast<uint4*>(a1_base[hh] + kb * 16384 + sw128(64 + r, ch)) = pack8(t8);
-                }
+                *reinterpret_cast<uint4*>(kt_img + kb * 8192 + sw128(r, ch)) = kp8;
+                *reinterpret_cast<uint4*>(qn_img + kb * 8192 + sw128(r, ch)) = qp8;
             }
         }
     }
     fence_async_smem();
     __syncthreads();
 
-    // ---- 2. Gram: D[0:128, 0:64] = [K; Q] K^T  (M=128, N=64, K=128)
+    // ---- 2. Gram: TMEM[0:128, 0:64] = [K; Q] K^T  (M=128, N=64, K=128); V loads meanwhile
     if (tid == 0) {
         tc_fence_after();
         const uint32_t idesc = idesc_bf16(128, 64, 0, 0);
 #pragma unroll
         for (int s = 0; s < 8; ++s) {
-            const uint32_t a = sb + kP_GRAM + (s >> 2) * 16384 + (s & 3) * 32;
+            const uint32_t a = sb + kP_GR + (s >> 2) * 16384 + (s & 3) * 32;
             mma_bf16(tmem, sdesc_sw128(a, 16, 1024), sdesc_sw128(a, 16, 1024), idesc, s > 0);
         }
         mma_commit(&ss.bar_mma);
-        // K as MN-major operand image -> workspace (read by the state kernel)
-        bulk_s2g(ws + L.kt + ((size_t)cid * hk + jq) * kKTBytes, sm + kP_KT, kKTBytes);
-        bulk_commit();
     }
-    bool ok = mbar_wait(&ss.bar_mma, 0);
-    if (__syncthreads_or(!ok)) { err = 1; goto cleanup; }
-    tc_fence_after();
-
-    // ---- 3. decay masks: A (fp32, smem) from K K^T rows; P (bf16, workspace) from Q K^T rows
     {
+        uint4 vr[2][4][2];
+#pragma unroll
+        for (int hh = 0; hh < 2; ++hh)
+#pragma unroll
+            for (int pass = 0; pass < 4; ++pass) {
+                const int r = pass * 16 + (tid >> 3);
+                if (r < len) {
+                    const uint4* vp = reinterpret_cast<const uint4*>(v + ((size_t)(t0 + r) * hv + h0 + hh) * kD + sub * 16);
+                    vr[hh][pass][0] = vp[0];
+                    vr[hh][pass][1] = vp[1];
+                } else {
+                    vr[hh][pass][0] = vr[hh][pass][1] = make_uint4(0, 0, 0, 0);
+                }
+            }
+        ok = mbar_wait(&ss.bar_mma, 0);
+        if (__syncthreads_or(!ok)) { err = 1; goto cleanup; }
+        tc_fence_after();
+
+        // ---- 3. decay masks: A (fp32, smem) from K K^T rows; P and gate factors to the workspace
         float row[64];
         tmem_ld64(tmem, warp, 0, row);
         const int r = tid & 63;
@@ -298,22 +323,22 @@ chunk_prep_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __re
 #pragma unroll
             for (int hh = 0; hh < 2; ++hh) {
                 const float Gr = ss.G[hh][r], br = ss.b[hh][r];
-                float4* af = reinterpret_cast<float4*>(sm + kP_AF + hh * 16384);
+                float4* a4 = reinterpret_cast<float4*>(af + hh * 4096);
 #pragma unroll
                 for (int m = 0; m < 16; ++m) {
-                    float a4[4];
+                    float t4[4];
 #pragma unroll
                     for (int e = 0; e < 4; ++e) {
                         const int i = 4 * m + e;
-                        a4[e] = (i < r) ? br * expf(Gr - ss.G[hh][i]) * row[i] : 0.f;
+                        t4[e] = (i < r) ? br * expf(Gr - ss.G[hh][i]) * row[i] : 0.f;
                     }
-                    af[r * 16 + (m ^ (r & 15))] = make_float4(a4[0], a4[1], a4[2], a4[3]);
+                    a4[r * 16 + (m ^ (r & 15))] = make_float4(t4[0], t4[1], t4[2], t4[3]);
                 }
             }
         } else {
 #pragma unroll
             for (int hh = 0; hh < 2; ++hh) {
-                const int h = jq * group + hh;
+                const int h = h0 + hh;
                 const float Gr = ss.G[hh][r];
                 unsigned char* pimg = ws + L.p + ((size_t)cid * hv + h) * kPBytes;
 #pragma unroll
@@ -329,79 +354,114 @@ chunk_prep_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __re
                 float* cv = reinterpret_cast<float*>(ws + L.cvec + ((size_t)cid * hv + h) * kCvecBytes);
                 const float Gl = ss.G[hh][len - 1];
                 cv[r] = (r < len) ? expf(Gl - Gr) : 0.f;
+                cv[128 + r] = ss.gam[hh][r];
                 if (r == 0) cv[64] = expf(Gl);
             }
         }
-    }
-    tc_fence_before();
-    __syncthreads();
-
-    // ---- 4. V images (MN-major, into the dead [K; Q] region), then T = (I + A)^-1
-    {
-        const int sub = tid & 7, kb = sub >> 2, c0 = (sub & 3) * 2;
-        for (int hh = 0; hh < 2; ++hh) {
-            const int h = jq * group + hh;
+        // V images (MN-major: token row, d_v contiguous) into the dead [K; Q] region
+#pragma unroll
+        for (int hh = 0; hh < 2; ++hh)
+#pragma unroll
             for (int pass = 0; pass < 4; ++pass) {
-                const int r = pass * 16 + (tid >> 3);
-                uint4 u0 = make_uint4(0, 0, 0, 0), u1 = u0;
-                if (r < len) {
-                    const uint4* vp = reinterpret_cast<const uint4*>(v + ((size_t)(t0 + r) * hv + h) * kD + sub * 16);
-                    u0 = vp[0];
-                    u1 = vp[1];
-                }
-                *reinterpret_cast<uint4*>(sm + kP_GRAM + hh * 16384 + kb * 8192 + sw128(r, c0)) = u0;
-                *reinterpret_cast<uint4*>(sm + kP_GRAM + hh * 16384 + kb * 8192 + sw128(r, c0 + 1)) = u1;
+                const int rr = pass * 16 + (tid >> 3);
+                *reinterpret_cast<uint4*>(sm + kP_GR + hh * 16384 + kb * 8192 + sw128(rr, c0)) = vr[hh][pass][0];
+                *reinterpret_cast<uint4*>(sm + kP_GR + hh * 16384 + kb * 8192 + sw128(rr, c0 + 1)) = vr[hh][pass][1];
             }
-        }
-    }
-    {
-        const int hh = tid >> 6, i = tid & 63;
-        const float4* af = reinterpret_cast<const float4*>(sm + kP_AF + hh * 16384);
-        float x[kChunk];
-#pragma unroll
-        for (int r = 0; r < kChunk; ++r) x[r] = 0.f;
-#pragma unroll
-        for (int r = 0; r < kChunk; ++r) {
-            float a0 = 0.f, a1 = 0.f, a2 = 0.f, a3 = 0.f;
-#pragma unroll
-            for (int m = 0; m < (r + 3) / 4; ++m) {
-                const float4 av = af[r * 16 + (m ^ (r & 15))];
-                a0 = fmaf(av.x, x[4 * m + 0], a0);
-                a1 = fmaf(av.y, x[4 * m + 1], a1);
-                a2 = fmaf(av.z, x[4 * m + 2], a2);
-                a3 = fmaf(av.w, x[4 * m + 3], a3);
-            }
-            x[r] = (r == i) ? 1.f : ((r < i) ? 0.f : -((a0 + a1) + (a2 + a3)));
-        }
-        // B operands (K-major, row r, K index i): T diag(b gam) for W, T diag(b) for U
-        const float bi = ss.b[hh][i], bgi = bi * ss.gam[hh][i];
-        const uint32_t bw = sb + kP_B + hh * 16384, bu = bw + 8192;
-        const uint32_t colo = (uint32_t)(i & 7) * 2;
-#pragma unroll
-        for (int r = 0; r < kChunk; ++r) {
-            const uint32_t o = sw128(r, i >> 3) + colo;
-            st_shared_b16(bw + o, x[r] * bgi);
-            st_shared_b16(bu + o, x[r] * bi);
-        }
     }
     fence_async_smem();
     tc_fence_before();
     __syncthreads();
 
-    // ---- 5. W^T = K^T (T diag(b gam))^T, U^T = V^T (T diag(b))^T  (M=128, N=64, K=64 each)
+    // ---- 4. T = (I + A)^-1 per head, by 16x16 blocks, in place in `af`
+    {
+        // 4a. diagonal blocks: thread = (head, block, column) forward substitution
+        const int hh = tid >> 6, blk = (tid >> 4) & 3, i = tid & 15;
+        const float* A = af + hh * 4096;
+        float x[16];
+#pragma unroll
+        for (int r = 0; r < 16; ++r) {
+            float acc = 0.f;
+#pragma unroll
+            for (int j = 0; j < r; ++j) acc = fmaf(A[af_idx(blk * 16 + r, blk * 16 + j)], x[j], acc);
+            x[r] = (r == i) ? 1.f : ((r < i) ? 0.f : -acc);
+        }
+        __syncthreads();
+#pragma unroll
+        for (int r = 0; r < 16; ++r) af[hh * 4096 + af_idx(blk * 16 + r, blk * 16 + i)] = x[r];
+        __syncthreads();
+    }
+    // 4b. block rows: X = sum_{k=bj}^{bi-1} A_{bi,k} T_{k,bj};  T_{bi,bj} = -Dinv_bi X
+#pragma unroll 1
+    for (int bi = 1; bi < 4; ++bi) {
+        const int hh = tid >> 6, l = tid & 63;
+        float* A = af + hh * 4096;
+        float* X = xs + hh * 768;
+        for (int o = l; o < 256 * bi; o += 64) {
+            const int bj = o >> 8, rr = (o >> 4) & 15, cc = o & 15;
+            const int R = bi * 16 + rr, C = bj * 16 + cc;
+            float acc = 0.f;
+            for (int kb2 = bj; kb2 < bi; ++kb2) {
+#pragma unroll
+                for (int m = 0; m < 16; ++m)
+                    acc = fmaf(A[af_idx(R, kb2 * 16 + m)], A[af_idx(kb2 * 16 + m, C)], acc);
+            }
+            X[o] = acc;
+        }
+        __syncthreads();
+        for (int o = l; o < 256 * bi; o += 64) {
+            const int bj = o >> 8, rr = (o >> 4) & 15, cc = o & 15;
+            float acc = 0.f;
+#pragma unroll
+            for (int m = 0; m < 16; ++m)
+                acc = fmaf(A[af_idx(bi * 16 + rr, bi * 16 + m)], X[(bj << 8) + (m << 4) + cc], acc);
+            A[af_idx(bi * 16 + rr, bj * 16 + cc)] = -acc;
+        }
+        __syncthreads();
+    }
+
+    // ---- 5. MMA operand images [T_0 diag(b_0 gam_0); T_1 diag(b_1 gam_1)] and [T_0 diag(b_0); ...]
+    {
+        const int hh = tid >> 6, r = tid & 63;
+        const float4* t4 = reinterpret_cast<const float4*>(af + hh * 4096);
+        uint4 wrow[8], urow[8];
+#pragma unroll
+        for (int ch = 0; ch < 8; ++ch) {
+            float w8[8], u8[8];
+#pragma unroll
+            for (int half4 = 0; half4 < 2; ++half4) {
+                const int m = 2 * ch + half4;   // float4 group: columns 4m .. 4m+3
+                const float4 tv = t4[r * 16 + (m ^ (r & 15))];
+                const float tt[4] = {tv.x, tv.y, tv.z, tv.w};
+#pragma unroll
+                for (int e = 0; e < 4; ++e) {
+                    const int j = 4 * m + e;
+                    u8[4 * half4 + e] = tt[e] * ss.b[hh][j];
+                    w8[4 * half4 + e] = u8[4 * half4 + e] * ss.gam[hh][j];
+                }
+            }
+            wrow[ch] = pack8(w8);
+            urow[ch] = pack8(u8);
+        }
+        __syncthreads();
+#pragma unroll
+        for (int ch = 0; ch < 8; ++ch) {
+            *reinterpret_cast<uint4*>(sm + kP_AF + sw128(tid, ch)) = wrow[ch];
+            *reinterpret_cast<uint4*>(sm + kP_AF + 16384 + sw128(tid, ch)) = urow[ch];
+        }
+    }
+    fence_async_smem();
+    __syncthreads();
+
+    // ---- 6. W (both heads) and U of head 0:  D[:, 0:128] = A_W K,  D[:, 128:256] = A_U V_0
     if (tid == 0) {
         tc_fence_after();
-        const uint32_t idesc = idesc_bf16(128, 64, 1, 0);
-        for (int hh = 0; hh < 2; ++hh) {
-            const uint32_t bw = sb + kP_B + hh * 16384, bu = bw + 8192;
-            const uint32_t vimg = sb + kP_GRAM + hh * 16384;
+        const uint32_t idesc = idesc_bf16(128, 128, 0, 1);
 #pragma unroll
-            for (int s = 0; s < 4; ++s) {
-                mma_bf16(tmem + 128 * hh, sdesc_sw128(sb + kP_KT + s * 2048, 8192, 1024),
-                         sdesc_sw128(bw + s * 32, 16, 1024), idesc, s > 0);
-                mma_bf16(tmem + 128 * hh + 64, sdesc_sw128(vimg + s * 2048, 8192, 1024),
-                         sdesc_sw128(bu + s * 32, 16, 1024), idesc, s > 0);
-            }
+        for (int s = 0; s < 4; ++s) {
+            mma_bf16(tmem, sdesc_sw128(sb + kP_AF + s * 32, 16, 1024),
+                     sdesc_sw128(sb + kP_KT + s * 2048, 8192, 1024), idesc, s > 0);
+            mma_bf16(tmem + 128, sdesc_sw128(sb + kP_AF + 16384 + s * 32, 16, 1024),
+                     sdesc_sw128(sb + kP_GR + s * 2048, 8192, 1024), idesc, s > 0);
         }
         mma_commit(&ss.bar_mma);
     }
@@ -409,38 +469,59 @@ chunk_prep_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __re
     if (__syncthreads_or(!ok)) { err = 1; goto cleanup; }
     tc_fence_after();
 
-    // ---- 6. epilogue: W rows 0..63 of A1 and U, staged K-major, bulk-stored
-    for (int hh = 0; hh < 2; ++hh) {
-        const int h = jq * group + hh;
-        unsigned char* stage = sm + (hh == 0 ? kP_AF : kP_B);
-        const int t = tid;  // TMEM lane = d_k (for W) or d_v (for U) index
-        const uint32_t so = (uint32_t)(t >> 6) * 8192, ch = (uint32_t)(t & 63) >> 3, colo = (uint32_t)(t & 7) * 2;
+    // ---- 7. epilogue: accumulator row r' is row r' % 64 of head r' / 64
+    {
+        const int hh = tid >> 6, r = tid & 63, h = h0 + hh;
+        unsigned char* wimg = ws + L.w + ((size_t)cid * hv + h) * kWBytes;
+        unsigned char* uimg = ws + L.u + ((size_t)cid * hv + h) * kUBytes;
         float col[64];
-        tmem_ld64(tmem, warp, 128 * hh, col);
 #pragma unroll
-        for (int r = 0; r < kChunk; ++r) st_shared_b16(smem_u32(stage) + so + sw128(r, ch) + colo, col[r]);
-        tmem_ld64(tmem, warp, 128 * hh + 64, col);
+        for (int half = 0; half < 2; ++half) {
+            tmem_ld64(tmem, warp, 64 * half, col);
 #pragma unroll
-        for (int r = 0; r < kChunk; ++r) st_shared_b16(smem_u32(stage) + 16384 + so + sw128(r, ch) + colo, col[r]);
-        fence_async_smem();
+            for (int ch = 0; ch < 8; ++ch)
+                *reinterpret_cast<uint4*>(wimg + half * 8192 + sw128(r, ch)) = pack8(col + 8 * ch);
+        }
+        if (hh == 0) {
+#pragma unroll
+            for (int half = 0; half < 2; ++half) {
+                tmem_ld64(tmem, warp, 128 + 64 * half, col);
+#pragma unroll
+                for (int ch = 0; ch < 8; ++ch)
+                    *reinterpret_cast<uint4*>(uimg + half * 8192 + sw128(r, ch)) = pack8(col + 8 * ch);
+            }
+        }
+        tc_fence_before();
         __syncthreads();
-        if (tid == 0) {
-            unsigned char* a1 = ws + L.a1 + ((size_t)cid * hv + h) * kA1Bytes;
-            bulk_s2g(a1, stage, 8192);              // W rows, d_k 0..63
-            bulk_s2g(a1 + 16384, stage + 8192, 8192);  // W rows, d_k 64..127
-            bulk_s2g(ws + L.u + ((size_t)cid * hv + h) * kUBytes, stage + 16384, kUBytes);
-            bulk_commit();
+        if (tid == 0) {  // U of head 1: D[:, 128:256] = A_U V_1 (rows 64..127 are head 1's)
+            tc_fence_after();
+            const uint32_t idesc = idesc_bf16(128, 128, 0, 1);
+#pragma unroll
+            for (int s = 0; s < 4; ++s)
+                mma_bf16(tmem + 128, sdesc_sw128(sb + kP_AF + 16384 + s * 32, 16, 1024),
+                         sdesc_sw128(sb + kP_GR + 16384 + s * 2048, 8192, 1024), idesc, s > 0);
+            mma_commit(&ss.bar_mma);
+        }
+        ok = mbar_wait(&ss.bar_mma, 0);
+        if (__syncthreads_or(!ok)) { err = 1; goto cleanup; }
+        tc_fence_after();
+        if (hh == 1) {
+#pragma unroll
+            for (int half = 0; half < 2; ++half) {
+                tmem_ld64(tmem, warp, 128 + 64 * half, col);
+#pragma unroll
+                for (int ch = 0; ch < 8; ++ch)
+                    *reinterpret_cast<uint4*>(uimg + half * 8192 + sw128(r, ch)) = pack8(col + 8 * ch);
+            }
         }
     }
 
 cleanup:
-    if (err) {
-        if (tid == 0) {
-            atomicOr(header, 1);
-            mma_commit(&ss.bar_mma);  // all MMAs issued so far complete before TMEM is freed
-        }
+    if (err && tid == 0) {
+        atomicOr(header, 1);
+        mma_commit(&ss.bar_mma);  // MMAs issued so far complete before TMEM is freed
+        mbar_wait(&ss.bar_mma, 1);
     }
-    if (tid == 0) bulk_wait_all();
     tc_fence_before();
     __syncthreads();
     if (warp == 3) {
@@ -450,38 +531,74 @@ cleanup:
 }
 
 // ===================================================================== K2
-constexpr uint32_t kS_A1 = 0, kS_KT = 32768, kS_A2 = 49152, kS_U = 65536, kS_CV = 73728;
+constexpr int kStateThreads = 160;                  // warps 0-3 compute, warp 4 copies + MMAs
+constexpr uint32_t kS_A1 = 0;                       // [W; Q] K-major, 2 K-blocks of 128 rows (32 KB)
+constexpr uint32_t kS_KT = 32768;                   // K MN-major (16 KB)
+constexpr uint32_t kS_A2 = 49152;                   // [0; P] K-major (16 KB)
+constexpr uint32_t kS_U = 65536;                    // U, this CTA's d_v half (8 KB)
+constexpr uint32_t kS_CV = 73728;                   // gate factors (1 KB)
 constexpr uint32_t kS_BUF = 74752;                  // one chunk buffer (73 KB)
 constexpr uint32_t kS_B1 = 2 * kS_BUF;              // S slice bf16, MN-major (16 KB)
 constexpr uint32_t kS_B2 = kS_B1 + 16384;           // Delta, MN-major (8 KB)
 constexpr uint32_t kS_B3 = kS_B2 + 8192;            // diag(c) Delta, MN-major (8 KB)
 constexpr uint32_t kS_SMALL = kS_B3 + 8192;
 constexpr uint32_t kStateSmem = kS_SMALL + 256 + 1024;
+// Tensor Memory columns
+constexpr uint32_t kT_XY = 0;     // [X; Y] of chunk parity p at kT_XY + 64 p
+constexpr uint32_t kT_PD = 128;   // P Delta of chunk parity p at kT_PD + 64 p
+constexpr uint32_t kT_SA = 256;   // K^T diag(c) Delta
 
 struct StateSmall {
     uint64_t full[2];
-    uint64_t bar_mma1, bar_mma23;
+    uint64_t b1, b23, mma1, mma2, mma3;
     uint32_t tmem_base;
+    int abort_flag;
 };
+
+// Bounded wait that also returns (false) as soon as another thread has given up.
+__device__ __forceinline__ bool wait_or_abort(uint64_t* bar, uint32_t parity, volatile int* abort_flag,
+                                              int32_t* header) {
+    if (mbar_try_wait(bar, parity)) return true;
+    const uint64_t t0 = global_timer_ns();
+    while (true) {
+        if (mbar_try_wait(bar, parity)) return true;
+        if (*abort_flag) return false;
+        if (global_timer_ns() - t0 > kWaitLimitNs) {
+            *abort_flag = 1;
+            atomicOr(header, 1);
+            return false;
+        }
+    }
+}
+
+__device__ __forceinline__ void mbar_arrive(uint64_t* bar) {
+    asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_u32(bar)) : "memory");
+}
 
 __device__ __forceinline__ void issue_chunk_loads(unsigned char* buf, uint64_t* bar, const unsigned char* ws,
                                                   const WsLayout& L, int cid, int h, int jq, int half,
                                                   int hk, int hv) {
     mbar_arrive_expect_tx(bar, kChunkLoadBytes);
-    bulk_g2s(buf + kS_A1, ws + L.a1 + ((size_t)cid * hv + h) * kA1Bytes, kA1Bytes, bar);
+    const unsigned char* w = ws + L.w + ((size_t)cid * hv + h) * kWBytes;
+    const unsigned char* qn = ws + L.qn + ((size_t)cid * hk + jq) * kQBytes;
+    bulk_g2s(buf + kS_A1, w, 8192, bar);                  // W rows, d_k 0..63
+    bulk_g2s(buf + kS_A1 + 8192, qn, 8192, bar);          // Q rows, d_k 0..63
+    bulk_g2s(buf + kS_A1 + 16384, w + 8192, 8192, bar);   // W rows, d_k 64..127
+    bulk_g2s(buf + kS_A1 + 24576, qn + 8192, 8192, bar);  // Q rows, d_k 64..127
     bulk_g2s(buf + kS_KT, ws + L.kt + ((size_t)cid * hk + jq) * kKTBytes, kKTBytes, bar);
     bulk_g2s(buf + kS_A2 + 8192, ws + L.p + ((size_t)cid * hv + h) * kPBytes, kPBytes, bar);
     bulk_g2s(buf + kS_U, ws + L.u + ((size_t)cid * hv + h) * kUBytes + half * (kUBytes / 2), kUBytes / 2, bar);
     bulk_g2s(buf + kS_CV, ws + L.cvec + ((size_t)cid * hv + h) * kCvecBytes, kCvecBytes, bar);
 }
 
-__global__ void __launch_bounds__(kThreads, 1)
+__global__ void __launch_bounds__(kStateThreads, 1)
 chunk_state_kernel(const float* s0, const int32_t* __restrict__ cu, __nv_bfloat16* __restrict__ out,
                    float* sT, unsigned char* ws, int num_seqs, int total_tokens, int hk, int hv) {
     extern __shared__ unsigned char smem_dyn[];
     unsigned char* sm = reinterpret_cast<unsigned char*>((reinterpret_cast<uintptr_t>(smem_dyn) + 1023) & ~uintptr_t(1023));
     const uint32_t sb = smem_u32(sm);
     StateSmall& ss = *reinterpret_cast<StateSmall*>(sm + kS_SMALL);
+    volatile int* abort_flag = &ss.abort_flag;
 
     const WsLayout L = ws_layout(num_seqs, total_tokens, hk, hv);
     int32_t* header = reinterpret_cast<int32_t*>(ws);
@@ -489,157 +606,187 @@ chunk_state_kernel(const float* s0, const int32_t* __restrict__ cu, __nv_bfloat1
     const int h = (blockIdx.x >> 1) % hv;
     const int n = (blockIdx.x >> 1) / hv;
     const int jq = h / (hv / hk);
-    const int tid = threadIdx.x, warp = tid >> 5;
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int32_t* seq_chunk0 = reinterpret_cast<const int32_t*>(ws + L.seq_chunk0);
     const int cs = seq_chunk0[n], nch = seq_chunk0[n + 1] - cs;
     const int t_begin = cu[n], t_end = cu[n + 1];
 
-    // zero the upper (unused) 64 rows of both P operands
-    for (int i = tid; i < 2 * 512; i += kThreads) {
+    // zero the upper (unused) 64 rows of both [0; P] operands
+    for (int i = tid; i < 2 * 512; i += kStateThreads) {
         const int b = i >> 9, o = (i & 511) * 16;
         *reinterpret_cast<uint4*>(sm + b * kS_BUF + kS_A2 + o) = make_uint4(0, 0, 0, 0);
     }
     if (warp == 0) {
-        tmem_alloc(&ss.tmem_base, 128);
+        tmem_alloc(&ss.tmem_base, 512);
         tmem_relinquish();
     }
     if (tid == 0) {
         mbar_init(&ss.full[0], 1);
         mbar_init(&ss.full[1], 1);
-        mbar_init(&ss.bar_mma1, 1);
-        mbar_init(&ss.bar_mma23, 1);
+        mbar_init(&ss.b1, 128);
+        mbar_init(&ss.b23, 64);
+        mbar_init(&ss.mma1, 1);
+        mbar_init(&ss.mma2, 1);
+        mbar_init(&ss.mma3, 1);
+        ss.abort_flag = 0;
         fence_mbar_init();
     }
-
-    // fp32 state slice: thread t owns S[half*64 + m][t], m = 0..63 (column t of S)
-    const int t = tid;
-    float S[64];
-    const size_t sbase = ((size_t)n * hv + h) * kD * kD + (size_t)(half * 64) * kD + t;
-#pragma unroll
-    for (int m = 0; m < 64; ++m) S[m] = s0 ? s0[sbase + (size_t)m * kD] : 0.f;
-#pragma unroll
-    for (int ch = 0; ch < 8; ++ch)
-        *reinterpret_cast<uint4*>(sm + kS_B1 + sw128(t, ch)) = pack8(S + 8 * ch);
     fence_async_smem();
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = ss.tmem_base;
-    if (tid == 0) {
-        for (int kk = 0; kk < 2 && kk < nch; ++kk)
-            issue_chunk_loads(sm + kk * kS_BUF, &ss.full[kk], ws, L, cs + kk, h, jq, half, hk, hv);
-    }
 
-    const uint32_t id_xy = idesc_bf16(128, 64, 0, 1);   // A K-major, B MN-major
-    const uint32_t id_s = idesc_bf16(128, 64, 1, 1);    // A MN-major, B MN-major
-    int err = 0;
-    int kk = 0;
-    for (; kk < nch; ++kk) {
-        const int b = kk & 1;
-        unsigned char* buf = sm + b * kS_BUF;
-        const uint32_t bufa = sb + b * kS_BUF;
-        const int t0 = t_begin + kk * kChunk;
-        const int len = min(kChunk, t_end - t0);
-        bool ok = mbar_wait(&ss.full[b], (kk >> 1) & 1);
-        if (__syncthreads_or(!ok)) { err = 1; break; }
-        const float* cvec = reinterpret_cast<const float*>(buf + kS_CV);
-        const float gl = cvec[64];
-
-        // [X; Y] = [W; diag(gam) Q] S^T
-        if (tid == 0) {
-            tc_fence_after();
-#pragma unroll
-            for (int s = 0; s < 8; ++s)
-                mma_bf16(tmem, sdesc_sw128(bufa + kS_A1 + (s >> 2) * 16384 + (s & 3) * 32, 16, 1024),
-                         sdesc_sw128(sb + kS_B1 + s * 2048, 16384, 1024), id_xy, s > 0);
-            mma_commit(&ss.bar_mma1);
-        }
-        ok = mbar_wait(&ss.bar_mma1, kk & 1);
-        if (__syncthreads_or(!ok)) { err = 1; break; }
-        tc_fence_after();
-
-        if (warp < 2) {  // Delta = U - X for token row r; write Delta and diag(c) Delta
-            const int r = tid;
-            float x[64];
-            tmem_ld64(tmem, warp, 0, x);
-            const float cr = cvec[r];
-#pragma unroll
-            for (int ch = 0; ch < 8; ++ch) {
-                float u8[8], d8[8], c8[8];
-                unpack8(*reinterpret_cast<const uint4*>(buf + kS_U + sw128(r, ch)), u8);
-#pragma unroll
-                for (int e = 0; e < 8; ++e) {
-                    d8[e] = u8[e] - x[8 * ch + e];
-                    c8[e] = d8[e] * cr;
+    if (warp == 4) {
+        // ------------------------------------------------ producer: bulk copies and MMAs
+        if (lane == 0) {
+            const uint32_t id_xy = idesc_bf16(128, 64, 0, 1);  // A K-major, B MN-major
+            const uint32_t id_s = idesc_bf16(128, 64, 1, 1);   // A MN-major, B MN-major
+            int issued = 0;  // chunks whose loads have been issued
+            if (nch > 0) {
+                issue_chunk_loads(sm, &ss.full[0], ws, L, cs, h, jq, half, hk, hv);
+                issued = 1;
+            }
+            int c = 0;
+            for (; c < nch; ++c) {
+                const int b = c & 1;
+                const uint32_t bufa = sb + b * kS_BUF;
+                if (!wait_or_abort(&ss.b1, c & 1, abort_flag, header)) break;   // B1 = S(c) written
+                if (c + 1 < nch) {
+                    // the other buffer held chunk c-1; its last reader, P Delta of c-1, is done
+                    if (c >= 1 && !wait_or_abort(&ss.mma2, (c - 1) & 1, abort_flag, header)) break;
+                    issue_chunk_loads(sm + (b ^ 1) * kS_BUF, &ss.full[b ^ 1], ws, L, cs + c + 1, h, jq,
+                                      half, hk, hv);
+                    issued = c + 2;
                 }
-                *reinterpret_cast<uint4*>(sm + kS_B2 + sw128(r, ch)) = pack8(d8);
-                *reinterpret_cast<uint4*>(sm + kS_B3 + sw128(r, ch)) = pack8(c8);
+                if (!wait_or_abort(&ss.full[b], (c >> 1) & 1, abort_flag, header)) break;
+                tc_fence_after();
+#pragma unroll
+                for (int s = 0; s < 8; ++s)
+                    mma_bf16(tmem + kT_XY + 64 * b,
+                             sdesc_sw128(bufa + kS_A1 + (s >> 2) * 16384 + (s & 3) * 32, 16, 1024),
+                             sdesc_sw128(sb + kS_B1 + s * 2048, 16384, 1024), id_xy, s > 0);
+                mma_commit(&ss.mma1);
+                if (!wait_or_abort(&ss.b23, c & 1, abort_flag, header)) break;  // Delta(c) written
+                tc_fence_after();
+#pragma unroll
+                for (int s = 0; s < 4; ++s)
+                    mma_bf16(tmem + kT_SA, sdesc_sw128(bufa + kS_KT + s * 2048, 8192, 1024),
+                             sdesc_sw128(sb + kS_B3 + s * 2048, 8192, 1024), id_s, s > 0);
+                mma_commit(&ss.mma3);
+#pragma unroll
+                for (int s = 0; s < 4; ++s)
+                    mma_bf16(tmem + kT_PD + 64 * b, sdesc_sw128(bufa + kS_A2 + s * 32, 16, 1024),
+                             sdesc_sw128(sb + kS_B2 + s * 2048, 8192, 1024), id_xy, s > 0);
+                mma_commit(&ss.mma2);
+            }
+            if (*abort_flag) {
+                // drain: every MMA issued so far, then every bulk copy still in flight
+                mma_commit(&ss.mma1);
+                mbar_wait(&ss.mma1, c & 1);
+                for (int j = c; j < issued; ++j) mbar_wait(&ss.full[j & 1], (j >> 1) & 1);
             }
         }
+    } else {
+        // ------------------------------------------------ compute warps 0-3
+        // fp32 state slice: thread t owns S[half*64 + m][t], m = 0..63 (column t of S)
+        const int t = tid;
+        float S[64];
+        const size_t sbase = ((size_t)n * hv + h) * kD * kD + (size_t)(half * 64) * kD + t;
+#pragma unroll
+        for (int m = 0; m < 64; ++m) S[m] = s0 ? s0[sbase + (size_t)m * kD] : 0.f;
+#pragma unroll
+        for (int ch = 0; ch < 8; ++ch)
+            *reinterpret_cast<uint4*>(sm + kS_B1 + sw128(t, ch)) = pack8(S + 8 * ch);
         fence_async_smem();
         tc_fence_before();
-        __syncthreads();
+        mbar_arrive(&ss.b1);
 
-        // Y += P Delta (rows 64..127 of the accumulator), S-update = K^T diag(c) Delta
-        if (tid == 0) {
+        const int r = tid & 63;  // token row (warps 0-1: Delta rows; warps 2-3: output rows)
+        for (int c = 0; c < nch; ++c) {
+            const int b = c & 1;
+            unsigned char* buf = sm + b * kS_BUF;
+            if (!wait_or_abort(&ss.full[b], (c >> 1) & 1, abort_flag, header)) break;
+            const float* cvec = reinterpret_cast<const float*>(buf + kS_CV);
+            const float gl = cvec[64];
+            const float crow = (warp < 2) ? cvec[r] : cvec[128 + r];  // c_r, or gam_r for outputs
+
+            if (warp < 2) {  // Delta = U - X for token row r; write Delta and diag(c) Delta
+                if (c >= 1 && !wait_or_abort(&ss.mma2, (c - 1) & 1, abort_flag, header)) break;
+                if (!wait_or_abort(&ss.mma1, c & 1, abort_flag, header)) break;
+                tc_fence_after();
+                float x[64];
+                tmem_ld64(tmem, warp, kT_XY + 64 * b, x);
+#pragma unroll
+                for (int ch = 0; ch < 8; ++ch) {
+                    float u8[8], d8[8], c8[8];
+                    unpack8(*reinterpret_cast<const uint4*>(buf + kS_U + sw128(r, ch)), u8);
+#pragma unroll
+                    for (int e = 0; e < 8; ++e) {
+                        d8[e] = u8[e] - x[8 * ch + e];
+                        c8[e] = d8[e] * crow;
+                    }
+                    *reinterpret_cast<uint4*>(sm + kS_B2 + sw128(r, ch)) = pack8(d8);
+                    *reinterpret_cast<uint4*>(sm + kS_B3 + sw128(r, ch)) = pack8(c8);
+                }
+                fence_async_smem();
+                tc_fence_before();
+                mbar_arrive(&ss.b23);
+            }
+            // state update S^T <- gam_L S^T + K^T diag(c) Delta (this thread: d_k row t)
+            if (!wait_or_abort(&ss.mma3, c & 1, abort_flag, header)) break;
             tc_fence_after();
+            {
+                float acc[64];
+                tmem_ld64(tmem, warp, kT_SA, acc);
 #pragma unroll
-            for (int s = 0; s < 4; ++s)
-                mma_bf16(tmem, sdesc_sw128(bufa + kS_A2 + s * 32, 16, 1024),
-                         sdesc_sw128(sb + kS_B2 + s * 2048, 8192, 1024), id_xy, 1);
+                for (int m = 0; m < 64; ++m) S[m] = fmaf(gl, S[m], acc[m]);
 #pragma unroll
-            for (int s = 0; s < 4; ++s)
-                mma_bf16(tmem + 64, sdesc_sw128(bufa + kS_KT + s * 2048, 8192, 1024),
-                         sdesc_sw128(sb + kS_B3 + s * 2048, 8192, 1024), id_s, s > 0);
-            mma_commit(&ss.bar_mma23);
-        }
-        ok = mbar_wait(&ss.bar_mma23, kk & 1);
-        if (__syncthreads_or(!ok)) { err = 1; break; }
-        tc_fence_after();
-        if (tid == 0 && kk + 2 < nch)
-            issue_chunk_loads(buf, &ss.full[b], ws, L, cs + kk + 2, h, jq, half, hk, hv);
+                for (int ch = 0; ch < 8; ++ch)
+                    *reinterpret_cast<uint4*>(sm + kS_B1 + sw128(t, ch)) = pack8(S + 8 * ch);
+            }
+            fence_async_smem();
+            tc_fence_before();
+            mbar_arrive(&ss.b1);
 
-        if (warp >= 2) {  // outputs of token row r
-            const int r = tid - 64;
-            float y[64];
-            tmem_ld64(tmem, warp, 0, y);
-            if (r < len) {
+            if (warp >= 2) {  // outputs of token row r: O = gam_r Y + P Delta
+                if (!wait_or_abort(&ss.mma2, c & 1, abort_flag, header)) break;
+                tc_fence_after();
+                const int t0 = t_begin + c * kChunk;
+                const int len = min(kChunk, t_end - t0);
                 uint4* op = reinterpret_cast<uint4*>(out + ((size_t)(t0 + r) * hv + h) * kD + half * 64);
 #pragma unroll
-                for (int ch = 0; ch < 8; ++ch) op[ch] = pack8(y + 8 * ch);
+                for (int part = 0; part < 2; ++part) {  // 32 columns at a time
+                    float y[32], pd[32];
+                    const uint32_t lq = (uint32_t)(warp & 3) * 32u << 16;
+                    tmem_ld16(tmem + lq + kT_XY + 64 * b + 32 * part, y);
+                    tmem_ld16(tmem + lq + kT_XY + 64 * b + 32 * part + 16, y + 16);
+                    tmem_ld16(tmem + lq + kT_PD + 64 * b + 32 * part, pd);
+                    tmem_ld16(tmem + lq + kT_PD + 64 * b + 32 * part + 16, pd + 16);
+                    tmem_ld_wait();
+                    if (r < len) {
+#pragma unroll
+                        for (int ch = 0; ch < 4; ++ch) {
+                            float o8[8];
+#pragma unroll
+                            for (int e = 0; e < 8; ++e) o8[e] = fmaf(crow, y[8 * ch + e], pd[8 * ch + e]);
+                            op[4 * part + ch] = pack8(o8);
+                        }
+                    }
+                }
+                tc_fence_before();
             }
         }
-        {
-            float acc[64];
-            tmem_ld64(tmem, warp, 64, acc);
+        if (!*abort_flag && sT) {
 #pragma unroll
-            for (int m = 0; m < 64; ++m) S[m] = fmaf(gl, S[m], acc[m]);
-#pragma unroll
-            for (int ch = 0; ch < 8; ++ch)
-                *reinterpret_cast<uint4*>(sm + kS_B1 + sw128(t, ch)) = pack8(S + 8 * ch);
+            for (int m = 0; m < 64; ++m) sT[sbase + (size_t)m * kD] = S[m];
         }
-        fence_async_smem();
-        tc_fence_before();
-        __syncthreads();
-    }
-
-    if (err) {
-        if (tid == 0) {
-            atomicOr(header, 1);
-            // drain: MMAs issued so far, and chunk loads still in flight (bounded waits)
-            mma_commit(&ss.bar_mma1);
-            mbar_wait(&ss.bar_mma1, kk & 1);
-            for (int j = kk; j < nch && j < kk + 2; ++j) mbar_wait(&ss.full[j & 1], (j >> 1) & 1);
-        }
-    } else if (sT) {
-#pragma unroll
-        for (int m = 0; m < 64; ++m) sT[sbase + (size_t)m * kD] = S[m];
     }
     tc_fence_before();
     __syncthreads();
     if (warp == 0) {
         tc_fence_after();
-        tmem_dealloc(tmem, 128);
+        tmem_dealloc(tmem, 512);
     }
 }
 
@@ -675,7 +822,7 @@ cudaError_t launch_prefill_tc_state(const float* s0, const int32_t* cu, void* ou
     cudaError_t e = cudaFuncSetAttribute(chunk_state_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          (int)kStateSmem);
     if (e != cudaSuccess) return e;
-    chunk_state_kernel<<<(unsigned)num_seqs * hv * 2, kThreads, kStateSmem, stream>>>(
+    chunk_state_kernel<<<(unsigned)num_seqs * hv * 2, kStateThreads, kStateSmem, stream>>>(
         s0, cu, (__nv_bfloat16*)out, sT, static_cast<unsigned char*>(workspace), num_seqs,
         total_tokens, hk, hv);
     return cudaGetLastError();
