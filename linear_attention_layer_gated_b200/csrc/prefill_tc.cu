@@ -14,21 +14,23 @@
 //  K1 chunk_prep_kernel   one CTA per (chunk, QK head), all chunks in parallel, both V
 //                         heads of the QK head:
 //                         - normalisation; K K^T and Q K^T as one M=128 MMA [K; Q] K^T;
-//                         - decay masks; T = (I + A)^-1 in fp32 by blocks (16x16 diagonal
-//                           inverses by forward substitution, then block products);
+//                         - decay masks A and P; T = (I + A)^-1 in fp32 by forward substitution,
+//                           one column per thread (128 threads = 64 columns x 2 heads);
 //                         - W and U of both heads as M=128 MMAs [T_0 D_0; T_1 D_1] x (K or V),
 //                           so each thread owns one output row and writes 16-byte chunks;
 //                         - bf16 operand images, already in the 128-byte swizzled layout the
-//                           state kernel's MMAs read, go to the workspace.
+//                           state kernel's MMAs read, go to the workspace, with the gate
+//                           factors (c, gam) of each V head.
 //  K2 chunk_state_kernel  one CTA per (sequence, V head, half of d_v), sequential over the
-//                         sequence's chunks.  Warp 4 issues the bulk copies (one chunk ahead)
-//                         and the MMAs; warps 0-3 compute.  Per chunk:
-//                           [X; Y] = [W; Q] S^T         (M=128, K=128)
-//                           Delta = U - X, c Delta      (warps 0-1, token rows)
-//                           K^T diag(c) Delta           (M=128: d_k rows)   <- on the chain
-//                           P Delta                     (M=128, zero upper half)
+//                         sequence's chunks.  Warp 8 issues the bulk copies (two chunks
+//                         ahead, three buffers) and the MMAs; warps 0-7 compute, each warp on
+//                         32 of the 64 d_v columns of its TMEM lane quarter.  Per chunk:
+//                           [X; Y] = [W; Q] S^T          (M=128)            <- on the chain
+//                           Delta = U - X, c Delta       (lanes 0-63: token rows)
+//                           K^T diag(c) Delta            (M=128: d_k rows)  <- on the chain
 //                           S^T <- gam_L S^T + K^T diag(c) Delta   (fp32 in registers)
-//                           O = diag(gam) Y + P Delta   (warps 2-3, off the chain)
+//                           P Delta                      (M=128 operand [U; P]: rows 64..127)
+//                           O = diag(gam) Y + P Delta    (lanes 64-127, off the chain)
 //                         Hand-offs between the producer and the compute warps are mbarriers;
 //                         the output accumulators are double-buffered in Tensor Memory so
 //                         the output epilogue stays off the state chain.
@@ -51,10 +53,11 @@ constexpr float kInvSqrtD = 0.08838834764831845f;  // 1 / sqrt(128)
 constexpr uint32_t kWBytes = 16384;    // W: 64 token rows x 128 d_k, K-major, [K-block][64 rows]
 constexpr uint32_t kQBytes = 16384;    // normalised Q, same layout (per QK head)
 constexpr uint32_t kUBytes = 16384;    // U: [d_v half][64 rows][64]
-constexpr uint32_t kPBytes = 8192;     // P: 64 rows x 64, K-major
-constexpr uint32_t kCvecBytes = 1024;  // c_j at [0,64), gam_L at [64], gam_r at [128,192)
-constexpr uint32_t kKTBytes = 16384;   // K as an MN-major operand (d_k x chunk)
-constexpr uint32_t kChunkLoadBytes = kWBytes + kQBytes + kKTBytes + kPBytes + kUBytes / 2 + kCvecBytes;
+constexpr uint32_t kPBytes = 8192;     // P: 64 token rows x 64, K-major
+constexpr uint32_t kCvecBytes = 1024;  // c_j at [0,64), gam_r at [64,128), gam_L at [128]
+constexpr uint32_t kCvecLoad = 528;    // the bytes of a gate-factor record the state kernel reads
+constexpr uint32_t kKTBytes = 16384;   // K, [d_k block][64 token rows] (MN-major A operand)
+constexpr uint32_t kChunkLoadBytes = kWBytes + kQBytes + kKTBytes + kUBytes / 2 + kPBytes + kCvecLoad;
 
 struct WsLayout {
     size_t seq_chunk0, table, w, u, p, cvec, kt, qn, total;
@@ -171,8 +174,7 @@ __device__ __forceinline__ int af_idx(int R, int J) { return R * 64 + 4 * ((J >>
 constexpr uint32_t kP_GR = 0;        // [K; Q] K-major (32 KB)  | after the Gram MMA: V images of both heads
 constexpr uint32_t kP_KT = 32768;    // K MN-major (16 KB)
 constexpr uint32_t kP_AF = 49152;    // A / T fp32, 2 heads (32 KB) | then [T0 D0; T1 D1] images for W and U
-constexpr uint32_t kP_XS = 81920;    // block-solve scratch, 2 heads x 3 blocks of 16x16 fp32 (6 KB)
-constexpr uint32_t kP_SMALL = 90112; // gates, barrier, TMEM address
+constexpr uint32_t kP_SMALL = 81920; // gates, barrier, TMEM address
 constexpr uint32_t kPrepSmem = kP_SMALL + 2048 + 1024;
 
 struct PrepSmall {
@@ -193,7 +195,6 @@ chunk_prep_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __re
     const uint32_t sb = smem_u32(sm);
     PrepSmall& ss = *reinterpret_cast<PrepSmall*>(sm + kP_SMALL);
     float* af = reinterpret_cast<float*>(sm + kP_AF);   // [head][64][64] (swizzled rows)
-    float* xs = reinterpret_cast<float*>(sm + kP_XS);   // [head][3][16][16]
 
     const WsLayout L = ws_layout(num_seqs, total_tokens, hk, hv);
     int32_t* header = reinterpret_cast<int32_t*>(ws);
@@ -311,51 +312,60 @@ chunk_prep_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __re
                     vr[hh][pass][0] = vr[hh][pass][1] = make_uint4(0, 0, 0, 0);
                 }
             }
+        // gate factors of both heads to the workspace (warps 2-3; token row r)
+        if (warp >= 2) {
+            const int r = tid - 64;
+#pragma unroll
+            for (int hh = 0; hh < 2; ++hh) {
+                float* cv = reinterpret_cast<float*>(ws + L.cvec + ((size_t)cid * hv + h0 + hh) * kCvecBytes);
+                const float Gl = ss.G[hh][len - 1], Gr = ss.G[hh][r];
+                cv[r] = (r < len) ? __expf(Gl - Gr) : 0.f;
+                cv[64 + r] = ss.gam[hh][r];
+                if (r == 0) cv[128] = __expf(Gl);
+            }
+        }
         ok = mbar_wait(&ss.bar_mma, 0);
         if (__syncthreads_or(!ok)) { err = 1; goto cleanup; }
         tc_fence_after();
 
-        // ---- 3. decay masks: A (fp32, smem) from K K^T rows; P and gate factors to the workspace
-        float row[64];
-        tmem_ld64(tmem, warp, 0, row);
-        const int r = tid & 63;
-        if (warp < 2) {
+        // ---- 3. decay masks from the Gram rows: A (fp32, smem) from K K^T (warps 0-1),
+        //         P = lower(exp(G_r - G_j) Q K^T) of both heads to the workspace (warps 2-3)
+        {
+            float row[64];
+            tmem_ld64(tmem, warp, 0, row);
+            const int r = tid & 63;
+            if (warp < 2) {
 #pragma unroll
-            for (int hh = 0; hh < 2; ++hh) {
-                const float Gr = ss.G[hh][r], br = ss.b[hh][r];
-                float4* a4 = reinterpret_cast<float4*>(af + hh * 4096);
+                for (int hh = 0; hh < 2; ++hh) {
+                    const float Gr = ss.G[hh][r], br = ss.b[hh][r];
+                    float4* a4 = reinterpret_cast<float4*>(af + hh * 4096);
 #pragma unroll
-                for (int m = 0; m < 16; ++m) {
-                    float t4[4];
+                    for (int m = 0; m < 16; ++m) {
+                        float t4[4];
 #pragma unroll
-                    for (int e = 0; e < 4; ++e) {
-                        const int i = 4 * m + e;
-                        t4[e] = (i < r) ? br * expf(Gr - ss.G[hh][i]) * row[i] : 0.f;
+                        for (int e = 0; e < 4; ++e) {
+                            const int i = 4 * m + e;
+                            t4[e] = (i < r) ? br * __expf(Gr - ss.G[hh][i]) * row[i] : 0.f;
+                        }
+                        a4[r * 16 + (m ^ (r & 15))] = make_float4(t4[0], t4[1], t4[2], t4[3]);
                     }
-                    a4[r * 16 + (m ^ (r & 15))] = make_float4(t4[0], t4[1], t4[2], t4[3]);
                 }
-            }
-        } else {
+            } else {
 #pragma unroll
-            for (int hh = 0; hh < 2; ++hh) {
-                const int h = h0 + hh;
-                const float Gr = ss.G[hh][r];
-                unsigned char* pimg = ws + L.p + ((size_t)cid * hv + h) * kPBytes;
+                for (int hh = 0; hh < 2; ++hh) {
+                    const float Gr = ss.G[hh][r];
+                    unsigned char* pimg = ws + L.p + ((size_t)cid * hv + h0 + hh) * kPBytes;
 #pragma unroll
-                for (int ch = 0; ch < 8; ++ch) {
-                    float p8[8];
+                    for (int ch = 0; ch < 8; ++ch) {
+                        float p8[8];
 #pragma unroll
-                    for (int e = 0; e < 8; ++e) {
-                        const int i = 8 * ch + e;
-                        p8[e] = (i <= r) ? expf(Gr - ss.G[hh][i]) * row[i] : 0.f;
+                        for (int e = 0; e < 8; ++e) {
+                            const int i = 8 * ch + e;
+                            p8[e] = (i <= r) ? __expf(Gr - ss.G[hh][i]) * row[i] : 0.f;
+                        }
+                        *reinterpret_cast<uint4*>(pimg + sw128(r, ch)) = pack8(p8);
                     }
-                    *reinterpret_cast<uint4*>(pimg + sw128(r, ch)) = pack8(p8);
                 }
-                float* cv = reinterpret_cast<float*>(ws + L.cvec + ((size_t)cid * hv + h) * kCvecBytes);
-                const float Gl = ss.G[hh][len - 1];
-                cv[r] = (r < len) ? expf(Gl - Gr) : 0.f;
-                cv[128 + r] = ss.gam[hh][r];
-                if (r == 0) cv[64] = expf(Gl);
             }
         }
         // V images (MN-major: token row, d_v contiguous) into the dead [K; Q] region
@@ -372,52 +382,34 @@ chunk_prep_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __re
     tc_fence_before();
     __syncthreads();
 
-    // ---- 4. T = (I + A)^-1 per head, by 16x16 blocks, in place in `af`
+    // ---- 4. T = (I + A)^-1: thread = (head, column i), forward substitution over the rows;
+    //         every index is a compile-time constant, the A reads are warp-wide broadcasts.
     {
-        // 4a. diagonal blocks: thread = (head, block, column) forward substitution
-        const int hh = tid >> 6, blk = (tid >> 4) & 3, i = tid & 15;
-        const float* A = af + hh * 4096;
-        float x[16];
+        const int hh = tid >> 6, i = tid & 63;
+        const float4* a4 = reinterpret_cast<const float4*>(af + hh * 4096);
+        float x[kChunk];
 #pragma unroll
-        for (int r = 0; r < 16; ++r) {
-            float acc = 0.f;
+        for (int r = 0; r < kChunk; ++r) x[r] = 0.f;
+        // column i of (I + A) x = e_i:  x_r = [r == i] - sum_{j<r} A[r][j] x_j  (x_r = 0 for r < i)
 #pragma unroll
-            for (int j = 0; j < r; ++j) acc = fmaf(A[af_idx(blk * 16 + r, blk * 16 + j)], x[j], acc);
-            x[r] = (r == i) ? 1.f : ((r < i) ? 0.f : -acc);
-        }
-        __syncthreads();
+        for (int r = 0; r < kChunk; ++r) {
+            float s0 = 0.f, s1 = 0.f, s2 = 0.f, s3 = 0.f;
 #pragma unroll
-        for (int r = 0; r < 16; ++r) af[hh * 4096 + af_idx(blk * 16 + r, blk * 16 + i)] = x[r];
-        __syncthreads();
-    }
-    // 4b. block rows: X = sum_{k=bj}^{bi-1} A_{bi,k} T_{k,bj};  T_{bi,bj} = -Dinv_bi X
-#pragma unroll 1
-    for (int bi = 1; bi < 4; ++bi) {
-        const int hh = tid >> 6, l = tid & 63;
-        float* A = af + hh * 4096;
-        float* X = xs + hh * 768;
-        for (int o = l; o < 256 * bi; o += 64) {
-            const int bj = o >> 8, rr = (o >> 4) & 15, cc = o & 15;
-            const int R = bi * 16 + rr, C = bj * 16 + cc;
-            float acc = 0.f;
-            for (int kb2 = bj; kb2 < bi; ++kb2) {
-#pragma unroll
-                for (int m = 0; m < 16; ++m)
-                    acc = fmaf(A[af_idx(R, kb2 * 16 + m)], A[af_idx(kb2 * 16 + m, C)], acc);
+            for (int m = 0; m < (r + 3) / 4; ++m) {
+                const float4 av = a4[r * 16 + (m ^ (r & 15))];
+                s0 = fmaf(av.x, x[4 * m + 0], s0);
+                s1 = fmaf(av.y, x[4 * m + 1], s1);
+                s2 = fmaf(av.z, x[4 * m + 2], s2);
+                s3 = fmaf(av.w, x[4 * m + 3], s3);
             }
-            X[o] = acc;
+            x[r] = (r == i) ? 1.f : -((s0 + s1) + (s2 + s3));
         }
         __syncthreads();
-        for (int o = l; o < 256 * bi; o += 64) {
-            const int bj = o >> 8, rr = (o >> 4) & 15, cc = o & 15;
-            float acc = 0.f;
+        // write column i of T back (row r: T[r][i]), then build the W / U operand rows
 #pragma unroll
-            for (int m = 0; m < 16; ++m)
-                acc = fmaf(A[af_idx(bi * 16 + rr, bi * 16 + m)], X[(bj << 8) + (m << 4) + cc], acc);
-            A[af_idx(bi * 16 + rr, bj * 16 + cc)] = -acc;
-        }
-        __syncthreads();
+        for (int r = 0; r < kChunk; ++r) af[hh * 4096 + af_idx(r, i)] = x[r];
     }
+    __syncthreads();
 
     // ---- 5. MMA operand images [T_0 diag(b_0 gam_0); T_1 diag(b_1 gam_1)] and [T_0 diag(b_0); ...]
     {
@@ -531,34 +523,39 @@ cleanup:
 }
 
 // ===================================================================== K2
-constexpr int kStateThreads = 160;                  // warps 0-3 compute, warp 4 copies + MMAs
+constexpr int kStateThreads = 288;                  // warps 0-7 compute, warp 8 copies + MMAs
+constexpr int kStages = 3;                          // chunk buffers (loads run two chunks ahead)
 constexpr uint32_t kS_A1 = 0;                       // [W; Q] K-major, 2 K-blocks of 128 rows (32 KB)
-constexpr uint32_t kS_KT = 32768;                   // K MN-major (16 KB)
-constexpr uint32_t kS_A2 = 49152;                   // [0; P] K-major (16 KB)
-constexpr uint32_t kS_U = 65536;                    // U, this CTA's d_v half (8 KB)
-constexpr uint32_t kS_CV = 73728;                   // gate factors (1 KB)
-constexpr uint32_t kS_BUF = 74752;                  // one chunk buffer (73 KB)
-constexpr uint32_t kS_B1 = 2 * kS_BUF;              // S slice bf16, MN-major (16 KB)
+constexpr uint32_t kS_KT = 32768;                   // K, MN-major A operand (16 KB)
+constexpr uint32_t kS_U = 49152;                    // U, this CTA's d_v half (8 KB)
+constexpr uint32_t kS_P = 57344;                    // P (8 KB); [U; P] is the A operand of P Delta
+constexpr uint32_t kS_BUF = 65536;                  // one chunk buffer (64 KB)
+constexpr uint32_t kS_B1 = kStages * kS_BUF;        // S slice bf16, MN-major (16 KB)
 constexpr uint32_t kS_B2 = kS_B1 + 16384;           // Delta, MN-major (8 KB)
 constexpr uint32_t kS_B3 = kS_B2 + 8192;            // diag(c) Delta, MN-major (8 KB)
-constexpr uint32_t kS_SMALL = kS_B3 + 8192;
-constexpr uint32_t kStateSmem = kS_SMALL + 256 + 1024;
+constexpr uint32_t kS_CV = kS_B3 + 8192;            // gate factors of each stage (3 x 528 B)
+constexpr uint32_t kS_SMALL = kS_CV + kStages * kCvecLoad;
+constexpr uint32_t kStateSmem = kS_SMALL + 128;     // needs a 1024-aligned dynamic base (checked)
 // Tensor Memory columns
 constexpr uint32_t kT_XY = 0;     // [X; Y] of chunk parity p at kT_XY + 64 p
-constexpr uint32_t kT_PD = 128;   // P Delta of chunk parity p at kT_PD + 64 p
+constexpr uint32_t kT_PD = 128;   // P Delta of chunk parity p at kT_PD + 64 p (rows 64..127)
 constexpr uint32_t kT_SA = 256;   // K^T diag(c) Delta
 
 struct StateSmall {
-    uint64_t full[2];
+    uint64_t full[kStages];
     uint64_t b1, b23, mma1, mma2, mma3;
     uint32_t tmem_base;
     int abort_flag;
 };
 
-// Bounded wait that also returns (false) as soon as another thread has given up.
+// Bounded wait that also returns (false) as soon as another thread has given up.  After a
+// few immediate polls the waiter backs off with a short sleep, so that idle waiters do not
+// take issue slots from the warps doing the work.
 __device__ __forceinline__ bool wait_or_abort(uint64_t* bar, uint32_t parity, volatile int* abort_flag,
                                               int32_t* header) {
-    if (mbar_try_wait(bar, parity)) return true;
+#pragma unroll 1
+    for (int i = 0; i < 4; ++i)
+        if (mbar_try_wait(bar, parity)) return true;
     const uint64_t t0 = global_timer_ns();
     while (true) {
         if (mbar_try_wait(bar, parity)) return true;
@@ -568,6 +565,7 @@ __device__ __forceinline__ bool wait_or_abort(uint64_t* bar, uint32_t parity, vo
             atomicOr(header, 1);
             return false;
         }
+        __nanosleep(32);
     }
 }
 
@@ -575,9 +573,17 @@ __device__ __forceinline__ void mbar_arrive(uint64_t* bar) {
     asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_u32(bar)) : "memory");
 }
 
-__device__ __forceinline__ void issue_chunk_loads(unsigned char* buf, uint64_t* bar, const unsigned char* ws,
-                                                  const WsLayout& L, int cid, int h, int jq, int half,
-                                                  int hk, int hv) {
+// 32 consecutive TMEM columns of this warp's lane quarter.
+__device__ __forceinline__ void tmem_ld32(uint32_t tmem_base, int warp, uint32_t col, float* v) {
+    const uint32_t a = tmem_base + ((uint32_t)(warp & 3) * 32u << 16) + col;
+    tmem_ld16(a, v);
+    tmem_ld16(a + 16, v + 16);
+    tmem_ld_wait();
+}
+
+__device__ __forceinline__ void issue_chunk_loads(unsigned char* buf, unsigned char* cv, uint64_t* bar,
+                                                  const unsigned char* ws, const WsLayout& L, int cid, int h,
+                                                  int jq, int half, int hk, int hv) {
     mbar_arrive_expect_tx(bar, kChunkLoadBytes);
     const unsigned char* w = ws + L.w + ((size_t)cid * hv + h) * kWBytes;
     const unsigned char* qn = ws + L.qn + ((size_t)cid * hk + jq) * kQBytes;
@@ -586,16 +592,15 @@ __device__ __forceinline__ void issue_chunk_loads(unsigned char* buf, uint64_t* 
     bulk_g2s(buf + kS_A1 + 16384, w + 8192, 8192, bar);   // W rows, d_k 64..127
     bulk_g2s(buf + kS_A1 + 24576, qn + 8192, 8192, bar);  // Q rows, d_k 64..127
     bulk_g2s(buf + kS_KT, ws + L.kt + ((size_t)cid * hk + jq) * kKTBytes, kKTBytes, bar);
-    bulk_g2s(buf + kS_A2 + 8192, ws + L.p + ((size_t)cid * hv + h) * kPBytes, kPBytes, bar);
     bulk_g2s(buf + kS_U, ws + L.u + ((size_t)cid * hv + h) * kUBytes + half * (kUBytes / 2), kUBytes / 2, bar);
-    bulk_g2s(buf + kS_CV, ws + L.cvec + ((size_t)cid * hv + h) * kCvecBytes, kCvecBytes, bar);
+    bulk_g2s(buf + kS_P, ws + L.p + ((size_t)cid * hv + h) * kPBytes, kPBytes, bar);
+    bulk_g2s(cv, ws + L.cvec + ((size_t)cid * hv + h) * kCvecBytes, kCvecLoad, bar);
 }
 
 __global__ void __launch_bounds__(kStateThreads, 1)
 chunk_state_kernel(const float* s0, const int32_t* __restrict__ cu, __nv_bfloat16* __restrict__ out,
                    float* sT, unsigned char* ws, int num_seqs, int total_tokens, int hk, int hv) {
-    extern __shared__ unsigned char smem_dyn[];
-    unsigned char* sm = reinterpret_cast<unsigned char*>((reinterpret_cast<uintptr_t>(smem_dyn) + 1023) & ~uintptr_t(1023));
+    extern __shared__ __align__(1024) unsigned char sm[];
     const uint32_t sb = smem_u32(sm);
     StateSmall& ss = *reinterpret_cast<StateSmall*>(sm + kS_SMALL);
     volatile int* abort_flag = &ss.abort_flag;
@@ -610,120 +615,127 @@ chunk_state_kernel(const float* s0, const int32_t* __restrict__ cu, __nv_bfloat1
     const int32_t* seq_chunk0 = reinterpret_cast<const int32_t*>(ws + L.seq_chunk0);
     const int cs = seq_chunk0[n], nch = seq_chunk0[n + 1] - cs;
     const int t_begin = cu[n], t_end = cu[n + 1];
-
-    // zero the upper (unused) 64 rows of both [0; P] operands
-    for (int i = tid; i < 2 * 512; i += kStateThreads) {
-        const int b = i >> 9, o = (i & 511) * 16;
-        *reinterpret_cast<uint4*>(sm + b * kS_BUF + kS_A2 + o) = make_uint4(0, 0, 0, 0);
+    if (sb & 1023u) {  // the swizzled operand layouts need a 1024-byte-aligned base
+        if (tid == 0) atomicOr(header, 2);
+        return;
     }
+
     if (warp == 0) {
         tmem_alloc(&ss.tmem_base, 512);
         tmem_relinquish();
     }
     if (tid == 0) {
-        mbar_init(&ss.full[0], 1);
-        mbar_init(&ss.full[1], 1);
-        mbar_init(&ss.b1, 128);
-        mbar_init(&ss.b23, 64);
+        for (int s = 0; s < kStages; ++s) mbar_init(&ss.full[s], 1);
+        mbar_init(&ss.b1, 256);
+        mbar_init(&ss.b23, 128);
         mbar_init(&ss.mma1, 1);
         mbar_init(&ss.mma2, 1);
         mbar_init(&ss.mma3, 1);
         ss.abort_flag = 0;
         fence_mbar_init();
     }
-    fence_async_smem();
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = ss.tmem_base;
 
-    if (warp == 4) {
+    if (warp == 8) {
         // ------------------------------------------------ producer: bulk copies and MMAs
         if (lane == 0) {
             const uint32_t id_xy = idesc_bf16(128, 64, 0, 1);  // A K-major, B MN-major
             const uint32_t id_s = idesc_bf16(128, 64, 1, 1);   // A MN-major, B MN-major
+            const uint64_t d_b1 = sdesc_sw128(sb + kS_B1, 16384, 1024);
+            const uint64_t d_b2 = sdesc_sw128(sb + kS_B2, 8192, 1024);
+            const uint64_t d_b3 = sdesc_sw128(sb + kS_B3, 8192, 1024);
             int issued = 0;  // chunks whose loads have been issued
-            if (nch > 0) {
-                issue_chunk_loads(sm, &ss.full[0], ws, L, cs, h, jq, half, hk, hv);
-                issued = 1;
-            }
+            for (; issued < kStages - 1 && issued < nch; ++issued)
+                issue_chunk_loads(sm + issued * kS_BUF, sm + kS_CV + issued * kCvecLoad, &ss.full[issued], ws, L,
+                                  cs + issued, h, jq, half, hk, hv);
             int c = 0;
             for (; c < nch; ++c) {
-                const int b = c & 1;
+                const int b = c % kStages, par = c & 1;
                 const uint32_t bufa = sb + b * kS_BUF;
-                if (!wait_or_abort(&ss.b1, c & 1, abort_flag, header)) break;   // B1 = S(c) written
-                if (c + 1 < nch) {
-                    // the other buffer held chunk c-1; its last reader, P Delta of c-1, is done
-                    if (c >= 1 && !wait_or_abort(&ss.mma2, (c - 1) & 1, abort_flag, header)) break;
-                    issue_chunk_loads(sm + (b ^ 1) * kS_BUF, &ss.full[b ^ 1], ws, L, cs + c + 1, h, jq,
-                                      half, hk, hv);
-                    issued = c + 2;
-                }
-                if (!wait_or_abort(&ss.full[b], (c >> 1) & 1, abort_flag, header)) break;
+                const uint64_t d_a1 = sdesc_sw128(bufa + kS_A1, 16, 1024);
+                const uint64_t d_kt = sdesc_sw128(bufa + kS_KT, 8192, 1024);
+                const uint64_t d_up = sdesc_sw128(bufa + kS_U, 16, 1024);  // rows 0..63 U (unused), 64..127 P
+                if (!wait_or_abort(&ss.b1, par, abort_flag, header)) break;   // S(c) in B1
+                if (!wait_or_abort(&ss.full[b], (c / kStages) & 1, abort_flag, header)) break;
                 tc_fence_after();
 #pragma unroll
-                for (int s = 0; s < 8; ++s)
-                    mma_bf16(tmem + kT_XY + 64 * b,
-                             sdesc_sw128(bufa + kS_A1 + (s >> 2) * 16384 + (s & 3) * 32, 16, 1024),
-                             sdesc_sw128(sb + kS_B1 + s * 2048, 16384, 1024), id_xy, s > 0);
+                for (int s = 0; s < 8; ++s)  // descriptor start addresses advance in 16-byte units
+                    mma_bf16(tmem + kT_XY + 64 * par, d_a1 + (((s >> 2) * 16384 + (s & 3) * 32) >> 4),
+                             d_b1 + ((s * 2048) >> 4), id_xy, s > 0);
                 mma_commit(&ss.mma1);
-                if (!wait_or_abort(&ss.b23, c & 1, abort_flag, header)) break;  // Delta(c) written
+                if (issued < nch) {
+                    // refill the buffer chunk c-1 used: its MMA readers (this thread's) are done
+                    // once P Delta of c-1 is; its thread readers finished before b1(c)
+                    if (c >= 1 && !wait_or_abort(&ss.mma2, (c - 1) & 1, abort_flag, header)) break;
+                    issue_chunk_loads(sm + (issued % kStages) * kS_BUF, sm + kS_CV + (issued % kStages) * kCvecLoad,
+                                      &ss.full[issued % kStages], ws, L, cs + issued, h, jq, half, hk, hv);
+                    ++issued;
+                }
+                if (!wait_or_abort(&ss.b23, par, abort_flag, header)) break;  // Delta(c) written
                 tc_fence_after();
 #pragma unroll
                 for (int s = 0; s < 4; ++s)
-                    mma_bf16(tmem + kT_SA, sdesc_sw128(bufa + kS_KT + s * 2048, 8192, 1024),
-                             sdesc_sw128(sb + kS_B3 + s * 2048, 8192, 1024), id_s, s > 0);
+                    mma_bf16(tmem + kT_SA, d_kt + ((s * 2048) >> 4), d_b3 + ((s * 2048) >> 4), id_s, s > 0);
                 mma_commit(&ss.mma3);
 #pragma unroll
                 for (int s = 0; s < 4; ++s)
-                    mma_bf16(tmem + kT_PD + 64 * b, sdesc_sw128(bufa + kS_A2 + s * 32, 16, 1024),
-                             sdesc_sw128(sb + kS_B2 + s * 2048, 8192, 1024), id_xy, s > 0);
+                    mma_bf16(tmem + kT_PD + 64 * par, d_up + ((s * 32) >> 4), d_b2 + ((s * 2048) >> 4), id_xy, s > 0);
                 mma_commit(&ss.mma2);
             }
             if (*abort_flag) {
                 // drain: every MMA issued so far, then every bulk copy still in flight
                 mma_commit(&ss.mma1);
                 mbar_wait(&ss.mma1, c & 1);
-                for (int j = c; j < issued; ++j) mbar_wait(&ss.full[j & 1], (j >> 1) & 1);
+                for (int j = c; j < issued; ++j) mbar_wait(&ss.full[j % kStages], (j / kStages) & 1);
             }
         }
     } else {
-        // ------------------------------------------------ compute warps 0-3
-        // fp32 state slice: thread t owns S[half*64 + m][t], m = 0..63 (column t of S)
-        const int t = tid;
-        float S[64];
-        const size_t sbase = ((size_t)n * hv + h) * kD * kD + (size_t)(half * 64) * kD + t;
+        // ------------------------------------------------ compute warps 0-7
+        // warp w: TMEM lane quarter q4 = w & 3, column half ch2 = w >> 2 of this CTA's 64 d_v
+        const int q4 = warp & 3, ch2 = warp >> 2;
+        const int t = q4 * 32 + lane;       // d_k row of S^T this thread owns (state update)
+        const int r = (q4 & 1) * 32 + lane; // token row (Delta: quarters 0-1; outputs: quarters 2-3)
+        const bool delta_warp = q4 < 2;
+        // fp32 state: S[half*64 + 32*ch2 + m][t], m = 0..31
+        float S[32];
+        const size_t sbase = ((size_t)n * hv + h) * kD * kD + (size_t)(half * 64 + 32 * ch2) * kD + t;
 #pragma unroll
-        for (int m = 0; m < 64; ++m) S[m] = s0 ? s0[sbase + (size_t)m * kD] : 0.f;
+        for (int m = 0; m < 32; ++m) S[m] = s0 ? s0[sbase + (size_t)m * kD] : 0.f;
 #pragma unroll
-        for (int ch = 0; ch < 8; ++ch)
-            *reinterpret_cast<uint4*>(sm + kS_B1 + sw128(t, ch)) = pack8(S + 8 * ch);
+        for (int cc = 0; cc < 4; ++cc)
+            *reinterpret_cast<uint4*>(sm + kS_B1 + sw128(t, 4 * ch2 + cc)) = pack8(S + 8 * cc);
         fence_async_smem();
         tc_fence_before();
         mbar_arrive(&ss.b1);
 
-        const int r = tid & 63;  // token row (warps 0-1: Delta rows; warps 2-3: output rows)
         for (int c = 0; c < nch; ++c) {
-            const int b = c & 1;
+            const int b = c % kStages, par = c & 1;
             unsigned char* buf = sm + b * kS_BUF;
-            if (!wait_or_abort(&ss.full[b], (c >> 1) & 1, abort_flag, header)) break;
-            const float* cvec = reinterpret_cast<const float*>(buf + kS_CV);
-            const float gl = cvec[64];
-            const float crow = (warp < 2) ? cvec[r] : cvec[128 + r];  // c_r, or gam_r for outputs
+            if (!wait_or_abort(&ss.full[b], (c / kStages) & 1, abort_flag, header)) break;
+            const float* cvec = reinterpret_cast<const float*>(sm + kS_CV + b * kCvecLoad);
+            const float gl = cvec[128];
+            const float crow = delta_warp ? cvec[r] : cvec[64 + r];  // c_r, or gam_r for outputs
 
-            if (warp < 2) {  // Delta = U - X for token row r; write Delta and diag(c) Delta
-                if (c >= 1 && !wait_or_abort(&ss.mma2, (c - 1) & 1, abort_flag, header)) break;
-                if (!wait_or_abort(&ss.mma1, c & 1, abort_flag, header)) break;
-                tc_fence_after();
-                float x[64];
-                tmem_ld64(tmem, warp, kT_XY + 64 * b, x);
+            if (delta_warp) {  // Delta = U - X for token row r, columns 32*ch2 .. +32
+                uint4 u4[4];    // this row's U values, read before any shared store of this phase
 #pragma unroll
-                for (int ch = 0; ch < 8; ++ch) {
+                for (int cc = 0; cc < 4; ++cc) u4[cc] = *reinterpret_cast<const uint4*>(buf + kS_U + sw128(r, 4 * ch2 + cc));
+                if (c >= 1 && !wait_or_abort(&ss.mma2, (c - 1) & 1, abort_flag, header)) break;  // B2 free
+                if (!wait_or_abort(&ss.mma1, par, abort_flag, header)) break;
+                tc_fence_after();
+                float x[32];
+                tmem_ld32(tmem, warp, kT_XY + 64 * par + 32 * ch2, x);
+#pragma unroll
+                for (int cc = 0; cc < 4; ++cc) {
+                    const int ch = 4 * ch2 + cc;
                     float u8[8], d8[8], c8[8];
-                    unpack8(*reinterpret_cast<const uint4*>(buf + kS_U + sw128(r, ch)), u8);
+                    unpack8(u4[cc], u8);
 #pragma unroll
                     for (int e = 0; e < 8; ++e) {
-                        d8[e] = u8[e] - x[8 * ch + e];
+                        d8[e] = u8[e] - x[8 * cc + e];
                         c8[e] = d8[e] * crow;
                     }
                     *reinterpret_cast<uint4*>(sm + kS_B2 + sw128(r, ch)) = pack8(d8);
@@ -733,45 +745,38 @@ chunk_state_kernel(const float* s0, const int32_t* __restrict__ cu, __nv_bfloat1
                 tc_fence_before();
                 mbar_arrive(&ss.b23);
             }
-            // state update S^T <- gam_L S^T + K^T diag(c) Delta (this thread: d_k row t)
-            if (!wait_or_abort(&ss.mma3, c & 1, abort_flag, header)) break;
+            // state update S^T <- gam_L S^T + K^T diag(c) Delta (d_k row t, 32 d_v columns)
+            if (!wait_or_abort(&ss.mma3, par, abort_flag, header)) break;
             tc_fence_after();
             {
-                float acc[64];
-                tmem_ld64(tmem, warp, kT_SA, acc);
+                float acc[32];
+                tmem_ld32(tmem, warp, kT_SA + 32 * ch2, acc);
 #pragma unroll
-                for (int m = 0; m < 64; ++m) S[m] = fmaf(gl, S[m], acc[m]);
+                for (int m = 0; m < 32; ++m) S[m] = fmaf(gl, S[m], acc[m]);
 #pragma unroll
-                for (int ch = 0; ch < 8; ++ch)
-                    *reinterpret_cast<uint4*>(sm + kS_B1 + sw128(t, ch)) = pack8(S + 8 * ch);
+                for (int cc = 0; cc < 4; ++cc)
+                    *reinterpret_cast<uint4*>(sm + kS_B1 + sw128(t, 4 * ch2 + cc)) = pack8(S + 8 * cc);
             }
             fence_async_smem();
             tc_fence_before();
             mbar_arrive(&ss.b1);
 
-            if (warp >= 2) {  // outputs of token row r: O = gam_r Y + P Delta
-                if (!wait_or_abort(&ss.mma2, c & 1, abort_flag, header)) break;
+            if (!delta_warp) {  // outputs of token row r: O = gam_r Y + P Delta
+                if (!wait_or_abort(&ss.mma2, par, abort_flag, header)) break;
                 tc_fence_after();
                 const int t0 = t_begin + c * kChunk;
                 const int len = min(kChunk, t_end - t0);
-                uint4* op = reinterpret_cast<uint4*>(out + ((size_t)(t0 + r) * hv + h) * kD + half * 64);
+                float y[32], pd[32];
+                tmem_ld32(tmem, warp, kT_XY + 64 * par + 32 * ch2, y);
+                tmem_ld32(tmem, warp, kT_PD + 64 * par + 32 * ch2, pd);
+                if (r < len) {
+                    uint4* op = reinterpret_cast<uint4*>(out + ((size_t)(t0 + r) * hv + h) * kD + half * 64 + 32 * ch2);
 #pragma unroll
-                for (int part = 0; part < 2; ++part) {  // 32 columns at a time
-                    float y[32], pd[32];
-                    const uint32_t lq = (uint32_t)(warp & 3) * 32u << 16;
-                    tmem_ld16(tmem + lq + kT_XY + 64 * b + 32 * part, y);
-                    tmem_ld16(tmem + lq + kT_XY + 64 * b + 32 * part + 16, y + 16);
-                    tmem_ld16(tmem + lq + kT_PD + 64 * b + 32 * part, pd);
-                    tmem_ld16(tmem + lq + kT_PD + 64 * b + 32 * part + 16, pd + 16);
-                    tmem_ld_wait();
-                    if (r < len) {
+                    for (int cc = 0; cc < 4; ++cc) {
+                        float o8[8];
 #pragma unroll
-                        for (int ch = 0; ch < 4; ++ch) {
-                            float o8[8];
-#pragma unroll
-                            for (int e = 0; e < 8; ++e) o8[e] = fmaf(crow, y[8 * ch + e], pd[8 * ch + e]);
-                            op[4 * part + ch] = pack8(o8);
-                        }
+                        for (int e = 0; e < 8; ++e) o8[e] = fmaf(crow, y[8 * cc + e], pd[8 * cc + e]);
+                        op[cc] = pack8(o8);
                     }
                 }
                 tc_fence_before();
@@ -779,7 +784,7 @@ chunk_state_kernel(const float* s0, const int32_t* __restrict__ cu, __nv_bfloat1
         }
         if (!*abort_flag && sT) {
 #pragma unroll
-            for (int m = 0; m < 64; ++m) sT[sbase + (size_t)m * kD] = S[m];
+            for (int m = 0; m < 32; ++m) sT[sbase + (size_t)m * kD] = S[m];
         }
     }
     tc_fence_before();
