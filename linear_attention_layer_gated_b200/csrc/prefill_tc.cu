@@ -22,17 +22,17 @@
 //                           state kernel's MMAs read, go to the workspace, with the gate
 //                           factors (c, gam) of each V head.
 //  K2 chunk_state_kernel  one CTA per (sequence, V head, half of d_v), sequential over the
-//                         sequence's chunks.  Warp 8 issues the bulk copies (two chunks
-//                         ahead, three buffers) and the MMAs; warps 0-7 compute, each warp on
+//                         sequence's chunks.  Warp 8 issues the MMAs, warp 9 the bulk copies
+//                         (two chunks ahead, three buffers); warps 0-7 compute, each warp on
 //                         32 of the 64 d_v columns of its TMEM lane quarter.  Per chunk:
 //                           [X; Y] = [W; Q] S^T          (M=128)            <- on the chain
 //                           Delta = U - X, c Delta       (lanes 0-63: token rows)
 //                           K^T diag(c) Delta            (M=128: d_k rows)  <- on the chain
 //                           S^T <- gam_L S^T + K^T diag(c) Delta   (fp32 in registers)
 //                           P Delta                      (M=128 operand [U; P]: rows 64..127)
-//                           O = diag(gam) Y + P Delta    (lanes 64-127, off the chain)
-//                         Hand-offs between the producer and the compute warps are mbarriers;
-//                         the output accumulators are double-buffered in Tensor Memory so
+//                           O = diag(gam) Y + P Delta    (lanes 64-127, one chunk later)
+//                         Hand-offs between the issuing and the compute warps are mbarriers;
+//                         the output accumulators are triple-buffered in Tensor Memory so
 //                         the output epilogue stays off the state chain.
 // Every mbarrier wait is bounded (1 s) and, in the state kernel, also gives up as soon as
 // another thread of the CTA has given up; the kernel then records an error in the
@@ -523,7 +523,7 @@ cleanup:
 }
 
 // ===================================================================== K2
-constexpr int kStateThreads = 288;                  // warps 0-7 compute, warp 8 copies + MMAs
+constexpr int kStateThreads = 320;                  // warps 0-7 compute, warp 8 MMAs, warp 9 bulk copies
 constexpr int kStages = 3;                          // chunk buffers (loads run two chunks ahead)
 constexpr uint32_t kS_A1 = 0;                       // [W; Q] K-major, 2 K-blocks of 128 rows (32 KB)
 constexpr uint32_t kS_KT = 32768;                   // K, MN-major A operand (16 KB)
@@ -537,35 +537,35 @@ constexpr uint32_t kS_CV = kS_B3 + 8192;            // gate factors of each stag
 constexpr uint32_t kS_SMALL = kS_CV + kStages * kCvecLoad;
 constexpr uint32_t kStateSmem = kS_SMALL + 128;     // needs a 1024-aligned dynamic base (checked)
 // Tensor Memory columns
-constexpr uint32_t kT_XY = 0;     // [X; Y] of chunk parity p at kT_XY + 64 p
-constexpr uint32_t kT_PD = 128;   // P Delta of chunk parity p at kT_PD + 64 p (rows 64..127)
-constexpr uint32_t kT_SA = 256;   // K^T diag(c) Delta
+constexpr int kTBufs = 3;        // output accumulators of three consecutive chunks stay live
+constexpr uint32_t kT_XY = 0;     // [X; Y] of chunk c at kT_XY + 64 (c % 3)
+constexpr uint32_t kT_PD = 192;   // P Delta of chunk c at kT_PD + 64 (c % 3) (rows 64..127)
+constexpr uint32_t kT_SA = 384;   // K^T diag(c) Delta
 
 struct StateSmall {
-    uint64_t full[kStages];
-    uint64_t b1, b23, mma1, mma2, mma3;
+    uint64_t full[kStages];   // stage loaded
+    uint64_t empty[kStages];  // stage consumed: 256 compute-thread arrivals + the MMAs' commit
+    uint64_t mma2[kTBufs];    // P Delta of chunk c done, on mma2[c % 3] (a waiter may lag one chunk)
+    uint64_t b1, b3, b2, mma1, mma3;
     uint32_t tmem_base;
     int abort_flag;
 };
 
-// Bounded wait that also returns (false) as soon as another thread has given up.  After a
-// few immediate polls the waiter backs off with a short sleep, so that idle waiters do not
-// take issue slots from the warps doing the work.
+// Bounded wait that also returns (false) as soon as another thread has given up.  The
+// waiting thread is suspended by the hardware between checks (it resumes when the phase
+// completes), so idle waiters neither spin on issue slots nor oversleep.
 __device__ __forceinline__ bool wait_or_abort(uint64_t* bar, uint32_t parity, volatile int* abort_flag,
                                               int32_t* header) {
-#pragma unroll 1
-    for (int i = 0; i < 4; ++i)
-        if (mbar_try_wait(bar, parity)) return true;
+    if (mbar_try_wait(bar, parity)) return true;
     const uint64_t t0 = global_timer_ns();
     while (true) {
-        if (mbar_try_wait(bar, parity)) return true;
+        if (mbar_try_wait_suspend(bar, parity, 20000u)) return true;
         if (*abort_flag) return false;
         if (global_timer_ns() - t0 > kWaitLimitNs) {
             *abort_flag = 1;
             atomicOr(header, 1);
             return false;
         }
-        __nanosleep(32);
     }
 }
 
@@ -625,11 +625,15 @@ chunk_state_kernel(const float* s0, const int32_t* __restrict__ cu, __nv_bfloat1
         tmem_relinquish();
     }
     if (tid == 0) {
-        for (int s = 0; s < kStages; ++s) mbar_init(&ss.full[s], 1);
+        for (int s = 0; s < kStages; ++s) {
+            mbar_init(&ss.full[s], 1);
+            mbar_init(&ss.empty[s], 257);
+        }
         mbar_init(&ss.b1, 256);
-        mbar_init(&ss.b23, 128);
+        mbar_init(&ss.b3, 128);
+        mbar_init(&ss.b2, 128);
         mbar_init(&ss.mma1, 1);
-        mbar_init(&ss.mma2, 1);
+        for (int s = 0; s < kTBufs; ++s) mbar_init(&ss.mma2[s], 1);
         mbar_init(&ss.mma3, 1);
         ss.abort_flag = 0;
         fence_mbar_init();
@@ -640,56 +644,63 @@ chunk_state_kernel(const float* s0, const int32_t* __restrict__ cu, __nv_bfloat1
     const uint32_t tmem = ss.tmem_base;
 
     if (warp == 8) {
-        // ------------------------------------------------ producer: bulk copies and MMAs
+        // ------------------------------------------------ MMA issuer
         if (lane == 0) {
             const uint32_t id_xy = idesc_bf16(128, 64, 0, 1);  // A K-major, B MN-major
             const uint32_t id_s = idesc_bf16(128, 64, 1, 1);   // A MN-major, B MN-major
             const uint64_t d_b1 = sdesc_sw128(sb + kS_B1, 16384, 1024);
             const uint64_t d_b2 = sdesc_sw128(sb + kS_B2, 8192, 1024);
             const uint64_t d_b3 = sdesc_sw128(sb + kS_B3, 8192, 1024);
-            int issued = 0;  // chunks whose loads have been issued
-            for (; issued < kStages - 1 && issued < nch; ++issued)
-                issue_chunk_loads(sm + issued * kS_BUF, sm + kS_CV + issued * kCvecLoad, &ss.full[issued], ws, L,
-                                  cs + issued, h, jq, half, hk, hv);
             int c = 0;
             for (; c < nch; ++c) {
-                const int b = c % kStages, par = c & 1;
+                const int b = c % kStages, par = c & 1, tb = c % kTBufs;
                 const uint32_t bufa = sb + b * kS_BUF;
                 const uint64_t d_a1 = sdesc_sw128(bufa + kS_A1, 16, 1024);
                 const uint64_t d_kt = sdesc_sw128(bufa + kS_KT, 8192, 1024);
                 const uint64_t d_up = sdesc_sw128(bufa + kS_U, 16, 1024);  // rows 0..63 U (unused), 64..127 P
-                if (!wait_or_abort(&ss.b1, par, abort_flag, header)) break;   // S(c) in B1
+                // the operands normally land long before the state does: check them first
                 if (!wait_or_abort(&ss.full[b], (c / kStages) & 1, abort_flag, header)) break;
+                if (!wait_or_abort(&ss.b1, par, abort_flag, header)) break;   // S(c) in B1
                 tc_fence_after();
 #pragma unroll
                 for (int s = 0; s < 8; ++s)  // descriptor start addresses advance in 16-byte units
-                    mma_bf16(tmem + kT_XY + 64 * par, d_a1 + (((s >> 2) * 16384 + (s & 3) * 32) >> 4),
+                    mma_bf16(tmem + kT_XY + 64 * tb, d_a1 + (((s >> 2) * 16384 + (s & 3) * 32) >> 4),
                              d_b1 + ((s * 2048) >> 4), id_xy, s > 0);
                 mma_commit(&ss.mma1);
-                if (issued < nch) {
-                    // refill the buffer chunk c-1 used: its MMA readers (this thread's) are done
-                    // once P Delta of c-1 is; its thread readers finished before b1(c)
-                    if (c >= 1 && !wait_or_abort(&ss.mma2, (c - 1) & 1, abort_flag, header)) break;
-                    issue_chunk_loads(sm + (issued % kStages) * kS_BUF, sm + kS_CV + (issued % kStages) * kCvecLoad,
-                                      &ss.full[issued % kStages], ws, L, cs + issued, h, jq, half, hk, hv);
-                    ++issued;
-                }
-                if (!wait_or_abort(&ss.b23, par, abort_flag, header)) break;  // Delta(c) written
+                if (!wait_or_abort(&ss.b3, par, abort_flag, header)) break;   // diag(c) Delta(c) written
                 tc_fence_after();
 #pragma unroll
                 for (int s = 0; s < 4; ++s)
                     mma_bf16(tmem + kT_SA, d_kt + ((s * 2048) >> 4), d_b3 + ((s * 2048) >> 4), id_s, s > 0);
                 mma_commit(&ss.mma3);
+                if (!wait_or_abort(&ss.b2, par, abort_flag, header)) break;   // Delta(c) written
+                tc_fence_after();
 #pragma unroll
                 for (int s = 0; s < 4; ++s)
-                    mma_bf16(tmem + kT_PD + 64 * par, d_up + ((s * 32) >> 4), d_b2 + ((s * 2048) >> 4), id_xy, s > 0);
-                mma_commit(&ss.mma2);
+                    mma_bf16(tmem + kT_PD + 64 * tb, d_up + ((s * 32) >> 4), d_b2 + ((s * 2048) >> 4), id_xy, s > 0);
+                mma_commit(&ss.mma2[tb]);
+                mma_commit(&ss.empty[b]);  // every MMA reading stage b has completed
             }
-            if (*abort_flag) {
-                // drain: every MMA issued so far, then every bulk copy still in flight
+            if (*abort_flag) {  // drain: every MMA issued so far completes before TMEM is freed
                 mma_commit(&ss.mma1);
                 mbar_wait(&ss.mma1, c & 1);
-                for (int j = c; j < issued; ++j) mbar_wait(&ss.full[j % kStages], (j / kStages) & 1);
+            }
+        }
+    } else if (warp == 9) {
+        // ------------------------------------------------ bulk copies, two chunks ahead
+        if (lane == 0) {
+            int issued = 0;
+            for (; issued < nch; ++issued) {
+                const int st = issued % kStages;
+                if (issued >= kStages &&
+                    !wait_or_abort(&ss.empty[st], ((issued / kStages) - 1) & 1, abort_flag, header))
+                    break;
+                issue_chunk_loads(sm + st * kS_BUF, sm + kS_CV + st * kCvecLoad, &ss.full[st], ws, L,
+                                  cs + issued, h, jq, half, hk, hv);
+            }
+            if (*abort_flag) {  // drain: copies in flight land before the CTA exits
+                for (int j = max(0, issued - kStages); j < issued; ++j)
+                    mbar_wait(&ss.full[j % kStages], (j / kStages) & 1);
             }
         }
     } else {
@@ -711,39 +722,79 @@ chunk_state_kernel(const float* s0, const int32_t* __restrict__ cu, __nv_bfloat1
         tc_fence_before();
         mbar_arrive(&ss.b1);
 
-        for (int c = 0; c < nch; ++c) {
-            const int b = c % kStages, par = c & 1;
+        // Outputs of chunk c are written one chunk later (after the state update of c+1), so
+        // that their global stores are not still in flight at the next shared-memory proxy
+        // fence on the state chain.  Three TMEM accumulator sets keep chunk c's [X; Y] and
+        // P Delta alive until then.
+        float prev_gam = 0.f;
+        auto write_outputs = [&](int cp, float gam_r) {
+            const int tb = cp % kTBufs;
+            if (!wait_or_abort(&ss.mma2[tb], (cp / kTBufs) & 1, abort_flag, header)) return false;
+            tc_fence_after();
+            const int t0 = t_begin + cp * kChunk;
+            const int len = min(kChunk, t_end - t0);
+            float y[32], pd[32];
+            tmem_ld32(tmem, warp, kT_XY + 64 * tb + 32 * ch2, y);
+            tmem_ld32(tmem, warp, kT_PD + 64 * tb + 32 * ch2, pd);
+            if (r < len) {
+                uint4* op = reinterpret_cast<uint4*>(out + ((size_t)(t0 + r) * hv + h) * kD + half * 64 + 32 * ch2);
+#pragma unroll
+                for (int cc = 0; cc < 4; ++cc) {
+                    float o8[8];
+#pragma unroll
+                    for (int e = 0; e < 8; ++e) o8[e] = fmaf(gam_r, y[8 * cc + e], pd[8 * cc + e]);
+                    op[cc] = pack8(o8);
+                }
+            }
+            tc_fence_before();
+            return true;
+        };
+        int c = 0;
+        for (; c < nch; ++c) {
+            const int b = c % kStages, par = c & 1, tb = c % kTBufs;
             unsigned char* buf = sm + b * kS_BUF;
             if (!wait_or_abort(&ss.full[b], (c / kStages) & 1, abort_flag, header)) break;
             const float* cvec = reinterpret_cast<const float*>(sm + kS_CV + b * kCvecLoad);
             const float gl = cvec[128];
             const float crow = delta_warp ? cvec[r] : cvec[64 + r];  // c_r, or gam_r for outputs
-
-            if (delta_warp) {  // Delta = U - X for token row r, columns 32*ch2 .. +32
-                uint4 u4[4];    // this row's U values, read before any shared store of this phase
+            uint4 u4[4];  // this row's U values (Delta warps)
+            if (delta_warp) {
 #pragma unroll
                 for (int cc = 0; cc < 4; ++cc) u4[cc] = *reinterpret_cast<const uint4*>(buf + kS_U + sw128(r, 4 * ch2 + cc));
-                if (c >= 1 && !wait_or_abort(&ss.mma2, (c - 1) & 1, abort_flag, header)) break;  // B2 free
+            }
+            mbar_arrive(&ss.empty[b]);  // this thread's reads of stage b are done (values in registers)
+
+            if (delta_warp) {  // Delta = U - X for token row r, columns 32*ch2 .. +32
+                if (c >= 1 && !wait_or_abort(&ss.mma2[(c - 1) % kTBufs], ((c - 1) / kTBufs) & 1, abort_flag, header))
+                    break;  // B2 and B3 are free once P Delta of c-1 is done
                 if (!wait_or_abort(&ss.mma1, par, abort_flag, header)) break;
                 tc_fence_after();
                 float x[32];
-                tmem_ld32(tmem, warp, kT_XY + 64 * par + 32 * ch2, x);
+                tmem_ld32(tmem, warp, kT_XY + 64 * tb + 32 * ch2, x);
+                float d[32];
 #pragma unroll
                 for (int cc = 0; cc < 4; ++cc) {
-                    const int ch = 4 * ch2 + cc;
-                    float u8[8], d8[8], c8[8];
+                    float u8[8];
                     unpack8(u4[cc], u8);
 #pragma unroll
-                    for (int e = 0; e < 8; ++e) {
-                        d8[e] = u8[e] - x[8 * cc + e];
-                        c8[e] = d8[e] * crow;
-                    }
-                    *reinterpret_cast<uint4*>(sm + kS_B2 + sw128(r, ch)) = pack8(d8);
-                    *reinterpret_cast<uint4*>(sm + kS_B3 + sw128(r, ch)) = pack8(c8);
+                    for (int e = 0; e < 8; ++e) d[8 * cc + e] = u8[e] - x[8 * cc + e];
+                }
+                // diag(c) Delta first: it feeds the state update, the next link of the chain
+#pragma unroll
+                for (int cc = 0; cc < 4; ++cc) {
+                    float c8[8];
+#pragma unroll
+                    for (int e = 0; e < 8; ++e) c8[e] = d[8 * cc + e] * crow;
+                    *reinterpret_cast<uint4*>(sm + kS_B3 + sw128(r, 4 * ch2 + cc)) = pack8(c8);
                 }
                 fence_async_smem();
                 tc_fence_before();
-                mbar_arrive(&ss.b23);
+                mbar_arrive(&ss.b3);
+#pragma unroll
+                for (int cc = 0; cc < 4; ++cc)
+                    *reinterpret_cast<uint4*>(sm + kS_B2 + sw128(r, 4 * ch2 + cc)) = pack8(d + 8 * cc);
+                fence_async_smem();
+                mbar_arrive(&ss.b2);
             }
             // state update S^T <- gam_L S^T + K^T diag(c) Delta (d_k row t, 32 d_v columns)
             if (!wait_or_abort(&ss.mma3, par, abort_flag, header)) break;
@@ -761,27 +812,12 @@ chunk_state_kernel(const float* s0, const int32_t* __restrict__ cu, __nv_bfloat1
             tc_fence_before();
             mbar_arrive(&ss.b1);
 
-            if (!delta_warp) {  // outputs of token row r: O = gam_r Y + P Delta
-                if (!wait_or_abort(&ss.mma2, par, abort_flag, header)) break;
-                tc_fence_after();
-                const int t0 = t_begin + c * kChunk;
-                const int len = min(kChunk, t_end - t0);
-                float y[32], pd[32];
-                tmem_ld32(tmem, warp, kT_XY + 64 * par + 32 * ch2, y);
-                tmem_ld32(tmem, warp, kT_PD + 64 * par + 32 * ch2, pd);
-                if (r < len) {
-                    uint4* op = reinterpret_cast<uint4*>(out + ((size_t)(t0 + r) * hv + h) * kD + half * 64 + 32 * ch2);
-#pragma unroll
-                    for (int cc = 0; cc < 4; ++cc) {
-                        float o8[8];
-#pragma unroll
-                        for (int e = 0; e < 8; ++e) o8[e] = fmaf(crow, y[8 * cc + e], pd[8 * cc + e]);
-                        op[cc] = pack8(o8);
-                    }
-                }
-                tc_fence_before();
+            if (!delta_warp) {  // outputs of the previous chunk: O = gam_r Y + P Delta
+                if (c >= 1 && !write_outputs(c - 1, prev_gam)) break;
+                prev_gam = crow;
             }
         }
+        if (!delta_warp && c == nch && nch > 0 && !*abort_flag) write_outputs(nch - 1, prev_gam);
         if (!*abort_flag && sT) {
 #pragma unroll
             for (int m = 0; m < 32; ++m) sT[sbase + (size_t)m * kD] = S[m];

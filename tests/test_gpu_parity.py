@@ -37,13 +37,17 @@ def assert_close(x, ref, tol, what):
 
 
 def run_prefill(x, algo, want_final=True):
+    """Runs the prefill and checks that no bounded device wait gave up."""
     try:
-        return gdn.prefill(x["q"], x["k"], x["v"], x["g"], x["beta"], x["cu_seqlens"],
-                           x["initial_state"], want_final, algo=algo)
+        ws = gdn.alloc_workspace(gdn.prefill_shape(x["q"], x["v"], x["cu_seqlens"], algo), x["q"].device)
+        res = gdn.prefill(x["q"], x["k"], x["v"], x["g"], x["beta"], x["cu_seqlens"],
+                          x["initial_state"], want_final, algo=algo, workspace=ws)
     except gdn.GdnError as e:
         if e.code == 9:
             pytest.skip("algorithm not available for these inputs")
         raise
+    assert gdn.STATUS[gdn.gdn_get_device_error(ws)] == "GDN_OK"
+    return res
 
 
 def to_dev(x, dev="cuda"):
