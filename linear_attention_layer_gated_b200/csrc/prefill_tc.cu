@@ -14,8 +14,9 @@
 //  K1 chunk_prep_kernel   one CTA per (chunk, QK head), all chunks in parallel, both V
 //                         heads of the QK head:
 //                         - normalisation; K K^T and Q K^T as one M=128 MMA [K; Q] K^T;
-//                         - decay masks A and P; T = (I + A)^-1 in fp32 by forward substitution,
-//                           one column per thread (128 threads = 64 columns x 2 heads);
+//                         - decay masks A and P; T = (I + A)^-1 in fp32 by 16x16 blocks:
+//                           diagonal inverses by forward substitution, then the blocks below
+//                           the diagonal as dense 16x16 products (64 threads per V head);
 //                         - W and U of both heads as M=128 MMAs [T_0 D_0; T_1 D_1] x (K or V),
 //                           so each thread owns one output row and writes 16-byte chunks;
 //                         - bf16 operand images, already in the 128-byte swizzled layout the
@@ -165,20 +166,30 @@ __device__ __forceinline__ float warp_inclusive_scan(float x, int lane) {
     return x;
 }
 
-// fp32 64x64 matrix in shared memory, rows of 64 floats; the float4 groups of row R are
-// XOR-permuted by R so that 32 threads writing 32 different rows hit different banks.
-__device__ __forceinline__ int af_idx(int R, int J) { return R * 64 + 4 * ((J >> 2) ^ (R & 15)) + (J & 3); }
+// fp32 64x64 matrices in shared memory: rows padded to 68 floats, so that 8 threads writing
+// float4s to 8 consecutive rows hit different banks and row reads stay contiguous.
+constexpr int kLdA = 68;
+constexpr int kAfHead = kChunk * kLdA;   // floats per head
+
+// 2^x on the special-function unit (PTX ex2.approx); callers pass arguments <= 0.
+__device__ __forceinline__ float fast_exp2(float x) {
+    float y;
+    asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+    return y;
+}
+constexpr float kLog2e = 1.4426950408889634f;
 
 // ===================================================================== K1
 // Shared memory map (bytes from a 1024-aligned base):
 constexpr uint32_t kP_GR = 0;        // [K; Q] K-major (32 KB)  | after the Gram MMA: V images of both heads
 constexpr uint32_t kP_KT = 32768;    // K MN-major (16 KB)
-constexpr uint32_t kP_AF = 49152;    // A / T fp32, 2 heads (32 KB) | then [T0 D0; T1 D1] images for W and U
-constexpr uint32_t kP_SMALL = 81920; // gates, barrier, TMEM address
+constexpr uint32_t kP_AF = 49152;    // A / T fp32, 2 heads (2 x 17 KB) | then [T0 D0; T1 D1] images for W and U
+constexpr uint32_t kP_XS = 49152 + 2 * kAfHead * 4;  // block-solve scratch, 2 heads x 768 floats (6 KB)
+constexpr uint32_t kP_SMALL = kP_XS + 2 * 768 * 4;   // gates, barrier, TMEM address
 constexpr uint32_t kPrepSmem = kP_SMALL + 2048 + 1024;
 
 struct PrepSmall {
-    float G[2][kChunk];
+    float G[2][kChunk];   // in-chunk gate sums, pre-scaled by log2(e)
     float b[2][kChunk];
     float gam[2][kChunk];
     uint64_t bar_mma;
@@ -194,7 +205,8 @@ chunk_prep_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __re
     unsigned char* sm = reinterpret_cast<unsigned char*>((reinterpret_cast<uintptr_t>(smem_dyn) + 1023) & ~uintptr_t(1023));
     const uint32_t sb = smem_u32(sm);
     PrepSmall& ss = *reinterpret_cast<PrepSmall*>(sm + kP_SMALL);
-    float* af = reinterpret_cast<float*>(sm + kP_AF);   // [head][64][64] (swizzled rows)
+    float* af = reinterpret_cast<float*>(sm + kP_AF);   // [head][64][kLdA]
+    float* xs = reinterpret_cast<float*>(sm + kP_XS);   // [head][768]
 
     const WsLayout L = ws_layout(num_seqs, total_tokens, hk, hv);
     int32_t* header = reinterpret_cast<int32_t*>(ws);
@@ -232,8 +244,8 @@ chunk_prep_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __re
         const float g1 = (lane + 32 < len) ? g[(size_t)(t0 + lane + 32) * hv + h] : 0.f;
         const float G0 = warp_inclusive_scan(g0, lane);
         const float G1 = warp_inclusive_scan(g1, lane) + __shfl_sync(0xffffffffu, G0, 31);
-        ss.G[warp][lane] = G0;
-        ss.G[warp][lane + 32] = G1;
+        ss.G[warp][lane] = G0 * kLog2e;
+        ss.G[warp][lane + 32] = G1 * kLog2e;
         ss.gam[warp][lane] = expf(G0);
         ss.gam[warp][lane + 32] = expf(G1);
         ss.b[warp][lane] = (lane < len) ? beta[(size_t)(t0 + lane) * hv + h] : 0.f;
@@ -319,9 +331,9 @@ chunk_prep_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __re
             for (int hh = 0; hh < 2; ++hh) {
                 float* cv = reinterpret_cast<float*>(ws + L.cvec + ((size_t)cid * hv + h0 + hh) * kCvecBytes);
                 const float Gl = ss.G[hh][len - 1], Gr = ss.G[hh][r];
-                cv[r] = (r < len) ? __expf(Gl - Gr) : 0.f;
+                cv[r] = (r < len) ? fast_exp2(Gl - Gr) : 0.f;
                 cv[64 + r] = ss.gam[hh][r];
-                if (r == 0) cv[128] = __expf(Gl);
+                if (r == 0) cv[128] = ss.gam[hh][len - 1];
             }
         }
         ok = mbar_wait(&ss.bar_mma, 0);
@@ -338,30 +350,36 @@ chunk_prep_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __re
 #pragma unroll
                 for (int hh = 0; hh < 2; ++hh) {
                     const float Gr = ss.G[hh][r], br = ss.b[hh][r];
-                    float4* a4 = reinterpret_cast<float4*>(af + hh * 4096);
+                    const float4* g4 = reinterpret_cast<const float4*>(ss.G[hh]);
+                    float4* a4 = reinterpret_cast<float4*>(af + hh * kAfHead + r * kLdA);
 #pragma unroll
                     for (int m = 0; m < 16; ++m) {
+                        const float4 gi = g4[m];
+                        const float gg[4] = {gi.x, gi.y, gi.z, gi.w};
                         float t4[4];
 #pragma unroll
                         for (int e = 0; e < 4; ++e) {
                             const int i = 4 * m + e;
-                            t4[e] = (i < r) ? br * __expf(Gr - ss.G[hh][i]) * row[i] : 0.f;
+                            t4[e] = (i < r) ? br * fast_exp2(fminf(Gr - gg[e], 0.f)) * row[i] : 0.f;
                         }
-                        a4[r * 16 + (m ^ (r & 15))] = make_float4(t4[0], t4[1], t4[2], t4[3]);
+                        a4[m] = make_float4(t4[0], t4[1], t4[2], t4[3]);
                     }
                 }
             } else {
 #pragma unroll
                 for (int hh = 0; hh < 2; ++hh) {
                     const float Gr = ss.G[hh][r];
+                    const float4* g4 = reinterpret_cast<const float4*>(ss.G[hh]);
                     unsigned char* pimg = ws + L.p + ((size_t)cid * hv + h0 + hh) * kPBytes;
 #pragma unroll
                     for (int ch = 0; ch < 8; ++ch) {
+                        const float4 ga = g4[2 * ch], gb = g4[2 * ch + 1];
+                        const float gg[8] = {ga.x, ga.y, ga.z, ga.w, gb.x, gb.y, gb.z, gb.w};
                         float p8[8];
 #pragma unroll
                         for (int e = 0; e < 8; ++e) {
                             const int i = 8 * ch + e;
-                            p8[e] = (i <= r) ? __expf(Gr - ss.G[hh][i]) * row[i] : 0.f;
+                            p8[e] = (i <= r) ? fast_exp2(fminf(Gr - gg[e], 0.f)) * row[i] : 0.f;
                         }
                         *reinterpret_cast<uint4*>(pimg + sw128(r, ch)) = pack8(p8);
                     }
@@ -382,39 +400,89 @@ chunk_prep_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __re
     tc_fence_before();
     __syncthreads();
 
-    // ---- 4. T = (I + A)^-1: thread = (head, column i), forward substitution over the rows;
-    //         every index is a compile-time constant, the A reads are warp-wide broadcasts.
+    // ---- 4. T = (I + A)^-1 per head, by 16x16 blocks, in place.  Each head uses 64 threads.
+    //         (a) diagonal blocks: D_b = (I + A_bb)^-1 by forward substitution, one column
+    //             per thread; (b) below the diagonal, block row by block row,
+    //             T_ij = -D_i (sum_{k=j}^{i-1} A_ik T_kj), as dense 16x16 products.
     {
-        const int hh = tid >> 6, i = tid & 63;
-        const float4* a4 = reinterpret_cast<const float4*>(af + hh * 4096);
-        float x[kChunk];
+        const int hh = tid >> 6, l = tid & 63;
+        float* A = af + hh * kAfHead;
+        float* X = xs + hh * 768;
+        {
+            const int base = 16 * (l >> 4), j = l & 15;
+            float x[16];
 #pragma unroll
-        for (int r = 0; r < kChunk; ++r) x[r] = 0.f;
-        // column i of (I + A) x = e_i:  x_r = [r == i] - sum_{j<r} A[r][j] x_j  (x_r = 0 for r < i)
+            for (int r = 0; r < 16; ++r) {
+                const float* arow = A + (base + r) * kLdA + base;
+                float acc = 0.f;
 #pragma unroll
-        for (int r = 0; r < kChunk; ++r) {
-            float s0 = 0.f, s1 = 0.f, s2 = 0.f, s3 = 0.f;
-#pragma unroll
-            for (int m = 0; m < (r + 3) / 4; ++m) {
-                const float4 av = a4[r * 16 + (m ^ (r & 15))];
-                s0 = fmaf(av.x, x[4 * m + 0], s0);
-                s1 = fmaf(av.y, x[4 * m + 1], s1);
-                s2 = fmaf(av.z, x[4 * m + 2], s2);
-                s3 = fmaf(av.w, x[4 * m + 3], s3);
+                for (int k = 0; k < r; ++k) acc = fmaf(arow[k], x[k], acc);
+                x[r] = (r == j) ? 1.f : ((r < j) ? 0.f : -acc);
             }
-            x[r] = (r == i) ? 1.f : -((s0 + s1) + (s2 + s3));
+            __syncthreads();
+#pragma unroll
+            for (int r = 0; r < 16; ++r) A[(base + r) * kLdA + base + j] = x[r];
         }
         __syncthreads();
-        // write column i of T back (row r: T[r][i]), then build the W / U operand rows
+        // Output mapping inside a 16x16 block: column cc = l & 15, rows rr0 + 4 q for q = 0..3.
+        const int cc = l & 15, rr0 = l >> 4;
+        // Block rows i = 1, 2, 3 in order.  Row i reads only its own A blocks (still intact)
+        // and blocks of rows < i (already T); it is overwritten only after all its X_ij are formed.
 #pragma unroll
-        for (int r = 0; r < kChunk; ++r) af[hh * 4096 + af_idx(r, i)] = x[r];
+        for (int i = 1; i < 4; ++i) {
+#pragma unroll
+            for (int j = 0; j < i; ++j) {              // X_ij = sum_{k=j}^{i-1} A_ik T_kj
+                float acc[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+                for (int k = j; k < i; ++k) {
+                    float tcol[16];
+#pragma unroll
+                    for (int m = 0; m < 16; ++m) tcol[m] = A[(16 * k + m) * kLdA + 16 * j + cc];
+#pragma unroll
+                    for (int q = 0; q < 4; ++q) {
+                        const float4* ar = reinterpret_cast<const float4*>(A + (16 * i + rr0 + 4 * q) * kLdA + 16 * k);
+#pragma unroll
+                        for (int m4 = 0; m4 < 4; ++m4) {
+                            const float4 a = ar[m4];
+                            acc[q] = fmaf(a.x, tcol[4 * m4 + 0], acc[q]);
+                            acc[q] = fmaf(a.y, tcol[4 * m4 + 1], acc[q]);
+                            acc[q] = fmaf(a.z, tcol[4 * m4 + 2], acc[q]);
+                            acc[q] = fmaf(a.w, tcol[4 * m4 + 3], acc[q]);
+                        }
+                    }
+                }
+#pragma unroll
+                for (int q = 0; q < 4; ++q) X[j * 256 + (rr0 + 4 * q) * 16 + cc] = acc[q];
+            }
+            __syncthreads();
+#pragma unroll
+            for (int j = 0; j < i; ++j) {              // T_ij = -D_i X_ij
+                float xcol[16];
+#pragma unroll
+                for (int m = 0; m < 16; ++m) xcol[m] = X[j * 256 + m * 16 + cc];
+#pragma unroll
+                for (int q = 0; q < 4; ++q) {
+                    const float4* dr = reinterpret_cast<const float4*>(A + (16 * i + rr0 + 4 * q) * kLdA + 16 * i);
+                    float acc = 0.f;
+#pragma unroll
+                    for (int m4 = 0; m4 < 4; ++m4) {
+                        const float4 d = dr[m4];
+                        acc = fmaf(d.x, xcol[4 * m4 + 0], acc);
+                        acc = fmaf(d.y, xcol[4 * m4 + 1], acc);
+                        acc = fmaf(d.z, xcol[4 * m4 + 2], acc);
+                        acc = fmaf(d.w, xcol[4 * m4 + 3], acc);
+                    }
+                    A[(16 * i + rr0 + 4 * q) * kLdA + 16 * j + cc] = -acc;
+                }
+            }
+            __syncthreads();
+        }
     }
-    __syncthreads();
 
     // ---- 5. MMA operand images [T_0 diag(b_0 gam_0); T_1 diag(b_1 gam_1)] and [T_0 diag(b_0); ...]
     {
         const int hh = tid >> 6, r = tid & 63;
-        const float4* t4 = reinterpret_cast<const float4*>(af + hh * 4096);
+        const float4* t4 = reinterpret_cast<const float4*>(af + hh * kAfHead + r * kLdA);
         uint4 wrow[8], urow[8];
 #pragma unroll
         for (int ch = 0; ch < 8; ++ch) {
@@ -422,7 +490,7 @@ chunk_prep_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __re
 #pragma unroll
             for (int half4 = 0; half4 < 2; ++half4) {
                 const int m = 2 * ch + half4;   // float4 group: columns 4m .. 4m+3
-                const float4 tv = t4[r * 16 + (m ^ (r & 15))];
+                const float4 tv = t4[m];
                 const float tt[4] = {tv.x, tv.y, tv.z, tv.w};
 #pragma unroll
                 for (int e = 0; e < 4; ++e) {
