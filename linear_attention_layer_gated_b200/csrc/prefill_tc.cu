@@ -347,7 +347,7 @@ chunk_prep_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __re
             tmem_ld64(tmem, warp, 0, row);
             const int r = tid & 63;
             if (warp < 2) {
-#pragma unroll
+#pragma unroll 1
                 for (int hh = 0; hh < 2; ++hh) {
                     const float Gr = ss.G[hh][r], br = ss.b[hh][r];
                     const float4* g4 = reinterpret_cast<const float4*>(ss.G[hh]);
@@ -366,7 +366,7 @@ chunk_prep_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __re
                     }
                 }
             } else {
-#pragma unroll
+#pragma unroll 1
                 for (int hh = 0; hh < 2; ++hh) {
                     const float Gr = ss.G[hh][r];
                     const float4* g4 = reinterpret_cast<const float4*>(ss.G[hh]);
@@ -428,19 +428,24 @@ chunk_prep_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __re
         const int cc = l & 15, rr0 = l >> 4;
         // Block rows i = 1, 2, 3 in order.  Row i reads only its own A blocks (still intact)
         // and blocks of rows < i (already T); it is overwritten only after all its X_ij are formed.
-#pragma unroll
+        // The block loops stay rolled (small code); each 16-term dot product is unrolled.
+#pragma unroll 1
         for (int i = 1; i < 4; ++i) {
+            const float* arow[4];
 #pragma unroll
+            for (int q = 0; q < 4; ++q) arow[q] = A + (16 * i + rr0 + 4 * q) * kLdA;
+#pragma unroll 1
             for (int j = 0; j < i; ++j) {              // X_ij = sum_{k=j}^{i-1} A_ik T_kj
                 float acc[4] = {0.f, 0.f, 0.f, 0.f};
-#pragma unroll
+#pragma unroll 1
                 for (int k = j; k < i; ++k) {
+                    const float* tc = A + (16 * k) * kLdA + 16 * j + cc;
                     float tcol[16];
 #pragma unroll
-                    for (int m = 0; m < 16; ++m) tcol[m] = A[(16 * k + m) * kLdA + 16 * j + cc];
+                    for (int m = 0; m < 16; ++m) tcol[m] = tc[m * kLdA];
 #pragma unroll
                     for (int q = 0; q < 4; ++q) {
-                        const float4* ar = reinterpret_cast<const float4*>(A + (16 * i + rr0 + 4 * q) * kLdA + 16 * k);
+                        const float4* ar = reinterpret_cast<const float4*>(arow[q] + 16 * k);
 #pragma unroll
                         for (int m4 = 0; m4 < 4; ++m4) {
                             const float4 a = ar[m4];
@@ -455,14 +460,14 @@ chunk_prep_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __re
                 for (int q = 0; q < 4; ++q) X[j * 256 + (rr0 + 4 * q) * 16 + cc] = acc[q];
             }
             __syncthreads();
-#pragma unroll
+#pragma unroll 1
             for (int j = 0; j < i; ++j) {              // T_ij = -D_i X_ij
                 float xcol[16];
 #pragma unroll
                 for (int m = 0; m < 16; ++m) xcol[m] = X[j * 256 + m * 16 + cc];
 #pragma unroll
                 for (int q = 0; q < 4; ++q) {
-                    const float4* dr = reinterpret_cast<const float4*>(A + (16 * i + rr0 + 4 * q) * kLdA + 16 * i);
+                    const float4* dr = reinterpret_cast<const float4*>(arow[q] + 16 * i);
                     float acc = 0.f;
 #pragma unroll
                     for (int m4 = 0; m4 < 4; ++m4) {
