@@ -17,16 +17,27 @@
 //
 // which is the token recurrence unrolled (delta_t is beta_t (v_t - alpha_t S_{t-1} k_t)).
 // The k.k and k.q scalars and the gate factors are per (n, h) and computed once per
-// CTA.  Each half-warp owns one state row per step: lane l holds columns 4l..4l+3 and
-// 64+4l..64+4l+3, so a row is two coalesced 256-byte loads and stores, and the dot
-// products reduce over 16 lanes with shuffles.
+// CTA.
+//
+// Memory: at entry every warp issues asynchronous 16-byte copies (cp.async, no waits
+// that could spin) of its 32 state rows into shared memory, so a CTA has its whole
+// 64 KiB head in flight before it does anything else; three CTAs fit on an SM.
+// Compute: a half-warp takes R rows at a time; lane l holds columns 4l..4l+3 and
+// 64+4l..64+4l+3 of each.  The 2m dot products of R rows (16 partial sums per lane)
+// are reduced over the 16 lanes with a transposing butterfly -- each exchange step
+// sends half of the remaining sums and keeps the other half -- so 15 shuffles leave
+// lane l with the complete sum number l, instead of 4 shuffles per sum.  The 16 sums
+// go through shared memory to every lane of the half-warp, each lane evaluates the
+// scalar recurrence for the R rows, and the new rows are streamed to HBM.
 #include "gdn_internal.cuh"
 
 namespace gdn {
 namespace {
 
 constexpr int kDecodeThreads = 128;  // 4 warps; warp w owns state rows [32w, 32w + 32)
+constexpr int kRowsPerWarp = kD / 4;
 constexpr float kInvSqrtD = 0.08838834764831845f;  // 1 / sqrt(128)
+constexpr size_t kStateSmemBytes = (size_t)kD * kD * sizeof(float);  // 64 KiB
 
 __device__ __forceinline__ float sum16(float x) {
     x += __shfl_xor_sync(0xffffffffu, x, 8);
@@ -50,12 +61,52 @@ __device__ __forceinline__ void load_cols(const IO* row, int l, float* dst) {
     dst[4] = b.x; dst[5] = b.y; dst[6] = b.z; dst[7] = b.w;
 }
 
-template <typename IO, int NTOK, int UNR>
-__global__ void __launch_bounds__(kDecodeThreads)
+__device__ __forceinline__ void cp_async16(void* dst_smem, const void* src) {
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(
+                     static_cast<uint32_t>(__cvta_generic_to_shared(dst_smem))),
+                 "l"(src)
+                 : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+template <int N>
+__device__ __forceinline__ void cp_async_wait() { asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory"); }
+
+// Transposing butterfly over the 16 lanes of a half-warp.  On entry a[0..CUR) are this
+// lane's partial sums of CUR quantities; each level with CUR >= 2 swaps half of them
+// with the partner lane (l ^ M) and keeps the other half, adding the partner's copy.
+// On exit (16 quantities) lane l holds in a[0] the full sum of quantity number l.
+template <int CUR, int M>
+__device__ __forceinline__ void xpose_reduce(float* a, int l) {
+    if constexpr (M > 0) {
+        static_assert(CUR >= 2, "needs at least as many quantities as lanes");
+        const bool up = (l & M) != 0;
+#pragma unroll
+        for (int i = 0; i < CUR / 2; ++i) {
+            const float send = up ? a[i] : a[i + CUR / 2];
+            const float keep = up ? a[i + CUR / 2] : a[i];
+            a[i] = keep + __shfl_xor_sync(0xffffffffu, send, M);
+        }
+        xpose_reduce<CUR / 2, M / 2>(a, l);
+    }
+}
+
+// NTOK tokens of one step; R rows per half-warp per iteration, with 2 * NT * R == 16
+// partial sums per lane (NT = NTOK rounded up to a power of two; a padding slot is 0).
+template <typename IO, int NTOK, int R>
+__global__ void __launch_bounds__(kDecodeThreads, 3)
 decode_kernel(const IO* __restrict__ q, const IO* __restrict__ k, const IO* __restrict__ v,
               const float* __restrict__ g, const float* __restrict__ beta,
               float* __restrict__ state, IO* __restrict__ out, int hk, int hv)
 {
+    constexpr int NT = NTOK == 3 ? 4 : NTOK;
+    constexpr int VR = 2 * NT;           // sums per row: x_0..x_{NT-1}, y_0..y_{NT-1}
+    static_assert(VR * R == 16, "one sum per lane after the butterfly");
+    constexpr int kRowsPerIter = 2 * R;  // both half-warps
+    constexpr int kIters = kRowsPerWarp / kRowsPerIter;
+    constexpr int kGroups = kIters < 4 ? kIters : 4;  // cp.async groups per warp
+    constexpr int kItersPerGroup = kIters / kGroups;
+    constexpr int kRowsPerGroup = kRowsPerWarp / kGroups;
+
     const int n = blockIdx.x / hv;
     const int h = blockIdx.x % hv;
     const int qh = h / (hv / hk);
@@ -64,15 +115,29 @@ decode_kernel(const IO* __restrict__ q, const IO* __restrict__ k, const IO* __re
     const int half = lane >> 4;
     const int l = lane & 15;
 
+    extern __shared__ __align__(16) float s_state[];  // [kD][kD], row-major like HBM
     __shared__ float v_s[NTOK][kD];
     __shared__ float o_s[NTOK][kD];
+    __shared__ __align__(16) float red_s[2][4][2][16];  // [parity][warp][half][sum]
 
+    float* S = state + ((size_t)n * hv + h) * kD * kD;
+
+    // 1. This warp's 32 rows start moving HBM -> shared memory immediately.
+#pragma unroll
+    for (int grp = 0; grp < kGroups; ++grp) {
+#pragma unroll
+        for (int j = 0; j < kRowsPerGroup; ++j) {
+            const int row = warp * kRowsPerWarp + grp * kRowsPerGroup + j;
+            cp_async16(s_state + row * kD + 4 * lane, S + row * kD + 4 * lane);
+        }
+        cp_async_commit();
+    }
+
+    // 2. Per-(n, h) inputs while the state is in flight.
     for (int idx = threadIdx.x; idx < NTOK * kD; idx += kDecodeThreads) {
         const int t = idx / kD, i = idx % kD;
         v_s[t][i] = to_f32(v[(((size_t)n * NTOK + t) * hv + h) * kD + i]);
     }
-
-    // Normalised key / query columns owned by this lane (both half-warps hold the same).
     float kr[NTOK][8], qr[NTOK][8];
 #pragma unroll
     for (int t = 0; t < NTOK; ++t) {
@@ -84,8 +149,6 @@ decode_kernel(const IO* __restrict__ q, const IO* __restrict__ k, const IO* __re
 #pragma unroll
         for (int c = 0; c < 8; ++c) { kr[t][c] *= rk; qr[t][c] *= rq; }
     }
-
-    // Per-(n, h) scalars: gate sums, decay-weighted k.k and k.q, final weights.
     float G[NTOK], bt[NTOK];
     {
         float acc = 0.f;
@@ -110,59 +173,90 @@ decode_kernel(const IO* __restrict__ q, const IO* __restrict__ k, const IO* __re
             if (j <= t) Em[t][j] = expf(G[t] - G[j]) * sum16(dot8(kr[j], qr[t]));
         }
     }
-    __syncthreads();
+    __syncthreads();  // v_s
 
-    float* S = state + ((size_t)n * hv + h) * kD * kD;
+    // 3. Rows, group by group as their copies land.
+#pragma unroll
+    for (int grp = 0; grp < kGroups; ++grp) {
+        if (grp == 0) cp_async_wait<kGroups - 1>();
+        else if (grp == 1) cp_async_wait<(kGroups > 1 ? kGroups - 2 : 0)>();
+        else if (grp == 2) cp_async_wait<(kGroups > 2 ? kGroups - 3 : 0)>();
+        else cp_async_wait<0>();
+        __syncwarp();  // every lane's copies of this group are visible to the warp
 #pragma unroll 1
-    for (int p0 = 0; p0 < 16; p0 += UNR) {
-        float4 sa[UNR], sb[UNR];
+        for (int it = grp * kItersPerGroup; it < (grp + 1) * kItersPerGroup; ++it) {
+            const int row0 = warp * kRowsPerWarp + it * kRowsPerIter + half * R;
+            float s[R][8];
+            float a[16];
 #pragma unroll
-        for (int u = 0; u < UNR; ++u) {
-            const int row = warp * 32 + 2 * (p0 + u) + half;
-            sa[u] = __ldcs(reinterpret_cast<const float4*>(S + row * kD + 4 * l));
-            sb[u] = __ldcs(reinterpret_cast<const float4*>(S + row * kD + 64 + 4 * l));
-        }
+            for (int r = 0; r < R; ++r) {
+                load_cols(s_state + (row0 + r) * kD, l, s[r]);
 #pragma unroll
-        for (int u = 0; u < UNR; ++u) {
-            const int row = warp * 32 + 2 * (p0 + u) + half;
-            float s[8] = {sa[u].x, sa[u].y, sa[u].z, sa[u].w, sb[u].x, sb[u].y, sb[u].z, sb[u].w};
-            float x[NTOK], y[NTOK];
-#pragma unroll
-            for (int t = 0; t < NTOK; ++t) {
-                x[t] = sum16(dot8(s, kr[t]));
-                y[t] = sum16(dot8(s, qr[t]));
+                for (int t = 0; t < NT; ++t) {
+                    a[r * VR + t] = t < NTOK ? dot8(s[r], kr[t < NTOK ? t : 0]) : 0.f;
+                    a[r * VR + NT + t] = t < NTOK ? dot8(s[r], qr[t < NTOK ? t : 0]) : 0.f;
+                }
             }
-            float delta[NTOK];
+            xpose_reduce<16, 8>(a, l);
+            float* red = red_s[it & 1][warp][half];
+            red[l] = a[0];
+            __syncwarp();
 #pragma unroll
-            for (int t = 0; t < NTOK; ++t) {
-                float a = Gam[t] * x[t];
+            for (int r = 0; r < R; ++r) {
+                float xy[VR];
 #pragma unroll
-                for (int j = 0; j < t; ++j) a = fmaf(Dm[t][j], delta[j], a);
-                delta[t] = bt[t] * (v_s[t][row] - a);
-                float o = Gam[t] * y[t];
+                for (int c4 = 0; c4 < VR; c4 += 4) {
+                    const float4 u = *reinterpret_cast<const float4*>(red + r * VR + c4);
+                    xy[c4] = u.x; xy[c4 + 1] = u.y; xy[c4 + 2] = u.z; xy[c4 + 3] = u.w;
+                }
+                const int row = row0 + r;
+                float delta[NTOK];
 #pragma unroll
-                for (int j = 0; j <= t; ++j) o = fmaf(Em[t][j], delta[j], o);
-                if (l == 0) o_s[t][row] = o;
+                for (int t = 0; t < NTOK; ++t) {
+                    float x = Gam[t] * xy[t];
+#pragma unroll
+                    for (int j = 0; j < t; ++j) x = fmaf(Dm[t][j], delta[j], x);
+                    delta[t] = bt[t] * (v_s[t][row] - x);
+                    float o = Gam[t] * xy[NT + t];
+#pragma unroll
+                    for (int j = 0; j <= t; ++j) o = fmaf(Em[t][j], delta[j], o);
+                    if (l == 0) o_s[t][row] = o;
+                }
+                float w[NTOK];
+#pragma unroll
+                for (int j = 0; j < NTOK; ++j) w[j] = F[j] * delta[j];
+#pragma unroll
+                for (int c = 0; c < 8; ++c) {
+                    float y = Gam[NTOK - 1] * s[r][c];
+#pragma unroll
+                    for (int j = 0; j < NTOK; ++j) y = fmaf(w[j], kr[j][c], y);
+                    s[r][c] = y;
+                }
+                __stcs(reinterpret_cast<float4*>(S + row * kD + 4 * l),
+                       make_float4(s[r][0], s[r][1], s[r][2], s[r][3]));
+                __stcs(reinterpret_cast<float4*>(S + row * kD + 64 + 4 * l),
+                       make_float4(s[r][4], s[r][5], s[r][6], s[r][7]));
             }
-            float w[NTOK];
-#pragma unroll
-            for (int j = 0; j < NTOK; ++j) w[j] = F[j] * delta[j];
-#pragma unroll
-            for (int c = 0; c < 8; ++c) {
-                float r = Gam[NTOK - 1] * s[c];
-#pragma unroll
-                for (int j = 0; j < NTOK; ++j) r = fmaf(w[j], kr[j][c], r);
-                s[c] = r;
-            }
-            __stcs(reinterpret_cast<float4*>(S + row * kD + 4 * l), make_float4(s[0], s[1], s[2], s[3]));
-            __stcs(reinterpret_cast<float4*>(S + row * kD + 64 + 4 * l), make_float4(s[4], s[5], s[6], s[7]));
         }
     }
-    __syncthreads();
+    __syncthreads();  // o_s
     for (int idx = threadIdx.x; idx < NTOK * kD; idx += kDecodeThreads) {
         const int t = idx / kD, i = idx % kD;
         out[(((size_t)n * NTOK + t) * hv + h) * kD + i] = from_f32<IO>(o_s[t][i]);
     }
+}
+
+template <typename IO, int NTOK, int R>
+cudaError_t launch_one(const IO* q, const IO* k, const IO* v, const float* g, const float* beta,
+                       float* state, IO* out, int num_seqs, int hk, int hv, cudaStream_t stream)
+{
+    auto kernel = decode_kernel<IO, NTOK, R>;
+    cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         (int)kStateSmemBytes);
+    if (e != cudaSuccess) return e;
+    kernel<<<dim3((unsigned)num_seqs * (unsigned)hv), dim3(kDecodeThreads), kStateSmemBytes,
+             stream>>>(q, k, v, g, beta, state, out, hk, hv);
+    return cudaGetLastError();
 }
 
 template <typename IO>
@@ -170,15 +264,12 @@ cudaError_t launch_typed(const IO* q, const IO* k, const IO* v, const float* g,
                          const float* beta, float* state, IO* out, int ntok, int num_seqs,
                          int hk, int hv, cudaStream_t stream)
 {
-    const dim3 grid((unsigned)num_seqs * (unsigned)hv);
-    const dim3 block(kDecodeThreads);
     switch (ntok) {
-    case 1: decode_kernel<IO, 1, 4><<<grid, block, 0, stream>>>(q, k, v, g, beta, state, out, hk, hv); break;
-    case 2: decode_kernel<IO, 2, 4><<<grid, block, 0, stream>>>(q, k, v, g, beta, state, out, hk, hv); break;
-    case 3: decode_kernel<IO, 3, 2><<<grid, block, 0, stream>>>(q, k, v, g, beta, state, out, hk, hv); break;
-    default: decode_kernel<IO, 4, 2><<<grid, block, 0, stream>>>(q, k, v, g, beta, state, out, hk, hv); break;
+    case 1: return launch_one<IO, 1, 8>(q, k, v, g, beta, state, out, num_seqs, hk, hv, stream);
+    case 2: return launch_one<IO, 2, 4>(q, k, v, g, beta, state, out, num_seqs, hk, hv, stream);
+    case 3: return launch_one<IO, 3, 2>(q, k, v, g, beta, state, out, num_seqs, hk, hv, stream);
+    default: return launch_one<IO, 4, 2>(q, k, v, g, beta, state, out, num_seqs, hk, hv, stream);
     }
-    return cudaGetLastError();
 }
 
 }  // namespace
