@@ -22,10 +22,12 @@
 //                         - bf16 operand images, already in the 128-byte swizzled layout the
 //                           state kernel's MMAs read, go to the workspace, with the gate
 //                           factors (c, gam) of each V head.
-//  K2 chunk_state_kernel  one CTA per (sequence, V head, half of d_v), sequential over the
-//                         sequence's chunks.  Warp 8 issues the MMAs, warp 9 the bulk copies
-//                         (two chunks ahead, three buffers); warps 0-7 compute, each warp on
-//                         32 of the 64 d_v columns of its TMEM lane quarter.  Per chunk:
+//  K2 chunk_state_kernel  one CTA per (sequence, V head, quarter of d_v): the rows of S (one
+//                         per d_v index) evolve independently, so the 32-row slices run on
+//                         separate SMs, sequentially over the sequence's chunks.  Warp 8
+//                         issues the MMAs (N = 32), warp 9 the bulk copies (two chunks
+//                         ahead, three buffers); warps 0-7 compute, each warp on 16 of the
+//                         32 d_v columns of its TMEM lane quarter.  Per chunk:
 //                           [X; Y] = [W; Q] S^T          (M=128)            <- on the chain
 //                           Delta = U - X, c Delta       (lanes 0-63: token rows)
 //                           K^T diag(c) Delta            (M=128: d_k rows)  <- on the chain
@@ -57,11 +59,12 @@ constexpr uint32_t kUBytes = 16384;    // U: [d_v half][64 rows][64]
 constexpr uint32_t kPBytes = 8192;     // P: 64 token rows x 64, K-major
 constexpr uint32_t kCvecBytes = 1024;  // c_j at [0,64), gam_r at [64,128), gam_L at [128]
 constexpr uint32_t kCvecLoad = 528;    // the bytes of a gate-factor record the state kernel reads
-constexpr uint32_t kKTBytes = 16384;   // K, [d_k block][64 token rows] (MN-major A operand)
-constexpr uint32_t kChunkLoadBytes = kWBytes + kQBytes + kKTBytes + kUBytes / 2 + kPBytes + kCvecLoad;
+constexpr uint32_t kKTBytes = 16384;   // diag(c) K (per V head), [d_k block][64 token rows] (MN-major A operand)
+constexpr uint32_t kMBytes = 8192;     // M = W K_prev^T diag(c_prev): 64 token rows x 64 previous-chunk tokens,
+                                       // K-major
 
 struct WsLayout {
-    size_t seq_chunk0, table, w, u, p, cvec, kt, qn, total;
+    size_t seq_chunk0, table, w, u, p, cvec, kt, qn, m, total;
     long long max_chunks;
 };
 
@@ -84,9 +87,11 @@ __host__ __device__ inline WsLayout ws_layout(int num_seqs, int total_tokens, in
     L.cvec = off;
     off += (size_t)L.max_chunks * hv * kCvecBytes;
     L.kt = off;
-    off += (size_t)L.max_chunks * hk * kKTBytes;
+    off += (size_t)L.max_chunks * hv * kKTBytes;
     L.qn = off;
     off += (size_t)L.max_chunks * hk * kQBytes;
+    L.m = off;
+    off += (size_t)L.max_chunks * hv * kMBytes;
     L.total = round_up(off, 1024);
     return L;
 }
@@ -157,6 +162,12 @@ __device__ __forceinline__ float sum8(float x) {  // over groups of 8 consecutiv
     return x;
 }
 
+__device__ __forceinline__ float warp_sum(float x) {
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) x += __shfl_xor_sync(0xffffffffu, x, o);
+    return x;
+}
+
 __device__ __forceinline__ float warp_inclusive_scan(float x, int lane) {
 #pragma unroll
     for (int o = 1; o < 32; o <<= 1) {
@@ -181,20 +192,31 @@ constexpr float kLog2e = 1.4426950408889634f;
 
 // ===================================================================== K1
 // Shared memory map (bytes from a 1024-aligned base):
-constexpr uint32_t kP_GR = 0;        // [K; Q] K-major (32 KB)  | after the Gram MMA: V images of both heads
-constexpr uint32_t kP_KT = 32768;    // K MN-major (16 KB)
-constexpr uint32_t kP_AF = 49152;    // A / T fp32, 2 heads (2 x 17 KB) | then [T0 D0; T1 D1] images for W and U
-constexpr uint32_t kP_XS = 49152 + 2 * kAfHead * 4;  // block-solve scratch, 2 heads x 768 floats (6 KB)
+//   kP_GR  per d_k block b (b = 0, 1) at b * kP_GRB: rows of Q | K | K_prev (8 KB each), K-major.
+//          The Gram MMA reads A = [Q; K] and B = [K; K_prev] (128 rows each) from it.  After
+//          the Gram, the Q and K_prev slots take the V images of both heads; the K slot stays
+//          (it is the MN-major B operand of W = [T D] K).
+//   kP_GX  K K_prev^T in bf16, MN-major B operand of M = [T D] (K K_prev^T) (8 KB)
+//   kP_AF  at entry: raw K_prev rows (16 KB); then A / T fp32 (2 heads x 17 KB); then the
+//          [T0 D0; T1 D1] and [T0 B0; T1 B1] operand images (2 x 16 KB)
+constexpr uint32_t kP_GR = 0;
+constexpr uint32_t kP_GRB = 24576;
+constexpr uint32_t kP_GX = 2 * kP_GRB;
+constexpr uint32_t kP_AF = kP_GX + 8192;
+constexpr uint32_t kP_XS = kP_AF + 2 * kAfHead * 4;  // block-solve scratch, 2 heads x 768 floats (6 KB)
 constexpr uint32_t kP_SMALL = kP_XS + 2 * 768 * 4;   // gates, barrier, TMEM address
-constexpr uint32_t kPrepSmem = kP_SMALL + 2048 + 1024;
+constexpr uint32_t kPrepSmem = kP_SMALL + 3072 + 1024;  // small struct + alignment slack
 
 struct PrepSmall {
     float G[2][kChunk];   // in-chunk gate sums, pre-scaled by log2(e)
     float b[2][kChunk];
     float gam[2][kChunk];
+    float cprev[2][kChunk];  // c of the previous chunk, exp(G_L - G_j), or 0 (16-byte aligned)
+    float gprev[2];       // exp(total gate sum of the previous chunk of the sequence), or 1
     uint64_t bar_mma;
     uint32_t tmem_base;
 };
+static_assert(sizeof(PrepSmall) <= 3072, "PrepSmall fits its region");
 
 __global__ void __launch_bounds__(kThreads, 2)
 chunk_prep_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __restrict__ k,
@@ -217,13 +239,24 @@ chunk_prep_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __re
     const int t0 = ent.y, len = ent.z;
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const int h0 = jq * 2;  // the two V heads of this QK head
+    // The previous chunk (always a full one) belongs to the same sequence unless this chunk
+    // is the sequence's first.
+    const bool has_prev = cid > reinterpret_cast<const int32_t*>(ws + L.seq_chunk0)[ent.x];
 
     // Thread's slice of a row for the row loads: 16 elements = 2 chunks of one 64-wide block.
     const int sub = tid & 7, kb = sub >> 2, c0 = (sub & 3) * 2;
     int err = 0;
     bool ok;
 
-    // ---- 0. issue the q, k row loads (4 passes of 16 rows), gates, TMEM, barrier
+    // ---- 0. K_prev rows to a staging area (async), the q, k row loads (4 passes of 16 rows),
+    //         gates, TMEM, barrier
+    if (has_prev) {
+        for (int i = tid; i < kChunk * 16; i += kThreads) {  // 64 rows x 16 pieces of 16 bytes
+            const int r = i >> 4, pc = i & 15;
+            cp_async16(sm + kP_AF + r * 256 + pc * 16, k + ((size_t)(t0 - kChunk + r) * hk + jq) * kD + pc * 8);
+        }
+        cp_async_commit();
+    }
     uint4 kr[4][2], qr[4][2];
 #pragma unroll
     for (int pass = 0; pass < 4; ++pass) {
@@ -250,6 +283,14 @@ chunk_prep_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __re
         ss.gam[warp][lane + 32] = expf(G1);
         ss.b[warp][lane] = (lane < len) ? beta[(size_t)(t0 + lane) * hv + h] : 0.f;
         ss.b[warp][lane + 32] = (lane + 32 < len) ? beta[(size_t)(t0 + lane + 32) * hv + h] : 0.f;
+        const float gp0 = has_prev ? g[(size_t)(t0 - kChunk + lane) * hv + h] : 0.f;
+        const float gp1 = has_prev ? g[(size_t)(t0 - kChunk + 32 + lane) * hv + h] : 0.f;
+        const float Gp0 = warp_inclusive_scan(gp0, lane);
+        const float Gp1 = warp_inclusive_scan(gp1, lane) + __shfl_sync(0xffffffffu, Gp0, 31);
+        const float GpL = __shfl_sync(0xffffffffu, Gp1, 31);
+        ss.cprev[warp][lane] = has_prev ? expf(GpL - Gp0) : 0.f;
+        ss.cprev[warp][lane + 32] = has_prev ? expf(GpL - Gp1) : 0.f;
+        if (lane == 0) ss.gprev[warp] = has_prev ? expf(GpL) : 1.f;
     }
     if (warp == 3) {
         tmem_alloc(&ss.tmem_base, 256);
@@ -264,9 +305,11 @@ chunk_prep_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __re
     tc_fence_after();
     const uint32_t tmem = ss.tmem_base;
 
-    // ---- 1. normalise; [K; Q] K-major and K MN-major in smem; K and Q images to the workspace
+    // ---- 1. normalise; Q, K and K_prev rows K-major in smem; Q and diag(c) K images to the
+    //         workspace (the latter once per V head)
     {
-        unsigned char* kt_img = ws + L.kt + ((size_t)cid * hk + jq) * kKTBytes;
+        unsigned char* kt_img0 = ws + L.kt + ((size_t)cid * hv + h0) * kKTBytes;
+        unsigned char* kt_img1 = kt_img0 + kKTBytes;
         unsigned char* qn_img = ws + L.qn + ((size_t)cid * hk + jq) * kQBytes;
 #pragma unroll
         for (int pass = 0; pass < 4; ++pass) {
@@ -283,29 +326,60 @@ chunk_prep_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __re
             const float rq = rsqrtf(sum8(ssq) + kNormEps) * kInvSqrtD;
 #pragma unroll
             for (int e = 0; e < 16; ++e) { kv[e] *= rk; qv[e] *= rq; }
+            // c_r = exp(G_L - G_r) of each V head (0 beyond the chunk's length)
+            const float cr0 = (r < len) ? fast_exp2(ss.G[0][len - 1] - ss.G[0][r]) : 0.f;
+            const float cr1 = (r < len) ? fast_exp2(ss.G[1][len - 1] - ss.G[1][r]) : 0.f;
 #pragma unroll
             for (int cc = 0; cc < 2; ++cc) {
                 const int ch = c0 + cc;
                 const uint4 kp8 = pack8(kv + 8 * cc), qp8 = pack8(qv + 8 * cc);
-                *reinterpret_cast<uint4*>(sm + kP_GR + kb * 16384 + sw128(r, ch)) = kp8;
-                *reinterpret_cast<uint4*>(sm + kP_GR + kb * 16384 + sw128(64 + r, ch)) = qp8;
-                *reinterpret_cast<uint4*>(sm + kP_KT + kb * 8192 + sw128(r, ch)) = kp8;
-                *reinterpret_cast<uint4*>(kt_img + kb * 8192 + sw128(r, ch)) = kp8;
+                float k0[8], k1[8];
+#pragma unroll
+                for (int e = 0; e < 8; ++e) { k0[e] = kv[8 * cc + e] * cr0; k1[e] = kv[8 * cc + e] * cr1; }
+                *reinterpret_cast<uint4*>(sm + kP_GR + kb * kP_GRB + sw128(r, ch)) = qp8;
+                *reinterpret_cast<uint4*>(sm + kP_GR + kb * kP_GRB + 8192 + sw128(r, ch)) = kp8;
+                *reinterpret_cast<uint4*>(kt_img0 + kb * 8192 + sw128(r, ch)) = pack8(k0);
+                *reinterpret_cast<uint4*>(kt_img1 + kb * 8192 + sw128(r, ch)) = pack8(k1);
                 *reinterpret_cast<uint4*>(qn_img + kb * 8192 + sw128(r, ch)) = qp8;
             }
         }
     }
+    if (has_prev) cp_async_wait_all();
+    __syncthreads();  // the staged K_prev rows are visible to every thread
+#pragma unroll 1
+    for (int pass = 0; pass < 4; ++pass) {
+        const int r = pass * 16 + (tid >> 3);
+        float kv[16];
+        if (has_prev) {
+            const uint4* src = reinterpret_cast<const uint4*>(sm + kP_AF + r * 256 + sub * 32);
+            unpack8(src[0], kv);
+            unpack8(src[1], kv + 8);
+        } else {
+#pragma unroll
+            for (int e = 0; e < 16; ++e) kv[e] = 0.f;
+        }
+        float ssk = 0.f;
+#pragma unroll
+        for (int e = 0; e < 16; ++e) ssk = fmaf(kv[e], kv[e], ssk);
+        const float rk = rsqrtf(sum8(ssk) + kNormEps);
+#pragma unroll
+        for (int e = 0; e < 16; ++e) kv[e] *= rk;
+#pragma unroll
+        for (int cc = 0; cc < 2; ++cc)
+            *reinterpret_cast<uint4*>(sm + kP_GR + kb * kP_GRB + 16384 + sw128(r, c0 + cc)) = pack8(kv + 8 * cc);
+    }
     fence_async_smem();
     __syncthreads();
 
-    // ---- 2. Gram: TMEM[0:128, 0:64] = [K; Q] K^T  (M=128, N=64, K=128); V loads meanwhile
+    // ---- 2. Gram: TMEM[0:128, 0:128] = [Q; K] [K; K_prev]^T  (M=128, N=128, K=128); V loads
+    //         meanwhile.  Rows 0..63: Q K^T | Q K_prev^T (unused); rows 64..127: K K^T | K K_prev^T.
     if (tid == 0) {
         tc_fence_after();
-        const uint32_t idesc = idesc_bf16(128, 64, 0, 0);
+        const uint32_t idesc = idesc_bf16(128, 128, 0, 0);
 #pragma unroll
         for (int s = 0; s < 8; ++s) {
-            const uint32_t a = sb + kP_GR + (s >> 2) * 16384 + (s & 3) * 32;
-            mma_bf16(tmem, sdesc_sw128(a, 16, 1024), sdesc_sw128(a, 16, 1024), idesc, s > 0);
+            const uint32_t a = sb + kP_GR + (s >> 2) * kP_GRB + (s & 3) * 32;
+            mma_bf16(tmem, sdesc_sw128(a, 16, 1024), sdesc_sw128(a + 8192, 16, 1024), idesc, s > 0);
         }
         mma_commit(&ss.bar_mma);
     }
@@ -324,9 +398,9 @@ chunk_prep_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __re
                     vr[hh][pass][0] = vr[hh][pass][1] = make_uint4(0, 0, 0, 0);
                 }
             }
-        // gate factors of both heads to the workspace (warps 2-3; token row r)
-        if (warp >= 2) {
-            const int r = tid - 64;
+        // gate factors of both heads to the workspace (warps 0-1; token row r)
+        if (warp < 2) {
+            const int r = tid;
 #pragma unroll
             for (int hh = 0; hh < 2; ++hh) {
                 float* cv = reinterpret_cast<float*>(ws + L.cvec + ((size_t)cid * hv + h0 + hh) * kCvecBytes);
@@ -340,13 +414,14 @@ chunk_prep_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __re
         if (__syncthreads_or(!ok)) { err = 1; goto cleanup; }
         tc_fence_after();
 
-        // ---- 3. decay masks from the Gram rows: A (fp32, smem) from K K^T (warps 0-1),
-        //         P = lower(exp(G_r - G_j) Q K^T) of both heads to the workspace (warps 2-3)
+        // ---- 3. from the Gram rows: P = lower(exp(G_r - G_j) Q K^T) of both heads to the
+        //         workspace (warps 0-1); A (fp32, smem) from K K^T and the bf16 image of
+        //         K K_prev^T (warps 2-3)
         {
             float row[64];
             tmem_ld64(tmem, warp, 0, row);
             const int r = tid & 63;
-            if (warp < 2) {
+            if (warp >= 2) {
 #pragma unroll 1
                 for (int hh = 0; hh < 2; ++hh) {
                     const float Gr = ss.G[hh][r], br = ss.b[hh][r];
@@ -365,6 +440,10 @@ chunk_prep_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __re
                         a4[m] = make_float4(t4[0], t4[1], t4[2], t4[3]);
                     }
                 }
+                tmem_ld64(tmem, warp, 64, row);  // K K_prev^T, row r (MN-major B: K index r)
+#pragma unroll
+                for (int ch = 0; ch < 8; ++ch)
+                    *reinterpret_cast<uint4*>(sm + kP_GX + sw128(r, ch)) = pack8(row + 8 * ch);
             } else {
 #pragma unroll 1
                 for (int hh = 0; hh < 2; ++hh) {
@@ -386,14 +465,16 @@ chunk_prep_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __re
                 }
             }
         }
-        // V images (MN-major: token row, d_v contiguous) into the dead [K; Q] region
+        // V images (MN-major: token row, d_v contiguous; d_v blocks kP_GRB apart) into the
+        // dead Q (head 0) and K_prev (head 1) slots
 #pragma unroll
         for (int hh = 0; hh < 2; ++hh)
 #pragma unroll
             for (int pass = 0; pass < 4; ++pass) {
                 const int rr = pass * 16 + (tid >> 3);
-                *reinterpret_cast<uint4*>(sm + kP_GR + hh * 16384 + kb * 8192 + sw128(rr, c0)) = vr[hh][pass][0];
-                *reinterpret_cast<uint4*>(sm + kP_GR + hh * 16384 + kb * 8192 + sw128(rr, c0 + 1)) = vr[hh][pass][1];
+                unsigned char* vb = sm + kP_GR + hh * 16384 + kb * kP_GRB;
+                *reinterpret_cast<uint4*>(vb + sw128(rr, c0)) = vr[hh][pass][0];
+                *reinterpret_cast<uint4*>(vb + sw128(rr, c0 + 1)) = vr[hh][pass][1];
             }
     }
     fence_async_smem();
@@ -524,9 +605,9 @@ chunk_prep_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __re
 #pragma unroll
         for (int s = 0; s < 4; ++s) {
             mma_bf16(tmem, sdesc_sw128(sb + kP_AF + s * 32, 16, 1024),
-                     sdesc_sw128(sb + kP_KT + s * 2048, 8192, 1024), idesc, s > 0);
+                     sdesc_sw128(sb + kP_GR + 8192 + s * 2048, kP_GRB, 1024), idesc, s > 0);
             mma_bf16(tmem + 128, sdesc_sw128(sb + kP_AF + 16384 + s * 32, 16, 1024),
-                     sdesc_sw128(sb + kP_GR + s * 2048, 8192, 1024), idesc, s > 0);
+                     sdesc_sw128(sb + kP_GR + s * 2048, kP_GRB, 1024), idesc, s > 0);
         }
         mma_commit(&ss.bar_mma);
     }
@@ -534,15 +615,19 @@ chunk_prep_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __re
     if (__syncthreads_or(!ok)) { err = 1; goto cleanup; }
     tc_fence_after();
 
-    // ---- 7. epilogue: accumulator row r' is row r' % 64 of head r' / 64
+    // ---- 7. epilogue: accumulator row r' is row r' % 64 of head r' / 64.  The W image is
+    //         stored pre-scaled by the previous chunk's total decay (W~ = gam_L,prev W).
     {
         const int hh = tid >> 6, r = tid & 63, h = h0 + hh;
         unsigned char* wimg = ws + L.w + ((size_t)cid * hv + h) * kWBytes;
         unsigned char* uimg = ws + L.u + ((size_t)cid * hv + h) * kUBytes;
+        const float gp = ss.gprev[hh];
         float col[64];
 #pragma unroll
         for (int half = 0; half < 2; ++half) {
             tmem_ld64(tmem, warp, 64 * half, col);
+#pragma unroll
+            for (int e = 0; e < 64; ++e) col[e] *= gp;
 #pragma unroll
             for (int ch = 0; ch < 8; ++ch)
                 *reinterpret_cast<uint4*>(wimg + half * 8192 + sw128(r, ch)) = pack8(col + 8 * ch);
@@ -559,12 +644,16 @@ chunk_prep_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __re
         tc_fence_before();
         __syncthreads();
         if (tid == 0) {  // U of head 1: D[:, 128:256] = A_U V_1 (rows 64..127 are head 1's)
-            tc_fence_after();
+            tc_fence_after();  // and M = [T0 D0; T1 D1] (K K_prev^T): D[:, 0:64]
             const uint32_t idesc = idesc_bf16(128, 128, 0, 1);
+            const uint32_t idesc_m = idesc_bf16(128, 64, 0, 1);
 #pragma unroll
-            for (int s = 0; s < 4; ++s)
+            for (int s = 0; s < 4; ++s) {
                 mma_bf16(tmem + 128, sdesc_sw128(sb + kP_AF + 16384 + s * 32, 16, 1024),
-                         sdesc_sw128(sb + kP_GR + 16384 + s * 2048, 8192, 1024), idesc, s > 0);
+                         sdesc_sw128(sb + kP_GR + 16384 + s * 2048, kP_GRB, 1024), idesc, s > 0);
+                mma_bf16(tmem, sdesc_sw128(sb + kP_AF + s * 32, 16, 1024),
+                         sdesc_sw128(sb + kP_GX + s * 2048, 8192, 1024), idesc_m, s > 0);
+            }
             mma_commit(&ss.bar_mma);
         }
         ok = mbar_wait(&ss.bar_mma, 0);
@@ -578,6 +667,19 @@ chunk_prep_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __re
                 for (int ch = 0; ch < 8; ++ch)
                     *reinterpret_cast<uint4*>(uimg + half * 8192 + sw128(r, ch)) = pack8(col + 8 * ch);
             }
+        }
+        {
+            unsigned char* mimg = ws + L.m + ((size_t)cid * hv + h) * kMBytes;
+            tmem_ld64(tmem, warp, 0, col);
+            const float4* cp4 = reinterpret_cast<const float4*>(ss.cprev[hh]);
+#pragma unroll
+            for (int j4 = 0; j4 < 16; ++j4) {
+                const float4 cv4 = cp4[j4];
+                col[4 * j4] *= cv4.x; col[4 * j4 + 1] *= cv4.y; col[4 * j4 + 2] *= cv4.z; col[4 * j4 + 3] *= cv4.w;
+            }
+#pragma unroll
+            for (int ch = 0; ch < 8; ++ch)
+                *reinterpret_cast<uint4*>(mimg + sw128(r, ch)) = pack8(col + 8 * ch);
         }
     }
 
@@ -596,30 +698,60 @@ cleanup:
 }
 
 // ===================================================================== K2
-constexpr int kStateThreads = 320;                  // warps 0-7 compute, warp 8 MMAs, warp 9 bulk copies
-constexpr int kStages = 3;                          // chunk buffers (loads run two chunks ahead)
-constexpr uint32_t kS_A1 = 0;                       // [W; Q] K-major, 2 K-blocks of 128 rows (32 KB)
-constexpr uint32_t kS_KT = 32768;                   // K, MN-major A operand (16 KB)
-constexpr uint32_t kS_U = 49152;                    // U, this CTA's d_v half (8 KB)
-constexpr uint32_t kS_P = 57344;                    // P (8 KB); [U; P] is the A operand of P Delta
-constexpr uint32_t kS_BUF = 65536;                  // one chunk buffer (64 KB)
-constexpr uint32_t kS_B1 = kStages * kS_BUF;        // S slice bf16, MN-major (16 KB)
-constexpr uint32_t kS_B2 = kS_B1 + 16384;           // Delta, MN-major (8 KB)
-constexpr uint32_t kS_B3 = kS_B2 + 8192;            // diag(c) Delta, MN-major (8 KB)
-constexpr uint32_t kS_CV = kS_B3 + 8192;            // gate factors of each stage (3 x 528 B)
+// Look-ahead form of the chunk recurrence.  With S_c the state entering chunk c and
+// X_c = W_c S_c^T, the state update of chunk c-1 gives
+//   X_c = gam_L,c-1 W_c S_{c-1}^T + (W_c K_{c-1}^T diag(c_{c-1})) Delta_{c-1}
+//       = W~_c S_{c-1}^T            + M~_c Delta_{c-1},
+// with W~ and M~ from the prep kernel.  The K = 128 product W~_c S_{c-1}^T (together with
+// Y_{c-1} = Q_{c-1} S_{c-1}^T, as one M = 128 MMA) is issued one chunk ahead; only the
+// K = 64 product M~_c Delta_{c-1} separates Delta_{c-1} from Delta_c, and it shares its
+// B operand with P_{c-1} Delta_{c-1} (the outputs of chunk c-1): [M~_c; P_{c-1}] Delta_{c-1}
+// is one M = 128 MMA.  The state update S_c = gam_L S_{c-1} + (K~_{c-1}^T Delta_{c-1})^T,
+// with K~ = diag(c) K from the prep kernel, reads the same B operand.  At these sizes every
+// tcgen05.mma costs the issuing thread about the same time whatever its N, so the schedule
+// is built around that one thread (16 MMAs per chunk).  In step c it waits for
+// Delta_{c-1}, issues (a) and (b) back to back, and (d) once S_c is written:
+//   (a) SA  = K~_{c-1}^T B2           (B2 = Delta_{c-1}, bf16)             -> state warps
+//   (b) CH  = [M~_c; P_{c-1}] B2      (rows 0..63 -> Delta warps; rows 64..127 -> outputs)
+//   (d) ZY  = [W~_{c+1}; Q_c] B1      (B1 = S_c, written by the state warps after (a))
+// Operand slot k (k = 0 .. nch) holds W~_k, M~_k and Q, P, K~ and the gate factors of chunk
+// k-1; step c reads slots c and c+1.  A slot is released in step k once (b) has completed;
+// the copy warp refills it two steps ahead of use and asks L2 for the slot after that.
+// Completion of (a) in step c+1 implies completion of everything issued before it, so the
+// outputs of chunk c-1 need no barrier of their own.
+//
+// Warps (TMEM lane quarter = warp % 4, 16-column half of the 32 d_v = (warp / 4) % 2):
+//   0, 1, 4, 5     Delta warps: token rows 0..63 of X_c, Delta_c and B2
+//   2, 3, 6, 7     state rows (d_k) 64..127 and the outputs (token rows of Y and PD)
+//   8, 9, 12, 13   state rows (d_k) 0..63
+//   10             MMA issuer;  11  bulk copies
+constexpr int kStateThreads = 448;
+constexpr int kIssuerWarp = 10, kCopyWarp = 11;
+constexpr int kStages = 3;                          // operand slots
+constexpr uint32_t kS_A1 = 0;                       // [W~_k; Q_{k-1}] K-major, 2 d_k blocks of 128 rows (32 KB)
+constexpr uint32_t kS_M = 32768;                    // M~_k (8 KB); [M~; P] is the A operand of (b)
+constexpr uint32_t kS_P = 40960;                    // P_{k-1} (8 KB)
+constexpr uint32_t kS_KT = 49152;                   // K~_{k-1}, MN-major A operand (16 KB)
+constexpr uint32_t kS_BUF = 65536;                  // one slot (64 KB)
+constexpr int kSlices = 4;                          // CTAs per (sequence, V head)
+constexpr int kSliceW = kD / kSlices;               // d_v columns per CTA (the MMAs' N)
+constexpr uint32_t kS_B1 = kStages * kS_BUF;        // S slice bf16, MN-major, 64-byte swizzle (8 KB)
+constexpr uint32_t kS_B2 = kS_B1 + 8192;            // Delta, two buffers (2 x 4 KB)
+constexpr uint32_t kS_CV = kS_B2 + 8192;            // gate factors of each slot (3 x 528 B)
 constexpr uint32_t kS_SMALL = kS_CV + kStages * kCvecLoad;
-constexpr uint32_t kStateSmem = kS_SMALL + 128;     // needs a 1024-aligned dynamic base (checked)
+constexpr uint32_t kStateSmem = kS_SMALL + 256;     // needs a 1024-aligned dynamic base (checked)
+constexpr uint32_t kEmptyArrivals = 257;            // state/output warps and the MMA commit (step k)
 // Tensor Memory columns
-constexpr int kTBufs = 3;        // output accumulators of three consecutive chunks stay live
-constexpr uint32_t kT_XY = 0;     // [X; Y] of chunk c at kT_XY + 64 (c % 3)
-constexpr uint32_t kT_PD = 192;   // P Delta of chunk c at kT_PD + 64 (c % 3) (rows 64..127)
-constexpr uint32_t kT_SA = 384;   // K^T diag(c) Delta
+constexpr uint32_t kT_ZY = 0;     // [Z~_c; Y_{c-1}] at 32 (c % 3)
+constexpr uint32_t kT_CH = 96;    // [M~_c Delta_{c-1}; P_{c-1} Delta_{c-1}] at 96 + 32 (c % 3)
+constexpr uint32_t kT_SA = 192;   // K~^T Delta
+constexpr uint32_t kTmemCols = 256;
 
 struct StateSmall {
-    uint64_t full[kStages];   // stage loaded
-    uint64_t empty[kStages];  // stage consumed: 256 compute-thread arrivals + the MMAs' commit
-    uint64_t mma2[kTBufs];    // P Delta of chunk c done, on mma2[c % 3] (a waiter may lag one chunk)
-    uint64_t b1, b3, b2, mma1, mma3;
+    uint64_t full[kStages];   // slot loaded
+    uint64_t empty[kStages];  // slot consumed (kEmptyArrivals arrivals)
+    uint64_t b2[2];           // Delta_c in B2[c & 1], on b2[c & 1]
+    uint64_t b1, mx, msa, fin, drain;
     uint32_t tmem_base;
     int abort_flag;
 };
@@ -646,28 +778,51 @@ __device__ __forceinline__ void mbar_arrive(uint64_t* bar) {
     asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_u32(bar)) : "memory");
 }
 
-// 32 consecutive TMEM columns of this warp's lane quarter.
-__device__ __forceinline__ void tmem_ld32(uint32_t tmem_base, int warp, uint32_t col, float* v) {
-    const uint32_t a = tmem_base + ((uint32_t)(warp & 3) * 32u << 16) + col;
-    tmem_ld16(a, v);
-    tmem_ld16(a + 16, v + 16);
+// 16 consecutive TMEM columns of this warp's lane quarter.
+__device__ __forceinline__ void tmem_ld16w(uint32_t tmem_base, int warp, uint32_t col, float* v) {
+    tmem_ld16(tmem_base + ((uint32_t)(warp & 3) * 32u << 16) + col, v);
     tmem_ld_wait();
 }
 
-__device__ __forceinline__ void issue_chunk_loads(unsigned char* buf, unsigned char* cv, uint64_t* bar,
-                                                  const unsigned char* ws, const WsLayout& L, int cid, int h,
-                                                  int jq, int half, int hk, int hv) {
-    mbar_arrive_expect_tx(bar, kChunkLoadBytes);
-    const unsigned char* w = ws + L.w + ((size_t)cid * hv + h) * kWBytes;
-    const unsigned char* qn = ws + L.qn + ((size_t)cid * hk + jq) * kQBytes;
-    bulk_g2s(buf + kS_A1, w, 8192, bar);                  // W rows, d_k 0..63
-    bulk_g2s(buf + kS_A1 + 8192, qn, 8192, bar);          // Q rows, d_k 0..63
-    bulk_g2s(buf + kS_A1 + 16384, w + 8192, 8192, bar);   // W rows, d_k 64..127
-    bulk_g2s(buf + kS_A1 + 24576, qn + 8192, 8192, bar);  // Q rows, d_k 64..127
-    bulk_g2s(buf + kS_KT, ws + L.kt + ((size_t)cid * hk + jq) * kKTBytes, kKTBytes, bar);
-    bulk_g2s(buf + kS_U, ws + L.u + ((size_t)cid * hv + h) * kUBytes + half * (kUBytes / 2), kUBytes / 2, bar);
-    bulk_g2s(buf + kS_P, ws + L.p + ((size_t)cid * hv + h) * kPBytes, kPBytes, bar);
-    bulk_g2s(cv, ws + L.cvec + ((size_t)cid * hv + h) * kCvecBytes, kCvecLoad, bar);
+// Operand slot k of a sequence whose chunks are cs .. cs + nch - 1.
+__device__ __forceinline__ void issue_slot_loads(unsigned char* buf, unsigned char* cv, uint64_t* bar,
+                                                 const unsigned char* ws, const WsLayout& L, int cs, int k,
+                                                 int nch, int h, int jq, int hk, int hv) {
+    const bool w_k = k < nch, m_k = k >= 1 && k < nch, prev = k >= 1;
+    uint32_t bytes = 0;
+    if (w_k) bytes += kWBytes;
+    if (m_k) bytes += kMBytes;
+    if (prev) bytes += kQBytes + kPBytes + kKTBytes + kCvecLoad;
+    mbar_arrive_expect_tx(bar, bytes);
+    if (w_k) {
+        const unsigned char* w = ws + L.w + ((size_t)(cs + k) * hv + h) * kWBytes;
+        bulk_g2s(buf + kS_A1, w, 8192, bar);                  // W~ rows, d_k 0..63
+        bulk_g2s(buf + kS_A1 + 16384, w + 8192, 8192, bar);   // W~ rows, d_k 64..127
+    }
+    if (m_k) bulk_g2s(buf + kS_M, ws + L.m + ((size_t)(cs + k) * hv + h) * kMBytes, kMBytes, bar);
+    if (prev) {
+        const int cp = cs + k - 1;
+        const unsigned char* qn = ws + L.qn + ((size_t)cp * hk + jq) * kQBytes;
+        bulk_g2s(buf + kS_A1 + 8192, qn, 8192, bar);          // Q rows, d_k 0..63
+        bulk_g2s(buf + kS_A1 + 24576, qn + 8192, 8192, bar);  // Q rows, d_k 64..127
+        bulk_g2s(buf + kS_P, ws + L.p + ((size_t)cp * hv + h) * kPBytes, kPBytes, bar);
+        bulk_g2s(buf + kS_KT, ws + L.kt + ((size_t)cp * hv + h) * kKTBytes, kKTBytes, bar);
+        bulk_g2s(cv, ws + L.cvec + ((size_t)cp * hv + h) * kCvecBytes, kCvecLoad, bar);
+    }
+}
+
+// The same bytes as issue_slot_loads, into L2 only.
+__device__ __forceinline__ void prefetch_slot(const unsigned char* ws, const WsLayout& L, int cs, int k, int nch,
+                                              int h, int jq, int hk, int hv) {
+    if (k < nch) bulk_prefetch_l2(ws + L.w + ((size_t)(cs + k) * hv + h) * kWBytes, kWBytes);
+    if (k >= 1 && k < nch) bulk_prefetch_l2(ws + L.m + ((size_t)(cs + k) * hv + h) * kMBytes, kMBytes);
+    if (k >= 1) {
+        const int cp = cs + k - 1;
+        bulk_prefetch_l2(ws + L.qn + ((size_t)cp * hk + jq) * kQBytes, kQBytes);
+        bulk_prefetch_l2(ws + L.p + ((size_t)cp * hv + h) * kPBytes, kPBytes);
+        bulk_prefetch_l2(ws + L.kt + ((size_t)cp * hv + h) * kKTBytes, kKTBytes);
+        bulk_prefetch_l2(ws + L.cvec + ((size_t)cp * hv + h) * kCvecBytes, kCvecLoad);
+    }
 }
 
 __global__ void __launch_bounds__(kStateThreads, 1)
@@ -680,9 +835,9 @@ chunk_state_kernel(const float* s0, const int32_t* __restrict__ cu, __nv_bfloat1
 
     const WsLayout L = ws_layout(num_seqs, total_tokens, hk, hv);
     int32_t* header = reinterpret_cast<int32_t*>(ws);
-    const int half = blockIdx.x & 1;
-    const int h = (blockIdx.x >> 1) % hv;
-    const int n = (blockIdx.x >> 1) / hv;
+    const int slice = blockIdx.x % kSlices;
+    const int h = (blockIdx.x / kSlices) % hv;
+    const int n = (blockIdx.x / kSlices) / hv;
     const int jq = h / (hv / hk);
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int32_t* seq_chunk0 = reinterpret_cast<const int32_t*>(ws + L.seq_chunk0);
@@ -694,20 +849,20 @@ chunk_state_kernel(const float* s0, const int32_t* __restrict__ cu, __nv_bfloat1
     }
 
     if (warp == 0) {
-        tmem_alloc(&ss.tmem_base, 512);
+        tmem_alloc(&ss.tmem_base, kTmemCols);
         tmem_relinquish();
     }
     if (tid == 0) {
         for (int s = 0; s < kStages; ++s) {
             mbar_init(&ss.full[s], 1);
-            mbar_init(&ss.empty[s], 257);
+            mbar_init(&ss.empty[s], kEmptyArrivals);
         }
+        for (int s = 0; s < 2; ++s) mbar_init(&ss.b2[s], 128);
         mbar_init(&ss.b1, 256);
-        mbar_init(&ss.b3, 128);
-        mbar_init(&ss.b2, 128);
-        mbar_init(&ss.mma1, 1);
-        for (int s = 0; s < kTBufs; ++s) mbar_init(&ss.mma2[s], 1);
-        mbar_init(&ss.mma3, 1);
+        mbar_init(&ss.mx, 1);
+        mbar_init(&ss.msa, 1);
+        mbar_init(&ss.fin, 1);
+        mbar_init(&ss.drain, 1);
         ss.abort_flag = 0;
         fence_mbar_init();
     }
@@ -716,60 +871,75 @@ chunk_state_kernel(const float* s0, const int32_t* __restrict__ cu, __nv_bfloat1
     tc_fence_after();
     const uint32_t tmem = ss.tmem_base;
 
-    if (warp == 8) {
+    if (warp == kIssuerWarp) {
         // ------------------------------------------------ MMA issuer
-        if (lane == 0) {
-            const uint32_t id_xy = idesc_bf16(128, 64, 0, 1);  // A K-major, B MN-major
-            const uint32_t id_s = idesc_bf16(128, 64, 1, 1);   // A MN-major, B MN-major
-            const uint64_t d_b1 = sdesc_sw128(sb + kS_B1, 16384, 1024);
-            const uint64_t d_b2 = sdesc_sw128(sb + kS_B2, 8192, 1024);
-            const uint64_t d_b3 = sdesc_sw128(sb + kS_B3, 8192, 1024);
-            int c = 0;
-            for (; c < nch; ++c) {
-                const int b = c % kStages, par = c & 1, tb = c % kTBufs;
-                const uint32_t bufa = sb + b * kS_BUF;
-                const uint64_t d_a1 = sdesc_sw128(bufa + kS_A1, 16, 1024);
-                const uint64_t d_kt = sdesc_sw128(bufa + kS_KT, 8192, 1024);
-                const uint64_t d_up = sdesc_sw128(bufa + kS_U, 16, 1024);  // rows 0..63 U (unused), 64..127 P
-                // the operands normally land long before the state does: check them first
-                if (!wait_or_abort(&ss.full[b], (c / kStages) & 1, abort_flag, header)) break;
-                if (!wait_or_abort(&ss.b1, par, abort_flag, header)) break;   // S(c) in B1
-                tc_fence_after();
+        if (lane == 0 && nch > 0) {
+            const uint32_t id_xy = idesc_bf16(128, kSliceW, 0, 1);  // A K-major, B MN-major
+            const uint32_t id_s = idesc_bf16(128, kSliceW, 1, 1);   // A MN-major, B MN-major
+            // B operands: one 32-wide atom along N (the N-block stride is never used), 8-K-row
+            // groups of 512 bytes
+            const uint64_t d_b1 = sdesc_sw64(sb + kS_B1, 512, 512);
+            auto issue_zy = [&](int k) {  // [W~_k; Q_{k-1}] S^T -> ZY buffer k % 3
+                const uint64_t d_a1 = sdesc_sw128(sb + (k % kStages) * kS_BUF + kS_A1, 16, 1024);
 #pragma unroll
                 for (int s = 0; s < 8; ++s)  // descriptor start addresses advance in 16-byte units
-                    mma_bf16(tmem + kT_XY + 64 * tb, d_a1 + (((s >> 2) * 16384 + (s & 3) * 32) >> 4),
-                             d_b1 + ((s * 2048) >> 4), id_xy, s > 0);
-                mma_commit(&ss.mma1);
-                if (!wait_or_abort(&ss.b3, par, abort_flag, header)) break;   // diag(c) Delta(c) written
+                    mma_bf16(tmem + kT_ZY + kSliceW * (k % 3), d_a1 + (((s >> 2) * 16384 + (s & 3) * 32) >> 4),
+                             d_b1 + ((s * 1024) >> 4), id_xy, s > 0);
+            };
+            int c = -1;
+            bool ok = wait_or_abort(&ss.full[0], 0, abort_flag, header) &&
+                      wait_or_abort(&ss.b1, 0, abort_flag, header);
+            if (ok) {  // X_0 = W_0 S_0^T
                 tc_fence_after();
+                issue_zy(0);
+                mma_commit(&ss.mx);
+                for (c = 0; c <= nch; ++c) {
+                    const int sc = c % kStages, sn = (c + 1) % kStages;
+                    const uint32_t bufc = sb + sc * kS_BUF;
+                    if (c >= 1) {
+                        const int pb = (c - 1) & 1;
+                        if (!wait_or_abort(&ss.b2[pb], ((c - 1) >> 1) & 1, abort_flag, header)) break;
+                        tc_fence_after();
+                        const uint64_t d_b2 = sdesc_sw64(sb + kS_B2 + 4096 * pb, 512, 512);
+                        const uint64_t d_kt = sdesc_sw128(bufc + kS_KT, 8192, 1024);
 #pragma unroll
-                for (int s = 0; s < 4; ++s)
-                    mma_bf16(tmem + kT_SA, d_kt + ((s * 2048) >> 4), d_b3 + ((s * 2048) >> 4), id_s, s > 0);
-                mma_commit(&ss.mma3);
-                if (!wait_or_abort(&ss.b2, par, abort_flag, header)) break;   // Delta(c) written
-                tc_fence_after();
+                        for (int s = 0; s < 4; ++s)  // (a)
+                            mma_bf16(tmem + kT_SA, d_kt + ((s * 2048) >> 4), d_b2 + ((s * 1024) >> 4), id_s, s > 0);
+                        mma_commit(&ss.msa);
+                        const uint64_t d_mp = sdesc_sw128(bufc + kS_M, 16, 1024);
 #pragma unroll
-                for (int s = 0; s < 4; ++s)
-                    mma_bf16(tmem + kT_PD + 64 * tb, d_up + ((s * 32) >> 4), d_b2 + ((s * 2048) >> 4), id_xy, s > 0);
-                mma_commit(&ss.mma2[tb]);
-                mma_commit(&ss.empty[b]);  // every MMA reading stage b has completed
+                        for (int s = 0; s < 4; ++s)  // (b)
+                            mma_bf16(tmem + kT_CH + kSliceW * (c % 3), d_mp + ((s * 32) >> 4), d_b2 + ((s * 1024) >> 4),
+                                     id_xy, s > 0);
+                        mma_commit(&ss.mx);
+                    }
+                    mma_commit(&ss.empty[sc]);  // every MMA reading slot c has been issued
+                    if (c < nch) {  // (d)
+                        if (!wait_or_abort(&ss.full[sn], ((c + 1) / kStages) & 1, abort_flag, header)) break;
+                        if (!wait_or_abort(&ss.b1, c & 1, abort_flag, header)) break;
+                        tc_fence_after();
+                        issue_zy(c + 1);
+                    }
+                }
+                if (c == nch + 1) mma_commit(&ss.fin);  // P Delta of the last chunk
             }
             if (*abort_flag) {  // drain: every MMA issued so far completes before TMEM is freed
-                mma_commit(&ss.mma1);
-                mbar_wait(&ss.mma1, c & 1);
+                mma_commit(&ss.drain);
+                mbar_wait(&ss.drain, 0);
             }
         }
-    } else if (warp == 9) {
-        // ------------------------------------------------ bulk copies, two chunks ahead
-        if (lane == 0) {
+    } else if (warp == kCopyWarp) {
+        // ------------------------------------------------ bulk copies, two slots ahead
+        if (lane == 0 && nch > 0) {
             int issued = 0;
-            for (; issued < nch; ++issued) {
+            for (; issued <= nch; ++issued) {
                 const int st = issued % kStages;
                 if (issued >= kStages &&
                     !wait_or_abort(&ss.empty[st], ((issued / kStages) - 1) & 1, abort_flag, header))
                     break;
-                issue_chunk_loads(sm + st * kS_BUF, sm + kS_CV + st * kCvecLoad, &ss.full[st], ws, L,
-                                  cs + issued, h, jq, half, hk, hv);
+                issue_slot_loads(sm + st * kS_BUF, sm + kS_CV + st * kCvecLoad, &ss.full[st], ws, L, cs, issued,
+                                 nch, h, jq, hk, hv);
+                if (issued + kStages <= nch) prefetch_slot(ws, L, cs, issued + kStages, nch, h, jq, hk, hv);
             }
             if (*abort_flag) {  // drain: copies in flight land before the CTA exits
                 for (int j = max(0, issued - kStages); j < issued; ++j)
@@ -777,130 +947,130 @@ chunk_state_kernel(const float* s0, const int32_t* __restrict__ cu, __nv_bfloat1
             }
         }
     } else {
-        // ------------------------------------------------ compute warps 0-7
-        // warp w: TMEM lane quarter q4 = w & 3, column half ch2 = w >> 2 of this CTA's 64 d_v
-        const int q4 = warp & 3, ch2 = warp >> 2;
-        const int t = q4 * 32 + lane;       // d_k row of S^T this thread owns (state update)
-        const int r = (q4 & 1) * 32 + lane; // token row (Delta: quarters 0-1; outputs: quarters 2-3)
-        const bool delta_warp = q4 < 2;
-        // fp32 state: S[half*64 + 32*ch2 + m][t], m = 0..31
-        float S[32];
-        const size_t sbase = ((size_t)n * hv + h) * kD * kD + (size_t)(half * 64 + 32 * ch2) * kD + t;
+        const int q4 = warp & 3, ch2 = (warp >> 2) & 1;
+        const int dv0 = slice * kSliceW + 16 * ch2;  // first d_v column of this thread
+        const int r = (q4 & 1) * 32 + lane;         // token row (Delta warps; output warps)
+        const bool delta_warp = warp < 8 && q4 < 2;
+        const bool out_warp = warp < 8 && q4 >= 2;
+        if (delta_warp) {
+            // ------------------------------------------------ Delta warps
+            // U rows of a chunk straight from the workspace (U image: [d_v half][64 rows][128 B])
+            auto load_u = [&](int cidx, uint4* u) {
+                const unsigned char* ub =
+                    ws + L.u + ((size_t)(cs + cidx) * hv + h) * kUBytes + (dv0 >> 6) * (kUBytes / 2);
 #pragma unroll
-        for (int m = 0; m < 32; ++m) S[m] = s0 ? s0[sbase + (size_t)m * kD] : 0.f;
-#pragma unroll
-        for (int cc = 0; cc < 4; ++cc)
-            *reinterpret_cast<uint4*>(sm + kS_B1 + sw128(t, 4 * ch2 + cc)) = pack8(S + 8 * cc);
-        fence_async_smem();
-        tc_fence_before();
-        mbar_arrive(&ss.b1);
-
-        // Outputs of chunk c are written one chunk later (after the state update of c+1), so
-        // that their global stores are not still in flight at the next shared-memory proxy
-        // fence on the state chain.  Three TMEM accumulator sets keep chunk c's [X; Y] and
-        // P Delta alive until then.
-        float prev_gam = 0.f;
-        auto write_outputs = [&](int cp, float gam_r) {
-            const int tb = cp % kTBufs;
-            if (!wait_or_abort(&ss.mma2[tb], (cp / kTBufs) & 1, abort_flag, header)) return false;
-            tc_fence_after();
-            const int t0 = t_begin + cp * kChunk;
-            const int len = min(kChunk, t_end - t0);
-            float y[32], pd[32];
-            tmem_ld32(tmem, warp, kT_XY + 64 * tb + 32 * ch2, y);
-            tmem_ld32(tmem, warp, kT_PD + 64 * tb + 32 * ch2, pd);
-            if (r < len) {
-                uint4* op = reinterpret_cast<uint4*>(out + ((size_t)(t0 + r) * hv + h) * kD + half * 64 + 32 * ch2);
-#pragma unroll
-                for (int cc = 0; cc < 4; ++cc) {
-                    float o8[8];
-#pragma unroll
-                    for (int e = 0; e < 8; ++e) o8[e] = fmaf(gam_r, y[8 * cc + e], pd[8 * cc + e]);
-                    op[cc] = pack8(o8);
-                }
-            }
-            tc_fence_before();
-            return true;
-        };
-        int c = 0;
-        for (; c < nch; ++c) {
-            const int b = c % kStages, par = c & 1, tb = c % kTBufs;
-            unsigned char* buf = sm + b * kS_BUF;
-            if (!wait_or_abort(&ss.full[b], (c / kStages) & 1, abort_flag, header)) break;
-            const float* cvec = reinterpret_cast<const float*>(sm + kS_CV + b * kCvecLoad);
-            const float gl = cvec[128];
-            const float crow = delta_warp ? cvec[r] : cvec[64 + r];  // c_r, or gam_r for outputs
-            uint4 u4[4];  // this row's U values (Delta warps)
-            if (delta_warp) {
-#pragma unroll
-                for (int cc = 0; cc < 4; ++cc) u4[cc] = *reinterpret_cast<const uint4*>(buf + kS_U + sw128(r, 4 * ch2 + cc));
-            }
-            mbar_arrive(&ss.empty[b]);  // this thread's reads of stage b are done (values in registers)
-
-            if (delta_warp) {  // Delta = U - X for token row r, columns 32*ch2 .. +32
-                if (c >= 1 && !wait_or_abort(&ss.mma2[(c - 1) % kTBufs], ((c - 1) / kTBufs) & 1, abort_flag, header))
-                    break;  // B2 and B3 are free once P Delta of c-1 is done
-                if (!wait_or_abort(&ss.mma1, par, abort_flag, header)) break;
+                for (int cc = 0; cc < 2; ++cc)
+                    u[cc] = *reinterpret_cast<const uint4*>(ub + sw128(r, (dv0 & 63) / 8 + cc));
+            };
+            uint4 u_next[2] = {make_uint4(0, 0, 0, 0), make_uint4(0, 0, 0, 0)};
+            if (nch > 0) load_u(0, u_next);
+            for (int c = 0; c < nch; ++c) {
+                // Delta_c = U_c - X_c,  X_c = Z~_c + M~_c Delta_{c-1}  (token row r)
+                uint4 u4[2] = {u_next[0], u_next[1]};
+                if (c + 1 < nch) load_u(c + 1, u_next);
+                if (!wait_or_abort(&ss.mx, c & 1, abort_flag, header)) break;
                 tc_fence_after();
-                float x[32];
-                tmem_ld32(tmem, warp, kT_XY + 64 * tb + 32 * ch2, x);
-                float d[32];
+                float x[16];
+                tmem_ld16w(tmem, warp, kT_ZY + kSliceW * (c % 3) + 16 * ch2, x);
+                if (c >= 1) {
+                    float xc[16];
+                    tmem_ld16w(tmem, warp, kT_CH + kSliceW * (c % 3) + 16 * ch2, xc);
 #pragma unroll
-                for (int cc = 0; cc < 4; ++cc) {
+                    for (int e = 0; e < 16; ++e) x[e] += xc[e];
+                }
+                float d[16];
+#pragma unroll
+                for (int cc = 0; cc < 2; ++cc) {
                     float u8[8];
                     unpack8(u4[cc], u8);
 #pragma unroll
                     for (int e = 0; e < 8; ++e) d[8 * cc + e] = u8[e] - x[8 * cc + e];
                 }
-                // diag(c) Delta first: it feeds the state update, the next link of the chain
 #pragma unroll
-                for (int cc = 0; cc < 4; ++cc) {
-                    float c8[8];
-#pragma unroll
-                    for (int e = 0; e < 8; ++e) c8[e] = d[8 * cc + e] * crow;
-                    *reinterpret_cast<uint4*>(sm + kS_B3 + sw128(r, 4 * ch2 + cc)) = pack8(c8);
-                }
+                for (int cc = 0; cc < 2; ++cc)
+                    *reinterpret_cast<uint4*>(sm + kS_B2 + 4096 * (c & 1) + sw64(r, 2 * ch2 + cc)) = pack8(d + 8 * cc);
                 fence_async_smem();
                 tc_fence_before();
-                mbar_arrive(&ss.b3);
+                mbar_arrive(&ss.b2[c & 1]);
+            }
+        } else {
+            // ------------------------------------------------ state warps (and outputs)
+            const int t = q4 * 32 + lane;  // d_k row of S^T this thread owns
+            // fp32 state: S[dv0 + m][t], m = 0..15
+            float S[16];
+            const size_t sbase = ((size_t)n * hv + h) * kD * kD + (size_t)dv0 * kD + t;
 #pragma unroll
-                for (int cc = 0; cc < 4; ++cc)
-                    *reinterpret_cast<uint4*>(sm + kS_B2 + sw128(r, 4 * ch2 + cc)) = pack8(d + 8 * cc);
+            for (int m = 0; m < 16; ++m) S[m] = s0 ? s0[sbase + (size_t)m * kD] : 0.f;
+            auto write_b1 = [&]() {
+#pragma unroll
+                for (int cc = 0; cc < 2; ++cc)
+                    *reinterpret_cast<uint4*>(sm + kS_B1 + sw64(t, 2 * ch2 + cc)) = pack8(S + 8 * cc);
                 fence_async_smem();
-                mbar_arrive(&ss.b2);
-            }
-            // state update S^T <- gam_L S^T + K^T diag(c) Delta (d_k row t, 32 d_v columns)
-            if (!wait_or_abort(&ss.mma3, par, abort_flag, header)) break;
-            tc_fence_after();
-            {
-                float acc[32];
-                tmem_ld32(tmem, warp, kT_SA + 32 * ch2, acc);
-#pragma unroll
-                for (int m = 0; m < 32; ++m) S[m] = fmaf(gl, S[m], acc[m]);
-#pragma unroll
-                for (int cc = 0; cc < 4; ++cc)
-                    *reinterpret_cast<uint4*>(sm + kS_B1 + sw128(t, 4 * ch2 + cc)) = pack8(S + 8 * cc);
-            }
-            fence_async_smem();
-            tc_fence_before();
-            mbar_arrive(&ss.b1);
+                tc_fence_before();
+                mbar_arrive(&ss.b1);
+            };
+            write_b1();  // S_0: phase 0 of b1
+            if (nch > 0) mbar_arrive(&ss.empty[0]);  // slot 0 has no gate factors to read
 
-            if (!delta_warp) {  // outputs of the previous chunk: O = gam_r Y + P Delta
-                if (c >= 1 && !write_outputs(c - 1, prev_gam)) break;
-                prev_gam = crow;
-            }
-        }
-        if (!delta_warp && c == nch && nch > 0 && !*abort_flag) write_outputs(nch - 1, prev_gam);
-        if (!*abort_flag && sT) {
+            // O_c = gam_r Y_c + P_c Delta_c, with Y_c in the ZY buffer of c+1 and P_c Delta_c in
+            // the CH buffer of c+1 (rows 64..127).  Written in step c+2, after the state update
+            // (whose wait on (a) of step c+2 covers (b) of step c+1), so that the global stores
+            // are not still in flight at the next proxy fence.
+            float prev_gam = 0.f;  // gam_r of the chunk whose outputs are written next
+            auto write_outputs = [&](int cpo, float gam_r) {
+                const int t0 = t_begin + cpo * kChunk;
+                const int len = min(kChunk, t_end - t0);
+                float y[16], pd[16];
+                tmem_ld16w(tmem, warp, kT_ZY + kSliceW * ((cpo + 1) % 3) + 16 * ch2, y);
+                tmem_ld16w(tmem, warp, kT_CH + kSliceW * ((cpo + 1) % 3) + 16 * ch2, pd);
+                if (r < len) {
+                    uint4* op = reinterpret_cast<uint4*>(out + ((size_t)(t0 + r) * hv + h) * kD + dv0);
 #pragma unroll
-            for (int m = 0; m < 32; ++m) sT[sbase + (size_t)m * kD] = S[m];
+                    for (int cc = 0; cc < 2; ++cc) {
+                        float o8[8];
+#pragma unroll
+                        for (int e = 0; e < 8; ++e) o8[e] = fmaf(gam_r, y[8 * cc + e], pd[8 * cc + e]);
+                        op[cc] = pack8(o8);
+                    }
+                }
+                tc_fence_before();
+            };
+            int c = 1;
+            for (; c <= nch; ++c) {
+                // S_c = gam_L S_{c-1} + SA  (gate factors of chunk c-1 are in slot c)
+                const int sc = c % kStages;
+                if (!wait_or_abort(&ss.full[sc], (c / kStages) & 1, abort_flag, header)) break;
+                const float* cvp = reinterpret_cast<const float*>(sm + kS_CV + sc * kCvecLoad);
+                const float gl = cvp[128];
+                const float gr = cvp[64 + r];
+                mbar_arrive(&ss.empty[sc]);
+                if (!wait_or_abort(&ss.msa, (c - 1) & 1, abort_flag, header)) break;
+                tc_fence_after();
+                float acc[16];
+                tmem_ld16w(tmem, warp, kT_SA + 16 * ch2, acc);
+#pragma unroll
+                for (int m = 0; m < 16; ++m) S[m] = fmaf(gl, S[m], acc[m]);
+                if (c < nch) write_b1();
+                if (out_warp) {
+                    if (c >= 2) write_outputs(c - 2, prev_gam);
+                    prev_gam = gr;
+                }
+            }
+            if (out_warp && nch > 0 && c == nch + 1 && wait_or_abort(&ss.fin, 0, abort_flag, header)) {
+                tc_fence_after();
+                write_outputs(nch - 1, prev_gam);
+            }
+            if (!*abort_flag && sT) {
+#pragma unroll
+                for (int m = 0; m < 16; ++m) sT[sbase + (size_t)m * kD] = S[m];
+            }
         }
     }
     tc_fence_before();
     __syncthreads();
     if (warp == 0) {
         tc_fence_after();
-        tmem_dealloc(tmem, 512);
+        tmem_dealloc(tmem, kTmemCols);
     }
 }
 
@@ -936,7 +1106,7 @@ cudaError_t launch_prefill_tc_state(const float* s0, const int32_t* cu, void* ou
     cudaError_t e = cudaFuncSetAttribute(chunk_state_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          (int)kStateSmem);
     if (e != cudaSuccess) return e;
-    chunk_state_kernel<<<(unsigned)num_seqs * hv * 2, kStateThreads, kStateSmem, stream>>>(
+    chunk_state_kernel<<<(unsigned)num_seqs * hv * kSlices, kStateThreads, kStateSmem, stream>>>(
         s0, cu, (__nv_bfloat16*)out, sT, static_cast<unsigned char*>(workspace), num_seqs,
         total_tokens, hk, hv);
     return cudaGetLastError();

@@ -91,11 +91,26 @@ __device__ __forceinline__ void bulk_s2g(void* dst_gmem, const void* src_smem, u
                  "r"(smem_u32(src_smem)), "r"(bytes)
                  : "memory");
 }
+// Asks for `bytes` (a multiple of 16) at a 16-byte-aligned global address to be brought
+// into L2; nothing waits for it.
+__device__ __forceinline__ void bulk_prefetch_l2(const void* src_gmem, uint32_t bytes) {
+    asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(src_gmem), "r"(bytes) : "memory");
+}
 __device__ __forceinline__ void bulk_commit() { asm volatile("cp.async.bulk.commit_group;" ::: "memory"); }
 __device__ __forceinline__ void bulk_wait_all() { asm volatile("cp.async.bulk.wait_group 0;" ::: "memory"); }
 __device__ __forceinline__ void bulk_wait_read_all() {
     asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory");
 }
+
+// ------------------------------------------------------------------ 16-byte async copies
+// (cp.async, global -> shared, bypassing L1; completion is waited for with cp_async_wait_all,
+// which is not a spin loop.)
+__device__ __forceinline__ void cp_async16(void* dst_smem, const void* src_gmem) {
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(smem_u32(dst_smem)), "l"(src_gmem)
+                 : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+__device__ __forceinline__ void cp_async_wait_all() { asm volatile("cp.async.wait_group 0;" ::: "memory"); }
 
 // ------------------------------------------------------------------ Tensor Memory
 // Allocation is warp-collective; the TMEM address is written to shared memory.
@@ -187,10 +202,27 @@ __device__ __forceinline__ uint64_t sdesc_sw128(uint32_t saddr, uint32_t lbo, ui
     return d;
 }
 
+// Same for the 64-byte-swizzled canonical layout (MN-major here: rows of 64 bytes, 32 bf16
+// along M/N, per K index; 8-K-row groups `sbo` apart, 32-wide M/N blocks `lbo` apart).
+// Atoms (8 rows, 512 bytes) must start on 512-byte boundaries.
+__device__ __forceinline__ uint64_t sdesc_sw64(uint32_t saddr, uint32_t lbo, uint32_t sbo) {
+    uint64_t d = 0;
+    d |= (uint64_t)((saddr >> 4) & 0x3FFFu);
+    d |= (uint64_t)((lbo >> 4) & 0x3FFFu) << 16;
+    d |= (uint64_t)((sbo >> 4) & 0x3FFFu) << 32;
+    d |= (uint64_t)1 << 46;  // descriptor version for sm_100
+    d |= (uint64_t)4 << 61;  // layout: 64-byte swizzle
+    return d;
+}
+
 // Byte offset of the 16-byte chunk `chunk` (0..7) of row `row` inside a 128-byte
 // swizzled row group: rows are 128 bytes apart, chunk positions XOR the row's low bits.
 __host__ __device__ constexpr uint32_t sw128(uint32_t row, uint32_t chunk) {
     return row * 128u + ((chunk ^ (row & 7u)) << 4);
+}
+// 64-byte swizzle: chunk (0..3) of a 64-byte row; address bits 4-5 XOR bits 7-8.
+__host__ __device__ constexpr uint32_t sw64(uint32_t row, uint32_t chunk) {
+    return row * 64u + ((chunk ^ ((row >> 1) & 3u)) << 4);
 }
 
 }  // namespace sm100
