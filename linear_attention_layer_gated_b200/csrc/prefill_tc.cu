@@ -203,8 +203,7 @@ constexpr uint32_t kP_GR = 0;
 constexpr uint32_t kP_GRB = 24576;
 constexpr uint32_t kP_GX = 2 * kP_GRB;
 constexpr uint32_t kP_AF = kP_GX + 8192;
-constexpr uint32_t kP_XS = kP_AF + 2 * kAfHead * 4;  // block-solve scratch, 2 heads x 768 floats (6 KB)
-constexpr uint32_t kP_SMALL = kP_XS + 2 * 768 * 4;   // gates, barrier, TMEM address
+constexpr uint32_t kP_SMALL = kP_AF + 2 * kAfHead * 4;  // gates, barrier, TMEM address
 constexpr uint32_t kPrepSmem = kP_SMALL + 3072 + 1024;  // small struct + alignment slack
 
 struct PrepSmall {
@@ -228,7 +227,6 @@ chunk_prep_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __re
     const uint32_t sb = smem_u32(sm);
     PrepSmall& ss = *reinterpret_cast<PrepSmall*>(sm + kP_SMALL);
     float* af = reinterpret_cast<float*>(sm + kP_AF);   // [head][64][kLdA]
-    float* xs = reinterpret_cast<float*>(sm + kP_XS);   // [head][768]
 
     const WsLayout L = ws_layout(num_seqs, total_tokens, hk, hv);
     int32_t* header = reinterpret_cast<int32_t*>(ws);
@@ -481,89 +479,81 @@ chunk_prep_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __re
     tc_fence_before();
     __syncthreads();
 
-    // ---- 4. T = (I + A)^-1 per head, by 16x16 blocks, in place.  Each head uses 64 threads.
-    //         (a) diagonal blocks: D_b = (I + A_bb)^-1 by forward substitution, one column
-    //             per thread; (b) below the diagonal, block row by block row,
-    //             T_ij = -D_i (sum_{k=j}^{i-1} A_ik T_kj), as dense 16x16 products.
+    // ---- 4. T = (I + A)^-1 per head, by 32x32 blocks, in place; 64 threads per head.
+    //         With A = [A11 0; A21 A22]:  T = [T1 0; T21 T2], T1 = (I + A11)^-1,
+    //         T2 = (I + A22)^-1, T21 = -T2 (A21 T1).
+    //         (a) T1 and T2 by forward substitution: warp (head, block), lane = column j;
+    //             every lane reads the same A row (a shared-memory broadcast);
+    //         (b) Y = A21 T1 into the (zero) upper-right block, then T21 = -T2 Y, each thread
+    //             a 4x4 tile; the upper-right block is cleared again afterwards.
     {
         const int hh = tid >> 6, l = tid & 63;
         float* A = af + hh * kAfHead;
-        float* X = xs + hh * 768;
         {
-            const int base = 16 * (l >> 4), j = l & 15;
-            float x[16];
+            const int base = 32 * (l >> 5), j = l & 31;
+            float x[32];
 #pragma unroll
-            for (int r = 0; r < 16; ++r) {
-                const float* arow = A + (base + r) * kLdA + base;
+            for (int r = 0; r < 32; ++r) {
+                const float4* arow = reinterpret_cast<const float4*>(A + (base + r) * kLdA + base);
                 float acc = 0.f;
 #pragma unroll
-                for (int k = 0; k < r; ++k) acc = fmaf(arow[k], x[k], acc);
+                for (int k4 = 0; k4 < (r + 3) / 4; ++k4) {
+                    const float4 a = arow[k4];
+                    const float av[4] = {a.x, a.y, a.z, a.w};
+#pragma unroll
+                    for (int e = 0; e < 4; ++e)
+                        if (4 * k4 + e < r) acc = fmaf(av[e], x[4 * k4 + e], acc);
+                }
                 x[r] = (r == j) ? 1.f : ((r < j) ? 0.f : -acc);
             }
-            __syncthreads();
+            __syncwarp();  // every lane of this block's warp is done reading A_bb
 #pragma unroll
-            for (int r = 0; r < 16; ++r) A[(base + r) * kLdA + base + j] = x[r];
+            for (int r = 0; r < 32; ++r) A[(base + r) * kLdA + base + j] = x[r];
         }
         __syncthreads();
-        // Output mapping inside a 16x16 block: column cc = l & 15, rows rr0 + 4 q for q = 0..3.
-        const int cc = l & 15, rr0 = l >> 4;
-        // Block rows i = 1, 2, 3 in order.  Row i reads only its own A blocks (still intact)
-        // and blocks of rows < i (already T); it is overwritten only after all its X_ij are formed.
-        // The block loops stay rolled (small code); each 16-term dot product is unrolled.
-#pragma unroll 1
-        for (int i = 1; i < 4; ++i) {
-            const float* arow[4];
+        const int tr = l >> 3, tc = l & 7;  // 4x4 output tile: rows 4 tr .., columns 4 tc ..
+        float acc[4][4];
+        auto tile_product = [&](const float* Lm, const float* Rm) {  // acc = Lm (32x32) Rm (32x32)
 #pragma unroll
-            for (int q = 0; q < 4; ++q) arow[q] = A + (16 * i + rr0 + 4 * q) * kLdA;
-#pragma unroll 1
-            for (int j = 0; j < i; ++j) {              // X_ij = sum_{k=j}^{i-1} A_ik T_kj
-                float acc[4] = {0.f, 0.f, 0.f, 0.f};
-#pragma unroll 1
-                for (int k = j; k < i; ++k) {
-                    const float* tc = A + (16 * k) * kLdA + 16 * j + cc;
-                    float tcol[16];
+            for (int i = 0; i < 4; ++i)
 #pragma unroll
-                    for (int m = 0; m < 16; ++m) tcol[m] = tc[m * kLdA];
+                for (int m = 0; m < 4; ++m) acc[i][m] = 0.f;
+#pragma unroll 2
+            for (int k4 = 0; k4 < 8; ++k4) {
+                float4 a[4], b[4];
 #pragma unroll
-                    for (int q = 0; q < 4; ++q) {
-                        const float4* ar = reinterpret_cast<const float4*>(arow[q] + 16 * k);
+                for (int i = 0; i < 4; ++i) a[i] = *reinterpret_cast<const float4*>(Lm + (4 * tr + i) * kLdA + 4 * k4);
 #pragma unroll
-                        for (int m4 = 0; m4 < 4; ++m4) {
-                            const float4 a = ar[m4];
-                            acc[q] = fmaf(a.x, tcol[4 * m4 + 0], acc[q]);
-                            acc[q] = fmaf(a.y, tcol[4 * m4 + 1], acc[q]);
-                            acc[q] = fmaf(a.z, tcol[4 * m4 + 2], acc[q]);
-                            acc[q] = fmaf(a.w, tcol[4 * m4 + 3], acc[q]);
-                        }
+                for (int e = 0; e < 4; ++e) b[e] = *reinterpret_cast<const float4*>(Rm + (4 * k4 + e) * kLdA + 4 * tc);
+#pragma unroll
+                for (int i = 0; i < 4; ++i) {
+                    const float av[4] = {a[i].x, a[i].y, a[i].z, a[i].w};
+#pragma unroll
+                    for (int e = 0; e < 4; ++e) {
+                        acc[i][0] = fmaf(av[e], b[e].x, acc[i][0]);
+                        acc[i][1] = fmaf(av[e], b[e].y, acc[i][1]);
+                        acc[i][2] = fmaf(av[e], b[e].z, acc[i][2]);
+                        acc[i][3] = fmaf(av[e], b[e].w, acc[i][3]);
                     }
                 }
-#pragma unroll
-                for (int q = 0; q < 4; ++q) X[j * 256 + (rr0 + 4 * q) * 16 + cc] = acc[q];
             }
-            __syncthreads();
-#pragma unroll 1
-            for (int j = 0; j < i; ++j) {              // T_ij = -D_i X_ij
-                float xcol[16];
+        };
+        tile_product(A + 32 * kLdA, A);  // Y = A21 T1
 #pragma unroll
-                for (int m = 0; m < 16; ++m) xcol[m] = X[j * 256 + m * 16 + cc];
+        for (int i = 0; i < 4; ++i)
+            *reinterpret_cast<float4*>(A + (4 * tr + i) * kLdA + 32 + 4 * tc) =
+                make_float4(acc[i][0], acc[i][1], acc[i][2], acc[i][3]);
+        __syncthreads();
+        tile_product(A + 32 * kLdA + 32, A + 32);  // T2 Y
+        __syncthreads();  // every thread is done reading Y and A21
 #pragma unroll
-                for (int q = 0; q < 4; ++q) {
-                    const float4* dr = reinterpret_cast<const float4*>(arow[q] + 16 * i);
-                    float acc = 0.f;
-#pragma unroll
-                    for (int m4 = 0; m4 < 4; ++m4) {
-                        const float4 d = dr[m4];
-                        acc = fmaf(d.x, xcol[4 * m4 + 0], acc);
-                        acc = fmaf(d.y, xcol[4 * m4 + 1], acc);
-                        acc = fmaf(d.z, xcol[4 * m4 + 2], acc);
-                        acc = fmaf(d.w, xcol[4 * m4 + 3], acc);
-                    }
-                    A[(16 * i + rr0 + 4 * q) * kLdA + 16 * j + cc] = -acc;
-                }
-            }
-            __syncthreads();
+        for (int i = 0; i < 4; ++i) {
+            *reinterpret_cast<float4*>(A + (32 + 4 * tr + i) * kLdA + 4 * tc) =
+                make_float4(-acc[i][0], -acc[i][1], -acc[i][2], -acc[i][3]);
+            *reinterpret_cast<float4*>(A + (4 * tr + i) * kLdA + 32 + 4 * tc) = make_float4(0.f, 0.f, 0.f, 0.f);
         }
     }
+    __syncthreads();
 
     // ---- 5. MMA operand images [T_0 diag(b_0 gam_0); T_1 diag(b_1 gam_1)] and [T_0 diag(b_0); ...]
     {
