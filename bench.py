@@ -46,6 +46,20 @@ STATE_BYTES = HV * D * D * 4                                                    
 #   state = [W; Q] S^T, P Delta and the state update (per V head)
 PREP_FLOP_PER_TOKEN = HK * (2 * 2 * C * D) + HV * (2 * 2 * C * D)                    # 1,572,864
 STATE_FLOP_PER_TOKEN = HV * (2 * C * D + 3 * 2 * D * D)                               # 3,670,016
+# Algorithmic HBM bytes per full 64-token chunk of each tensor-core phase (the roofline
+# of both phases is the HBM one: their flop/byte ratios, about 30 and 90, are far below
+# the B200's bf16 ridge point).
+#   prep  reads q, k (bf16, per QK head), v (bf16), g, beta (fp32, per V head) once and
+#         writes the chunk's operand images: per V head W~ and U (64 x 128 bf16 each),
+#         P and M~ (64 x 64 bf16 each), diag(c) K (64 x 128 bf16) and the gate factors
+#         (129 fp32); per QK head the normalised Q (64 x 128 bf16).
+#   state reads those images once (Q, W~, M~, P, diag(c) K, U, gate factors) and writes
+#         the outputs (64 x 128 bf16 per V head); the state itself enters and leaves once
+#         per sequence (fp32, counted separately).
+PREP_BYTES_PER_CHUNK = (C * (2 * HK * D * 2 + HV * D * 2 + HV * 4 * 2)
+                        + HV * (3 * C * D * 2 + 2 * C * C * 2 + 129 * 4) + HK * C * D * 2)   # 3,440,768
+STATE_BYTES_PER_CHUNK = (HK * C * D * 2 + HV * (3 * C * D * 2 + 2 * C * C * 2 + 129 * 4)
+                         + HV * C * D * 2)                                                  # 2,900,096
 
 
 def decode_bytes(num_seqs, ntok):
@@ -258,21 +272,26 @@ def main_ours(args, rank, world, local_rank):
         timed_ev = phase_ev[-args.steps:]
         prep_ms = max_over_ranks(sum(e[0].elapsed_time(e[1]) for e in timed_ev) / args.steps)
         state_ms = max_over_ranks(sum(e[1].elapsed_time(e[2]) for e in timed_ev) / args.steps)
+        chunks = T // C  # one sequence of T tokens, T a multiple of the chunk size
         phases = {
             "prep": {"kernels": "chunk_table_kernel + chunk_prep_kernel", "ms": prep_ms,
-                     "flop": PREP_FLOP_PER_TOKEN * T,
-                     "tflops": PREP_FLOP_PER_TOKEN * T / (prep_ms * 1e-3) / 1e12},
+                     "flop": PREP_FLOP_PER_TOKEN * T, "bytes": PREP_BYTES_PER_CHUNK * chunks},
             "state": {"kernels": "chunk_state_kernel", "ms": state_ms,
                       "flop": STATE_FLOP_PER_TOKEN * T,
-                      "tflops": STATE_FLOP_PER_TOKEN * T / (state_ms * 1e-3) / 1e12}}
+                      "bytes": STATE_BYTES_PER_CHUNK * chunks + 2 * STATE_BYTES}}
+        for ph in phases.values():
+            ph["tflops"] = ph["flop"] / (ph["ms"] * 1e-3) / 1e12
+            ph["gbs"] = ph["bytes"] / (ph["ms"] * 1e-3) / 1e9
+            ph["frac_hbm"] = ph["gbs"] / peaks["hbm_gbs"]
+            ph["frac_tensor"] = ph["tflops"] / peak
         dom = max(phases, key=lambda k2: phases[k2]["ms"])
-        achieved = phases[dom]["tflops"]
-        roofline = {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
-                    "frac": achieved / peak, "traffic": None,
-                    "peak_source": peaks["source"] + " bf16 dense (burst)",
-                    "kernel": phases[dom]["kernels"],
-                    "algorithmic_flop_per_launch": phases[dom]["flop"],
-                    "step_frac": PREFILL_FLOP_PER_TOKEN * T / (ms_step * 1e-3) / 1e12 / peak}
+        d = phases[dom]
+        roofline = {"bound": "hbm", "achieved": d["gbs"], "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                    "frac": d["frac_hbm"], "traffic": None,
+                    "peak_source": peaks["source"] + " HBM copy",
+                    "kernel": d["kernels"], "algorithmic_bytes_per_launch": d["bytes"],
+                    "tensor_frac": d["frac_tensor"],
+                    "step_frac_tensor": PREFILL_FLOP_PER_TOKEN * T / (ms_step * 1e-3) / 1e12 / peak}
     else:
         flop = PREFILL_FLOP_PER_TOKEN * T
         achieved = flop / (ms_step * 1e-3) / 1e12
