@@ -49,7 +49,6 @@ namespace {
 
 using namespace sm100;
 
-constexpr int kThreads = 128;
 constexpr float kInvSqrtD = 0.08838834764831845f;  // 1 / sqrt(128)
 
 // Operand image sizes (bytes)
@@ -217,7 +216,11 @@ struct PrepSmall {
 };
 static_assert(sizeof(PrepSmall) <= 3072, "PrepSmall fits its region");
 
-__global__ void __launch_bounds__(kThreads, 2)
+// 256 threads: warp w reads Tensor Memory lane quarter w % 4; the two warps of a quarter
+// split the columns (column half hf = w / 4).
+constexpr int kPrepThreads = 256;
+
+__global__ void __launch_bounds__(kPrepThreads, 2)
 chunk_prep_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __restrict__ k,
                   const __nv_bfloat16* __restrict__ v, const float* __restrict__ g,
                   const float* __restrict__ beta, unsigned char* ws, int num_seqs,
@@ -236,29 +239,31 @@ chunk_prep_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __re
     const int4 ent = reinterpret_cast<const int4*>(ws + L.table)[cid];
     const int t0 = ent.y, len = ent.z;
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    const int qw = warp & 3, hf = warp >> 2;  // TMEM lane quarter, column half
     const int h0 = jq * 2;  // the two V heads of this QK head
     // The previous chunk (always a full one) belongs to the same sequence unless this chunk
     // is the sequence's first.
     const bool has_prev = cid > reinterpret_cast<const int32_t*>(ws + L.seq_chunk0)[ent.x];
 
-    // Thread's slice of a row for the row loads: 16 elements = 2 chunks of one 64-wide block.
+    // Row loads: 8 threads per row, 16 elements (2 chunks of one 64-wide block) each;
+    // 32 rows per pass.
     const int sub = tid & 7, kb = sub >> 2, c0 = (sub & 3) * 2;
     int err = 0;
     bool ok;
 
-    // ---- 0. K_prev rows to a staging area (async), the q, k row loads (4 passes of 16 rows),
-    //         gates, TMEM, barrier
+    // ---- 0. K_prev rows to a staging area (async), the q, k row loads (2 passes), gates,
+    //         TMEM, barrier
     if (has_prev) {
-        for (int i = tid; i < kChunk * 16; i += kThreads) {  // 64 rows x 16 pieces of 16 bytes
+        for (int i = tid; i < kChunk * 16; i += kPrepThreads) {  // 64 rows x 16 pieces of 16 bytes
             const int r = i >> 4, pc = i & 15;
             cp_async16(sm + kP_AF + r * 256 + pc * 16, k + ((size_t)(t0 - kChunk + r) * hk + jq) * kD + pc * 8);
         }
         cp_async_commit();
     }
-    uint4 kr[4][2], qr[4][2];
+    uint4 kr[2][2], qr[2][2];
 #pragma unroll
-    for (int pass = 0; pass < 4; ++pass) {
-        const int r = pass * 16 + (tid >> 3);
+    for (int pass = 0; pass < 2; ++pass) {
+        const int r = pass * 32 + (tid >> 3);
         if (r < len) {
             const size_t base = ((size_t)(t0 + r) * hk + jq) * kD + sub * 16;
             kr[pass][0] = *reinterpret_cast<const uint4*>(k + base);
@@ -273,16 +278,18 @@ chunk_prep_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __re
         const int h = h0 + warp;
         const float g0 = (lane < len) ? g[(size_t)(t0 + lane) * hv + h] : 0.f;
         const float g1 = (lane + 32 < len) ? g[(size_t)(t0 + lane + 32) * hv + h] : 0.f;
+        const float gp0 = has_prev ? g[(size_t)(t0 - kChunk + lane) * hv + h] : 0.f;
+        const float gp1 = has_prev ? g[(size_t)(t0 - kChunk + 32 + lane) * hv + h] : 0.f;
+        const float b0 = (lane < len) ? beta[(size_t)(t0 + lane) * hv + h] : 0.f;
+        const float b1 = (lane + 32 < len) ? beta[(size_t)(t0 + lane + 32) * hv + h] : 0.f;
         const float G0 = warp_inclusive_scan(g0, lane);
         const float G1 = warp_inclusive_scan(g1, lane) + __shfl_sync(0xffffffffu, G0, 31);
         ss.G[warp][lane] = G0 * kLog2e;
         ss.G[warp][lane + 32] = G1 * kLog2e;
         ss.gam[warp][lane] = expf(G0);
         ss.gam[warp][lane + 32] = expf(G1);
-        ss.b[warp][lane] = (lane < len) ? beta[(size_t)(t0 + lane) * hv + h] : 0.f;
-        ss.b[warp][lane + 32] = (lane + 32 < len) ? beta[(size_t)(t0 + lane + 32) * hv + h] : 0.f;
-        const float gp0 = has_prev ? g[(size_t)(t0 - kChunk + lane) * hv + h] : 0.f;
-        const float gp1 = has_prev ? g[(size_t)(t0 - kChunk + 32 + lane) * hv + h] : 0.f;
+        ss.b[warp][lane] = b0;
+        ss.b[warp][lane + 32] = b1;
         const float Gp0 = warp_inclusive_scan(gp0, lane);
         const float Gp1 = warp_inclusive_scan(gp1, lane) + __shfl_sync(0xffffffffu, Gp0, 31);
         const float GpL = __shfl_sync(0xffffffffu, Gp1, 31);
@@ -294,7 +301,7 @@ chunk_prep_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __re
         tmem_alloc(&ss.tmem_base, 256);
         tmem_relinquish();
     }
-    if (tid == 0) {
+    if (tid == 64) {
         mbar_init(&ss.bar_mma, 1);
         fence_mbar_init();
     }
@@ -310,8 +317,8 @@ chunk_prep_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __re
         unsigned char* kt_img1 = kt_img0 + kKTBytes;
         unsigned char* qn_img = ws + L.qn + ((size_t)cid * hk + jq) * kQBytes;
 #pragma unroll
-        for (int pass = 0; pass < 4; ++pass) {
-            const int r = pass * 16 + (tid >> 3);
+        for (int pass = 0; pass < 2; ++pass) {
+            const int r = pass * 32 + (tid >> 3);
             float kv[16], qv[16];
             unpack8(kr[pass][0], kv);
             unpack8(kr[pass][1], kv + 8);
@@ -345,8 +352,8 @@ chunk_prep_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __re
     if (has_prev) cp_async_wait_all();
     __syncthreads();  // the staged K_prev rows are visible to every thread
 #pragma unroll 1
-    for (int pass = 0; pass < 4; ++pass) {
-        const int r = pass * 16 + (tid >> 3);
+    for (int pass = 0; pass < 2; ++pass) {
+        const int r = pass * 32 + (tid >> 3);
         float kv[16];
         if (has_prev) {
             const uint4* src = reinterpret_cast<const uint4*>(sm + kP_AF + r * 256 + sub * 32);
@@ -382,12 +389,12 @@ chunk_prep_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __re
         mma_commit(&ss.bar_mma);
     }
     {
-        uint4 vr[2][4][2];
+        uint4 vr[2][2][2];
 #pragma unroll
         for (int hh = 0; hh < 2; ++hh)
 #pragma unroll
-            for (int pass = 0; pass < 4; ++pass) {
-                const int r = pass * 16 + (tid >> 3);
+            for (int pass = 0; pass < 2; ++pass) {
+                const int r = pass * 32 + (tid >> 3);
                 if (r < len) {
                     const uint4* vp = reinterpret_cast<const uint4*>(v + ((size_t)(t0 + r) * hv + h0 + hh) * kD + sub * 16);
                     vr[hh][pass][0] = vp[0];
@@ -412,53 +419,59 @@ chunk_prep_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __re
         if (__syncthreads_or(!ok)) { err = 1; goto cleanup; }
         tc_fence_after();
 
-        // ---- 3. from the Gram rows: P = lower(exp(G_r - G_j) Q K^T) of both heads to the
-        //         workspace (warps 0-1); A (fp32, smem) from K K^T and the bf16 image of
-        //         K K_prev^T (warps 2-3)
+        // ---- 3. from the Gram rows, columns 32 hf .. 32 hf + 31 of each block:
+        //         warps of quarters 0-1 (Q rows): P = lower(exp(G_r - G_j) Q K^T) of both heads
+        //         to the workspace; quarters 2-3 (K rows): A = strictly_lower(b_r exp(G_r - G_j)
+        //         K K^T) in fp32 -- the two 32x32 diagonal blocks stored transposed, for the
+        //         forward substitution -- and the bf16 image of K K_prev^T.
         {
-            float row[64];
-            tmem_ld64(tmem, warp, 0, row);
-            const int r = tid & 63;
-            if (warp >= 2) {
+            float row[32];
+            const uint32_t ta = tmem + ((uint32_t)qw * 32u << 16) + 32u * hf;
+            tmem_ld16(ta, row);
+            tmem_ld16(ta + 16, row + 16);
+            tmem_ld_wait();
+            const int r = (qw & 1) * 32 + lane;  // token row
+            const int j0 = 32 * hf;              // first column of this thread
+            if (qw >= 2) {
 #pragma unroll 1
                 for (int hh = 0; hh < 2; ++hh) {
                     const float Gr = ss.G[hh][r], br = ss.b[hh][r];
-                    const float4* g4 = reinterpret_cast<const float4*>(ss.G[hh]);
-                    float4* a4 = reinterpret_cast<float4*>(af + hh * kAfHead + r * kLdA);
+                    const float* gj = ss.G[hh] + j0;
+                    float* A = af + hh * kAfHead;
+                    float a[32];
 #pragma unroll
-                    for (int m = 0; m < 16; ++m) {
-                        const float4 gi = g4[m];
-                        const float gg[4] = {gi.x, gi.y, gi.z, gi.w};
-                        float t4[4];
+                    for (int e = 0; e < 32; ++e)
+                        a[e] = (j0 + e < r) ? br * fast_exp2(fminf(Gr - gj[e], 0.f)) * row[e] : 0.f;
+                    if ((r >> 5) == hf) {  // diagonal block, transposed: A^T[j][r]
 #pragma unroll
-                        for (int e = 0; e < 4; ++e) {
-                            const int i = 4 * m + e;
-                            t4[e] = (i < r) ? br * fast_exp2(fminf(Gr - gg[e], 0.f)) * row[i] : 0.f;
-                        }
-                        a4[m] = make_float4(t4[0], t4[1], t4[2], t4[3]);
+                        for (int e = 0; e < 32; ++e) A[(j0 + e) * kLdA + r] = a[e];
+                    } else if (hf < (r >> 5)) {  // A21, row-major
+                        float4* a4 = reinterpret_cast<float4*>(A + r * kLdA + j0);
+#pragma unroll
+                        for (int m = 0; m < 8; ++m) a4[m] = make_float4(a[4 * m], a[4 * m + 1], a[4 * m + 2], a[4 * m + 3]);
                     }
                 }
-                tmem_ld64(tmem, warp, 64, row);  // K K_prev^T, row r (MN-major B: K index r)
+                tmem_ld16(ta + 64, row);
+                tmem_ld16(ta + 80, row + 16);
+                tmem_ld_wait();
 #pragma unroll
-                for (int ch = 0; ch < 8; ++ch)
-                    *reinterpret_cast<uint4*>(sm + kP_GX + sw128(r, ch)) = pack8(row + 8 * ch);
+                for (int ch = 0; ch < 4; ++ch)
+                    *reinterpret_cast<uint4*>(sm + kP_GX + sw128(r, 4 * hf + ch)) = pack8(row + 8 * ch);
             } else {
 #pragma unroll 1
                 for (int hh = 0; hh < 2; ++hh) {
                     const float Gr = ss.G[hh][r];
-                    const float4* g4 = reinterpret_cast<const float4*>(ss.G[hh]);
+                    const float* gj = ss.G[hh] + j0;
                     unsigned char* pimg = ws + L.p + ((size_t)cid * hv + h0 + hh) * kPBytes;
 #pragma unroll
-                    for (int ch = 0; ch < 8; ++ch) {
-                        const float4 ga = g4[2 * ch], gb = g4[2 * ch + 1];
-                        const float gg[8] = {ga.x, ga.y, ga.z, ga.w, gb.x, gb.y, gb.z, gb.w};
+                    for (int ch = 0; ch < 4; ++ch) {
                         float p8[8];
 #pragma unroll
                         for (int e = 0; e < 8; ++e) {
-                            const int i = 8 * ch + e;
-                            p8[e] = (i <= r) ? fast_exp2(fminf(Gr - gg[e], 0.f)) * row[i] : 0.f;
+                            const int i = j0 + 8 * ch + e;
+                            p8[e] = (i <= r) ? fast_exp2(fminf(Gr - gj[8 * ch + e], 0.f)) * row[8 * ch + e] : 0.f;
                         }
-                        *reinterpret_cast<uint4*>(pimg + sw128(r, ch)) = pack8(p8);
+                        *reinterpret_cast<uint4*>(pimg + sw128(r, 4 * hf + ch)) = pack8(p8);
                     }
                 }
             }
@@ -468,8 +481,8 @@ chunk_prep_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __re
 #pragma unroll
         for (int hh = 0; hh < 2; ++hh)
 #pragma unroll
-            for (int pass = 0; pass < 4; ++pass) {
-                const int rr = pass * 16 + (tid >> 3);
+            for (int pass = 0; pass < 2; ++pass) {
+                const int rr = pass * 32 + (tid >> 3);
                 unsigned char* vb = sm + kP_GR + hh * 16384 + kb * kP_GRB;
                 *reinterpret_cast<uint4*>(vb + sw128(rr, c0)) = vr[hh][pass][0];
                 *reinterpret_cast<uint4*>(vb + sw128(rr, c0 + 1)) = vr[hh][pass][1];
@@ -479,110 +492,108 @@ chunk_prep_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __re
     tc_fence_before();
     __syncthreads();
 
-    // ---- 4. T = (I + A)^-1 per head, by 32x32 blocks, in place; 64 threads per head.
+    // ---- 4. T = (I + A)^-1 per head, by 32x32 blocks, in place; 128 threads per head.
     //         With A = [A11 0; A21 A22]:  T = [T1 0; T21 T2], T1 = (I + A11)^-1,
     //         T2 = (I + A22)^-1, T21 = -T2 (A21 T1).
-    //         (a) T1 and T2 by forward substitution: warp (head, block), lane = column j;
-    //             every lane reads the same A row (a shared-memory broadcast);
+    //         (a) T1 and T2 by forward substitution, one warp per block, lane = column j,
+    //             column-oriented: once x_k is known every later row's partial sum takes its
+    //             term (independent updates), reading row k of the transposed block;
     //         (b) Y = A21 T1 into the (zero) upper-right block, then T21 = -T2 Y, each thread
-    //             a 4x4 tile; the upper-right block is cleared again afterwards.
+    //             a 4x2 tile; the upper-right block is cleared again afterwards.
     {
-        const int hh = tid >> 6, l = tid & 63;
+        const int hh = tid >> 7, l = tid & 127;
         float* A = af + hh * kAfHead;
-        {
+        if (l < 64) {
             const int base = 32 * (l >> 5), j = l & 31;
-            float x[32];
+            float acc[32];
 #pragma unroll
-            for (int r = 0; r < 32; ++r) {
-                const float4* arow = reinterpret_cast<const float4*>(A + (base + r) * kLdA + base);
-                float acc = 0.f;
+            for (int r = 0; r < 32; ++r) acc[r] = 0.f;
 #pragma unroll
-                for (int k4 = 0; k4 < (r + 3) / 4; ++k4) {
-                    const float4 a = arow[k4];
+            for (int kk = 0; kk < 32; ++kk) {
+                const float xk = (kk == j) ? 1.f : ((kk < j) ? 0.f : -acc[kk]);
+                acc[kk] = xk;
+                const float4* at = reinterpret_cast<const float4*>(A + (base + kk) * kLdA + base);  // A^T row kk
+#pragma unroll
+                for (int r4 = (kk + 1) / 4; r4 < 8; ++r4) {
+                    const float4 a = at[r4];
                     const float av[4] = {a.x, a.y, a.z, a.w};
 #pragma unroll
                     for (int e = 0; e < 4; ++e)
-                        if (4 * k4 + e < r) acc = fmaf(av[e], x[4 * k4 + e], acc);
+                        if (4 * r4 + e > kk) acc[4 * r4 + e] = fmaf(av[e], xk, acc[4 * r4 + e]);
                 }
-                x[r] = (r == j) ? 1.f : ((r < j) ? 0.f : -acc);
             }
-            __syncwarp();  // every lane of this block's warp is done reading A_bb
+            __syncwarp();  // every lane of this block's warp is done reading A^T
 #pragma unroll
-            for (int r = 0; r < 32; ++r) A[(base + r) * kLdA + base + j] = x[r];
+            for (int r = 0; r < 32; ++r) A[(base + r) * kLdA + base + j] = acc[r];
         }
         __syncthreads();
-        const int tr = l >> 3, tc = l & 7;  // 4x4 output tile: rows 4 tr .., columns 4 tc ..
-        float acc[4][4];
-        auto tile_product = [&](const float* Lm, const float* Rm) {  // acc = Lm (32x32) Rm (32x32)
+        const int tr = l >> 4, tc = l & 15;  // 4x2 output tile: rows 4 tr .., columns 2 tc ..
+        float2 acc2[4];
+        auto tile_product = [&](const float* Lm, const float* Rm) {  // acc2 = Lm (32x32) Rm (32x32)
 #pragma unroll
-            for (int i = 0; i < 4; ++i)
-#pragma unroll
-                for (int m = 0; m < 4; ++m) acc[i][m] = 0.f;
+            for (int i = 0; i < 4; ++i) acc2[i] = make_float2(0.f, 0.f);
 #pragma unroll 2
             for (int k4 = 0; k4 < 8; ++k4) {
-                float4 a[4], b[4];
+                float4 a[4];
+                float2 b[4];
 #pragma unroll
                 for (int i = 0; i < 4; ++i) a[i] = *reinterpret_cast<const float4*>(Lm + (4 * tr + i) * kLdA + 4 * k4);
 #pragma unroll
-                for (int e = 0; e < 4; ++e) b[e] = *reinterpret_cast<const float4*>(Rm + (4 * k4 + e) * kLdA + 4 * tc);
+                for (int e = 0; e < 4; ++e) b[e] = *reinterpret_cast<const float2*>(Rm + (4 * k4 + e) * kLdA + 2 * tc);
 #pragma unroll
                 for (int i = 0; i < 4; ++i) {
-                    const float av[4] = {a[i].x, a[i].y, a[i].z, a[i].w};
-#pragma unroll
-                    for (int e = 0; e < 4; ++e) {
-                        acc[i][0] = fmaf(av[e], b[e].x, acc[i][0]);
-                        acc[i][1] = fmaf(av[e], b[e].y, acc[i][1]);
-                        acc[i][2] = fmaf(av[e], b[e].z, acc[i][2]);
-                        acc[i][3] = fmaf(av[e], b[e].w, acc[i][3]);
-                    }
+                    acc2[i] = __ffma2_rn(make_float2(a[i].x, a[i].x), b[0], acc2[i]);
+                    acc2[i] = __ffma2_rn(make_float2(a[i].y, a[i].y), b[1], acc2[i]);
+                    acc2[i] = __ffma2_rn(make_float2(a[i].z, a[i].z), b[2], acc2[i]);
+                    acc2[i] = __ffma2_rn(make_float2(a[i].w, a[i].w), b[3], acc2[i]);
                 }
             }
         };
         tile_product(A + 32 * kLdA, A);  // Y = A21 T1
 #pragma unroll
-        for (int i = 0; i < 4; ++i)
-            *reinterpret_cast<float4*>(A + (4 * tr + i) * kLdA + 32 + 4 * tc) =
-                make_float4(acc[i][0], acc[i][1], acc[i][2], acc[i][3]);
+        for (int i = 0; i < 4; ++i) *reinterpret_cast<float2*>(A + (4 * tr + i) * kLdA + 32 + 2 * tc) = acc2[i];
         __syncthreads();
         tile_product(A + 32 * kLdA + 32, A + 32);  // T2 Y
         __syncthreads();  // every thread is done reading Y and A21
 #pragma unroll
         for (int i = 0; i < 4; ++i) {
-            *reinterpret_cast<float4*>(A + (32 + 4 * tr + i) * kLdA + 4 * tc) =
-                make_float4(-acc[i][0], -acc[i][1], -acc[i][2], -acc[i][3]);
-            *reinterpret_cast<float4*>(A + (4 * tr + i) * kLdA + 32 + 4 * tc) = make_float4(0.f, 0.f, 0.f, 0.f);
+            *reinterpret_cast<float2*>(A + (32 + 4 * tr + i) * kLdA + 2 * tc) = make_float2(-acc2[i].x, -acc2[i].y);
+            *reinterpret_cast<float2*>(A + (4 * tr + i) * kLdA + 32 + 2 * tc) = make_float2(0.f, 0.f);
         }
     }
     __syncthreads();
 
     // ---- 5. MMA operand images [T_0 diag(b_0 gam_0); T_1 diag(b_1 gam_1)] and [T_0 diag(b_0); ...]
+    //         (two threads per row, 32 columns each)
     {
-        const int hh = tid >> 6, r = tid & 63;
-        const float4* t4 = reinterpret_cast<const float4*>(af + hh * kAfHead + r * kLdA);
-        uint4 wrow[8], urow[8];
+        const int hh = tid >> 7, r = (tid & 127) >> 1, hc = tid & 1;
+        const float4* t4 = reinterpret_cast<const float4*>(af + hh * kAfHead + r * kLdA + 32 * hc);
+        const float* bj = ss.b[hh] + 32 * hc;
+        const float* gj = ss.gam[hh] + 32 * hc;
+        uint4 wrow[4], urow[4];
 #pragma unroll
-        for (int ch = 0; ch < 8; ++ch) {
+        for (int ch = 0; ch < 4; ++ch) {
             float w8[8], u8[8];
 #pragma unroll
             for (int half4 = 0; half4 < 2; ++half4) {
-                const int m = 2 * ch + half4;   // float4 group: columns 4m .. 4m+3
-                const float4 tv = t4[m];
+                const float4 tv = t4[2 * ch + half4];
                 const float tt[4] = {tv.x, tv.y, tv.z, tv.w};
 #pragma unroll
                 for (int e = 0; e < 4; ++e) {
-                    const int j = 4 * m + e;
-                    u8[4 * half4 + e] = tt[e] * ss.b[hh][j];
-                    w8[4 * half4 + e] = u8[4 * half4 + e] * ss.gam[hh][j];
+                    const int jj = 8 * ch + 4 * half4 + e;
+                    u8[4 * half4 + e] = tt[e] * bj[jj];
+                    w8[4 * half4 + e] = u8[4 * half4 + e] * gj[jj];
                 }
             }
             wrow[ch] = pack8(w8);
             urow[ch] = pack8(u8);
         }
         __syncthreads();
+        const int row = hh * 64 + r;
 #pragma unroll
-        for (int ch = 0; ch < 8; ++ch) {
-            *reinterpret_cast<uint4*>(sm + kP_AF + sw128(tid, ch)) = wrow[ch];
-            *reinterpret_cast<uint4*>(sm + kP_AF + 16384 + sw128(tid, ch)) = urow[ch];
+        for (int ch = 0; ch < 4; ++ch) {
+            *reinterpret_cast<uint4*>(sm + kP_AF + sw128(row, 4 * hc + ch)) = wrow[ch];
+            *reinterpret_cast<uint4*>(sm + kP_AF + 16384 + sw128(row, 4 * hc + ch)) = urow[ch];
         }
     }
     fence_async_smem();
@@ -605,31 +616,32 @@ chunk_prep_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __re
     if (__syncthreads_or(!ok)) { err = 1; goto cleanup; }
     tc_fence_after();
 
-    // ---- 7. epilogue: accumulator row r' is row r' % 64 of head r' / 64.  The W image is
-    //         stored pre-scaled by the previous chunk's total decay (W~ = gam_L,prev W).
+    // ---- 7. epilogue: accumulator row r' (lane quarter qw) is row r' % 64 of head r' / 64;
+    //         each warp takes 64 of the 128 columns.  The W image is stored pre-scaled by the
+    //         previous chunk's total decay (W~ = gam_L,prev W).
     {
-        const int hh = tid >> 6, r = tid & 63, h = h0 + hh;
+        const int hh = qw >> 1, r = (qw & 1) * 32 + lane, h = h0 + hh;
+        const uint32_t tq = tmem + ((uint32_t)qw * 32u << 16);
         unsigned char* wimg = ws + L.w + ((size_t)cid * hv + h) * kWBytes;
         unsigned char* uimg = ws + L.u + ((size_t)cid * hv + h) * kUBytes;
         const float gp = ss.gprev[hh];
-        float col[64];
+        float col[32];
+        auto store32 = [&](unsigned char* img, uint32_t tcol, int chunk0, float scale) {
+            tmem_ld16(tq + tcol, col);
+            tmem_ld16(tq + tcol + 16, col + 16);
+            tmem_ld_wait();
 #pragma unroll
-        for (int half = 0; half < 2; ++half) {
-            tmem_ld64(tmem, warp, 64 * half, col);
+            for (int e = 0; e < 32; ++e) col[e] *= scale;
 #pragma unroll
-            for (int e = 0; e < 64; ++e) col[e] *= gp;
-#pragma unroll
-            for (int ch = 0; ch < 8; ++ch)
-                *reinterpret_cast<uint4*>(wimg + half * 8192 + sw128(r, ch)) = pack8(col + 8 * ch);
-        }
-        if (hh == 0) {
-#pragma unroll
-            for (int half = 0; half < 2; ++half) {
-                tmem_ld64(tmem, warp, 128 + 64 * half, col);
-#pragma unroll
-                for (int ch = 0; ch < 8; ++ch)
-                    *reinterpret_cast<uint4*>(uimg + half * 8192 + sw128(r, ch)) = pack8(col + 8 * ch);
-            }
+            for (int ch = 0; ch < 4; ++ch)
+                *reinterpret_cast<uint4*>(img + sw128(r, chunk0 + ch)) = pack8(col + 8 * ch);
+        };
+        // W columns 64 hf .. 64 hf + 63 = d_k block hf (8 KB image half)
+        store32(wimg + hf * 8192, 64 * hf, 0, gp);
+        store32(wimg + hf * 8192, 64 * hf + 32, 4, gp);
+        if (hh == 0) {  // U of head 0: columns 128 + 64 hf ..
+            store32(uimg + hf * 8192, 128 + 64 * hf, 0, 1.f);
+            store32(uimg + hf * 8192, 128 + 64 * hf + 32, 4, 1.f);
         }
         tc_fence_before();
         __syncthreads();
@@ -650,26 +662,20 @@ chunk_prep_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __re
         if (__syncthreads_or(!ok)) { err = 1; goto cleanup; }
         tc_fence_after();
         if (hh == 1) {
-#pragma unroll
-            for (int half = 0; half < 2; ++half) {
-                tmem_ld64(tmem, warp, 128 + 64 * half, col);
-#pragma unroll
-                for (int ch = 0; ch < 8; ++ch)
-                    *reinterpret_cast<uint4*>(uimg + half * 8192 + sw128(r, ch)) = pack8(col + 8 * ch);
-            }
+            store32(uimg + hf * 8192, 128 + 64 * hf, 0, 1.f);
+            store32(uimg + hf * 8192, 128 + 64 * hf + 32, 4, 1.f);
         }
-        {
+        {   // M~ = M diag(c_prev): columns 32 hf .. 32 hf + 31
             unsigned char* mimg = ws + L.m + ((size_t)cid * hv + h) * kMBytes;
-            tmem_ld64(tmem, warp, 0, col);
-            const float4* cp4 = reinterpret_cast<const float4*>(ss.cprev[hh]);
+            tmem_ld16(tq + 32 * hf, col);
+            tmem_ld16(tq + 32 * hf + 16, col + 16);
+            tmem_ld_wait();
+            const float* cp = ss.cprev[hh] + 32 * hf;
 #pragma unroll
-            for (int j4 = 0; j4 < 16; ++j4) {
-                const float4 cv4 = cp4[j4];
-                col[4 * j4] *= cv4.x; col[4 * j4 + 1] *= cv4.y; col[4 * j4 + 2] *= cv4.z; col[4 * j4 + 3] *= cv4.w;
-            }
+            for (int e = 0; e < 32; ++e) col[e] *= cp[e];
 #pragma unroll
-            for (int ch = 0; ch < 8; ++ch)
-                *reinterpret_cast<uint4*>(mimg + sw128(r, ch)) = pack8(col + 8 * ch);
+            for (int ch = 0; ch < 4; ++ch)
+                *reinterpret_cast<uint4*>(mimg + sw128(r, 4 * hf + ch)) = pack8(col + 8 * ch);
         }
     }
 
@@ -1082,7 +1088,7 @@ cudaError_t launch_prefill_tc_prep(const void* q, const void* k, const void* v, 
     if (e != cudaSuccess) return e;
     chunk_table_kernel<<<1, 1024, 0, stream>>>(cu, num_seqs, ws);
     if (L.max_chunks > 0 && total_tokens > 0) {
-        chunk_prep_kernel<<<(unsigned)(L.max_chunks * hk), kThreads, kPrepSmem, stream>>>(
+        chunk_prep_kernel<<<(unsigned)(L.max_chunks * hk), kPrepThreads, kPrepSmem, stream>>>(
             (const __nv_bfloat16*)q, (const __nv_bfloat16*)k, (const __nv_bfloat16*)v, g, beta, ws,
             num_seqs, total_tokens, hk, hv);
     }
