@@ -11,32 +11,21 @@
 // Three kernels, all on the caller's stream:
 //  K0 chunk_table_kernel  cu_seqlens -> per-sequence first chunk id and a (seq, start,
 //                         length) entry per chunk, on the device (no host read).
-//  K1 chunk_prep_kernel   one CTA per (chunk, QK head), all chunks in parallel, both V
-//                         heads of the QK head:
-//                         - normalisation; K K^T and Q K^T as one M=128 MMA [K; Q] K^T;
-//                         - decay masks A and P; T = (I + A)^-1 in fp32 by 16x16 blocks:
-//                           diagonal inverses by forward substitution, then the blocks below
-//                           the diagonal as dense 16x16 products (64 threads per V head);
+//  K1 chunk_prep_kernel   one CTA (256 threads) per (chunk, QK head), all chunks in
+//                         parallel, both V heads of the QK head:
+//                         - normalisation; Q K^T, K K^T and the cross Gram K K_prev^T with
+//                           the previous chunk's keys as one M=128, N=128 MMA;
+//                         - decay masks A and P; T = (I + A)^-1 in fp32 by 32x32 blocks
+//                           (forward substitution per diagonal block, then one off-diagonal
+//                           block as two dense products);
 //                         - W and U of both heads as M=128 MMAs [T_0 D_0; T_1 D_1] x (K or V),
-//                           so each thread owns one output row and writes 16-byte chunks;
+//                           and M~ = [T D] (K K_prev^T) diag(c_prev);
 //                         - bf16 operand images, already in the 128-byte swizzled layout the
-//                           state kernel's MMAs read, go to the workspace, with the gate
+//                           state kernel's MMAs read, go to the workspace: W~ = gam_L,prev W,
+//                           U, P, M~, diag(c) K per V head and Q per QK head, with the gate
 //                           factors (c, gam) of each V head.
-//  K2 chunk_state_kernel  one CTA per (sequence, V head, quarter of d_v): the rows of S (one
-//                         per d_v index) evolve independently, so the 32-row slices run on
-//                         separate SMs, sequentially over the sequence's chunks.  Warp 8
-//                         issues the MMAs (N = 32), warp 9 the bulk copies (two chunks
-//                         ahead, three buffers); warps 0-7 compute, each warp on 16 of the
-//                         32 d_v columns of its TMEM lane quarter.  Per chunk:
-//                           [X; Y] = [W; Q] S^T          (M=128)            <- on the chain
-//                           Delta = U - X, c Delta       (lanes 0-63: token rows)
-//                           K^T diag(c) Delta            (M=128: d_k rows)  <- on the chain
-//                           S^T <- gam_L S^T + K^T diag(c) Delta   (fp32 in registers)
-//                           P Delta                      (M=128 operand [U; P]: rows 64..127)
-//                           O = diag(gam) Y + P Delta    (lanes 64-127, one chunk later)
-//                         Hand-offs between the issuing and the compute warps are mbarriers;
-//                         the output accumulators are triple-buffered in Tensor Memory so
-//                         the output epilogue stays off the state chain.
+//  K2 chunk_state_kernel  one CTA per (sequence, V head, quarter of d_v), sequential over the
+//                         sequence's chunks, in the look-ahead form described at the kernel.
 // Every mbarrier wait is bounded (1 s) and, in the state kernel, also gives up as soon as
 // another thread of the CTA has given up; the kernel then records an error in the
 // workspace header, drains its own copies and MMAs (bounded), frees Tensor Memory and
