@@ -299,12 +299,11 @@ chunk_prep_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __re
     tc_fence_after();
     const uint32_t tmem = ss.tmem_base;
 
-    // ---- 1. normalise; Q, K and K_prev rows K-major in smem; Q and diag(c) K images to the
-    //         workspace (the latter once per V head)
+    // ---- 1. normalise; Q, K and K_prev rows K-major in smem.  (Global stores wait until
+    //         after the proxy fences below: a fence.proxy.async also waits for the thread's
+    //         stores in flight, so each phase writes shared memory, fences, and only then
+    //         stores to the workspace.)
     {
-        unsigned char* kt_img0 = ws + L.kt + ((size_t)cid * hv + h0) * kKTBytes;
-        unsigned char* kt_img1 = kt_img0 + kKTBytes;
-        unsigned char* qn_img = ws + L.qn + ((size_t)cid * hk + jq) * kQBytes;
 #pragma unroll
         for (int pass = 0; pass < 2; ++pass) {
             const int r = pass * 32 + (tid >> 3);
@@ -320,21 +319,11 @@ chunk_prep_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __re
             const float rq = rsqrtf(sum8(ssq) + kNormEps) * kInvSqrtD;
 #pragma unroll
             for (int e = 0; e < 16; ++e) { kv[e] *= rk; qv[e] *= rq; }
-            // c_r = exp(G_L - G_r) of each V head (0 beyond the chunk's length)
-            const float cr0 = (r < len) ? fast_exp2(ss.G[0][len - 1] - ss.G[0][r]) : 0.f;
-            const float cr1 = (r < len) ? fast_exp2(ss.G[1][len - 1] - ss.G[1][r]) : 0.f;
 #pragma unroll
             for (int cc = 0; cc < 2; ++cc) {
                 const int ch = c0 + cc;
-                const uint4 kp8 = pack8(kv + 8 * cc), qp8 = pack8(qv + 8 * cc);
-                float k0[8], k1[8];
-#pragma unroll
-                for (int e = 0; e < 8; ++e) { k0[e] = kv[8 * cc + e] * cr0; k1[e] = kv[8 * cc + e] * cr1; }
-                *reinterpret_cast<uint4*>(sm + kP_GR + kb * kP_GRB + sw128(r, ch)) = qp8;
-                *reinterpret_cast<uint4*>(sm + kP_GR + kb * kP_GRB + 8192 + sw128(r, ch)) = kp8;
-                *reinterpret_cast<uint4*>(kt_img0 + kb * 8192 + sw128(r, ch)) = pack8(k0);
-                *reinterpret_cast<uint4*>(kt_img1 + kb * 8192 + sw128(r, ch)) = pack8(k1);
-                *reinterpret_cast<uint4*>(qn_img + kb * 8192 + sw128(r, ch)) = qp8;
+                *reinterpret_cast<uint4*>(sm + kP_GR + kb * kP_GRB + sw128(r, ch)) = pack8(qv + 8 * cc);
+                *reinterpret_cast<uint4*>(sm + kP_GR + kb * kP_GRB + 8192 + sw128(r, ch)) = pack8(kv + 8 * cc);
             }
         }
     }
@@ -377,6 +366,12 @@ chunk_prep_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __re
         }
         mma_commit(&ss.bar_mma);
     }
+    if (tid == 32) {  // the Q image is the Q slot as it stands: two 8 KB bulk stores
+        unsigned char* qn_img = ws + L.qn + ((size_t)cid * hk + jq) * kQBytes;
+        bulk_s2g(qn_img, sm + kP_GR, 8192);
+        bulk_s2g(qn_img + 8192, sm + kP_GR + kP_GRB, 8192);
+        bulk_commit();
+    }
     {
         uint4 vr[2][2][2];
 #pragma unroll
@@ -405,6 +400,7 @@ chunk_prep_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __re
             }
         }
         ok = mbar_wait(&ss.bar_mma, 0);
+        if (tid == 32) bulk_wait_read_all();  // the Q slot is read before V overwrites it
         if (__syncthreads_or(!ok)) { err = 1; goto cleanup; }
         tc_fence_after();
 
@@ -413,57 +409,38 @@ chunk_prep_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __re
         //         to the workspace; quarters 2-3 (K rows): A = strictly_lower(b_r exp(G_r - G_j)
         //         K K^T) in fp32 -- the two 32x32 diagonal blocks stored transposed, for the
         //         forward substitution -- and the bf16 image of K K_prev^T.
-        {
-            float row[32];
-            const uint32_t ta = tmem + ((uint32_t)qw * 32u << 16) + 32u * hf;
+        float row[32];
+        const uint32_t ta = tmem + ((uint32_t)qw * 32u << 16) + 32u * hf;
+        const int r = (qw & 1) * 32 + lane;  // token row
+        const int j0 = 32 * hf;              // first column of this thread
+        if (qw >= 2) {
             tmem_ld16(ta, row);
             tmem_ld16(ta + 16, row + 16);
             tmem_ld_wait();
-            const int r = (qw & 1) * 32 + lane;  // token row
-            const int j0 = 32 * hf;              // first column of this thread
-            if (qw >= 2) {
 #pragma unroll 1
-                for (int hh = 0; hh < 2; ++hh) {
-                    const float Gr = ss.G[hh][r], br = ss.b[hh][r];
-                    const float* gj = ss.G[hh] + j0;
-                    float* A = af + hh * kAfHead;
-                    float a[32];
+            for (int hh = 0; hh < 2; ++hh) {
+                const float Gr = ss.G[hh][r], br = ss.b[hh][r];
+                const float* gj = ss.G[hh] + j0;
+                float* A = af + hh * kAfHead;
+                float a[32];
 #pragma unroll
-                    for (int e = 0; e < 32; ++e)
-                        a[e] = (j0 + e < r) ? br * fast_exp2(fminf(Gr - gj[e], 0.f)) * row[e] : 0.f;
-                    if ((r >> 5) == hf) {  // diagonal block, transposed: A^T[j][r]
+                for (int e = 0; e < 32; ++e)
+                    a[e] = (j0 + e < r) ? br * fast_exp2(fminf(Gr - gj[e], 0.f)) * row[e] : 0.f;
+                if ((r >> 5) == hf) {  // diagonal block, transposed: A^T[j][r]
 #pragma unroll
-                        for (int e = 0; e < 32; ++e) A[(j0 + e) * kLdA + r] = a[e];
-                    } else if (hf < (r >> 5)) {  // A21, row-major
-                        float4* a4 = reinterpret_cast<float4*>(A + r * kLdA + j0);
+                    for (int e = 0; e < 32; ++e) A[(j0 + e) * kLdA + r] = a[e];
+                } else if (hf < (r >> 5)) {  // A21, row-major
+                    float4* a4 = reinterpret_cast<float4*>(A + r * kLdA + j0);
 #pragma unroll
-                        for (int m = 0; m < 8; ++m) a4[m] = make_float4(a[4 * m], a[4 * m + 1], a[4 * m + 2], a[4 * m + 3]);
-                    }
-                }
-                tmem_ld16(ta + 64, row);
-                tmem_ld16(ta + 80, row + 16);
-                tmem_ld_wait();
-#pragma unroll
-                for (int ch = 0; ch < 4; ++ch)
-                    *reinterpret_cast<uint4*>(sm + kP_GX + sw128(r, 4 * hf + ch)) = pack8(row + 8 * ch);
-            } else {
-#pragma unroll 1
-                for (int hh = 0; hh < 2; ++hh) {
-                    const float Gr = ss.G[hh][r];
-                    const float* gj = ss.G[hh] + j0;
-                    unsigned char* pimg = ws + L.p + ((size_t)cid * hv + h0 + hh) * kPBytes;
-#pragma unroll
-                    for (int ch = 0; ch < 4; ++ch) {
-                        float p8[8];
-#pragma unroll
-                        for (int e = 0; e < 8; ++e) {
-                            const int i = j0 + 8 * ch + e;
-                            p8[e] = (i <= r) ? fast_exp2(fminf(Gr - gj[8 * ch + e], 0.f)) * row[8 * ch + e] : 0.f;
-                        }
-                        *reinterpret_cast<uint4*>(pimg + sw128(r, 4 * hf + ch)) = pack8(p8);
-                    }
+                    for (int m = 0; m < 8; ++m) a4[m] = make_float4(a[4 * m], a[4 * m + 1], a[4 * m + 2], a[4 * m + 3]);
                 }
             }
+            tmem_ld16(ta + 64, row);
+            tmem_ld16(ta + 80, row + 16);
+            tmem_ld_wait();
+#pragma unroll
+            for (int ch = 0; ch < 4; ++ch)
+                *reinterpret_cast<uint4*>(sm + kP_GX + sw128(r, 4 * hf + ch)) = pack8(row + 8 * ch);
         }
         // V images (MN-major: token row, d_v contiguous; d_v blocks kP_GRB apart) into the
         // dead Q (head 0) and K_prev (head 1) slots
@@ -476,8 +453,29 @@ chunk_prep_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __re
                 *reinterpret_cast<uint4*>(vb + sw128(rr, c0)) = vr[hh][pass][0];
                 *reinterpret_cast<uint4*>(vb + sw128(rr, c0 + 1)) = vr[hh][pass][1];
             }
+        fence_async_smem();
+        if (qw < 2) {  // P rows, after the fence: these stores may stay in flight
+            tmem_ld16(ta, row);
+            tmem_ld16(ta + 16, row + 16);
+            tmem_ld_wait();
+#pragma unroll 1
+            for (int hh = 0; hh < 2; ++hh) {
+                const float Gr = ss.G[hh][r];
+                const float* gj = ss.G[hh] + j0;
+                unsigned char* pimg = ws + L.p + ((size_t)cid * hv + h0 + hh) * kPBytes;
+#pragma unroll
+                for (int ch = 0; ch < 4; ++ch) {
+                    float p8[8];
+#pragma unroll
+                    for (int e = 0; e < 8; ++e) {
+                        const int i = j0 + 8 * ch + e;
+                        p8[e] = (i <= r) ? fast_exp2(fminf(Gr - gj[8 * ch + e], 0.f)) * row[8 * ch + e] : 0.f;
+                    }
+                    *reinterpret_cast<uint4*>(pimg + sw128(r, 4 * hf + ch)) = pack8(p8);
+                }
+            }
+        }
     }
-    fence_async_smem();
     tc_fence_before();
     __syncthreads();
 
@@ -514,6 +512,25 @@ chunk_prep_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __re
             __syncwarp();  // every lane of this block's warp is done reading A^T
 #pragma unroll
             for (int r = 0; r < 32; ++r) A[(base + r) * kLdA + base + j] = acc[r];
+        } else {
+            // meanwhile the other 64 threads of the head write its diag(c) K image from the
+            // K slot, rows scaled by c_r = exp(G_L - G_r) (0 beyond the chunk's length); eight
+            // lanes cover one 128-byte image row, so every store instruction writes whole lines
+            const int lk = l - 64, pc = lk & 7;
+            unsigned char* kt_img = ws + L.kt + ((size_t)cid * hv + h0 + hh) * kKTBytes;
+            const float GL = ss.G[hh][len - 1];
+#pragma unroll 2
+            for (int i = 0; i < 16; ++i) {  // 16 passes of 8 rows: (d_k block, row) pairs
+                const int rowi = i * 8 + (lk >> 3);
+                const int kb2 = rowi >> 6, r = rowi & 63;
+                const float cr = (r < len) ? fast_exp2(GL - ss.G[hh][r]) : 0.f;
+                const uint32_t off = kb2 * 8192 + r * 128 + pc * 16;  // same swizzled position
+                float kv8[8];
+                unpack8(*reinterpret_cast<const uint4*>(sm + kP_GR + kb2 * kP_GRB + 8192 + r * 128 + pc * 16), kv8);
+#pragma unroll
+                for (int e = 0; e < 8; ++e) kv8[e] *= cr;
+                *reinterpret_cast<uint4*>(kt_img + off) = pack8(kv8);
+            }
         }
         __syncthreads();
         const int tr = l >> 4, tc = l & 15;  // 4x2 output tile: rows 4 tr .., columns 2 tc ..
