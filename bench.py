@@ -312,14 +312,58 @@ def main_ours(args, rank, world, local_rank):
                               dbuf["cu_seqlens"], out, fin, workspace=ws, algo=algo, stream=stream)
         hout.copy_(out, non_blocking=True)
 
+    def e2e_pipelined(steps):
+        """`steps` prefills back to back, each with its own host->device input copy and
+        device->host output copy, pipelined over three streams with double-buffered device
+        inputs and outputs: the copies of neighbouring steps overlap each other (PCIe is
+        full duplex) and the kernels.  Returns ms per step (device events, whole loop)."""
+        s_in, s_out = torch.cuda.Stream(dev), torch.cuda.Stream(dev)
+        bufs = [{k2: torch.empty_like(x[k2]) for k2 in host} for _ in range(2)]
+        outs = [torch.empty_like(out) for _ in range(2)]
+        houts = [hout, torch.empty(out.shape, dtype=out.dtype).pin_memory()]
+        ev = lambda: torch.cuda.Event()  # noqa: E731
+        h2d_done, comp_done, d2h_done = [ev() for _ in range(steps)], [ev() for _ in range(steps)], [ev() for _ in range(steps)]
+        torch.cuda.synchronize(dev)
+        barrier()
+        t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        t0.record(s_in)
+        for i in range(steps):
+            b2 = i % 2
+            if i >= 2:
+                s_in.wait_event(comp_done[i - 2])
+            with torch.cuda.stream(s_in):
+                for k2 in host:
+                    bufs[b2][k2].copy_(host[k2], non_blocking=True)
+            h2d_done[i].record(s_in)
+            stream.wait_event(h2d_done[i])
+            if i >= 2:
+                stream.wait_event(d2h_done[i - 2])
+            gdn.gdn_chunk_prefill(bufs[b2]["q"], bufs[b2]["k"], bufs[b2]["v"], bufs[b2]["g"], bufs[b2]["beta"],
+                                  None, bufs[b2]["cu_seqlens"], outs[b2], fin, workspace=ws, algo=algo,
+                                  stream=stream)
+            comp_done[i].record(stream)
+            s_out.wait_event(comp_done[i])
+            with torch.cuda.stream(s_out):
+                houts[b2].copy_(outs[b2], non_blocking=True)
+            d2h_done[i].record(s_out)
+        s_out.wait_event(d2h_done[steps - 1])
+        t1.record(s_out)
+        torch.cuda.synchronize(dev)
+        barrier()
+        return t0.elapsed_time(t1) / steps
+
     e2e = None
     if not args.no_e2e:
         e2e_ms = timed(e2e_once, max(3, args.steps // 2), 2)
-        e2e_step = max_over_ranks(sum(e2e_ms) / len(e2e_ms))
+        serial_step = max_over_ranks(sum(e2e_ms) / len(e2e_ms))
+        e2e_pipelined(3)  # warm-up
+        e2e_step = max_over_ranks(e2e_pipelined(max(4, args.steps)))
         h2d = sum(t.numel() * t.element_size() for t in host.values())
         d2h = hout.numel() * hout.element_size()
         e2e = {"value": world * T / (e2e_step * 1e-3), "unit": UNIT,
-               "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h}
+               "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+               "ms_per_step": e2e_step, "pipelined": True,
+               "serial_value": world * T / (serial_step * 1e-3)}
 
     # ---- decode: 256 sequences, 1 token and 4-token verify
     dec = {}
