@@ -240,12 +240,15 @@ chunk_prep_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __re
     int err = 0;
     bool ok;
 
-    // ---- 0. K_prev rows to a staging area (async), the q, k row loads (2 passes), gates,
-    //         TMEM, barrier
+    // ---- 0. loads: each thread stages (async) exactly the K_prev pieces it normalises
+    //         below, and loads its q, k rows (2 passes); warps 0-1 the gates; TMEM; barrier
     if (has_prev) {
-        for (int i = tid; i < kChunk * 16; i += kPrepThreads) {  // 64 rows x 16 pieces of 16 bytes
-            const int r = i >> 4, pc = i & 15;
-            cp_async16(sm + kP_AF + r * 256 + pc * 16, k + ((size_t)(t0 - kChunk + r) * hk + jq) * kD + pc * 8);
+#pragma unroll
+        for (int pass = 0; pass < 2; ++pass) {
+            const int r = pass * 32 + (tid >> 3);
+            const __nv_bfloat16* src = k + ((size_t)(t0 - kChunk + r) * hk + jq) * kD + sub * 16;
+            cp_async16(sm + kP_AF + r * 256 + sub * 32, src);
+            cp_async16(sm + kP_AF + r * 256 + sub * 32 + 16, src + 8);
         }
         cp_async_commit();
     }
@@ -294,41 +297,35 @@ chunk_prep_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __re
         mbar_init(&ss.bar_mma, 1);
         fence_mbar_init();
     }
-    tc_fence_before();
-    __syncthreads();
-    tc_fence_after();
-    const uint32_t tmem = ss.tmem_base;
 
-    // ---- 1. normalise; Q, K and K_prev rows K-major in smem.  (Global stores wait until
-    //         after the proxy fences below: a fence.proxy.async also waits for the thread's
-    //         stores in flight, so each phase writes shared memory, fences, and only then
-    //         stores to the workspace.)
-    {
+    // ---- 1. normalise q, k and K_prev rows into their K-major smem slots (no dependency on
+    //         the gates, so no barrier before it).  (Global stores wait until after the proxy
+    //         fences below: a fence.proxy.async also waits for the thread's stores in flight,
+    //         so each phase writes shared memory, fences, and only then stores to the
+    //         workspace.)
 #pragma unroll
-        for (int pass = 0; pass < 2; ++pass) {
-            const int r = pass * 32 + (tid >> 3);
-            float kv[16], qv[16];
-            unpack8(kr[pass][0], kv);
-            unpack8(kr[pass][1], kv + 8);
-            unpack8(qr[pass][0], qv);
-            unpack8(qr[pass][1], qv + 8);
-            float ssk = 0.f, ssq = 0.f;
+    for (int pass = 0; pass < 2; ++pass) {
+        const int r = pass * 32 + (tid >> 3);
+        float kv[16], qv[16];
+        unpack8(kr[pass][0], kv);
+        unpack8(kr[pass][1], kv + 8);
+        unpack8(qr[pass][0], qv);
+        unpack8(qr[pass][1], qv + 8);
+        float ssk = 0.f, ssq = 0.f;
 #pragma unroll
-            for (int e = 0; e < 16; ++e) { ssk = fmaf(kv[e], kv[e], ssk); ssq = fmaf(qv[e], qv[e], ssq); }
-            const float rk = rsqrtf(sum8(ssk) + kNormEps);
-            const float rq = rsqrtf(sum8(ssq) + kNormEps) * kInvSqrtD;
+        for (int e = 0; e < 16; ++e) { ssk = fmaf(kv[e], kv[e], ssk); ssq = fmaf(qv[e], qv[e], ssq); }
+        const float rk = rsqrtf(sum8(ssk) + kNormEps);
+        const float rq = rsqrtf(sum8(ssq) + kNormEps) * kInvSqrtD;
 #pragma unroll
-            for (int e = 0; e < 16; ++e) { kv[e] *= rk; qv[e] *= rq; }
+        for (int e = 0; e < 16; ++e) { kv[e] *= rk; qv[e] *= rq; }
 #pragma unroll
-            for (int cc = 0; cc < 2; ++cc) {
-                const int ch = c0 + cc;
-                *reinterpret_cast<uint4*>(sm + kP_GR + kb * kP_GRB + sw128(r, ch)) = pack8(qv + 8 * cc);
-                *reinterpret_cast<uint4*>(sm + kP_GR + kb * kP_GRB + 8192 + sw128(r, ch)) = pack8(kv + 8 * cc);
-            }
+        for (int cc = 0; cc < 2; ++cc) {
+            const int ch = c0 + cc;
+            *reinterpret_cast<uint4*>(sm + kP_GR + kb * kP_GRB + sw128(r, ch)) = pack8(qv + 8 * cc);
+            *reinterpret_cast<uint4*>(sm + kP_GR + kb * kP_GRB + 8192 + sw128(r, ch)) = pack8(kv + 8 * cc);
         }
     }
-    if (has_prev) cp_async_wait_all();
-    __syncthreads();  // the staged K_prev rows are visible to every thread
+    if (has_prev) cp_async_wait_all();  // this thread's own staged pieces
 #pragma unroll 1
     for (int pass = 0; pass < 2; ++pass) {
         const int r = pass * 32 + (tid >> 3);
@@ -352,7 +349,10 @@ chunk_prep_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __re
             *reinterpret_cast<uint4*>(sm + kP_GR + kb * kP_GRB + 16384 + sw128(r, c0 + cc)) = pack8(kv + 8 * cc);
     }
     fence_async_smem();
-    __syncthreads();
+    tc_fence_before();
+    __syncthreads();  // gates, TMEM address, barrier and the three row slots are ready
+    tc_fence_after();
+    const uint32_t tmem = ss.tmem_base;
 
     // ---- 2. Gram: TMEM[0:128, 0:128] = [Q; K] [K; K_prev]^T  (M=128, N=128, K=128); V loads
     //         meanwhile.  Rows 0..63: Q K^T | Q K_prev^T (unused); rows 64..127: K K^T | K K_prev^T.
