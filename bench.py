@@ -385,6 +385,36 @@ def main_ours(args, rank, world, local_rank):
                          "frac": gbs / peaks["hbm_gbs"], "frac_of_8TBs": gbs / 8000.0,
                          "traffic": None, "algorithmic_bytes_per_launch": nbytes}}
 
+    # ---- speculative verify (4 draft tokens, per-token state snapshots) and the commit of
+    #      the accepted prefix (2 of 4 accepted everywhere), 256 sequences
+    if args.only != "prefill":
+        ntok = 4
+        d = inputs.make_decode(256, ntok, seed=3, device=dev)
+        dout = torch.empty_like(d["v"])
+        snaps = torch.empty((256, ntok, HV, D, D), dtype=torch.float32, device=dev)
+        acc = torch.full((256,), 2, dtype=torch.int32, device=dev)
+
+        def verify_once():
+            gdn.gdn_decode_verify(d["q"], d["k"], d["v"], d["g"], d["beta"], d["state"], dout, snaps,
+                                  stream=stream)
+
+        def commit_once():
+            gdn.gdn_decode_commit(d["state"], snaps, acc, stream=stream)
+
+        for name, fn, nbytes in (
+                ("verify4_snapshots", verify_once,
+                 256 * (STATE_BYTES * (1 + ntok) + ntok * PREFILL_BYTES_PER_TOKEN)),
+                ("commit", commit_once, 256 * STATE_BYTES * 2 + 256 * 4)):
+            dms = timed(fn, max(args.steps, 10), args.warmup)
+            dstep = max_over_ranks(sum(dms) / len(dms))
+            gbs = nbytes / (dstep * 1e-3) / 1e9
+            dec[name] = {
+                "ms_per_step": dstep,
+                "roofline": {"bound": "hbm", "achieved": gbs, "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                             "frac": gbs / peaks["hbm_gbs"], "traffic": None,
+                             "algorithmic_bytes_per_launch": nbytes}}
+        dec["verify4_snapshots"]["tokens_per_s"] = world * 256 * ntok / (dec["verify4_snapshots"]["ms_per_step"] * 1e-3)
+
     # ---- CPU baseline: the oracle on a bounded sample (rank 0, N=1 only)
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline and not args.tokens:

@@ -162,6 +162,35 @@ gdn_status gdn_decode_step(const void *q, const void *k, const void *v,
                            void *stream);
 
 /*
+ * Speculative verify with per-token state snapshots (the multi-token prediction
+ * serving of the pages -- vLLM blog post, "Multi-Token Prediction"; Qwen3-Next model
+ * card, "Deployment" -- checks up to 4 draft tokens per step and keeps only the
+ * accepted ones, so the state must be recoverable after any prefix of the drafts).
+ *
+ * gdn_decode_verify: same inputs and outputs as gdn_decode_step, except that `state`
+ *   is only read, and the state after each token t (t = 0 .. num_tokens-1) is written
+ *   to `snapshots`:
+ *     state       [N][HV][D][D] fp32, read only
+ *     snapshots   [N][num_tokens][HV][D][D] fp32, written; snapshots[n][t] is the state
+ *                 after tokens 0..t of sequence n (must not overlap state, inputs or out)
+ *   The outputs are those gdn_decode_step gives for the same tokens.
+ * gdn_decode_commit: for every sequence n with 1 <= accepted[n] <= num_tokens, copies
+ *   snapshots[n][accepted[n] - 1] into state[n]; a sequence with any other count (0:
+ *   every draft rejected) keeps its state.
+ *     accepted    [N] int32, DEVICE memory (typically written by the sampler on the GPU)
+ *   num_tokens must be the value the snapshots were written with.
+ * Errors as for gdn_decode_step (GDN_ERR_NULL for a missing snapshots or accepted
+ * pointer); the commit reads num_seqs, num_v_heads and head_dim of `shape`.  Bytes moved: verify reads the state once and writes num_tokens states;
+ * commit reads and writes one state per sequence that accepted a draft.
+ */
+gdn_status gdn_decode_verify(const void *q, const void *k, const void *v,
+                             const float *g, const float *beta, const float *state,
+                             void *out, float *snapshots, int32_t num_tokens,
+                             const gdn_shape *shape, void *stream);
+gdn_status gdn_decode_commit(float *state, const float *snapshots, const int32_t *accepted,
+                             int32_t num_tokens, const gdn_shape *shape, void *stream);
+
+/*
  * Reads the device error word of a prefill workspace (synchronises `stream`; meant for
  * tests and debugging).  Returns GDN_ERR_DEVICE_TIMEOUT if a bounded device wait of a
  * previous prefill gave up, GDN_ERR_CUDA if the runtime reports an error, else GDN_OK.

@@ -95,11 +95,15 @@ __device__ __forceinline__ void xpose_reduce(float* a, int l) {
 
 // NTOK tokens of one step; R rows per half-warp per iteration, with 2 * NT * R == 16
 // partial sums per lane (NT = NTOK rounded up to a power of two; a padding slot is 0).
-template <typename IO, int NTOK, int R>
+// SNAP = false: the state after the last token overwrites `state` in place.
+// SNAP = true (speculative verify): `state` is only read; the state after each token t,
+//   s_t = Gam_t s0 + sum_{j<=t} exp(G_t - G_j) delta_j k_j (the same closed form), goes to
+//   snap[n][t][h] ([N][NTOK][HV][D][D] fp32).
+template <typename IO, int NTOK, int R, bool SNAP>
 __global__ void __launch_bounds__(kDecodeThreads, 3)
 decode_kernel(const IO* __restrict__ q, const IO* __restrict__ k, const IO* __restrict__ v,
               const float* __restrict__ g, const float* __restrict__ beta,
-              float* __restrict__ state, IO* __restrict__ out, int hk, int hv)
+              float* __restrict__ state, IO* __restrict__ out, float* __restrict__ snap, int hk, int hv)
 {
     constexpr int NT = NTOK == 3 ? 4 : NTOK;
     constexpr int VR = 2 * NT;           // sums per row: x_0..x_{NT-1}, y_0..y_{NT-1}
@@ -166,17 +170,17 @@ decode_kernel(const IO* __restrict__ q, const IO* __restrict__ k, const IO* __re
             bt[t] = beta[gi];
         }
     }
-    float Dm[NTOK][NTOK], Em[NTOK][NTOK], Gam[NTOK], F[NTOK];
+    float Dm[NTOK][NTOK], Em[NTOK][NTOK], Et[NTOK][NTOK], Gam[NTOK];
 #pragma unroll
     for (int t = 0; t < NTOK; ++t) {
         Gam[t] = expf(G[t]);
-        F[t] = expf(G[NTOK - 1] - G[t]);
 #pragma unroll
         for (int j = 0; j < NTOK; ++j) {
             Dm[t][j] = 0.f;
             Em[t][j] = 0.f;
-            if (j < t) Dm[t][j] = expf(G[t] - G[j]) * sum16(dot8(kr[j], kr[t]));
-            if (j <= t) Em[t][j] = expf(G[t] - G[j]) * sum16(dot8(kr[j], qr[t]));
+            Et[t][j] = (j <= t) ? expf(G[t] - G[j]) : 0.f;  // decay from token j to token t
+            if (j < t) Dm[t][j] = Et[t][j] * sum16(dot8(kr[j], kr[t]));
+            if (j <= t) Em[t][j] = Et[t][j] * sum16(dot8(kr[j], qr[t]));
         }
     }
     __syncthreads();  // v_s
@@ -228,21 +232,42 @@ decode_kernel(const IO* __restrict__ q, const IO* __restrict__ k, const IO* __re
                     for (int j = 0; j <= t; ++j) o = fmaf(Em[t][j], delta[j], o);
                     if (l == 0) o_s[t][row] = o;
                 }
-                float2 w[NTOK];
+                if constexpr (SNAP) {
 #pragma unroll
-                for (int j = 0; j < NTOK; ++j) w[j] = make_float2(F[j] * delta[j], F[j] * delta[j]);
-                const float2 gl = make_float2(Gam[NTOK - 1], Gam[NTOK - 1]);
+                    for (int t = 0; t < NTOK; ++t) {
+                        float2 w[NTOK];
 #pragma unroll
-                for (int c = 0; c < 4; ++c) {
-                    float2 y = __fmul2_rn(gl, s[r][c]);
+                        for (int j = 0; j <= t; ++j) w[j] = make_float2(Et[t][j] * delta[j], Et[t][j] * delta[j]);
+                        const float2 gt = make_float2(Gam[t], Gam[t]);
+                        float2 y[4];
 #pragma unroll
-                    for (int j = 0; j < NTOK; ++j) y = __ffma2_rn(w[j], kr[j][c], y);
-                    s[r][c] = y;
+                        for (int c = 0; c < 4; ++c) {
+                            y[c] = __fmul2_rn(gt, s[r][c]);
+#pragma unroll
+                            for (int j = 0; j <= t; ++j) y[c] = __ffma2_rn(w[j], kr[j][c], y[c]);
+                        }
+                        float* St = snap + (((size_t)n * NTOK + t) * hv + h) * kD * kD + row * kD;
+                        __stcs(reinterpret_cast<float4*>(St + 4 * l), make_float4(y[0].x, y[0].y, y[1].x, y[1].y));
+                        __stcs(reinterpret_cast<float4*>(St + 64 + 4 * l), make_float4(y[2].x, y[2].y, y[3].x, y[3].y));
+                    }
+                } else {
+                    float2 w[NTOK];
+#pragma unroll
+                    for (int j = 0; j < NTOK; ++j)
+                        w[j] = make_float2(Et[NTOK - 1][j] * delta[j], Et[NTOK - 1][j] * delta[j]);
+                    const float2 gl = make_float2(Gam[NTOK - 1], Gam[NTOK - 1]);
+#pragma unroll
+                    for (int c = 0; c < 4; ++c) {
+                        float2 y = __fmul2_rn(gl, s[r][c]);
+#pragma unroll
+                        for (int j = 0; j < NTOK; ++j) y = __ffma2_rn(w[j], kr[j][c], y);
+                        s[r][c] = y;
+                    }
+                    __stcs(reinterpret_cast<float4*>(S + row * kD + 4 * l),
+                           make_float4(s[r][0].x, s[r][0].y, s[r][1].x, s[r][1].y));
+                    __stcs(reinterpret_cast<float4*>(S + row * kD + 64 + 4 * l),
+                           make_float4(s[r][2].x, s[r][2].y, s[r][3].x, s[r][3].y));
                 }
-                __stcs(reinterpret_cast<float4*>(S + row * kD + 4 * l),
-                       make_float4(s[r][0].x, s[r][0].y, s[r][1].x, s[r][1].y));
-                __stcs(reinterpret_cast<float4*>(S + row * kD + 64 + 4 * l),
-                       make_float4(s[r][2].x, s[r][2].y, s[r][3].x, s[r][3].y));
             }
         }
     }
@@ -253,46 +278,77 @@ decode_kernel(const IO* __restrict__ q, const IO* __restrict__ k, const IO* __re
     }
 }
 
-template <typename IO, int NTOK, int R>
+template <typename IO, int NTOK, int R, bool SNAP>
 cudaError_t launch_one(const IO* q, const IO* k, const IO* v, const float* g, const float* beta,
-                       float* state, IO* out, int num_seqs, int hk, int hv, cudaStream_t stream)
+                       float* state, IO* out, float* snap, int num_seqs, int hk, int hv,
+                       cudaStream_t stream)
 {
-    auto kernel = decode_kernel<IO, NTOK, R>;
+    auto kernel = decode_kernel<IO, NTOK, R, SNAP>;
     cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          (int)kStateSmemBytes);
     if (e != cudaSuccess) return e;
     kernel<<<dim3((unsigned)num_seqs * (unsigned)hv), dim3(kDecodeThreads), kStateSmemBytes,
-             stream>>>(q, k, v, g, beta, state, out, hk, hv);
+             stream>>>(q, k, v, g, beta, state, out, snap, hk, hv);
     return cudaGetLastError();
 }
 
-template <typename IO>
+template <typename IO, bool SNAP>
 cudaError_t launch_typed(const IO* q, const IO* k, const IO* v, const float* g,
-                         const float* beta, float* state, IO* out, int ntok, int num_seqs,
-                         int hk, int hv, cudaStream_t stream)
+                         const float* beta, float* state, IO* out, float* snap, int ntok,
+                         int num_seqs, int hk, int hv, cudaStream_t stream)
 {
     switch (ntok) {
-    case 1: return launch_one<IO, 1, 8>(q, k, v, g, beta, state, out, num_seqs, hk, hv, stream);
-    case 2: return launch_one<IO, 2, 4>(q, k, v, g, beta, state, out, num_seqs, hk, hv, stream);
-    case 3: return launch_one<IO, 3, 2>(q, k, v, g, beta, state, out, num_seqs, hk, hv, stream);
-    default: return launch_one<IO, 4, 2>(q, k, v, g, beta, state, out, num_seqs, hk, hv, stream);
+    case 1: return launch_one<IO, 1, 8, SNAP>(q, k, v, g, beta, state, out, snap, num_seqs, hk, hv, stream);
+    case 2: return launch_one<IO, 2, 4, SNAP>(q, k, v, g, beta, state, out, snap, num_seqs, hk, hv, stream);
+    case 3: return launch_one<IO, 3, 2, SNAP>(q, k, v, g, beta, state, out, snap, num_seqs, hk, hv, stream);
+    default: return launch_one<IO, 4, 2, SNAP>(q, k, v, g, beta, state, out, snap, num_seqs, hk, hv, stream);
     }
+}
+
+// Commit of a verify step: state[n][h] <- snap[n][accepted[n] - 1][h] for accepted[n] in
+// 1..ntok; any other count leaves the state as it was.  One CTA per (n, h), 64 KiB each.
+__global__ void __launch_bounds__(kDecodeThreads)
+commit_kernel(float* __restrict__ state, const float* __restrict__ snap,
+              const int32_t* __restrict__ accepted, int ntok, int hv)
+{
+    const int n = blockIdx.x / hv, h = blockIdx.x % hv;
+    const int acc = accepted[n];
+    if (acc < 1 || acc > ntok) return;
+    const float4* src = reinterpret_cast<const float4*>(snap + (((size_t)n * ntok + acc - 1) * hv + h) * kD * kD);
+    float4* dst = reinterpret_cast<float4*>(state + ((size_t)n * hv + h) * kD * kD);
+#pragma unroll 4
+    for (int i = threadIdx.x; i < kD * kD / 4; i += kDecodeThreads) __stcs(dst + i, __ldcs(src + i));
 }
 
 }  // namespace
 
 cudaError_t launch_decode(const void* q, const void* k, const void* v, const float* g,
-                          const float* beta, float* state, void* out, int num_tokens,
+                          const float* beta, float* state, void* out, float* snap, int num_tokens,
                           int num_seqs, int hk, int hv, gdn_dtype io, cudaStream_t stream)
 {
     if (num_seqs == 0) return cudaSuccess;
     if (io == GDN_BF16) {
         using T = __nv_bfloat16;
-        return launch_typed<T>((const T*)q, (const T*)k, (const T*)v, g, beta, state, (T*)out,
-                               num_tokens, num_seqs, hk, hv, stream);
+        if (snap)
+            return launch_typed<T, true>((const T*)q, (const T*)k, (const T*)v, g, beta, state, (T*)out, snap,
+                                         num_tokens, num_seqs, hk, hv, stream);
+        return launch_typed<T, false>((const T*)q, (const T*)k, (const T*)v, g, beta, state, (T*)out, nullptr,
+                                      num_tokens, num_seqs, hk, hv, stream);
     }
-    return launch_typed<float>((const float*)q, (const float*)k, (const float*)v, g, beta, state,
-                               (float*)out, num_tokens, num_seqs, hk, hv, stream);
+    if (snap)
+        return launch_typed<float, true>((const float*)q, (const float*)k, (const float*)v, g, beta, state,
+                                         (float*)out, snap, num_tokens, num_seqs, hk, hv, stream);
+    return launch_typed<float, false>((const float*)q, (const float*)k, (const float*)v, g, beta, state,
+                                      (float*)out, nullptr, num_tokens, num_seqs, hk, hv, stream);
+}
+
+cudaError_t launch_decode_commit(float* state, const float* snap, const int32_t* accepted, int num_tokens,
+                                 int num_seqs, int hv, cudaStream_t stream)
+{
+    if (num_seqs == 0) return cudaSuccess;
+    commit_kernel<<<dim3((unsigned)num_seqs * (unsigned)hv), dim3(kDecodeThreads), 0, stream>>>(
+        state, snap, accepted, num_tokens, hv);
+    return cudaGetLastError();
 }
 
 }  // namespace gdn

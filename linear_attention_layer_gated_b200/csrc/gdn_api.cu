@@ -170,10 +170,45 @@ gdn_status gdn_decode_step(const void* q, const void* k, const void* v, const fl
     const void* ptrs[] = {q, k, v, g, beta, state_inout, out};
     for (const void* p : ptrs)
         if (!aligned16(p)) return GDN_ERR_ALIGN;
-    cudaError_t e = gdn::launch_decode(q, k, v, g, beta, state_inout, out, num_tokens,
+    cudaError_t e = gdn::launch_decode(q, k, v, g, beta, state_inout, out, nullptr, num_tokens,
                                        shape->num_seqs, shape->num_qk_heads, shape->num_v_heads,
                                        (gdn_dtype)shape->io_dtype,
                                        reinterpret_cast<cudaStream_t>(stream));
+    return e == cudaSuccess ? GDN_OK : GDN_ERR_CUDA;
+}
+
+gdn_status gdn_decode_verify(const void* q, const void* k, const void* v, const float* g,
+                             const float* beta, const float* state, void* out, float* snapshots,
+                             int32_t num_tokens, const gdn_shape* shape, void* stream) {
+    gdn_status st = check_common(shape);
+    if (st != GDN_OK) return st;
+    if (num_tokens < 1 || num_tokens > 4) return GDN_ERR_NUM_TOKENS;
+    if ((int64_t)shape->num_seqs * shape->num_v_heads * num_tokens > INT32_MAX) return GDN_ERR_SHAPE;
+    if (shape->num_seqs == 0) return GDN_OK;
+    if (!q || !k || !v || !g || !beta || !state || !out || !snapshots) return GDN_ERR_NULL;
+    const void* ptrs[] = {q, k, v, g, beta, state, out, snapshots};
+    for (const void* p : ptrs)
+        if (!aligned16(p)) return GDN_ERR_ALIGN;
+    cudaError_t e = gdn::launch_decode(q, k, v, g, beta, const_cast<float*>(state), out, snapshots,
+                                       num_tokens, shape->num_seqs, shape->num_qk_heads,
+                                       shape->num_v_heads, (gdn_dtype)shape->io_dtype,
+                                       reinterpret_cast<cudaStream_t>(stream));
+    return e == cudaSuccess ? GDN_OK : GDN_ERR_CUDA;
+}
+
+gdn_status gdn_decode_commit(float* state, const float* snapshots, const int32_t* accepted,
+                             int32_t num_tokens, const gdn_shape* shape, void* stream) {
+    gdn_status st = check_common(shape);
+    if (st != GDN_OK) return st;
+    if (num_tokens < 1 || num_tokens > 4) return GDN_ERR_NUM_TOKENS;
+    if ((int64_t)shape->num_seqs * shape->num_v_heads > INT32_MAX) return GDN_ERR_SHAPE;
+    if (shape->num_seqs == 0) return GDN_OK;
+    if (!state || !snapshots || !accepted) return GDN_ERR_NULL;
+    const void* ptrs[] = {state, snapshots, accepted};
+    for (const void* p : ptrs)
+        if (!aligned16(p)) return GDN_ERR_ALIGN;
+    cudaError_t e = gdn::launch_decode_commit(state, snapshots, accepted, num_tokens, shape->num_seqs,
+                                              shape->num_v_heads, reinterpret_cast<cudaStream_t>(stream));
     return e == cudaSuccess ? GDN_OK : GDN_ERR_CUDA;
 }
 

@@ -46,9 +46,13 @@ __device__ __forceinline__ void store4(__nv_bfloat16* p, float4 v) {
 
 // ---------------------------------------------------------------- launchers
 // Each returns cudaSuccess or the launch error; arguments were validated by the caller.
+// snap == nullptr: decode step in place; otherwise verify (state read only, per-token
+// states to snap).
 cudaError_t launch_decode(const void* q, const void* k, const void* v, const float* g,
-                          const float* beta, float* state, void* out, int num_tokens,
+                          const float* beta, float* state, void* out, float* snap, int num_tokens,
                           int num_seqs, int hk, int hv, gdn_dtype io, cudaStream_t stream);
+cudaError_t launch_decode_commit(float* state, const float* snap, const int32_t* accepted, int num_tokens,
+                                 int num_seqs, int hv, cudaStream_t stream);
 
 cudaError_t launch_prefill_simt(const void* q, const void* k, const void* v, const float* g,
                                 const float* beta, const float* s0, const int32_t* cu,

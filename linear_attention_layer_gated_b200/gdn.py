@@ -25,7 +25,7 @@ STATUS = {0: "GDN_OK", 1: "GDN_ERR_NULL", 2: "GDN_ERR_SHAPE", 3: "GDN_ERR_ALIGN"
 EXPORTED = ["gdn_prefill_workspace_bytes", "gdn_chunk_prefill", "gdn_chunk_prefill_prep",
             "gdn_chunk_prefill_state", "gdn_decode_step", "gdn_get_device_error",
             "gdn_selftest_wait_timeout", "gdn_status_string", "gdn_abi_version",
-            "gdn_chunk_prefill_noalloc"]
+            "gdn_chunk_prefill_noalloc", "gdn_decode_verify", "gdn_decode_commit"]
 
 
 class GdnShape(ctypes.Structure):
@@ -67,6 +67,10 @@ def lib() -> ctypes.CDLL:
             L.gdn_chunk_prefill_state.argtypes = [fp, ip, vp, fp, sp, vp, ctypes.c_size_t, vp]
             L.gdn_decode_step.restype = ctypes.c_int
             L.gdn_decode_step.argtypes = [vp, vp, vp, fp, fp, fp, vp, ctypes.c_int32, sp, vp]
+            L.gdn_decode_verify.restype = ctypes.c_int
+            L.gdn_decode_verify.argtypes = [vp, vp, vp, fp, fp, fp, vp, fp, ctypes.c_int32, sp, vp]
+            L.gdn_decode_commit.restype = ctypes.c_int
+            L.gdn_decode_commit.argtypes = [fp, fp, ip, ctypes.c_int32, sp, vp]
             L.gdn_get_device_error.restype = ctypes.c_int
             L.gdn_get_device_error.argtypes = [vp, vp]
             L.gdn_chunk_prefill_noalloc.restype = ctypes.c_int
@@ -195,6 +199,32 @@ def gdn_decode_step(q, k, v, g, beta, state_inout, out, num_tokens=None, stream=
         raise GdnError(rc, "gdn_decode_step")
 
 
+def gdn_decode_verify(q, k, v, g, beta, state, out, snapshots, num_tokens=None, stream=None):
+    """Calls gdn_decode_verify.  Shapes as gdn_decode_step; state [N, HV, 128, 128] fp32 is
+    only read; snapshots [N, m, HV, 128, 128] fp32 receives the state after each token."""
+    N, m, HK, D = q.shape
+    if num_tokens is None:
+        num_tokens = m
+    shape = make_shape(N, N * m, HK, v.shape[2], D, _io_dtype(q))
+    rc = lib().gdn_decode_verify(_ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(beta), _ptr(state), _ptr(out),
+                                 _ptr(snapshots), int(num_tokens), ctypes.byref(shape), _stream(stream))
+    if rc != GDN_OK:
+        raise GdnError(rc, "gdn_decode_verify")
+
+
+def gdn_decode_commit(state, snapshots, accepted, num_tokens=None, stream=None):
+    """Calls gdn_decode_commit: state[n] <- snapshots[n, accepted[n] - 1] where
+    1 <= accepted[n] <= num_tokens (accepted: [N] int32 on the device)."""
+    N, m, HV, D, _ = snapshots.shape
+    if num_tokens is None:
+        num_tokens = m
+    shape = make_shape(N, N * m, 1, HV, D, GDN_BF16)  # the commit reads num_seqs, num_v_heads, head_dim
+    rc = lib().gdn_decode_commit(_ptr(state), _ptr(snapshots), _ptr(accepted), int(num_tokens),
+                                 ctypes.byref(shape), _stream(stream))
+    if rc != GDN_OK:
+        raise GdnError(rc, "gdn_decode_commit")
+
+
 def gdn_chunk_prefill_noalloc(q, k, v, g, beta, initial_state, cu_seqlens, out, final_state,
                               stream=None):
     """Calls gdn_chunk_prefill_noalloc: the tensor-core prefill with the library's own
@@ -239,3 +269,14 @@ def decode(q, k, v, g, beta, state_inout, stream=None):
     out = torch.empty_like(v)
     gdn_decode_step(q, k, v, g, beta, state_inout, out, stream=stream)
     return out
+
+
+def verify(q, k, v, g, beta, state, stream=None):
+    """Allocates out and the snapshots and runs gdn_decode_verify (state is not changed).
+    Returns (out, snapshots)."""
+    N, m = q.shape[:2]
+    HV, D = v.shape[2], v.shape[3]
+    out = torch.empty_like(v)
+    snaps = torch.empty((N, m, HV, D, D), dtype=torch.float32, device=v.device)
+    gdn_decode_verify(q, k, v, g, beta, state, out, snaps, stream=stream)
+    return out, snaps

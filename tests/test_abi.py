@@ -132,3 +132,22 @@ def test_selftest_rejects_bad_arguments(L):
     assert gdn.STATUS[L.gdn_selftest_wait_timeout(FAKE, 16, 1000, None)] == "GDN_ERR_WORKSPACE"
     assert gdn.STATUS[L.gdn_selftest_wait_timeout(FAKE + 16, 256, 1000, None)] == "GDN_ERR_ALIGN"
     assert gdn.STATUS[L.gdn_selftest_wait_timeout(FAKE, 256, 0, None)] == "GDN_ERR_SHAPE"
+
+
+def test_verify_and_commit_reject_bad_arguments(L):
+    s = shape(num_seqs=4)
+    verify = lambda ntok=2, **kw: L.gdn_decode_verify(  # noqa: E731
+        kw.get("q", FAKE), FAKE, FAKE, FAKE, FAKE, kw.get("st", FAKE), FAKE, kw.get("snap", FAKE), ntok,
+        ctypes.byref(s), None)
+    assert gdn.STATUS[verify(ntok=0)] == "GDN_ERR_NUM_TOKENS"
+    assert gdn.STATUS[verify(ntok=5)] == "GDN_ERR_NUM_TOKENS"
+    assert gdn.STATUS[verify(snap=None)] == "GDN_ERR_NULL"
+    assert gdn.STATUS[verify(st=None)] == "GDN_ERR_NULL"
+    assert gdn.STATUS[verify(snap=FAKE + 4)] == "GDN_ERR_ALIGN"
+    commit = lambda ntok=2, **kw: L.gdn_decode_commit(  # noqa: E731
+        kw.get("st", FAKE), kw.get("snap", FAKE), kw.get("acc", FAKE), ntok, ctypes.byref(s), None)
+    assert gdn.STATUS[commit(ntok=7)] == "GDN_ERR_NUM_TOKENS"
+    assert gdn.STATUS[commit(acc=None)] == "GDN_ERR_NULL"
+    assert gdn.STATUS[commit(acc=FAKE + 4)] == "GDN_ERR_ALIGN"
+    empty = shape(num_seqs=0)
+    assert L.gdn_decode_commit(None, None, None, 2, ctypes.byref(empty), None) == 0

@@ -99,6 +99,39 @@ def test_decode_four_tokens_equals_four_single_steps_and_prefill():
     assert_close(sp, s4.double().cpu().numpy(), 1e-5, "decode vs prefill state")
 
 
+# ------------------------------------------------------------------ speculative verify
+@pytest.mark.parametrize("ntok", [1, 2, 3, 4])
+def test_verify_snapshots_match_oracle_and_keep_state(ntok):
+    x = inputs.make_decode(32, ntok, hk=4, hv=8, seed=40 + ntok, device="cuda")
+    st = x["state"].clone()
+    out_v, snaps = gdn.verify(x["q"], x["k"], x["v"], x["g"], x["beta"], st)
+    torch.cuda.synchronize()
+    torch.testing.assert_close(st, x["state"], rtol=0, atol=0)  # verify leaves the state alone
+    st_d = x["state"].clone()
+    out_d = gdn.decode(x["q"], x["k"], x["v"], x["g"], x["beta"], st_d)
+    torch.testing.assert_close(out_v, out_d, rtol=0, atol=0)            # same outputs as decode
+    torch.testing.assert_close(snaps[:, ntok - 1], st_d, rtol=0, atol=0)  # last snapshot = decode state
+    for t in range(ntok):  # snapshot t = the oracle's state after tokens 0..t
+        sl = lambda a: a[:, : t + 1].contiguous()  # noqa: E731
+        _, s_ref = oracle.decode(sl(x["q"]), sl(x["k"]), sl(x["v"]), sl(x["g"]), sl(x["beta"]), x["state"])
+        assert_close(snaps[:, t], s_ref, TOL_BF16, "verify snapshot %d of %d" % (t, ntok))
+
+
+def test_commit_installs_the_accepted_snapshot():
+    ntok = 4
+    x = inputs.make_decode(40, ntok, hk=4, hv=8, seed=45, device="cuda")
+    st = x["state"].clone()
+    _, snaps = gdn.verify(x["q"], x["k"], x["v"], x["g"], x["beta"], st)
+    accepted = torch.tensor([i % (ntok + 2) - (1 if i % 7 == 0 else 0) for i in range(40)],
+                            dtype=torch.int32, device="cuda")  # 0..ntok, plus -1 and ntok+1
+    gdn.gdn_decode_commit(st, snaps, accepted)
+    torch.cuda.synchronize()
+    for n in range(40):
+        a = int(accepted[n])
+        want = snaps[n, a - 1] if 1 <= a <= ntok else x["state"][n]
+        torch.testing.assert_close(st[n], want, rtol=0, atol=0)
+
+
 # ------------------------------------------------------------------ prefill, small
 def test_prefill_tiny_fp32_matches_oracle():
     x = inputs.make(inputs.workload("tiny"), device="cuda")
