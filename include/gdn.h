@@ -191,6 +191,41 @@ gdn_status gdn_decode_commit(float *state, const float *snapshots, const int32_t
                              int32_t num_tokens, const gdn_shape *shape, void *stream);
 
 /*
+ * State-slot indirection (the pages' hybrid cache manager keeps the linear-attention
+ * states of running requests in one preallocated pool -- vLLM blog post, "Hybrid KV
+ * Cache Management"): the same prefill, decode, verify and commit on states held in
+ *     state_pool    [num_slots][HV][D][D] fp32
+ * where sequence n's state is state_pool[state_slots[n]].
+ *     state_slots   [N] int32, DEVICE memory.  A slot outside [0, num_slots) marks a
+ *                   sequence without a state: decode and verify skip it (its outputs and
+ *                   snapshots are not written) and commit leaves the pool unchanged for it;
+ *                   prefill runs it from a zero state and writes no final state.
+ * gdn_chunk_prefill_slots reads each sequence's initial state from its slot and writes
+ * the final state back to the same slot (in place); otherwise the arguments are those of
+ * gdn_chunk_prefill.  Two sequences of one call must not share a valid slot.
+ * GDN_ERR_NULL for a missing pool or slot table, GDN_ERR_SHAPE for num_slots < 0; the
+ * rest as for the dense entry points.
+ */
+gdn_status gdn_chunk_prefill_slots(const void *q, const void *k, const void *v,
+                                   const float *g, const float *beta, float *state_pool,
+                                   const int32_t *state_slots, int32_t num_slots,
+                                   const int32_t *cu_seqlens, void *out, const gdn_shape *shape,
+                                   void *workspace, size_t workspace_bytes, void *stream);
+gdn_status gdn_decode_step_slots(const void *q, const void *k, const void *v,
+                                 const float *g, const float *beta, float *state_pool,
+                                 const int32_t *state_slots, int32_t num_slots, void *out,
+                                 int32_t num_tokens, const gdn_shape *shape, void *stream);
+gdn_status gdn_decode_verify_slots(const void *q, const void *k, const void *v,
+                                   const float *g, const float *beta, const float *state_pool,
+                                   const int32_t *state_slots, int32_t num_slots, void *out,
+                                   float *snapshots, int32_t num_tokens, const gdn_shape *shape,
+                                   void *stream);
+gdn_status gdn_decode_commit_slots(float *state_pool, const int32_t *state_slots,
+                                   int32_t num_slots, const float *snapshots,
+                                   const int32_t *accepted, int32_t num_tokens,
+                                   const gdn_shape *shape, void *stream);
+
+/*
  * Reads the device error word of a prefill workspace (synchronises `stream`; meant for
  * tests and debugging).  Returns GDN_ERR_DEVICE_TIMEOUT if a bounded device wait of a
  * previous prefill gave up, GDN_ERR_CUDA if the runtime reports an error, else GDN_OK.

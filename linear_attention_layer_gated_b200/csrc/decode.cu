@@ -103,7 +103,8 @@ template <typename IO, int NTOK, int R, bool SNAP>
 __global__ void __launch_bounds__(kDecodeThreads, 3)
 decode_kernel(const IO* __restrict__ q, const IO* __restrict__ k, const IO* __restrict__ v,
               const float* __restrict__ g, const float* __restrict__ beta,
-              float* __restrict__ state, IO* __restrict__ out, float* __restrict__ snap, int hk, int hv)
+              float* __restrict__ state, StateSlots map, IO* __restrict__ out, float* __restrict__ snap,
+              int hk, int hv)
 {
     constexpr int NT = NTOK == 3 ? 4 : NTOK;
     constexpr int VR = 2 * NT;           // sums per row: x_0..x_{NT-1}, y_0..y_{NT-1}
@@ -127,7 +128,10 @@ decode_kernel(const IO* __restrict__ q, const IO* __restrict__ k, const IO* __re
     __shared__ float o_s[NTOK][kD];
     __shared__ __align__(16) float red_s[2][4][2][16];  // [parity][warp][half][sum]
 
-    float* S = state + ((size_t)n * hv + h) * kD * kD;
+    bool has_state;
+    const int sidx = state_index(map, n, has_state);
+    if (!has_state) return;  // a sequence without a state slot is skipped (whole CTA)
+    float* S = state + ((size_t)sidx * hv + h) * kD * kD;
 
     // 1. This warp's 32 rows start moving HBM -> shared memory immediately.
 #pragma unroll
@@ -280,7 +284,7 @@ decode_kernel(const IO* __restrict__ q, const IO* __restrict__ k, const IO* __re
 
 template <typename IO, int NTOK, int R, bool SNAP>
 cudaError_t launch_one(const IO* q, const IO* k, const IO* v, const float* g, const float* beta,
-                       float* state, IO* out, float* snap, int num_seqs, int hk, int hv,
+                       float* state, StateSlots map, IO* out, float* snap, int num_seqs, int hk, int hv,
                        cudaStream_t stream)
 {
     auto kernel = decode_kernel<IO, NTOK, R, SNAP>;
@@ -288,34 +292,36 @@ cudaError_t launch_one(const IO* q, const IO* k, const IO* v, const float* g, co
                                          (int)kStateSmemBytes);
     if (e != cudaSuccess) return e;
     kernel<<<dim3((unsigned)num_seqs * (unsigned)hv), dim3(kDecodeThreads), kStateSmemBytes,
-             stream>>>(q, k, v, g, beta, state, out, snap, hk, hv);
+             stream>>>(q, k, v, g, beta, state, map, out, snap, hk, hv);
     return cudaGetLastError();
 }
 
 template <typename IO, bool SNAP>
 cudaError_t launch_typed(const IO* q, const IO* k, const IO* v, const float* g,
-                         const float* beta, float* state, IO* out, float* snap, int ntok,
+                         const float* beta, float* state, StateSlots map, IO* out, float* snap, int ntok,
                          int num_seqs, int hk, int hv, cudaStream_t stream)
 {
     switch (ntok) {
-    case 1: return launch_one<IO, 1, 8, SNAP>(q, k, v, g, beta, state, out, snap, num_seqs, hk, hv, stream);
-    case 2: return launch_one<IO, 2, 4, SNAP>(q, k, v, g, beta, state, out, snap, num_seqs, hk, hv, stream);
-    case 3: return launch_one<IO, 3, 2, SNAP>(q, k, v, g, beta, state, out, snap, num_seqs, hk, hv, stream);
-    default: return launch_one<IO, 4, 2, SNAP>(q, k, v, g, beta, state, out, snap, num_seqs, hk, hv, stream);
+    case 1: return launch_one<IO, 1, 8, SNAP>(q, k, v, g, beta, state, map, out, snap, num_seqs, hk, hv, stream);
+    case 2: return launch_one<IO, 2, 4, SNAP>(q, k, v, g, beta, state, map, out, snap, num_seqs, hk, hv, stream);
+    case 3: return launch_one<IO, 3, 2, SNAP>(q, k, v, g, beta, state, map, out, snap, num_seqs, hk, hv, stream);
+    default: return launch_one<IO, 4, 2, SNAP>(q, k, v, g, beta, state, map, out, snap, num_seqs, hk, hv, stream);
     }
 }
 
 // Commit of a verify step: state[n][h] <- snap[n][accepted[n] - 1][h] for accepted[n] in
 // 1..ntok; any other count leaves the state as it was.  One CTA per (n, h), 64 KiB each.
 __global__ void __launch_bounds__(kDecodeThreads)
-commit_kernel(float* __restrict__ state, const float* __restrict__ snap,
+commit_kernel(float* __restrict__ state, StateSlots map, const float* __restrict__ snap,
               const int32_t* __restrict__ accepted, int ntok, int hv)
 {
     const int n = blockIdx.x / hv, h = blockIdx.x % hv;
     const int acc = accepted[n];
-    if (acc < 1 || acc > ntok) return;
+    bool has_state;
+    const int sidx = state_index(map, n, has_state);
+    if (acc < 1 || acc > ntok || !has_state) return;
     const float4* src = reinterpret_cast<const float4*>(snap + (((size_t)n * ntok + acc - 1) * hv + h) * kD * kD);
-    float4* dst = reinterpret_cast<float4*>(state + ((size_t)n * hv + h) * kD * kD);
+    float4* dst = reinterpret_cast<float4*>(state + ((size_t)sidx * hv + h) * kD * kD);
 #pragma unroll 4
     for (int i = threadIdx.x; i < kD * kD / 4; i += kDecodeThreads) __stcs(dst + i, __ldcs(src + i));
 }
@@ -323,31 +329,31 @@ commit_kernel(float* __restrict__ state, const float* __restrict__ snap,
 }  // namespace
 
 cudaError_t launch_decode(const void* q, const void* k, const void* v, const float* g,
-                          const float* beta, float* state, void* out, float* snap, int num_tokens,
-                          int num_seqs, int hk, int hv, gdn_dtype io, cudaStream_t stream)
+                          const float* beta, float* state, StateSlots map, void* out, float* snap,
+                          int num_tokens, int num_seqs, int hk, int hv, gdn_dtype io, cudaStream_t stream)
 {
     if (num_seqs == 0) return cudaSuccess;
     if (io == GDN_BF16) {
         using T = __nv_bfloat16;
         if (snap)
-            return launch_typed<T, true>((const T*)q, (const T*)k, (const T*)v, g, beta, state, (T*)out, snap,
+            return launch_typed<T, true>((const T*)q, (const T*)k, (const T*)v, g, beta, state, map, (T*)out, snap,
                                          num_tokens, num_seqs, hk, hv, stream);
-        return launch_typed<T, false>((const T*)q, (const T*)k, (const T*)v, g, beta, state, (T*)out, nullptr,
+        return launch_typed<T, false>((const T*)q, (const T*)k, (const T*)v, g, beta, state, map, (T*)out, nullptr,
                                       num_tokens, num_seqs, hk, hv, stream);
     }
     if (snap)
         return launch_typed<float, true>((const float*)q, (const float*)k, (const float*)v, g, beta, state,
-                                         (float*)out, snap, num_tokens, num_seqs, hk, hv, stream);
+                                         map, (float*)out, snap, num_tokens, num_seqs, hk, hv, stream);
     return launch_typed<float, false>((const float*)q, (const float*)k, (const float*)v, g, beta, state,
-                                      (float*)out, nullptr, num_tokens, num_seqs, hk, hv, stream);
+                                      map, (float*)out, nullptr, num_tokens, num_seqs, hk, hv, stream);
 }
 
-cudaError_t launch_decode_commit(float* state, const float* snap, const int32_t* accepted, int num_tokens,
-                                 int num_seqs, int hv, cudaStream_t stream)
+cudaError_t launch_decode_commit(float* state, StateSlots map, const float* snap, const int32_t* accepted,
+                                 int num_tokens, int num_seqs, int hv, cudaStream_t stream)
 {
     if (num_seqs == 0) return cudaSuccess;
     commit_kernel<<<dim3((unsigned)num_seqs * (unsigned)hv), dim3(kDecodeThreads), 0, stream>>>(
-        state, snap, accepted, num_tokens, hv);
+        state, map, snap, accepted, num_tokens, hv);
     return cudaGetLastError();
 }
 

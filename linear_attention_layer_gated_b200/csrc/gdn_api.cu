@@ -71,11 +71,14 @@ size_t gdn_prefill_workspace_bytes(const gdn_shape* shape) {
     return kHeaderBytes;
 }
 
-gdn_status gdn_chunk_prefill(const void* q, const void* k, const void* v, const float* g,
-                             const float* beta, const float* initial_state,
-                             const int32_t* cu_seqlens, void* out, float* final_state,
-                             const gdn_shape* shape, void* workspace, size_t workspace_bytes,
-                             void* stream) {
+}  // extern "C"
+
+namespace {
+
+gdn_status prefill_impl(const void* q, const void* k, const void* v, const float* g, const float* beta,
+                        const float* initial_state, const int32_t* cu_seqlens, void* out, float* final_state,
+                        gdn::StateSlots map, const gdn_shape* shape, void* workspace, size_t workspace_bytes,
+                        void* stream) {
     gdn_status st = check_prefill_shape(shape);
     if (st != GDN_OK) return st;
     const size_t need = gdn_prefill_workspace_bytes(shape);
@@ -99,14 +102,81 @@ gdn_status gdn_chunk_prefill(const void* q, const void* k, const void* v, const 
                                         shape->total_tokens, shape->num_qk_heads,
                                         shape->num_v_heads, workspace, s);
         if (e == cudaSuccess)
-            e = gdn::launch_prefill_tc_state(initial_state, cu_seqlens, out, final_state,
+            e = gdn::launch_prefill_tc_state(initial_state, cu_seqlens, out, final_state, map,
                                              shape->num_seqs, shape->total_tokens,
                                              shape->num_qk_heads, shape->num_v_heads, workspace, s);
     } else
         e = gdn::launch_prefill_simt(q, k, v, g, beta, initial_state, cu_seqlens, out,
-                                     final_state, shape->num_seqs, shape->num_qk_heads,
+                                     final_state, map, shape->num_seqs, shape->num_qk_heads,
                                      shape->num_v_heads, io, s);
     return e == cudaSuccess ? GDN_OK : GDN_ERR_CUDA;
+}
+
+gdn_status decode_impl(const void* q, const void* k, const void* v, const float* g, const float* beta,
+                       float* state, gdn::StateSlots map, void* out, float* snapshots, int32_t num_tokens,
+                       const gdn_shape* shape, void* stream) {
+    gdn_status st = check_common(shape);
+    if (st != GDN_OK) return st;
+    if (num_tokens < 1 || num_tokens > 4) return GDN_ERR_NUM_TOKENS;
+    if ((int64_t)shape->num_seqs * shape->num_v_heads * num_tokens > INT32_MAX) return GDN_ERR_SHAPE;
+    if (shape->num_seqs == 0) return GDN_OK;
+    if (!q || !k || !v || !g || !beta || !state || !out) return GDN_ERR_NULL;
+    const void* ptrs[] = {q, k, v, g, beta, state, out, snapshots, map.slots};
+    for (const void* p : ptrs)
+        if (p && !aligned16(p)) return GDN_ERR_ALIGN;
+    cudaError_t e = gdn::launch_decode(q, k, v, g, beta, state, map, out, snapshots, num_tokens,
+                                       shape->num_seqs, shape->num_qk_heads, shape->num_v_heads,
+                                       (gdn_dtype)shape->io_dtype, reinterpret_cast<cudaStream_t>(stream));
+    return e == cudaSuccess ? GDN_OK : GDN_ERR_CUDA;
+}
+
+gdn_status commit_impl(float* state, gdn::StateSlots map, const float* snapshots, const int32_t* accepted,
+                       int32_t num_tokens, const gdn_shape* shape, void* stream) {
+    gdn_status st = check_common(shape);
+    if (st != GDN_OK) return st;
+    if (num_tokens < 1 || num_tokens > 4) return GDN_ERR_NUM_TOKENS;
+    if ((int64_t)shape->num_seqs * shape->num_v_heads > INT32_MAX) return GDN_ERR_SHAPE;
+    if (shape->num_seqs == 0) return GDN_OK;
+    if (!state || !snapshots || !accepted) return GDN_ERR_NULL;
+    const void* ptrs[] = {state, snapshots, accepted, map.slots};
+    for (const void* p : ptrs)
+        if (p && !aligned16(p)) return GDN_ERR_ALIGN;
+    cudaError_t e = gdn::launch_decode_commit(state, map, snapshots, accepted, num_tokens, shape->num_seqs,
+                                              shape->num_v_heads, reinterpret_cast<cudaStream_t>(stream));
+    return e == cudaSuccess ? GDN_OK : GDN_ERR_CUDA;
+}
+
+constexpr gdn::StateSlots kDense{nullptr, 0};
+
+gdn_status check_slots(const float* pool, const int32_t* slots, int32_t num_slots) {
+    if (!pool || !slots) return GDN_ERR_NULL;
+    if (num_slots < 0) return GDN_ERR_SHAPE;
+    return GDN_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+gdn_status gdn_chunk_prefill(const void* q, const void* k, const void* v, const float* g,
+                             const float* beta, const float* initial_state,
+                             const int32_t* cu_seqlens, void* out, float* final_state,
+                             const gdn_shape* shape, void* workspace, size_t workspace_bytes,
+                             void* stream) {
+    return prefill_impl(q, k, v, g, beta, initial_state, cu_seqlens, out, final_state, kDense, shape,
+                        workspace, workspace_bytes, stream);
+}
+
+gdn_status gdn_chunk_prefill_slots(const void* q, const void* k, const void* v, const float* g,
+                                   const float* beta, float* state_pool, const int32_t* state_slots,
+                                   int32_t num_slots, const int32_t* cu_seqlens, void* out,
+                                   const gdn_shape* shape, void* workspace, size_t workspace_bytes,
+                                   void* stream) {
+    if (shape && shape->num_seqs == 0) return check_prefill_shape(shape);
+    gdn_status st = check_slots(state_pool, state_slots, num_slots);
+    if (st != GDN_OK) return st;
+    return prefill_impl(q, k, v, g, beta, state_pool, cu_seqlens, out, state_pool,
+                        gdn::StateSlots{state_slots, num_slots}, shape, workspace, workspace_bytes, stream);
 }
 
 // Shared validation of the two tensor-core prefill phases.
@@ -151,7 +221,7 @@ gdn_status gdn_chunk_prefill_state(const float* initial_state, const int32_t* cu
     const void* ptrs[] = {initial_state, out, final_state};
     for (const void* p : ptrs)
         if (p && !aligned16(p)) return GDN_ERR_ALIGN;
-    cudaError_t e = gdn::launch_prefill_tc_state(initial_state, cu_seqlens, out, final_state,
+    cudaError_t e = gdn::launch_prefill_tc_state(initial_state, cu_seqlens, out, final_state, kDense,
                                                  shape->num_seqs, shape->total_tokens,
                                                  shape->num_qk_heads, shape->num_v_heads,
                                                  workspace, reinterpret_cast<cudaStream_t>(stream));
@@ -161,55 +231,56 @@ gdn_status gdn_chunk_prefill_state(const float* initial_state, const int32_t* cu
 gdn_status gdn_decode_step(const void* q, const void* k, const void* v, const float* g,
                            const float* beta, float* state_inout, void* out, int32_t num_tokens,
                            const gdn_shape* shape, void* stream) {
-    gdn_status st = check_common(shape);
-    if (st != GDN_OK) return st;
-    if (num_tokens < 1 || num_tokens > 4) return GDN_ERR_NUM_TOKENS;
-    if ((int64_t)shape->num_seqs * shape->num_v_heads > INT32_MAX) return GDN_ERR_SHAPE;
-    if (shape->num_seqs == 0) return GDN_OK;
-    if (!q || !k || !v || !g || !beta || !state_inout || !out) return GDN_ERR_NULL;
-    const void* ptrs[] = {q, k, v, g, beta, state_inout, out};
-    for (const void* p : ptrs)
-        if (!aligned16(p)) return GDN_ERR_ALIGN;
-    cudaError_t e = gdn::launch_decode(q, k, v, g, beta, state_inout, out, nullptr, num_tokens,
-                                       shape->num_seqs, shape->num_qk_heads, shape->num_v_heads,
-                                       (gdn_dtype)shape->io_dtype,
-                                       reinterpret_cast<cudaStream_t>(stream));
-    return e == cudaSuccess ? GDN_OK : GDN_ERR_CUDA;
+    return decode_impl(q, k, v, g, beta, state_inout, kDense, out, nullptr, num_tokens, shape, stream);
 }
 
 gdn_status gdn_decode_verify(const void* q, const void* k, const void* v, const float* g,
                              const float* beta, const float* state, void* out, float* snapshots,
                              int32_t num_tokens, const gdn_shape* shape, void* stream) {
-    gdn_status st = check_common(shape);
-    if (st != GDN_OK) return st;
-    if (num_tokens < 1 || num_tokens > 4) return GDN_ERR_NUM_TOKENS;
-    if ((int64_t)shape->num_seqs * shape->num_v_heads * num_tokens > INT32_MAX) return GDN_ERR_SHAPE;
-    if (shape->num_seqs == 0) return GDN_OK;
-    if (!q || !k || !v || !g || !beta || !state || !out || !snapshots) return GDN_ERR_NULL;
-    const void* ptrs[] = {q, k, v, g, beta, state, out, snapshots};
-    for (const void* p : ptrs)
-        if (!aligned16(p)) return GDN_ERR_ALIGN;
-    cudaError_t e = gdn::launch_decode(q, k, v, g, beta, const_cast<float*>(state), out, snapshots,
-                                       num_tokens, shape->num_seqs, shape->num_qk_heads,
-                                       shape->num_v_heads, (gdn_dtype)shape->io_dtype,
-                                       reinterpret_cast<cudaStream_t>(stream));
-    return e == cudaSuccess ? GDN_OK : GDN_ERR_CUDA;
+    if (shape && shape->num_seqs > 0 && !snapshots) return GDN_ERR_NULL;
+    return decode_impl(q, k, v, g, beta, const_cast<float*>(state), kDense, out, snapshots, num_tokens,
+                       shape, stream);
 }
 
 gdn_status gdn_decode_commit(float* state, const float* snapshots, const int32_t* accepted,
                              int32_t num_tokens, const gdn_shape* shape, void* stream) {
-    gdn_status st = check_common(shape);
-    if (st != GDN_OK) return st;
-    if (num_tokens < 1 || num_tokens > 4) return GDN_ERR_NUM_TOKENS;
-    if ((int64_t)shape->num_seqs * shape->num_v_heads > INT32_MAX) return GDN_ERR_SHAPE;
-    if (shape->num_seqs == 0) return GDN_OK;
-    if (!state || !snapshots || !accepted) return GDN_ERR_NULL;
-    const void* ptrs[] = {state, snapshots, accepted};
-    for (const void* p : ptrs)
-        if (!aligned16(p)) return GDN_ERR_ALIGN;
-    cudaError_t e = gdn::launch_decode_commit(state, snapshots, accepted, num_tokens, shape->num_seqs,
-                                              shape->num_v_heads, reinterpret_cast<cudaStream_t>(stream));
-    return e == cudaSuccess ? GDN_OK : GDN_ERR_CUDA;
+    return commit_impl(state, kDense, snapshots, accepted, num_tokens, shape, stream);
+}
+
+gdn_status gdn_decode_step_slots(const void* q, const void* k, const void* v, const float* g,
+                                 const float* beta, float* state_pool, const int32_t* state_slots,
+                                 int32_t num_slots, void* out, int32_t num_tokens, const gdn_shape* shape,
+                                 void* stream) {
+    if (shape && shape->num_seqs > 0) {
+        gdn_status st = check_slots(state_pool, state_slots, num_slots);
+        if (st != GDN_OK) return st;
+    }
+    return decode_impl(q, k, v, g, beta, state_pool, gdn::StateSlots{state_slots, num_slots}, out, nullptr,
+                       num_tokens, shape, stream);
+}
+
+gdn_status gdn_decode_verify_slots(const void* q, const void* k, const void* v, const float* g,
+                                   const float* beta, const float* state_pool, const int32_t* state_slots,
+                                   int32_t num_slots, void* out, float* snapshots, int32_t num_tokens,
+                                   const gdn_shape* shape, void* stream) {
+    if (shape && shape->num_seqs > 0) {
+        gdn_status st = check_slots(state_pool, state_slots, num_slots);
+        if (st != GDN_OK) return st;
+        if (!snapshots) return GDN_ERR_NULL;
+    }
+    return decode_impl(q, k, v, g, beta, const_cast<float*>(state_pool), gdn::StateSlots{state_slots, num_slots},
+                       out, snapshots, num_tokens, shape, stream);
+}
+
+gdn_status gdn_decode_commit_slots(float* state_pool, const int32_t* state_slots, int32_t num_slots,
+                                   const float* snapshots, const int32_t* accepted, int32_t num_tokens,
+                                   const gdn_shape* shape, void* stream) {
+    if (shape && shape->num_seqs > 0) {
+        gdn_status st = check_slots(state_pool, state_slots, num_slots);
+        if (st != GDN_OK) return st;
+    }
+    return commit_impl(state_pool, gdn::StateSlots{state_slots, num_slots}, snapshots, accepted, num_tokens,
+                       shape, stream);
 }
 
 gdn_status gdn_selftest_wait_timeout(void* workspace, size_t workspace_bytes, uint32_t limit_us,

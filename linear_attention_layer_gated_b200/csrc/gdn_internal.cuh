@@ -44,19 +44,35 @@ __device__ __forceinline__ void store4(__nv_bfloat16* p, float4 v) {
     *reinterpret_cast<uint2*>(p) = u;
 }
 
+// ---------------------------------------------------------------- state addressing
+// States are either dense ([N][HV][D][D], state of sequence n at index n) or held in a
+// pool indexed through a slot table: sequence n's state is pool[slots[n]].  A slot outside
+// [0, num_slots) marks a sequence without a state (decode skips it; prefill starts it from
+// zeros and writes no final state).
+struct StateSlots {
+    const int32_t* slots;  // nullptr: dense
+    int num_slots;
+};
+__device__ __forceinline__ int state_index(const StateSlots& m, int n, bool& valid) {
+    if (!m.slots) { valid = true; return n; }
+    const int s = m.slots[n];
+    valid = s >= 0 && s < m.num_slots;
+    return valid ? s : 0;
+}
+
 // ---------------------------------------------------------------- launchers
 // Each returns cudaSuccess or the launch error; arguments were validated by the caller.
 // snap == nullptr: decode step in place; otherwise verify (state read only, per-token
 // states to snap).
 cudaError_t launch_decode(const void* q, const void* k, const void* v, const float* g,
-                          const float* beta, float* state, void* out, float* snap, int num_tokens,
-                          int num_seqs, int hk, int hv, gdn_dtype io, cudaStream_t stream);
-cudaError_t launch_decode_commit(float* state, const float* snap, const int32_t* accepted, int num_tokens,
-                                 int num_seqs, int hv, cudaStream_t stream);
+                          const float* beta, float* state, StateSlots map, void* out, float* snap,
+                          int num_tokens, int num_seqs, int hk, int hv, gdn_dtype io, cudaStream_t stream);
+cudaError_t launch_decode_commit(float* state, StateSlots map, const float* snap, const int32_t* accepted,
+                                 int num_tokens, int num_seqs, int hv, cudaStream_t stream);
 
 cudaError_t launch_prefill_simt(const void* q, const void* k, const void* v, const float* g,
                                 const float* beta, const float* s0, const int32_t* cu,
-                                void* out, float* sT, int num_seqs, int hk, int hv,
+                                void* out, float* sT, StateSlots map, int num_seqs, int hk, int hv,
                                 gdn_dtype io, cudaStream_t stream);
 
 // Tensor-core prefill (bf16 I/O): total workspace bytes (header included) and launch.
@@ -67,7 +83,7 @@ cudaError_t launch_prefill_tc_prep(const void* q, const void* k, const void* v, 
                                    int total_tokens, int hk, int hv, void* workspace,
                                    cudaStream_t stream);
 cudaError_t launch_prefill_tc_state(const float* s0, const int32_t* cu, void* out, float* sT,
-                                    int num_seqs, int total_tokens, int hk, int hv,
+                                    StateSlots map, int num_seqs, int total_tokens, int hk, int hv,
                                     void* workspace, cudaStream_t stream);
 
 // Diagnostic: a bounded wait that is guaranteed to expire (failure-path self-test).

@@ -65,7 +65,7 @@ __global__ void __launch_bounds__(kSimtThreads, 1)
 prefill_simt_kernel(const IO* __restrict__ q, const IO* __restrict__ k, const IO* __restrict__ v,
                     const float* __restrict__ g, const float* __restrict__ beta,
                     const float* s0, const int32_t* __restrict__ cu, IO* __restrict__ out,
-                    float* sT, int hk, int hv)
+                    float* sT, StateSlots map, int hk, int hv)
 {
     extern __shared__ __align__(16) unsigned char smem_raw[];
     SimtSmem& sm = *reinterpret_cast<SimtSmem*>(smem_raw);
@@ -78,7 +78,10 @@ prefill_simt_kernel(const IO* __restrict__ q, const IO* __restrict__ k, const IO
     const int ty = tid / 16, tx = tid % 16;
     const int cv0 = slice * kSlice;
     const int seq_begin = cu[n], seq_end = cu[n + 1];
-    const size_t state_base = ((size_t)n * hv + h) * kD * kD + (size_t)cv0 * kD;
+    bool has_state;
+    const int sidx = state_index(map, n, has_state);
+    if (!has_state) { s0 = nullptr; sT = nullptr; }  // no slot: start from zeros, keep no state
+    const size_t state_base = ((size_t)sidx * hv + h) * kD * kD + (size_t)cv0 * kD;
 
     for (int idx = tid; idx < kSlice * kD; idx += kSimtThreads) {
         const int i = idx / kD, j = idx % kD;
@@ -312,7 +315,7 @@ prefill_simt_kernel(const IO* __restrict__ q, const IO* __restrict__ k, const IO
 template <typename IO>
 cudaError_t launch_typed(const IO* q, const IO* k, const IO* v, const float* g,
                          const float* beta, const float* s0, const int32_t* cu, IO* out,
-                         float* sT, int num_seqs, int hk, int hv, cudaStream_t stream)
+                         float* sT, StateSlots map, int num_seqs, int hk, int hv, cudaStream_t stream)
 {
     const size_t smem = sizeof(SimtSmem);
     cudaError_t e = cudaFuncSetAttribute(prefill_simt_kernel<IO>,
@@ -320,7 +323,7 @@ cudaError_t launch_typed(const IO* q, const IO* k, const IO* v, const float* g,
     if (e != cudaSuccess) return e;
     const dim3 grid((unsigned)num_seqs * (unsigned)hv * kSlices);
     prefill_simt_kernel<IO><<<grid, kSimtThreads, smem, stream>>>(q, k, v, g, beta, s0, cu, out,
-                                                                   sT, hk, hv);
+                                                                   sT, map, hk, hv);
     return cudaGetLastError();
 }
 
@@ -328,17 +331,17 @@ cudaError_t launch_typed(const IO* q, const IO* k, const IO* v, const float* g,
 
 cudaError_t launch_prefill_simt(const void* q, const void* k, const void* v, const float* g,
                                 const float* beta, const float* s0, const int32_t* cu,
-                                void* out, float* sT, int num_seqs, int hk, int hv,
+                                void* out, float* sT, StateSlots map, int num_seqs, int hk, int hv,
                                 gdn_dtype io, cudaStream_t stream)
 {
     if (num_seqs == 0) return cudaSuccess;
     if (io == GDN_BF16) {
         using T = __nv_bfloat16;
         return launch_typed<T>((const T*)q, (const T*)k, (const T*)v, g, beta, s0, cu, (T*)out,
-                               sT, num_seqs, hk, hv, stream);
+                               sT, map, num_seqs, hk, hv, stream);
     }
     return launch_typed<float>((const float*)q, (const float*)k, (const float*)v, g, beta, s0, cu,
-                               (float*)out, sT, num_seqs, hk, hv, stream);
+                               (float*)out, sT, map, num_seqs, hk, hv, stream);
 }
 
 }  // namespace gdn

@@ -829,7 +829,7 @@ __device__ __forceinline__ void prefetch_slot(const unsigned char* ws, const WsL
 
 __global__ void __launch_bounds__(kStateThreads, 1)
 chunk_state_kernel(const float* s0, const int32_t* __restrict__ cu, __nv_bfloat16* __restrict__ out,
-                   float* sT, unsigned char* ws, int num_seqs, int total_tokens, int hk, int hv) {
+                   float* sT, StateSlots map, unsigned char* ws, int num_seqs, int total_tokens, int hk, int hv) {
     extern __shared__ __align__(1024) unsigned char sm[];
     const uint32_t sb = smem_u32(sm);
     StateSmall& ss = *reinterpret_cast<StateSmall*>(sm + kS_SMALL);
@@ -1000,7 +1000,10 @@ chunk_state_kernel(const float* s0, const int32_t* __restrict__ cu, __nv_bfloat1
             const int t = q4 * 32 + lane;  // d_k row of S^T this thread owns
             // fp32 state: S[dv0 + m][t], m = 0..15
             float S[16];
-            const size_t sbase = ((size_t)n * hv + h) * kD * kD + (size_t)dv0 * kD + t;
+            bool has_state;
+            const int sidx = state_index(map, n, has_state);
+            if (!has_state) { s0 = nullptr; sT = nullptr; }  // no slot: start from zeros, keep no state
+            const size_t sbase = ((size_t)sidx * hv + h) * kD * kD + (size_t)dv0 * kD + t;
 #pragma unroll
             for (int m = 0; m < 16; ++m) S[m] = s0 ? s0[sbase + (size_t)m * kD] : 0.f;
             auto write_b1 = [&]() {
@@ -1102,14 +1105,14 @@ cudaError_t launch_prefill_tc_prep(const void* q, const void* k, const void* v, 
 }
 
 cudaError_t launch_prefill_tc_state(const float* s0, const int32_t* cu, void* out, float* sT,
-                                    int num_seqs, int total_tokens, int hk, int hv,
+                                    StateSlots map, int num_seqs, int total_tokens, int hk, int hv,
                                     void* workspace, cudaStream_t stream) {
     if (num_seqs == 0) return cudaSuccess;
     cudaError_t e = cudaFuncSetAttribute(chunk_state_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          (int)kStateSmem);
     if (e != cudaSuccess) return e;
     chunk_state_kernel<<<(unsigned)num_seqs * hv * kSlices, kStateThreads, kStateSmem, stream>>>(
-        s0, cu, (__nv_bfloat16*)out, sT, static_cast<unsigned char*>(workspace), num_seqs,
+        s0, cu, (__nv_bfloat16*)out, sT, map, static_cast<unsigned char*>(workspace), num_seqs,
         total_tokens, hk, hv);
     return cudaGetLastError();
 }

@@ -25,7 +25,9 @@ STATUS = {0: "GDN_OK", 1: "GDN_ERR_NULL", 2: "GDN_ERR_SHAPE", 3: "GDN_ERR_ALIGN"
 EXPORTED = ["gdn_prefill_workspace_bytes", "gdn_chunk_prefill", "gdn_chunk_prefill_prep",
             "gdn_chunk_prefill_state", "gdn_decode_step", "gdn_get_device_error",
             "gdn_selftest_wait_timeout", "gdn_status_string", "gdn_abi_version",
-            "gdn_chunk_prefill_noalloc", "gdn_decode_verify", "gdn_decode_commit"]
+            "gdn_chunk_prefill_noalloc", "gdn_decode_verify", "gdn_decode_commit",
+            "gdn_chunk_prefill_slots", "gdn_decode_step_slots", "gdn_decode_verify_slots",
+            "gdn_decode_commit_slots"]
 
 
 class GdnShape(ctypes.Structure):
@@ -71,6 +73,16 @@ def lib() -> ctypes.CDLL:
             L.gdn_decode_verify.argtypes = [vp, vp, vp, fp, fp, fp, vp, fp, ctypes.c_int32, sp, vp]
             L.gdn_decode_commit.restype = ctypes.c_int
             L.gdn_decode_commit.argtypes = [fp, fp, ip, ctypes.c_int32, sp, vp]
+            i32 = ctypes.c_int32
+            L.gdn_chunk_prefill_slots.restype = ctypes.c_int
+            L.gdn_chunk_prefill_slots.argtypes = [vp, vp, vp, fp, fp, fp, ip, i32, ip, vp, sp, vp,
+                                                  ctypes.c_size_t, vp]
+            L.gdn_decode_step_slots.restype = ctypes.c_int
+            L.gdn_decode_step_slots.argtypes = [vp, vp, vp, fp, fp, fp, ip, i32, vp, i32, sp, vp]
+            L.gdn_decode_verify_slots.restype = ctypes.c_int
+            L.gdn_decode_verify_slots.argtypes = [vp, vp, vp, fp, fp, fp, ip, i32, vp, fp, i32, sp, vp]
+            L.gdn_decode_commit_slots.restype = ctypes.c_int
+            L.gdn_decode_commit_slots.argtypes = [fp, ip, i32, fp, ip, i32, sp, vp]
             L.gdn_get_device_error.restype = ctypes.c_int
             L.gdn_get_device_error.argtypes = [vp, vp]
             L.gdn_chunk_prefill_noalloc.restype = ctypes.c_int
@@ -223,6 +235,53 @@ def gdn_decode_commit(state, snapshots, accepted, num_tokens=None, stream=None):
                                  ctypes.byref(shape), _stream(stream))
     if rc != GDN_OK:
         raise GdnError(rc, "gdn_decode_commit")
+
+
+def gdn_chunk_prefill_slots(q, k, v, g, beta, state_pool, state_slots, cu_seqlens, out,
+                            workspace=None, algo=GDN_ALGO_AUTO, stream=None):
+    """Calls gdn_chunk_prefill_slots: initial and final states live in state_pool
+    [num_slots, HV, 128, 128] fp32 at the rows state_slots [N] (int32, device) names."""
+    shape = prefill_shape(q, v, cu_seqlens, algo)
+    if workspace is None:
+        workspace = alloc_workspace(shape, q.device)
+    rc = lib().gdn_chunk_prefill_slots(_ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(beta), _ptr(state_pool),
+                                       _ptr(state_slots), int(state_pool.shape[0]), _ptr(cu_seqlens), _ptr(out),
+                                       ctypes.byref(shape), _ptr(workspace), workspace.numel(), _stream(stream))
+    if rc != GDN_OK:
+        raise GdnError(rc, "gdn_chunk_prefill_slots")
+
+
+def gdn_decode_step_slots(q, k, v, g, beta, state_pool, state_slots, out, stream=None):
+    """Calls gdn_decode_step_slots (the pool rows named by state_slots are updated in place)."""
+    N, m, HK, D = q.shape
+    shape = make_shape(N, N * m, HK, v.shape[2], D, _io_dtype(q))
+    rc = lib().gdn_decode_step_slots(_ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(beta), _ptr(state_pool),
+                                     _ptr(state_slots), int(state_pool.shape[0]), _ptr(out), int(m),
+                                     ctypes.byref(shape), _stream(stream))
+    if rc != GDN_OK:
+        raise GdnError(rc, "gdn_decode_step_slots")
+
+
+def gdn_decode_verify_slots(q, k, v, g, beta, state_pool, state_slots, out, snapshots, stream=None):
+    """Calls gdn_decode_verify_slots (the pool is only read)."""
+    N, m, HK, D = q.shape
+    shape = make_shape(N, N * m, HK, v.shape[2], D, _io_dtype(q))
+    rc = lib().gdn_decode_verify_slots(_ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(beta), _ptr(state_pool),
+                                       _ptr(state_slots), int(state_pool.shape[0]), _ptr(out), _ptr(snapshots),
+                                       int(m), ctypes.byref(shape), _stream(stream))
+    if rc != GDN_OK:
+        raise GdnError(rc, "gdn_decode_verify_slots")
+
+
+def gdn_decode_commit_slots(state_pool, state_slots, snapshots, accepted, stream=None):
+    """Calls gdn_decode_commit_slots."""
+    N, m, HV, D, _ = snapshots.shape
+    shape = make_shape(N, N * m, 1, HV, D, GDN_BF16)
+    rc = lib().gdn_decode_commit_slots(_ptr(state_pool), _ptr(state_slots), int(state_pool.shape[0]),
+                                       _ptr(snapshots), _ptr(accepted), int(m), ctypes.byref(shape),
+                                       _stream(stream))
+    if rc != GDN_OK:
+        raise GdnError(rc, "gdn_decode_commit_slots")
 
 
 def gdn_chunk_prefill_noalloc(q, k, v, g, beta, initial_state, cu_seqlens, out, final_state,

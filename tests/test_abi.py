@@ -151,3 +151,25 @@ def test_verify_and_commit_reject_bad_arguments(L):
     assert gdn.STATUS[commit(acc=FAKE + 4)] == "GDN_ERR_ALIGN"
     empty = shape(num_seqs=0)
     assert L.gdn_decode_commit(None, None, None, 2, ctypes.byref(empty), None) == 0
+
+
+def test_slot_entry_points_reject_missing_pool_or_table(L):
+    s = shape(num_seqs=4)
+    assert gdn.STATUS[L.gdn_decode_step_slots(FAKE, FAKE, FAKE, FAKE, FAKE, None, FAKE, 8, FAKE, 1,
+                                              ctypes.byref(s), None)] == "GDN_ERR_NULL"
+    assert gdn.STATUS[L.gdn_decode_step_slots(FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, None, 8, FAKE, 1,
+                                              ctypes.byref(s), None)] == "GDN_ERR_NULL"
+    assert gdn.STATUS[L.gdn_decode_step_slots(FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, -1, FAKE, 1,
+                                              ctypes.byref(s), None)] == "GDN_ERR_SHAPE"
+    assert gdn.STATUS[L.gdn_decode_step_slots(FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE + 4, 8, FAKE, 1,
+                                              ctypes.byref(s), None)] == "GDN_ERR_ALIGN"
+    assert gdn.STATUS[L.gdn_decode_verify_slots(FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, 8, FAKE, None, 2,
+                                                ctypes.byref(s), None)] == "GDN_ERR_NULL"
+    assert gdn.STATUS[L.gdn_decode_commit_slots(FAKE, None, 8, FAKE, FAKE, 2, ctypes.byref(s),
+                                                None)] == "GDN_ERR_NULL"
+    ps = shape()
+    ws_bytes = L.gdn_prefill_workspace_bytes(ctypes.byref(ps))
+    assert gdn.STATUS[L.gdn_chunk_prefill_slots(FAKE, FAKE, FAKE, FAKE, FAKE, None, FAKE, 8, FAKE, FAKE,
+                                                ctypes.byref(ps), FAKE, ws_bytes, None)] == "GDN_ERR_NULL"
+    assert gdn.STATUS[L.gdn_chunk_prefill_slots(FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, -3, FAKE, FAKE,
+                                                ctypes.byref(ps), FAKE, ws_bytes, None)] == "GDN_ERR_SHAPE"

@@ -132,6 +132,82 @@ def test_commit_installs_the_accepted_snapshot():
         torch.testing.assert_close(st[n], want, rtol=0, atol=0)
 
 
+# ------------------------------------------------------------------ state-slot indirection
+def _slot_table(n, num_slots, seed):
+    """Distinct slots for n sequences from a pool of num_slots, every 5th one invalid."""
+    gen = torch.Generator().manual_seed(seed)
+    slots = torch.randperm(num_slots, generator=gen)[:n].to(torch.int32)
+    slots[::5] = -1
+    return slots.cuda()
+
+
+def test_decode_verify_commit_through_slots_match_dense():
+    N, ntok, S = 20, 3, 48
+    x = inputs.make_decode(N, ntok, hk=4, hv=8, seed=50, device="cuda")
+    pool = torch.randn(S, 8, 128, 128, device="cuda") * 0.02
+    slots = _slot_table(N, S, 51)
+    valid = slots >= 0
+    dense = torch.zeros_like(x["state"])
+    dense[valid] = pool[slots[valid].long()]
+    # decode step in place on the pool
+    p1 = pool.clone()
+    out_s = torch.full_like(x["v"], float("nan"))
+    gdn.gdn_decode_step_slots(x["q"], x["k"], x["v"], x["g"], x["beta"], p1, slots, out_s)
+    d1 = dense.clone()
+    out_d = gdn.decode(x["q"], x["k"], x["v"], x["g"], x["beta"], d1)
+    torch.cuda.synchronize()
+    torch.testing.assert_close(out_s[valid], out_d[valid], rtol=0, atol=0)
+    assert torch.isnan(out_s[~valid]).all()  # sequences without a slot are skipped
+    torch.testing.assert_close(p1[slots[valid].long()], d1[valid], rtol=0, atol=0)
+    untouched = torch.ones(S, dtype=torch.bool, device="cuda")
+    untouched[slots[valid].long()] = False
+    torch.testing.assert_close(p1[untouched], pool[untouched], rtol=0, atol=0)
+    # verify reads the pool, commit writes the accepted snapshot back into it
+    p2 = pool.clone()
+    out_v = torch.empty_like(x["v"])
+    snaps = torch.empty(N, ntok, 8, 128, 128, device="cuda")
+    gdn.gdn_decode_verify_slots(x["q"], x["k"], x["v"], x["g"], x["beta"], p2, slots, out_v, snaps)
+    torch.testing.assert_close(p2, pool, rtol=0, atol=0)
+    torch.testing.assert_close(out_v[valid], out_d[valid], rtol=0, atol=0)
+    accepted = torch.tensor([n % (ntok + 1) for n in range(N)], dtype=torch.int32, device="cuda")
+    gdn.gdn_decode_commit_slots(p2, slots, snaps, accepted)
+    torch.cuda.synchronize()
+    for n in range(N):
+        a, sl = int(accepted[n]), int(slots[n])
+        if sl < 0:
+            continue
+        want = snaps[n, a - 1] if a >= 1 else pool[sl]
+        torch.testing.assert_close(p2[sl], want, rtol=0, atol=0)
+
+
+@pytest.mark.parametrize("algo", ALGOS)
+def test_prefill_through_slots_matches_dense(algo):
+    lens = [70, 0, 130, 64, 1, 200]
+    x = inputs.make_prefill(lens, hk=2, hv=4, state_std=0.02, seed=52, device="cuda")
+    N, S = len(lens), 16
+    pool = torch.randn(S, 4, 128, 128, device="cuda") * 0.02
+    slots = _slot_table(N, S, 53)
+    valid = slots >= 0
+    init = torch.zeros(N, 4, 128, 128, device="cuda")
+    init[valid] = pool[slots[valid].long()]
+    out_d, fin_d = run_prefill(dict(x, initial_state=init), algo)
+    p1 = pool.clone()
+    out_s = torch.empty_like(x["v"])
+    try:
+        gdn.gdn_chunk_prefill_slots(x["q"], x["k"], x["v"], x["g"], x["beta"], p1, slots, x["cu_seqlens"],
+                                    out_s, algo=algo)
+    except gdn.GdnError as e:
+        if e.code == 9:
+            pytest.skip("algorithm not available")
+        raise
+    torch.cuda.synchronize()
+    torch.testing.assert_close(out_s, out_d, rtol=0, atol=0)
+    torch.testing.assert_close(p1[slots[valid].long()], fin_d[valid], rtol=0, atol=0)
+    untouched = torch.ones(S, dtype=torch.bool, device="cuda")
+    untouched[slots[valid].long()] = False
+    torch.testing.assert_close(p1[untouched], pool[untouched], rtol=0, atol=0)
+
+
 # ------------------------------------------------------------------ prefill, small
 def test_prefill_tiny_fp32_matches_oracle():
     x = inputs.make(inputs.workload("tiny"), device="cuda")
