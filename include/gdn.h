@@ -191,6 +191,25 @@ gdn_status gdn_decode_commit(float *state, const float *snapshots, const int32_t
                              int32_t num_tokens, const gdn_shape *shape, void *stream);
 
 /*
+ * Prefill that also keeps the state at every chunk boundary (for prefix caching: the
+ * pages' roadmap lists automatic prefix caching for hybrid models -- vLLM blog post,
+ * "Future Work" -- which needs the linear-attention state at cached prefix lengths).
+ * Same arguments and results as gdn_chunk_prefill, plus
+ *     chunk_states  [C][HV][D][D] fp32, C = sum over sequences of ceil(T_n / 64): the
+ *                   state after chunk c of sequence n (after token min(64 (c+1), T_n) - 1)
+ *                   is row sum_{m<n} ceil(T_m / 64) + c.  The last row of a sequence equals
+ *                   its final state.  Must not overlap the other buffers.
+ * GDN_ERR_NULL if chunk_states is missing while there are tokens.  Bytes: one extra state
+ * write per chunk (2 MiB per 64 tokens at 32 V heads).
+ */
+gdn_status gdn_chunk_prefill_chunk_states(const void *q, const void *k, const void *v,
+                                          const float *g, const float *beta,
+                                          const float *initial_state, const int32_t *cu_seqlens,
+                                          void *out, float *final_state, float *chunk_states,
+                                          const gdn_shape *shape, void *workspace,
+                                          size_t workspace_bytes, void *stream);
+
+/*
  * State-slot indirection (the pages' hybrid cache manager keeps the linear-attention
  * states of running requests in one preallocated pool -- vLLM blog post, "Hybrid KV
  * Cache Management"): the same prefill, decode, verify and commit on states held in

@@ -77,8 +77,8 @@ namespace {
 
 gdn_status prefill_impl(const void* q, const void* k, const void* v, const float* g, const float* beta,
                         const float* initial_state, const int32_t* cu_seqlens, void* out, float* final_state,
-                        gdn::StateSlots map, const gdn_shape* shape, void* workspace, size_t workspace_bytes,
-                        void* stream) {
+                        gdn::StateSlots map, float* chunk_states, const gdn_shape* shape, void* workspace,
+                        size_t workspace_bytes, void* stream) {
     gdn_status st = check_prefill_shape(shape);
     if (st != GDN_OK) return st;
     const size_t need = gdn_prefill_workspace_bytes(shape);
@@ -87,7 +87,7 @@ gdn_status prefill_impl(const void* q, const void* k, const void* v, const float
     if (shape->num_seqs == 0) return GDN_OK;
     if (!cu_seqlens) return GDN_ERR_NULL;
     if (shape->total_tokens > 0 && (!q || !k || !v || !g || !beta || !out)) return GDN_ERR_NULL;
-    const void* ptrs[] = {q, k, v, g, beta, initial_state, cu_seqlens, out, final_state};
+    const void* ptrs[] = {q, k, v, g, beta, initial_state, cu_seqlens, out, final_state, chunk_states};
     for (const void* p : ptrs)
         if (p && !aligned16(p)) return GDN_ERR_ALIGN;
 
@@ -102,12 +102,12 @@ gdn_status prefill_impl(const void* q, const void* k, const void* v, const float
                                         shape->total_tokens, shape->num_qk_heads,
                                         shape->num_v_heads, workspace, s);
         if (e == cudaSuccess)
-            e = gdn::launch_prefill_tc_state(initial_state, cu_seqlens, out, final_state, map,
+            e = gdn::launch_prefill_tc_state(initial_state, cu_seqlens, out, final_state, map, chunk_states,
                                              shape->num_seqs, shape->total_tokens,
                                              shape->num_qk_heads, shape->num_v_heads, workspace, s);
     } else
         e = gdn::launch_prefill_simt(q, k, v, g, beta, initial_state, cu_seqlens, out,
-                                     final_state, map, shape->num_seqs, shape->num_qk_heads,
+                                     final_state, map, chunk_states, shape->num_seqs, shape->num_qk_heads,
                                      shape->num_v_heads, io, s);
     return e == cudaSuccess ? GDN_OK : GDN_ERR_CUDA;
 }
@@ -163,8 +163,18 @@ gdn_status gdn_chunk_prefill(const void* q, const void* k, const void* v, const 
                              const int32_t* cu_seqlens, void* out, float* final_state,
                              const gdn_shape* shape, void* workspace, size_t workspace_bytes,
                              void* stream) {
-    return prefill_impl(q, k, v, g, beta, initial_state, cu_seqlens, out, final_state, kDense, shape,
+    return prefill_impl(q, k, v, g, beta, initial_state, cu_seqlens, out, final_state, kDense, nullptr, shape,
                         workspace, workspace_bytes, stream);
+}
+
+gdn_status gdn_chunk_prefill_chunk_states(const void* q, const void* k, const void* v, const float* g,
+                                          const float* beta, const float* initial_state,
+                                          const int32_t* cu_seqlens, void* out, float* final_state,
+                                          float* chunk_states, const gdn_shape* shape, void* workspace,
+                                          size_t workspace_bytes, void* stream) {
+    if (shape && shape->num_seqs > 0 && shape->total_tokens > 0 && !chunk_states) return GDN_ERR_NULL;
+    return prefill_impl(q, k, v, g, beta, initial_state, cu_seqlens, out, final_state, kDense, chunk_states,
+                        shape, workspace, workspace_bytes, stream);
 }
 
 gdn_status gdn_chunk_prefill_slots(const void* q, const void* k, const void* v, const float* g,
@@ -176,7 +186,7 @@ gdn_status gdn_chunk_prefill_slots(const void* q, const void* k, const void* v, 
     gdn_status st = check_slots(state_pool, state_slots, num_slots);
     if (st != GDN_OK) return st;
     return prefill_impl(q, k, v, g, beta, state_pool, cu_seqlens, out, state_pool,
-                        gdn::StateSlots{state_slots, num_slots}, shape, workspace, workspace_bytes, stream);
+                        gdn::StateSlots{state_slots, num_slots}, nullptr, shape, workspace, workspace_bytes, stream);
 }
 
 // Shared validation of the two tensor-core prefill phases.
@@ -221,7 +231,7 @@ gdn_status gdn_chunk_prefill_state(const float* initial_state, const int32_t* cu
     const void* ptrs[] = {initial_state, out, final_state};
     for (const void* p : ptrs)
         if (p && !aligned16(p)) return GDN_ERR_ALIGN;
-    cudaError_t e = gdn::launch_prefill_tc_state(initial_state, cu_seqlens, out, final_state, kDense,
+    cudaError_t e = gdn::launch_prefill_tc_state(initial_state, cu_seqlens, out, final_state, kDense, nullptr,
                                                  shape->num_seqs, shape->total_tokens,
                                                  shape->num_qk_heads, shape->num_v_heads,
                                                  workspace, reinterpret_cast<cudaStream_t>(stream));

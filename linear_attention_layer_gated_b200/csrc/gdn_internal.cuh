@@ -72,8 +72,8 @@ cudaError_t launch_decode_commit(float* state, StateSlots map, const float* snap
 
 cudaError_t launch_prefill_simt(const void* q, const void* k, const void* v, const float* g,
                                 const float* beta, const float* s0, const int32_t* cu,
-                                void* out, float* sT, StateSlots map, int num_seqs, int hk, int hv,
-                                gdn_dtype io, cudaStream_t stream);
+                                void* out, float* sT, StateSlots map, float* cstates, int num_seqs, int hk,
+                                int hv, gdn_dtype io, cudaStream_t stream);
 
 // Tensor-core prefill (bf16 I/O): total workspace bytes (header included) and launch.
 size_t tc_workspace_bytes(int num_seqs, int total_tokens, int hk, int hv);
@@ -82,9 +82,11 @@ cudaError_t launch_prefill_tc_prep(const void* q, const void* k, const void* v, 
                                    const float* beta, const int32_t* cu, int num_seqs,
                                    int total_tokens, int hk, int hv, void* workspace,
                                    cudaStream_t stream);
+// cstates (nullable): the state after every chunk, [total chunks][HV][D][D], chunks in
+// sequence order.
 cudaError_t launch_prefill_tc_state(const float* s0, const int32_t* cu, void* out, float* sT,
-                                    StateSlots map, int num_seqs, int total_tokens, int hk, int hv,
-                                    void* workspace, cudaStream_t stream);
+                                    StateSlots map, float* cstates, int num_seqs, int total_tokens, int hk,
+                                    int hv, void* workspace, cudaStream_t stream);
 
 // Diagnostic: a bounded wait that is guaranteed to expire (failure-path self-test).
 cudaError_t launch_wait_timeout_selftest(void* workspace, uint64_t limit_ns, cudaStream_t stream);

@@ -65,7 +65,7 @@ __global__ void __launch_bounds__(kSimtThreads, 1)
 prefill_simt_kernel(const IO* __restrict__ q, const IO* __restrict__ k, const IO* __restrict__ v,
                     const float* __restrict__ g, const float* __restrict__ beta,
                     const float* s0, const int32_t* __restrict__ cu, IO* __restrict__ out,
-                    float* sT, StateSlots map, int hk, int hv)
+                    float* sT, StateSlots map, float* cstates, int hk, int hv)
 {
     extern __shared__ __align__(16) unsigned char smem_raw[];
     SimtSmem& sm = *reinterpret_cast<SimtSmem*>(smem_raw);
@@ -88,7 +88,21 @@ prefill_simt_kernel(const IO* __restrict__ q, const IO* __restrict__ k, const IO
         sm.St[i][j] = s0 ? s0[state_base + (size_t)i * kD + j] : 0.f;
     }
 
-    for (int t0 = seq_begin; t0 < seq_end; t0 += kChunk) {
+    // Chunk-end states (optional): chunk c of sequence n goes to row chunk0 + c of
+    // cstates, chunk0 = sum over earlier sequences of their chunk counts.
+    __shared__ int s_chunk0;
+    if (cstates) {
+        int part = 0;
+        for (int m = tid; m < n; m += kSimtThreads) part += (cu[m + 1] - cu[m] + kChunk - 1) / kChunk;
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) part += __shfl_xor_sync(0xffffffffu, part, o);
+        if (tid == 0) s_chunk0 = 0;
+        __syncthreads();
+        if (lane == 0) atomicAdd(&s_chunk0, part);
+    }
+    int chunk_no = 0;
+
+    for (int t0 = seq_begin; t0 < seq_end; t0 += kChunk, ++chunk_no) {
         const int L = min(kChunk, seq_end - t0);
         __syncthreads();
 
@@ -301,6 +315,13 @@ prefill_simt_kernel(const IO* __restrict__ q, const IO* __restrict__ k, const IO
             for (int i = 0; i < 2; ++i)
 #pragma unroll
                 for (int cc = 0; cc < 8; ++cc) sm.St[ty + 16 * i][tx + 16 * cc] = acc[i][cc];
+            if (cstates) {
+                float* cs_row = cstates + ((size_t)(s_chunk0 + chunk_no) * hv + h) * kD * kD + (size_t)cv0 * kD;
+#pragma unroll
+                for (int i = 0; i < 2; ++i)
+#pragma unroll
+                    for (int cc = 0; cc < 8; ++cc) cs_row[(size_t)(ty + 16 * i) * kD + tx + 16 * cc] = acc[i][cc];
+            }
         }
     }
     __syncthreads();
@@ -315,7 +336,8 @@ prefill_simt_kernel(const IO* __restrict__ q, const IO* __restrict__ k, const IO
 template <typename IO>
 cudaError_t launch_typed(const IO* q, const IO* k, const IO* v, const float* g,
                          const float* beta, const float* s0, const int32_t* cu, IO* out,
-                         float* sT, StateSlots map, int num_seqs, int hk, int hv, cudaStream_t stream)
+                         float* sT, StateSlots map, float* cstates, int num_seqs, int hk, int hv,
+                         cudaStream_t stream)
 {
     const size_t smem = sizeof(SimtSmem);
     cudaError_t e = cudaFuncSetAttribute(prefill_simt_kernel<IO>,
@@ -323,7 +345,7 @@ cudaError_t launch_typed(const IO* q, const IO* k, const IO* v, const float* g,
     if (e != cudaSuccess) return e;
     const dim3 grid((unsigned)num_seqs * (unsigned)hv * kSlices);
     prefill_simt_kernel<IO><<<grid, kSimtThreads, smem, stream>>>(q, k, v, g, beta, s0, cu, out,
-                                                                   sT, map, hk, hv);
+                                                                   sT, map, cstates, hk, hv);
     return cudaGetLastError();
 }
 
@@ -331,17 +353,17 @@ cudaError_t launch_typed(const IO* q, const IO* k, const IO* v, const float* g,
 
 cudaError_t launch_prefill_simt(const void* q, const void* k, const void* v, const float* g,
                                 const float* beta, const float* s0, const int32_t* cu,
-                                void* out, float* sT, StateSlots map, int num_seqs, int hk, int hv,
-                                gdn_dtype io, cudaStream_t stream)
+                                void* out, float* sT, StateSlots map, float* cstates, int num_seqs, int hk,
+                                int hv, gdn_dtype io, cudaStream_t stream)
 {
     if (num_seqs == 0) return cudaSuccess;
     if (io == GDN_BF16) {
         using T = __nv_bfloat16;
         return launch_typed<T>((const T*)q, (const T*)k, (const T*)v, g, beta, s0, cu, (T*)out,
-                               sT, map, num_seqs, hk, hv, stream);
+                               sT, map, cstates, num_seqs, hk, hv, stream);
     }
     return launch_typed<float>((const float*)q, (const float*)k, (const float*)v, g, beta, s0, cu,
-                               (float*)out, sT, map, num_seqs, hk, hv, stream);
+                               (float*)out, sT, map, cstates, num_seqs, hk, hv, stream);
 }
 
 }  // namespace gdn

@@ -829,7 +829,8 @@ __device__ __forceinline__ void prefetch_slot(const unsigned char* ws, const WsL
 
 __global__ void __launch_bounds__(kStateThreads, 1)
 chunk_state_kernel(const float* s0, const int32_t* __restrict__ cu, __nv_bfloat16* __restrict__ out,
-                   float* sT, StateSlots map, unsigned char* ws, int num_seqs, int total_tokens, int hk, int hv) {
+                   float* sT, StateSlots map, float* cstates, unsigned char* ws, int num_seqs, int total_tokens,
+                   int hk, int hv) {
     extern __shared__ __align__(1024) unsigned char sm[];
     const uint32_t sb = smem_u32(sm);
     StateSmall& ss = *reinterpret_cast<StateSmall*>(sm + kS_SMALL);
@@ -1056,6 +1057,11 @@ chunk_state_kernel(const float* s0, const int32_t* __restrict__ cu, __nv_bfloat1
 #pragma unroll
                 for (int m = 0; m < 16; ++m) S[m] = fmaf(gl, S[m], acc[m]);
                 if (c < nch) write_b1();
+                if (cstates) {  // the state after chunk c-1, after the proxy fence (stores may stay in flight)
+                    float* cr = cstates + ((size_t)(cs + c - 1) * hv + h) * kD * kD + (size_t)dv0 * kD + t;
+#pragma unroll
+                    for (int m = 0; m < 16; ++m) cr[(size_t)m * kD] = S[m];
+                }
                 if (out_warp) {
                     if (c >= 2) write_outputs(c - 2, prev_gam);
                     prev_gam = gr;
@@ -1105,14 +1111,14 @@ cudaError_t launch_prefill_tc_prep(const void* q, const void* k, const void* v, 
 }
 
 cudaError_t launch_prefill_tc_state(const float* s0, const int32_t* cu, void* out, float* sT,
-                                    StateSlots map, int num_seqs, int total_tokens, int hk, int hv,
-                                    void* workspace, cudaStream_t stream) {
+                                    StateSlots map, float* cstates, int num_seqs, int total_tokens, int hk,
+                                    int hv, void* workspace, cudaStream_t stream) {
     if (num_seqs == 0) return cudaSuccess;
     cudaError_t e = cudaFuncSetAttribute(chunk_state_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          (int)kStateSmem);
     if (e != cudaSuccess) return e;
     chunk_state_kernel<<<(unsigned)num_seqs * hv * kSlices, kStateThreads, kStateSmem, stream>>>(
-        s0, cu, (__nv_bfloat16*)out, sT, map, static_cast<unsigned char*>(workspace), num_seqs,
+        s0, cu, (__nv_bfloat16*)out, sT, map, cstates, static_cast<unsigned char*>(workspace), num_seqs,
         total_tokens, hk, hv);
     return cudaGetLastError();
 }

@@ -27,7 +27,7 @@ EXPORTED = ["gdn_prefill_workspace_bytes", "gdn_chunk_prefill", "gdn_chunk_prefi
             "gdn_selftest_wait_timeout", "gdn_status_string", "gdn_abi_version",
             "gdn_chunk_prefill_noalloc", "gdn_decode_verify", "gdn_decode_commit",
             "gdn_chunk_prefill_slots", "gdn_decode_step_slots", "gdn_decode_verify_slots",
-            "gdn_decode_commit_slots"]
+            "gdn_decode_commit_slots", "gdn_chunk_prefill_chunk_states"]
 
 
 class GdnShape(ctypes.Structure):
@@ -83,6 +83,9 @@ def lib() -> ctypes.CDLL:
             L.gdn_decode_verify_slots.argtypes = [vp, vp, vp, fp, fp, fp, ip, i32, vp, fp, i32, sp, vp]
             L.gdn_decode_commit_slots.restype = ctypes.c_int
             L.gdn_decode_commit_slots.argtypes = [fp, ip, i32, fp, ip, i32, sp, vp]
+            L.gdn_chunk_prefill_chunk_states.restype = ctypes.c_int
+            L.gdn_chunk_prefill_chunk_states.argtypes = [vp, vp, vp, fp, fp, fp, ip, vp, fp, fp, sp, vp,
+                                                         ctypes.c_size_t, vp]
             L.gdn_get_device_error.restype = ctypes.c_int
             L.gdn_get_device_error.argtypes = [vp, vp]
             L.gdn_chunk_prefill_noalloc.restype = ctypes.c_int
@@ -235,6 +238,21 @@ def gdn_decode_commit(state, snapshots, accepted, num_tokens=None, stream=None):
                                  ctypes.byref(shape), _stream(stream))
     if rc != GDN_OK:
         raise GdnError(rc, "gdn_decode_commit")
+
+
+def gdn_chunk_prefill_chunk_states(q, k, v, g, beta, initial_state, cu_seqlens, out, final_state,
+                                   chunk_states, workspace=None, algo=GDN_ALGO_AUTO, stream=None):
+    """Calls gdn_chunk_prefill_chunk_states: as gdn_chunk_prefill, plus the state after every
+    64-token chunk in chunk_states [sum_n ceil(T_n / 64), HV, 128, 128] fp32."""
+    shape = prefill_shape(q, v, cu_seqlens, algo)
+    if workspace is None:
+        workspace = alloc_workspace(shape, q.device)
+    rc = lib().gdn_chunk_prefill_chunk_states(_ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(beta),
+                                              _ptr(initial_state), _ptr(cu_seqlens), _ptr(out),
+                                              _ptr(final_state), _ptr(chunk_states), ctypes.byref(shape),
+                                              _ptr(workspace), workspace.numel(), _stream(stream))
+    if rc != GDN_OK:
+        raise GdnError(rc, "gdn_chunk_prefill_chunk_states")
 
 
 def gdn_chunk_prefill_slots(q, k, v, g, beta, state_pool, state_slots, cu_seqlens, out,

@@ -173,3 +173,14 @@ def test_slot_entry_points_reject_missing_pool_or_table(L):
                                                 ctypes.byref(ps), FAKE, ws_bytes, None)] == "GDN_ERR_NULL"
     assert gdn.STATUS[L.gdn_chunk_prefill_slots(FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, -3, FAKE, FAKE,
                                                 ctypes.byref(ps), FAKE, ws_bytes, None)] == "GDN_ERR_SHAPE"
+
+
+def test_chunk_states_prefill_requires_its_buffer(L):
+    s = shape()
+    ws_bytes = L.gdn_prefill_workspace_bytes(ctypes.byref(s))
+    assert gdn.STATUS[L.gdn_chunk_prefill_chunk_states(FAKE, FAKE, FAKE, FAKE, FAKE, None, FAKE, FAKE, None,
+                                                       None, ctypes.byref(s), FAKE, ws_bytes,
+                                                       None)] == "GDN_ERR_NULL"
+    assert gdn.STATUS[L.gdn_chunk_prefill_chunk_states(FAKE, FAKE, FAKE, FAKE, FAKE, None, FAKE, FAKE, None,
+                                                       FAKE + 8, ctypes.byref(s), FAKE, ws_bytes,
+                                                       None)] == "GDN_ERR_ALIGN"

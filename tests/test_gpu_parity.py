@@ -208,6 +208,42 @@ def test_prefill_through_slots_matches_dense(algo):
     torch.testing.assert_close(p1[untouched], pool[untouched], rtol=0, atol=0)
 
 
+# ------------------------------------------------------------------ chunk-boundary states
+@pytest.mark.parametrize("algo", ALGOS)
+def test_prefill_chunk_states_match_oracle_prefixes(algo):
+    lens = [70, 0, 130, 64]
+    x = inputs.make_prefill(lens, hk=2, hv=4, state_std=0.02, seed=54, device="cuda")
+    nchunks = sum((L + 63) // 64 for L in lens)
+    cst = torch.full((nchunks, 4, 128, 128), float("nan"), device="cuda")
+    out = torch.empty_like(x["v"])
+    fin = torch.empty_like(x["initial_state"])
+    try:
+        gdn.gdn_chunk_prefill_chunk_states(x["q"], x["k"], x["v"], x["g"], x["beta"], x["initial_state"],
+                                           x["cu_seqlens"], out, fin, cst, algo=algo)
+    except gdn.GdnError as e:
+        if e.code == 9:
+            pytest.skip("algorithm not available")
+        raise
+    torch.cuda.synchronize()
+    out_ref, _ = run_prefill(x, algo)
+    torch.testing.assert_close(out, out_ref, rtol=0, atol=0)  # outputs unchanged by the extra writes
+    tol = TOL_F32 if x["q"].dtype == torch.float32 else TOL_BF16
+    cu = x["cu_seqlens"].cpu().tolist()
+    row = 0
+    for n, L in enumerate(lens):
+        for c in range((L + 63) // 64):
+            end = cu[n] + min(64 * (c + 1), L)
+            sl = slice(cu[n], end)
+            cu1 = torch.tensor([0, end - cu[n]], dtype=torch.int32)
+            _, s_ref = oracle.forward(x["q"][sl], x["k"][sl], x["v"][sl], x["g"][sl], x["beta"][sl], cu1,
+                                      x["initial_state"][n:n + 1])
+            assert_close(cst[row], s_ref[0], tol, "chunk state %d (sequence %d, chunk %d)" % (row, n, c))
+            if 64 * (c + 1) >= L:
+                torch.testing.assert_close(cst[row], fin[n], rtol=0, atol=0)
+            row += 1
+    assert row == nchunks
+
+
 # ------------------------------------------------------------------ prefill, small
 def test_prefill_tiny_fp32_matches_oracle():
     x = inputs.make(inputs.workload("tiny"), device="cuda")
