@@ -624,11 +624,16 @@ chunk_prep_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __re
 
     // ---- 7. epilogue: accumulator row r' (lane quarter qw) is row r' % 64 of head r' / 64;
     //         each warp takes 64 of the 128 columns.  The W image is stored pre-scaled by the
-    //         previous chunk's total decay (W~ = gam_L,prev W).
+    //         previous chunk's total decay (W~ = gam_L,prev W).  Images are assembled in
+    //         shared memory that is free by then, in their final (swizzled) layout, and leave
+    //         as 8 KB bulk copies: round 1 W~ of both heads (K and Q slots), round 2 U of head
+    //         1 and M~ of both heads (the same four 8 KB pieces).  U of head 0 goes straight to
+    //         the workspace (its accumulator is reused before round 2).
     {
         const int hh = qw >> 1, r = (qw & 1) * 32 + lane, h = h0 + hh;
         const uint32_t tq = tmem + ((uint32_t)qw * 32u << 16);
-        unsigned char* wimg = ws + L.w + ((size_t)cid * hv + h) * kWBytes;
+        // piece i: the Q (i even) or K (i odd) slot of d_k block i / 2, 8 KB each
+        auto piece = [&](int i) { return sm + kP_GR + (i >> 1) * kP_GRB + (i & 1) * 8192; };
         unsigned char* uimg = ws + L.u + ((size_t)cid * hv + h) * kUBytes;
         const float gp = ss.gprev[hh];
         float col[32];
@@ -642,13 +647,14 @@ chunk_prep_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __re
             for (int ch = 0; ch < 4; ++ch)
                 *reinterpret_cast<uint4*>(img + sw128(r, chunk0 + ch)) = pack8(col + 8 * ch);
         };
-        // W columns 64 hf .. 64 hf + 63 = d_k block hf (8 KB image half)
-        store32(wimg + hf * 8192, 64 * hf, 0, gp);
-        store32(wimg + hf * 8192, 64 * hf + 32, 4, gp);
+        // W columns 64 hf .. 64 hf + 63 = d_k block hf (8 KB image half) -> piece 2 hh + hf
+        store32(piece(2 * hh + hf), 64 * hf, 0, gp);
+        store32(piece(2 * hh + hf), 64 * hf + 32, 4, gp);
         if (hh == 0) {  // U of head 0: columns 128 + 64 hf ..
             store32(uimg + hf * 8192, 128 + 64 * hf, 0, 1.f);
             store32(uimg + hf * 8192, 128 + 64 * hf + 32, 4, 1.f);
         }
+        fence_async_smem();
         tc_fence_before();
         __syncthreads();
         if (tid == 0) {  // U of head 1: D[:, 128:256] = A_U V_1 (rows 64..127 are head 1's)
@@ -664,15 +670,21 @@ chunk_prep_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __re
             }
             mma_commit(&ss.bar_mma);
         }
+        if (tid == 32) {  // round 1 out: W~ of both heads
+            unsigned char* w0 = ws + L.w + ((size_t)cid * hv + h0) * kWBytes;
+#pragma unroll
+            for (int i = 0; i < 4; ++i) bulk_s2g(w0 + (i >> 1) * kWBytes + (i & 1) * 8192, piece(i), 8192);
+            bulk_commit();
+            bulk_wait_read_all();  // the pieces are read before round 2 refills them
+        }
         ok = mbar_wait(&ss.bar_mma, 0);
         if (__syncthreads_or(!ok)) { err = 1; goto cleanup; }
         tc_fence_after();
-        if (hh == 1) {
-            store32(uimg + hf * 8192, 128 + 64 * hf, 0, 1.f);
-            store32(uimg + hf * 8192, 128 + 64 * hf + 32, 4, 1.f);
+        if (hh == 1) {  // U of head 1 -> pieces 0 (d_v block 0) and 1 (d_v block 1)
+            store32(piece(hf), 128 + 64 * hf, 0, 1.f);
+            store32(piece(hf), 128 + 64 * hf + 32, 4, 1.f);
         }
-        {   // M~ = M diag(c_prev): columns 32 hf .. 32 hf + 31
-            unsigned char* mimg = ws + L.m + ((size_t)cid * hv + h) * kMBytes;
+        {   // M~ = M diag(c_prev): columns 32 hf .. 32 hf + 31 of head hh -> piece 2 + hh
             tmem_ld16(tq + 32 * hf, col);
             tmem_ld16(tq + 32 * hf + 16, col + 16);
             tmem_ld_wait();
@@ -681,7 +693,19 @@ chunk_prep_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __re
             for (int e = 0; e < 32; ++e) col[e] *= cp[e];
 #pragma unroll
             for (int ch = 0; ch < 4; ++ch)
-                *reinterpret_cast<uint4*>(mimg + sw128(r, 4 * hf + ch)) = pack8(col + 8 * ch);
+                *reinterpret_cast<uint4*>(piece(2 + hh) + sw128(r, 4 * hf + ch)) = pack8(col + 8 * ch);
+        }
+        fence_async_smem();
+        __syncthreads();
+        if (tid == 32) {  // round 2 out: U of head 1, M~ of both heads
+            unsigned char* u1 = ws + L.u + ((size_t)cid * hv + h0 + 1) * kUBytes;
+            unsigned char* m0 = ws + L.m + ((size_t)cid * hv + h0) * kMBytes;
+            bulk_s2g(u1, piece(0), 8192);
+            bulk_s2g(u1 + 8192, piece(1), 8192);
+            bulk_s2g(m0, piece(2), 8192);
+            bulk_s2g(m0 + kMBytes, piece(3), 8192);
+            bulk_commit();
+            bulk_wait_read_all();  // shared memory is read before the CTA exits
         }
     }
 
