@@ -67,6 +67,29 @@ def decode_bytes(num_seqs, ntok):
     return num_seqs * (STATE_BYTES * 2 + ntok * PREFILL_BYTES_PER_TOKEN)
 
 
+def load_traffic():
+    """DRAM bytes per launch of the prefill kernels from the committed ncu record, or {} if
+    the record is missing or was taken on a different version of the kernel source."""
+    import hashlib
+    rec = os.path.join(ROOT, "profiles", "traffic_layer_T8192.txt")
+    try:
+        lines = open(rec).read().splitlines()
+    except OSError:
+        return {}
+    fields = dict(l.split(": ", 1) for l in lines if ": " in l and not l.startswith("#"))
+    try:
+        src = os.path.join(ROOT, fields["source"])
+        if hashlib.sha256(open(src, "rb").read()).hexdigest() != fields["source_sha256"]:
+            return {}
+        out = {}
+        for kname in ("chunk_table_kernel", "chunk_prep_kernel", "chunk_state_kernel"):
+            parts = fields[kname].split()
+            out[kname] = int(parts[1]) + int(parts[3])
+        return out
+    except (KeyError, OSError, ValueError, IndexError):
+        return {}
+
+
 def load_peaks():
     path = os.path.join(ROOT, "MEASURED_PEAKS.json")
     try:
@@ -286,8 +309,12 @@ def main_ours(args, rank, world, local_rank):
             ph["frac_tensor"] = ph["tflops"] / peak
         dom = max(phases, key=lambda k2: phases[k2]["ms"])
         d = phases[dom]
+        traffic = None
+        tr = load_traffic() if T == 8192 and len(x["cu_seqlens"]) == 2 else {}
+        if tr:
+            traffic = (tr["chunk_table_kernel"] + tr["chunk_prep_kernel"]) if dom == "prep" else tr["chunk_state_kernel"]
         roofline = {"bound": "hbm", "achieved": d["gbs"], "peak": peaks["hbm_gbs"], "unit": "GB/s",
-                    "frac": d["frac_hbm"], "traffic": None,
+                    "frac": d["frac_hbm"], "traffic": traffic,
                     "peak_source": peaks["source"] + " HBM copy",
                     "kernel": d["kernels"], "algorithmic_bytes_per_launch": d["bytes"],
                     "tensor_frac": d["frac_tensor"],
