@@ -212,8 +212,7 @@ def reference_arm(args, rank, world):
 # ---------------------------------------------------------------- our arm
 def main_ours(args, rank, world, local_rank):
     import torch
-    import torch.distributed as dist
-    from linear_attention_layer_gated_b200 import build, gdn, inputs
+    from linear_attention_layer_gated_b200 import build, gdn, inputs, replicas
 
     build.build()
     torch.cuda.set_device(local_rank)
@@ -254,8 +253,7 @@ def main_ours(args, rank, world, local_rank):
         phase_ev.append(e)
 
     def barrier():
-        if world > 1:
-            dist.barrier()
+        replicas.barrier(world)
         torch.cuda.synchronize(dev)
 
     def timed(fn, steps, warmup, flush_between=True):
@@ -274,18 +272,14 @@ def main_ours(args, rank, world, local_rank):
         return [a.elapsed_time(b) for a, b in ev]
 
     def max_over_ranks(v):
-        if world == 1:
-            return v
-        t = torch.tensor([v], dtype=torch.float64, device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        return float(t.item())
+        return replicas.max_over_ranks(v, world, device=dev)
 
     step_fn = prefill_phased if tensor_path else prefill_once
     with ClockSampler(local_rank) as clk:
         ms = timed(step_fn, args.steps, args.warmup)
     clocks = clk.summary()
     ms_step = max_over_ranks(sum(ms) / len(ms))
-    value = world * T / (ms_step * 1e-3)
+    value = replicas.job_throughput(T, world, ms_step * 1e-3)
 
     # ---- dominant kernel roofline, from CUDA events on the launching stream
     launches_per_step = gdn_launches_per_prefill(algo, x["q"].dtype)
@@ -496,24 +490,15 @@ def main():
     args = ap.parse_args()
     if args.warmup < 3 and args.impl == "ours":
         args.warmup = 3
-    world = int(os.environ.get("WORLD_SIZE", "1"))
-    rank = int(os.environ.get("RANK", "0"))
-    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+    from linear_attention_layer_gated_b200 import replicas
+    rank, world, local_rank = replicas.rank_info()
     if args.impl == "reference":
         return reference_arm(args, rank, world)
-    if world > 1:
-        import datetime
-        import torch
-        import torch.distributed as dist
-        torch.cuda.set_device(local_rank)
-        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
-                                device_id=torch.device("cuda", local_rank))
+    replicas.init(world, local_rank, "nccl")
     try:
         return main_ours(args, rank, world, local_rank)
     finally:
-        if world > 1:
-            import torch.distributed as dist
-            dist.destroy_process_group()
+        replicas.finish(world)
 
 
 if __name__ == "__main__":
