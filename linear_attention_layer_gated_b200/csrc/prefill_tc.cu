@@ -87,6 +87,7 @@ __host__ __device__ inline WsLayout ws_layout(int num_seqs, int total_tokens, in
 // ===================================================================== K0
 __global__ void __launch_bounds__(1024)
 chunk_table_kernel(const int32_t* __restrict__ cu, int num_seqs, unsigned char* ws) {
+    allow_dependent_launch();
     int32_t* header = reinterpret_cast<int32_t*>(ws);
     const WsLayout L = ws_layout(num_seqs, 0, 1, 1);  // seq_chunk0 and table do not depend on T
     int32_t* seq_chunk0 = reinterpret_cast<int32_t*>(ws + L.seq_chunk0);
@@ -116,11 +117,18 @@ chunk_table_kernel(const int32_t* __restrict__ cu, int num_seqs, unsigned char* 
         header[1] = carry;
     }
     __syncthreads();
-    for (int n = threadIdx.x; n < num_seqs; n += blockDim.x) {
-        const int t0 = cu[n], len = cu[n + 1] - cu[n];
-        const int first = seq_chunk0[n];
-        for (int kk = 0; kk * kChunk < len; ++kk)
-            table[first + kk] = make_int4(n, t0 + kk * kChunk, min(kChunk, len - kk * kChunk), 0);
+    // one entry per thread: chunk c belongs to the last sequence n with seq_chunk0[n] <= c
+    const int total = carry;
+    for (int c = threadIdx.x; c < total; c += blockDim.x) {
+        int lo = 0, hi = num_seqs - 1;
+        while (lo < hi) {
+            const int mid = (lo + hi + 1) >> 1;
+            if (seq_chunk0[mid] <= c) lo = mid;
+            else hi = mid - 1;
+        }
+        const int n = lo, kk = c - seq_chunk0[n];
+        const int t0 = cu[n], len = cu[n + 1] - t0;
+        table[c] = make_int4(n, t0 + kk * kChunk, min(kChunk, len - kk * kChunk), 0);
     }
 }
 
@@ -224,6 +232,8 @@ chunk_prep_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __re
     int32_t* header = reinterpret_cast<int32_t*>(ws);
     const int cid = blockIdx.x / hk;
     const int jq = blockIdx.x % hk;
+    grid_dependency_wait();    // the chunk table is written
+    allow_dependent_launch();  // the state kernel may be scheduled as SMs free up
     if (cid >= header[1]) return;
     const int4 ent = reinterpret_cast<const int4*>(ws + L.table)[cid];
     const int t0 = ent.y, len = ent.z;
@@ -867,6 +877,7 @@ chunk_state_kernel(const float* s0, const int32_t* __restrict__ cu, __nv_bfloat1
     const int n = (blockIdx.x / kSlices) / hv;
     const int jq = h / (hv / hk);
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    grid_dependency_wait();  // the prep kernel's workspace is complete and visible
     const int32_t* seq_chunk0 = reinterpret_cast<const int32_t*>(ws + L.seq_chunk0);
     const int cs = seq_chunk0[n], nch = seq_chunk0[n + 1] - cs;
     const int t_begin = cu[n], t_end = cu[n + 1];
@@ -1109,6 +1120,24 @@ chunk_state_kernel(const float* s0, const int32_t* __restrict__ cu, __nv_bfloat1
     }
 }
 
+// Launch with programmatic stream serialization: the kernel may begin (and run its set-up)
+// while the previous kernel on the stream finishes; it waits with grid_dependency_wait.
+template <typename... KArgs, typename... Args>
+cudaError_t launch_dependent(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t stream,
+                             Args... args) {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = grid;
+    cfg.blockDim = block;
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, kernel, static_cast<KArgs>(args)...);
+}
+
 }  // namespace
 
 size_t tc_workspace_bytes(int num_seqs, int total_tokens, int hk, int hv) {
@@ -1127,9 +1156,10 @@ cudaError_t launch_prefill_tc_prep(const void* q, const void* k, const void* v, 
     if (e != cudaSuccess) return e;
     chunk_table_kernel<<<1, 1024, 0, stream>>>(cu, num_seqs, ws);
     if (L.max_chunks > 0 && total_tokens > 0) {
-        chunk_prep_kernel<<<(unsigned)(L.max_chunks * hk), kPrepThreads, kPrepSmem, stream>>>(
-            (const __nv_bfloat16*)q, (const __nv_bfloat16*)k, (const __nv_bfloat16*)v, g, beta, ws,
-            num_seqs, total_tokens, hk, hv);
+        e = launch_dependent(chunk_prep_kernel, dim3((unsigned)(L.max_chunks * hk)), dim3(kPrepThreads),
+                             kPrepSmem, stream, (const __nv_bfloat16*)q, (const __nv_bfloat16*)k,
+                             (const __nv_bfloat16*)v, g, beta, ws, num_seqs, total_tokens, hk, hv);
+        if (e != cudaSuccess) return e;
     }
     return cudaGetLastError();
 }
@@ -1141,9 +1171,10 @@ cudaError_t launch_prefill_tc_state(const float* s0, const int32_t* cu, void* ou
     cudaError_t e = cudaFuncSetAttribute(chunk_state_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          (int)kStateSmem);
     if (e != cudaSuccess) return e;
-    chunk_state_kernel<<<(unsigned)num_seqs * hv * kSlices, kStateThreads, kStateSmem, stream>>>(
-        s0, cu, (__nv_bfloat16*)out, sT, map, cstates, static_cast<unsigned char*>(workspace), num_seqs,
-        total_tokens, hk, hv);
+    e = launch_dependent(chunk_state_kernel, dim3((unsigned)num_seqs * hv * kSlices), dim3(kStateThreads),
+                         kStateSmem, stream, s0, cu, (__nv_bfloat16*)out, sT, map, cstates,
+                         static_cast<unsigned char*>(workspace), num_seqs, total_tokens, hk, hv);
+    if (e != cudaSuccess) return e;
     return cudaGetLastError();
 }
 

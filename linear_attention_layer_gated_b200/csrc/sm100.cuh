@@ -102,6 +102,16 @@ __device__ __forceinline__ void bulk_wait_read_all() {
     asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory");
 }
 
+// ------------------------------------------------------------------ programmatic dependent launch
+// A kernel launched with programmatic stream serialization may start before the previous
+// kernel on the stream has finished; grid_dependency_wait blocks (in hardware, no spin)
+// until that kernel has completed and its memory is visible, and is a no-op otherwise.
+// allow_dependent_launch lets the next kernel's CTAs be scheduled as SMs become free.
+__device__ __forceinline__ void grid_dependency_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void allow_dependent_launch() {
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+
 // ------------------------------------------------------------------ 16-byte async copies
 // (cp.async, global -> shared, bypassing L1; completion is waited for with cp_async_wait_all,
 // which is not a spin loop.)
