@@ -221,7 +221,7 @@ __global__ void __launch_bounds__(kPrepThreads, 2)
 chunk_prep_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __restrict__ k,
                   const __nv_bfloat16* __restrict__ v, const float* __restrict__ g,
                   const float* __restrict__ beta, unsigned char* ws, int num_seqs,
-                  int total_tokens, int hk, int hv) {
+                  int total_tokens, int hk, int hv, int resident) {
     extern __shared__ unsigned char smem_dyn[];
     unsigned char* sm = reinterpret_cast<unsigned char*>((reinterpret_cast<uintptr_t>(smem_dyn) + 1023) & ~uintptr_t(1023));
     const uint32_t sb = smem_u32(sm);
@@ -234,8 +234,14 @@ chunk_prep_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __re
     const int jq = blockIdx.x % hk;
     grid_dependency_wait();    // the chunk table is written
     allow_dependent_launch();  // the state kernel may be scheduled as SMs free up
-    if (cid >= header[1]) return;
+    const int nchunks = header[1];
+    if (cid >= nchunks) return;
     const int4 ent = reinterpret_cast<const int4*>(ws + L.table)[cid];
+    // The CTA that takes this one's place on the SM (CTAs start in index order, `resident`
+    // at a time): its chunk entry, for the L2 prefetch of its inputs in phase 3.
+    const int nb = blockIdx.x + resident;
+    const int ncid = nb / hk, njq = nb % hk;
+    const int4 nent = (ncid < nchunks) ? reinterpret_cast<const int4*>(ws + L.table)[ncid] : make_int4(0, 0, 0, 0);
     const int t0 = ent.y, len = ent.z;
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const int qw = warp & 3, hf = warp >> 2;  // TMEM lane quarter, column half
@@ -464,6 +470,21 @@ chunk_prep_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __re
                 *reinterpret_cast<uint4*>(vb + sw128(rr, c0 + 1)) = vr[hh][pass][1];
             }
         fence_async_smem();
+        // This CTA's own loads are done: ask L2 for the next CTA's q, k (one 128-byte line per
+        // thread), v of both heads (four lines per token) and gates.  Its K_prev rows and
+        // previous gates belong to the chunk before it, which a CTA now running has just read.
+        if (nent.z > 0) {
+            const int nt0 = nent.y, nlen = nent.z;
+            const int pr = tid >> 1, pl = tid & 1;
+            if ((pr & 63) < nlen) {
+                const __nv_bfloat16* src = (pr < 64 ? q : k) + ((size_t)(nt0 + (pr & 63)) * hk + njq) * kD + pl * 64;
+                prefetch_l2(src);
+            }
+            const int vrow = tid >> 2, vl = tid & 3;
+            if (vrow < nlen) prefetch_l2(v + ((size_t)(nt0 + vrow) * hv + 2 * njq) * kD + vl * 64);
+            if (tid < 128 && (tid & 63) < nlen)
+                prefetch_l2((tid < 64 ? g : beta) + (size_t)(nt0 + (tid & 63)) * hv + 2 * njq);
+        }
         if (qw < 2) {  // P rows, after the fence: these stores may stay in flight
             tmem_ld16(ta, row);
             tmem_ld16(ta + 16, row + 16);
@@ -1154,11 +1175,18 @@ cudaError_t launch_prefill_tc_prep(const void* q, const void* k, const void* v, 
     cudaError_t e = cudaFuncSetAttribute(chunk_prep_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          (int)kPrepSmem);
     if (e != cudaSuccess) return e;
+    int dev = 0, sms = 0, per_sm = 0;
+    if ((e = cudaGetDevice(&dev)) != cudaSuccess) return e;
+    if ((e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev)) != cudaSuccess) return e;
+    if ((e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, chunk_prep_kernel, kPrepThreads, kPrepSmem)) !=
+        cudaSuccess)
+        return e;
     chunk_table_kernel<<<1, 1024, 0, stream>>>(cu, num_seqs, ws);
     if (L.max_chunks > 0 && total_tokens > 0) {
         e = launch_dependent(chunk_prep_kernel, dim3((unsigned)(L.max_chunks * hk)), dim3(kPrepThreads),
                              kPrepSmem, stream, (const __nv_bfloat16*)q, (const __nv_bfloat16*)k,
-                             (const __nv_bfloat16*)v, g, beta, ws, num_seqs, total_tokens, hk, hv);
+                             (const __nv_bfloat16*)v, g, beta, ws, num_seqs, total_tokens, hk, hv,
+                             sms * per_sm);
         if (e != cudaSuccess) return e;
     }
     return cudaGetLastError();

@@ -93,6 +93,10 @@ __device__ __forceinline__ void bulk_s2g(void* dst_gmem, const void* src_smem, u
 }
 // Asks for `bytes` (a multiple of 16) at a 16-byte-aligned global address to be brought
 // into L2; nothing waits for it.
+// Asks L2 for the 128-byte line holding src (no register result, no completion to wait for).
+__device__ __forceinline__ void prefetch_l2(const void* src_gmem) {
+    asm volatile("prefetch.global.L2 [%0];" ::"l"(src_gmem));
+}
 __device__ __forceinline__ void bulk_prefetch_l2(const void* src_gmem, uint32_t bytes) {
     asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(src_gmem), "r"(bytes) : "memory");
 }
