@@ -67,10 +67,21 @@ def decode_bytes(num_seqs, ntok):
     return num_seqs * (STATE_BYTES * 2 + ntok * PREFILL_BYTES_PER_TOKEN)
 
 
+def source_code_sha256(path):
+    """sha256 of a C/CUDA source with its comments removed and its whitespace collapsed, so
+    that a record of measured counters stays keyed to the code it was taken on across edits
+    of comments and layout only."""
+    import hashlib
+    import re
+    text = open(path, encoding="utf-8").read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    text = re.sub(r"//[^\n]*", "", text)
+    return hashlib.sha256(" ".join(text.split()).encode()).hexdigest()
+
+
 def load_traffic():
     """DRAM bytes per launch of the prefill kernels from the committed ncu record, or {} if
-    the record is missing or was taken on a different version of the kernel source."""
-    import hashlib
+    the record is missing or was taken on a different version of the kernel code."""
     rec = os.path.join(ROOT, "profiles", "traffic_layer_T8192.txt")
     try:
         lines = open(rec).read().splitlines()
@@ -79,7 +90,7 @@ def load_traffic():
     fields = dict(l.split(": ", 1) for l in lines if ": " in l and not l.startswith("#"))
     try:
         src = os.path.join(ROOT, fields["source"])
-        if hashlib.sha256(open(src, "rb").read()).hexdigest() != fields["source_sha256"]:
+        if source_code_sha256(src) != fields["source_code_sha256"]:
             return {}
         out = {}
         for kname in ("chunk_table_kernel", "chunk_prep_kernel", "chunk_state_kernel"):

@@ -657,9 +657,9 @@ chunk_prep_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __re
     //         each warp takes 64 of the 128 columns.  The W image is stored pre-scaled by the
     //         previous chunk's total decay (W~ = gam_L,prev W).  Images are assembled in
     //         shared memory that is free by then, in their final (swizzled) layout, and leave
-    //         as 8 KB bulk copies: round 1 W~ of both heads (K and Q slots), round 2 U of head
+    //         as 8 KB bulk copies: batch 1 W~ of both heads (K and Q slots), batch 2 U of head
     //         1 and M~ of both heads (the same four 8 KB pieces).  U of head 0 goes straight to
-    //         the workspace (its accumulator is reused before round 2).
+    //         the workspace (its accumulator is reused before batch 2).
     {
         const int hh = qw >> 1, r = (qw & 1) * 32 + lane, h = h0 + hh;
         const uint32_t tq = tmem + ((uint32_t)qw * 32u << 16);
@@ -701,12 +701,12 @@ chunk_prep_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __re
             }
             mma_commit(&ss.bar_mma);
         }
-        if (tid == 32) {  // round 1 out: W~ of both heads
+        if (tid == 32) {  // batch 1 out: W~ of both heads
             unsigned char* w0 = ws + L.w + ((size_t)cid * hv + h0) * kWBytes;
 #pragma unroll
             for (int i = 0; i < 4; ++i) bulk_s2g(w0 + (i >> 1) * kWBytes + (i & 1) * 8192, piece(i), 8192);
             bulk_commit();
-            bulk_wait_read_all();  // the pieces are read before round 2 refills them
+            bulk_wait_read_all();  // the pieces are read before batch 2 refills them
         }
         ok = mbar_wait(&ss.bar_mma, 0);
         if (__syncthreads_or(!ok)) { err = 1; goto cleanup; }
@@ -728,7 +728,7 @@ chunk_prep_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __re
         }
         fence_async_smem();
         __syncthreads();
-        if (tid == 32) {  // round 2 out: U of head 1, M~ of both heads
+        if (tid == 32) {  // batch 2 out: U of head 1, M~ of both heads
             unsigned char* u1 = ws + L.u + ((size_t)cid * hv + h0 + 1) * kUBytes;
             unsigned char* m0 = ws + L.m + ((size_t)cid * hv + h0) * kMBytes;
             bulk_s2g(u1, piece(0), 8192);
