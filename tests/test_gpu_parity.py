@@ -422,3 +422,68 @@ def test_bounded_wait_expiry_is_reported_and_context_survives():
     assert gdn.gdn_get_device_error(ws2) == gdn.GDN_OK
     o_ref, _ = oracle.forward(x["q"], x["k"], x["v"], x["g"], x["beta"], x["cu_seqlens"], None)
     assert_close(out, o_ref, TOL_BF16, "prefill after a reported timeout")
+
+
+# ------------------------------------------------------------------ poisoned buffers
+# Outputs and states sit inside NaN-filled buffers with a guard row on each side: every
+# element a call owns must be written (finite and matching the oracle) and nothing outside
+# it touched.  The prefill workspace starts as 0xFF bytes (NaN in fp32 and bf16), so an
+# operand image the kernels forget to write shows up as NaN in the results.
+NAN = float("nan")
+
+
+@pytest.mark.parametrize("algo", ALGOS)
+def test_prefill_writes_exactly_its_outputs(algo):
+    lens = [65, 0, 130, 1, 64]
+    hv = 4
+    x = inputs.make_prefill(lens, hk=2, hv=hv, state_std=0.02, seed=61, device="cuda")
+    T, N = x["q"].shape[0], len(lens)
+    out_buf = torch.full((T + 2, hv, 128), NAN, dtype=x["v"].dtype, device="cuda")
+    fin_buf = torch.full((N + 2, hv, 128, 128), NAN, device="cuda")
+    out, fin = out_buf[1:T + 1], fin_buf[1:N + 1]
+    ws = gdn.alloc_workspace(gdn.prefill_shape(x["q"], x["v"], x["cu_seqlens"], algo), "cuda")
+    ws.fill_(0xFF)
+    try:
+        gdn.gdn_chunk_prefill(x["q"], x["k"], x["v"], x["g"], x["beta"], x["initial_state"],
+                              x["cu_seqlens"], out, fin, workspace=ws, algo=algo)
+    except gdn.GdnError as e:
+        if e.code == 9:
+            pytest.skip("algorithm not available for these inputs")
+        raise
+    torch.cuda.synchronize()
+    assert gdn.STATUS[gdn.gdn_get_device_error(ws)] == "GDN_OK"
+    for guard in (out_buf[0], out_buf[-1], fin_buf[0], fin_buf[-1]):
+        assert torch.isnan(guard).all(), "a write outside the output buffers"
+    assert torch.isfinite(out).all() and torch.isfinite(fin).all(), "an output element left unwritten"
+    o_ref, s_ref = oracle.forward(x["q"], x["k"], x["v"], x["g"], x["beta"], x["cu_seqlens"],
+                                  x["initial_state"])
+    assert_close(out, o_ref, TOL_BF16, "poisoned prefill out")
+    assert_close(fin, s_ref, TOL_BF16, "poisoned prefill state")
+
+
+@pytest.mark.parametrize("ntok", [1, 3, 4])
+def test_decode_and_verify_write_exactly_their_outputs(ntok):
+    N, hv = 6, 8
+    x = inputs.make_decode(N, ntok, hk=4, hv=hv, seed=62 + ntok, device="cuda")
+    st_buf = torch.full((N + 2, hv, 128, 128), NAN, device="cuda")
+    st_buf[1:N + 1] = x["state"]
+    out_buf = torch.full((N + 2, ntok, hv, 128), NAN, dtype=x["v"].dtype, device="cuda")
+    st, out = st_buf[1:N + 1], out_buf[1:N + 1]
+    gdn.gdn_decode_step(x["q"], x["k"], x["v"], x["g"], x["beta"], st, out)
+    torch.cuda.synchronize()
+    for guard in (st_buf[0], st_buf[-1], out_buf[0], out_buf[-1]):
+        assert torch.isnan(guard).all(), "a write outside the decode buffers"
+    assert torch.isfinite(out).all() and torch.isfinite(st).all()
+    o_ref, s_ref = oracle.decode(x["q"], x["k"], x["v"], x["g"], x["beta"], x["state"])
+    assert_close(out, o_ref, TOL_BF16, "poisoned decode out")
+    assert_close(st, s_ref, TOL_BF16, "poisoned decode state")
+    # verify: the snapshots too
+    snap_buf = torch.full((N + 2, ntok, hv, 128, 128), NAN, device="cuda")
+    out_buf.fill_(NAN)
+    snaps = snap_buf[1:N + 1]
+    gdn.gdn_decode_verify(x["q"], x["k"], x["v"], x["g"], x["beta"], x["state"], out, snaps)
+    torch.cuda.synchronize()
+    for guard in (snap_buf[0], snap_buf[-1], out_buf[0], out_buf[-1]):
+        assert torch.isnan(guard).all(), "a write outside the verify buffers"
+    assert torch.isfinite(snaps).all() and torch.isfinite(out).all()
+    assert_close(snaps[:, ntok - 1], s_ref, TOL_BF16, "poisoned verify last snapshot")
