@@ -95,7 +95,9 @@ gdn_status prefill_impl(const void* q, const void* k, const void* v, const float
     const bool tensor = use_tensor_path(shape);
     if (tensor && io != GDN_BF16) return GDN_ERR_UNSUPPORTED;
     cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
-    if (cudaMemsetAsync(workspace, 0, kHeaderBytes, s) != cudaSuccess) return GDN_ERR_CUDA;
+    // The tensor-core path's first kernel (the chunk table) clears the device error word
+    // itself; the fp32 path's header is cleared here.
+    if (!tensor && cudaMemsetAsync(workspace, 0, kHeaderBytes, s) != cudaSuccess) return GDN_ERR_CUDA;
     cudaError_t e;
     if (tensor) {
         e = gdn::launch_prefill_tc_prep(q, k, v, g, beta, cu_seqlens, shape->num_seqs,
@@ -214,7 +216,6 @@ gdn_status gdn_chunk_prefill_prep(const void* q, const void* k, const void* v, c
     for (const void* p : ptrs)
         if (p && !aligned16(p)) return GDN_ERR_ALIGN;
     cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
-    if (cudaMemsetAsync(workspace, 0, kHeaderBytes, s) != cudaSuccess) return GDN_ERR_CUDA;
     cudaError_t e = gdn::launch_prefill_tc_prep(q, k, v, g, beta, cu_seqlens, shape->num_seqs,
                                                 shape->total_tokens, shape->num_qk_heads,
                                                 shape->num_v_heads, workspace, s);

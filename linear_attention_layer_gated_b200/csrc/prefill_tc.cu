@@ -9,8 +9,9 @@
 //   Delta = U - W S^T,   O = diag(gam) Q S^T + P Delta,   S <- gam_L S + Delta^T diag(c) K
 //
 // Three kernels, all on the caller's stream:
-//  K0 chunk_table_kernel  cu_seqlens -> per-sequence first chunk id and a (seq, start,
-//                         length) entry per chunk, on the device (no host read).
+//  K0 chunk_table_kernel  clears the workspace's device error word; cu_seqlens -> per-sequence
+//                         first chunk id and a (seq, start, length) entry per chunk, on the
+//                         device (no host read).
 //  K1 chunk_prep_kernel   one CTA (256 threads) per (chunk, QK head), all chunks in
 //                         parallel, both V heads of the QK head:
 //                         - normalisation; Q K^T, K K^T and the cross Gram K K_prev^T with
@@ -89,6 +90,7 @@ __global__ void __launch_bounds__(1024)
 chunk_table_kernel(const int32_t* __restrict__ cu, int num_seqs, unsigned char* ws) {
     allow_dependent_launch();
     int32_t* header = reinterpret_cast<int32_t*>(ws);
+    if (threadIdx.x == 0) header[0] = 0;  // the device error word of this call
     const WsLayout L = ws_layout(num_seqs, 0, 1, 1);  // seq_chunk0 and table do not depend on T
     int32_t* seq_chunk0 = reinterpret_cast<int32_t*>(ws + L.seq_chunk0);
     int4* table = reinterpret_cast<int4*>(ws + L.table);
