@@ -35,6 +35,7 @@ def errs(x, ref):
 
 def assert_close(x, ref, tol, what):
     rel, mx = errs(x, ref)
+    print("%s: rel-L2 %.3e (tol %.0e), max-abs %.3e" % (what, rel, tol, mx))  # shown with pytest -rP
     assert np.isfinite(rel) and rel <= tol, "%s: rel-L2 %.3e (tol %.0e), max-abs %.3e" % (what, rel, tol, mx)
     return rel, mx
 
@@ -402,6 +403,7 @@ def test_long_context_split_carry_and_sampled_heads(algo):
         for a_, b_, what in ((out_s, out, "out"), (st, fin, "state")):
             rel = float(torch.linalg.vector_norm((a_.float() - b_.float()).flatten()) /
                         torch.linalg.vector_norm(b_.float().flatten()))
+            print("split vs whole %s: rel-L2 %.3e (tol %.0e)" % (what, rel, TOL_SPLIT))
             assert np.isfinite(rel) and rel <= TOL_SPLIT, "split vs whole %s: rel-L2 %.3e" % (what, rel)
     heads = [5]
     o_ref, s_ref, vh = oracle.forward_heads(x["q"], x["k"], x["v"], x["g"], x["beta"],
