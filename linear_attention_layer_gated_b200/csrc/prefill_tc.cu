@@ -96,11 +96,19 @@ chunk_table_kernel(const int32_t* __restrict__ cu, int num_seqs, unsigned char* 
     int4* table = reinterpret_cast<int4*>(ws + L.table);
     __shared__ int32_t scan[1024];
     __shared__ int32_t carry;
+    // up to 1024 sequences: chunk starts and cu_seqlens stay in shared memory for the entries
+    __shared__ int32_t start_s[1025], cu_s[1025];
+    const bool small = num_seqs <= 1024;
     if (threadIdx.x == 0) carry = 0;
     __syncthreads();
     for (int base = 0; base < num_seqs; base += 1024) {
         const int n = base + threadIdx.x;
-        const int cnt = (n < num_seqs) ? (cu[n + 1] - cu[n] + kChunk - 1) / kChunk : 0;
+        const int c0n = (n < num_seqs) ? cu[n] : 0, c1n = (n < num_seqs) ? cu[n + 1] : 0;
+        const int cnt = (n < num_seqs) ? (c1n - c0n + kChunk - 1) / kChunk : 0;
+        if (small && n < num_seqs) {
+            cu_s[n] = c0n;
+            if (n == num_seqs - 1) cu_s[num_seqs] = c1n;
+        }
         scan[threadIdx.x] = cnt;
         __syncthreads();
         for (int o = 1; o < 1024; o <<= 1) {  // inclusive Hillis-Steele scan
@@ -109,7 +117,10 @@ chunk_table_kernel(const int32_t* __restrict__ cu, int num_seqs, unsigned char* 
             scan[threadIdx.x] += add;
             __syncthreads();
         }
-        if (n < num_seqs) seq_chunk0[n] = carry + scan[threadIdx.x] - cnt;
+        if (n < num_seqs) {
+            seq_chunk0[n] = carry + scan[threadIdx.x] - cnt;
+            if (small) start_s[n] = carry + scan[threadIdx.x] - cnt;
+        }
         __syncthreads();
         if (threadIdx.x == 1023) carry += scan[1023];
         __syncthreads();
@@ -117,19 +128,22 @@ chunk_table_kernel(const int32_t* __restrict__ cu, int num_seqs, unsigned char* 
     if (threadIdx.x == 0) {
         seq_chunk0[num_seqs] = carry;
         header[1] = carry;
+        if (small) start_s[num_seqs] = carry;
     }
     __syncthreads();
     // one entry per thread: chunk c belongs to the last sequence n with seq_chunk0[n] <= c
     const int total = carry;
+    const int32_t* starts = small ? start_s : seq_chunk0;
+    const int32_t* cus = small ? cu_s : cu;
     for (int c = threadIdx.x; c < total; c += blockDim.x) {
         int lo = 0, hi = num_seqs - 1;
         while (lo < hi) {
             const int mid = (lo + hi + 1) >> 1;
-            if (seq_chunk0[mid] <= c) lo = mid;
+            if (starts[mid] <= c) lo = mid;
             else hi = mid - 1;
         }
-        const int n = lo, kk = c - seq_chunk0[n];
-        const int t0 = cu[n], len = cu[n + 1] - t0;
+        const int n = lo, kk = c - starts[n];
+        const int t0 = cus[n], len = cus[n + 1] - t0;
         table[c] = make_int4(n, t0 + kk * kChunk, min(kChunk, len - kk * kChunk), 0);
     }
 }
@@ -157,12 +171,6 @@ __device__ __forceinline__ float sum8(float x) {  // over groups of 8 consecutiv
     x += __shfl_xor_sync(0xffffffffu, x, 4);
     x += __shfl_xor_sync(0xffffffffu, x, 2);
     x += __shfl_xor_sync(0xffffffffu, x, 1);
-    return x;
-}
-
-__device__ __forceinline__ float warp_sum(float x) {
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) x += __shfl_xor_sync(0xffffffffu, x, o);
     return x;
 }
 
@@ -900,15 +908,15 @@ chunk_state_kernel(const float* s0, const int32_t* __restrict__ cu, __nv_bfloat1
     const int n = (blockIdx.x / kSlices) / hv;
     const int jq = h / (hv / hk);
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-    grid_dependency_wait();  // the prep kernel's workspace is complete and visible
-    const int32_t* seq_chunk0 = reinterpret_cast<const int32_t*>(ws + L.seq_chunk0);
-    const int cs = seq_chunk0[n], nch = seq_chunk0[n + 1] - cs;
-    const int t_begin = cu[n], t_end = cu[n + 1];
     if (sb & 1023u) {  // the swizzled operand layouts need a 1024-byte-aligned base
+        grid_dependency_wait();
         if (tid == 0) atomicOr(header, 2);
         return;
     }
 
+    // Set-up that needs nothing from the prep kernel runs before the dependency wait (a
+    // CTA of this kernel never shares an SM with a prep CTA: their shared memory does not
+    // fit together, so the Tensor Memory columns are free).
     if (warp == 0) {
         tmem_alloc(&ss.tmem_base, kTmemCols);
         tmem_relinquish();
@@ -931,6 +939,10 @@ chunk_state_kernel(const float* s0, const int32_t* __restrict__ cu, __nv_bfloat1
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = ss.tmem_base;
+    grid_dependency_wait();  // the prep kernel's workspace is complete and visible
+    const int32_t* seq_chunk0 = reinterpret_cast<const int32_t*>(ws + L.seq_chunk0);
+    const int cs = seq_chunk0[n], nch = seq_chunk0[n + 1] - cs;
+    const int t_begin = cu[n], t_end = cu[n + 1];
 
     if (warp == kIssuerWarp) {
         // ------------------------------------------------ MMA issuer
