@@ -489,3 +489,21 @@ def test_decode_and_verify_write_exactly_their_outputs(ntok):
         assert torch.isnan(guard).all(), "a write outside the verify buffers"
     assert torch.isfinite(snaps).all() and torch.isfinite(out).all()
     assert_close(snaps[:, ntok - 1], s_ref, TOL_BF16, "poisoned verify last snapshot")
+
+
+@pytest.mark.parametrize("algo", ALGOS)
+def test_prefill_more_than_1024_sequences(algo):
+    """More sequences than one thread block of the chunk-table scan covers: the scan runs
+    in several batches with a carry, and the chunk entries are found in global memory."""
+    gen = np.random.default_rng(70)
+    lens = [int(x) for x in gen.integers(0, 140, size=1100)]
+    lens[5] = 0
+    lens[1023] = 64
+    x = inputs.make_prefill(lens, hk=2, hv=4, state_std=0.02, seed=71, device="cuda")
+    o_ref, s_ref = oracle.forward(x["q"], x["k"], x["v"], x["g"], x["beta"], x["cu_seqlens"],
+                                  x["initial_state"])
+    out, fin = run_prefill(x, algo)
+    torch.cuda.synchronize()
+    assert_close(out, o_ref, TOL_BF16, "1100 sequences out")
+    assert_close(fin, s_ref, TOL_BF16, "1100 sequences final state")
+    torch.testing.assert_close(fin[5], x["initial_state"][5], rtol=0, atol=0)
