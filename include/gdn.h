@@ -267,10 +267,15 @@ gdn_status gdn_get_device_error(void *workspace, void *stream);
  *     one sequence of up to 1,728 tokens); fp32 I/O or GDN_ALGO_SIMT give
  *     GDN_ERR_UNSUPPORTED.
  *   - The first call on each device (with that device current) looks up the array's
- *     device address once and caches it; make that first call before any stream capture.
+ *     device address and caches it with the identity of the device's current context;
+ *     make that first call before any stream capture.  If the context changes (after
+ *     cudaDeviceReset, for instance) the next call looks the address up again, so make
+ *     the first call after a reset before any capture as well.
  *   - Every call on a device shares the one array, which keeps the previous call's
  *     contents; each call clears what must start at zero.  Calls that overlap on the GPU
  *     (e.g. on unordered streams) race on the array.
+ *   - A bounded device wait that gave up is recorded in the array's header; read it with
+ *     gdn_get_noalloc_device_error.
  */
 #define GDN_NOALLOC_SCRATCH_BYTES ((size_t)64 << 20)
 gdn_status gdn_chunk_prefill_noalloc(const void *q, const void *k, const void *v,
@@ -278,6 +283,15 @@ gdn_status gdn_chunk_prefill_noalloc(const void *q, const void *k, const void *v
                                      const float *initial_state, const int32_t *cu_seqlens,
                                      void *out, float *final_state, const gdn_shape *shape,
                                      void *stream);
+
+/*
+ * The device error word of gdn_chunk_prefill_noalloc's static scratch on the current
+ * device (its callers never see the array's address, so gdn_get_device_error cannot be
+ * given it).  Synchronises `stream` and returns GDN_ERR_DEVICE_TIMEOUT if a bounded
+ * device wait of the last allocation-free prefill on this device gave up, GDN_ERR_CUDA
+ * if the runtime reports an error, else GDN_OK.  Meant for tests and debugging.
+ */
+gdn_status gdn_get_noalloc_device_error(void *stream);
 
 /*
  * Failure-path self-test.  Clears the workspace header, then launches a kernel that waits

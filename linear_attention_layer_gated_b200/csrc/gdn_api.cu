@@ -2,8 +2,9 @@
 // dispatch on the caller's stream.  Declarations and contracts are in include/gdn.h.
 //
 // Nothing here allocates, synchronises or reads device memory inside the prefill and
-// decode entry points, so both are stream-ordered and graph-capturable; the only
-// device-side work besides kernels is a 256-byte memset of the workspace header.
+// decode entry points, so both are stream-ordered and graph-capturable.  On the
+// tensor-core prefill path every piece of device work is a kernel (its first kernel
+// clears the workspace header); the fp32 path clears the 256-byte header with a memset.
 #include <cstdint>
 #include <cstring>
 

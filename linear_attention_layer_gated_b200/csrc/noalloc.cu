@@ -11,15 +11,20 @@
 //
 // The array's name is only a host-side stand-in in host code, not a device address, so
 // the first call on each device (with that device current) looks up its real address
-// with cudaGetSymbolAddress and caches it; later calls on that device reuse it.  That
-// first call therefore does a little one-time set-up work and should come before any
-// stream capture.
+// with cudaGetSymbolAddress and caches it together with the identity of the device's
+// current context; later calls in the same context reuse it.  When the context changes
+// (cudaDeviceReset, or the primary context released and created again, reloads the
+// library's device code, so the array may sit elsewhere) the next call looks the address
+// up again.  The first call in a context therefore does a little one-time set-up work and
+// should come before any stream capture.
 //
 // All calls on a device share the one array and it keeps the previous call's contents.
 // The prefill clears what must start at zero (the header with the device error word)
 // on every call, and everything else is written before it is read.  Calls whose
 // executions overlap on the GPU (different streams, no ordering between them) race on
 // the array; order them on one stream or with events.
+#include <cuda.h>
+
 #include <mutex>
 
 #include "gdn_internal.cuh"
@@ -31,21 +36,57 @@ constexpr int kMaxDevices = 64;
 
 static __device__ __align__(256) unsigned char g_prefill_scratch[kScratchBytes];
 
-std::mutex g_mutex;
-void* g_scratch_ptr[kMaxDevices] = {};
+struct CachedAddress {
+    unsigned long long ctx_id;  // unique id of the context the address was taken in
+    void* ptr;
+};
 
-// Device address of g_prefill_scratch on the current device (set up once per device).
+std::mutex g_mutex;
+CachedAddress g_cache[kMaxDevices] = {};
+
+using CtxGetCurrentFn = CUresult (*)(CUcontext*);
+using CtxGetIdFn = CUresult (*)(CUcontext, unsigned long long*);
+
+// Unique id of the calling thread's current context (CUDA 12 context ids are never reused
+// within a process), or 0 if the driver cannot tell; 0 makes every call look the address up.
+unsigned long long current_context_id() {
+    static CtxGetCurrentFn get_current = nullptr;
+    static CtxGetIdFn get_id = nullptr;
+    static std::once_flag once;
+    std::call_once(once, [] {
+        void* f = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuCtxGetCurrent", &f, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            get_current = reinterpret_cast<CtxGetCurrentFn>(f);
+        f = nullptr;
+        if (cudaGetDriverEntryPoint("cuCtxGetId", &f, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            get_id = reinterpret_cast<CtxGetIdFn>(f);
+    });
+    if (!get_current || !get_id) return 0;
+    CUcontext ctx = nullptr;
+    unsigned long long id = 0;
+    if (get_current(&ctx) != CUDA_SUCCESS || !ctx || get_id(ctx, &id) != CUDA_SUCCESS) return 0;
+    return id;
+}
+
+// Device address of g_prefill_scratch on the current device, in its current context.
 gdn_status scratch_address(void** out) {
     int dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess) return GDN_ERR_CUDA;
     if (dev < 0 || dev >= kMaxDevices) return GDN_ERR_UNSUPPORTED;
     std::lock_guard<std::mutex> lock(g_mutex);
-    if (!g_scratch_ptr[dev]) {
+    CachedAddress& c = g_cache[dev];
+    unsigned long long id = current_context_id();
+    if (!c.ptr || id == 0 || id != c.ctx_id) {
         void* p = nullptr;
         if (cudaGetSymbolAddress(&p, g_prefill_scratch) != cudaSuccess || !p) return GDN_ERR_CUDA;
-        g_scratch_ptr[dev] = p;
+        if (id == 0) id = current_context_id();  // the lookup may have created the context
+        c.ptr = p;
+        c.ctx_id = id;
     }
-    *out = g_scratch_ptr[dev];
+    *out = c.ptr;
     return GDN_OK;
 }
 
@@ -67,4 +108,13 @@ extern "C" gdn_status gdn_chunk_prefill_noalloc(const void* q, const void* k, co
     if (st != GDN_OK) return st;
     return gdn_chunk_prefill(q, k, v, g, beta, initial_state, cu_seqlens, out, final_state, shape,
                              scratch, kScratchBytes, stream);
+}
+
+// The device error word of the static scratch: the caller of gdn_chunk_prefill_noalloc
+// never sees the array's address, so it cannot pass it to gdn_get_device_error.
+extern "C" gdn_status gdn_get_noalloc_device_error(void* stream) {
+    void* scratch = nullptr;
+    const gdn_status st = scratch_address(&scratch);
+    if (st != GDN_OK) return st;
+    return gdn_get_device_error(scratch, stream);
 }

@@ -27,7 +27,8 @@ EXPORTED = ["gdn_prefill_workspace_bytes", "gdn_chunk_prefill", "gdn_chunk_prefi
             "gdn_selftest_wait_timeout", "gdn_status_string", "gdn_abi_version",
             "gdn_chunk_prefill_noalloc", "gdn_decode_verify", "gdn_decode_commit",
             "gdn_chunk_prefill_slots", "gdn_decode_step_slots", "gdn_decode_verify_slots",
-            "gdn_decode_commit_slots", "gdn_chunk_prefill_chunk_states"]
+            "gdn_decode_commit_slots", "gdn_chunk_prefill_chunk_states",
+            "gdn_get_noalloc_device_error"]
 
 
 class GdnShape(ctypes.Structure):
@@ -90,6 +91,8 @@ def lib() -> ctypes.CDLL:
             L.gdn_get_device_error.argtypes = [vp, vp]
             L.gdn_chunk_prefill_noalloc.restype = ctypes.c_int
             L.gdn_chunk_prefill_noalloc.argtypes = [vp, vp, vp, fp, fp, fp, ip, vp, fp, sp, vp]
+            L.gdn_get_noalloc_device_error.restype = ctypes.c_int
+            L.gdn_get_noalloc_device_error.argtypes = [vp]
             L.gdn_selftest_wait_timeout.restype = ctypes.c_int
             L.gdn_selftest_wait_timeout.argtypes = [vp, ctypes.c_size_t, ctypes.c_uint32, vp]
             L.gdn_status_string.restype = ctypes.c_char_p
@@ -312,6 +315,12 @@ def gdn_chunk_prefill_noalloc(q, k, v, g, beta, initial_state, cu_seqlens, out, 
                                          _ptr(final_state), ctypes.byref(shape), _stream(stream))
     if rc != GDN_OK:
         raise GdnError(rc, "gdn_chunk_prefill_noalloc")
+
+
+def gdn_get_noalloc_device_error(stream=None) -> int:
+    """Calls gdn_get_noalloc_device_error: the device error word of the static scratch
+    the allocation-free prefill uses on the current device."""
+    return int(lib().gdn_get_noalloc_device_error(_stream(stream)))
 
 
 def gdn_selftest_wait_timeout(workspace, limit_us=20000, stream=None):

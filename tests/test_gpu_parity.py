@@ -3,7 +3,9 @@ seeded inputs.
 
 Tolerances are relative L2 errors over whole flattened tensors, computed separately
 for outputs and states: <= 1e-4 for fp32 I/O (fp32 arithmetic throughout), <= 1e-2 for
-bf16 I/O with fp32 state.  Max-abs error is reported in the assertion message.
+bf16 I/O with fp32 state.  Max-abs error is reported in the assertion message.  The
+full-size tests also bound every row (token and V head of the output, sequence and V
+head of the state) on its own, so that a few wrong rows cannot hide in the norm.
 Full-size workloads compare a sample of heads: every (sequence, V head) recurrence is
 independent, so the oracle on a subset of QK heads (and the V heads that read them) is
 an exact sample of the full result.
@@ -15,29 +17,14 @@ import torch
 
 import oracle
 from linear_attention_layer_gated_b200 import gdn, inputs
+from parity_util import TOL_BF16, TOL_F32, TOL_ROW_BF16, assert_close, assert_rows_close, errs  # noqa: F401
 
 pytestmark = pytest.mark.gpu
 
-TOL_F32 = 1e-4
-TOL_BF16 = 1e-2
 # Two tensor-core runs of the same inputs that differ only in where the bf16 operands are
 # rounded (split vs whole sequence): an order of magnitude inside the bf16 tolerance.
 TOL_SPLIT = 1e-3
 ALGOS = [gdn.GDN_ALGO_SIMT, gdn.GDN_ALGO_TENSOR]
-
-
-def errs(x, ref):
-    x = x.detach().double().cpu().numpy() if hasattr(x, "detach") else np.asarray(x, np.float64)
-    ref = np.asarray(ref, np.float64)
-    rel = float(np.linalg.norm(x - ref) / max(np.linalg.norm(ref), 1e-300))
-    return rel, float(np.max(np.abs(x - ref))) if x.size else 0.0
-
-
-def assert_close(x, ref, tol, what):
-    rel, mx = errs(x, ref)
-    print("%s: rel-L2 %.3e (tol %.0e), max-abs %.3e" % (what, rel, tol, mx))  # shown with pytest -rP
-    assert np.isfinite(rel) and rel <= tol, "%s: rel-L2 %.3e (tol %.0e), max-abs %.3e" % (what, rel, tol, mx)
-    return rel, mx
 
 
 def run_prefill(x, algo, want_final=True):
@@ -70,6 +57,8 @@ def test_decode_full_batch_matches_oracle(ntok):
     torch.cuda.synchronize()
     assert_close(out, o_ref, TOL_BF16, "decode out ntok=%d" % ntok)
     assert_close(st, sn_ref, TOL_BF16, "decode state ntok=%d" % ntok)
+    assert_rows_close(out, o_ref, 3, TOL_ROW_BF16, "decode out rows ntok=%d" % ntok)
+    assert_rows_close(st, sn_ref, 2, TOL_ROW_BF16, "decode state rows ntok=%d" % ntok)
 
 
 def test_decode_fp32_io_tight():
@@ -135,10 +124,14 @@ def test_commit_installs_the_accepted_snapshot():
 
 # ------------------------------------------------------------------ state-slot indirection
 def _slot_table(n, num_slots, seed):
-    """Distinct slots for n sequences from a pool of num_slots, every 5th one invalid."""
+    """Distinct slots for n sequences from a pool of num_slots (a permutation, so the pool
+    order differs from the sequence order); every 5th one is outside [0, num_slots) in one
+    of three ways: -1, num_slots itself, or far beyond it."""
     gen = torch.Generator().manual_seed(seed)
     slots = torch.randperm(num_slots, generator=gen)[:n].to(torch.int32)
-    slots[::5] = -1
+    bad = [-1, num_slots, num_slots + 1000]
+    for i, j in enumerate(range(0, n, 5)):
+        slots[j] = bad[i % 3]
     return slots.cuda()
 
 
@@ -147,7 +140,7 @@ def test_decode_verify_commit_through_slots_match_dense():
     x = inputs.make_decode(N, ntok, hk=4, hv=8, seed=50, device="cuda")
     pool = torch.randn(S, 8, 128, 128, device="cuda") * 0.02
     slots = _slot_table(N, S, 51)
-    valid = slots >= 0
+    valid = (slots >= 0) & (slots < S)
     dense = torch.zeros_like(x["state"])
     dense[valid] = pool[slots[valid].long()]
     # decode step in place on the pool
@@ -159,6 +152,12 @@ def test_decode_verify_commit_through_slots_match_dense():
     torch.cuda.synchronize()
     torch.testing.assert_close(out_s[valid], out_d[valid], rtol=0, atol=0)
     assert torch.isnan(out_s[~valid]).all()  # sequences without a slot are skipped
+    # against the definition: the oracle run on the states the slot table names
+    sel = lambda a: a[valid]  # noqa: E731
+    o_ref, s_ref = oracle.decode(sel(x["q"]), sel(x["k"]), sel(x["v"]), sel(x["g"]), sel(x["beta"]),
+                                 pool[slots[valid].long()])
+    assert_close(out_s[valid], o_ref, TOL_BF16, "decode through slots out vs oracle")
+    assert_close(p1[slots[valid].long()], s_ref, TOL_BF16, "decode through slots state vs oracle")
     torch.testing.assert_close(p1[slots[valid].long()], d1[valid], rtol=0, atol=0)
     untouched = torch.ones(S, dtype=torch.bool, device="cuda")
     untouched[slots[valid].long()] = False
@@ -175,7 +174,7 @@ def test_decode_verify_commit_through_slots_match_dense():
     torch.cuda.synchronize()
     for n in range(N):
         a, sl = int(accepted[n]), int(slots[n])
-        if sl < 0:
+        if not 0 <= sl < S:
             continue
         want = snaps[n, a - 1] if a >= 1 else pool[sl]
         torch.testing.assert_close(p2[sl], want, rtol=0, atol=0)
@@ -188,7 +187,7 @@ def test_prefill_through_slots_matches_dense(algo):
     N, S = len(lens), 16
     pool = torch.randn(S, 4, 128, 128, device="cuda") * 0.02
     slots = _slot_table(N, S, 53)
-    valid = slots >= 0
+    valid = (slots >= 0) & (slots < S)
     init = torch.zeros(N, 4, 128, 128, device="cuda")
     init[valid] = pool[slots[valid].long()]
     out_d, fin_d = run_prefill(dict(x, initial_state=init), algo)
@@ -204,6 +203,12 @@ def test_prefill_through_slots_matches_dense(algo):
     torch.cuda.synchronize()
     torch.testing.assert_close(out_s, out_d, rtol=0, atol=0)
     torch.testing.assert_close(p1[slots[valid].long()], fin_d[valid], rtol=0, atol=0)
+    # against the definition: sequences with a slot start from the pool row it names,
+    # the others from zeros
+    o_ref, s_ref = oracle.forward(x["q"], x["k"], x["v"], x["g"], x["beta"], x["cu_seqlens"], init)
+    tol = TOL_F32 if x["q"].dtype == torch.float32 else TOL_BF16
+    assert_close(out_s, o_ref, tol, "prefill through slots out vs oracle")
+    assert_close(p1[slots[valid].long()], s_ref[valid.cpu().numpy()], tol, "prefill through slots state vs oracle")
     untouched = torch.ones(S, dtype=torch.bool, device="cuda")
     untouched[slots[valid].long()] = False
     torch.testing.assert_close(p1[untouched], pool[untouched], rtol=0, atol=0)
@@ -360,6 +365,8 @@ def test_layer_prefill_8192_sampled_heads(algo):
                                             x["cu_seqlens"], heads)
     assert_close(out[:, vh], o_ref, TOL_BF16, "T=8192 out (sampled heads)")
     assert_close(fin[:, vh], s_ref, TOL_BF16, "T=8192 state (sampled heads)")
+    assert_rows_close(out[:, vh], o_ref, 2, TOL_ROW_BF16, "T=8192 out rows")
+    assert_rows_close(fin[:, vh], s_ref, 2, TOL_ROW_BF16, "T=8192 state rows")
 
 
 @pytest.mark.parametrize("algo", ALGOS)
@@ -373,6 +380,8 @@ def test_varlen_8_sequences_sampled_heads(algo):
                                             x["cu_seqlens"], heads, x["initial_state"])
     assert_close(out[:, vh], o_ref, TOL_BF16, "varlen out (sampled heads)")
     assert_close(fin[:, vh], s_ref, TOL_BF16, "varlen state (sampled heads)")
+    assert_rows_close(out[:, vh], o_ref, 2, TOL_ROW_BF16, "varlen out rows")
+    assert_rows_close(fin[:, vh], s_ref, 2, TOL_ROW_BF16, "varlen state rows (sequence, head)")
 
 
 @pytest.mark.parametrize("algo", ALGOS)
@@ -410,6 +419,8 @@ def test_long_context_split_carry_and_sampled_heads(algo):
                                             x["cu_seqlens"], heads)
     assert_close(out[:, vh], o_ref, TOL_BF16, "T=262144 out (sampled heads)")
     assert_close(fin[:, vh], s_ref, TOL_BF16, "T=262144 state (sampled heads)")
+    assert_rows_close(out[:, vh], o_ref, 2, TOL_ROW_BF16, "T=262144 out rows")
+    assert_rows_close(fin[:, vh], s_ref, 2, TOL_ROW_BF16, "T=262144 state rows")
 
 
 def test_bounded_wait_expiry_is_reported_and_context_survives():

@@ -348,3 +348,38 @@ def test_pins_reject_planted_mistakes():
     for t in range(T):
         M = M @ (np.exp(g[t]) * (np.eye(d) - b[t] * np.outer(k[t], k[t])))
     assert np.max(np.abs((s_with - s_zero) - S0 @ M)) > 1e-3
+
+
+# ------------------- the head-subset oracle (checker of the full-size GPU parity tests)
+def _forward_heads_wrong_grouping(q, k, v, g, b, cu, qk_heads, s0):
+    """A plausible bug planted on the CPU: the V heads of QK head j listed as j + r * HK
+    (strided) instead of the contiguous j * group + r."""
+    HK, HV = q.shape[1], v.shape[1]
+    vh = [j + r * HK for j in qk_heads for r in range(HV // HK)]
+    out, fin = oracle.forward(q[:, list(qk_heads)], k[:, list(qk_heads)], v[:, vh], g[:, vh],
+                              b[:, vh], cu, s0[:, vh])
+    return out, fin, vh
+
+
+@pytest.mark.parametrize("qk_heads", [[0], [2, 1], [3, 0, 2], [0, 1, 2, 3]])
+def test_forward_heads_is_an_exact_sample_of_forward(qk_heads):
+    """forward_heads on a subset of QK heads returns exactly the columns of the full
+    oracle for the V heads that read those QK heads (contiguous groups, R3), in the
+    order of the QK heads given, with their initial and final states."""
+    r = rng(120)
+    lens = [23, 0, 41, 9]
+    T, HK, HV, d = sum(lens), 4, 8, 16
+    cu = np.concatenate([[0], np.cumsum(lens)]).astype(np.int32)
+    q, k = r.standard_normal((T, HK, d)), r.standard_normal((T, HK, d))
+    v = r.standard_normal((T, HV, d))
+    g, b = -r.uniform(0, 0.3, (T, HV)), r.uniform(0.05, 0.95, (T, HV))
+    s0 = r.standard_normal((len(lens), HV, d, d)) * 0.1
+    out, fin = oracle.forward(q, k, v, g, b, cu, s0)
+    o_s, f_s, vh = oracle.forward_heads(q, k, v, g, b, cu, qk_heads, s0)
+    assert vh == [2 * j + rr for j in qk_heads for rr in range(2)]
+    np.testing.assert_array_equal(o_s, out[:, vh])
+    np.testing.assert_array_equal(f_s, fin[:, vh])
+    # the same comparison rejects a strided listing of the V heads
+    if qk_heads != [0]:
+        o_w, f_w, vh_w = _forward_heads_wrong_grouping(q, k, v, g, b, cu, qk_heads, s0)
+        assert np.max(np.abs(o_w - out[:, [2 * j + rr for j in qk_heads for rr in range(2)]])) > 1e-3

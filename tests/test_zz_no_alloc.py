@@ -24,6 +24,10 @@ def rel_l2(x, ref):
     return float(np.linalg.norm(x - ref) / np.linalg.norm(ref))
 
 
+def stream_handle():
+    return torch.cuda.current_stream().cuda_stream
+
+
 def run_noalloc(L, x, out, fin):
     shape = gdn.prefill_shape(x["q"], x["v"], x["cu_seqlens"])
     stream = torch.cuda.current_stream().cuda_stream
@@ -43,6 +47,8 @@ def test_noalloc_prefill_matches_workspace_prefill_twice_in_a_row():
         out = torch.full_like(x["v"], float("nan"))
         fin = torch.full_like(x["initial_state"], float("nan"))
         assert run_noalloc(L, x, out, fin) == gdn.GDN_OK
+        # no bounded device wait of this call gave up (the word lives in the static scratch)
+        assert gdn.STATUS[L.gdn_get_noalloc_device_error(stream_handle())] == "GDN_OK"
         ref_out, ref_fin = gdn.prefill(x["q"], x["k"], x["v"], x["g"], x["beta"],
                                        x["cu_seqlens"], x["initial_state"])
         torch.cuda.synchronize()
