@@ -37,29 +37,48 @@ UNIT = "tokens/s"
 WORKLOAD = "layer_prefill"
 HK, HV, D, C = 16, 32, 128, 64
 
-# Algorithmic work per token of prefill (GEMM flops of the chunked form) and bytes.
+# Algorithmic work of the method (what any implementation must do; no intermediate of
+# ours is counted).  Prefill reads q, k (bf16, per QK head), v (bf16) and g, beta (fp32,
+# per V head) once, writes out (bf16) once, and reads / writes each sequence's fp32 state
+# once when an initial / final state is given.  GEMM flops are those of the chunked form.
+INPUT_BYTES_PER_TOKEN = 2 * HK * D * 2 + HV * D * 2 + 2 * HV * 4                      # 16,640
+OUTPUT_BYTES_PER_TOKEN = HV * D * 2                                                   # 8,192
+PREFILL_BYTES_PER_TOKEN = INPUT_BYTES_PER_TOKEN + OUTPUT_BYTES_PER_TOKEN              # 24,832
 PREFILL_FLOP_PER_TOKEN = HV * (3 * 2 * C * D + 3 * 2 * D * D) + HK * (2 * 2 * C * D)  # 5,242,880
-PREFILL_BYTES_PER_TOKEN = 2 * HK * D * 2 + HV * D * 2 * 2 + HV * 4 * 2                # 24,832
 STATE_BYTES = HV * D * D * 4                                                          # per sequence
-# Split of the GEMM flops between the two tensor-core phases:
-#   prep  = Gram matrices (per QK head) + W and U (per V head)
-#   state = [W; Q] S^T, P Delta and the state update (per V head)
+# The two tensor-core phases split that work:
+#   prep  = Gram matrices (per QK head) and W, U (per V head); reads every input
+#   state = [W; Q] S^T, P Delta and the state update (per V head); writes every output and
+#           reads / writes the states
 PREP_FLOP_PER_TOKEN = HK * (2 * 2 * C * D) + HV * (2 * 2 * C * D)                    # 1,572,864
 STATE_FLOP_PER_TOKEN = HV * (2 * C * D + 3 * 2 * D * D)                               # 3,670,016
-# Algorithmic HBM bytes per full 64-token chunk of each tensor-core phase (the roofline
-# of both phases is the HBM one: their flop/byte ratios, about 30 and 90, are far below
-# the B200's bf16 ridge point).
-#   prep  reads q, k (bf16, per QK head), v (bf16), g, beta (fp32, per V head) once and
-#         writes the chunk's operand images: per V head W~ and U (64 x 128 bf16 each),
-#         P and M~ (64 x 64 bf16 each), diag(c) K (64 x 128 bf16) and the gate factors
-#         (129 fp32); per QK head the normalised Q (64 x 128 bf16).
-#   state reads those images once (Q, W~, M~, P, diag(c) K, U, gate factors) and writes
-#         the outputs (64 x 128 bf16 per V head); the state itself enters and leaves once
-#         per sequence (fp32, counted separately).
-PREP_BYTES_PER_CHUNK = (C * (2 * HK * D * 2 + HV * D * 2 + HV * 4 * 2)
-                        + HV * (3 * C * D * 2 + 2 * C * C * 2 + 129 * 4) + HK * C * D * 2)   # 3,440,768
-STATE_BYTES_PER_CHUNK = (HK * C * D * 2 + HV * (3 * C * D * 2 + 2 * C * C * 2 + 129 * 4)
-                         + HV * C * D * 2)                                                  # 2,900,096
+
+
+def prefill_work(T, N, with_initial, with_final):
+    """Algorithmic (bytes, flop) of one prefill of T packed tokens in N sequences."""
+    nbytes = T * PREFILL_BYTES_PER_TOKEN + N * STATE_BYTES * (int(with_initial) + int(with_final))
+    return nbytes, T * PREFILL_FLOP_PER_TOKEN
+
+
+def phase_work(T, N, with_initial, with_final):
+    """Algorithmic (bytes, flop) of each tensor-core phase: prep reads the inputs, state
+    writes the outputs and moves the states."""
+    return {"prep": (T * INPUT_BYTES_PER_TOKEN, T * PREP_FLOP_PER_TOKEN),
+            "state": (T * OUTPUT_BYTES_PER_TOKEN + N * STATE_BYTES * (int(with_initial) + int(with_final)),
+                      T * STATE_FLOP_PER_TOKEN)}
+
+
+def roofline_of(nbytes, flop, ms, peaks):
+    """Achieved rates of a kernel (or step) against both peaks; its bound is the one its
+    arithmetic intensity selects (tensor above the ridge point flop/byte, HBM below)."""
+    s = ms * 1e-3
+    gbs, tflops = nbytes / s / 1e9, flop / s / 1e12
+    ridge = peaks["bf16_tflops"] * 1e12 / (peaks["hbm_gbs"] * 1e9)
+    bound = "tensor" if nbytes == 0 or flop / nbytes >= ridge else "hbm"
+    r = {"gbs": gbs, "tflops": tflops, "frac_hbm": gbs / peaks["hbm_gbs"],
+         "frac_tensor": tflops / peaks["bf16_tflops"], "bound": bound,
+         "intensity_flop_per_byte": flop / nbytes if nbytes else None, "ridge_flop_per_byte": ridge}
+    return r
 
 
 def decode_bytes(num_seqs, ntok):
@@ -232,36 +251,7 @@ def main_ours(args, rank, world, local_rank):
     stream = torch.cuda.current_stream(dev)
     algo = {"auto": gdn.GDN_ALGO_AUTO, "simt": gdn.GDN_ALGO_SIMT,
             "tensor": gdn.GDN_ALGO_TENSOR}[args.algo]
-
-    w = inputs.workload(WORKLOAD)
-    if args.tokens:
-        w.seqlens = [args.tokens]
-    x = inputs.make(w, device=dev)
-    T = x["q"].shape[0]
-    out = torch.empty_like(x["v"])
-    fin = torch.empty((1, HV, D, D), dtype=torch.float32, device=dev)
-    shape = gdn.prefill_shape(x["q"], x["v"], x["cu_seqlens"], algo)
-    ws = gdn.alloc_workspace(shape, dev)
     flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
-
-    tensor_path = gdn_launches_per_prefill(algo, x["q"].dtype) == 3
-    phase_ev = []
-
-    def prefill_once():
-        gdn.gdn_chunk_prefill(x["q"], x["k"], x["v"], x["g"], x["beta"], None, x["cu_seqlens"],
-                              out, fin, workspace=ws, algo=algo, stream=stream)
-
-    def prefill_phased():
-        # the same two launches gdn_chunk_prefill makes, with events between them
-        e = [torch.cuda.Event(enable_timing=True) for _ in range(3)]
-        e[0].record(stream)
-        gdn.gdn_chunk_prefill_prep(x["q"], x["k"], x["v"], x["g"], x["beta"], x["cu_seqlens"],
-                                   ws, algo=algo, stream=stream)
-        e[1].record(stream)
-        gdn.gdn_chunk_prefill_state(None, x["cu_seqlens"], out, fin, ws, x["q"], algo=algo,
-                                    stream=stream)
-        e[2].record(stream)
-        phase_ev.append(e)
 
     def barrier():
         replicas.barrier(world)
@@ -285,55 +275,127 @@ def main_ours(args, rank, world, local_rank):
     def max_over_ranks(v):
         return replicas.max_over_ranks(v, world, device=dev)
 
-    # the step as a user runs it: one gdn_chunk_prefill call
-    with ClockSampler(local_rank) as clk:
-        ms = timed(prefill_once, args.steps, args.warmup)
-    clocks = clk.summary()
-    if tensor_path:  # the same launches with events between them, for the phase rooflines
-        timed(prefill_phased, args.steps, args.warmup)
-    ms_step = max_over_ranks(sum(ms) / len(ms))
-    value = replicas.job_throughput(T, world, ms_step * 1e-3)
+    def prefill_step_fn(x, out, fin, ws, with_initial, segments=1):
+        """One step: gdn_chunk_prefill over the workload, or over `segments` equal pieces of
+        its single sequence with the state carried in place from one call to the next."""
+        s0 = x["initial_state"] if with_initial else None
+        if segments == 1:
+            return lambda: gdn.gdn_chunk_prefill(x["q"], x["k"], x["v"], x["g"], x["beta"], s0,
+                                                 x["cu_seqlens"], out, fin, workspace=ws, algo=algo,
+                                                 stream=stream)
+        T = x["q"].shape[0]
+        seg = T // segments
+        cu = torch.tensor([0, seg], dtype=torch.int32, device=dev)
+        views = [{k2: x[k2][i * seg:(i + 1) * seg] for k2 in ("q", "k", "v", "g", "beta")}
+                 for i in range(segments)]
+        outs = [out[i * seg:(i + 1) * seg] for i in range(segments)]
 
-    # ---- dominant kernel roofline, from CUDA events on the launching stream
+        def run():
+            for i in range(segments):
+                v = views[i]
+                gdn.gdn_chunk_prefill(v["q"], v["k"], v["v"], v["g"], v["beta"], s0 if i == 0 else fin,
+                                      cu, outs[i], fin, workspace=ws, algo=algo, stream=stream)
+        return run
+
+    tensor_path = gdn_launches_per_prefill(algo, torch.bfloat16) == 3
+
+    def measure_prefill(w, steps, warmup, with_initial, segments=1, phased=False, clocks=False):
+        """Times one prefill workload; returns (record, x, out, fin, ws)."""
+        x = inputs.make(w, device=dev)
+        T, N = x["q"].shape[0], x["cu_seqlens"].numel() - 1
+        out = torch.empty_like(x["v"])
+        fin = torch.empty((N, HV, D, D), dtype=torch.float32, device=dev)
+        if segments == 1:
+            shape = gdn.prefill_shape(x["q"], x["v"], x["cu_seqlens"], algo)
+        else:  # every call sees one sequence of T / segments tokens
+            shape = gdn.make_shape(1, T // segments, HK, HV, D, gdn.GDN_BF16, algo)
+        ws = gdn.alloc_workspace(shape, dev)
+        fn = prefill_step_fn(x, out, fin, ws, with_initial, segments)
+        clk = ClockSampler(local_rank) if clocks else None
+        if clk:
+            with clk:
+                ms = timed(fn, steps, warmup)
+        else:
+            ms = timed(fn, steps, warmup)
+        ms_step = max_over_ranks(sum(ms) / len(ms))
+        nbytes, flop = prefill_work(T, N, with_initial, True)
+        rec = {"tokens": T, "sequences": N, "ms_per_step": ms_step,
+               "tokens_per_s": replicas.job_throughput(T, world, ms_step * 1e-3),
+               "step": roofline_of(nbytes, flop, ms_step, peaks),
+               "algorithmic_bytes": nbytes, "algorithmic_flop": flop}
+        if segments > 1:
+            rec["segments"] = segments
+        if clk:
+            rec["clocks"] = clk.summary()
+        if phased and tensor_path and segments == 1:
+            # the same two launches gdn_chunk_prefill makes, with events between them
+            evs = []
+
+            def phased_fn():
+                e = [torch.cuda.Event(enable_timing=True) for _ in range(3)]
+                e[0].record(stream)
+                gdn.gdn_chunk_prefill_prep(x["q"], x["k"], x["g"], x["beta"], x["cu_seqlens"], ws, x["v"],
+                                           algo=algo, stream=stream)
+                e[1].record(stream)
+                gdn.gdn_chunk_prefill_state(x["k"], x["v"], x["initial_state"] if with_initial else None,
+                                            x["cu_seqlens"], out, fin, ws, algo=algo, stream=stream)
+                e[2].record(stream)
+                evs.append(e)
+            timed(phased_fn, steps, warmup)
+            tev = evs[-steps:]
+            phase_ms = {"prep": max_over_ranks(sum(e[0].elapsed_time(e[1]) for e in tev) / steps),
+                        "state": max_over_ranks(sum(e[1].elapsed_time(e[2]) for e in tev) / steps)}
+            kernels = {"prep": "chunk_table_kernel + chunk_prep_kernel", "state": "chunk_state_kernel"}
+            rec["phases"] = {}
+            for ph, (pb, pf) in phase_work(T, N, with_initial, True).items():
+                r = roofline_of(pb, pf, phase_ms[ph], peaks)
+                r.update(kernels=kernels[ph], ms=phase_ms[ph], algorithmic_bytes=pb, algorithmic_flop=pf)
+                rec["phases"][ph] = r
+            # north_star's GEMM-phase figure: all GEMM flops over the time of the GEMM phases
+            gemm_ms = phase_ms["prep"] + phase_ms["state"]
+            rec["gemm_phases_frac_tensor"] = flop / (gemm_ms * 1e-3) / 1e12 / peaks["bf16_tflops"]
+        return rec, x, out, fin, ws
+
+    # ---- the headline: the layer workload (B=1, T=8192), one gdn_chunk_prefill call per step
+    w = inputs.workload(WORKLOAD)
+    if args.tokens:
+        w.seqlens = [args.tokens]
+    main_rec, x, out, fin, ws = measure_prefill(w, args.steps, args.warmup, False, phased=True, clocks=True)
+    T = main_rec["tokens"]
+    ms_step = main_rec["ms_per_step"]
+    value = main_rec["tokens_per_s"]
+    clocks = main_rec.pop("clocks", None)
     launches_per_step = gdn_launches_per_prefill(algo, x["q"].dtype)
-    peak = peaks["bf16_tflops"]
-    phases = None
-    if tensor_path:
-        timed_ev = phase_ev[-args.steps:]
-        prep_ms = max_over_ranks(sum(e[0].elapsed_time(e[1]) for e in timed_ev) / args.steps)
-        state_ms = max_over_ranks(sum(e[1].elapsed_time(e[2]) for e in timed_ev) / args.steps)
-        chunks = T // C  # one sequence of T tokens, T a multiple of the chunk size
-        phases = {
-            "prep": {"kernels": "chunk_table_kernel + chunk_prep_kernel", "ms": prep_ms,
-                     "flop": PREP_FLOP_PER_TOKEN * T, "bytes": PREP_BYTES_PER_CHUNK * chunks},
-            "state": {"kernels": "chunk_state_kernel", "ms": state_ms,
-                      "flop": STATE_FLOP_PER_TOKEN * T,
-                      "bytes": STATE_BYTES_PER_CHUNK * chunks + 2 * STATE_BYTES}}
-        for ph in phases.values():
-            ph["tflops"] = ph["flop"] / (ph["ms"] * 1e-3) / 1e12
-            ph["gbs"] = ph["bytes"] / (ph["ms"] * 1e-3) / 1e9
-            ph["frac_hbm"] = ph["gbs"] / peaks["hbm_gbs"]
-            ph["frac_tensor"] = ph["tflops"] / peak
+    phases = main_rec.get("phases")
+    step = main_rec["step"]
+    if phases:
         dom = max(phases, key=lambda k2: phases[k2]["ms"])
         d = phases[dom]
         traffic = None
-        tr = load_traffic() if T == 8192 and len(x["cu_seqlens"]) == 2 else {}
+        tr = load_traffic() if T == 8192 else {}
         if tr:
             traffic = (tr["chunk_table_kernel"] + tr["chunk_prep_kernel"]) if dom == "prep" else tr["chunk_state_kernel"]
-        roofline = {"bound": "hbm", "achieved": d["gbs"], "peak": peaks["hbm_gbs"], "unit": "GB/s",
-                    "frac": d["frac_hbm"], "traffic": traffic,
-                    "peak_source": peaks["source"] + " HBM copy",
-                    "kernel": d["kernels"], "algorithmic_bytes_per_launch": d["bytes"],
-                    "tensor_frac": d["frac_tensor"],
-                    "step_frac_tensor": PREFILL_FLOP_PER_TOKEN * T / (ms_step * 1e-3) / 1e12 / peak}
+        unit_hbm = d["bound"] == "hbm"
+        roofline = {"bound": d["bound"],
+                    "achieved": d["gbs"] if unit_hbm else d["tflops"],
+                    "peak": peaks["hbm_gbs"] if unit_hbm else peaks["bf16_tflops"],
+                    "unit": "GB/s" if unit_hbm else "TFLOP/s",
+                    "frac": d["frac_hbm"] if unit_hbm else d["frac_tensor"],
+                    "traffic": traffic,
+                    "traffic_over_algorithmic_bytes": (traffic / d["algorithmic_bytes"]) if traffic else None,
+                    "peak_source": peaks["source"] + (" HBM copy" if unit_hbm else " bf16 dense (burst)"),
+                    "kernel": d["kernels"], "algorithmic_bytes_per_launch": d["algorithmic_bytes"],
+                    "algorithmic_flop_per_launch": d["algorithmic_flop"],
+                    "frac_hbm": d["frac_hbm"], "frac_tensor": d["frac_tensor"],
+                    "step_frac_tensor": step["frac_tensor"], "step_frac_hbm": step["frac_hbm"],
+                    "gemm_phases_frac_tensor": main_rec["gemm_phases_frac_tensor"]}
     else:
-        flop = PREFILL_FLOP_PER_TOKEN * T
-        achieved = flop / (ms_step * 1e-3) / 1e12
-        roofline = {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
-                    "frac": achieved / peak, "traffic": None,
+        nbytes, flop = prefill_work(T, 1, False, True)
+        roofline = {"bound": "tensor", "achieved": step["tflops"], "peak": peaks["bf16_tflops"],
+                    "unit": "TFLOP/s", "frac": step["frac_tensor"], "traffic": None,
                     "peak_source": peaks["source"] + " bf16 dense (burst)",
-                    "kernel": "prefill_simt_kernel", "algorithmic_flop_per_launch": flop}
-
+                    "kernel": "prefill_simt_kernel", "algorithmic_flop_per_launch": flop,
+                    "step_frac_tensor": step["frac_tensor"], "step_frac_hbm": step["frac_hbm"]}
     # ---- end to end through the C ABI with pinned host buffers
     host = {k2: x[k2].cpu().pin_memory() for k2 in ("q", "k", "v", "g", "beta", "cu_seqlens")}
     dbuf = {k2: torch.empty_like(x[k2]) for k2 in host}
@@ -449,15 +511,63 @@ def main_ours(args, rank, world, local_rank):
                              "algorithmic_bytes_per_launch": nbytes}}
         dec["verify4_snapshots"]["tokens_per_s"] = world * 256 * ntok / (dec["verify4_snapshots"]["ms_per_step"] * 1e-3)
 
-    # ---- CPU baseline: the oracle on a bounded sample (rank 0, N=1 only)
+    # ---- the other prefill workloads: varlen (8 sequences with initial and final states) and
+    #      long context (T = 262,144 whole, and as 4 segments of 65,536 with the state carried)
+    others = {}
+    want_cpu = rank == 0 and world == 1 and not args.no_cpu_baseline and not args.tokens
+    cpu_samples = {}
+    if want_cpu:  # the layer workload's inputs, as the GPU drew them
+        cpu_samples["layer"] = {k2: x[k2].cpu() for k2 in ("q", "k", "v", "g", "beta", "cu_seqlens")}
+    if not args.tokens and args.only != "prefill":
+        del x, out, fin, ws
+        torch.cuda.empty_cache()
+        for name, w2, kw in (("varlen", inputs.workload("varlen"), dict(with_initial=True)),
+                             ("long", inputs.workload("long"), dict(with_initial=False)),
+                             ("long_4x65536_carry", inputs.workload("long"), dict(with_initial=False, segments=4))):
+            rec, x2, *_bufs = measure_prefill(w2, max(5, args.steps // 2), args.warmup,
+                                              phased=(name != "long_4x65536_carry"), **kw)
+            if want_cpu and name == "varlen":  # 4 of the 16 QK heads and the 8 V heads that read them
+                cpu_samples[name] = {"q": x2["q"][:, :4].cpu(), "k": x2["k"][:, :4].cpu(), "v": x2["v"][:, :8].cpu(),
+                                     "g": x2["g"][:, :8].cpu(), "beta": x2["beta"][:, :8].cpu(),
+                                     "cu_seqlens": x2["cu_seqlens"].cpu(),
+                                     "initial_state": x2["initial_state"][:, :8].cpu()}
+            if want_cpu and name == "long":  # every head of the first 16,384 tokens
+                cpu_samples[name] = {k2: x2[k2][:16384].cpu() for k2 in ("q", "k", "v", "g", "beta")}
+                cpu_samples[name]["cu_seqlens"] = torch.tensor([0, 16384], dtype=torch.int32)
+            del x2, _bufs
+            torch.cuda.empty_cache()
+            others[name] = rec
+
+    # ---- CPU baseline: the fp64 oracle on bounded samples of the same inputs (rank 0, N=1 only)
     cpu = None
-    if rank == 0 and world == 1 and not args.no_cpu_baseline and not args.tokens:
+    if want_cpu:
         import oracle
-        xs = {k2: (x[k2].cpu() if hasattr(x[k2], "cpu") else x[k2]) for k2 in x}
-        v_cpu, dt = oracle_tokens_per_s(xs, HK)
-        cpu = {"value": v_cpu, "unit": UNIT, "cores": oracle.host_threads(), "kind": "oracle",
+        cores = oracle.host_threads()
+
+        def oracle_rate(xs, with_initial, scale_heads):
+            t0 = time.perf_counter()
+            oracle.forward(xs["q"], xs["k"], xs["v"], xs["g"], xs["beta"], xs["cu_seqlens"],
+                           xs["initial_state"] if with_initial else None)
+            dt = time.perf_counter() - t0
+            return xs["q"].shape[0] / (dt * scale_heads), dt
+
+        v_cpu, dt = oracle_rate(cpu_samples["layer"], False, 1)
+        cpu = {"value": v_cpu, "unit": UNIT, "cores": cores, "kind": "oracle",
                "sample": "fp64 oracle (token recurrence) on the whole T=8192, 16/32-head "
                          "workload, one pass, %.1f s" % dt}
+        if "varlen" in cpu_samples:
+            vv, dtv = oracle_rate(cpu_samples["varlen"], True, HK / 4)
+            others["varlen"]["cpu_baseline"] = {
+                "value": vv, "unit": UNIT, "cores": cores, "kind": "oracle",
+                "sample": "4 of 16 QK heads (8 of 32 V heads) of all %d packed tokens with their "
+                          "initial states, %.1f s, scaled to 16 heads" % (cpu_samples["varlen"]["q"].shape[0], dtv)}
+        if "long" in cpu_samples:
+            vl, dtl = oracle_rate(cpu_samples["long"], False, 1)
+            for nm in ("long", "long_4x65536_carry"):
+                others[nm]["cpu_baseline"] = {
+                    "value": vl, "unit": UNIT, "cores": cores, "kind": "oracle",
+                    "sample": "every head of the first 16384 tokens, %.1f s (the recurrence's cost is "
+                              "linear in tokens)" % dtl}
 
     if rank == 0:
         line = {"metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world,
@@ -472,7 +582,8 @@ def main_ours(args, rank, world, local_rank):
                 "roofline": roofline, "cpu_baseline": cpu,
                 "e2e": e2e,
                 "gpu_launches": launches_per_step * args.steps, "phases": phases,
-                "decode": dec, "clocks": clocks, "peaks": peaks}
+                "gemm_phases_frac_tensor": main_rec.get("gemm_phases_frac_tensor"),
+                "configs": others, "decode": dec, "clocks": clocks, "peaks": peaks}
         print(json.dumps(line), flush=True)
     return 0
 

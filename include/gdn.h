@@ -51,7 +51,7 @@
 extern "C" {
 #endif
 
-#define GDN_ABI_VERSION 1
+#define GDN_ABI_VERSION 2
 
 typedef enum {
     GDN_OK = 0,
@@ -70,9 +70,10 @@ typedef enum { GDN_BF16 = 0, GDN_F32 = 1 } gdn_dtype;
 
 /* Prefill algorithm selection (gdn_shape.algo). */
 typedef enum {
-    GDN_ALGO_AUTO = 0,          /* tensor-core path for bf16 I/O, SIMT fp32 path for fp32 I/O */
+    GDN_ALGO_AUTO = 0,          /* tensor-core path where it applies, else the SIMT fp32 path */
     GDN_ALGO_SIMT = 1,          /* chunked form on CUDA cores in fp32 (any io dtype) */
-    GDN_ALGO_TENSOR = 2         /* chunked form on tcgen05 tensor cores (bf16 I/O only) */
+    GDN_ALGO_TENSOR = 2         /* chunked form on tcgen05 tensor cores: bf16 I/O and an even
+                                   number of V heads per QK head only */
 } gdn_algo;
 
 typedef struct {
@@ -123,23 +124,25 @@ gdn_status gdn_chunk_prefill(const void *q, const void *k, const void *v,
  * The tensor-core prefill in two phases, for callers that want to schedule or time
  * them separately (gdn_chunk_prefill is exactly prep followed by state on one stream).
  *
- * gdn_chunk_prefill_prep: builds the chunk table from cu_seqlens and, for every chunk
- *   and head in parallel, the chunk's UT representation (W, U, P, decay factors and the
- *   normalised keys) into `workspace`.  Reads q, k, v, g, beta, cu_seqlens.
- * gdn_chunk_prefill_state: carries each sequence's fp32 state across its chunks using
- *   the workspace written by the prep phase of the same shape, writing out and
- *   final_state.  Reads initial_state, cu_seqlens.
- * Both require io_dtype == GDN_BF16 and an algo of GDN_ALGO_AUTO or GDN_ALGO_TENSOR
- * (GDN_ERR_UNSUPPORTED otherwise); arguments as for gdn_chunk_prefill.  The workspace
- * header is cleared by the prep phase.
+ * gdn_chunk_prefill_prep: builds the chunk table from cu_seqlens and, for every chunk and
+ *   V head in parallel, the chunk's coefficient images into `workspace`: the solved UT
+ *   system T = (I + strictly_lower(beta K K^T decay))^-1 applied to the keys (W) and folded
+ *   into the queries, T diag(beta) and its product with the decay-masked Q K^T, and the gate
+ *   factors.  Reads q, k, g, beta, cu_seqlens.
+ * gdn_chunk_prefill_state: carries each sequence's fp32 state across its chunks using the
+ *   workspace written by the prep phase of the same shape, reading the raw keys and values
+ *   again, and writes out and final_state.  Reads k, v, initial_state, cu_seqlens.
+ * Both require io_dtype == GDN_BF16, an even number of V heads per QK head and an algo of
+ * GDN_ALGO_AUTO or GDN_ALGO_TENSOR (GDN_ERR_UNSUPPORTED otherwise); arguments as for
+ * gdn_chunk_prefill.  The workspace header is cleared by the prep phase.
  */
-gdn_status gdn_chunk_prefill_prep(const void *q, const void *k, const void *v,
-                                  const float *g, const float *beta,
+gdn_status gdn_chunk_prefill_prep(const void *q, const void *k, const float *g, const float *beta,
                                   const int32_t *cu_seqlens, const gdn_shape *shape,
                                   void *workspace, size_t workspace_bytes, void *stream);
-gdn_status gdn_chunk_prefill_state(const float *initial_state, const int32_t *cu_seqlens,
-                                   void *out, float *final_state, const gdn_shape *shape,
-                                   void *workspace, size_t workspace_bytes, void *stream);
+gdn_status gdn_chunk_prefill_state(const void *k, const void *v, const float *initial_state,
+                                   const int32_t *cu_seqlens, void *out, float *final_state,
+                                   const gdn_shape *shape, void *workspace, size_t workspace_bytes,
+                                   void *stream);
 
 /*
  * Decode / multi-token verify step: advances every sequence's state by num_tokens

@@ -57,16 +57,21 @@ const char* gdn_status_string(gdn_status status) {
     return "unknown gdn_status";
 }
 
-// Which kernel family serves a (validated) shape: true = tensor cores.
+// Which kernel family serves a (validated) shape: true = tensor cores.  The tensor-core
+// kernels take the V heads in pairs that read one QK head, so they need an even number of V
+// heads per QK head; GDN_ALGO_AUTO takes the fp32 kernels otherwise.
+static bool tensor_shape_ok(const gdn_shape* s) {
+    return s->io_dtype == GDN_BF16 && (s->num_v_heads / s->num_qk_heads) % 2 == 0;
+}
 static bool use_tensor_path(const gdn_shape* s) {
     if (s->algo == GDN_ALGO_TENSOR) return true;
     if (s->algo == GDN_ALGO_SIMT) return false;
-    return s->io_dtype == GDN_BF16;
+    return tensor_shape_ok(s);
 }
 
 size_t gdn_prefill_workspace_bytes(const gdn_shape* shape) {
     if (check_prefill_shape(shape) != GDN_OK) return 0;
-    if (use_tensor_path(shape) && shape->io_dtype == GDN_BF16)
+    if (use_tensor_path(shape) && tensor_shape_ok(shape))
         return gdn::tc_workspace_bytes(shape->num_seqs, shape->total_tokens, shape->num_qk_heads,
                                        shape->num_v_heads);
     return kHeaderBytes;
@@ -94,18 +99,17 @@ gdn_status prefill_impl(const void* q, const void* k, const void* v, const float
 
     gdn_dtype io = (gdn_dtype)shape->io_dtype;
     const bool tensor = use_tensor_path(shape);
-    if (tensor && io != GDN_BF16) return GDN_ERR_UNSUPPORTED;
+    if (tensor && !tensor_shape_ok(shape)) return GDN_ERR_UNSUPPORTED;
     cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
     // The tensor-core path's first kernel (the chunk table) clears the device error word
     // itself; the fp32 path's header is cleared here.
     if (!tensor && cudaMemsetAsync(workspace, 0, kHeaderBytes, s) != cudaSuccess) return GDN_ERR_CUDA;
     cudaError_t e;
     if (tensor) {
-        e = gdn::launch_prefill_tc_prep(q, k, v, g, beta, cu_seqlens, shape->num_seqs,
-                                        shape->total_tokens, shape->num_qk_heads,
-                                        shape->num_v_heads, workspace, s);
+        e = gdn::launch_prefill_tc_prep(q, k, g, beta, cu_seqlens, shape->num_seqs, shape->total_tokens,
+                                        shape->num_qk_heads, shape->num_v_heads, workspace, s);
         if (e == cudaSuccess)
-            e = gdn::launch_prefill_tc_state(initial_state, cu_seqlens, out, final_state, map, chunk_states,
+            e = gdn::launch_prefill_tc_state(k, v, initial_state, cu_seqlens, out, final_state, map, chunk_states,
                                              shape->num_seqs, shape->total_tokens,
                                              shape->num_qk_heads, shape->num_v_heads, workspace, s);
     } else
@@ -197,7 +201,7 @@ static gdn_status check_phase(const gdn_shape* shape, const int32_t* cu_seqlens,
                               size_t workspace_bytes) {
     gdn_status st = check_prefill_shape(shape);
     if (st != GDN_OK) return st;
-    if (shape->io_dtype != GDN_BF16 || !use_tensor_path(shape)) return GDN_ERR_UNSUPPORTED;
+    if (!use_tensor_path(shape) || !tensor_shape_ok(shape)) return GDN_ERR_UNSUPPORTED;
     if (!workspace || workspace_bytes < gdn_prefill_workspace_bytes(shape)) return GDN_ERR_WORKSPACE;
     if ((reinterpret_cast<uintptr_t>(workspace) & 255u) != 0) return GDN_ERR_ALIGN;
     if (shape->num_seqs > 0 && !cu_seqlens) return GDN_ERR_NULL;
@@ -205,35 +209,34 @@ static gdn_status check_phase(const gdn_shape* shape, const int32_t* cu_seqlens,
     return GDN_OK;
 }
 
-gdn_status gdn_chunk_prefill_prep(const void* q, const void* k, const void* v, const float* g,
-                                  const float* beta, const int32_t* cu_seqlens,
-                                  const gdn_shape* shape, void* workspace, size_t workspace_bytes,
-                                  void* stream) {
+gdn_status gdn_chunk_prefill_prep(const void* q, const void* k, const float* g, const float* beta,
+                                  const int32_t* cu_seqlens, const gdn_shape* shape, void* workspace,
+                                  size_t workspace_bytes, void* stream) {
     gdn_status st = check_phase(shape, cu_seqlens, workspace, workspace_bytes);
     if (st != GDN_OK) return st;
     if (shape->num_seqs == 0) return GDN_OK;
-    if (shape->total_tokens > 0 && (!q || !k || !v || !g || !beta)) return GDN_ERR_NULL;
-    const void* ptrs[] = {q, k, v, g, beta};
+    if (shape->total_tokens > 0 && (!q || !k || !g || !beta)) return GDN_ERR_NULL;
+    const void* ptrs[] = {q, k, g, beta};
     for (const void* p : ptrs)
         if (p && !aligned16(p)) return GDN_ERR_ALIGN;
     cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
-    cudaError_t e = gdn::launch_prefill_tc_prep(q, k, v, g, beta, cu_seqlens, shape->num_seqs,
-                                                shape->total_tokens, shape->num_qk_heads,
-                                                shape->num_v_heads, workspace, s);
+    cudaError_t e = gdn::launch_prefill_tc_prep(q, k, g, beta, cu_seqlens, shape->num_seqs, shape->total_tokens,
+                                                shape->num_qk_heads, shape->num_v_heads, workspace, s);
     return e == cudaSuccess ? GDN_OK : GDN_ERR_CUDA;
 }
 
-gdn_status gdn_chunk_prefill_state(const float* initial_state, const int32_t* cu_seqlens,
-                                   void* out, float* final_state, const gdn_shape* shape,
-                                   void* workspace, size_t workspace_bytes, void* stream) {
+gdn_status gdn_chunk_prefill_state(const void* k, const void* v, const float* initial_state,
+                                   const int32_t* cu_seqlens, void* out, float* final_state,
+                                   const gdn_shape* shape, void* workspace, size_t workspace_bytes,
+                                   void* stream) {
     gdn_status st = check_phase(shape, cu_seqlens, workspace, workspace_bytes);
     if (st != GDN_OK) return st;
     if (shape->num_seqs == 0) return GDN_OK;
-    if (shape->total_tokens > 0 && !out) return GDN_ERR_NULL;
-    const void* ptrs[] = {initial_state, out, final_state};
+    if (shape->total_tokens > 0 && (!k || !v || !out)) return GDN_ERR_NULL;
+    const void* ptrs[] = {k, v, initial_state, out, final_state};
     for (const void* p : ptrs)
         if (p && !aligned16(p)) return GDN_ERR_ALIGN;
-    cudaError_t e = gdn::launch_prefill_tc_state(initial_state, cu_seqlens, out, final_state, kDense, nullptr,
+    cudaError_t e = gdn::launch_prefill_tc_state(k, v, initial_state, cu_seqlens, out, final_state, kDense, nullptr,
                                                  shape->num_seqs, shape->total_tokens,
                                                  shape->num_qk_heads, shape->num_v_heads,
                                                  workspace, reinterpret_cast<cudaStream_t>(stream));

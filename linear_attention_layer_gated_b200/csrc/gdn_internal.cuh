@@ -75,17 +75,18 @@ cudaError_t launch_prefill_simt(const void* q, const void* k, const void* v, con
                                 void* out, float* sT, StateSlots map, float* cstates, int num_seqs, int hk,
                                 int hv, gdn_dtype io, cudaStream_t stream);
 
-// Tensor-core prefill (bf16 I/O): total workspace bytes (header included) and launch.
+// Tensor-core prefill (bf16 I/O, num_v_heads / num_qk_heads even): total workspace bytes
+// (header included) and launch.
 size_t tc_workspace_bytes(int num_seqs, int total_tokens, int hk, int hv);
-// Phase 1 (chunk table + per-chunk UT representation) and phase 2 (state pass).
-cudaError_t launch_prefill_tc_prep(const void* q, const void* k, const void* v, const float* g,
-                                   const float* beta, const int32_t* cu, int num_seqs,
-                                   int total_tokens, int hk, int hv, void* workspace,
-                                   cudaStream_t stream);
+// Phase 1 (chunk table + per-chunk coefficient images, from q, k and the gates) and phase 2
+// (state pass, from k, v and the images).
+cudaError_t launch_prefill_tc_prep(const void* q, const void* k, const float* g, const float* beta,
+                                   const int32_t* cu, int num_seqs, int total_tokens, int hk, int hv,
+                                   void* workspace, cudaStream_t stream);
 // cstates (nullable): the state after every chunk, [total chunks][HV][D][D], chunks in
 // sequence order.
-cudaError_t launch_prefill_tc_state(const float* s0, const int32_t* cu, void* out, float* sT,
-                                    StateSlots map, float* cstates, int num_seqs, int total_tokens, int hk,
+cudaError_t launch_prefill_tc_state(const void* k, const void* v, const float* s0, const int32_t* cu, void* out,
+                                    float* sT, StateSlots map, float* cstates, int num_seqs, int total_tokens, int hk,
                                     int hv, void* workspace, cudaStream_t stream);
 
 // Diagnostic: a bounded wait that is guaranteed to expire (failure-path self-test).

@@ -65,9 +65,9 @@ def lib() -> ctypes.CDLL:
             L.gdn_chunk_prefill.argtypes = [vp, vp, vp, fp, fp, fp, ip, vp, fp, sp, vp,
                                             ctypes.c_size_t, vp]
             L.gdn_chunk_prefill_prep.restype = ctypes.c_int
-            L.gdn_chunk_prefill_prep.argtypes = [vp, vp, vp, fp, fp, ip, sp, vp, ctypes.c_size_t, vp]
+            L.gdn_chunk_prefill_prep.argtypes = [vp, vp, fp, fp, ip, sp, vp, ctypes.c_size_t, vp]
             L.gdn_chunk_prefill_state.restype = ctypes.c_int
-            L.gdn_chunk_prefill_state.argtypes = [fp, ip, vp, fp, sp, vp, ctypes.c_size_t, vp]
+            L.gdn_chunk_prefill_state.argtypes = [vp, vp, fp, ip, vp, fp, sp, vp, ctypes.c_size_t, vp]
             L.gdn_decode_step.restype = ctypes.c_int
             L.gdn_decode_step.argtypes = [vp, vp, vp, fp, fp, fp, vp, ctypes.c_int32, sp, vp]
             L.gdn_decode_verify.restype = ctypes.c_int
@@ -181,23 +181,24 @@ def gdn_chunk_prefill(q, k, v, g, beta, initial_state, cu_seqlens, out, final_st
     return workspace
 
 
-def gdn_chunk_prefill_prep(q, k, v, g, beta, cu_seqlens, workspace, algo=GDN_ALGO_AUTO,
+def gdn_chunk_prefill_prep(q, k, g, beta, cu_seqlens, workspace, v_shape_like, algo=GDN_ALGO_AUTO,
                            stream=None):
-    """Calls gdn_chunk_prefill_prep (tensor-core path, phase 1)."""
-    shape = prefill_shape(q, v, cu_seqlens, algo)
-    rc = lib().gdn_chunk_prefill_prep(_ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(beta),
-                                      _ptr(cu_seqlens), ctypes.byref(shape), _ptr(workspace),
-                                      workspace.numel(), _stream(stream))
+    """Calls gdn_chunk_prefill_prep (tensor-core path, phase 1).  ``v_shape_like`` is v (or
+    any tensor of v's shape) -- only its head count is used."""
+    shape = prefill_shape(q, v_shape_like, cu_seqlens, algo)
+    rc = lib().gdn_chunk_prefill_prep(_ptr(q), _ptr(k), _ptr(g), _ptr(beta), _ptr(cu_seqlens),
+                                      ctypes.byref(shape), _ptr(workspace), workspace.numel(),
+                                      _stream(stream))
     if rc != GDN_OK:
         raise GdnError(rc, "gdn_chunk_prefill_prep")
 
 
-def gdn_chunk_prefill_state(initial_state, cu_seqlens, out, final_state, workspace, q_shape_like,
+def gdn_chunk_prefill_state(k, v, initial_state, cu_seqlens, out, final_state, workspace,
                             algo=GDN_ALGO_AUTO, stream=None):
-    """Calls gdn_chunk_prefill_state (tensor-core path, phase 2).  ``q_shape_like`` is the
-    q tensor (or any tensor of q's shape and dtype) the prep phase was given."""
-    shape = prefill_shape(q_shape_like, out, cu_seqlens, algo)
-    rc = lib().gdn_chunk_prefill_state(_ptr(initial_state), _ptr(cu_seqlens), _ptr(out),
+    """Calls gdn_chunk_prefill_state (tensor-core path, phase 2) on the workspace the prep
+    phase of the same shape wrote."""
+    shape = prefill_shape(k, v, cu_seqlens, algo)
+    rc = lib().gdn_chunk_prefill_state(_ptr(k), _ptr(v), _ptr(initial_state), _ptr(cu_seqlens), _ptr(out),
                                        _ptr(final_state), ctypes.byref(shape), _ptr(workspace),
                                        workspace.numel(), _stream(stream))
     if rc != GDN_OK:

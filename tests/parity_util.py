@@ -39,15 +39,20 @@ def assert_close(x, ref, tol, what):
 
 def assert_rows_close(x, ref, row_dims, tol, what):
     """Relative L2 error of every row, rows being the first ``row_dims`` axes flattened.
-    A row whose reference norm is below 1e-2 of the median row norm (legitimately near
-    zero, e.g. a strongly decayed state) is measured against that floor instead."""
+    A row whose reference norm is below 0.1 of the median row norm is measured against that
+    floor instead: a bf16 dot product of normalised vectors carries an absolute rounding
+    error set by the vectors' scale, not by the product's value, so a row whose exact value
+    is nearly zero (a query almost orthogonal to the only key left after a strong decay)
+    has a large relative error that says nothing about the kernel.  A structurally wrong
+    row (a missing or misplaced contribution) is off by the order of the median norm and
+    still fails."""
     x, ref = as_f64(x), as_f64(ref)
     if x.size == 0:
         return 0.0
     nrows = int(np.prod(x.shape[:row_dims]))
     xr, rr = x.reshape(nrows, -1), ref.reshape(nrows, -1)
     rn = np.linalg.norm(rr, axis=1)
-    floor = max(1e-2 * float(np.median(rn)), 1e-300)
+    floor = max(0.1 * float(np.median(rn)), 1e-300)
     rel = np.linalg.norm(xr - rr, axis=1) / np.maximum(rn, floor)
     worst = int(np.argmax(rel))
     idx = np.unravel_index(worst, x.shape[:row_dims])

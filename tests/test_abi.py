@@ -36,7 +36,7 @@ def test_exports_every_declared_symbol(L):
 
 
 def test_abi_version_and_status_strings(L):
-    assert gdn.gdn_abi_version() == 1
+    assert gdn.gdn_abi_version() == 2
     for code, name in gdn.STATUS.items():
         assert gdn.gdn_status_string(code).startswith(name)
 
@@ -184,3 +184,17 @@ def test_chunk_states_prefill_requires_its_buffer(L):
     assert gdn.STATUS[L.gdn_chunk_prefill_chunk_states(FAKE, FAKE, FAKE, FAKE, FAKE, None, FAKE, FAKE, None,
                                                        FAKE + 8, ctypes.byref(s), FAKE, ws_bytes,
                                                        None)] == "GDN_ERR_ALIGN"
+
+
+def test_tensor_path_needs_pairs_of_v_heads_per_qk_head(L):
+    """The tensor-core kernels take V heads in pairs that read one QK head: an odd number of
+    V heads per QK head is refused on that path (before any device work) and served by the
+    fp32 path under GDN_ALGO_AUTO (whose workspace is just the header)."""
+    odd = shape(num_qk_heads=8, num_v_heads=8, algo=gdn.GDN_ALGO_TENSOR)
+    assert gdn.STATUS[prefill_call(L, odd, ws_bytes=1 << 30)] == "GDN_ERR_UNSUPPORTED"
+    assert L.gdn_prefill_workspace_bytes(ctypes.byref(shape(num_qk_heads=8, num_v_heads=8))) == 256
+    assert L.gdn_prefill_workspace_bytes(ctypes.byref(shape(num_qk_heads=8, num_v_heads=16))) > 256
+    assert gdn.STATUS[L.gdn_chunk_prefill_prep(FAKE, FAKE, FAKE, FAKE, FAKE, ctypes.byref(odd), FAKE, 1 << 30,
+                                               None)] == "GDN_ERR_UNSUPPORTED"
+    assert gdn.STATUS[L.gdn_chunk_prefill_state(FAKE, FAKE, None, FAKE, FAKE, None, ctypes.byref(odd), FAKE,
+                                                1 << 30, None)] == "GDN_ERR_UNSUPPORTED"
