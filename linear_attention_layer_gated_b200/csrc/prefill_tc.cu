@@ -20,6 +20,10 @@
 // operand is split into a bf16 high part and a bf16 remainder and both are multiplied, which
 // keeps about 16 significant bits.
 //
+// The state update runs as a tf32 product: it reads Delta^T (fp32) straight out of the
+// accumulator of the previous product and Kt = diag(c r_k) K in fp32, so Delta never passes
+// through the CUDA cores or bf16 (tf32 keeps 10 bits of each operand).
+//
 // Three kernels, all on the caller's stream:
 //  K0 chunk_table_kernel  clears the workspace's device error word; cu_seqlens -> per-sequence
 //                         first chunk id and a (seq, start, length) entry per chunk.
@@ -29,8 +33,8 @@
 //                         blocked forward substitution and P T in fp32; then per V head the
 //                         coefficient rows are written to Tensor Memory and W and
 //                         diag(gam r_q) Q - (P T diag(b gam r_k)) K come out of one tcgen05
-//                         product with K; W, Qt, the split [T diag(b); At] images and the
-//                         gate factors go to the workspace.
+//                         product with K; -W, Qt, the split [T diag(b); At] images, Kt in fp32
+//                         and gam_L go to the workspace.
 //  K2 chunk_state_kernel  one CTA per (sequence, V head), sequential over the sequence's chunks:
 //                         the state is the A operand of its MMAs, held in Tensor Memory (M =
 //                         d_v = 128 rows), so every product reads only its B operand from shared
@@ -50,17 +54,23 @@ using namespace sm100;
 constexpr float kInvSqrtD = 0.08838834764831845f;  // 1 / sqrt(128)
 constexpr float kLog2e = 1.4426950408889634f;
 
-// Workspace record per (chunk, V head), bf16 images in the 128-byte-swizzled K-major layout the
-// state kernel's MMAs read:
-//   WQ     [W; Qt]: per d_k block b (64 columns) at b * 16384, 64 rows of W then 64 rows of Qt
-//   TA_hi  [T diag(b); At] high part: 128 rows (64 of T diag(b), 64 of At) x 64 tokens
+// Workspace record per (chunk, V head), images in the 128-byte-swizzled layouts the state
+// kernel's MMAs read:
+//   WQ     [-W; Qt] bf16, K-major: per d_k block b (64 columns) at b * 16384, 64 rows of -W then
+//          64 rows of Qt
+//   TA_hi  [T diag(b); At] bf16 high part, K-major: 128 rows (64 of T diag(b), 64 of At) x 64
+//          tokens
 //   TA_lo  the remainders of the same
-//   F      c_r r_k,r for the chunk's 64 rows (0 beyond its length), gam_L at [64]
+//   KT     Kt = diag(c r_k) K in fp32 (the tf32 B operand of the state update), K-major: per
+//          32-token block b at b * 16384, 128 d_k rows of 128 bytes (32 tokens)
+//   F      gam_L
 constexpr uint32_t kWQBytes = 32768;
 constexpr uint32_t kTABytes = 16384;
-constexpr uint32_t kFacOff = kWQBytes + 2 * kTABytes;  // 65536
-constexpr uint32_t kFacLoad = 272;                      // bytes of F the state kernel reads
-constexpr uint32_t kRecBytes = kFacOff + 1024;          // 66,560
+constexpr uint32_t kKTOff = kWQBytes + 2 * kTABytes;  // 65536
+constexpr uint32_t kKTBytes = 32768;
+constexpr uint32_t kFacOff = kKTOff + kKTBytes;       // 98304
+constexpr uint32_t kFacLoad = 16;                     // bytes of F the state kernel reads
+constexpr uint32_t kRecBytes = kFacOff + 1024;        // 99,328
 
 struct WsLayout {
     size_t seq_chunk0, table, rec, total;
@@ -493,55 +503,93 @@ chunk_prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
     }
     __syncthreads();
 
-    // ---- 6. per head, 128 threads; thread l takes row l & 63 of T (l < 64) or of P T (l >= 64):
-    //         - image rows of [T diag(b); At = P T diag(b)], split high / low, to the workspace;
-    //         - Tensor Memory A-operand row l: T diag(b gam r_k) split high / low (l < 64), or
-    //           -P T diag(b gam r_k) with a zero low part (l >= 64);
-    //         - the gate factors c r_k and gam_L (threads l < 64).
+    // ---- 6. per head, 128 threads.
+    //   (a) thread l takes row l & 63 of T (l < 64) or of P T (l >= 64) and writes Tensor Memory
+    //       A-operand row l: T diag(b gam r_k) split high / low (l < 64), or -P T diag(b gam r_k)
+    //       with a zero low part (l >= 64); thread 0 also writes gam_L.
+    //   (b) the [T diag(b); At = P T diag(b)] images, split high / low, straight to the
+    //       workspace: thread l takes the 16-byte chunk l & 7 of rows l / 8 + 16 m, so that a
+    //       warp's store covers four whole 128-byte rows.
     {
         const int hh = tid >> 7, l = tid & 127, rr = l & 63;
         const bool trow = l < 64;
         const int h = h0 + hh;
-        const float* src = (trow ? AT : PP) + hh * kMat + rr * kLdA;
         unsigned char* rec = ws + L.rec + ((size_t)cid * hv + h) * kRecBytes;
-        unsigned char* ta_hi = rec + kWQBytes;
-        unsigned char* ta_lo = ta_hi + kTABytes;
         const float* bb = ss.b[hh];
         const float* gm = ss.gam[hh];
-        const uint32_t ta = tmem + ((uint32_t)(l & ~31) << 16) + 128 + 64 * hh;
-        uint32_t whi[32], wlo[32];
+        {
+            const float* src = (trow ? AT : PP) + hh * kMat + rr * kLdA;
+            const uint32_t ta = tmem + ((uint32_t)(l & ~31) << 16) + 128 + 64 * hh;
+            uint32_t whi[32], wlo[32];
 #pragma unroll
-        for (int ch = 0; ch < 8; ++ch) {
-            const float4 x0 = *reinterpret_cast<const float4*>(src + 8 * ch);
-            const float4 x1 = *reinterpret_cast<const float4*>(src + 8 * ch + 4);
-            const float v[8] = {x0.x, x0.y, x0.z, x0.w, x1.x, x1.y, x1.z, x1.w};
-            float tb[8], cw[8];
+            for (int ch = 0; ch < 8; ++ch) {
+                const float4 x0 = *reinterpret_cast<const float4*>(src + 8 * ch);
+                const float4 x1 = *reinterpret_cast<const float4*>(src + 8 * ch + 4);
+                const float v[8] = {x0.x, x0.y, x0.z, x0.w, x1.x, x1.y, x1.z, x1.w};
+                float cw[8];
 #pragma unroll
-            for (int e = 0; e < 8; ++e) {
-                const int i = 8 * ch + e;
-                tb[e] = v[e] * bb[i];
-                cw[e] = trow ? tb[e] * gm[i] * ss.rk[i] : -(tb[e] * gm[i] * ss.rk[i]);
+                for (int e = 0; e < 8; ++e) {
+                    const int i = 8 * ch + e;
+                    const float x = v[e] * bb[i] * gm[i] * ss.rk[i];
+                    cw[e] = trow ? x : -x;
+                }
+#pragma unroll
+                for (int e = 0; e < 4; ++e) {
+                    uint32_t hi, lo;
+                    split2(cw[2 * e], cw[2 * e + 1], hi, lo);
+                    whi[4 * ch + e] = hi;
+                    wlo[4 * ch + e] = trow ? lo : 0u;
+                }
             }
-            uint32_t th[4], tl[4];
-#pragma unroll
-            for (int e = 0; e < 4; ++e) {
-                split2(tb[2 * e], tb[2 * e + 1], th[e], tl[e]);
-                uint32_t ch_, cl_;
-                split2(cw[2 * e], cw[2 * e + 1], ch_, cl_);
-                whi[4 * ch + e] = ch_;
-                wlo[4 * ch + e] = trow ? cl_ : 0u;
+            tmem_st16(ta, whi);
+            tmem_st16(ta + 16, whi + 16);
+            tmem_st16(ta + 32, wlo);
+            tmem_st16(ta + 48, wlo + 16);
+            if (l == 0) {
+                float* fac = reinterpret_cast<float*>(rec + kFacOff);
+                fac[0] = ss.gam[hh][kChunk - 1];  // gam_L (G is constant past the length)
             }
-            *reinterpret_cast<uint4*>(ta_hi + sw128(l, ch)) = make_uint4(th[0], th[1], th[2], th[3]);
-            *reinterpret_cast<uint4*>(ta_lo + sw128(l, ch)) = make_uint4(tl[0], tl[1], tl[2], tl[3]);
         }
-        tmem_st16(ta, whi);
-        tmem_st16(ta + 16, whi + 16);
-        tmem_st16(ta + 32, wlo);
-        tmem_st16(ta + 48, wlo + 16);
-        if (trow) {
-            float* fac = reinterpret_cast<float*>(rec + kFacOff);
-            fac[rr] = ss.c[hh][rr] * ss.rk[rr];
-            if (rr == 0) fac[64] = ss.gam[hh][kChunk - 1];  // gam_L (G is constant past the length)
+        {
+            unsigned char* ta_hi = rec + kWQBytes;
+            unsigned char* ta_lo = ta_hi + kTABytes;
+            const int ch = l & 7;
+            float b8[8];
+#pragma unroll
+            for (int e = 0; e < 8; ++e) b8[e] = bb[8 * ch + e];
+#pragma unroll 2
+            for (int m = 0; m < 8; ++m) {
+                const int row = (l >> 3) + 16 * m;  // image row: T rows 0..63, then P T rows
+                const float* src = (row < 64 ? AT + row * kLdA : PP + (row - 64) * kLdA) + hh * kMat + 8 * ch;
+                const float4 x0 = *reinterpret_cast<const float4*>(src);
+                const float4 x1 = *reinterpret_cast<const float4*>(src + 4);
+                const float v[8] = {x0.x * b8[0], x0.y * b8[1], x0.z * b8[2], x0.w * b8[3],
+                                    x1.x * b8[4], x1.y * b8[5], x1.z * b8[6], x1.w * b8[7]};
+                uint32_t th[4], tl[4];
+#pragma unroll
+                for (int e = 0; e < 4; ++e) split2(v[2 * e], v[2 * e + 1], th[e], tl[e]);
+                *reinterpret_cast<uint4*>(ta_hi + sw128(row, ch)) = make_uint4(th[0], th[1], th[2], th[3]);
+                *reinterpret_cast<uint4*>(ta_lo + sw128(row, ch)) = make_uint4(tl[0], tl[1], tl[2], tl[3]);
+            }
+        }
+        {   // (c) Kt = diag(c r_k) K in fp32, K-major (tokens contiguous): 16-byte chunk i = l + 128 m
+            //     of the image is token block i / 1024, d_k row (i / 8) % 128, chunk i % 8 (tokens
+            //     32 (i / 1024) + 4 (i % 8) ..) -- a warp's store covers four whole 128-byte rows
+            unsigned char* kt = rec + kKTOff;
+            const float* cc = ss.c[hh];
+#pragma unroll 4
+            for (int m = 0; m < 16; ++m) {
+                const int i = l + 128 * m;
+                const int kb = i >> 10, dk = (i >> 3) & 127, ch = i & 7;
+                const int t = 32 * kb + 4 * ch;  // first of the chunk's 4 tokens
+                const unsigned char* kcol = sm + kP_QK + (dk >> 6) * 16384 + 8192 + (dk & 7) * 2;
+                float v4[4];
+#pragma unroll
+                for (int e = 0; e < 4; ++e)
+                    v4[e] = __bfloat162float(*reinterpret_cast<const __nv_bfloat16*>(kcol + sw128(t + e, (dk & 63) >> 3))) *
+                            (cc[t + e] * ss.rk[t + e]);
+                *reinterpret_cast<float4*>(kt + kb * 16384 + sw128(dk, ch)) = make_float4(v4[0], v4[1], v4[2], v4[3]);
+            }
         }
         tmem_st_wait();
     }
@@ -549,8 +597,9 @@ chunk_prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
     __syncthreads();
 
     // ---- 7. per head: TMEM[0:128, 0:128] = A_hi K + A_lo K (rows 0-63: W, rows 64-127:
-    //         -P T diag(b gam r_k) K), then the W and Qt = diag(gam r_q) Q + (rows 64-127) images
-    //         straight to the workspace (each thread one row, 8 16-byte chunks per d_k block).
+    //         -P T diag(b gam r_k) K); the -W and Qt = diag(gam r_q) Q + (rows 64-127) images are
+    //         assembled in the (now free) fp32 region in their final swizzled layout and leave
+    //         as one 32 KB bulk copy per head.
 #pragma unroll 1
     for (int hh = 0; hh < 2; ++hh) {
         if (tid == 0) {
@@ -567,8 +616,7 @@ chunk_prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
         if (__syncthreads_or(!ok)) { err = 1; goto cleanup; }
         tc_fence_after();
         {
-            const int h = h0 + hh;
-            unsigned char* wq = ws + L.rec + ((size_t)(cid * hv + h)) * kRecBytes;
+            unsigned char* img = sm + kP_AT + hh * kWQBytes;  // staging image of this head
             const uint32_t trow = tmem + ((uint32_t)qw * 32u << 16);
             const int r = (qw & 1) * 32 + lane;
             const float sq = (qw >= 2) ? ss.gam[hh][r] * ss.rq[r] : 0.f;
@@ -577,10 +625,12 @@ chunk_prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
             for (int half = 0; half < 2; ++half) {
                 tmem_ld32(trow + 64 * hf + 32 * half, col);
                 tmem_ld_wait();
-                if (qw < 2) {  // W row r, d_k block hf
+                if (qw < 2) {  // -W row r, d_k block hf
+#pragma unroll
+                    for (int e = 0; e < 32; ++e) col[e] = -col[e];
 #pragma unroll
                     for (int ch = 0; ch < 4; ++ch)
-                        *reinterpret_cast<uint4*>(wq + hf * 16384 + sw128(r, 4 * half + ch)) = pack8(col + 8 * ch);
+                        *reinterpret_cast<uint4*>(img + hf * 16384 + sw128(r, 4 * half + ch)) = pack8(col + 8 * ch);
                 } else {  // Qt row r = gam_r r_q,r q_r + (the product row), d_k block hf
 #pragma unroll
                     for (int ch = 0; ch < 4; ++ch) {
@@ -588,16 +638,21 @@ chunk_prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
                         unpack8(*reinterpret_cast<const uint4*>(sm + kP_QK + hf * 16384 + sw128(r, 4 * half + ch)), q8);
 #pragma unroll
                         for (int e = 0; e < 8; ++e) q8[e] = fmaf(sq, q8[e], col[8 * ch + e]);
-                        *reinterpret_cast<uint4*>(wq + hf * 16384 + 8192 + sw128(r, 4 * half + ch)) = pack8(q8);
+                        *reinterpret_cast<uint4*>(img + hf * 16384 + 8192 + sw128(r, 4 * half + ch)) = pack8(q8);
                     }
                 }
             }
+            fence_async_smem();
         }
         tc_fence_before();
         __syncthreads();  // the product is read before the next head's MMA overwrites it
+        if (tid == 32) {
+            bulk_s2g(ws + L.rec + ((size_t)cid * hv + h0 + hh) * kRecBytes, sm + kP_AT + hh * kWQBytes, kWQBytes);
+            bulk_commit();
+        }
     }
-
 cleanup:
+    if (tid == 32) bulk_wait_read_all();  // the image copies have read shared memory before the CTA exits
     if (err && tid == 0) {
         atomicOr(header, 1);
         mma_commit(&ss.bar_mma);  // MMAs issued so far complete before TMEM is freed
@@ -614,43 +669,45 @@ cleanup:
 
 // ===================================================================== K2
 // State pass, one CTA per (sequence, V head).  With S the fp32 state entering chunk c (held in
-// registers by the row workers, its bf16 copy in Tensor Memory as the A operand):
-//   (1x) X^T  = S W^T                       N = 64  -> Delta
-//   (1o) O^T  = S Qt^T                      N = 64  (output, first part)
-//   (2a) O^T += V^T At_hi^T + V^T At_lo^T   N = 64  (output, second part)
-//   (2b) U^T  = V^T Tb_hi^T + V^T Tb_lo^T   N = 64  (issued one chunk ahead)
-//   (3)  SA   = Dt_hi K + Dt_lo K           N = 128, Dt = (diag(c r_k)(U - X))^T split hi/lo
+// registers by the row workers, its bf16 copy in Tensor Memory as the A operand), per chunk
+// three groups of eight N = 128 MMAs (an MMA instruction costs the issuing thread about the
+// same whatever its N up to 128, so the products are merged into as few as possible):
+//   (2) D_c  = V^T [Tb; At]_hi^T + V^T [Tb; At]_lo^T   D_c = [U^T | O^T]    (no dependence on S)
+//   (1) D_c += S [-W; Qt]^T  (bf16)                   D_c = [Delta^T | O^T]
+//   (3) SA   = Delta^T Kt    (tf32, A = D_c's first 64 columns, Kt = diag(c r_k) K in fp32)
 //   S <- gam_L S + SA
-// The chain per chunk is S -> (1x) -> Delta -> (3) -> S; (1o), (2a) and (2b) fill the tensor
-// pipe while the row workers compute.  The tensor-pipe order is (1x) (1o) (2a) (3) (2b)_{c+1}.
+// (1) and (3) follow each other in the tensor pipe with no thread in between; the chain per
+// chunk is S -> (1) -> (3) -> S.  D is double-buffered so that (2) of chunk c+1 runs while the
+// row workers update the state; the tensor-pipe order is (1)_c (3)_c (2)_{c+1}.
 //
-// Warps: 0 loads (bulk copies and TMA), 1 issues MMAs, 2..9 row workers: lane quarter
-// warp % 4 (d_v rows 32 q .. 32 q + 31), half (warp - 2) / 4 of the columns.
-constexpr int kStateThreads = 320;
+// Warps: 0 loads (bulk copies and TMA), 1 issues MMAs, 2..9 row workers (the state: lane
+// quarter warp % 4 = d_v rows 32 q .. 32 q + 31, half (warp - 2) / 4 of the d_k columns),
+// 10..13 output warps (lane quarter warp % 4, all 64 tokens).  The outputs of a full chunk are
+// staged in the slot's V tile, which (2) has finished with, and leave by TMA store.
+constexpr int kStateThreads = 448;
 constexpr int kRowThreads = 256;
-constexpr uint32_t kSl_WQ = 0;          // [W; Qt] image (32 KB)
+constexpr int kOutWarp0 = 10;
+constexpr uint32_t kSl_WQ = 0;          // [-W; Qt] image (32 KB)
 constexpr uint32_t kSl_TA = 32768;      // TA_hi (16 KB) then TA_lo (16 KB)
-constexpr uint32_t kSl_V = 65536;       // V tile: 2 d_v blocks x 64 tokens x 128 B (TMA)
-constexpr uint32_t kSl_K = 81920;       // K tile: 2 d_k blocks x 64 tokens x 128 B (TMA)
-constexpr uint32_t kSl_F = 98304;       // gate factors (272 B)
-constexpr uint32_t kSlotBytes = 99328;  // 97 KB, a multiple of 1024
-constexpr uint32_t kSlotTx = 65536 + kFacLoad + 32768;
+constexpr uint32_t kSl_V = 65536;       // V tile: 2 d_v blocks x 64 tokens x 128 B (TMA); later the outputs
+constexpr uint32_t kSl_KT = 81920;      // Kt^T, fp32, K-major (32 KB)
+constexpr uint32_t kSlotBytes = 114688; // 112 KB, a multiple of 1024
+constexpr uint32_t kSlotTx = 65536 + 16384 + kKTBytes + kFacLoad;
 constexpr uint32_t kS_SMALL = 2 * kSlotBytes;
 constexpr uint32_t kStateSmem = kS_SMALL + 256 + 1024;  // small struct + alignment slack
+constexpr uint32_t kEmptyArrivals = 5;                  // the MMA commit and the 4 output warps
 // Tensor Memory columns
-constexpr uint32_t kT_X = 0;     // X^T (64)
-constexpr uint32_t kT_O = 64;    // O^T (64)
-constexpr uint32_t kT_U = 128;   // U^T (64)
+constexpr uint32_t kT_D = 0;     // D buffers at 0 and 128: [Delta^T | O^T] (2 x 128)
 constexpr uint32_t kT_SA = 256;  // state update (128)
-constexpr uint32_t kT_SB = 384;  // S in bf16, the A operand of (1x) and (1o) (64)
-constexpr uint32_t kT_DH = 448;  // Dt high part (32)
-constexpr uint32_t kT_DL = 480;  // Dt low part (32)
+constexpr uint32_t kT_SB = 384;  // S in bf16, the A operand of (1) (64)
 constexpr uint32_t kTmemCols = 512;
 
 struct StateSmall {
+    alignas(16) float gl[2][4];  // gam_L of the chunk in each slot (a 16-byte bulk-copy target)
     uint64_t full[2], empty[2];
-    uint64_t s_ready, d_ready, o_done;  // row workers -> issuer (256 arrivals)
-    uint64_t mx, mo, mu, msa;           // MMA commits -> row workers
+    uint64_t s_ready;            // row workers -> issuer (256 arrivals)
+    uint64_t o_done;             // output warps -> issuer (128 arrivals)
+    uint64_t mo, msa;            // MMA commits -> output warps, row workers
     uint64_t drain;
     uint32_t tmem_base;
     int abort_flag;
@@ -680,7 +737,7 @@ __device__ __forceinline__ void mbar_arrive(uint64_t* bar) {
 }
 
 __global__ void __launch_bounds__(kStateThreads, 1)
-chunk_state_kernel(const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_k,
+chunk_state_kernel(const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_out,
                    const float* s0, const int32_t* __restrict__ cu, __nv_bfloat16* __restrict__ out, float* sT,
                    StateSlots map, float* cstates, unsigned char* ws, int num_seqs, int total_tokens, int hk,
                    int hv) {
@@ -694,8 +751,8 @@ chunk_state_kernel(const __grid_constant__ CUtensorMap tm_v, const __grid_consta
     int32_t* header = reinterpret_cast<int32_t*>(ws);
     const int h = blockIdx.x % hv;
     const int n = blockIdx.x / hv;
-    const int jq = h / (hv / hk);
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    (void)hk;
 
     // Set-up that needs nothing from the prep kernel runs before the dependency wait (a
     // CTA of this kernel never shares an SM with a prep CTA: their shared memory does not
@@ -707,20 +764,17 @@ chunk_state_kernel(const __grid_constant__ CUtensorMap tm_v, const __grid_consta
     if (tid == 32) {
         for (int s = 0; s < 2; ++s) {
             mbar_init(&ss.full[s], 1);
-            mbar_init(&ss.empty[s], 1);
+            mbar_init(&ss.empty[s], kEmptyArrivals);
         }
         mbar_init(&ss.s_ready, kRowThreads);
-        mbar_init(&ss.d_ready, kRowThreads);
-        mbar_init(&ss.o_done, kRowThreads);
-        mbar_init(&ss.mx, 1);
+        mbar_init(&ss.o_done, 128);
         mbar_init(&ss.mo, 1);
-        mbar_init(&ss.mu, 1);
         mbar_init(&ss.msa, 1);
         mbar_init(&ss.drain, 1);
         ss.abort_flag = 0;
         fence_mbar_init();
         tma_prefetch_desc(&tm_v);
-        tma_prefetch_desc(&tm_k);
+        tma_prefetch_desc(&tm_out);
     }
     tc_fence_before();
     __syncthreads();
@@ -735,8 +789,21 @@ chunk_state_kernel(const __grid_constant__ CUtensorMap tm_v, const __grid_consta
     if (warp == 0) {
         // ------------------------------------------------ loads, one slot ahead
         if (lane == 0 && nch > 0) {
+            // chunk j's workspace record and V tile into L2, kAhead chunks before its slot load,
+            // so that the slot fills are L2 hits
+            auto prefetch = [&](int j) {
+                if (j >= nch) return;
+                const unsigned char* rec = rec_of(j);
+                bulk_prefetch_l2(rec, kFacOff + kFacLoad);
+                const int tj = t_begin + j * kChunk;
+                tma_prefetch_l2_2d(&tm_v, h * kD, tj);
+                tma_prefetch_l2_2d(&tm_v, h * kD + 64, tj);
+            };
+            constexpr int kAhead = 4;
+            for (int j = 2; j < kAhead; ++j) prefetch(j);
             int k = 0;
             for (; k < nch; ++k) {
+                prefetch(k + kAhead);
                 const int st = k & 1;
                 if (k >= 2 && !wait_or_abort(&ss.empty[st], ((k >> 1) - 1) & 1, abort_flag, header)) break;
                 unsigned char* slot = sm + st * kSlotBytes;
@@ -744,12 +811,10 @@ chunk_state_kernel(const __grid_constant__ CUtensorMap tm_v, const __grid_consta
                 const int tk = t_begin + k * kChunk;
                 mbar_arrive_expect_tx(&ss.full[st], kSlotTx);
                 bulk_g2s(slot + kSl_WQ, rec, 65536, &ss.full[st]);
-                bulk_g2s(slot + kSl_F, rec + kFacOff, kFacLoad, &ss.full[st]);
-#pragma unroll
-                for (int b = 0; b < 2; ++b) {
-                    tma_load_2d(slot + kSl_V + b * 8192, &tm_v, h * kD + b * 64, tk, &ss.full[st]);
-                    tma_load_2d(slot + kSl_K + b * 8192, &tm_k, jq * kD + b * 64, tk, &ss.full[st]);
-                }
+                bulk_g2s(slot + kSl_KT, rec + kKTOff, kKTBytes, &ss.full[st]);
+                bulk_g2s(&ss.gl[st][0], rec + kFacOff, kFacLoad, &ss.full[st]);
+                tma_load_2d(slot + kSl_V, &tm_v, h * kD, tk, &ss.full[st]);
+                tma_load_2d(slot + kSl_V + 8192, &tm_v, h * kD + 64, tk, &ss.full[st]);
             }
             if (*abort_flag) {  // drain: copies in flight land before the CTA exits
                 for (int j = max(0, k - 2); j < k; ++j) mbar_wait(&ss.full[j & 1], (j >> 1) & 1);
@@ -758,59 +823,48 @@ chunk_state_kernel(const __grid_constant__ CUtensorMap tm_v, const __grid_consta
     } else if (warp == 1) {
         // ------------------------------------------------ MMA issuer
         if (lane == 0 && nch > 0) {
-            const uint32_t id_x = idesc_bf16(128, 64, 0, 0);   // A TMEM, B K-major
-            const uint32_t id_v = idesc_bf16(128, 64, 1, 0);   // A (V^T) MN-major, B K-major
-            const uint32_t id_s = idesc_bf16(128, 128, 0, 1);  // A TMEM, B (K) MN-major
-            auto issue_u = [&](int c) {  // (2b): U^T = V^T Tb^T, hi and lo
+            const uint32_t id_s = idesc_bf16(128, 128, 0, 0);   // (1): A TMEM, B K-major
+            const uint32_t id_v = idesc_bf16(128, 128, 1, 0);   // (2): A (V^T) MN-major, B K-major
+            const uint32_t id_k = idesc_tf32(128, 128, 0, 0);   // (3): A TMEM (fp32), B (Kt) K-major
+            auto issue_2 = [&](int c) {  // D_c = V^T [Tb; At]^T, high then low part
                 const uint32_t slot = sb + (c & 1) * kSlotBytes;
 #pragma unroll
                 for (int s = 0; s < 8; ++s)
-                    mma_bf16(tmem + kT_U, sdesc_sw128(slot + kSl_V + (s & 3) * 2048, 8192, 1024),
+                    mma_bf16(tmem + kT_D + 128 * (c & 1), sdesc_sw128(slot + kSl_V + (s & 3) * 2048, 8192, 1024),
                              sdesc_sw128(slot + kSl_TA + (s >> 2) * kTABytes + (s & 3) * 32, 16, 1024), id_v, s > 0);
-                mma_commit(&ss.mu);
             };
             bool ok = wait_or_abort(&ss.full[0], 0, abort_flag, header);
             if (ok) {
                 tc_fence_after();
-                issue_u(0);
+                issue_2(0);
             }
             for (int c = 0; ok && c < nch; ++c) {
                 const uint32_t slot = sb + (c & 1) * kSlotBytes;
-                // (1x): X^T = S W^T once S_c is in Tensor Memory
+                const uint32_t dcol = tmem + kT_D + 128 * (c & 1);
+                // (1) once S_c is in Tensor Memory.  The output warps released D_{c-1} (o_done);
+                // waiting for it here, before the commit below, keeps the wait from ever falling
+                // two phases behind.
                 if (!(ok = wait_or_abort(&ss.s_ready, c & 1, abort_flag, header))) break;
-                tc_fence_after();
-#pragma unroll
-                for (int s = 0; s < 8; ++s)
-                    mma_bf16_tmem_a(tmem + kT_X, tmem + kT_SB + 8 * s,
-                                    sdesc_sw128(slot + kSl_WQ + (s >> 2) * 16384 + (s & 3) * 32, 16, 1024), id_x, s > 0);
-                mma_commit(&ss.mx);
-                // (1o) + (2a): O^T once the previous chunk's outputs are read
                 if (c >= 1 && !(ok = wait_or_abort(&ss.o_done, (c - 1) & 1, abort_flag, header))) break;
                 tc_fence_after();
 #pragma unroll
                 for (int s = 0; s < 8; ++s)
-                    mma_bf16_tmem_a(tmem + kT_O, tmem + kT_SB + 8 * s,
-                                    sdesc_sw128(slot + kSl_WQ + 8192 + (s >> 2) * 16384 + (s & 3) * 32, 16, 1024),
-                                    id_x, s > 0);
-#pragma unroll
-                for (int s = 0; s < 8; ++s)
-                    mma_bf16(tmem + kT_O, sdesc_sw128(slot + kSl_V + (s & 3) * 2048, 8192, 1024),
-                             sdesc_sw128(slot + kSl_TA + 8192 + (s >> 2) * kTABytes + (s & 3) * 32, 16, 1024), id_v, 1);
+                    mma_bf16_tmem_a(dcol, tmem + kT_SB + 8 * s,
+                                    sdesc_sw128(slot + kSl_WQ + (s >> 2) * 16384 + (s & 3) * 32, 16, 1024), id_s, 1);
                 mma_commit(&ss.mo);
-                // (3): the state update once Dt is in Tensor Memory
-                if (!(ok = wait_or_abort(&ss.d_ready, c & 1, abort_flag, header))) break;
-                tc_fence_after();
+                // (3): SA = Delta^T Kt, Delta^T from the first 64 columns of D_c
 #pragma unroll
                 for (int s = 0; s < 8; ++s)
-                    mma_bf16_tmem_a(tmem + kT_SA, tmem + ((s >> 2) ? kT_DL : kT_DH) + 8 * (s & 3),
-                                    sdesc_sw128(slot + kSl_K + (s & 3) * 2048, 8192, 1024), id_s, s > 0);
+                    mma_tf32_tmem_a(tmem + kT_SA, dcol + 8 * s,
+                                    sdesc_sw128(slot + kSl_KT + (s >> 2) * 16384 + (s & 3) * 32, 16, 1024), id_k, s > 0);
                 mma_commit(&ss.msa);
                 mma_commit(&ss.empty[c & 1]);  // every MMA reading slot c has been issued
-                // (2b) of the next chunk
+                // (2) of the next chunk into the other D buffer (released with D_{c-1} above); it
+                // runs while the row workers update the state
                 if (c + 1 < nch) {
                     if (!(ok = wait_or_abort(&ss.full[(c + 1) & 1], ((c + 1) >> 1) & 1, abort_flag, header))) break;
                     tc_fence_after();
-                    issue_u(c + 1);
+                    issue_2(c + 1);
                 }
             }
             if (*abort_flag) {  // drain: every MMA issued so far completes before TMEM is freed
@@ -818,10 +872,10 @@ chunk_state_kernel(const __grid_constant__ CUtensorMap tm_v, const __grid_consta
                 mbar_wait(&ss.drain, 0);
             }
         }
-    } else {
-        // ------------------------------------------------ row workers
+    } else if (warp < kOutWarp0) {
+        // ------------------------------------------------ row workers: the state
         const int q4 = warp & 3, hf = (warp - 2) >> 2;
-        const int dv = 32 * q4 + lane;  // d_v row of S this thread owns
+        const int dv = 32 * q4 + lane;  // d_v row of S this thread owns, d_k columns 64 hf ..
         const uint32_t trow = tmem + ((uint32_t)q4 * 32u << 16);
         bool has_state;
         const int sidx = state_index(map, n, has_state);
@@ -852,66 +906,23 @@ chunk_state_kernel(const __grid_constant__ CUtensorMap tm_v, const __grid_consta
         if (nch > 0) write_sb();
         bool alive = true;
         for (int c = 0; c < nch && alive; ++c) {
-            const unsigned char* slot = sm + (c & 1) * kSlotBytes;
-            const int t0 = t_begin + c * kChunk;
-            const int len = min(kChunk, t_end - t0);
-            // Delta: Dt = (U - X) diag(c r_k), tokens 32 hf .. 32 hf + 31 of row dv (the slot's
-            // gate factors are read after this thread's own wait on the slot's load)
             if (!(alive = wait_or_abort(&ss.full[c & 1], (c >> 1) & 1, abort_flag, header))) break;
-            if (!(alive = wait_or_abort(&ss.mx, c & 1, abort_flag, header))) break;
-            if (!(alive = wait_or_abort(&ss.mu, c & 1, abort_flag, header))) break;
-            tc_fence_after();
-            const float* fac = reinterpret_cast<const float*>(slot + kSl_F);
-            const float gl = fac[64];
-            {
-                float x[32], u[32];
-                tmem_ld32(trow + kT_X + 32 * hf, x);
-                tmem_ld32(trow + kT_U + 32 * hf, u);
-                tmem_ld_wait();
-                uint32_t dh[16], dl[16];
-#pragma unroll
-                for (int m = 0; m < 16; ++m) {
-                    const int e = 2 * m;
-                    split2((u[e] - x[e]) * fac[32 * hf + e], (u[e + 1] - x[e + 1]) * fac[32 * hf + e + 1], dh[m], dl[m]);
-                }
-                tmem_st16(trow + kT_DH + 16 * hf, dh);
-                tmem_st16(trow + kT_DL + 16 * hf, dl);
-                tmem_st_wait();
-                tc_fence_before();
-                mbar_arrive(&ss.d_ready);
-            }
-            // the state update
+            const float gl = ss.gl[c & 1][0];
             if (!(alive = wait_or_abort(&ss.msa, c & 1, abort_flag, header))) break;
             tc_fence_after();
-            {
+#pragma unroll
+            for (int half = 0; half < 2; ++half) {
                 float sa[32];
+                tmem_ld32(trow + kT_SA + 64 * hf + 32 * half, sa);
+                tmem_ld_wait();
 #pragma unroll
-                for (int half = 0; half < 2; ++half) {
-                    tmem_ld32(trow + kT_SA + 64 * hf + 32 * half, sa);
-                    tmem_ld_wait();
-#pragma unroll
-                    for (int m = 0; m < 32; ++m) S[32 * half + m] = fmaf(gl, S[32 * half + m], sa[m]);
-                }
+                for (int m = 0; m < 32; ++m) S[32 * half + m] = fmaf(gl, S[32 * half + m], sa[m]);
             }
             if (c + 1 < nch) write_sb();
-            if (cstates) {  // the state after this chunk, after the proxy fence (stores may stay in flight)
+            if (cstates) {  // the state after this chunk
                 float4* cr = reinterpret_cast<float4*>(cstates + ((size_t)(cs + c) * hv + h) * kD * kD + (size_t)dv * kD + 64 * hf);
 #pragma unroll
                 for (int m = 0; m < 16; ++m) cr[m] = make_float4(S[4 * m], S[4 * m + 1], S[4 * m + 2], S[4 * m + 3]);
-            }
-            // the outputs of this chunk: O^T row dv, tokens 32 hf .. 32 hf + 31
-            if (!(alive = wait_or_abort(&ss.mo, c & 1, abort_flag, header))) break;
-            tc_fence_after();
-            {
-                float o[32];
-                tmem_ld32(trow + kT_O + 32 * hf, o);
-                tmem_ld_wait();
-                __nv_bfloat16* op = out + ((size_t)(t0 + 32 * hf) * hv + h) * kD + dv;
-#pragma unroll
-                for (int e = 0; e < 32; ++e)
-                    if (32 * hf + e < len) op[(size_t)e * hv * kD] = __float2bfloat16_rn(o[e]);
-                tc_fence_before();
-                mbar_arrive(&ss.o_done);
             }
         }
         if (alive && !*abort_flag && srow_out) {
@@ -919,6 +930,47 @@ chunk_state_kernel(const __grid_constant__ CUtensorMap tm_v, const __grid_consta
 #pragma unroll
             for (int m = 0; m < 16; ++m) dst[m] = make_float4(S[4 * m], S[4 * m + 1], S[4 * m + 2], S[4 * m + 3]);
         }
+    } else {
+        // ------------------------------------------------ output warps
+        const int q4 = warp & 3;
+        const int dv = 32 * q4 + lane;  // d_v row of O^T this thread reads, all 64 tokens
+        const uint32_t trow = tmem + ((uint32_t)q4 * 32u << 16);
+        for (int c = 0; c < nch; ++c) {
+            if (!wait_or_abort(&ss.mo, c & 1, abort_flag, header)) break;
+            tc_fence_after();
+            const uint32_t dcol = kT_D + 128 * (c & 1) + 64;
+            float o[64];
+            tmem_ld32(trow + dcol, o);
+            tmem_ld32(trow + dcol + 32, o + 32);
+            tmem_ld_wait();
+            tc_fence_before();
+            mbar_arrive(&ss.o_done);  // D_c has been read
+            const int t0 = t_begin + c * kChunk;
+            const int len = min(kChunk, t_end - t0);
+            if (len == kChunk) {
+                // a 64-token x 32-d_v tile, row-major in the slot's V area (its (2) is complete:
+                // (1) of this chunk, which follows it in the pipe, has completed), one TMA store
+                unsigned char* st = sm + (c & 1) * kSlotBytes + kSl_V + q4 * 4096;
+#pragma unroll
+                for (int e = 0; e < 64; ++e)
+                    *reinterpret_cast<__nv_bfloat16*>(st + e * 64 + lane * 2) = __float2bfloat16_rn(o[e]);
+                fence_async_smem();
+                __syncwarp();
+                if (lane == 0) {
+                    tma_store_2d(&tm_out, h * kD + 32 * q4, t0, st);
+                    bulk_commit();
+                    bulk_wait_read_all();  // the tile is read before the slot is released
+                }
+            } else {
+                __nv_bfloat16* op = out + ((size_t)t0 * hv + h) * kD + dv;
+#pragma unroll
+                for (int e = 0; e < 64; ++e)
+                    if (e < len) op[(size_t)e * hv * kD] = __float2bfloat16_rn(o[e]);
+            }
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&ss.empty[c & 1]);
+        }
+        if (lane == 0) bulk_wait_all();  // this warp's output TMA stores have completed
     }
     tc_fence_before();
     __syncthreads();
@@ -946,8 +998,9 @@ cudaError_t launch_dependent(void (*kernel)(KArgs...), dim3 grid, dim3 block, si
     return cudaLaunchKernelEx(&cfg, kernel, static_cast<KArgs>(args)...);
 }
 
-// ---- TMA descriptors: a bf16 [rows][heads * 128] tensor, boxes of 64 rows x 64 elements
-//      (128 bytes, the 128-byte swizzle width), rows past the end read as zeros.
+// ---- TMA descriptors: a bf16 [rows][heads * 128] tensor, boxes of box_y rows x box_x elements
+//      (64 x 64 by default: 128 bytes, the 128-byte swizzle width); loads read rows past the end
+//      as zeros, stores do not write them.
 using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
                                    const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
                                    CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
@@ -964,15 +1017,17 @@ EncodeTiledFn encode_fn() {
     return fn;
 }
 
-cudaError_t encode_rows(CUtensorMap* m, const void* base, int rows, int heads) {
+cudaError_t encode_rows(CUtensorMap* m, const void* base, int rows, int heads,
+                        CUtensorMapSwizzle swizzle = CU_TENSOR_MAP_SWIZZLE_128B, unsigned box_x = 64,
+                        unsigned box_y = 64) {
     EncodeTiledFn fn = encode_fn();
     if (!fn) return cudaErrorNotSupported;
     const cuuint64_t dims[2] = {(cuuint64_t)heads * kD, (cuuint64_t)rows};
     const cuuint64_t strides[1] = {(cuuint64_t)heads * kD * 2};
-    const cuuint32_t box[2] = {64, 64};
+    const cuuint32_t box[2] = {box_x, box_y};
     const cuuint32_t estr[2] = {1, 1};
     const CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box, estr,
-                          CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                          CU_TENSOR_MAP_INTERLEAVE_NONE, swizzle, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                           CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
     return r == CUDA_SUCCESS ? cudaSuccess : cudaErrorInvalidValue;
 }
@@ -1008,19 +1063,23 @@ cudaError_t launch_prefill_tc_prep(const void* q, const void* k, const float* g,
 cudaError_t launch_prefill_tc_state(const void* k, const void* v, const float* s0, const int32_t* cu, void* out,
                                     float* sT, StateSlots map, float* cstates, int num_seqs, int total_tokens, int hk,
                                     int hv, void* workspace, cudaStream_t stream) {
+    (void)k;  // the keys reach the state pass as Kt, in the workspace
     if (num_seqs == 0) return cudaSuccess;
     // a zero-token batch still hands every initial state through; the descriptors then cover
     // one (never read) row of the caller's buffers
     const int rows = total_tokens > 0 ? total_tokens : 1;
-    CUtensorMap tv, tk;
+    CUtensorMap tv, to;
     cudaError_t e;
     if ((e = encode_rows(&tv, v ? v : workspace, rows, v ? hv : 1)) != cudaSuccess) return e;
-    if ((e = encode_rows(&tk, k ? k : workspace, rows, k ? hk : 1)) != cudaSuccess) return e;
+    // the outputs leave row-major (unswizzled) staging tiles of 64 tokens x 32 d_v
+    if ((e = encode_rows(&to, out ? out : workspace, rows, out ? hv : 1, CU_TENSOR_MAP_SWIZZLE_NONE, 32, 64)) !=
+        cudaSuccess)
+        return e;
     if ((e = cudaFuncSetAttribute(chunk_state_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kStateSmem)) !=
         cudaSuccess)
         return e;
     e = launch_dependent(chunk_state_kernel, dim3((unsigned)num_seqs * hv), dim3(kStateThreads), kStateSmem, stream, tv,
-                         tk, s0, cu, (__nv_bfloat16*)out, sT, map, cstates, static_cast<unsigned char*>(workspace),
+                         to, s0, cu, (__nv_bfloat16*)out, sT, map, cstates, static_cast<unsigned char*>(workspace),
                          num_seqs, total_tokens, hk, hv);
     if (e != cudaSuccess) return e;
     return cudaGetLastError();
