@@ -29,8 +29,8 @@
 //                         first chunk id and a (seq, start, length) entry per chunk.
 //  K1 chunk_prep_kernel   one CTA (256 threads) per (chunk, pair of V heads sharing a QK head),
 //                         all chunks in parallel: q and k tiles by TMA; the Gram [Q;K][Q;K]^T
-//                         (tcgen05), whose diagonal gives the norms; decay masks A and P; T by
-//                         blocked forward substitution and P T in fp32; then per V head the
+//                         (tcgen05), whose diagonal gives the norms; decay masks A and P; the
+//                         rows of T and of P T by substitution in fp32; then per V head the
 //                         coefficient rows are written to Tensor Memory and W and
 //                         diag(gam r_q) Q - (P T diag(b gam r_k)) K come out of one tcgen05
 //                         product with K; -W, Qt, the split [T diag(b); At] images, Kt in fp32
@@ -209,15 +209,15 @@ constexpr int kMat = kChunk * kLdA;  // floats per matrix
 //   kP_QK  per d_k block b at b * 16384: 64 rows of Q then 64 rows of K (TMA, 128-byte swizzle).
 //          The Gram reads it as A = B = [Q; K] (K-major); the W product reads the K rows as an
 //          MN-major B operand (tokens along K, d_k along N).
-//   kP_AT  per head: A, then T in place (fp32)
-//   kP_PP  per head: P, then P T in place (fp32)
+//   kP_AT  per head: A, then T (fp32, row-major)
+//   kP_PP  per head: P, then P T (fp32, row-major)
 // Tensor Memory (256 columns): 0..127 the Gram, later the [W; -P T diag(b gam r_k) K] product of
 // one head at a time; 128 + 64 h .. : head h's A operand rows (32 columns high part, 32 low).
 constexpr uint32_t kP_QK = 0;
 constexpr uint32_t kP_AT = 32768;
 constexpr uint32_t kP_PP = kP_AT + 2 * kMat * 4;
 constexpr uint32_t kP_SMALL = kP_PP + 2 * kMat * 4;
-constexpr uint32_t kPrepSmem = kP_SMALL + 3072 + 1024;  // small struct + alignment slack
+constexpr uint32_t kPrepSmem = kP_SMALL + 4096 + 1024;  // small struct + alignment slack
 constexpr int kPrepThreads = 256;
 
 struct PrepSmall {
@@ -227,10 +227,12 @@ struct PrepSmall {
     float c[2][kChunk];    // exp(G_L - G_r), 0 past the chunk's length
     float rq[kChunk];      // 1 / (sqrt(|q|^2 + eps) sqrt(128))
     float rk[kChunk];      // 1 / sqrt(|k|^2 + eps)
+    float fw[2][kChunk];   // b gam r_k per column (the W / P T coefficient scaling)
+    float fk[2][kChunk];   // c r_k per token (Kt's row scaling)
     uint64_t bar_tma, bar_mma;
     uint32_t tmem_base;
 };
-static_assert(sizeof(PrepSmall) <= 3072, "PrepSmall fits its region");
+static_assert(sizeof(PrepSmall) <= 4096, "PrepSmall fits its region");
 
 __global__ void __launch_bounds__(kPrepThreads, 2)
 chunk_prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
@@ -337,8 +339,7 @@ chunk_prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
 
         // ---- 3. decay masks from the Gram's key columns (64 + 32 hf ..): quarters 0-1 (Q rows)
         //         P = lower(exp(G_r - G_j) r_q r_k Q K^T) of both heads, row-major; quarters 2-3
-        //         (K rows) A = strictly_lower(b_r exp(G_r - G_j) r_k r_k K K^T), its two 32x32
-        //         diagonal blocks stored transposed (for the forward substitution).
+        //         (K rows) A = strictly_lower(b_r exp(G_r - G_j) r_k r_k K K^T), row-major.
         float row[32];
         const int r = (qw & 1) * 32 + lane;  // token row
         const int j0 = 32 * hf;              // first key column of this thread
@@ -369,18 +370,16 @@ chunk_prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
             for (int hh = 0; hh < 2; ++hh) {
                 const float Gr = ss.G[hh][r], br = ss.b[hh][r] * sr;
                 const float* gj = ss.G[hh] + j0;
-                float* A = AT + hh * kMat;
-                float a[32];
+                float4* a4 = reinterpret_cast<float4*>(AT + hh * kMat + r * kLdA + j0);
 #pragma unroll
-                for (int e = 0; e < 32; ++e)
-                    a[e] = (j0 + e < r) ? br * fast_exp2(fminf(Gr - gj[e], 0.f)) * rkj[e] * row[e] : 0.f;
-                if ((r >> 5) == hf) {  // diagonal block, transposed: A^T[j][r]
+                for (int m = 0; m < 8; ++m) {
+                    float x4[4];
 #pragma unroll
-                    for (int e = 0; e < 32; ++e) A[(j0 + e) * kLdA + r] = a[e];
-                } else if (hf < (r >> 5)) {  // A21, row-major
-                    float4* a4 = reinterpret_cast<float4*>(A + r * kLdA + j0);
-#pragma unroll
-                    for (int m = 0; m < 8; ++m) a4[m] = make_float4(a[4 * m], a[4 * m + 1], a[4 * m + 2], a[4 * m + 3]);
+                    for (int e = 0; e < 4; ++e) {
+                        const int i = 4 * m + e;
+                        x4[e] = (j0 + i < r) ? br * fast_exp2(fminf(Gr - gj[i], 0.f)) * rkj[i] * row[i] : 0.f;
+                    }
+                    a4[m] = make_float4(x4[0], x4[1], x4[2], x4[3]);
                 }
             }
         }
@@ -388,118 +387,61 @@ chunk_prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
     tc_fence_before();
     __syncthreads();
 
-    // ---- 4. T = (I + A)^-1 per head, by 32x32 blocks, in place; 128 threads per head.
-    //         With A = [A11 0; A21 A22]:  T = [T1 0; T21 T2], T1 = (I + A11)^-1,
-    //         T2 = (I + A22)^-1, T21 = -T2 (A21 T1).
-    //         (a) T1 and T2 by forward substitution, one warp per block, lane = column j,
-    //             column-oriented: once x_k is known every later row's partial sum takes its
-    //             term, reading row k of the transposed block;
-    //         (b) Y = A21 T1 into the (unused) upper-right block, then T21 = -T2 Y, each thread
-    //             a 4x2 tile; the upper-right block is cleared afterwards.
+    // ---- 4. T = (I + A)^-1 and P T per head, one row per thread: a row x of either satisfies
+    //         x (I + A) = rhs, with rhs = e_r for row r of T and rhs = P_r for row r of P T, and A
+    //         strictly lower triangular, so x_j = rhs_j - sum_{i > j} x_i A_ij.  Taking i from the
+    //         top down, x_i is final when reached and its terms go to every lower x_j at once
+    //         (row i of A, read by all threads of the head as broadcasts).  Both right-hand sides
+    //         vanish past column r, so x does too: a warp starts at its last row.
     {
-        const int hh = tid >> 7, l = tid & 127;
-        float* A = AT + hh * kMat;
-        if (l < 64) {
-            const int base = 32 * (l >> 5), j = l & 31;
-            float acc[32];
+        // Rows 32..63 take about four times the work of rows 0..31; warp w runs on scheduler w % 4,
+        // so the second head takes its row halves the other way round and every scheduler gets
+        // one long and one short warp of each CTA.
+        const int hh = tid >> 7, l = tid & 127, rr = (l & 63) ^ (32 * hh);
+        const bool trow = l < 64;
+        const float* A = AT + hh * kMat;
+        float2 x[kChunk / 2];  // x_{2m}, x_{2m+1}
+        if (trow) {
 #pragma unroll
-            for (int rr = 0; rr < 32; ++rr) acc[rr] = 0.f;
+            for (int m = 0; m < kChunk / 2; ++m) x[m] = make_float2(2 * m == rr ? 1.f : 0.f, 2 * m + 1 == rr ? 1.f : 0.f);
+        } else {
+            const float4* pr = reinterpret_cast<const float4*>(PP + hh * kMat + rr * kLdA);
 #pragma unroll
-            for (int kk = 0; kk < 32; ++kk) {
-                const float xk = (kk == j) ? 1.f : ((kk < j) ? 0.f : -acc[kk]);
-                acc[kk] = xk;
-                const float4* at = reinterpret_cast<const float4*>(A + (base + kk) * kLdA + base);  // A^T row kk
+            for (int m = 0; m < kChunk / 4; ++m) {
+                const float4 v = pr[m];
+                x[2 * m] = make_float2(v.x, v.y);
+                x[2 * m + 1] = make_float2(v.z, v.w);
+            }
+        }
+        const int imax = (rr | 31);  // the warp's last row (warp-uniform)
 #pragma unroll
-                for (int r4 = (kk + 1) / 4; r4 < 8; ++r4) {
-                    const float4 a = at[r4];
-                    const float av[4] = {a.x, a.y, a.z, a.w};
+        for (int i = kChunk - 1; i >= 1; --i) {
+            if (i <= imax) {
+                const float xi = (i & 1) ? x[i >> 1].y : x[i >> 1].x;
+                const float2 nx = make_float2(-xi, -xi);
+                const float4* ar = reinterpret_cast<const float4*>(A + i * kLdA);
+                // highest columns first: x_{i-1} is final soonest, so the next step can start while
+                // this one's other terms are still in flight
 #pragma unroll
-                    for (int e = 0; e < 4; ++e)
-                        if (4 * r4 + e > kk) acc[4 * r4 + e] = fmaf(av[e], xk, acc[4 * r4 + e]);
+                for (int m = (i - 1) / 4; m >= 0; --m) {
+                    const float4 a = ar[m];
+                    // pairs (4m, 4m+1) and (4m+2, 4m+3); only columns below i take the term
+                    if (4 * m + 3 < i) x[2 * m + 1] = __ffma2_rn(nx, make_float2(a.z, a.w), x[2 * m + 1]);
+                    else if (4 * m + 2 < i) x[2 * m + 1].x = fmaf(-xi, a.z, x[2 * m + 1].x);
+                    if (4 * m + 1 < i) x[2 * m] = __ffma2_rn(nx, make_float2(a.x, a.y), x[2 * m]);
+                    else x[2 * m].x = fmaf(-xi, a.x, x[2 * m].x);
                 }
             }
-            __syncwarp();  // every lane of this block's warp is done reading A^T
-#pragma unroll
-            for (int rr = 0; rr < 32; ++rr) A[(base + rr) * kLdA + base + j] = acc[rr];
         }
-        __syncthreads();
-        const int tr = l >> 4, tc = l & 15;  // 4x2 output tile: rows 4 tr .., columns 2 tc ..
-        float2 acc2[4];
-        auto tile_product = [&](const float* Lm, const float* Rm) {  // acc2 = Lm (32x32) Rm (32x32)
+        __syncthreads();  // every thread is done reading A and P
+        float4* dst = reinterpret_cast<float4*>((trow ? AT : PP) + hh * kMat + rr * kLdA);
 #pragma unroll
-            for (int i = 0; i < 4; ++i) acc2[i] = make_float2(0.f, 0.f);
-#pragma unroll 2
-            for (int k4 = 0; k4 < 8; ++k4) {
-                float4 a[4];
-                float2 b[4];
-#pragma unroll
-                for (int i = 0; i < 4; ++i) a[i] = *reinterpret_cast<const float4*>(Lm + (4 * tr + i) * kLdA + 4 * k4);
-#pragma unroll
-                for (int e = 0; e < 4; ++e) b[e] = *reinterpret_cast<const float2*>(Rm + (4 * k4 + e) * kLdA + 2 * tc);
-#pragma unroll
-                for (int i = 0; i < 4; ++i) {
-                    acc2[i] = __ffma2_rn(make_float2(a[i].x, a[i].x), b[0], acc2[i]);
-                    acc2[i] = __ffma2_rn(make_float2(a[i].y, a[i].y), b[1], acc2[i]);
-                    acc2[i] = __ffma2_rn(make_float2(a[i].z, a[i].z), b[2], acc2[i]);
-                    acc2[i] = __ffma2_rn(make_float2(a[i].w, a[i].w), b[3], acc2[i]);
-                }
-            }
-        };
-        tile_product(A + 32 * kLdA, A);  // Y = A21 T1
-#pragma unroll
-        for (int i = 0; i < 4; ++i) *reinterpret_cast<float2*>(A + (4 * tr + i) * kLdA + 32 + 2 * tc) = acc2[i];
-        __syncthreads();
-        tile_product(A + 32 * kLdA + 32, A + 32);  // T2 Y
-        __syncthreads();  // every thread is done reading Y and A21
-#pragma unroll
-        for (int i = 0; i < 4; ++i) {
-            *reinterpret_cast<float2*>(A + (32 + 4 * tr + i) * kLdA + 2 * tc) = make_float2(-acc2[i].x, -acc2[i].y);
-            *reinterpret_cast<float2*>(A + (4 * tr + i) * kLdA + 32 + 2 * tc) = make_float2(0.f, 0.f);
-        }
+        for (int m = 0; m < kChunk / 4; ++m) dst[m] = make_float4(x[2 * m].x, x[2 * m].y, x[2 * m + 1].x, x[2 * m + 1].y);
     }
-    __syncthreads();
-
-    // ---- 5. P T per head in fp32, over P in place.  Both are lower triangular, so row block
-    //         r0 .. r0+3 only needs i <= r0 + 3.  A warp takes 16 rows; lane = (row quad, 8
-    //         columns); every warp's loop bound is uniform.
-    {
-        const int hh = tid >> 7, l = tid & 127, wh = l >> 5, ln = l & 31;
-        const int r0 = 16 * wh + 4 * (ln >> 3), c0 = 8 * (ln & 7);
-        float* Pm = PP + hh * kMat;
-        const float* Tm = AT + hh * kMat;
-        float2 acc[4][4];
-#pragma unroll
-        for (int rr = 0; rr < 4; ++rr)
-#pragma unroll
-            for (int e = 0; e < 4; ++e) acc[rr][e] = make_float2(0.f, 0.f);
-        const int iend = 16 * wh + 16;
-#pragma unroll 1
-        for (int i = 0; i < iend; i += 4) {
-            float4 p[4];
-#pragma unroll
-            for (int rr = 0; rr < 4; ++rr) p[rr] = *reinterpret_cast<const float4*>(Pm + (r0 + rr) * kLdA + i);
-#pragma unroll
-            for (int ii = 0; ii < 4; ++ii) {
-                const float4 ta = *reinterpret_cast<const float4*>(Tm + (i + ii) * kLdA + c0);
-                const float4 tb = *reinterpret_cast<const float4*>(Tm + (i + ii) * kLdA + c0 + 4);
-                const float2 t2[4] = {make_float2(ta.x, ta.y), make_float2(ta.z, ta.w), make_float2(tb.x, tb.y),
-                                      make_float2(tb.z, tb.w)};
-#pragma unroll
-                for (int rr = 0; rr < 4; ++rr) {
-                    const float pv = ii == 0 ? p[rr].x : ii == 1 ? p[rr].y : ii == 2 ? p[rr].z : p[rr].w;
-                    const float2 p2 = make_float2(pv, pv);
-#pragma unroll
-                    for (int e = 0; e < 4; ++e) acc[rr][e] = __ffma2_rn(p2, t2[e], acc[rr][e]);
-                }
-            }
-        }
-        __syncthreads();  // P is read by everyone before it is overwritten
-#pragma unroll
-        for (int rr = 0; rr < 4; ++rr) {
-            float4* dst = reinterpret_cast<float4*>(Pm + (r0 + rr) * kLdA + c0);
-            dst[0] = make_float4(acc[rr][0].x, acc[rr][0].y, acc[rr][1].x, acc[rr][1].y);
-            dst[1] = make_float4(acc[rr][2].x, acc[rr][2].y, acc[rr][3].x, acc[rr][3].y);
-        }
+    if (tid < 128) {  // per-column factors of step 6, once
+        const int hh = tid >> 6, i = tid & 63;
+        ss.fw[hh][i] = ss.b[hh][i] * ss.gam[hh][i] * ss.rk[i];
+        ss.fk[hh][i] = ss.c[hh][i] * ss.rk[i];
     }
     __syncthreads();
 
@@ -516,7 +458,7 @@ chunk_prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
         const int h = h0 + hh;
         unsigned char* rec = ws + L.rec + ((size_t)cid * hv + h) * kRecBytes;
         const float* bb = ss.b[hh];
-        const float* gm = ss.gam[hh];
+        const float* fw = ss.fw[hh];
         {
             const float* src = (trow ? AT : PP) + hh * kMat + rr * kLdA;
             const uint32_t ta = tmem + ((uint32_t)(l & ~31) << 16) + 128 + 64 * hh;
@@ -525,14 +467,11 @@ chunk_prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
             for (int ch = 0; ch < 8; ++ch) {
                 const float4 x0 = *reinterpret_cast<const float4*>(src + 8 * ch);
                 const float4 x1 = *reinterpret_cast<const float4*>(src + 8 * ch + 4);
-                const float v[8] = {x0.x, x0.y, x0.z, x0.w, x1.x, x1.y, x1.z, x1.w};
-                float cw[8];
-#pragma unroll
-                for (int e = 0; e < 8; ++e) {
-                    const int i = 8 * ch + e;
-                    const float x = v[e] * bb[i] * gm[i] * ss.rk[i];
-                    cw[e] = trow ? x : -x;
-                }
+                const float4 f0 = *reinterpret_cast<const float4*>(fw + 8 * ch);
+                const float4 f1 = *reinterpret_cast<const float4*>(fw + 8 * ch + 4);
+                const float sg = trow ? 1.f : -1.f;
+                const float cw[8] = {sg * x0.x * f0.x, sg * x0.y * f0.y, sg * x0.z * f0.z, sg * x0.w * f0.w,
+                                     sg * x1.x * f1.x, sg * x1.y * f1.y, sg * x1.z * f1.z, sg * x1.w * f1.w};
 #pragma unroll
                 for (int e = 0; e < 4; ++e) {
                     uint32_t hi, lo;
@@ -572,23 +511,31 @@ chunk_prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
                 *reinterpret_cast<uint4*>(ta_lo + sw128(row, ch)) = make_uint4(tl[0], tl[1], tl[2], tl[3]);
             }
         }
-        {   // (c) Kt = diag(c r_k) K in fp32, K-major (tokens contiguous): 16-byte chunk i = l + 128 m
-            //     of the image is token block i / 1024, d_k row (i / 8) % 128, chunk i % 8 (tokens
-            //     32 (i / 1024) + 4 (i % 8) ..) -- a warp's store covers four whole 128-byte rows
+        {   // (c) Kt = diag(c r_k) K in fp32, K-major (tokens contiguous).  Thread item i = l + 128 m:
+            //     token block i / 256, d_k rows 4 ((i / 8) % 32) .. + 3, tokens 32 (i / 256) + 4 (i % 8)
+            //     .. + 3: four 8-byte reads of K rows, four 16-byte chunks of Kt rows -- a warp's store
+            //     covers four whole 128-byte rows
             unsigned char* kt = rec + kKTOff;
-            const float* cc = ss.c[hh];
-#pragma unroll 4
-            for (int m = 0; m < 16; ++m) {
+            const float* fk = ss.fk[hh];
+#pragma unroll 2
+            for (int m = 0; m < 4; ++m) {
                 const int i = l + 128 * m;
-                const int kb = i >> 10, dk = (i >> 3) & 127, ch = i & 7;
-                const int t = 32 * kb + 4 * ch;  // first of the chunk's 4 tokens
-                const unsigned char* kcol = sm + kP_QK + (dk >> 6) * 16384 + 8192 + (dk & 7) * 2;
-                float v4[4];
+                const int kb = i >> 8, dk = 4 * ((i >> 3) & 31), tc = i & 7;
+                const int t = 32 * kb + 4 * tc;  // first of the 4 tokens
+                const unsigned char* kblk = sm + kP_QK + (dk >> 6) * 16384 + 8192 + (dk & 7) * 2;
+                float v[4][4];  // [token][d_k]
 #pragma unroll
-                for (int e = 0; e < 4; ++e)
-                    v4[e] = __bfloat162float(*reinterpret_cast<const __nv_bfloat16*>(kcol + sw128(t + e, (dk & 63) >> 3))) *
-                            (cc[t + e] * ss.rk[t + e]);
-                *reinterpret_cast<float4*>(kt + kb * 16384 + sw128(dk, ch)) = make_float4(v4[0], v4[1], v4[2], v4[3]);
+                for (int e = 0; e < 4; ++e) {
+                    const uint2 kr = *reinterpret_cast<const uint2*>(kblk + sw128(t + e, (dk & 63) >> 3));
+                    const float2 a = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&kr.x));
+                    const float2 b = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&kr.y));
+                    const float sc = fk[t + e];
+                    v[e][0] = a.x * sc; v[e][1] = a.y * sc; v[e][2] = b.x * sc; v[e][3] = b.y * sc;
+                }
+#pragma unroll
+                for (int d = 0; d < 4; ++d)
+                    *reinterpret_cast<float4*>(kt + kb * 16384 + sw128(dk + d, tc)) =
+                        make_float4(v[0][d], v[1][d], v[2][d], v[3][d]);
             }
         }
         tmem_st_wait();
