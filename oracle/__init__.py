@@ -14,6 +14,10 @@ Two independent formulations live here:
   UT/WY triangular system, state carry between chunks), used only to cross-check
   :func:`forward` on small inputs.
 
+:func:`gates_from_projections` (and the ``*_from_projections`` wrappers) derive the
+activated gates from raw per-token projections, g = -a softplus(x + b) and
+beta = sigmoid(y); that activation is a stated reading, not given by the pages.
+
 The layer is Gated DeltaNet as named in the Qwen3-Next-80B-A3B model card
 ("Highlights", "Model Overview": 16 QK heads, 32 V heads, head dimension 128); the
 recurrence is S_t = exp(g_t) S_{t-1} (I - beta_t k_t k_t^T) + beta_t v_t k_t^T,
@@ -160,3 +164,53 @@ def forward_heads(q, k, v, g, beta, cu_seqlens, qk_heads, initial_state=None,
                        sel(g, v_heads), sel(beta, v_heads), cu_seqlens, s0, eps=eps,
                        threads=threads)
     return out, fin, v_heads
+
+
+# ---------------------------------------------------------------- gates from raw projections
+# The pages specify the layer in terms of the activated gates: a decay exp(g_t) in (0, 1] and
+# a write strength beta_t in [0, 1].  Serving stacks usually produce both from per-token raw
+# projections.  The reading used here (stated, not on the pages): per V head h,
+#     g_t    = -a_h * softplus(x_t + b_h),   softplus(z) = log(1 + exp(z)),
+#     beta_t = sigmoid(y_t)              = 1 / (1 + exp(-y_t)),
+# with x_t, y_t the raw projections [T, HV], a_h > 0 a per-head decay rate [HV] (the positive
+# rate itself, not its logarithm) and b_h a per-head bias [HV].
+
+def softplus(z):
+    """log(1 + exp(z)) in fp64, written as max(z, 0) + log1p(exp(-|z|)) (the same value,
+    without overflow for large z)."""
+    z = np.asarray(z, dtype=np.float64)
+    return np.maximum(z, 0.0) + np.log1p(np.exp(-np.abs(z)))
+
+
+def sigmoid(y):
+    """1 / (1 + exp(-y)) in fp64 (exp overflow for y << 0 gives the limit 0)."""
+    y = np.asarray(y, dtype=np.float64)
+    with np.errstate(over="ignore"):
+        return 1.0 / (1.0 + np.exp(-y))
+
+
+def gates_from_projections(x, y, a, b):
+    """Activated gates from raw projections: ``(g, beta)``, both ``[T, HV]`` fp64.
+
+    x, y: ``[T, HV]`` raw decay and write-strength projections; a, b: ``[HV]`` per-V-head
+    decay rate and bias.  g = -a * softplus(x + b); beta = sigmoid(y)."""
+    x, y, a, b = (_f64(t) for t in (x, y, a, b))
+    if x.shape != y.shape or x.ndim != 2 or a.shape != (x.shape[1],) or b.shape != (x.shape[1],):
+        raise ValueError("x, y must be [T, HV] and a, b [HV]")
+    return -a[None, :] * softplus(x + b[None, :]), sigmoid(y)
+
+
+def forward_from_projections(q, k, v, x, y, a, b, cu_seqlens, initial_state=None,
+                             eps: float = EPS, threads: int | None = None):
+    """:func:`forward` with the gates taken from raw projections (:func:`gates_from_projections`)."""
+    g, beta = gates_from_projections(x, y, a, b)
+    return forward(q, k, v, g, beta, cu_seqlens, initial_state, eps=eps, threads=threads)
+
+
+def decode_from_projections(q, k, v, x, y, a, b, state, eps: float = EPS, threads: int | None = None):
+    """:func:`decode` with the gates taken from raw projections; x, y are ``[N, ntok, HV]``."""
+    x, y = _f64(x), _f64(y)
+    N, ntok, HV = x.shape
+    g, beta = gates_from_projections(x.reshape(N * ntok, HV), y.reshape(N * ntok, HV), a, b)
+    return decode(q, k, v, g.reshape(N, ntok, HV), beta.reshape(N, ntok, HV), state, eps=eps,
+                  threads=threads)
