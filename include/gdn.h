@@ -194,6 +194,39 @@ gdn_status gdn_decode_commit(float *state, const float *snapshots, const int32_t
                              int32_t num_tokens, const gdn_shape *shape, void *stream);
 
 /*
+ * Gates from raw projections.  The entry points above take the activated gates g <= 0 and
+ * beta in (0, 1).  These three take instead, per token and V head, the raw projections x
+ * (decay) and y (write strength) and per V head a decay rate a > 0 and a bias b, and apply
+ *
+ *     g = -a[h] * softplus(x + b[h]),   softplus(z) = log(1 + exp(z)),
+ *     beta = sigmoid(y) = 1 / (1 + exp(-y))
+ *
+ * in fp32 where the kernels load the gates (no separate pass, nothing written back).  The
+ * pages give only the activated gates; this activation is the usual parameterisation of
+ * the decay and write strength of gated delta rules, offered as an option.
+ *   x, y        same layout as g and beta of the corresponding call ([T][HV], or
+ *               [N][num_tokens][HV] for decode), fp32
+ *   a, b        [HV] fp32, DEVICE memory, 16-byte aligned (GDN_ERR_NULL / GDN_ERR_ALIGN)
+ * Everything else, and every error, as for gdn_chunk_prefill, gdn_decode_step and
+ * gdn_decode_verify.
+ */
+gdn_status gdn_chunk_prefill_raw_gates(const void *q, const void *k, const void *v,
+                                       const float *x, const float *y, const float *a,
+                                       const float *b, const float *initial_state,
+                                       const int32_t *cu_seqlens, void *out, float *final_state,
+                                       const gdn_shape *shape, void *workspace,
+                                       size_t workspace_bytes, void *stream);
+gdn_status gdn_decode_step_raw_gates(const void *q, const void *k, const void *v,
+                                     const float *x, const float *y, const float *a,
+                                     const float *b, float *state_inout, void *out,
+                                     int32_t num_tokens, const gdn_shape *shape, void *stream);
+gdn_status gdn_decode_verify_raw_gates(const void *q, const void *k, const void *v,
+                                       const float *x, const float *y, const float *a,
+                                       const float *b, const float *state, void *out,
+                                       float *snapshots, int32_t num_tokens,
+                                       const gdn_shape *shape, void *stream);
+
+/*
  * Prefill that also keeps the state at every chunk boundary (for prefix caching: the
  * pages' roadmap lists automatic prefix caching for hybrid models -- vLLM blog post,
  * "Future Work" -- which needs the linear-attention state at cached prefix lengths).
@@ -295,6 +328,16 @@ gdn_status gdn_chunk_prefill_noalloc(const void *q, const void *k, const void *v
  * if the runtime reports an error, else GDN_OK.  Meant for tests and debugging.
  */
 gdn_status gdn_get_noalloc_device_error(void *stream);
+
+/*
+ * The device error word of the decode and verify kernels on the current device.  The
+ * multi-token kernels (num_tokens 2..4) wait on asynchronous copies with a bounded wait;
+ * if one gives up, the kernel stops early (the results of that call are undefined) and
+ * records it here.  Synchronises `stream`, returns GDN_ERR_DEVICE_TIMEOUT if a wait gave up
+ * since the last read (and clears the word), GDN_ERR_CUDA if the runtime reports an error,
+ * else GDN_OK.  Meant for tests and debugging.
+ */
+gdn_status gdn_get_decode_device_error(void *stream);
 
 /*
  * Failure-path self-test.  Clears the workspace header, then launches a kernel that waits

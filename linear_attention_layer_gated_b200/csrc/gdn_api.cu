@@ -84,7 +84,7 @@ namespace {
 gdn_status prefill_impl(const void* q, const void* k, const void* v, const float* g, const float* beta,
                         const float* initial_state, const int32_t* cu_seqlens, void* out, float* final_state,
                         gdn::StateSlots map, float* chunk_states, const gdn_shape* shape, void* workspace,
-                        size_t workspace_bytes, void* stream) {
+                        size_t workspace_bytes, gdn::GateAct act, void* stream) {
     gdn_status st = check_prefill_shape(shape);
     if (st != GDN_OK) return st;
     const size_t need = gdn_prefill_workspace_bytes(shape);
@@ -107,7 +107,7 @@ gdn_status prefill_impl(const void* q, const void* k, const void* v, const float
     cudaError_t e;
     if (tensor) {
         e = gdn::launch_prefill_tc_prep(q, k, g, beta, cu_seqlens, shape->num_seqs, shape->total_tokens,
-                                        shape->num_qk_heads, shape->num_v_heads, workspace, s);
+                                        shape->num_qk_heads, shape->num_v_heads, workspace, act, s);
         if (e == cudaSuccess)
             e = gdn::launch_prefill_tc_state(k, v, initial_state, cu_seqlens, out, final_state, map, chunk_states,
                                              shape->num_seqs, shape->total_tokens,
@@ -115,13 +115,13 @@ gdn_status prefill_impl(const void* q, const void* k, const void* v, const float
     } else
         e = gdn::launch_prefill_simt(q, k, v, g, beta, initial_state, cu_seqlens, out,
                                      final_state, map, chunk_states, shape->num_seqs, shape->num_qk_heads,
-                                     shape->num_v_heads, io, s);
+                                     shape->num_v_heads, io, act, s);
     return e == cudaSuccess ? GDN_OK : GDN_ERR_CUDA;
 }
 
 gdn_status decode_impl(const void* q, const void* k, const void* v, const float* g, const float* beta,
                        float* state, gdn::StateSlots map, void* out, float* snapshots, int32_t num_tokens,
-                       const gdn_shape* shape, void* stream) {
+                       const gdn_shape* shape, gdn::GateAct act, void* stream) {
     gdn_status st = check_common(shape);
     if (st != GDN_OK) return st;
     if (num_tokens < 1 || num_tokens > 4) return GDN_ERR_NUM_TOKENS;
@@ -133,7 +133,7 @@ gdn_status decode_impl(const void* q, const void* k, const void* v, const float*
         if (p && !aligned16(p)) return GDN_ERR_ALIGN;
     cudaError_t e = gdn::launch_decode(q, k, v, g, beta, state, map, out, snapshots, num_tokens,
                                        shape->num_seqs, shape->num_qk_heads, shape->num_v_heads,
-                                       (gdn_dtype)shape->io_dtype, reinterpret_cast<cudaStream_t>(stream));
+                                       (gdn_dtype)shape->io_dtype, act, reinterpret_cast<cudaStream_t>(stream));
     return e == cudaSuccess ? GDN_OK : GDN_ERR_CUDA;
 }
 
@@ -154,6 +154,14 @@ gdn_status commit_impl(float* state, gdn::StateSlots map, const float* snapshots
 }
 
 constexpr gdn::StateSlots kDense{nullptr, 0};
+constexpr gdn::GateAct kActivated{nullptr, nullptr};  // g and beta are the activated gates
+
+// The raw-gate parameters: both present and aligned like every other device pointer.
+gdn_status check_gate_params(const float* a, const float* b) {
+    if (!a || !b) return GDN_ERR_NULL;
+    if (!aligned16(a) || !aligned16(b)) return GDN_ERR_ALIGN;
+    return GDN_OK;
+}
 
 gdn_status check_slots(const float* pool, const int32_t* slots, int32_t num_slots) {
     if (!pool || !slots) return GDN_ERR_NULL;
@@ -171,7 +179,7 @@ gdn_status gdn_chunk_prefill(const void* q, const void* k, const void* v, const 
                              const gdn_shape* shape, void* workspace, size_t workspace_bytes,
                              void* stream) {
     return prefill_impl(q, k, v, g, beta, initial_state, cu_seqlens, out, final_state, kDense, nullptr, shape,
-                        workspace, workspace_bytes, stream);
+                        workspace, workspace_bytes, kActivated, stream);
 }
 
 gdn_status gdn_chunk_prefill_chunk_states(const void* q, const void* k, const void* v, const float* g,
@@ -181,7 +189,7 @@ gdn_status gdn_chunk_prefill_chunk_states(const void* q, const void* k, const vo
                                           size_t workspace_bytes, void* stream) {
     if (shape && shape->num_seqs > 0 && shape->total_tokens > 0 && !chunk_states) return GDN_ERR_NULL;
     return prefill_impl(q, k, v, g, beta, initial_state, cu_seqlens, out, final_state, kDense, chunk_states,
-                        shape, workspace, workspace_bytes, stream);
+                        shape, workspace, workspace_bytes, kActivated, stream);
 }
 
 gdn_status gdn_chunk_prefill_slots(const void* q, const void* k, const void* v, const float* g,
@@ -193,7 +201,8 @@ gdn_status gdn_chunk_prefill_slots(const void* q, const void* k, const void* v, 
     gdn_status st = check_slots(state_pool, state_slots, num_slots);
     if (st != GDN_OK) return st;
     return prefill_impl(q, k, v, g, beta, state_pool, cu_seqlens, out, state_pool,
-                        gdn::StateSlots{state_slots, num_slots}, nullptr, shape, workspace, workspace_bytes, stream);
+                        gdn::StateSlots{state_slots, num_slots}, nullptr, shape, workspace, workspace_bytes, kActivated,
+                        stream);
 }
 
 // Shared validation of the two tensor-core prefill phases.
@@ -221,7 +230,7 @@ gdn_status gdn_chunk_prefill_prep(const void* q, const void* k, const float* g, 
         if (p && !aligned16(p)) return GDN_ERR_ALIGN;
     cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
     cudaError_t e = gdn::launch_prefill_tc_prep(q, k, g, beta, cu_seqlens, shape->num_seqs, shape->total_tokens,
-                                                shape->num_qk_heads, shape->num_v_heads, workspace, s);
+                                                shape->num_qk_heads, shape->num_v_heads, workspace, kActivated, s);
     return e == cudaSuccess ? GDN_OK : GDN_ERR_CUDA;
 }
 
@@ -246,7 +255,7 @@ gdn_status gdn_chunk_prefill_state(const void* k, const void* v, const float* in
 gdn_status gdn_decode_step(const void* q, const void* k, const void* v, const float* g,
                            const float* beta, float* state_inout, void* out, int32_t num_tokens,
                            const gdn_shape* shape, void* stream) {
-    return decode_impl(q, k, v, g, beta, state_inout, kDense, out, nullptr, num_tokens, shape, stream);
+    return decode_impl(q, k, v, g, beta, state_inout, kDense, out, nullptr, num_tokens, shape, kActivated, stream);
 }
 
 gdn_status gdn_decode_verify(const void* q, const void* k, const void* v, const float* g,
@@ -254,7 +263,44 @@ gdn_status gdn_decode_verify(const void* q, const void* k, const void* v, const 
                              int32_t num_tokens, const gdn_shape* shape, void* stream) {
     if (shape && shape->num_seqs > 0 && !snapshots) return GDN_ERR_NULL;
     return decode_impl(q, k, v, g, beta, const_cast<float*>(state), kDense, out, snapshots, num_tokens,
-                       shape, stream);
+                       shape, kActivated, stream);
+}
+
+gdn_status gdn_chunk_prefill_raw_gates(const void* q, const void* k, const void* v, const float* x,
+                                       const float* y, const float* a, const float* b,
+                                       const float* initial_state, const int32_t* cu_seqlens, void* out,
+                                       float* final_state, const gdn_shape* shape, void* workspace,
+                                       size_t workspace_bytes, void* stream) {
+    if (shape && shape->num_seqs > 0 && shape->total_tokens > 0) {
+        gdn_status st = check_gate_params(a, b);
+        if (st != GDN_OK) return st;
+    }
+    return prefill_impl(q, k, v, x, y, initial_state, cu_seqlens, out, final_state, kDense, nullptr, shape,
+                        workspace, workspace_bytes, gdn::GateAct{a, b}, stream);
+}
+
+gdn_status gdn_decode_step_raw_gates(const void* q, const void* k, const void* v, const float* x,
+                                     const float* y, const float* a, const float* b, float* state_inout,
+                                     void* out, int32_t num_tokens, const gdn_shape* shape, void* stream) {
+    if (shape && shape->num_seqs > 0) {
+        gdn_status st = check_gate_params(a, b);
+        if (st != GDN_OK) return st;
+    }
+    return decode_impl(q, k, v, x, y, state_inout, kDense, out, nullptr, num_tokens, shape, gdn::GateAct{a, b},
+                       stream);
+}
+
+gdn_status gdn_decode_verify_raw_gates(const void* q, const void* k, const void* v, const float* x,
+                                       const float* y, const float* a, const float* b, const float* state,
+                                       void* out, float* snapshots, int32_t num_tokens, const gdn_shape* shape,
+                                       void* stream) {
+    if (shape && shape->num_seqs > 0) {
+        gdn_status st = check_gate_params(a, b);
+        if (st != GDN_OK) return st;
+        if (!snapshots) return GDN_ERR_NULL;
+    }
+    return decode_impl(q, k, v, x, y, const_cast<float*>(state), kDense, out, snapshots, num_tokens, shape,
+                       gdn::GateAct{a, b}, stream);
 }
 
 gdn_status gdn_decode_commit(float* state, const float* snapshots, const int32_t* accepted,
@@ -271,7 +317,7 @@ gdn_status gdn_decode_step_slots(const void* q, const void* k, const void* v, co
         if (st != GDN_OK) return st;
     }
     return decode_impl(q, k, v, g, beta, state_pool, gdn::StateSlots{state_slots, num_slots}, out, nullptr,
-                       num_tokens, shape, stream);
+                       num_tokens, shape, kActivated, stream);
 }
 
 gdn_status gdn_decode_verify_slots(const void* q, const void* k, const void* v, const float* g,
@@ -284,7 +330,7 @@ gdn_status gdn_decode_verify_slots(const void* q, const void* k, const void* v, 
         if (!snapshots) return GDN_ERR_NULL;
     }
     return decode_impl(q, k, v, g, beta, const_cast<float*>(state_pool), gdn::StateSlots{state_slots, num_slots},
-                       out, snapshots, num_tokens, shape, stream);
+                       out, snapshots, num_tokens, shape, kActivated, stream);
 }
 
 gdn_status gdn_decode_commit_slots(float* state_pool, const int32_t* state_slots, int32_t num_slots,

@@ -60,20 +60,44 @@ __device__ __forceinline__ int state_index(const StateSlots& m, int n, bool& val
     return valid ? s : 0;
 }
 
+// ---------------------------------------------------------------- gates
+// Gates given as raw projections (the *_raw_gates entry points): when `a` is non-null the g
+// and beta arrays hold the raw projections x and y, and every kernel applies, per V head h,
+// g = -a[h] * softplus(x + b[h]) and beta = sigmoid(y) where it loads them.  With `a` null
+// they are the activated gates and are used as they are.
+struct GateAct {
+    const float* a;  // [HV] decay rates (> 0), or nullptr
+    const float* b;  // [HV] biases of the decay projection
+};
+__device__ __forceinline__ float softplus_f32(float z) {  // log(1 + e^z) without overflow
+    return fmaxf(z, 0.f) + log1pf(expf(-fabsf(z)));
+}
+__device__ __forceinline__ float act_g(float x, float a, float b) { return -a * softplus_f32(x + b); }
+__device__ __forceinline__ float act_beta(float y) { return 1.f / (1.f + expf(-y)); }
+__device__ __forceinline__ float load_g(const float* g, size_t idx, const GateAct& act, int h) {
+    const float x = g[idx];
+    return act.a ? act_g(x, act.a[h], act.b[h]) : x;
+}
+__device__ __forceinline__ float load_beta(const float* beta, size_t idx, const GateAct& act) {
+    const float y = beta[idx];
+    return act.a ? act_beta(y) : y;
+}
+
 // ---------------------------------------------------------------- launchers
 // Each returns cudaSuccess or the launch error; arguments were validated by the caller.
 // snap == nullptr: decode step in place; otherwise verify (state read only, per-token
 // states to snap).
 cudaError_t launch_decode(const void* q, const void* k, const void* v, const float* g,
                           const float* beta, float* state, StateSlots map, void* out, float* snap,
-                          int num_tokens, int num_seqs, int hk, int hv, gdn_dtype io, cudaStream_t stream);
+                          int num_tokens, int num_seqs, int hk, int hv, gdn_dtype io, GateAct act,
+                          cudaStream_t stream);
 cudaError_t launch_decode_commit(float* state, StateSlots map, const float* snap, const int32_t* accepted,
                                  int num_tokens, int num_seqs, int hv, cudaStream_t stream);
 
 cudaError_t launch_prefill_simt(const void* q, const void* k, const void* v, const float* g,
                                 const float* beta, const float* s0, const int32_t* cu,
                                 void* out, float* sT, StateSlots map, float* cstates, int num_seqs, int hk,
-                                int hv, gdn_dtype io, cudaStream_t stream);
+                                int hv, gdn_dtype io, GateAct act, cudaStream_t stream);
 
 // Tensor-core prefill (bf16 I/O, num_v_heads / num_qk_heads even): total workspace bytes
 // (header included) and launch.
@@ -82,7 +106,7 @@ size_t tc_workspace_bytes(int num_seqs, int total_tokens, int hk, int hv);
 // (state pass, from k, v and the images).
 cudaError_t launch_prefill_tc_prep(const void* q, const void* k, const float* g, const float* beta,
                                    const int32_t* cu, int num_seqs, int total_tokens, int hk, int hv,
-                                   void* workspace, cudaStream_t stream);
+                                   void* workspace, GateAct act, cudaStream_t stream);
 // cstates (nullable): the state after every chunk, [total chunks][HV][D][D], chunks in
 // sequence order.
 cudaError_t launch_prefill_tc_state(const void* k, const void* v, const float* s0, const int32_t* cu, void* out,

@@ -65,7 +65,7 @@ __global__ void __launch_bounds__(kSimtThreads, 1)
 prefill_simt_kernel(const IO* __restrict__ q, const IO* __restrict__ k, const IO* __restrict__ v,
                     const float* __restrict__ g, const float* __restrict__ beta,
                     const float* s0, const int32_t* __restrict__ cu, IO* __restrict__ out,
-                    float* sT, StateSlots map, float* cstates, int hk, int hv)
+                    float* sT, StateSlots map, float* cstates, int hk, int hv, GateAct act)
 {
     extern __shared__ __align__(16) unsigned char smem_raw[];
     SimtSmem& sm = *reinterpret_cast<SimtSmem*>(smem_raw);
@@ -128,14 +128,14 @@ prefill_simt_kernel(const IO* __restrict__ q, const IO* __restrict__ k, const IO
             sm.V[r][cc] = (r < L) ? to_f32(v[((size_t)(t0 + r) * hv + h) * kD + cv0 + cc]) : 0.f;
         }
         if (warp == 0) {
-            const float g0 = (lane < L) ? g[(size_t)(t0 + lane) * hv + h] : 0.f;
-            const float g1 = (lane + 32 < L) ? g[(size_t)(t0 + lane + 32) * hv + h] : 0.f;
+            const float g0 = (lane < L) ? load_g(g, (size_t)(t0 + lane) * hv + h, act, h) : 0.f;
+            const float g1 = (lane + 32 < L) ? load_g(g, (size_t)(t0 + lane + 32) * hv + h, act, h) : 0.f;
             const float G0 = warp_inclusive_scan(g0, lane);
             const float G1 = warp_inclusive_scan(g1, lane) + __shfl_sync(0xffffffffu, G0, 31);
             sm.G[lane] = G0;
             sm.G[lane + 32] = G1;   // rows >= L repeat the last sum (their g is 0)
-            sm.b[lane] = (lane < L) ? beta[(size_t)(t0 + lane) * hv + h] : 0.f;
-            sm.b[lane + 32] = (lane + 32 < L) ? beta[(size_t)(t0 + lane + 32) * hv + h] : 0.f;
+            sm.b[lane] = (lane < L) ? load_beta(beta, (size_t)(t0 + lane) * hv + h, act) : 0.f;
+            sm.b[lane + 32] = (lane + 32 < L) ? load_beta(beta, (size_t)(t0 + lane + 32) * hv + h, act) : 0.f;
         }
         __syncthreads();
         if (tid < kChunk) {
@@ -337,7 +337,7 @@ template <typename IO>
 cudaError_t launch_typed(const IO* q, const IO* k, const IO* v, const float* g,
                          const float* beta, const float* s0, const int32_t* cu, IO* out,
                          float* sT, StateSlots map, float* cstates, int num_seqs, int hk, int hv,
-                         cudaStream_t stream)
+                         GateAct act, cudaStream_t stream)
 {
     const size_t smem = sizeof(SimtSmem);
     cudaError_t e = cudaFuncSetAttribute(prefill_simt_kernel<IO>,
@@ -345,7 +345,7 @@ cudaError_t launch_typed(const IO* q, const IO* k, const IO* v, const float* g,
     if (e != cudaSuccess) return e;
     const dim3 grid((unsigned)num_seqs * (unsigned)hv * kSlices);
     prefill_simt_kernel<IO><<<grid, kSimtThreads, smem, stream>>>(q, k, v, g, beta, s0, cu, out,
-                                                                   sT, map, cstates, hk, hv);
+                                                                   sT, map, cstates, hk, hv, act);
     return cudaGetLastError();
 }
 
@@ -354,16 +354,16 @@ cudaError_t launch_typed(const IO* q, const IO* k, const IO* v, const float* g,
 cudaError_t launch_prefill_simt(const void* q, const void* k, const void* v, const float* g,
                                 const float* beta, const float* s0, const int32_t* cu,
                                 void* out, float* sT, StateSlots map, float* cstates, int num_seqs, int hk,
-                                int hv, gdn_dtype io, cudaStream_t stream)
+                                int hv, gdn_dtype io, GateAct act, cudaStream_t stream)
 {
     if (num_seqs == 0) return cudaSuccess;
     if (io == GDN_BF16) {
         using T = __nv_bfloat16;
         return launch_typed<T>((const T*)q, (const T*)k, (const T*)v, g, beta, s0, cu, (T*)out,
-                               sT, map, cstates, num_seqs, hk, hv, stream);
+                               sT, map, cstates, num_seqs, hk, hv, act, stream);
     }
     return launch_typed<float>((const float*)q, (const float*)k, (const float*)v, g, beta, s0, cu,
-                               (float*)out, sT, map, cstates, num_seqs, hk, hv, stream);
+                               (float*)out, sT, map, cstates, num_seqs, hk, hv, act, stream);
 }
 
 }  // namespace gdn

@@ -237,7 +237,7 @@ static_assert(sizeof(PrepSmall) <= 4096, "PrepSmall fits its region");
 __global__ void __launch_bounds__(kPrepThreads, 2)
 chunk_prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                   const float* __restrict__ g, const float* __restrict__ beta, unsigned char* ws,
-                  int num_seqs, int total_tokens, int hk, int hv) {
+                  int num_seqs, int total_tokens, int hk, int hv, GateAct act) {
     extern __shared__ unsigned char smem_dyn[];
     unsigned char* sm = reinterpret_cast<unsigned char*>((reinterpret_cast<uintptr_t>(smem_dyn) + 1023) & ~uintptr_t(1023));
     const uint32_t sb = smem_u32(sm);
@@ -283,10 +283,10 @@ chunk_prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
     }
     if (warp < 2) {
         const int h = h0 + warp;
-        const float g0 = (lane < len) ? g[(size_t)(t0 + lane) * hv + h] : 0.f;
-        const float g1 = (lane + 32 < len) ? g[(size_t)(t0 + lane + 32) * hv + h] : 0.f;
-        const float b0 = (lane < len) ? beta[(size_t)(t0 + lane) * hv + h] : 0.f;
-        const float b1 = (lane + 32 < len) ? beta[(size_t)(t0 + lane + 32) * hv + h] : 0.f;
+        const float g0 = (lane < len) ? load_g(g, (size_t)(t0 + lane) * hv + h, act, h) : 0.f;
+        const float g1 = (lane + 32 < len) ? load_g(g, (size_t)(t0 + lane + 32) * hv + h, act, h) : 0.f;
+        const float b0 = (lane < len) ? load_beta(beta, (size_t)(t0 + lane) * hv + h, act) : 0.f;
+        const float b1 = (lane + 32 < len) ? load_beta(beta, (size_t)(t0 + lane + 32) * hv + h, act) : 0.f;
         const float G0 = warp_inclusive_scan(g0, lane);
         const float G1 = warp_inclusive_scan(g1, lane) + __shfl_sync(0xffffffffu, G0, 31);
         const float GL = __shfl_sync(0xffffffffu, G1, 31);  // g = 0 past the length: the last row's sum
@@ -679,10 +679,6 @@ __device__ __forceinline__ bool wait_or_abort(uint64_t* bar, uint32_t parity, vo
     }
 }
 
-__device__ __forceinline__ void mbar_arrive(uint64_t* bar) {
-    asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_u32(bar)) : "memory");
-}
-
 __global__ void __launch_bounds__(kStateThreads, 1)
 chunk_state_kernel(const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_out,
                    const float* s0, const int32_t* __restrict__ cu, __nv_bfloat16* __restrict__ out, float* sT,
@@ -988,7 +984,7 @@ size_t tc_workspace_bytes(int num_seqs, int total_tokens, int hk, int hv) {
 
 cudaError_t launch_prefill_tc_prep(const void* q, const void* k, const float* g, const float* beta,
                                    const int32_t* cu, int num_seqs, int total_tokens, int hk, int hv,
-                                   void* workspace, cudaStream_t stream) {
+                                   void* workspace, GateAct act, cudaStream_t stream) {
     if (num_seqs == 0) return cudaSuccess;
     unsigned char* ws = static_cast<unsigned char*>(workspace);
     const WsLayout L = ws_layout(num_seqs, total_tokens, hv);
@@ -1002,7 +998,7 @@ cudaError_t launch_prefill_tc_prep(const void* q, const void* k, const float* g,
         cudaSuccess)
         return e;
     e = launch_dependent(chunk_prep_kernel, dim3((unsigned)(L.max_chunks * (hv / 2))), dim3(kPrepThreads), kPrepSmem,
-                         stream, tq, tk, g, beta, ws, num_seqs, total_tokens, hk, hv);
+                         stream, tq, tk, g, beta, ws, num_seqs, total_tokens, hk, hv, act);
     if (e != cudaSuccess) return e;
     return cudaGetLastError();
 }

@@ -28,7 +28,8 @@ EXPORTED = ["gdn_prefill_workspace_bytes", "gdn_chunk_prefill", "gdn_chunk_prefi
             "gdn_chunk_prefill_noalloc", "gdn_decode_verify", "gdn_decode_commit",
             "gdn_chunk_prefill_slots", "gdn_decode_step_slots", "gdn_decode_verify_slots",
             "gdn_decode_commit_slots", "gdn_chunk_prefill_chunk_states",
-            "gdn_get_noalloc_device_error"]
+            "gdn_get_noalloc_device_error", "gdn_get_decode_device_error",
+            "gdn_chunk_prefill_raw_gates", "gdn_decode_step_raw_gates", "gdn_decode_verify_raw_gates"]
 
 
 class GdnShape(ctypes.Structure):
@@ -93,6 +94,16 @@ def lib() -> ctypes.CDLL:
             L.gdn_chunk_prefill_noalloc.argtypes = [vp, vp, vp, fp, fp, fp, ip, vp, fp, sp, vp]
             L.gdn_get_noalloc_device_error.restype = ctypes.c_int
             L.gdn_get_noalloc_device_error.argtypes = [vp]
+            L.gdn_get_decode_device_error.restype = ctypes.c_int
+            L.gdn_get_decode_device_error.argtypes = [vp]
+            L.gdn_chunk_prefill_raw_gates.restype = ctypes.c_int
+            L.gdn_chunk_prefill_raw_gates.argtypes = [vp, vp, vp, fp, fp, fp, fp, fp, ip, vp, fp, sp, vp,
+                                                      ctypes.c_size_t, vp]
+            L.gdn_decode_step_raw_gates.restype = ctypes.c_int
+            L.gdn_decode_step_raw_gates.argtypes = [vp, vp, vp, fp, fp, fp, fp, fp, vp, ctypes.c_int32, sp, vp]
+            L.gdn_decode_verify_raw_gates.restype = ctypes.c_int
+            L.gdn_decode_verify_raw_gates.argtypes = [vp, vp, vp, fp, fp, fp, fp, fp, vp, fp, ctypes.c_int32,
+                                                      sp, vp]
             L.gdn_selftest_wait_timeout.restype = ctypes.c_int
             L.gdn_selftest_wait_timeout.argtypes = [vp, ctypes.c_size_t, ctypes.c_uint32, vp]
             L.gdn_status_string.restype = ctypes.c_char_p
@@ -231,6 +242,53 @@ def gdn_decode_verify(q, k, v, g, beta, state, out, snapshots, num_tokens=None, 
         raise GdnError(rc, "gdn_decode_verify")
 
 
+def gdn_chunk_prefill_raw_gates(q, k, v, x, y, a, b, initial_state, cu_seqlens, out, final_state,
+                                workspace=None, algo=GDN_ALGO_AUTO, max_seqlen=0, stream=None):
+    """Calls gdn_chunk_prefill_raw_gates: as gdn_chunk_prefill with the gates given as raw
+    projections x, y [T, HV] and per-V-head a, b [HV] (all fp32)."""
+    if q.dtype != k.dtype or q.dtype != v.dtype or out.dtype != q.dtype:
+        raise TypeError("q, k, v and out must share one dtype")
+    if cu_seqlens.dtype != torch.int32:
+        raise TypeError("cu_seqlens must be int32")
+    shape = prefill_shape(q, v, cu_seqlens, algo, max_seqlen)
+    if workspace is None:
+        workspace = alloc_workspace(shape, q.device)
+    rc = lib().gdn_chunk_prefill_raw_gates(_ptr(q), _ptr(k), _ptr(v), _ptr(x), _ptr(y), _ptr(a), _ptr(b),
+                                           _ptr(initial_state), _ptr(cu_seqlens), _ptr(out),
+                                           _ptr(final_state), ctypes.byref(shape), _ptr(workspace),
+                                           workspace.numel(), _stream(stream))
+    if rc != GDN_OK:
+        raise GdnError(rc, "gdn_chunk_prefill_raw_gates")
+    return workspace
+
+
+def gdn_decode_step_raw_gates(q, k, v, x, y, a, b, state_inout, out, num_tokens=None, stream=None):
+    """Calls gdn_decode_step_raw_gates: as gdn_decode_step with raw projections x, y
+    [N, m, HV] and per-V-head a, b [HV] (all fp32)."""
+    N, m, HK, D = q.shape
+    if num_tokens is None:
+        num_tokens = m
+    shape = make_shape(N, N * m, HK, v.shape[2], D, _io_dtype(q))
+    rc = lib().gdn_decode_step_raw_gates(_ptr(q), _ptr(k), _ptr(v), _ptr(x), _ptr(y), _ptr(a), _ptr(b),
+                                         _ptr(state_inout), _ptr(out), int(num_tokens), ctypes.byref(shape),
+                                         _stream(stream))
+    if rc != GDN_OK:
+        raise GdnError(rc, "gdn_decode_step_raw_gates")
+
+
+def gdn_decode_verify_raw_gates(q, k, v, x, y, a, b, state, out, snapshots, num_tokens=None, stream=None):
+    """Calls gdn_decode_verify_raw_gates: as gdn_decode_verify with raw projections."""
+    N, m, HK, D = q.shape
+    if num_tokens is None:
+        num_tokens = m
+    shape = make_shape(N, N * m, HK, v.shape[2], D, _io_dtype(q))
+    rc = lib().gdn_decode_verify_raw_gates(_ptr(q), _ptr(k), _ptr(v), _ptr(x), _ptr(y), _ptr(a), _ptr(b),
+                                           _ptr(state), _ptr(out), _ptr(snapshots), int(num_tokens),
+                                           ctypes.byref(shape), _stream(stream))
+    if rc != GDN_OK:
+        raise GdnError(rc, "gdn_decode_verify_raw_gates")
+
+
 def gdn_decode_commit(state, snapshots, accepted, num_tokens=None, stream=None):
     """Calls gdn_decode_commit: state[n] <- snapshots[n, accepted[n] - 1] where
     1 <= accepted[n] <= num_tokens (accepted: [N] int32 on the device)."""
@@ -316,6 +374,12 @@ def gdn_chunk_prefill_noalloc(q, k, v, g, beta, initial_state, cu_seqlens, out, 
                                          _ptr(final_state), ctypes.byref(shape), _stream(stream))
     if rc != GDN_OK:
         raise GdnError(rc, "gdn_chunk_prefill_noalloc")
+
+
+def gdn_get_decode_device_error(stream=None) -> int:
+    """Calls gdn_get_decode_device_error: reads and clears the decode kernels' device error
+    word (synchronises the stream).  Returns the gdn_status code."""
+    return int(lib().gdn_get_decode_device_error(_stream(stream)))
 
 
 def gdn_get_noalloc_device_error(stream=None) -> int:

@@ -118,6 +118,21 @@ def make_decode(num_seqs, ntok, *, hk=HK, hv=HV, d=D, io_dtype=torch.bfloat16,
                 state=state)
 
 
+def make_raw_gates(shape, hv=HV, *, scale=1.0, seed=0, device="cpu"):
+    """Raw gate projections for the *_raw_gates entry points: x, y ``shape`` (the token
+    layout of g and beta, last axis = V heads) drawn N(0, scale^2), and per V head a decay
+    rate a ~ U[0.02, 0.2] and a bias b ~ N(0, 0.5^2), all fp32.  (With these, g = -a
+    softplus(x + b) lands mostly in [-0.4, 0]; a large ``scale`` drives both activations
+    into saturation.)"""
+    gen = torch.Generator(device=device)
+    gen.manual_seed(seed)
+    x = torch.randn(shape, generator=gen, device=device, dtype=torch.float32) * scale
+    y = torch.randn(shape, generator=gen, device=device, dtype=torch.float32) * scale
+    a = 0.02 + 0.18 * torch.rand((hv,), generator=gen, device=device, dtype=torch.float32)
+    b = 0.5 * torch.randn((hv,), generator=gen, device=device, dtype=torch.float32)
+    return dict(x=x, y=y, a=a, b=b)
+
+
 def make(w: Workload, device="cpu", **overrides):
     """Materialise a named workload on ``device``."""
     if w.kind == "prefill":

@@ -198,3 +198,24 @@ def test_tensor_path_needs_pairs_of_v_heads_per_qk_head(L):
                                                None)] == "GDN_ERR_UNSUPPORTED"
     assert gdn.STATUS[L.gdn_chunk_prefill_state(FAKE, FAKE, None, FAKE, FAKE, None, ctypes.byref(odd), FAKE,
                                                 1 << 30, None)] == "GDN_ERR_UNSUPPORTED"
+
+
+def test_raw_gate_entry_points_reject_bad_gate_parameters(L):
+    s = shape(num_seqs=4)
+    dec = lambda a=FAKE, b=FAKE, ntok=2: L.gdn_decode_step_raw_gates(  # noqa: E731
+        FAKE, FAKE, FAKE, FAKE, FAKE, a, b, FAKE, FAKE, ntok, ctypes.byref(s), None)
+    ver = lambda a=FAKE, b=FAKE, snap=FAKE: L.gdn_decode_verify_raw_gates(  # noqa: E731
+        FAKE, FAKE, FAKE, FAKE, FAKE, a, b, FAKE, FAKE, snap, 2, ctypes.byref(s), None)
+    for f in (dec, ver):
+        assert gdn.STATUS[f(a=None)] == "GDN_ERR_NULL"
+        assert gdn.STATUS[f(b=None)] == "GDN_ERR_NULL"
+        assert gdn.STATUS[f(a=FAKE + 4)] == "GDN_ERR_ALIGN"
+        assert gdn.STATUS[f(b=FAKE + 8)] == "GDN_ERR_ALIGN"
+    assert gdn.STATUS[ver(snap=None)] == "GDN_ERR_NULL"
+    assert gdn.STATUS[dec(ntok=5)] == "GDN_ERR_NUM_TOKENS"  # then the decode checks
+    ps = shape(num_seqs=1, total_tokens=64)
+    pre = lambda a=FAKE, b=FAKE: L.gdn_chunk_prefill_raw_gates(  # noqa: E731
+        FAKE, FAKE, FAKE, FAKE, FAKE, a, b, None, FAKE, FAKE, None, ctypes.byref(ps), FAKE, 0, None)
+    assert gdn.STATUS[pre(a=None)] == "GDN_ERR_NULL"
+    assert gdn.STATUS[pre(b=FAKE + 4)] == "GDN_ERR_ALIGN"
+    assert gdn.STATUS[pre()] == "GDN_ERR_WORKSPACE"  # then the prefill checks

@@ -56,6 +56,7 @@ def test_decode_full_batch_matches_oracle(ntok):
     assert_close(st, sn_ref, TOL_BF16, "decode state ntok=%d" % ntok)
     assert_rows_close(out, o_ref, 3, TOL_ROW_BF16, "decode out rows ntok=%d" % ntok)
     assert_rows_close(st, sn_ref, 2, TOL_ROW_BF16, "decode state rows ntok=%d" % ntok)
+    assert gdn.STATUS[gdn.gdn_get_decode_device_error()] == "GDN_OK"
 
 
 def test_decode_fp32_io_tight():
@@ -102,6 +103,7 @@ def test_verify_snapshots_match_oracle_and_keep_state(ntok):
         sl = lambda a: a[:, : t + 1].contiguous()  # noqa: E731
         _, s_ref = oracle.decode(sl(x["q"]), sl(x["k"]), sl(x["v"]), sl(x["g"]), sl(x["beta"]), x["state"])
         assert_close(snaps[:, t], s_ref, TOL_BF16, "verify snapshot %d of %d" % (t, ntok))
+    assert gdn.STATUS[gdn.gdn_get_decode_device_error()] == "GDN_OK"
 
 
 def test_commit_installs_the_accepted_snapshot():
