@@ -4,8 +4,8 @@
 // tokens per step, Qwen3-Next model card "Deployment" and the vLLM blog post,
 // "Multi-Token Prediction").
 //
-// One CTA per (sequence n, V head h) streams that head's 128x128 fp32 state (64 KiB)
-// once from HBM and once back, whatever the number of tokens m = 1..4.  The m tokens
+// Each (sequence n, V head h) streams that head's 128x128 fp32 state (64 KiB) once from
+// HBM and once back, whatever the number of tokens m = 1..4.  The m tokens
 // are folded into one pass over the state with the closed form of m consecutive
 // updates.  For state row s0 (one d_v index i) with cumulative gate sums
 // G_t = g_1 + ... + g_t and Gam_t = exp(G_t):
@@ -17,8 +17,13 @@
 //
 // which is the token recurrence unrolled (delta_t is beta_t (v_t - alpha_t S_{t-1} k_t)).
 // The k.k and k.q scalars and the gate factors are per (n, h) and computed once per
-// CTA.
+// (n, h).
 //
+// Two kernels evaluate this.  decode_kernel (the 1-token step, every verify, and fp32 I/O)
+// is described here; decode_mma_kernel (2..4 tokens in place with bf16 I/O) runs the same
+// closed form with its two contractions on warp MMAs and is described at its definition.
+//
+// decode_kernel, one CTA per (sequence n, V head h).
 // Memory: at entry every warp issues asynchronous 16-byte copies (cp.async, no waits
 // that could spin) of its 32 state rows into shared memory, so a CTA has its whole
 // 64 KiB head in flight before it does anything else; three CTAs fit on an SM.
@@ -29,12 +34,14 @@
 // lane l with the complete sum number l, instead of 4 shuffles per sum.  The 16 sums
 // go through shared memory to every lane of the half-warp, each lane evaluates the
 // scalar recurrence for the R rows, and the new rows are streamed to HBM.
+#include <cuda.h>
+
 #include "gdn_internal.cuh"
 #include "sm100.cuh"
 
 namespace gdn {
 
-__device__ unsigned int g_decode_error;  // set when a bounded wait of the streaming kernel gives up
+__device__ unsigned int g_decode_error;  // set when a bounded wait of a decode kernel gives up
 
 namespace {
 
@@ -70,6 +77,12 @@ __device__ __forceinline__ void load_cols(const IO* row, int l, float2* dst) {
 
 __device__ __forceinline__ void cp_async16(void* dst_smem, const void* src) {
     asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(
+                     static_cast<uint32_t>(__cvta_generic_to_shared(dst_smem))),
+                 "l"(src)
+                 : "memory");
+}
+__device__ __forceinline__ void cp_async4(void* dst_smem, const void* src) {
+    asm volatile("cp.async.ca.shared.global [%0], [%1], 4;" ::"r"(
                      static_cast<uint32_t>(__cvta_generic_to_shared(dst_smem))),
                  "l"(src)
                  : "memory");
@@ -286,104 +299,76 @@ decode_kernel(const IO* __restrict__ q, const IO* __restrict__ k, const IO* __re
     }
 }
 
-// ---------------------------------------------------------------- streaming multi-token step
-// For 2..4 tokens the per-row work is several times the 1-token step's.  This kernel keeps
-// one 512-thread CTA per SM and streams (sequence, V head) items through a ring of three
-// shared-memory slots, so that while item i is computed the states of items i+1 and i+2 are
-// on their way.  Each state (64 KiB, contiguous in HBM) arrives by one bulk asynchronous copy
-// that completes on the slot's mbarrier; the small per-item vectors (q, k, v rows and the
-// gates) come by cp.async.  The updated rows go back by bulk copies too (one 4 KiB copy per
-// warp), so the threads issue only shared-memory accesses and arithmetic.
+// ---------------------------------------------------------------- multi-token step on warp MMAs (bf16 I/O)
+// For 2..4 tokens in place with bf16 q, k, v.  The two contractions of the closed form are
+// small matrix products:  the raw products X = S [k_0..k_{m-1} q_0..q_{m-1}]^T (128 x 8, K =
+// 128) and the rank-m update S <- Gam_m S + W K (W: 128 x m per-row coefficients).  Here they
+// run as m16n8k8 tf32 warp MMAs with fp32 accumulation, which takes the multiply-adds, the
+// reductions over the 128 columns and the row update off the CUDA cores (about a third of the
+// instructions of the SIMT kernel).  tf32 keeps 10 mantissa bits, so every fp32 operand x goes
+// in as two terms, x = hi + lo with hi = x rounded to tf32 and lo = x - hi (together about 21
+// bits); bf16 values (q, k, v) are exact in tf32 and need no split.
 //
-// Per item, with three CTA barriers:
-//   B1  the item's state and vectors have landed;
-//       the raw dot products among k_0.., q_0.. (8 lanes per product) and
-//   pass 1: the 2m raw products s.k_t, s.q_t of every state row (a half-warp per R rows,
-//       the transposing butterfly);
-//   B2  the next free slot is refilled (item i+2);
-//   pass 2: one thread per row turns the raw products into the norms, decays and
-//       coefficients and runs the scalar recurrence of the m tokens;
-//   B3
-//   pass 3: the row update s <- Gam_m s + sum_j Et[m-1][j] delta_j k_j / |k_j|, written
-//       back into the slot and copied to HBM by each warp for its 8 rows (with SNAP, every
-//       intermediate state s_t goes straight to the snapshots instead and the state is left
-//       alone; the last snapshot is computed with the same operations as the in-place state).
-constexpr int kStrThreads = 512;
+// One CTA per SM (8 warps) streams (sequence, V head) items through three shared-memory slots:
+// the state (four 2-D tensor copies of 128 rows x 32 columns with the 128-byte swizzle) and the
+// q, k, v rows (bulk copies) of item i+2 are in flight while item i is computed; one barrier per
+// item.  Warp w owns 16 state rows of the item: MMA rows g = 0..7 are state rows 16w + 2g and
+// MMA rows g + 8 are 16w + 2g + 1, which with the swizzle makes every fragment load free of
+// bank conflicts.  The columns are permuted the same way in both products: in k-step / n-tile
+// p, slot t of the MMA is column 8p + 2t and slot t + 4 is column 8p + 2t + 1, so the A
+// fragments of S for the first product are exactly the accumulator fragments of S for the
+// second, and each thread loads its 64 state values once.  The new rows go straight to HBM
+// (each 8-byte store completes a 32-byte sector with its three neighbours).
+constexpr int kMmaWarps = 8;
+constexpr int kVecStride = 272;  // bytes between staged q / k / v rows (bank-conflict padding)
 
-template <typename IO, int NTOK, bool SNAP>
-struct StrLayout {
-    static constexpr int kTokBytes = kD * (int)sizeof(IO);   // one q, k or v row
+template <int NTOK>
+struct MmaLayout {
     static constexpr int kStateBytes = kD * kD * 4;
-    static constexpr int kVec = kStateBytes;                  // q_0.., k_0.., v_0.. rows
-    static constexpr int kG = kVec + 3 * NTOK * kTokBytes;    // g[NTOK], beta[NTOK], a_h, b_h
-    static constexpr int kSlot = (kG + (2 * NTOK + 2) * 4 + 127) / 128 * 128;
-    static constexpr int kCoefStride = SNAP ? 16 : 4;          // per row: [t][j] with SNAP, else [j]
-    static constexpr int kSums = 3 * kSlot;                    // [128][8] raw products
-    static constexpr int kCoef = kSums + 128 * 8 * 4;          // [128][kCoefStride]
-    static constexpr int kOst = kCoef + 128 * kCoefStride * 4;  // [4][128] outputs
-    static constexpr int kDots = kOst + 4 * 128 * 4;           // [8][8] raw vector products
-    static constexpr int kGam = kDots + 64 * 4;                // Gam_t
-    static constexpr int kBar = kGam + 16;                     // full[3], abort flag
-    static constexpr int kSmem = kBar + 32;
+    static constexpr int kVec = kStateBytes;                            // rows k_0.., q_0.., v_0..
+    static constexpr int kTx = kStateBytes + 3 * NTOK * kD * 2;
+    static constexpr int kGate = kVec + 3 * NTOK * kVecStride;         // g_t, beta_t, a_h, b_h; then the slot index
+    static constexpr int kSidx = kGate + 16 * 4;
+    static constexpr int kSlot = (kSidx + 16 + 1023) / 1024 * 1024;
+    static constexpr int kDots = 3 * kSlot;                             // per warp [8][8] floats
+    static constexpr int kBar = kDots + kMmaWarps * 64 * 4;             // full[3], abort flag
+    static constexpr int kSmem = kBar + 32 + 1024;                      // + alignment of the base
 };
 
-template <typename IO>
-__device__ __forceinline__ void load16f(const IO* p, float* x) {  // 16 consecutive elements
-    if constexpr (sizeof(IO) == 4) {
-#pragma unroll
-        for (int c = 0; c < 4; ++c) {
-            const float4 v = reinterpret_cast<const float4*>(p)[c];
-            x[4 * c] = v.x; x[4 * c + 1] = v.y; x[4 * c + 2] = v.z; x[4 * c + 3] = v.w;
-        }
-    } else {
-#pragma unroll
-        for (int c = 0; c < 2; ++c) {
-            const uint4 u = reinterpret_cast<const uint4*>(p)[c];
-            const uint32_t w[4] = {u.x, u.y, u.z, u.w};
-#pragma unroll
-            for (int e = 0; e < 4; ++e) {  // a bf16 value is the upper half of the fp32 with its bits
-                x[8 * c + 2 * e] = __uint_as_float(w[e] << 16);
-                x[8 * c + 2 * e + 1] = __uint_as_float(w[e] & 0xffff0000u);
-            }
-        }
-    }
+__device__ __forceinline__ uint32_t tf32_hi(float x) {
+    uint32_t r;
+    asm("cvt.rna.tf32.f32 %0, %1;" : "=r"(r) : "f"(x));
+    return r;
+}
+// d += a b, m16n8k8, tf32 inputs, fp32 accumulators.
+__device__ __forceinline__ void mma_tf32(float* d, uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3,
+                                         uint32_t b0, uint32_t b1) {
+    asm volatile("mma.sync.aligned.m16n8k8.row.col.f32.tf32.tf32.f32 {%0, %1, %2, %3}, {%4, %5, %6, %7}, "
+                 "{%8, %9}, {%0, %1, %2, %3};"
+                 : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+                 : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
 }
 
-__device__ __forceinline__ void cp_async4(void* dst_smem, const void* src) {
-    asm volatile("cp.async.ca.shared.global [%0], [%1], 4;" ::"r"(
-                     static_cast<uint32_t>(__cvta_generic_to_shared(dst_smem))),
-                 "l"(src)
-                 : "memory");
-}
-
-template <typename IO, int NTOK, bool SNAP>
-__global__ void __launch_bounds__(kStrThreads, 1)
-decode_stream_kernel(const IO* __restrict__ q, const IO* __restrict__ k, const IO* __restrict__ v,
-                     const float* __restrict__ g, const float* __restrict__ beta, float* __restrict__ state,
-                     StateSlots map, IO* __restrict__ out, float* __restrict__ snap, int num_seqs, int hk,
-                     int hv, GateAct act) {
+template <int NTOK>
+__global__ void __launch_bounds__(kMmaWarps * 32, 1)
+decode_mma_kernel(const __grid_constant__ CUtensorMap tm_state, const __nv_bfloat16* __restrict__ q,
+                  const __nv_bfloat16* __restrict__ k, const __nv_bfloat16* __restrict__ v,
+                  const float* __restrict__ g, const float* __restrict__ beta, float* __restrict__ state,
+                  StateSlots map, __nv_bfloat16* __restrict__ out, int num_seqs, int hk, int hv, GateAct act) {
     using namespace sm100;
-    using Lay = StrLayout<IO, NTOK, SNAP>;
-    constexpr int NT = NTOK == 3 ? 4 : NTOK;  // sums per kind, padded to a power of two
-    constexpr int VR = 2 * NT;                // sums per row: x_0.., y_0..
-    constexpr int R = 16 / VR;                // rows per half-warp per butterfly
-    constexpr int kIters = 8 / (2 * R);       // a warp owns 8 rows
-    constexpr int NV = 2 * NTOK;              // vectors k_0.., q_0..
-    constexpr int ND = NV * (NV + 1) / 2;     // products among them
-    constexpr int kDotWarps = (ND * 8 + 31) / 32;
-    constexpr int CS = Lay::kCoefStride;
-    extern __shared__ __align__(128) unsigned char smem[];
-    float* sums = reinterpret_cast<float*>(smem + Lay::kSums);
-    float* coefr = reinterpret_cast<float*>(smem + Lay::kCoef);
-    float* ostage = reinterpret_cast<float*>(smem + Lay::kOst);
-    float* dots = reinterpret_cast<float*>(smem + Lay::kDots);
-    float* gam = reinterpret_cast<float*>(smem + Lay::kGam);
+    using Lay = MmaLayout<NTOK>;
+    constexpr int NV = 2 * NTOK;  // vectors k_0.., q_0.. (n = 0 .. NV-1 of the first product)
+    constexpr int NG = 2 * NTOK + 2;
+    extern __shared__ unsigned char smem_raw[];
+    unsigned char* smem =
+        reinterpret_cast<unsigned char*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    const int gq = lane >> 2, tq = lane & 3;  // MMA group and thread in group
+    float* dots = reinterpret_cast<float*>(smem + Lay::kDots) + warp * 64;
     uint64_t* full = reinterpret_cast<uint64_t*>(smem + Lay::kBar);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + Lay::kBar + 24);
-    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5, half = lane >> 4, l = lane & 15;
     const int items = num_seqs * hv;
     const int first = blockIdx.x, stride = gridDim.x;
-
     if (tid == 0) {
 #pragma unroll
         for (int s = 0; s < 3; ++s) mbar_init(&full[s], 1);
@@ -392,254 +377,266 @@ decode_stream_kernel(const IO* __restrict__ q, const IO* __restrict__ k, const I
     }
     __syncthreads();
 
-    // The vectors of an item: cp.async by the threads, one group per item (empty past the end
-    // or without a state slot, so that every thread's group count stays aligned with the items).
-    auto issue_vectors = [&](int item, int slot) {
-        if (item < items) {
-            const int n = item / hv, h = item % hv, qh = h / (hv / hk);
-            bool has;
-            state_index(map, n, has);
-            if (has) {
-                unsigned char* base = smem + slot * Lay::kSlot;
-                constexpr int kRowChunks = Lay::kTokBytes / 16;
-                for (int c = tid; c < 3 * NTOK * kRowChunks; c += kStrThreads) {
-                    const int which = c / (NTOK * kRowChunks), rem = c % (NTOK * kRowChunks);
-                    const int t = rem / kRowChunks, ch = rem % kRowChunks;
-                    const IO* src = which == 0   ? q + (((size_t)n * NTOK + t) * hk + qh) * kD
-                                    : which == 1 ? k + (((size_t)n * NTOK + t) * hk + qh) * kD
-                                                 : v + (((size_t)n * NTOK + t) * hv + h) * kD;
-                    cp_async16(base + Lay::kVec + (which * NTOK + t) * Lay::kTokBytes + ch * 16,
-                               reinterpret_cast<const unsigned char*>(src) + ch * 16);
-                }
-                if (tid >= kStrThreads - 2 * NTOK - 2) {  // the gates (and a_h, b_h for raw gates)
-                    const int e = tid - (kStrThreads - 2 * NTOK - 2), t = e % NTOK;
-                    if (e < 2 * NTOK)
-                        cp_async4(base + Lay::kG + e * 4, (e < NTOK ? g : beta) + ((size_t)n * NTOK + t) * hv + h);
-                    else if (act.a)
-                        cp_async4(base + Lay::kG + e * 4, (e == 2 * NTOK ? act.a : act.b) + h);
-                }
-            }
+    // Thread 0: the state slot of an item (-1: none).  With a slot table this is a load, which
+    // thread 0 issues one item before it needs the value.
+    auto slot_of = [&](int item) -> int {
+        if (item >= items) return -1;
+        bool has;
+        const int sidx = state_index(map, item / hv, has);
+        return has ? sidx : -1;
+    };
+    // Thread 0: the copies of an item into slot s, completing on full[s] (a plain arrival for
+    // an item without a state, so that every item moves its slot's phase on by one).
+    auto issue = [&](int item, int s, int sidx) {
+        const int n = item / hv, h = item % hv, qh = h / (hv / hk);
+        unsigned char* sl = smem + s * Lay::kSlot;
+        *reinterpret_cast<int*>(sl + Lay::kSidx) = sidx;
+        if (sidx < 0) {
+            mbar_arrive(&full[s]);
+            return;
+        }
+        fence_async_smem();  // the CTA's earlier reads of this slot come first
+        mbar_arrive_expect_tx(&full[s], Lay::kTx);
+        const int row0 = (sidx * hv + h) * kD;
+#pragma unroll
+        for (int cb = 0; cb < 4; ++cb) tma_load_2d(sl + cb * 16384, &tm_state, cb * 32, row0, &full[s]);
+#pragma unroll
+        for (int t = 0; t < NTOK; ++t) {
+            const size_t tok = (size_t)n * NTOK + t;
+            bulk_g2s(sl + Lay::kVec + t * kVecStride, k + (tok * hk + qh) * kD, kD * 2, &full[s]);
+            bulk_g2s(sl + Lay::kVec + (NTOK + t) * kVecStride, q + (tok * hk + qh) * kD, kD * 2, &full[s]);
+            bulk_g2s(sl + Lay::kVec + (2 * NTOK + t) * kVecStride, v + (tok * hv + h) * kD, kD * 2, &full[s]);
+        }
+    };
+    // Threads 0 .. NG-1: gate value number `tid` of an item into slot s by cp.async (raw or
+    // activated as given); one cp.async group per item and thread, empty past the end.
+    auto issue_gates = [&](int item, int s) {
+        if (item < items && tid < NG) {
+            const int n = item / hv, h = item % hv, t = tid % NTOK;
+            const float* src = tid < NTOK       ? g + ((size_t)n * NTOK + t) * hv + h
+                               : tid < 2 * NTOK ? beta + ((size_t)n * NTOK + t) * hv + h
+                               : act.a          ? (tid == 2 * NTOK ? act.a + h : act.b + h)
+                                                : nullptr;
+            if (src) cp_async4(smem + s * Lay::kSlot + Lay::kGate + tid * 4, src);
         }
         cp_async_commit();
     };
-    // The state of an item: one bulk copy issued by thread 0 that completes on full[slot]
-    // (a plain arrival completes the phase for an item without a state slot).
-    auto issue_state = [&](int item, int slot) {
-        if (tid == 0 && item < items) {
-            bool has;
-            const int sidx = state_index(map, item / hv, has);
-            if (has) {
-                mbar_arrive_expect_tx(&full[slot], Lay::kStateBytes);
-                bulk_g2s(smem + slot * Lay::kSlot, state + ((size_t)sidx * hv + item % hv) * kD * kD,
-                         Lay::kStateBytes, &full[slot]);
-            } else {
-                mbar_arrive(&full[slot]);
-            }
-        }
-    };
 
-    issue_vectors(first, 0);
-    issue_state(first, 0);
-    issue_vectors(first + stride, 1);
-    issue_state(first + stride, 1);
+    int sidx_ahead = -1;  // thread 0: the state slot of the next item to copy
+    if (tid == 0) {
+        if (first < items) issue(first, 0, slot_of(first));
+        if (first + stride < items) issue(first + stride, 1, slot_of(first + stride));
+        sidx_ahead = slot_of(first + 2 * stride);
+    }
+    if (warp == 0) {
+        issue_gates(first, 0);
+        issue_gates(first + stride, 1);
+    }
+    const int rowA = 16 * warp + 2 * gq, rowB = rowA + 1;  // state rows of MMA rows gq and gq + 8
     int i = 0;
     for (;; ++i) {
         const int item = first + i * stride;
         if (item >= items) break;
         const int slot = i % 3;
         const uint32_t parity = (i / 3) & 1;
-        cp_async_wait<1>();  // this thread's vectors of item i (item i+1's may still be in flight)
+        if (warp == 0) cp_async_wait<1>();  // this thread's gates of item i (item i+1's may be in flight)
         if (tid == 0 && !mbar_wait(&full[slot], parity)) {
             *abort_flag = 1;
             atomicOr(&g_decode_error, 1u);
         }
-        __syncthreads();  // B1
+        __syncthreads();  // item i has landed; every warp is done with item i-1's slot
         if (*abort_flag) break;
-        mbar_try_wait(&full[slot], parity);  // completed: makes the bulk copy's data visible here too
-        const int n = item / hv, h = item % hv;
-        bool has;
-        const int sidx = state_index(map, n, has);
-        issue_vectors(item + 2 * stride, (i + 2) % 3);  // the slot item i-1 used, free since B1
-
-        unsigned char* base = smem + slot * Lay::kSlot;
-        float* Ss = reinterpret_cast<float*>(base);
-        const IO* vecs = reinterpret_cast<const IO*>(base + Lay::kVec);  // q_0.. k_0.. v_0.. rows
-        float2 kv[NTOK][4];
-        if (has) {
-            // ---- raw products among k_0.. (vectors 0..NTOK-1) and q_0.. (NTOK..), 8 lanes each
-            if (warp < kDotWarps) {
-                const int d = tid >> 3, part = tid & 7;
-                float acc = 0.f;
-                int a = 0, b = 0;
-                if (d < ND) {
-                    int rem = d;
-                    while (rem >= NV - a) { rem -= NV - a; ++a; }
-                    b = a + rem;
-                    auto vec = [&](int idx) { return vecs + (idx < NTOK ? NTOK + idx : idx - NTOK) * kD; };
-                    float xa[16], xb[16];
-                    load16f<IO>(vec(a) + 16 * part, xa);
-                    load16f<IO>(vec(b) + 16 * part, xb);
-                    float2 s2 = __fmul2_rn(make_float2(xa[0], xa[1]), make_float2(xb[0], xb[1]));
-#pragma unroll
-                    for (int e = 2; e < 16; e += 2)
-                        s2 = __ffma2_rn(make_float2(xa[e], xa[e + 1]), make_float2(xb[e], xb[e + 1]), s2);
-                    acc = s2.x + s2.y;
-                }
-                acc += __shfl_xor_sync(0xffffffffu, acc, 1);
-                acc += __shfl_xor_sync(0xffffffffu, acc, 2);
-                acc += __shfl_xor_sync(0xffffffffu, acc, 4);
-                if (d < ND && part == 0) {
-                    dots[a * 8 + b] = acc;
-                    dots[b * 8 + a] = acc;
-                }
-            }
-            // ---- pass 1: raw products of every state row with k_t and q_t
-            float2 qv[NTOK][4];
-#pragma unroll
-            for (int t = 0; t < NTOK; ++t) {
-                load_cols(vecs + (NTOK + t) * kD, l, kv[t]);
-                load_cols(vecs + t * kD, l, qv[t]);
-            }
-#pragma unroll
-            for (int it = 0; it < kIters; ++it) {
-                const int row0 = 8 * warp + it * 2 * R + half * R;
-                float a[16];
-#pragma unroll
-                for (int r = 0; r < R; ++r) {
-                    float2 s2[4];
-                    load_cols(Ss + (row0 + r) * kD, l, s2);
-#pragma unroll
-                    for (int t = 0; t < NT; ++t) {
-                        a[r * VR + t] = t < NTOK ? dot8(s2, kv[t < NTOK ? t : 0]) : 0.f;
-                        a[r * VR + NT + t] = t < NTOK ? dot8(s2, qv[t < NTOK ? t : 0]) : 0.f;
-                    }
-                }
-                xpose_reduce<16, 8>(a, l);
-                sums[(row0 + l / VR) * 8 + l % VR] = a[0];
-            }
+        mbar_try_wait(&full[slot], parity);  // completed: makes the copies' data visible here too
+        if (tid == 0 && item + 2 * stride < items) {
+            issue(item + 2 * stride, (i + 2) % 3, sidx_ahead);
+            sidx_ahead = slot_of(item + 3 * stride);
         }
-        if (lane == 0) bulk_wait_read_all();  // this warp's copies of item i-1's rows have left the slot
-        __syncthreads();                      // B2
-        issue_state(item + 2 * stride, (i + 2) % 3);
-        if (has) {
-            // ---- pass 2: coefficients and the recurrence, one thread per row
-            if (tid < kD) {
-                const int row = tid;
-                const float* gg = reinterpret_cast<const float*>(base + Lay::kG);
-                const bool raw = act.a != nullptr;
-                float G[NTOK], bt[NTOK], rk[NTOK], rq[NTOK], Gm[NTOK], Et[NTOK][NTOK];
-                float acc = 0.f;
+        if (warp == 0) issue_gates(item + 2 * stride, (i + 2) % 3);
+        const int n = item / hv, h = item % hv;
+        const unsigned char* sl = smem + slot * Lay::kSlot;
+        const int sidx = *reinterpret_cast<const int*>(sl + Lay::kSidx);
+        if (sidx >= 0) {
+            const unsigned char* vec = sl + Lay::kVec;
+            // ---- fragments: this thread's 64 state values, its vector n = gq (k_gq or q_{gq-m},
+            //      zero past 2m) at columns 8p + 2t, 8p + 2t + 1, and key t at columns 8p + gq
+            float2 sa[16], sb[16];
+            uint32_t vb0[16], vb1[16];
+            float kb[16];
+#pragma unroll
+            for (int p = 0; p < 16; ++p) {
+                const int box = (p >> 2) * 16384;
+                const int chunk = 2 * (p & 3) + (tq >> 1);
+                sa[p] = *reinterpret_cast<const float2*>(sl + box + rowA * 128 + ((chunk ^ (rowA & 7)) << 4) +
+                                                         8 * (tq & 1));
+                sb[p] = *reinterpret_cast<const float2*>(sl + box + rowB * 128 + ((chunk ^ (rowB & 7)) << 4) +
+                                                         8 * (tq & 1));
+                if (gq < NV) {
+                    const uint32_t w = *reinterpret_cast<const uint32_t*>(vec + gq * kVecStride + (8 * p + 2 * tq) * 2);
+                    vb0[p] = w << 16;            // bf16 -> fp32 (exact, and exact in tf32)
+                    vb1[p] = w & 0xffff0000u;
+                } else {
+                    vb0[p] = 0u;
+                    vb1[p] = 0u;
+                }
+                kb[p] = tq < NTOK ? to_f32(reinterpret_cast<const __nv_bfloat16*>(vec + tq * kVecStride)[8 * p + gq])
+                                  : 0.f;
+            }
+            // ---- products among the vectors (rows gq, columns 2t, 2t+1 of V V^T), for the norms
+            //      and the key-key / key-query coefficients, and X = S V^T
+            //      (four accumulators per product, so that the MMAs of one chain are 4-8 long)
+            float d[4] = {0.f, 0.f, 0.f, 0.f};
+            {
+                float dv[4][4], dx[4][4];
+#pragma unroll
+                for (int c = 0; c < 4; ++c)
+#pragma unroll
+                    for (int e = 0; e < 4; ++e) dv[c][e] = dx[c][e] = 0.f;
+#pragma unroll
+                for (int p = 0; p < 16; ++p) {
+                    mma_tf32(dv[p & 3], vb0[p], 0u, vb1[p], 0u, vb0[p], vb1[p]);
+                    // ---- X = S V^T: rows rowA (d[0], d[1]) and rowB (d[2], d[3]), vectors 2t, 2t + 1
+                    const uint32_t a0 = tf32_hi(sa[p].x), a1 = tf32_hi(sb[p].x);
+                    const uint32_t a2 = tf32_hi(sa[p].y), a3 = tf32_hi(sb[p].y);
+                    mma_tf32(dx[p & 3], a0, a1, a2, a3, vb0[p], vb1[p]);
+                    mma_tf32(dx[p & 3], __float_as_uint(sa[p].x - __uint_as_float(a0)),
+                             __float_as_uint(sb[p].x - __uint_as_float(a1)), __float_as_uint(sa[p].y - __uint_as_float(a2)),
+                             __float_as_uint(sb[p].y - __uint_as_float(a3)), vb0[p], vb1[p]);
+                }
+#pragma unroll
+                for (int e = 0; e < 4; ++e) d[e] = (dx[0][e] + dx[1][e]) + (dx[2][e] + dx[3][e]);
+                dots[gq * 8 + 2 * tq] = (dv[0][0] + dv[1][0]) + (dv[2][0] + dv[3][0]);
+                dots[gq * 8 + 2 * tq + 1] = (dv[0][1] + dv[1][1]) + (dv[2][1] + dv[3][1]);
+            }
+            __syncwarp();  // dots
+            // ---- gates and the coefficients every row shares
+            float bt[NTOK], Gm[NTOK], rk[NTOK], rq[NTOK], Et[NTOK][NTOK];
+            {
+                const float* gs = reinterpret_cast<const float*>(sl + Lay::kGate);
+                const float ga = gs[2 * NTOK], gb = gs[2 * NTOK + 1];
+                float G[NTOK], acc = 0.f;
 #pragma unroll
                 for (int t = 0; t < NTOK; ++t) {
-                    acc += raw ? act_g(gg[t], gg[2 * NTOK], gg[2 * NTOK + 1]) : gg[t];
-                    bt[t] = raw ? act_beta(gg[NTOK + t]) : gg[NTOK + t];
+                    const float graw = gs[t];
+                    const float braw = gs[NTOK + t];
+                    acc += act.a ? act_g(graw, ga, gb) : graw;
                     G[t] = acc;
+                    bt[t] = act.a ? act_beta(braw) : braw;
+                    Gm[t] = expf(G[t]);
                     rk[t] = rsqrtf(dots[t * 8 + t] + kNormEps);
                     rq[t] = rsqrtf(dots[(NTOK + t) * 8 + NTOK + t] + kNormEps) * kInvSqrtD;
-                    Gm[t] = expf(G[t]);
                 }
 #pragma unroll
                 for (int t = 0; t < NTOK; ++t)
 #pragma unroll
                     for (int j = 0; j <= t; ++j) Et[t][j] = (j == t) ? 1.f : expf(G[t] - G[j]);
-                if (row == 0) {
+            }
+            // ---- the 8 raw products of rows rowA and rowB, gathered from the 4 threads of the group
+            float xa[8], xb[8];
 #pragma unroll
-                    for (int t = 0; t < NTOK; ++t) gam[t] = Gm[t];
-                }
+            for (int src = 0; src < 4; ++src) {
+                const int from = (lane & ~3) | src;
+                xa[2 * src] = __shfl_sync(0xffffffffu, d[0], from);
+                xa[2 * src + 1] = __shfl_sync(0xffffffffu, d[1], from);
+                xb[2 * src] = __shfl_sync(0xffffffffu, d[2], from);
+                xb[2 * src + 1] = __shfl_sync(0xffffffffu, d[3], from);
+            }
+            // ---- the recurrence of the m tokens for both rows; thread t writes o_t
+            const __nv_bfloat16* vrow = reinterpret_cast<const __nv_bfloat16*>(vec + 2 * NTOK * kVecStride);
+            float wa = 0.f, wb = 0.f;  // Et[m-1][t] delta_t / |k_t| of rows rowA, rowB for t = tq
+#pragma unroll
+            for (int rr = 0; rr < 2; ++rr) {
+                const float* xr = rr ? xb : xa;
+                const int row = rr ? rowB : rowA;
                 float delta[NTOK];
 #pragma unroll
                 for (int t = 0; t < NTOK; ++t) {
-                    float x = Gm[t] * (rk[t] * sums[row * 8 + t]);
+                    float x = Gm[t] * (rk[t] * xr[t]);
 #pragma unroll
                     for (int j = 0; j < t; ++j) x = fmaf(Et[t][j] * dots[j * 8 + t] * rk[j] * rk[t], delta[j], x);
-                    delta[t] = bt[t] * (to_f32(vecs[(2 * NTOK + t) * kD + row]) - x);
-                    float o = Gm[t] * (rq[t] * sums[row * 8 + NT + t]);
+                    delta[t] = bt[t] * (to_f32(vrow[t * (kVecStride / 2) + row]) - x);
+                    float o = Gm[t] * (rq[t] * xr[NTOK + t]);
 #pragma unroll
                     for (int j = 0; j <= t; ++j)
                         o = fmaf(Et[t][j] * dots[j * 8 + NTOK + t] * rk[j] * rq[t], delta[j], o);
-                    ostage[t * kD + row] = o;
+                    if (t == tq) out[(((size_t)n * NTOK + t) * hv + h) * kD + row] = from_f32<__nv_bfloat16>(o);
                 }
 #pragma unroll
-                for (int t = SNAP ? 0 : NTOK - 1; t < NTOK; ++t)
-#pragma unroll
-                    for (int j = 0; j <= t; ++j)
-                        coefr[row * CS + (SNAP ? t * 4 : 0) + j] = Et[t][j] * rk[j] * delta[j];
+                for (int j = 0; j < NTOK; ++j)
+                    if (j == tq) (rr ? wb : wa) = Et[NTOK - 1][j] * rk[j] * delta[j];
             }
-            __syncthreads();  // B3
-            // ---- pass 3: the new rows (or the snapshots); the outputs
+            // ---- S <- Gam_m S + W K: A = [W_hi | W_lo] (slots t, t + 4 = key t), B = key t at
+            //      columns 8p + gq (twice), C = Gam_m S
+            const uint32_t wa_hi = tf32_hi(wa), wb_hi = tf32_hi(wb);
+            const uint32_t wa_lo = __float_as_uint(wa - __uint_as_float(wa_hi));
+            const uint32_t wb_lo = __float_as_uint(wb - __uint_as_float(wb_hi));
+            const float gl = Gm[NTOK - 1];
+            float* dstA = state + ((size_t)sidx * hv + h) * kD * kD + rowA * kD + 2 * tq;
+            float* dstB = dstA + kD;
 #pragma unroll
-            for (int it = 0; it < kIters; ++it) {
-                const int row0 = 8 * warp + it * 2 * R + half * R;
-#pragma unroll
-                for (int r = 0; r < R; ++r) {
-                    const int row = row0 + r;
-                    float2 s2[4];
-                    load_cols(Ss + row * kD, l, s2);
-#pragma unroll
-                    for (int t = SNAP ? 0 : NTOK - 1; t < NTOK; ++t) {
-                        const float2 gt = make_float2(gam[t], gam[t]);
-                        float2 y[4];
-#pragma unroll
-                        for (int c = 0; c < 4; ++c) y[c] = __fmul2_rn(gt, s2[c]);
-#pragma unroll
-                        for (int j = 0; j <= t; ++j) {
-                            const float w = coefr[row * CS + (SNAP ? t * 4 : 0) + j];
-#pragma unroll
-                            for (int c = 0; c < 4; ++c) y[c] = __ffma2_rn(make_float2(w, w), kv[j][c], y[c]);
-                        }
-                        float* dst = SNAP ? snap + (((size_t)n * NTOK + t) * hv + h) * kD * kD + row * kD
-                                          : Ss + row * kD;
-                        const float4 lo = make_float4(y[0].x, y[0].y, y[1].x, y[1].y);
-                        const float4 hi = make_float4(y[2].x, y[2].y, y[3].x, y[3].y);
-                        if constexpr (SNAP) {
-                            __stcs(reinterpret_cast<float4*>(dst + 4 * l), lo);
-                            __stcs(reinterpret_cast<float4*>(dst + 64 + 4 * l), hi);
-                        } else {
-                            *reinterpret_cast<float4*>(dst + 4 * l) = lo;
-                            *reinterpret_cast<float4*>(dst + 64 + 4 * l) = hi;
-                        }
-                    }
-                }
-            }
-            if constexpr (!SNAP) {  // this warp's 8 rows, 4 KiB contiguous in HBM
-                fence_async_smem();
-                __syncwarp();
-                if (lane == 0) {
-                    bulk_s2g(state + ((size_t)sidx * hv + h) * kD * kD + 8 * warp * kD, Ss + 8 * warp * kD,
-                             8 * kD * 4);
-                    bulk_commit();
-                }
-            }
-            if (tid < NTOK * kD) {
-                const int t = tid / kD, row = tid % kD;
-                out[(((size_t)n * NTOK + t) * hv + h) * kD + row] = from_f32<IO>(ostage[t * kD + row]);
+            for (int p = 0; p < 16; ++p) {
+                float y[4] = {gl * sa[p].x, gl * sa[p].y, gl * sb[p].x, gl * sb[p].y};
+                const uint32_t kbits = __float_as_uint(kb[p]);
+                mma_tf32(y, wa_hi, wb_hi, wa_lo, wb_lo, kbits, kbits);
+                __stcs(reinterpret_cast<float2*>(dstA + 8 * p), make_float2(y[0], y[1]));
+                __stcs(reinterpret_cast<float2*>(dstB + 8 * p), make_float2(y[2], y[3]));
             }
         }
     }
-    // Drain: the state copies this CTA still has in flight, then the vectors.
-    if (lane == 0) bulk_wait_all();
-    if (tid == 0 && *abort_flag) {  // loads issued for items i (gave up) and i+1
+    // Drain: after giving up, the next item's copies may still be in flight.
+    if (tid == 0 && *abort_flag) {
         const int nxt = i + 1;
         if (first + nxt * stride < items) mbar_wait(&full[nxt % 3], (nxt / 3) & 1);
     }
     cp_async_wait<0>();
 }
 
-template <typename IO, int NTOK, bool SNAP>
-cudaError_t launch_stream(const IO* q, const IO* k, const IO* v, const float* g, const float* beta, float* state,
-                          StateSlots map, IO* out, float* snap, int num_seqs, int hk, int hv, GateAct act,
-                          cudaStream_t stream) {
-    auto kernel = decode_stream_kernel<IO, NTOK, SNAP>;
-    using Lay = StrLayout<IO, NTOK, SNAP>;
+using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                   const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                   CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+    static EncodeTiledFn fn = [] {
+        void* f = nullptr;
+        cudaDriverEntryPointQueryResult qr;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &f, cudaEnableDefault, &qr) != cudaSuccess ||
+            qr != cudaDriverEntryPointSuccess)
+            return static_cast<EncodeTiledFn>(nullptr);
+        return reinterpret_cast<EncodeTiledFn>(f);
+    }();
+    return fn;
+}
+
+template <int NTOK>
+cudaError_t launch_mma(const __nv_bfloat16* q, const __nv_bfloat16* k, const __nv_bfloat16* v, const float* g,
+                       const float* beta, float* state, StateSlots map, __nv_bfloat16* out, int num_seqs, int hk,
+                       int hv, GateAct act, cudaStream_t stream) {
+    using Lay = MmaLayout<NTOK>;
     static_assert(Lay::kSmem <= 227 * 1024, "shared memory");
+    // The states as a 2-D fp32 tensor [slots * HV * 128 rows][128], boxes of 128 rows x 32
+    // columns (128 bytes, the swizzle width).
+    const long long slots = map.slots ? map.num_slots : num_seqs;
+    if (slots <= 0) return cudaSuccess;  // no sequence has a state: nothing to do
+    if (slots * hv * kD > INT32_MAX) return cudaErrorInvalidValue;  // row numbers are 32-bit
+    EncodeTiledFn fn = encode_fn();
+    if (!fn) return cudaErrorNotSupported;
+    CUtensorMap tm;
+    const cuuint64_t dims[2] = {(cuuint64_t)kD, (cuuint64_t)(slots * hv * kD)};
+    const cuuint64_t strides[1] = {(cuuint64_t)kD * 4};
+    const cuuint32_t box[2] = {32, (cuuint32_t)kD};
+    const cuuint32_t estr[2] = {1, 1};
+    if (fn(&tm, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 2, state, dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+           CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) !=
+        CUDA_SUCCESS)
+        return cudaErrorInvalidValue;
+    auto kernel = decode_mma_kernel<NTOK>;
     cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, Lay::kSmem);
     if (e != cudaSuccess) return e;
     int dev = 0, sms = 0;
     if ((e = cudaGetDevice(&dev)) != cudaSuccess) return e;
     if ((e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev)) != cudaSuccess) return e;
-    const int items = num_seqs * hv;
-    kernel<<<dim3((unsigned)(items < sms ? items : sms)), dim3(kStrThreads), Lay::kSmem, stream>>>(
-        q, k, v, g, beta, state, map, out, snap, num_seqs, hk, hv, act);
+    const long long items = (long long)num_seqs * hv;
+    kernel<<<dim3((unsigned)(items < sms ? items : sms)), dim3(kMmaWarps * 32), Lay::kSmem, stream>>>(
+        tm, q, k, v, g, beta, state, map, out, num_seqs, hk, hv, act);
     return cudaGetLastError();
 }
 
@@ -662,11 +659,28 @@ cudaError_t launch_typed(const IO* q, const IO* k, const IO* v, const float* g,
                          const float* beta, float* state, StateSlots map, IO* out, float* snap, int ntok,
                          int num_seqs, int hk, int hv, GateAct act, cudaStream_t stream)
 {
-    switch (ntok) {  // one token: one CTA per head; 2..4 tokens: the streaming kernel
-    case 1: return launch_one<IO, 1, 8, SNAP>(q, k, v, g, beta, state, map, out, snap, num_seqs, hk, hv, act, stream);
-    case 2: return launch_stream<IO, 2, SNAP>(q, k, v, g, beta, state, map, out, snap, num_seqs, hk, hv, act, stream);
-    case 3: return launch_stream<IO, 3, SNAP>(q, k, v, g, beta, state, map, out, snap, num_seqs, hk, hv, act, stream);
-    default: return launch_stream<IO, 4, SNAP>(q, k, v, g, beta, state, map, out, snap, num_seqs, hk, hv, act, stream);
+    if constexpr (!SNAP) {  // in place
+        if constexpr (sizeof(IO) == 2) {  // bf16: 2..4 tokens on warp MMAs
+            switch (ntok) {
+            case 2: return launch_mma<2>(q, k, v, g, beta, state, map, out, num_seqs, hk, hv, act, stream);
+            case 3: return launch_mma<3>(q, k, v, g, beta, state, map, out, num_seqs, hk, hv, act, stream);
+            case 4: return launch_mma<4>(q, k, v, g, beta, state, map, out, num_seqs, hk, hv, act, stream);
+            default: break;
+            }
+        }
+        switch (ntok) {  // one token, and fp32 I/O: one CTA per (sequence, V head)
+        case 1: return launch_one<IO, 1, 8, false>(q, k, v, g, beta, state, map, out, snap, num_seqs, hk, hv, act, stream);
+        case 2: return launch_one<IO, 2, 4, false>(q, k, v, g, beta, state, map, out, snap, num_seqs, hk, hv, act, stream);
+        case 3: return launch_one<IO, 3, 2, false>(q, k, v, g, beta, state, map, out, snap, num_seqs, hk, hv, act, stream);
+        default: return launch_one<IO, 4, 2, false>(q, k, v, g, beta, state, map, out, snap, num_seqs, hk, hv, act, stream);
+        }
+    } else {  // verify: one CTA per (sequence, V head)
+        switch (ntok) {
+        case 1: return launch_one<IO, 1, 8, true>(q, k, v, g, beta, state, map, out, snap, num_seqs, hk, hv, act, stream);
+        case 2: return launch_one<IO, 2, 4, true>(q, k, v, g, beta, state, map, out, snap, num_seqs, hk, hv, act, stream);
+        case 3: return launch_one<IO, 3, 2, true>(q, k, v, g, beta, state, map, out, snap, num_seqs, hk, hv, act, stream);
+        default: return launch_one<IO, 4, 2, true>(q, k, v, g, beta, state, map, out, snap, num_seqs, hk, hv, act, stream);
+        }
     }
 }
 

@@ -97,8 +97,12 @@ def test_verify_snapshots_match_oracle_and_keep_state(ntok):
     torch.testing.assert_close(st, x["state"], rtol=0, atol=0)  # verify leaves the state alone
     st_d = x["state"].clone()
     out_d = gdn.decode(x["q"], x["k"], x["v"], x["g"], x["beta"], st_d)
-    torch.testing.assert_close(out_v, out_d, rtol=0, atol=0)            # same outputs as decode
-    torch.testing.assert_close(snaps[:, ntok - 1], st_d, rtol=0, atol=0)  # last snapshot = decode state
+    if ntok == 1:  # one kernel serves both: the same operations
+        torch.testing.assert_close(out_v, out_d, rtol=0, atol=0)
+        torch.testing.assert_close(snaps[:, 0], st_d, rtol=0, atol=0)
+    else:  # decode has its own kernel for 2..4 tokens: the same values up to fp32 rounding order
+        assert_close(out_v, out_d.double().cpu().numpy(), 5e-3, "verify vs decode out ntok=%d" % ntok)
+        assert_close(snaps[:, ntok - 1], st_d.double().cpu().numpy(), 1e-5, "last snapshot vs decode state")
     for t in range(ntok):  # snapshot t = the oracle's state after tokens 0..t
         sl = lambda a: a[:, : t + 1].contiguous()  # noqa: E731
         _, s_ref = oracle.decode(sl(x["q"]), sl(x["k"]), sl(x["v"]), sl(x["g"]), sl(x["beta"]), x["state"])
@@ -167,7 +171,8 @@ def test_decode_verify_commit_through_slots_match_dense():
     snaps = torch.empty(N, ntok, 8, 128, 128, device="cuda")
     gdn.gdn_decode_verify_slots(x["q"], x["k"], x["v"], x["g"], x["beta"], p2, slots, out_v, snaps)
     torch.testing.assert_close(p2, pool, rtol=0, atol=0)
-    torch.testing.assert_close(out_v[valid], out_d[valid], rtol=0, atol=0)
+    # verify's kernel differs from the 3-token decode's: the same values up to fp32 rounding order
+    assert_close(out_v[valid], out_d[valid].double().cpu().numpy(), 5e-3, "verify vs decode through slots")
     accepted = torch.tensor([n % (ntok + 1) for n in range(N)], dtype=torch.int32, device="cuda")
     gdn.gdn_decode_commit_slots(p2, slots, snaps, accepted)
     torch.cuda.synchronize()
