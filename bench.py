@@ -351,7 +351,7 @@ def main_ours(args, rank, world, local_rank):
                 r = roofline_of(pb, pf, phase_ms[ph], peaks)
                 r.update(kernels=kernels[ph], ms=phase_ms[ph], algorithmic_bytes=pb, algorithmic_flop=pf)
                 rec["phases"][ph] = r
-            # the benchmark spec's GEMM-phase figure: all GEMM flops over the time of the GEMM phases
+            # the GEMM-phase figure: all GEMM flops over the time of the GEMM phases
             gemm_ms = phase_ms["prep"] + phase_ms["state"]
             rec["gemm_phases_frac_tensor"] = flop / (gemm_ms * 1e-3) / 1e12 / peaks["bf16_tflops"]
         return rec, x, out, fin, ws
@@ -518,7 +518,7 @@ def main_ours(args, rank, world, local_rank):
     cpu_samples = {}
     if want_cpu:  # the layer workload's inputs, as the GPU drew them
         cpu_samples["layer"] = {k2: x[k2].cpu() for k2 in ("q", "k", "v", "g", "beta", "cu_seqlens")}
-    if not args.tokens and args.only != "prefill":
+    if not args.tokens and args.only == "all":
         del x, out, fin, ws
         torch.cuda.empty_cache()
         for name, w2, kw in (("varlen", inputs.workload("varlen"), dict(with_initial=True)),
@@ -607,8 +607,9 @@ def main():
     ap.add_argument("--algo", default="auto", choices=["auto", "simt", "tensor"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true", help="skip the host-buffer end-to-end leg")
-    ap.add_argument("--only", default="all", choices=["all", "prefill"],
-                    help="prefill: skip the decode measurements (profiling runs)")
+    ap.add_argument("--only", default="all", choices=["all", "prefill", "decode"],
+                    help="profiling runs: prefill = the layer workload only; decode = the layer "
+                         "workload and the decode measurements, without the other prefill configs")
     ap.add_argument("--tokens", type=int, default=0,
                     help="override the prefill length (profiling runs; not a bench line)")
     args = ap.parse_args()

@@ -299,8 +299,8 @@ gdn_status gdn_get_device_error(void *workspace, void *stream);
  * inside libgdn.so, which every GPU that loads the library holds until exit.
  *   - Calls no cudaMalloc, cudaFree or other allocating routine.
  *   - Workloads whose gdn_prefill_workspace_bytes(shape) exceeds the maximum are rejected
- *     with GDN_ERR_WORKSPACE (about 28 chunks of 64 tokens with 16 QK / 32 V heads, e.g.
- *     one sequence of up to 1,728 tokens); fp32 I/O or GDN_ALGO_SIMT give
+ *     with GDN_ERR_WORKSPACE (about 21 chunks of 64 tokens with 16 QK / 32 V heads, e.g.
+ *     one sequence of up to 1,343 tokens); fp32 I/O or GDN_ALGO_SIMT give
  *     GDN_ERR_UNSUPPORTED.
  *   - The first call on each device (with that device current) looks up the array's
  *     device address and caches it with the identity of the device's current context;
