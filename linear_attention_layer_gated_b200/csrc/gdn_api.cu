@@ -105,7 +105,11 @@ gdn_status prefill_impl(const void* q, const void* k, const void* v, const float
     // itself; the fp32 path's header is cleared here.
     if (!tensor && cudaMemsetAsync(workspace, 0, kHeaderBytes, s) != cudaSuccess) return GDN_ERR_CUDA;
     cudaError_t e;
-    if (tensor) {
+    if (tensor && gdn::fused_prefill_applies(shape->num_seqs, shape->total_tokens, shape->num_v_heads)) {
+        e = gdn::launch_prefill_tc_fused(q, k, v, g, beta, initial_state, cu_seqlens, out, final_state, map,
+                                         chunk_states, shape->num_seqs, shape->total_tokens, shape->num_qk_heads,
+                                         shape->num_v_heads, workspace, act, s);
+    } else if (tensor) {
         e = gdn::launch_prefill_tc_prep(q, k, g, beta, cu_seqlens, shape->num_seqs, shape->total_tokens,
                                         shape->num_qk_heads, shape->num_v_heads, workspace, act, s);
         if (e == cudaSuccess)

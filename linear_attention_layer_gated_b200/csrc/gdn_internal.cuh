@@ -113,6 +113,15 @@ cudaError_t launch_prefill_tc_state(const void* k, const void* v, const float* s
                                     float* sT, StateSlots map, float* cstates, int num_seqs, int total_tokens, int hk,
                                     int hv, void* workspace, cudaStream_t stream);
 
+// Both phases in one cooperative launch (the state passes wait per chunk for the prep
+// workers of the same launch); applies when the (sequence, V head) chains fill at most half of
+// the SMs and the device supports cooperative launches.
+bool fused_prefill_applies(int num_seqs, int total_tokens, int hv);
+cudaError_t launch_prefill_tc_fused(const void* q, const void* k, const void* v, const float* g, const float* beta,
+                                   const float* s0, const int32_t* cu, void* out, float* sT, StateSlots map,
+                                   float* cstates, int num_seqs, int total_tokens, int hk, int hv, void* workspace,
+                                   GateAct act, cudaStream_t stream);
+
 // Diagnostic: a bounded wait that is guaranteed to expire (failure-path self-test).
 cudaError_t launch_wait_timeout_selftest(void* workspace, uint64_t limit_ns, cudaStream_t stream);
 

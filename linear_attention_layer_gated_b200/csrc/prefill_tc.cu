@@ -73,7 +73,7 @@ constexpr uint32_t kFacLoad = 16;                     // bytes of F the state ke
 constexpr uint32_t kRecBytes = kFacOff + 1024;        // 99,328
 
 struct WsLayout {
-    size_t seq_chunk0, table, rec, total;
+    size_t seq_chunk0, table, flags, rec, total;
     long long max_chunks;
 };
 
@@ -87,6 +87,8 @@ __host__ __device__ inline WsLayout ws_layout(int num_seqs, int total_tokens, in
     off = round_up(off + (size_t)(num_seqs + 1) * 4, 1024);
     L.table = off;
     off = round_up(off + (size_t)L.max_chunks * 16, 1024);
+    L.flags = off;  // per (chunk, pair of V heads): the fused pass's "records complete" flags
+    off = round_up(off + (size_t)L.max_chunks * (hv / 2 > 0 ? hv / 2 : 1) * 4, 1024);
     L.rec = off;
     off += (size_t)L.max_chunks * hv * kRecBytes;
     L.total = round_up(off, 1024);
@@ -95,11 +97,16 @@ __host__ __device__ inline WsLayout ws_layout(int num_seqs, int total_tokens, in
 
 // ===================================================================== K0
 __global__ void __launch_bounds__(1024)
-chunk_table_kernel(const int32_t* __restrict__ cu, int num_seqs, unsigned char* ws) {
+chunk_table_kernel(const int32_t* __restrict__ cu, int num_seqs, int total_tokens, int hv, unsigned char* ws) {
     allow_dependent_launch();
     int32_t* header = reinterpret_cast<int32_t*>(ws);
     if (threadIdx.x == 0) header[0] = 0;  // the device error word of this call
-    const WsLayout L = ws_layout(num_seqs, 0, 1);  // seq_chunk0 and table do not depend on T
+    const WsLayout L = ws_layout(num_seqs, total_tokens, hv);
+    {
+        int32_t* flags = reinterpret_cast<int32_t*>(ws + L.flags);
+        const long long nflags = L.max_chunks * (hv / 2);
+        for (long long i = threadIdx.x; i < nflags; i += blockDim.x) flags[i] = 0;
+    }
     int32_t* seq_chunk0 = reinterpret_cast<int32_t*>(ws + L.seq_chunk0);
     int4* table = reinterpret_cast<int4*>(ws + L.table);
     __shared__ int32_t scan[1024];
@@ -229,56 +236,67 @@ struct PrepSmall {
     float rk[kChunk];      // 1 / sqrt(|k|^2 + eps)
     float fw[2][kChunk];   // b gam r_k per column (the W / P T coefficient scaling)
     float fk[2][kChunk];   // c r_k per token (Kt's row scaling)
-    uint64_t bar_tma, bar_mma;
+    uint64_t bar_tma, bar_mma, bar_drain;
     uint32_t tmem_base;
 };
 static_assert(sizeof(PrepSmall) <= 4096, "PrepSmall fits its region");
+constexpr uint32_t kPrepRegion = kP_SMALL + 4096;  // one prep item's shared memory (1024-aligned)
 
-__global__ void __launch_bounds__(kPrepThreads, 2)
-chunk_prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
-                  const float* __restrict__ g, const float* __restrict__ beta, unsigned char* ws,
-                  int num_seqs, int total_tokens, int hk, int hv, GateAct act) {
-    extern __shared__ unsigned char smem_dyn[];
-    unsigned char* sm = reinterpret_cast<unsigned char*>((reinterpret_cast<uintptr_t>(smem_dyn) + 1023) & ~uintptr_t(1023));
+// Everything one prep item needs besides its place in the CTA.
+struct PrepArgs {
+    const CUtensorMap* tm_q;
+    const CUtensorMap* tm_k;
+    const float* g;
+    const float* beta;
+    unsigned char* ws;
+    int num_seqs, total_tokens, hk, hv;
+    GateAct act;
+    int32_t* ready;  // per (chunk, pair of V heads): set once the item's records are complete, or nullptr
+};
+
+// The barriers of a prep item's 256 threads, initialised once (thread 32 of the item).
+__device__ __forceinline__ void prep_init_barriers(PrepSmall& ss) {
+    mbar_init(&ss.bar_tma, 1);
+    mbar_init(&ss.bar_mma, 1);
+    mbar_init(&ss.bar_drain, 1);
+    fence_mbar_init();
+}
+
+// One prep item, the chunk cid for the V heads 2 pair and 2 pair + 1, by 256 threads (tid
+// 0..255, their warps a multiple-of-4-aligned group of the CTA) that synchronise on named
+// barrier bid.  sm is the item's 1024-aligned shared memory (kPrepRegion bytes), tmem its 256
+// Tensor Memory columns; j counts the items these threads have run before, so that the
+// mbarrier phases continue across items.  Returns false (on all 256 threads) if a bounded wait
+// gave up; the caller then records the error and drains.
+__device__ bool prep_item(const PrepArgs& a, int cid, int pair, unsigned char* sm, uint32_t tmem, int tid,
+                          uint32_t bid, uint32_t j) {
     const uint32_t sb = smem_u32(sm);
     PrepSmall& ss = *reinterpret_cast<PrepSmall*>(sm + kP_SMALL);
     float* AT = reinterpret_cast<float*>(sm + kP_AT);  // [head][64][kLdA]
     float* PP = reinterpret_cast<float*>(sm + kP_PP);
-
-    const WsLayout L = ws_layout(num_seqs, total_tokens, hv);
-    int32_t* header = reinterpret_cast<int32_t*>(ws);
-    const int npairs = hv / 2;
-    const int cid = blockIdx.x / npairs;
-    const int h0 = 2 * (blockIdx.x % npairs);  // the two V heads of this CTA
-    const int jq = h0 / (hv / hk);             // their QK head
-    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    const int hv = a.hv;
+    const GateAct act = a.act;
+    const float* g = a.g;
+    const float* beta = a.beta;
+    unsigned char* ws = a.ws;
+    const WsLayout L = ws_layout(a.num_seqs, a.total_tokens, hv);
+    const int h0 = 2 * pair;             // the two V heads of this item
+    const int jq = h0 / (hv / a.hk);     // their QK head
+    const int lane = tid & 31, warp = tid >> 5;
     const int qw = warp & 3, hf = warp >> 2;  // TMEM lane quarter, column half
-    grid_dependency_wait();    // the chunk table is written
-    allow_dependent_launch();  // the state kernel may be scheduled as SMs free up
-    const int nchunks = header[1];
-    if (cid >= nchunks) return;
     const int4 ent = reinterpret_cast<const int4*>(ws + L.table)[cid];
     const int t0 = ent.y, len = ent.z;
-    int err = 0;
+    const uint32_t ph = j & 1;  // parity of this item's first completion of each barrier
     bool ok;
 
-    // ---- 0. TMEM, barriers; q and k tiles by TMA; warps 0-1 the gates of one head each
-    if (warp == 0) {
-        tmem_alloc(&ss.tmem_base, 256);
-        tmem_relinquish();
-    }
+    // ---- 0. q and k tiles by TMA; warps 0-1 the gates of one head each
     if (tid == 32) {
-        mbar_init(&ss.bar_tma, 1);
-        mbar_init(&ss.bar_mma, 1);
-        fence_mbar_init();
-    }
-    __syncthreads();
-    if (tid == 32) {
+        fence_async_smem();  // a previous item's reads of the tiles come first
         mbar_arrive_expect_tx(&ss.bar_tma, 32768);
 #pragma unroll
         for (int b = 0; b < 2; ++b) {
-            tma_load_2d(sm + kP_QK + b * 16384, &tm_q, jq * kD + b * 64, t0, &ss.bar_tma);
-            tma_load_2d(sm + kP_QK + b * 16384 + 8192, &tm_k, jq * kD + b * 64, t0, &ss.bar_tma);
+            tma_load_2d(sm + kP_QK + b * 16384, a.tm_q, jq * kD + b * 64, t0, &ss.bar_tma);
+            tma_load_2d(sm + kP_QK + b * 16384 + 8192, a.tm_k, jq * kD + b * 64, t0, &ss.bar_tma);
         }
     }
     if (warp < 2) {
@@ -300,13 +318,12 @@ chunk_prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
         ss.c[warp][lane + 32] = (lane + 32 < len) ? expf(GL - G1) : 0.f;
     }
     tc_fence_before();
-    __syncthreads();
+    hbar(bid, 256);
     tc_fence_after();
-    const uint32_t tmem = ss.tmem_base;
 
     // ---- 1. Gram: TMEM[0:128, 0:128] = [Q; K] [Q; K]^T  (M = N = 128, K = 128)
     if (tid == 0) {
-        if (mbar_wait(&ss.bar_tma, 0)) {
+        if (mbar_wait(&ss.bar_tma, ph)) {
             tc_fence_after();
             const uint32_t idesc = idesc_bf16(128, 128, 0, 0);
 #pragma unroll
@@ -317,8 +334,8 @@ chunk_prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
             mma_commit(&ss.bar_mma);
         }
     }
-    ok = mbar_wait(&ss.bar_mma, 0);
-    if (__syncthreads_or(!ok)) { err = 1; goto cleanup; }
+    ok = mbar_wait(&ss.bar_mma, ph);
+    if (hbar_or(bid, 256, !ok)) return false;
     tc_fence_after();
 
     // ---- 2. norms from the Gram's diagonal: row R = 32 qw + lane has q_R.q_R (R < 64) or
@@ -335,7 +352,7 @@ chunk_prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
             if (qw < 2) ss.rq[32 * qw + lane] = rsqrtf(x + kNormEps) * kInvSqrtD;
             else ss.rk[32 * (qw - 2) + lane] = rsqrtf(x + kNormEps);
         }
-        __syncthreads();
+        hbar(bid, 256);
 
         // ---- 3. decay masks from the Gram's key columns (64 + 32 hf ..): quarters 0-1 (Q rows)
         //         P = lower(exp(G_r - G_j) r_q r_k Q K^T) of both heads, row-major; quarters 2-3
@@ -385,7 +402,7 @@ chunk_prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
         }
     }
     tc_fence_before();
-    __syncthreads();
+    hbar(bid, 256);
 
     // ---- 4. T = (I + A)^-1 and P T per head, one row per thread: a row x of either satisfies
     //         x (I + A) = rhs, with rhs = e_r for row r of T and rhs = P_r for row r of P T, and A
@@ -433,7 +450,7 @@ chunk_prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
                 }
             }
         }
-        __syncthreads();  // every thread is done reading A and P
+        hbar(bid, 256);  // every thread is done reading A and P
         float4* dst = reinterpret_cast<float4*>((trow ? AT : PP) + hh * kMat + rr * kLdA);
 #pragma unroll
         for (int m = 0; m < kChunk / 4; ++m) dst[m] = make_float4(x[2 * m].x, x[2 * m].y, x[2 * m + 1].x, x[2 * m + 1].y);
@@ -443,7 +460,7 @@ chunk_prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
         ss.fw[hh][i] = ss.b[hh][i] * ss.gam[hh][i] * ss.rk[i];
         ss.fk[hh][i] = ss.c[hh][i] * ss.rk[i];
     }
-    __syncthreads();
+    hbar(bid, 256);
 
     // ---- 6. per head, 128 threads.
     //   (a) thread l takes row l & 63 of T (l < 64) or of P T (l >= 64) and writes Tensor Memory
@@ -541,7 +558,7 @@ chunk_prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
         tmem_st_wait();
     }
     tc_fence_before();
-    __syncthreads();
+    hbar(bid, 256);
 
     // ---- 7. per head: TMEM[0:128, 0:128] = A_hi K + A_lo K (rows 0-63: W, rows 64-127:
     //         -P T diag(b gam r_k) K); the -W and Qt = diag(gam r_q) Q + (rows 64-127) images are
@@ -559,8 +576,8 @@ chunk_prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
                                 sdesc_sw128(sb + kP_QK + 8192 + (s & 3) * 2048, 16384, 1024), idesc, s > 0);
             mma_commit(&ss.bar_mma);
         }
-        ok = mbar_wait(&ss.bar_mma, (hh + 1) & 1);
-        if (__syncthreads_or(!ok)) { err = 1; goto cleanup; }
+        ok = mbar_wait(&ss.bar_mma, (ph + 1 + hh) & 1);
+        if (hbar_or(bid, 256, !ok)) return false;
         tc_fence_after();
         {
             unsigned char* img = sm + kP_AT + hh * kWQBytes;  // staging image of this head
@@ -592,19 +609,65 @@ chunk_prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
             fence_async_smem();
         }
         tc_fence_before();
-        __syncthreads();  // the product is read before the next head's MMA overwrites it
+        hbar(bid, 256);  // the product is read before the next head's MMA overwrites it
         if (tid == 32) {
             bulk_s2g(ws + L.rec + ((size_t)cid * hv + h0 + hh) * kRecBytes, sm + kP_AT + hh * kWQBytes, kWQBytes);
             bulk_commit();
         }
     }
-cleanup:
-    if (tid == 32) bulk_wait_read_all();  // the image copies have read shared memory before the CTA exits
-    if (err && tid == 0) {
-        atomicOr(header, 1);
-        mma_commit(&ss.bar_mma);  // MMAs issued so far complete before TMEM is freed
-        mbar_wait(&ss.bar_mma, 0);
-        mbar_wait(&ss.bar_mma, 1);
+    // The item's records are complete when the image copies have finished (not only read shared
+    // memory, whose regions the next item reuses) and every thread's direct stores are visible.
+    if (a.ready) {
+        __threadfence();
+        if (tid == 32) {
+            bulk_wait_all();
+            fence_async_global();
+        }
+        hbar(bid, 256);
+        if (tid == 0) st_release_gpu(a.ready + (size_t)cid * (hv / 2) + pair, 1);
+    } else if (tid == 32) {
+        bulk_wait_read_all();
+    }
+    return true;
+}
+
+// After a failed item: this item's MMAs complete before its Tensor Memory is freed or reused
+// (thread 0 of the item; d counts the drains these threads have done before).
+__device__ __forceinline__ void prep_drain(PrepSmall& ss, int tid, uint32_t d) {
+    if (tid == 0) {
+        mma_commit(&ss.bar_drain);
+        mbar_wait(&ss.bar_drain, d & 1);
+    }
+    if (tid == 32) bulk_wait_all();
+}
+
+__global__ void __launch_bounds__(kPrepThreads, 2)
+chunk_prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
+                  const float* __restrict__ g, const float* __restrict__ beta, unsigned char* ws,
+                  int num_seqs, int total_tokens, int hk, int hv, GateAct act) {
+    extern __shared__ unsigned char smem_dyn[];
+    unsigned char* sm = reinterpret_cast<unsigned char*>((reinterpret_cast<uintptr_t>(smem_dyn) + 1023) & ~uintptr_t(1023));
+    PrepSmall& ss = *reinterpret_cast<PrepSmall*>(sm + kP_SMALL);
+    int32_t* header = reinterpret_cast<int32_t*>(ws);
+    const int npairs = hv / 2;
+    const int cid = blockIdx.x / npairs;
+    const int tid = threadIdx.x, warp = tid >> 5;
+    grid_dependency_wait();    // the chunk table is written
+    allow_dependent_launch();  // the state kernel may be scheduled as SMs free up
+    if (cid >= header[1]) return;
+    if (warp == 0) {
+        tmem_alloc(&ss.tmem_base, 256);
+        tmem_relinquish();
+    }
+    if (tid == 32) prep_init_barriers(ss);
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = ss.tmem_base;
+    const PrepArgs a{&tm_q, &tm_k, g, beta, ws, num_seqs, total_tokens, hk, hv, act, nullptr};
+    if (!prep_item(a, cid, blockIdx.x % npairs, sm, tmem, tid, 1, 0)) {
+        if (tid == 0) atomicOr(header, 1);
+        prep_drain(ss, tid, 0);
     }
     tc_fence_before();
     __syncthreads();
@@ -679,31 +742,51 @@ __device__ __forceinline__ bool wait_or_abort(uint64_t* bar, uint32_t parity, vo
     }
 }
 
-__global__ void __launch_bounds__(kStateThreads, 1)
-chunk_state_kernel(const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_out,
-                   const float* s0, const int32_t* __restrict__ cu, __nv_bfloat16* __restrict__ out, float* sT,
-                   StateSlots map, float* cstates, unsigned char* ws, int num_seqs, int total_tokens, int hk,
-                   int hv) {
-    extern __shared__ unsigned char smem_dyn[];
-    unsigned char* sm = reinterpret_cast<unsigned char*>((reinterpret_cast<uintptr_t>(smem_dyn) + 1023) & ~uintptr_t(1023));
+// Bounded wait (one thread) for a flag another CTA of the same launch raises; returns false
+// if it gave up or another thread or CTA has recorded an error.
+__device__ bool wait_flag(const int32_t* flag, volatile int* abort_flag, int32_t* header) {
+    if (ld_acquire_gpu(flag) != 0) {
+        fence_async_global();
+        return true;
+    }
+    const uint64_t t0 = global_timer_ns();
+    while (true) {
+        __nanosleep(200);
+        if (ld_acquire_gpu(flag) != 0) {
+            fence_async_global();  // the bulk copies that follow read what the flag released
+            return true;
+        }
+        if (*abort_flag || *reinterpret_cast<volatile int32_t*>(header) != 0) {
+            *abort_flag = 1;
+            return false;
+        }
+        if (global_timer_ns() - t0 > kWaitLimitNs) {
+            *abort_flag = 1;
+            atomicOr(header, 1);
+            return false;
+        }
+    }
+}
+
+// The state pass of sequence n, V head h, by the CTA's threads 0..447 (any further threads of
+// the CTA take part in its barriers only).  sm is the CTA's 1024-aligned shared memory
+// (kStateSmem bytes), tmem its kTmemCols Tensor Memory columns.  With `ready` set, the loads of
+// chunk c first wait (bounded) for that chunk's flag: the records are then produced while this
+// pass runs, by the other CTAs of the same launch.
+__device__ void state_body(const CUtensorMap* tm_v_p, const CUtensorMap* tm_out_p, const float* s0,
+                           const int32_t* __restrict__ cu, __nv_bfloat16* __restrict__ out, float* sT,
+                           StateSlots map, float* cstates, unsigned char* ws, int num_seqs, int total_tokens,
+                           int hv, int n, int h, unsigned char* sm, uint32_t tmem, const int32_t* ready) {
     const uint32_t sb = smem_u32(sm);
     StateSmall& ss = *reinterpret_cast<StateSmall*>(sm + kS_SMALL);
     volatile int* abort_flag = &ss.abort_flag;
+    const CUtensorMap& tm_v = *tm_v_p;
+    const CUtensorMap& tm_out = *tm_out_p;
 
     const WsLayout L = ws_layout(num_seqs, total_tokens, hv);
     int32_t* header = reinterpret_cast<int32_t*>(ws);
-    const int h = blockIdx.x % hv;
-    const int n = blockIdx.x / hv;
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-    (void)hk;
 
-    // Set-up that needs nothing from the prep kernel runs before the dependency wait (a
-    // CTA of this kernel never shares an SM with a prep CTA: their shared memory does not
-    // fit together, so the Tensor Memory columns are free).
-    if (warp == 0) {
-        tmem_alloc(&ss.tmem_base, kTmemCols);
-        tmem_relinquish();
-    }
     if (tid == 32) {
         for (int s = 0; s < 2; ++s) {
             mbar_init(&ss.full[s], 1);
@@ -722,8 +805,7 @@ chunk_state_kernel(const __grid_constant__ CUtensorMap tm_v, const __grid_consta
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
-    const uint32_t tmem = ss.tmem_base;
-    grid_dependency_wait();  // the prep kernel's workspace is complete and visible
+    grid_dependency_wait();  // (two-phase launch) the prep kernel's workspace is complete and visible
     const int32_t* seq_chunk0 = reinterpret_cast<const int32_t*>(ws + L.seq_chunk0);
     const int cs = seq_chunk0[n], nch = seq_chunk0[n + 1] - cs;
     const int t_begin = cu[n], t_end = cu[n + 1];
@@ -737,7 +819,7 @@ chunk_state_kernel(const __grid_constant__ CUtensorMap tm_v, const __grid_consta
             auto prefetch = [&](int j) {
                 if (j >= nch) return;
                 const unsigned char* rec = rec_of(j);
-                bulk_prefetch_l2(rec, kFacOff + kFacLoad);
+                if (!ready) bulk_prefetch_l2(rec, kFacOff + kFacLoad);  // fused: not written yet
                 const int tj = t_begin + j * kChunk;
                 tma_prefetch_l2_2d(&tm_v, h * kD, tj);
                 tma_prefetch_l2_2d(&tm_v, h * kD + 64, tj);
@@ -752,6 +834,7 @@ chunk_state_kernel(const __grid_constant__ CUtensorMap tm_v, const __grid_consta
                 unsigned char* slot = sm + st * kSlotBytes;
                 const unsigned char* rec = rec_of(k);
                 const int tk = t_begin + k * kChunk;
+                if (ready && !wait_flag(ready + (size_t)(cs + k) * (hv / 2) + h / 2, abort_flag, header)) break;
                 mbar_arrive_expect_tx(&ss.full[st], kSlotTx);
                 bulk_g2s(slot + kSl_WQ, rec, 65536, &ss.full[st]);
                 bulk_g2s(slot + kSl_KT, rec + kKTOff, kKTBytes, &ss.full[st]);
@@ -873,7 +956,7 @@ chunk_state_kernel(const __grid_constant__ CUtensorMap tm_v, const __grid_consta
 #pragma unroll
             for (int m = 0; m < 16; ++m) dst[m] = make_float4(S[4 * m], S[4 * m + 1], S[4 * m + 2], S[4 * m + 3]);
         }
-    } else {
+    } else if (warp < kOutWarp0 + 4) {
         // ------------------------------------------------ output warps
         const int q4 = warp & 3;
         const int dv = 32 * q4 + lane;  // d_v row of O^T this thread reads, all 64 tokens
@@ -915,11 +998,103 @@ chunk_state_kernel(const __grid_constant__ CUtensorMap tm_v, const __grid_consta
         }
         if (lane == 0) bulk_wait_all();  // this warp's output TMA stores have completed
     }
+}
+
+__global__ void __launch_bounds__(kStateThreads, 1)
+chunk_state_kernel(const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_out,
+                   const float* s0, const int32_t* __restrict__ cu, __nv_bfloat16* __restrict__ out, float* sT,
+                   StateSlots map, float* cstates, unsigned char* ws, int num_seqs, int total_tokens, int hk,
+                   int hv) {
+    extern __shared__ unsigned char smem_dyn[];
+    unsigned char* sm = reinterpret_cast<unsigned char*>((reinterpret_cast<uintptr_t>(smem_dyn) + 1023) & ~uintptr_t(1023));
+    StateSmall& ss = *reinterpret_cast<StateSmall*>(sm + kS_SMALL);
+    (void)hk;
+    // Set-up that needs nothing from the prep kernel runs before the dependency wait (a CTA of
+    // this kernel never shares an SM with a prep CTA: their shared memory does not fit
+    // together, so the Tensor Memory columns are free).
+    if (threadIdx.x < 32) {
+        tmem_alloc(&ss.tmem_base, kTmemCols);
+        tmem_relinquish();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = ss.tmem_base;
+    state_body(&tm_v, &tm_out, s0, cu, out, sT, map, cstates, ws, num_seqs, total_tokens, hv, blockIdx.x / hv,
+               blockIdx.x % hv, sm, tmem, nullptr);
+    tc_fence_before();
+    __syncthreads();
+    if (threadIdx.x < 32) {
+        tc_fence_after();
+        tmem_dealloc(tmem, kTmemCols);
+    }
+}
+
+// ===================================================================== K1 + K2 in one launch
+// For a batch with few (sequence, V head) chains the state pass occupies few SMs and the prep
+// pass must finish before it starts.  This cooperative launch runs both at once: CTAs
+// 0 .. nstate-1 are the state passes (one per chain), every other CTA runs two prep workers of
+// 256 threads (halves of the CTA, named barriers 1 and 2, 256 Tensor Memory columns each) that
+// take the (chunk, pair) items in chunk order and raise each item's flag once its records are
+// complete; a state pass waits for a chunk's flag before it loads the chunk.  All CTAs are
+// resident at once (cooperative launch, one CTA per SM), and no prep worker waits for a state
+// pass, so every flag is eventually raised; all waits are bounded and give up when another CTA
+// has recorded an error.
+constexpr int kFusedThreads = 512;
+constexpr uint32_t kFusedSmem = (kStateSmem > 2 * kPrepRegion + 1024) ? kStateSmem : 2 * kPrepRegion + 1024;
+
+__global__ void __launch_bounds__(kFusedThreads, 1)
+chunk_fused_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
+                   const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_out,
+                   const float* __restrict__ g, const float* __restrict__ beta, const float* s0,
+                   const int32_t* __restrict__ cu, __nv_bfloat16* __restrict__ out, float* sT, StateSlots map,
+                   float* cstates, unsigned char* ws, int num_seqs, int total_tokens, int hk, int hv, GateAct act,
+                   int nstate) {
+    extern __shared__ unsigned char smem_dyn[];
+    unsigned char* sm = reinterpret_cast<unsigned char*>((reinterpret_cast<uintptr_t>(smem_dyn) + 1023) & ~uintptr_t(1023));
+    __shared__ uint32_t tmem_s;
+    const int tid = threadIdx.x, warp = tid >> 5;
+    int32_t* header = reinterpret_cast<int32_t*>(ws);
+    const WsLayout L = ws_layout(num_seqs, total_tokens, hv);
+    int32_t* ready = reinterpret_cast<int32_t*>(ws + L.flags);
+    const bool is_state = (int)blockIdx.x < nstate;
+    if (warp == 0) {
+        tmem_alloc(&tmem_s, 512);
+        tmem_relinquish();
+    }
+    if (!is_state && (tid & 255) == 32) prep_init_barriers(*reinterpret_cast<PrepSmall*>(sm + (tid >> 8) * kPrepRegion + kP_SMALL));
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = tmem_s;
+    if (is_state) {
+        state_body(&tm_v, &tm_out, s0, cu, out, sT, map, cstates, ws, num_seqs, total_tokens, hv, blockIdx.x / hv,
+                   blockIdx.x % hv, sm, tmem, ready);
+    } else {
+        const int half = tid >> 8, ltid = tid & 255;
+        const uint32_t bid = 1 + half;
+        unsigned char* hsm = sm + half * kPrepRegion;
+        PrepSmall& ss = *reinterpret_cast<PrepSmall*>(hsm + kP_SMALL);
+        const int npairs = hv / 2;
+        const long long items = (long long)header[1] * npairs;
+        const long long worker = (long long)(blockIdx.x - nstate) * 2 + half;
+        const long long nworkers = (long long)(gridDim.x - nstate) * 2;
+        const PrepArgs a{&tm_q, &tm_k, g, beta, ws, num_seqs, total_tokens, hk, hv, act, ready};
+        uint32_t j = 0;
+        for (long long it = worker; it < items; it += nworkers, ++j) {
+            if (hbar_or(bid, 256, *reinterpret_cast<volatile int32_t*>(header) != 0)) break;  // another CTA gave up
+            if (!prep_item(a, (int)(it / npairs), (int)(it % npairs), hsm, tmem + 256u * half, ltid, bid, j)) {
+                if (ltid == 0) atomicOr(header, 1);
+                prep_drain(ss, ltid, 0);
+                break;
+            }
+        }
+    }
     tc_fence_before();
     __syncthreads();
     if (warp == 0) {
         tc_fence_after();
-        tmem_dealloc(tmem, kTmemCols);
+        tmem_dealloc(tmem, 512);
     }
 }
 
@@ -988,7 +1163,7 @@ cudaError_t launch_prefill_tc_prep(const void* q, const void* k, const float* g,
     if (num_seqs == 0) return cudaSuccess;
     unsigned char* ws = static_cast<unsigned char*>(workspace);
     const WsLayout L = ws_layout(num_seqs, total_tokens, hv);
-    chunk_table_kernel<<<1, 1024, 0, stream>>>(cu, num_seqs, ws);
+    chunk_table_kernel<<<1, 1024, 0, stream>>>(cu, num_seqs, total_tokens, hv, ws);
     cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess || L.max_chunks == 0 || total_tokens == 0) return e;
     CUtensorMap tq, tk;
@@ -1024,6 +1199,55 @@ cudaError_t launch_prefill_tc_state(const void* k, const void* v, const float* s
     e = launch_dependent(chunk_state_kernel, dim3((unsigned)num_seqs * hv), dim3(kStateThreads), kStateSmem, stream, tv,
                          to, s0, cu, (__nv_bfloat16*)out, sT, map, cstates, static_cast<unsigned char*>(workspace),
                          num_seqs, total_tokens, hk, hv);
+    if (e != cudaSuccess) return e;
+    return cudaGetLastError();
+}
+
+bool fused_prefill_applies(int num_seqs, int total_tokens, int hv) {
+    if (num_seqs <= 0 || total_tokens <= 0) return false;
+    int dev = 0, sms = 0, coop = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return false;
+    if (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return false;
+    if (cudaDeviceGetAttribute(&coop, cudaDevAttrCooperativeLaunch, dev) != cudaSuccess || !coop) return false;
+    return 2LL * num_seqs * hv <= sms;
+}
+
+cudaError_t launch_prefill_tc_fused(const void* q, const void* k, const void* v, const float* g, const float* beta,
+                                   const float* s0, const int32_t* cu, void* out, float* sT, StateSlots map,
+                                   float* cstates, int num_seqs, int total_tokens, int hk, int hv, void* workspace,
+                                   GateAct act, cudaStream_t stream) {
+    unsigned char* ws = static_cast<unsigned char*>(workspace);
+    chunk_table_kernel<<<1, 1024, 0, stream>>>(cu, num_seqs, total_tokens, hv, ws);
+    cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess) return e;
+    CUtensorMap tq, tk, tv, to;
+    if ((e = encode_rows(&tq, q, total_tokens, hk)) != cudaSuccess) return e;
+    if ((e = encode_rows(&tk, k, total_tokens, hk)) != cudaSuccess) return e;
+    if ((e = encode_rows(&tv, v, total_tokens, hv)) != cudaSuccess) return e;
+    if ((e = encode_rows(&to, out, total_tokens, hv, CU_TENSOR_MAP_SWIZZLE_NONE, 32, 64)) != cudaSuccess) return e;
+    if ((e = cudaFuncSetAttribute(chunk_fused_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kFusedSmem)) !=
+        cudaSuccess)
+        return e;
+    int dev = 0, sms = 0, per_sm = 0;
+    if ((e = cudaGetDevice(&dev)) != cudaSuccess) return e;
+    if ((e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev)) != cudaSuccess) return e;
+    if ((e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, chunk_fused_kernel, kFusedThreads, kFusedSmem)) !=
+        cudaSuccess)
+        return e;
+    if (per_sm < 1) return cudaErrorInvalidConfiguration;
+    const int nstate = num_seqs * hv;
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3((unsigned)sms);  // one CTA per SM, all resident (cooperative launch)
+    cfg.blockDim = dim3(kFusedThreads);
+    cfg.dynamicSmemBytes = kFusedSmem;
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeCooperative;
+    attr[0].val.cooperative = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    e = cudaLaunchKernelEx(&cfg, chunk_fused_kernel, tq, tk, tv, to, g, beta, s0, cu, (__nv_bfloat16*)out, sT, map,
+                           cstates, ws, num_seqs, total_tokens, hk, hv, act, nstate);
     if (e != cudaSuccess) return e;
     return cudaGetLastError();
 }
