@@ -112,9 +112,10 @@ def load_traffic():
         if source_code_sha256(src) != fields["source_code_sha256"]:
             return {}
         out = {}
-        for kname in ("chunk_table_kernel", "chunk_prep_kernel", "chunk_state_kernel"):
-            parts = fields[kname].split()
-            out[kname] = int(parts[1]) + int(parts[3])
+        for kname in ("chunk_table_kernel", "chunk_prep_kernel", "chunk_state_kernel", "chunk_fused_kernel"):
+            if kname in fields:
+                parts = fields[kname].split()
+                out[kname] = int(parts[1]) + int(parts[3])
         return out
     except (KeyError, OSError, ValueError, IndexError):
         return {}
@@ -368,7 +369,29 @@ def main_ours(args, rank, world, local_rank):
     launches_per_step = gdn_launches_per_prefill(algo, x["q"].dtype)
     phases = main_rec.get("phases")
     step = main_rec["step"]
-    if phases:
+    fused = launches_per_step == 2
+    if fused:
+        # one chunk-table launch and one fused launch per step: the step's events time exactly
+        # them, and the whole step's algorithmic work is the fused kernel's
+        nbytes, flop = prefill_work(T, 1, False, True)
+        tr = load_traffic() if T == 8192 else {}
+        traffic = (tr["chunk_table_kernel"] + tr["chunk_fused_kernel"]) if "chunk_fused_kernel" in tr else None
+        unit_hbm = step["bound"] == "hbm"
+        roofline = {"bound": step["bound"],
+                    "achieved": step["gbs"] if unit_hbm else step["tflops"],
+                    "peak": peaks["hbm_gbs"] if unit_hbm else peaks["bf16_tflops"],
+                    "unit": "GB/s" if unit_hbm else "TFLOP/s",
+                    "frac": step["frac_hbm"] if unit_hbm else step["frac_tensor"],
+                    "traffic": traffic,
+                    "traffic_over_algorithmic_bytes": (traffic / nbytes) if traffic else None,
+                    "peak_source": peaks["source"] + (" HBM copy" if unit_hbm else " bf16 dense (burst)"),
+                    "kernel": "chunk_table_kernel + chunk_fused_kernel (prep and state passes in one cooperative launch)",
+                    "algorithmic_bytes_per_launch": nbytes, "algorithmic_flop_per_launch": flop,
+                    "frac_hbm": step["frac_hbm"], "frac_tensor": step["frac_tensor"],
+                    "step_frac_tensor": step["frac_tensor"], "step_frac_hbm": step["frac_hbm"],
+                    "gemm_phases_frac_tensor": step["frac_tensor"],
+                    "two_phase_path_frac_tensor": main_rec.get("gemm_phases_frac_tensor")}
+    elif phases:
         dom = max(phases, key=lambda k2: phases[k2]["ms"])
         d = phases[dom]
         traffic = None
@@ -582,20 +605,33 @@ def main_ours(args, rank, world, local_rank):
                 "roofline": roofline, "cpu_baseline": cpu,
                 "e2e": e2e,
                 "gpu_launches": launches_per_step * args.steps, "phases": phases,
+                "phases_path": "gdn_chunk_prefill_prep and gdn_chunk_prefill_state, the two-kernel path, timed as "
+                               "separate launches on the same inputs",
                 "gemm_phases_frac_tensor": main_rec.get("gemm_phases_frac_tensor"),
                 "configs": others, "decode": dec, "clocks": clocks, "peaks": peaks}
         print(json.dumps(line), flush=True)
     return 0
 
 
-def gdn_launches_per_prefill(algo, dtype):
+def fused_prefill_applies(num_seqs, hv):
+    """The library's rule for the one-launch tensor-core prefill (prep and state passes in one
+    cooperative kernel): the (sequence, V head) chains fill at most half of the SMs."""
+    import torch
+    props = torch.cuda.get_device_properties(torch.cuda.current_device())
+    return 2 * num_seqs * hv <= props.multi_processor_count
+
+
+def gdn_launches_per_prefill(algo, dtype, num_seqs=1, hv=HV):
     """Kernels libgdn.so launches per gdn_chunk_prefill call on the chosen path:
-    the SIMT path is one kernel; the tensor-core path is chunk table, chunk prep and
-    chunk state (the workspace-header memset is not a kernel of ours)."""
+    the SIMT path is one kernel; the tensor-core path is the chunk table and then either the
+    fused kernel or chunk prep and chunk state (the fp32 path's header memset is not a
+    kernel of ours)."""
     from linear_attention_layer_gated_b200 import gdn
     import torch
     tensor = algo == gdn.GDN_ALGO_TENSOR or (algo == gdn.GDN_ALGO_AUTO and dtype == torch.bfloat16)
-    return 3 if tensor else 1
+    if not tensor:
+        return 1
+    return 2 if fused_prefill_applies(num_seqs, hv) else 3
 
 
 def main():
