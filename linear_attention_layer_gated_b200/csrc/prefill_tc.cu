@@ -71,6 +71,12 @@ constexpr uint32_t kKTBytes = 32768;
 constexpr uint32_t kFacOff = kKTOff + kKTBytes;       // 98304
 constexpr uint32_t kFacLoad = 16;                     // bytes of F the state kernel reads
 constexpr uint32_t kRecBytes = kFacOff + 1024;        // 99,328
+// The one-launch pass keeps the records of at most kRing chunks (a ring: 14 x 32 heads x 99 KB =
+// 44.5 MB at 32 V heads, which stays in L2, so the records rarely reach DRAM) instead of one
+// slot per chunk.  Its prep workers run about 14.5 chunks ahead of the state passes at B = 1
+// (232 workers, 16 items per chunk); a larger ring lets L2 evict records to DRAM before they
+// are overwritten, a smaller one stalls the workers.
+constexpr int kRing = 14;
 
 struct WsLayout {
     size_t seq_chunk0, table, flags, rec, total;
@@ -87,8 +93,9 @@ __host__ __device__ inline WsLayout ws_layout(int num_seqs, int total_tokens, in
     off = round_up(off + (size_t)(num_seqs + 1) * 4, 1024);
     L.table = off;
     off = round_up(off + (size_t)L.max_chunks * 16, 1024);
-    L.flags = off;  // per (chunk, pair of V heads): the fused pass's "records complete" flags
-    off = round_up(off + (size_t)L.max_chunks * (hv / 2 > 0 ? hv / 2 : 1) * 4, 1024);
+    L.flags = off;  // the one-launch pass: per (chunk, pair of V heads) "records complete" flags,
+                    // then per (ring slot, V head) the last chunk consumed + 1
+    off = round_up(off + ((size_t)L.max_chunks * (hv / 2 > 0 ? hv / 2 : 1) + (size_t)kRing * hv) * 4, 1024);
     L.rec = off;
     off += (size_t)L.max_chunks * hv * kRecBytes;
     L.total = round_up(off, 1024);
@@ -104,7 +111,7 @@ chunk_table_kernel(const int32_t* __restrict__ cu, int num_seqs, int total_token
     const WsLayout L = ws_layout(num_seqs, total_tokens, hv);
     {
         int32_t* flags = reinterpret_cast<int32_t*>(ws + L.flags);
-        const long long nflags = L.max_chunks * (hv / 2);
+        const long long nflags = L.max_chunks * (hv / 2) + (long long)kRing * hv;
         for (long long i = threadIdx.x; i < nflags; i += blockDim.x) flags[i] = 0;
     }
     int32_t* seq_chunk0 = reinterpret_cast<int32_t*>(ws + L.seq_chunk0);
@@ -252,6 +259,8 @@ struct PrepArgs {
     int num_seqs, total_tokens, hk, hv;
     GateAct act;
     int32_t* ready;  // per (chunk, pair of V heads): set once the item's records are complete, or nullptr
+    const int32_t* consumed;  // per (ring slot, V head): last chunk whose records a state pass has taken + 1
+    int ring;                 // records go to ring slot chunk % ring (0: to slot chunk, no ring)
 };
 
 // The barriers of a prep item's 256 threads, initialised once (thread 32 of the item).
@@ -260,6 +269,22 @@ __device__ __forceinline__ void prep_init_barriers(PrepSmall& ss) {
     mbar_init(&ss.bar_mma, 1);
     mbar_init(&ss.bar_drain, 1);
     fence_mbar_init();
+}
+
+// Bounded wait (one thread) until both V heads' state passes have taken chunk `need` - 1 from
+// a ring slot: marks[0] and marks[1] reach `need`.  Gives up (false) after the wait limit or as
+// soon as another CTA has recorded an error in the header.
+__device__ bool wait_consumed(const int32_t* marks, int need, int32_t* header) {
+    const uint64_t t0 = global_timer_ns();
+    while (ld_acquire_gpu(marks) < need || ld_acquire_gpu(marks + 1) < need) {
+        if (*reinterpret_cast<volatile int32_t*>(header) != 0) return false;
+        if (global_timer_ns() - t0 > kWaitLimitNs) {
+            atomicOr(header, 1);
+            return false;
+        }
+        __nanosleep(200);
+    }
+    return true;
 }
 
 // One prep item, the chunk cid for the V heads 2 pair and 2 pair + 1, by 256 threads (tid
@@ -281,6 +306,7 @@ __device__ bool prep_item(const PrepArgs& a, int cid, int pair, unsigned char* s
     unsigned char* ws = a.ws;
     const WsLayout L = ws_layout(a.num_seqs, a.total_tokens, hv);
     const int h0 = 2 * pair;             // the two V heads of this item
+    const size_t rslot = a.ring ? (size_t)(cid % a.ring) : (size_t)cid;  // the item's record slot
     const int jq = h0 / (hv / a.hk);     // their QK head
     const int lane = tid & 31, warp = tid >> 5;
     const int qw = warp & 3, hf = warp >> 2;  // TMEM lane quarter, column half
@@ -460,7 +486,14 @@ __device__ bool prep_item(const PrepArgs& a, int cid, int pair, unsigned char* s
         ss.fw[hh][i] = ss.b[hh][i] * ss.gam[hh][i] * ss.rk[i];
         ss.fk[hh][i] = ss.c[hh][i] * ss.rk[i];
     }
-    hbar(bid, 256);
+    // With a ring, the slot's previous chunk (cid - ring) must have been taken by the state
+    // passes of both heads before its records are overwritten.
+    ok = true;
+    if (a.ring && cid >= a.ring && tid == 0) {
+        ok = wait_consumed(a.consumed + rslot * hv + h0, cid - a.ring + 1, reinterpret_cast<int32_t*>(ws));
+        if (ok) fence_async_global();
+    }
+    if (hbar_or(bid, 256, !ok)) return false;
 
     // ---- 6. per head, 128 threads.
     //   (a) thread l takes row l & 63 of T (l < 64) or of P T (l >= 64) and writes Tensor Memory
@@ -473,7 +506,7 @@ __device__ bool prep_item(const PrepArgs& a, int cid, int pair, unsigned char* s
         const int hh = tid >> 7, l = tid & 127, rr = l & 63;
         const bool trow = l < 64;
         const int h = h0 + hh;
-        unsigned char* rec = ws + L.rec + ((size_t)cid * hv + h) * kRecBytes;
+        unsigned char* rec = ws + L.rec + (rslot * hv + h) * kRecBytes;
         const float* bb = ss.b[hh];
         const float* fw = ss.fw[hh];
         {
@@ -611,7 +644,7 @@ __device__ bool prep_item(const PrepArgs& a, int cid, int pair, unsigned char* s
         tc_fence_before();
         hbar(bid, 256);  // the product is read before the next head's MMA overwrites it
         if (tid == 32) {
-            bulk_s2g(ws + L.rec + ((size_t)cid * hv + h0 + hh) * kRecBytes, sm + kP_AT + hh * kWQBytes, kWQBytes);
+            bulk_s2g(ws + L.rec + (rslot * hv + h0 + hh) * kRecBytes, sm + kP_AT + hh * kWQBytes, kWQBytes);
             bulk_commit();
         }
     }
@@ -664,7 +697,7 @@ chunk_prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = ss.tmem_base;
-    const PrepArgs a{&tm_q, &tm_k, g, beta, ws, num_seqs, total_tokens, hk, hv, act, nullptr};
+    const PrepArgs a{&tm_q, &tm_k, g, beta, ws, num_seqs, total_tokens, hk, hv, act, nullptr, nullptr, 0};
     if (!prep_item(a, cid, blockIdx.x % npairs, sm, tmem, tid, 1, 0)) {
         if (tid == 0) atomicOr(header, 1);
         prep_drain(ss, tid, 0);
@@ -776,7 +809,8 @@ __device__ bool wait_flag(const int32_t* flag, volatile int* abort_flag, int32_t
 __device__ void state_body(const CUtensorMap* tm_v_p, const CUtensorMap* tm_out_p, const float* s0,
                            const int32_t* __restrict__ cu, __nv_bfloat16* __restrict__ out, float* sT,
                            StateSlots map, float* cstates, unsigned char* ws, int num_seqs, int total_tokens,
-                           int hv, int n, int h, unsigned char* sm, uint32_t tmem, const int32_t* ready) {
+                           int hv, int n, int h, unsigned char* sm, uint32_t tmem, const int32_t* ready,
+                           int32_t* consumed, int ring) {
     const uint32_t sb = smem_u32(sm);
     StateSmall& ss = *reinterpret_cast<StateSmall*>(sm + kS_SMALL);
     volatile int* abort_flag = &ss.abort_flag;
@@ -809,7 +843,10 @@ __device__ void state_body(const CUtensorMap* tm_v_p, const CUtensorMap* tm_out_
     const int32_t* seq_chunk0 = reinterpret_cast<const int32_t*>(ws + L.seq_chunk0);
     const int cs = seq_chunk0[n], nch = seq_chunk0[n + 1] - cs;
     const int t_begin = cu[n], t_end = cu[n + 1];
-    auto rec_of = [&](int c) { return ws + L.rec + ((size_t)(cs + c) * hv + h) * kRecBytes; };
+    auto rec_of = [&](int c) {
+        const size_t slot_c = ring ? (size_t)((cs + c) % ring) : (size_t)(cs + c);
+        return ws + L.rec + (slot_c * hv + h) * kRecBytes;
+    };
 
     if (warp == 0) {
         // ------------------------------------------------ loads, one slot ahead
@@ -933,6 +970,8 @@ __device__ void state_body(const CUtensorMap* tm_v_p, const CUtensorMap* tm_out_
         bool alive = true;
         for (int c = 0; c < nch && alive; ++c) {
             if (!(alive = wait_or_abort(&ss.full[c & 1], (c >> 1) & 1, abort_flag, header))) break;
+            if (consumed && warp == 2 && lane == 0)  // the chunk's records are in shared memory: its ring slot is free
+                st_release_gpu(consumed + (size_t)((cs + c) % ring) * hv + h, cs + c + 1);
             const float gl = ss.gl[c & 1][0];
             if (!(alive = wait_or_abort(&ss.msa, c & 1, abort_flag, header))) break;
             tc_fence_after();
@@ -1021,7 +1060,7 @@ chunk_state_kernel(const __grid_constant__ CUtensorMap tm_v, const __grid_consta
     tc_fence_after();
     const uint32_t tmem = ss.tmem_base;
     state_body(&tm_v, &tm_out, s0, cu, out, sT, map, cstates, ws, num_seqs, total_tokens, hv, blockIdx.x / hv,
-               blockIdx.x % hv, sm, tmem, nullptr);
+               blockIdx.x % hv, sm, tmem, nullptr, nullptr, 0);
     tc_fence_before();
     __syncthreads();
     if (threadIdx.x < 32) {
@@ -1057,6 +1096,8 @@ chunk_fused_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
     int32_t* header = reinterpret_cast<int32_t*>(ws);
     const WsLayout L = ws_layout(num_seqs, total_tokens, hv);
     int32_t* ready = reinterpret_cast<int32_t*>(ws + L.flags);
+    int32_t* consumed = ready + L.max_chunks * (hv / 2);
+    const int ring = L.max_chunks > kRing ? kRing : 0;
     const bool is_state = (int)blockIdx.x < nstate;
     if (warp == 0) {
         tmem_alloc(&tmem_s, 512);
@@ -1069,7 +1110,7 @@ chunk_fused_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
     const uint32_t tmem = tmem_s;
     if (is_state) {
         state_body(&tm_v, &tm_out, s0, cu, out, sT, map, cstates, ws, num_seqs, total_tokens, hv, blockIdx.x / hv,
-                   blockIdx.x % hv, sm, tmem, ready);
+                   blockIdx.x % hv, sm, tmem, ready, ring ? consumed : nullptr, ring);
     } else {
         const int half = tid >> 8, ltid = tid & 255;
         const uint32_t bid = 1 + half;
@@ -1079,7 +1120,7 @@ chunk_fused_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
         const long long items = (long long)header[1] * npairs;
         const long long worker = (long long)(blockIdx.x - nstate) * 2 + half;
         const long long nworkers = (long long)(gridDim.x - nstate) * 2;
-        const PrepArgs a{&tm_q, &tm_k, g, beta, ws, num_seqs, total_tokens, hk, hv, act, ready};
+        const PrepArgs a{&tm_q, &tm_k, g, beta, ws, num_seqs, total_tokens, hk, hv, act, ready, consumed, ring};
         uint32_t j = 0;
         for (long long it = worker; it < items; it += nworkers, ++j) {
             if (hbar_or(bid, 256, *reinterpret_cast<volatile int32_t*>(header) != 0)) break;  // another CTA gave up
