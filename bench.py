@@ -298,7 +298,7 @@ def main_ours(args, rank, world, local_rank):
                                       cu, outs[i], fin, workspace=ws, algo=algo, stream=stream)
         return run
 
-    tensor_path = gdn_launches_per_prefill(algo, torch.bfloat16) == 3
+    tensor_path = gdn_launches_per_prefill(algo, torch.bfloat16) > 1
 
     def measure_prefill(w, steps, warmup, with_initial, segments=1, phased=False, clocks=False):
         """Times one prefill workload; returns (record, x, out, fin, ws)."""
@@ -310,7 +310,7 @@ def main_ours(args, rank, world, local_rank):
             shape = gdn.prefill_shape(x["q"], x["v"], x["cu_seqlens"], algo)
         else:  # every call sees one sequence of T / segments tokens
             shape = gdn.make_shape(1, T // segments, HK, HV, D, gdn.GDN_BF16, algo)
-        ws = gdn.alloc_workspace(shape, dev)
+        ws = gdn.alloc_workspace(shape, dev, phases=phased)
         fn = prefill_step_fn(x, out, fin, ws, with_initial, segments)
         clk = ClockSampler(local_rank) if clocks else None
         if clk:

@@ -88,11 +88,24 @@ typedef struct {
 } gdn_shape;
 
 /*
- * Workspace the caller must provide to gdn_chunk_prefill for `shape` (bytes, a
- * multiple of 256).  It depends on total_tokens, num_seqs, the head counts and the
- * algorithm.  Returns 0 if the shape is invalid.
+ * Workspace the caller must provide to gdn_chunk_prefill (and its _slots, _chunk_states,
+ * _raw_gates variants) for `shape` (bytes, a multiple of 256).  It depends on
+ * total_tokens, num_seqs, the head counts, the algorithm and the current device: when the
+ * (sequence, V head) chains fill at most half of the device's SMs the tensor-core prefill
+ * runs both of its passes in one cooperative launch and keeps its per-chunk operands in
+ * a ring of a few chunks (about 46 MB at 32 V heads, whatever the length); otherwise the
+ * workspace holds the operands of every chunk (about 50 KB per token at 16/32 heads).
+ * Query it with the device current that will run the call: a call whose path needs more
+ * than it is given returns GDN_ERR_WORKSPACE.  Returns 0 if the shape is invalid.
  */
 size_t gdn_prefill_workspace_bytes(const gdn_shape *shape);
+
+/*
+ * Workspace of the two-phase entry points gdn_chunk_prefill_prep / gdn_chunk_prefill_state
+ * (the operands of every chunk; at least gdn_prefill_workspace_bytes).  Returns 0 if the
+ * shape is invalid or does not take the tensor-core path.
+ */
+size_t gdn_prefill_phase_workspace_bytes(const gdn_shape *shape);
 
 /*
  * Chunked prefill over a packed varlen batch.  The chunked form of the gated delta
@@ -299,8 +312,9 @@ gdn_status gdn_get_device_error(void *workspace, void *stream);
  * inside libgdn.so, which every GPU that loads the library holds until exit.
  *   - Calls no cudaMalloc, cudaFree or other allocating routine.
  *   - Workloads whose gdn_prefill_workspace_bytes(shape) exceeds the maximum are rejected
- *     with GDN_ERR_WORKSPACE (about 21 chunks of 64 tokens with 16 QK / 32 V heads, e.g.
- *     one sequence of up to 1,343 tokens); fp32 I/O or GDN_ALGO_SIMT give
+ *     with GDN_ERR_WORKSPACE.  With 16 QK / 32 V heads on a 148-SM device one or two
+ *     sequences of any length fit (their operands live in a ring of a few chunks); larger
+ *     batches fit up to about 21 chunks of 64 tokens in all.  fp32 I/O or GDN_ALGO_SIMT give
  *     GDN_ERR_UNSUPPORTED.
  *   - The first call on each device (with that device current) looks up the array's
  *     device address and caches it with the identity of the device's current context;

@@ -71,10 +71,20 @@ static bool use_tensor_path(const gdn_shape* s) {
 
 size_t gdn_prefill_workspace_bytes(const gdn_shape* shape) {
     if (check_prefill_shape(shape) != GDN_OK) return 0;
-    if (use_tensor_path(shape) && tensor_shape_ok(shape))
+    if (use_tensor_path(shape) && tensor_shape_ok(shape)) {
+        if (gdn::fused_prefill_applies(shape->num_seqs, shape->total_tokens, shape->num_v_heads))
+            return gdn::tc_fused_workspace_bytes(shape->num_seqs, shape->total_tokens, shape->num_qk_heads,
+                                                 shape->num_v_heads);
         return gdn::tc_workspace_bytes(shape->num_seqs, shape->total_tokens, shape->num_qk_heads,
                                        shape->num_v_heads);
+    }
     return kHeaderBytes;
+}
+
+size_t gdn_prefill_phase_workspace_bytes(const gdn_shape* shape) {
+    if (check_prefill_shape(shape) != GDN_OK) return 0;
+    if (!use_tensor_path(shape) || !tensor_shape_ok(shape)) return 0;
+    return gdn::tc_workspace_bytes(shape->num_seqs, shape->total_tokens, shape->num_qk_heads, shape->num_v_heads);
 }
 
 }  // extern "C"
@@ -215,7 +225,7 @@ static gdn_status check_phase(const gdn_shape* shape, const int32_t* cu_seqlens,
     gdn_status st = check_prefill_shape(shape);
     if (st != GDN_OK) return st;
     if (!use_tensor_path(shape) || !tensor_shape_ok(shape)) return GDN_ERR_UNSUPPORTED;
-    if (!workspace || workspace_bytes < gdn_prefill_workspace_bytes(shape)) return GDN_ERR_WORKSPACE;
+    if (!workspace || workspace_bytes < gdn_prefill_phase_workspace_bytes(shape)) return GDN_ERR_WORKSPACE;
     if ((reinterpret_cast<uintptr_t>(workspace) & 255u) != 0) return GDN_ERR_ALIGN;
     if (shape->num_seqs > 0 && !cu_seqlens) return GDN_ERR_NULL;
     if (cu_seqlens && !aligned16(cu_seqlens)) return GDN_ERR_ALIGN;

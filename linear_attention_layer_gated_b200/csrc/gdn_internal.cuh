@@ -102,6 +102,8 @@ cudaError_t launch_prefill_simt(const void* q, const void* k, const void* v, con
 // Tensor-core prefill (bf16 I/O, num_v_heads / num_qk_heads even): total workspace bytes
 // (header included) and launch.
 size_t tc_workspace_bytes(int num_seqs, int total_tokens, int hk, int hv);
+// The one-launch pass's smaller workspace: its records live in a ring of a few chunks.
+size_t tc_fused_workspace_bytes(int num_seqs, int total_tokens, int hk, int hv);
 // Phase 1 (chunk table + per-chunk coefficient images, from q, k and the gates) and phase 2
 // (state pass, from k, v and the images).
 cudaError_t launch_prefill_tc_prep(const void* q, const void* k, const float* g, const float* beta,

@@ -1198,6 +1198,13 @@ size_t tc_workspace_bytes(int num_seqs, int total_tokens, int hk, int hv) {
     return ws_layout(num_seqs, total_tokens, hv).total;
 }
 
+size_t tc_fused_workspace_bytes(int num_seqs, int total_tokens, int hk, int hv) {
+    (void)hk;
+    const WsLayout L = ws_layout(num_seqs, total_tokens, hv);
+    const long long slots = L.max_chunks > kRing ? kRing : L.max_chunks;  // the record ring
+    return round_up(L.rec + (size_t)slots * hv * kRecBytes, 1024);
+}
+
 cudaError_t launch_prefill_tc_prep(const void* q, const void* k, const float* g, const float* beta,
                                    const int32_t* cu, int num_seqs, int total_tokens, int hk, int hv,
                                    void* workspace, GateAct act, cudaStream_t stream) {

@@ -22,7 +22,8 @@ GDN_ALGO_AUTO, GDN_ALGO_SIMT, GDN_ALGO_TENSOR = 0, 1, 2
 STATUS = {0: "GDN_OK", 1: "GDN_ERR_NULL", 2: "GDN_ERR_SHAPE", 3: "GDN_ERR_ALIGN",
           4: "GDN_ERR_DTYPE", 5: "GDN_ERR_NUM_TOKENS", 6: "GDN_ERR_WORKSPACE",
           7: "GDN_ERR_CUDA", 8: "GDN_ERR_DEVICE_TIMEOUT", 9: "GDN_ERR_UNSUPPORTED"}
-EXPORTED = ["gdn_prefill_workspace_bytes", "gdn_chunk_prefill", "gdn_chunk_prefill_prep",
+EXPORTED = ["gdn_prefill_workspace_bytes", "gdn_prefill_phase_workspace_bytes", "gdn_chunk_prefill",
+            "gdn_chunk_prefill_prep",
             "gdn_chunk_prefill_state", "gdn_decode_step", "gdn_get_device_error",
             "gdn_selftest_wait_timeout", "gdn_status_string", "gdn_abi_version",
             "gdn_chunk_prefill_noalloc", "gdn_decode_verify", "gdn_decode_commit",
@@ -62,6 +63,8 @@ def lib() -> ctypes.CDLL:
             sp = ctypes.POINTER(GdnShape)
             L.gdn_prefill_workspace_bytes.restype = ctypes.c_size_t
             L.gdn_prefill_workspace_bytes.argtypes = [sp]
+            L.gdn_prefill_phase_workspace_bytes.restype = ctypes.c_size_t
+            L.gdn_prefill_phase_workspace_bytes.argtypes = [sp]
             L.gdn_chunk_prefill.restype = ctypes.c_int
             L.gdn_chunk_prefill.argtypes = [vp, vp, vp, fp, fp, fp, ip, vp, fp, sp, vp,
                                             ctypes.c_size_t, vp]
@@ -160,15 +163,23 @@ def gdn_prefill_workspace_bytes(shape: GdnShape) -> int:
     return int(lib().gdn_prefill_workspace_bytes(ctypes.byref(shape)))
 
 
+def gdn_prefill_phase_workspace_bytes(shape: GdnShape) -> int:
+    return int(lib().gdn_prefill_phase_workspace_bytes(ctypes.byref(shape)))
+
+
 def prefill_shape(q, v, cu_seqlens, algo=GDN_ALGO_AUTO, max_seqlen=0) -> GdnShape:
     T, HK, D = q.shape
     return make_shape(cu_seqlens.numel() - 1, T, HK, v.shape[1], D, _io_dtype(q), algo, max_seqlen)
 
 
-def alloc_workspace(shape: GdnShape, device) -> torch.Tensor:
+def alloc_workspace(shape: GdnShape, device, phases=False) -> torch.Tensor:
+    """A workspace for gdn_chunk_prefill on `shape` (with phases=True, large enough for the
+    two-phase entry points gdn_chunk_prefill_prep / _state as well)."""
     n = gdn_prefill_workspace_bytes(shape)
     if n == 0:
         raise ValueError("invalid prefill shape")
+    if phases:
+        n = max(n, gdn_prefill_phase_workspace_bytes(shape))
     return torch.empty(n, dtype=torch.uint8, device=device)
 
 

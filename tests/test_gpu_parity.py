@@ -319,6 +319,30 @@ def test_prefill_paired_heads_identical(algo):
     torch.testing.assert_close(fin[:, 1], fin[:, 0], rtol=0, atol=0)
 
 
+@pytest.mark.parametrize("lens", [[700], [130, 1, 300]])
+def test_split_entry_points_match_one_call_and_oracle(lens):
+    """gdn_chunk_prefill_prep + gdn_chunk_prefill_state (two launches, a workspace slot per
+    chunk) against one gdn_chunk_prefill call (here the one-launch pass with its record ring):
+    the same operations, so the same bits; and both against the oracle."""
+    x = inputs.make_prefill(lens, hk=4, hv=8, state_std=0.02, seed=60, device="cuda")
+    N = len(lens)
+    shape = gdn.prefill_shape(x["q"], x["v"], x["cu_seqlens"])
+    assert gdn.gdn_prefill_phase_workspace_bytes(shape) >= gdn.gdn_prefill_workspace_bytes(shape)
+    ws = gdn.alloc_workspace(shape, "cuda", phases=True)
+    out_p = torch.full_like(x["v"], float("nan"))
+    fin_p = torch.full((N, 8, 128, 128), float("nan"), device="cuda")
+    gdn.gdn_chunk_prefill_prep(x["q"], x["k"], x["g"], x["beta"], x["cu_seqlens"], ws, x["v"])
+    gdn.gdn_chunk_prefill_state(x["k"], x["v"], x["initial_state"], x["cu_seqlens"], out_p, fin_p, ws)
+    out_1, fin_1 = gdn.prefill(x["q"], x["k"], x["v"], x["g"], x["beta"], x["cu_seqlens"], x["initial_state"])
+    torch.cuda.synchronize()
+    assert gdn.STATUS[gdn.gdn_get_device_error(ws)] == "GDN_OK"
+    torch.testing.assert_close(out_p, out_1, rtol=0, atol=0)
+    torch.testing.assert_close(fin_p, fin_1, rtol=0, atol=0)
+    o_ref, s_ref = oracle.forward(x["q"], x["k"], x["v"], x["g"], x["beta"], x["cu_seqlens"], x["initial_state"])
+    assert_close(out_p, o_ref, TOL_BF16, "split prefill out")
+    assert_close(fin_p, s_ref, TOL_BF16, "split prefill state")
+
+
 def test_device_error_word_is_clear_after_prefill():
     x = inputs.make_prefill([100], hk=2, hv=4, seed=25, device="cuda")
     ws = gdn.alloc_workspace(gdn.prefill_shape(x["q"], x["v"], x["cu_seqlens"]), "cuda")

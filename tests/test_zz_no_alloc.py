@@ -56,9 +56,27 @@ def test_noalloc_prefill_matches_workspace_prefill_twice_in_a_row():
         assert rel_l2(fin, ref_fin) <= TOL_BF16
 
 
+def test_noalloc_prefill_takes_one_long_sequence():
+    """One sequence runs in the one-launch pass, whose operands live in a ring of a few
+    chunks: the static scratch holds a sequence of any length."""
+    L = gdn.lib()
+    x = inputs.make_prefill([20000], state_std=0.02, seed=33, device="cuda")
+    shape = gdn.prefill_shape(x["q"], x["v"], x["cu_seqlens"])
+    assert L.gdn_prefill_workspace_bytes(ctypes.byref(shape)) <= (64 << 20)
+    out = torch.full_like(x["v"], float("nan"))
+    fin = torch.full_like(x["initial_state"], float("nan"))
+    assert run_noalloc(L, x, out, fin) == gdn.GDN_OK
+    assert gdn.STATUS[L.gdn_get_noalloc_device_error(stream_handle())] == "GDN_OK"
+    ref_out, ref_fin = gdn.prefill(x["q"], x["k"], x["v"], x["g"], x["beta"], x["cu_seqlens"], x["initial_state"])
+    torch.cuda.synchronize()
+    assert rel_l2(out, ref_out) <= 1e-5 and rel_l2(fin, ref_fin) <= 1e-5  # the same pass, the same scratch layout
+
+
 def test_noalloc_prefill_rejects_workloads_beyond_its_scratch():
     L = gdn.lib()
-    shape = gdn.make_shape(1, 1 << 16, 16, 32)   # 65,536 tokens need far more than 64 MiB
+    # 8 sequences of 8,192 tokens: too many chains for the one-launch pass, and the operands of
+    # every chunk need far more than 64 MiB
+    shape = gdn.make_shape(8, 1 << 16, 16, 32)
     assert L.gdn_prefill_workspace_bytes(ctypes.byref(shape)) > (64 << 20)
     rc = L.gdn_chunk_prefill_noalloc(None, None, None, None, None, None, None, None, None,
                                      ctypes.byref(shape), None)
