@@ -354,10 +354,11 @@ gdn_status gdn_get_noalloc_device_error(void *stream);
 gdn_status gdn_get_decode_device_error(void *stream);
 
 /*
- * Failure-path self-test.  Clears the workspace header, then launches a kernel that waits
- * on a barrier nothing completes, using the same bounded wait as the prefill kernels
- * but with a limit of `limit_us` microseconds (1 .. 2,000,000).  When the limit expires
- * the kernel records the timeout in the header and returns normally; a following
+ * Failure-path self-test.  Clears the workspace header, then launches a kernel that runs
+ * each kind of bounded wait the kernels use -- on a flag another CTA would raise, on a pair
+ * of marks, and on an mbarrier phase -- against something nothing completes, with a limit
+ * of `limit_us` microseconds each (1 .. 2,000,000).  When the limits expire the kernel
+ * records the timeout in the header and returns normally; a following
  * gdn_get_device_error(workspace, stream) then returns GDN_ERR_DEVICE_TIMEOUT and the
  * CUDA context remains usable.  `workspace` needs >= 256 bytes, 256-byte aligned.
  */

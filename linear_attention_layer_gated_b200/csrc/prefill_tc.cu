@@ -272,19 +272,12 @@ __device__ __forceinline__ void prep_init_barriers(PrepSmall& ss) {
 }
 
 // Bounded wait (one thread) until both V heads' state passes have taken chunk `need` - 1 from
-// a ring slot: marks[0] and marks[1] reach `need`.  Gives up (false) after the wait limit or as
-// soon as another CTA has recorded an error in the header.
+// a ring slot: marks[0] and marks[1] reach `need`.  Gives up (false, recording the error) after
+// the wait limit, or at once when another CTA has recorded an error in the header.
 __device__ bool wait_consumed(const int32_t* marks, int need, int32_t* header) {
-    const uint64_t t0 = global_timer_ns();
-    while (ld_acquire_gpu(marks) < need || ld_acquire_gpu(marks + 1) < need) {
-        if (*reinterpret_cast<volatile int32_t*>(header) != 0) return false;
-        if (global_timer_ns() - t0 > kWaitLimitNs) {
-            atomicOr(header, 1);
-            return false;
-        }
-        __nanosleep(200);
-    }
-    return true;
+    if (wait_marks_reach(marks, need, header, kWaitLimitNs)) return true;
+    atomicOr(header, 1);
+    return false;
 }
 
 // One prep item, the chunk cid for the V heads 2 pair and 2 pair + 1, by 256 threads (tid
@@ -776,29 +769,13 @@ __device__ __forceinline__ bool wait_or_abort(uint64_t* bar, uint32_t parity, vo
 }
 
 // Bounded wait (one thread) for a flag another CTA of the same launch raises; returns false
-// if it gave up or another thread or CTA has recorded an error.
+// (and raises the CTA's abort flag, recording the error) if it gave up, or at once if another
+// CTA has recorded an error.
 __device__ bool wait_flag(const int32_t* flag, volatile int* abort_flag, int32_t* header) {
-    if (ld_acquire_gpu(flag) != 0) {
-        fence_async_global();
-        return true;
-    }
-    const uint64_t t0 = global_timer_ns();
-    while (true) {
-        __nanosleep(200);
-        if (ld_acquire_gpu(flag) != 0) {
-            fence_async_global();  // the bulk copies that follow read what the flag released
-            return true;
-        }
-        if (*abort_flag || *reinterpret_cast<volatile int32_t*>(header) != 0) {
-            *abort_flag = 1;
-            return false;
-        }
-        if (global_timer_ns() - t0 > kWaitLimitNs) {
-            *abort_flag = 1;
-            atomicOr(header, 1);
-            return false;
-        }
-    }
+    if (wait_flag_set(flag, header, kWaitLimitNs)) return true;
+    *abort_flag = 1;
+    atomicOr(header, 1);
+    return false;
 }
 
 // The state pass of sequence n, V head h, by the CTA's threads 0..447 (any further threads of

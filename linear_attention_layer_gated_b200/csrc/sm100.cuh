@@ -95,6 +95,31 @@ __device__ __forceinline__ int32_t ld_acquire_gpu(const int32_t* p) {
     return v;
 }
 
+// Bounded waits (one thread) on values that another CTA of the same launch writes.  Each gives
+// up (false) after limit_ns, or as soon as *stop (if given) is non-zero: another thread or CTA
+// has given up already.  On success the thread's later bulk copies are ordered after what the
+// writer released.
+__device__ __forceinline__ bool wait_flag_set(const int32_t* flag, const volatile int32_t* stop, uint64_t limit_ns) {
+    const uint64_t t0 = global_timer_ns();
+    while (ld_acquire_gpu(flag) == 0) {
+        if ((stop && *stop != 0) || global_timer_ns() - t0 > limit_ns) return false;
+        __nanosleep(200);
+    }
+    fence_async_global();
+    return true;
+}
+// Until marks[0] and marks[1] both reach `need`.
+__device__ __forceinline__ bool wait_marks_reach(const int32_t* marks, int32_t need, const volatile int32_t* stop,
+                                                 uint64_t limit_ns) {
+    const uint64_t t0 = global_timer_ns();
+    while (ld_acquire_gpu(marks) < need || ld_acquire_gpu(marks + 1) < need) {
+        if ((stop && *stop != 0) || global_timer_ns() - t0 > limit_ns) return false;
+        __nanosleep(200);
+    }
+    fence_async_global();
+    return true;
+}
+
 // ------------------------------------------------------------------ named barriers
 // A barrier among `count` threads (a multiple of 32) of the CTA, numbered id (1..15; 0 is
 // __syncthreads); hbar_or also returns whether any of them passed a non-zero x.

@@ -443,11 +443,17 @@ def test_long_context_split_carry_and_sampled_heads(algo):
 
 
 def test_bounded_wait_expiry_is_reported_and_context_survives():
-    """A device wait that nothing completes gives up after its limit, records the
-    timeout in the workspace header and returns; the next calls still work."""
+    """Device waits that nothing completes (an inter-CTA flag, a pair of ring marks and an
+    mbarrier phase) give up after their limit, record the timeout in the workspace header
+    and return; the next calls still work."""
     ws = torch.zeros(256, dtype=torch.uint8, device="cuda")
+    a = torch.cuda.Event(enable_timing=True)
+    b = torch.cuda.Event(enable_timing=True)
+    a.record()
     gdn.gdn_selftest_wait_timeout(ws, limit_us=20000)
+    b.record()
     assert gdn.STATUS[gdn.gdn_get_device_error(ws)] == "GDN_ERR_DEVICE_TIMEOUT"
+    assert a.elapsed_time(b) >= 3 * 20.0 * 0.9  # each of the three waits ran to its 20 ms limit
     x = inputs.make_prefill([80], hk=2, hv=4, seed=28, device="cuda")
     ws2 = gdn.alloc_workspace(gdn.prefill_shape(x["q"], x["v"], x["cu_seqlens"]), "cuda")
     out, fin = gdn.prefill(x["q"], x["k"], x["v"], x["g"], x["beta"], x["cu_seqlens"], workspace=ws2)
