@@ -81,12 +81,6 @@ __device__ __forceinline__ void cp_async16(void* dst_smem, const void* src) {
                  "l"(src)
                  : "memory");
 }
-__device__ __forceinline__ void cp_async4(void* dst_smem, const void* src) {
-    asm volatile("cp.async.ca.shared.global [%0], [%1], 4;" ::"r"(
-                     static_cast<uint32_t>(__cvta_generic_to_shared(dst_smem))),
-                 "l"(src)
-                 : "memory");
-}
 __device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
 template <int N>
 __device__ __forceinline__ void cp_async_wait() { asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory"); }
@@ -309,30 +303,32 @@ decode_kernel(const IO* __restrict__ q, const IO* __restrict__ k, const IO* __re
 // in as two terms, x = hi + lo with hi = x rounded to tf32 and lo = x - hi (together about 21
 // bits); bf16 values (q, k, v) are exact in tf32 and need no split.
 //
-// One CTA per SM (8 warps) streams (sequence, V head) items through three shared-memory slots:
-// the state (four 2-D tensor copies of 128 rows x 32 columns with the 128-byte swizzle) and the
-// q, k, v rows (bulk copies) of item i+2 are in flight while item i is computed; one barrier per
-// item.  Warp w owns 16 state rows of the item: MMA rows g = 0..7 are state rows 16w + 2g and
-// MMA rows g + 8 are 16w + 2g + 1, which with the swizzle makes every fragment load free of
+// One CTA of 4 warps per (sequence, V head), three CTAs per SM, so that the copies of one CTA
+// overlap the arithmetic of the others.  At entry one thread issues the whole head's state as
+// eight 2-D tensor copies (64 rows x 32 columns, 128-byte swizzle) and the item's q, k, v rows
+// as bulk copies; rows 0..63 and the vectors complete one barrier, rows 64..127 a second, so
+// that each warp starts on its first 16-row tile (rows 16 w ..) while its second (rows 16 (w +
+// 4) ..) is still arriving.  Within a tile, MMA rows g = 0..7 are state rows 16 tile + 2 g and
+// MMA rows g + 8 are 16 tile + 2 g + 1, which with the swizzle makes every fragment load free of
 // bank conflicts.  The columns are permuted the same way in both products: in k-step / n-tile
 // p, slot t of the MMA is column 8p + 2t and slot t + 4 is column 8p + 2t + 1, so the A
 // fragments of S for the first product are exactly the accumulator fragments of S for the
-// second, and each thread loads its 64 state values once.  The new rows go straight to HBM
-// (each 8-byte store completes a 32-byte sector with its three neighbours).
-constexpr int kMmaWarps = 8;
+// second.  The new rows go straight to HBM (each 8-byte store completes a 32-byte sector with
+// its three neighbours).
+constexpr int kCtaWarps = 4;
 constexpr int kVecStride = 272;  // bytes between staged q / k / v rows (bank-conflict padding)
+constexpr int kHalfRows = kD / 2;
 
 template <int NTOK>
 struct MmaLayout {
-    static constexpr int kStateBytes = kD * kD * 4;
+    static constexpr int kStateBytes = kD * kD * 4;                     // 4 column boxes of 128 rows
+    static constexpr int kHalfBytes = kStateBytes / 2;
     static constexpr int kVec = kStateBytes;                            // rows k_0.., q_0.., v_0..
-    static constexpr int kTx = kStateBytes + 3 * NTOK * kD * 2;
-    static constexpr int kGate = kVec + 3 * NTOK * kVecStride;         // g_t, beta_t, a_h, b_h; then the slot index
-    static constexpr int kSidx = kGate + 16 * 4;
-    static constexpr int kSlot = (kSidx + 16 + 1023) / 1024 * 1024;
-    static constexpr int kDots = 3 * kSlot;                             // per warp [8][8] floats
-    static constexpr int kBar = kDots + kMmaWarps * 64 * 4;             // full[3], abort flag
-    static constexpr int kSmem = kBar + 32 + 1024;                      // + alignment of the base
+    static constexpr int kTx0 = kHalfBytes + 3 * NTOK * kD * 2;         // rows 0..63 and the vectors
+    static constexpr int kGate = kVec + 3 * NTOK * kVecStride;          // g_t, beta_t, a_h, b_h
+    static constexpr int kDots = (kGate + 16 * 4 + 15) / 16 * 16;       // per warp [8][8] floats
+    static constexpr int kBar = kDots + kCtaWarps * 64 * 4;             // two barriers
+    static constexpr int kSmem = kBar + 16 + 1024;                      // + alignment of the base
 };
 
 __device__ __forceinline__ uint32_t tf32_hi(float x) {
@@ -350,244 +346,183 @@ __device__ __forceinline__ void mma_tf32(float* d, uint32_t a0, uint32_t a1, uin
 }
 
 template <int NTOK>
-__global__ void __launch_bounds__(kMmaWarps * 32, 1)
+__global__ void __launch_bounds__(kCtaWarps * 32, 3)
 decode_mma_kernel(const __grid_constant__ CUtensorMap tm_state, const __nv_bfloat16* __restrict__ q,
                   const __nv_bfloat16* __restrict__ k, const __nv_bfloat16* __restrict__ v,
                   const float* __restrict__ g, const float* __restrict__ beta, float* __restrict__ state,
-                  StateSlots map, __nv_bfloat16* __restrict__ out, int num_seqs, int hk, int hv, GateAct act) {
+                  StateSlots map, __nv_bfloat16* __restrict__ out, int hk, int hv, GateAct act) {
     using namespace sm100;
     using Lay = MmaLayout<NTOK>;
-    constexpr int NV = 2 * NTOK;  // vectors k_0.., q_0.. (n = 0 .. NV-1 of the first product)
+    constexpr int NV = 2 * NTOK;
     constexpr int NG = 2 * NTOK + 2;
     extern __shared__ unsigned char smem_raw[];
-    unsigned char* smem =
+    unsigned char* sl =
         reinterpret_cast<unsigned char*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-    const int gq = lane >> 2, tq = lane & 3;  // MMA group and thread in group
-    float* dots = reinterpret_cast<float*>(smem + Lay::kDots) + warp * 64;
-    uint64_t* full = reinterpret_cast<uint64_t*>(smem + Lay::kBar);
-    volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + Lay::kBar + 24);
-    const int items = num_seqs * hv;
-    const int first = blockIdx.x, stride = gridDim.x;
+    const int gq = lane >> 2, tq = lane & 3;
+    float* dots = reinterpret_cast<float*>(sl + Lay::kDots) + warp * 64;
+    uint64_t* full = reinterpret_cast<uint64_t*>(sl + Lay::kBar);  // [0] rows 0..63 + vectors, [1] rows 64..127
+    const int n = blockIdx.x / hv, h = blockIdx.x % hv, qh = h / (hv / hk);
+    bool has;
+    const int sidx = state_index(map, n, has);
+    if (!has) return;  // a sequence without a state slot is skipped (whole CTA)
     if (tid == 0) {
-#pragma unroll
-        for (int s = 0; s < 3; ++s) mbar_init(&full[s], 1);
-        *abort_flag = 0;
+        mbar_init(full, 1);
+        mbar_init(full + 1, 1);
         fence_mbar_init();
     }
     __syncthreads();
-
-    // Thread 0: the state slot of an item (-1: none).  With a slot table this is a load, which
-    // thread 0 issues one item before it needs the value.
-    auto slot_of = [&](int item) -> int {
-        if (item >= items) return -1;
-        bool has;
-        const int sidx = state_index(map, item / hv, has);
-        return has ? sidx : -1;
-    };
-    // Thread 0: the copies of an item into slot s, completing on full[s] (a plain arrival for
-    // an item without a state, so that every item moves its slot's phase on by one).
-    auto issue = [&](int item, int s, int sidx) {
-        const int n = item / hv, h = item % hv, qh = h / (hv / hk);
-        unsigned char* sl = smem + s * Lay::kSlot;
-        *reinterpret_cast<int*>(sl + Lay::kSidx) = sidx;
-        if (sidx < 0) {
-            mbar_arrive(&full[s]);
-            return;
-        }
-        fence_async_smem();  // the CTA's earlier reads of this slot come first
-        mbar_arrive_expect_tx(&full[s], Lay::kTx);
+    if (tid == 0) {
+        mbar_arrive_expect_tx(full, Lay::kTx0);
+        mbar_arrive_expect_tx(full + 1, Lay::kHalfBytes);
         const int row0 = (sidx * hv + h) * kD;
+        // box (column block cb, half hf) lands at cb * 16 KiB + hf * 8 KiB: the same bytes as
+        // one 128-row box, so the swizzled addressing below does not depend on the split
 #pragma unroll
-        for (int cb = 0; cb < 4; ++cb) tma_load_2d(sl + cb * 16384, &tm_state, cb * 32, row0, &full[s]);
+        for (int cb = 0; cb < 4; ++cb) tma_load_2d(sl + cb * 16384, &tm_state, cb * 32, row0, full);
 #pragma unroll
         for (int t = 0; t < NTOK; ++t) {
             const size_t tok = (size_t)n * NTOK + t;
-            bulk_g2s(sl + Lay::kVec + t * kVecStride, k + (tok * hk + qh) * kD, kD * 2, &full[s]);
-            bulk_g2s(sl + Lay::kVec + (NTOK + t) * kVecStride, q + (tok * hk + qh) * kD, kD * 2, &full[s]);
-            bulk_g2s(sl + Lay::kVec + (2 * NTOK + t) * kVecStride, v + (tok * hv + h) * kD, kD * 2, &full[s]);
+            bulk_g2s(sl + Lay::kVec + t * kVecStride, k + (tok * hk + qh) * kD, kD * 2, full);
+            bulk_g2s(sl + Lay::kVec + (NTOK + t) * kVecStride, q + (tok * hk + qh) * kD, kD * 2, full);
+            bulk_g2s(sl + Lay::kVec + (2 * NTOK + t) * kVecStride, v + (tok * hv + h) * kD, kD * 2, full);
         }
-    };
-    // Threads 0 .. NG-1: gate value number `tid` of an item into slot s by cp.async (raw or
-    // activated as given); one cp.async group per item and thread, empty past the end.
-    auto issue_gates = [&](int item, int s) {
-        if (item < items && tid < NG) {
-            const int n = item / hv, h = item % hv, t = tid % NTOK;
-            const float* src = tid < NTOK       ? g + ((size_t)n * NTOK + t) * hv + h
-                               : tid < 2 * NTOK ? beta + ((size_t)n * NTOK + t) * hv + h
-                               : act.a          ? (tid == 2 * NTOK ? act.a + h : act.b + h)
-                                                : nullptr;
-            if (src) cp_async4(smem + s * Lay::kSlot + Lay::kGate + tid * 4, src);
-        }
-        cp_async_commit();
-    };
+#pragma unroll
+        for (int cb = 0; cb < 4; ++cb)
+            tma_load_2d(sl + cb * 16384 + kHalfRows * 128, &tm_state, cb * 32, row0 + kHalfRows, full + 1);
+    }
+    if (tid >= 32 && tid < 32 + NG) {  // the gates, by plain loads while the copies fly
+        const int e = tid - 32, t = e % NTOK;
+        float val = 0.f;
+        if (e < NTOK) val = g[((size_t)n * NTOK + t) * hv + h];
+        else if (e < 2 * NTOK) val = beta[((size_t)n * NTOK + t) * hv + h];
+        else if (act.a) val = (e == 2 * NTOK ? act.a : act.b)[h];
+        reinterpret_cast<float*>(sl + Lay::kGate)[e] = val;
+    }
+    __syncthreads();  // the barriers are armed and the gates stored; no block barrier follows
+    // Each warp waits (bounded) for what it reads; a warp whose wait gives up records the error
+    // and leaves.  Nothing after this point synchronises the whole CTA.
+    if (!mbar_wait(full, 0)) {
+        if (lane == 0) atomicOr(&g_decode_error, 1u);
+        return;
+    }
+    const unsigned char* vec = sl + Lay::kVec;
 
-    int sidx_ahead = -1;  // thread 0: the state slot of the next item to copy
-    if (tid == 0) {
-        if (first < items) issue(first, 0, slot_of(first));
-        if (first + stride < items) issue(first + stride, 1, slot_of(first + stride));
-        sidx_ahead = slot_of(first + 2 * stride);
-    }
-    if (warp == 0) {
-        issue_gates(first, 0);
-        issue_gates(first + stride, 1);
-    }
-    const int rowA = 16 * warp + 2 * gq, rowB = rowA + 1;  // state rows of MMA rows gq and gq + 8
-    int i = 0;
-    for (;; ++i) {
-        const int item = first + i * stride;
-        if (item >= items) break;
-        const int slot = i % 3;
-        const uint32_t parity = (i / 3) & 1;
-        if (warp == 0) cp_async_wait<1>();  // this thread's gates of item i (item i+1's may be in flight)
-        if (tid == 0 && !mbar_wait(&full[slot], parity)) {
-            *abort_flag = 1;
-            atomicOr(&g_decode_error, 1u);
+    // ---- this thread's vector n = gq at columns 8p + 2t, 8p + 2t + 1 and key t at 8p + gq
+    uint32_t vb0[16], vb1[16];
+    float kb[16];
+#pragma unroll
+    for (int p = 0; p < 16; ++p) {
+        if (gq < NV) {
+            const uint32_t w = *reinterpret_cast<const uint32_t*>(vec + gq * kVecStride + (8 * p + 2 * tq) * 2);
+            vb0[p] = w << 16;
+            vb1[p] = w & 0xffff0000u;
+        } else {
+            vb0[p] = 0u;
+            vb1[p] = 0u;
         }
-        __syncthreads();  // item i has landed; every warp is done with item i-1's slot
-        if (*abort_flag) break;
-        mbar_try_wait(&full[slot], parity);  // completed: makes the copies' data visible here too
-        if (tid == 0 && item + 2 * stride < items) {
-            issue(item + 2 * stride, (i + 2) % 3, sidx_ahead);
-            sidx_ahead = slot_of(item + 3 * stride);
+        kb[p] = tq < NTOK ? to_f32(reinterpret_cast<const __nv_bfloat16*>(vec + tq * kVecStride)[8 * p + gq]) : 0.f;
+    }
+    {   // products among the vectors
+        float dv[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+        for (int p = 0; p < 16; ++p) mma_tf32(dv, vb0[p], 0u, vb1[p], 0u, vb0[p], vb1[p]);
+        dots[gq * 8 + 2 * tq] = dv[0];
+        dots[gq * 8 + 2 * tq + 1] = dv[1];
+    }
+    __syncwarp();
+    float bt[NTOK], Gm[NTOK], rk[NTOK], rq[NTOK], Et[NTOK][NTOK];
+    {
+        const float* gs = reinterpret_cast<const float*>(sl + Lay::kGate);
+        const float ga = gs[2 * NTOK], gb = gs[2 * NTOK + 1];
+        float G[NTOK], acc = 0.f;
+#pragma unroll
+        for (int t = 0; t < NTOK; ++t) {
+            acc += act.a ? act_g(gs[t], ga, gb) : gs[t];
+            G[t] = acc;
+            bt[t] = act.a ? act_beta(gs[NTOK + t]) : gs[NTOK + t];
+            Gm[t] = expf(G[t]);
+            rk[t] = rsqrtf(dots[t * 8 + t] + kNormEps);
+            rq[t] = rsqrtf(dots[(NTOK + t) * 8 + NTOK + t] + kNormEps) * kInvSqrtD;
         }
-        if (warp == 0) issue_gates(item + 2 * stride, (i + 2) % 3);
-        const int n = item / hv, h = item % hv;
-        const unsigned char* sl = smem + slot * Lay::kSlot;
-        const int sidx = *reinterpret_cast<const int*>(sl + Lay::kSidx);
-        if (sidx >= 0) {
-            const unsigned char* vec = sl + Lay::kVec;
-            // ---- fragments: this thread's 64 state values, its vector n = gq (k_gq or q_{gq-m},
-            //      zero past 2m) at columns 8p + 2t, 8p + 2t + 1, and key t at columns 8p + gq
-            float2 sa[16], sb[16];
-            uint32_t vb0[16], vb1[16];
-            float kb[16];
 #pragma unroll
-            for (int p = 0; p < 16; ++p) {
-                const int box = (p >> 2) * 16384;
-                const int chunk = 2 * (p & 3) + (tq >> 1);
-                sa[p] = *reinterpret_cast<const float2*>(sl + box + rowA * 128 + ((chunk ^ (rowA & 7)) << 4) +
-                                                         8 * (tq & 1));
-                sb[p] = *reinterpret_cast<const float2*>(sl + box + rowB * 128 + ((chunk ^ (rowB & 7)) << 4) +
-                                                         8 * (tq & 1));
-                if (gq < NV) {
-                    const uint32_t w = *reinterpret_cast<const uint32_t*>(vec + gq * kVecStride + (8 * p + 2 * tq) * 2);
-                    vb0[p] = w << 16;            // bf16 -> fp32 (exact, and exact in tf32)
-                    vb1[p] = w & 0xffff0000u;
-                } else {
-                    vb0[p] = 0u;
-                    vb1[p] = 0u;
-                }
-                kb[p] = tq < NTOK ? to_f32(reinterpret_cast<const __nv_bfloat16*>(vec + tq * kVecStride)[8 * p + gq])
-                                  : 0.f;
+        for (int t = 0; t < NTOK; ++t)
+#pragma unroll
+            for (int j = 0; j <= t; ++j) Et[t][j] = (j == t) ? 1.f : expf(G[t] - G[j]);
+    }
+    const __nv_bfloat16* vrow = reinterpret_cast<const __nv_bfloat16*>(vec + 2 * NTOK * kVecStride);
+    const float gl = Gm[NTOK - 1];
+#pragma unroll 1
+    for (int tt = 0; tt < 2; ++tt) {
+        if (tt == 1 && !mbar_wait(full + 1, 0)) {
+            if (lane == 0) atomicOr(&g_decode_error, 1u);
+            return;
+        }
+        const int tile = warp + kCtaWarps * tt;
+        const int rowA = 16 * tile + 2 * gq, rowB = rowA + 1;
+        // the rows' fragments are read from shared memory twice (here and in the update), which
+        // keeps them out of registers across the recurrence
+        auto frag = [&](int p, int row) {
+            const int chunk = 2 * (p & 3) + (tq >> 1);
+            return *reinterpret_cast<const float2*>(sl + (p >> 2) * 16384 + row * 128 +
+                                                    ((chunk ^ (row & 7)) << 4) + 8 * (tq & 1));
+        };
+        float d[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+        for (int p = 0; p < 16; ++p) {
+            const float2 sa = frag(p, rowA), sb = frag(p, rowB);
+            const uint32_t a0 = tf32_hi(sa.x), a1 = tf32_hi(sb.x);
+            const uint32_t a2 = tf32_hi(sa.y), a3 = tf32_hi(sb.y);
+            mma_tf32(d, a0, a1, a2, a3, vb0[p], vb1[p]);
+            mma_tf32(d, __float_as_uint(sa.x - __uint_as_float(a0)), __float_as_uint(sb.x - __uint_as_float(a1)),
+                     __float_as_uint(sa.y - __uint_as_float(a2)), __float_as_uint(sb.y - __uint_as_float(a3)),
+                     vb0[p], vb1[p]);
+        }
+        float xa[8], xb[8];
+#pragma unroll
+        for (int src = 0; src < 4; ++src) {
+            const int from = (lane & ~3) | src;
+            xa[2 * src] = __shfl_sync(0xffffffffu, d[0], from);
+            xa[2 * src + 1] = __shfl_sync(0xffffffffu, d[1], from);
+            xb[2 * src] = __shfl_sync(0xffffffffu, d[2], from);
+            xb[2 * src + 1] = __shfl_sync(0xffffffffu, d[3], from);
+        }
+        float wa = 0.f, wb = 0.f;
+#pragma unroll
+        for (int rr = 0; rr < 2; ++rr) {
+            const float* xr = rr ? xb : xa;
+            const int row = rr ? rowB : rowA;
+            float delta[NTOK];
+#pragma unroll
+            for (int t = 0; t < NTOK; ++t) {
+                float x = Gm[t] * (rk[t] * xr[t]);
+#pragma unroll
+                for (int j = 0; j < t; ++j) x = fmaf(Et[t][j] * dots[j * 8 + t] * rk[j] * rk[t], delta[j], x);
+                delta[t] = bt[t] * (to_f32(vrow[t * (kVecStride / 2) + row]) - x);
+                float o = Gm[t] * (rq[t] * xr[NTOK + t]);
+#pragma unroll
+                for (int j = 0; j <= t; ++j) o = fmaf(Et[t][j] * dots[j * 8 + NTOK + t] * rk[j] * rq[t], delta[j], o);
+                if (t == tq) out[(((size_t)n * NTOK + t) * hv + h) * kD + row] = from_f32<__nv_bfloat16>(o);
             }
-            // ---- products among the vectors (rows gq, columns 2t, 2t+1 of V V^T), for the norms
-            //      and the key-key / key-query coefficients, and X = S V^T
-            //      (four accumulators per product, so that the MMAs of one chain are 4-8 long)
-            float d[4] = {0.f, 0.f, 0.f, 0.f};
-            {
-                float dv[4][4], dx[4][4];
 #pragma unroll
-                for (int c = 0; c < 4; ++c)
+            for (int j = 0; j < NTOK; ++j)
+                if (j == tq) (rr ? wb : wa) = Et[NTOK - 1][j] * rk[j] * delta[j];
+        }
+        const uint32_t wa_hi = tf32_hi(wa), wb_hi = tf32_hi(wb);
+        const uint32_t wa_lo = __float_as_uint(wa - __uint_as_float(wa_hi));
+        const uint32_t wb_lo = __float_as_uint(wb - __uint_as_float(wb_hi));
+        float* dstA = state + ((size_t)sidx * hv + h) * kD * kD + rowA * kD + 2 * tq;
+        float* dstB = dstA + kD;
 #pragma unroll
-                    for (int e = 0; e < 4; ++e) dv[c][e] = dx[c][e] = 0.f;
-#pragma unroll
-                for (int p = 0; p < 16; ++p) {
-                    mma_tf32(dv[p & 3], vb0[p], 0u, vb1[p], 0u, vb0[p], vb1[p]);
-                    // ---- X = S V^T: rows rowA (d[0], d[1]) and rowB (d[2], d[3]), vectors 2t, 2t + 1
-                    const uint32_t a0 = tf32_hi(sa[p].x), a1 = tf32_hi(sb[p].x);
-                    const uint32_t a2 = tf32_hi(sa[p].y), a3 = tf32_hi(sb[p].y);
-                    mma_tf32(dx[p & 3], a0, a1, a2, a3, vb0[p], vb1[p]);
-                    mma_tf32(dx[p & 3], __float_as_uint(sa[p].x - __uint_as_float(a0)),
-                             __float_as_uint(sb[p].x - __uint_as_float(a1)), __float_as_uint(sa[p].y - __uint_as_float(a2)),
-                             __float_as_uint(sb[p].y - __uint_as_float(a3)), vb0[p], vb1[p]);
-                }
-#pragma unroll
-                for (int e = 0; e < 4; ++e) d[e] = (dx[0][e] + dx[1][e]) + (dx[2][e] + dx[3][e]);
-                dots[gq * 8 + 2 * tq] = (dv[0][0] + dv[1][0]) + (dv[2][0] + dv[3][0]);
-                dots[gq * 8 + 2 * tq + 1] = (dv[0][1] + dv[1][1]) + (dv[2][1] + dv[3][1]);
-            }
-            __syncwarp();  // dots
-            // ---- gates and the coefficients every row shares
-            float bt[NTOK], Gm[NTOK], rk[NTOK], rq[NTOK], Et[NTOK][NTOK];
-            {
-                const float* gs = reinterpret_cast<const float*>(sl + Lay::kGate);
-                const float ga = gs[2 * NTOK], gb = gs[2 * NTOK + 1];
-                float G[NTOK], acc = 0.f;
-#pragma unroll
-                for (int t = 0; t < NTOK; ++t) {
-                    const float graw = gs[t];
-                    const float braw = gs[NTOK + t];
-                    acc += act.a ? act_g(graw, ga, gb) : graw;
-                    G[t] = acc;
-                    bt[t] = act.a ? act_beta(braw) : braw;
-                    Gm[t] = expf(G[t]);
-                    rk[t] = rsqrtf(dots[t * 8 + t] + kNormEps);
-                    rq[t] = rsqrtf(dots[(NTOK + t) * 8 + NTOK + t] + kNormEps) * kInvSqrtD;
-                }
-#pragma unroll
-                for (int t = 0; t < NTOK; ++t)
-#pragma unroll
-                    for (int j = 0; j <= t; ++j) Et[t][j] = (j == t) ? 1.f : expf(G[t] - G[j]);
-            }
-            // ---- the 8 raw products of rows rowA and rowB, gathered from the 4 threads of the group
-            float xa[8], xb[8];
-#pragma unroll
-            for (int src = 0; src < 4; ++src) {
-                const int from = (lane & ~3) | src;
-                xa[2 * src] = __shfl_sync(0xffffffffu, d[0], from);
-                xa[2 * src + 1] = __shfl_sync(0xffffffffu, d[1], from);
-                xb[2 * src] = __shfl_sync(0xffffffffu, d[2], from);
-                xb[2 * src + 1] = __shfl_sync(0xffffffffu, d[3], from);
-            }
-            // ---- the recurrence of the m tokens for both rows; thread t writes o_t
-            const __nv_bfloat16* vrow = reinterpret_cast<const __nv_bfloat16*>(vec + 2 * NTOK * kVecStride);
-            float wa = 0.f, wb = 0.f;  // Et[m-1][t] delta_t / |k_t| of rows rowA, rowB for t = tq
-#pragma unroll
-            for (int rr = 0; rr < 2; ++rr) {
-                const float* xr = rr ? xb : xa;
-                const int row = rr ? rowB : rowA;
-                float delta[NTOK];
-#pragma unroll
-                for (int t = 0; t < NTOK; ++t) {
-                    float x = Gm[t] * (rk[t] * xr[t]);
-#pragma unroll
-                    for (int j = 0; j < t; ++j) x = fmaf(Et[t][j] * dots[j * 8 + t] * rk[j] * rk[t], delta[j], x);
-                    delta[t] = bt[t] * (to_f32(vrow[t * (kVecStride / 2) + row]) - x);
-                    float o = Gm[t] * (rq[t] * xr[NTOK + t]);
-#pragma unroll
-                    for (int j = 0; j <= t; ++j)
-                        o = fmaf(Et[t][j] * dots[j * 8 + NTOK + t] * rk[j] * rq[t], delta[j], o);
-                    if (t == tq) out[(((size_t)n * NTOK + t) * hv + h) * kD + row] = from_f32<__nv_bfloat16>(o);
-                }
-#pragma unroll
-                for (int j = 0; j < NTOK; ++j)
-                    if (j == tq) (rr ? wb : wa) = Et[NTOK - 1][j] * rk[j] * delta[j];
-            }
-            // ---- S <- Gam_m S + W K: A = [W_hi | W_lo] (slots t, t + 4 = key t), B = key t at
-            //      columns 8p + gq (twice), C = Gam_m S
-            const uint32_t wa_hi = tf32_hi(wa), wb_hi = tf32_hi(wb);
-            const uint32_t wa_lo = __float_as_uint(wa - __uint_as_float(wa_hi));
-            const uint32_t wb_lo = __float_as_uint(wb - __uint_as_float(wb_hi));
-            const float gl = Gm[NTOK - 1];
-            float* dstA = state + ((size_t)sidx * hv + h) * kD * kD + rowA * kD + 2 * tq;
-            float* dstB = dstA + kD;
-#pragma unroll
-            for (int p = 0; p < 16; ++p) {
-                float y[4] = {gl * sa[p].x, gl * sa[p].y, gl * sb[p].x, gl * sb[p].y};
-                const uint32_t kbits = __float_as_uint(kb[p]);
-                mma_tf32(y, wa_hi, wb_hi, wa_lo, wb_lo, kbits, kbits);
-                __stcs(reinterpret_cast<float2*>(dstA + 8 * p), make_float2(y[0], y[1]));
-                __stcs(reinterpret_cast<float2*>(dstB + 8 * p), make_float2(y[2], y[3]));
-            }
+        for (int p = 0; p < 16; ++p) {
+            const float2 sa = frag(p, rowA), sb = frag(p, rowB);
+            float y[4] = {gl * sa.x, gl * sa.y, gl * sb.x, gl * sb.y};
+            const uint32_t kbits = __float_as_uint(kb[p]);
+            mma_tf32(y, wa_hi, wb_hi, wa_lo, wb_lo, kbits, kbits);
+            __stcs(reinterpret_cast<float2*>(dstA + 8 * p), make_float2(y[0], y[1]));
+            __stcs(reinterpret_cast<float2*>(dstB + 8 * p), make_float2(y[2], y[3]));
         }
     }
-    // Drain: after giving up, the next item's copies may still be in flight.
-    if (tid == 0 && *abort_flag) {
-        const int nxt = i + 1;
-        if (first + nxt * stride < items) mbar_wait(&full[nxt % 3], (nxt / 3) & 1);
-    }
-    cp_async_wait<0>();
 }
 
 using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
@@ -611,18 +546,20 @@ cudaError_t launch_mma(const __nv_bfloat16* q, const __nv_bfloat16* k, const __n
                        const float* beta, float* state, StateSlots map, __nv_bfloat16* out, int num_seqs, int hk,
                        int hv, GateAct act, cudaStream_t stream) {
     using Lay = MmaLayout<NTOK>;
-    static_assert(Lay::kSmem <= 227 * 1024, "shared memory");
-    // The states as a 2-D fp32 tensor [slots * HV * 128 rows][128], boxes of 128 rows x 32
+    static_assert(3 * (Lay::kSmem + 1024) <= 228 * 1024, "three CTAs per SM");
+    // The states as a 2-D fp32 tensor [slots * HV * 128 rows][128], boxes of 64 rows x 32
     // columns (128 bytes, the swizzle width).
     const long long slots = map.slots ? map.num_slots : num_seqs;
     if (slots <= 0) return cudaSuccess;  // no sequence has a state: nothing to do
     if (slots * hv * kD > INT32_MAX) return cudaErrorInvalidValue;  // row numbers are 32-bit
+    const long long items = (long long)num_seqs * hv;
+    if (items > INT32_MAX) return cudaErrorInvalidValue;
     EncodeTiledFn fn = encode_fn();
     if (!fn) return cudaErrorNotSupported;
     CUtensorMap tm;
     const cuuint64_t dims[2] = {(cuuint64_t)kD, (cuuint64_t)(slots * hv * kD)};
     const cuuint64_t strides[1] = {(cuuint64_t)kD * 4};
-    const cuuint32_t box[2] = {32, (cuuint32_t)kD};
+    const cuuint32_t box[2] = {32, (cuuint32_t)kHalfRows};
     const cuuint32_t estr[2] = {1, 1};
     if (fn(&tm, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 2, state, dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
            CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) !=
@@ -631,12 +568,8 @@ cudaError_t launch_mma(const __nv_bfloat16* q, const __nv_bfloat16* k, const __n
     auto kernel = decode_mma_kernel<NTOK>;
     cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, Lay::kSmem);
     if (e != cudaSuccess) return e;
-    int dev = 0, sms = 0;
-    if ((e = cudaGetDevice(&dev)) != cudaSuccess) return e;
-    if ((e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev)) != cudaSuccess) return e;
-    const long long items = (long long)num_seqs * hv;
-    kernel<<<dim3((unsigned)(items < sms ? items : sms)), dim3(kMmaWarps * 32), Lay::kSmem, stream>>>(
-        tm, q, k, v, g, beta, state, map, out, num_seqs, hk, hv, act);
+    kernel<<<dim3((unsigned)items), dim3(kCtaWarps * 32), Lay::kSmem, stream>>>(tm, q, k, v, g, beta, state, map,
+                                                                                out, hk, hv, act);
     return cudaGetLastError();
 }
 
