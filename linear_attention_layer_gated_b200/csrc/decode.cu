@@ -331,20 +331,6 @@ struct MmaLayout {
     static constexpr int kSmem = kBar + 16 + 1024;                      // + alignment of the base
 };
 
-__device__ __forceinline__ uint32_t tf32_hi(float x) {
-    uint32_t r;
-    asm("cvt.rna.tf32.f32 %0, %1;" : "=r"(r) : "f"(x));
-    return r;
-}
-// d += a b, m16n8k8, tf32 inputs, fp32 accumulators.
-__device__ __forceinline__ void mma_tf32(float* d, uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3,
-                                         uint32_t b0, uint32_t b1) {
-    asm volatile("mma.sync.aligned.m16n8k8.row.col.f32.tf32.tf32.f32 {%0, %1, %2, %3}, {%4, %5, %6, %7}, "
-                 "{%8, %9}, {%0, %1, %2, %3};"
-                 : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
-                 : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
-}
-
 template <int NTOK>
 __global__ void __launch_bounds__(kCtaWarps * 32, 3)
 decode_mma_kernel(const __grid_constant__ CUtensorMap tm_state, const __nv_bfloat16* __restrict__ q,

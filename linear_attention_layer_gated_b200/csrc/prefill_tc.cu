@@ -30,7 +30,8 @@
 //  K1 chunk_prep_kernel   one CTA (256 threads) per (chunk, pair of V heads sharing a QK head),
 //                         all chunks in parallel: q and k tiles by TMA; the Gram [Q;K][Q;K]^T
 //                         (tcgen05), whose diagonal gives the norms; decay masks A and P; the
-//                         rows of T and of P T by substitution in fp32; then per V head the
+//                         rows of T by substitution in fp32 and P T from warp tf32 MMAs with
+//                         both factors split high / low; then per V head the
 //                         coefficient rows are written to Tensor Memory and W and
 //                         diag(gam r_q) Q - (P T diag(b gam r_k)) K come out of one tcgen05
 //                         product with K; -W, Qt, the split [T diag(b); At] images, Kt in fp32
@@ -423,56 +424,175 @@ __device__ bool prep_item(const PrepArgs& a, int cid, int pair, unsigned char* s
     tc_fence_before();
     hbar(bid, 256);
 
-    // ---- 4. T = (I + A)^-1 and P T per head, one row per thread: a row x of either satisfies
-    //         x (I + A) = rhs, with rhs = e_r for row r of T and rhs = P_r for row r of P T, and A
-    //         strictly lower triangular, so x_j = rhs_j - sum_{i > j} x_i A_ij.  Taking i from the
-    //         top down, x_i is final when reached and its terms go to every lower x_j at once
-    //         (row i of A, read by all threads of the head as broadcasts).  Both right-hand sides
-    //         vanish past column r, so x does too: a warp starts at its last row.
+    // ---- 4. T = (I + A)^-1 per head in 32 x 32 blocks.  With A11, A22 the diagonal blocks and
+    //         A21 the lower-left one (A strictly lower triangular),
+    //           T11 = (I + A11)^-1,  T22 = (I + A22)^-1,  T21 = -T22 A21 T11,  T12 = 0.
+    //  (a) T11 and T22 one row per thread (warps 0-3): row r of a diagonal block satisfies
+    //      x (I + Abb) = e_r, so x_j = [j == r] - sum_{i > j} x_i A_ij within the block.  Taking i
+    //      from the top down, x_i is final when reached and its terms go to every lower x_j at
+    //      once (row i of A, read by all threads of the head as broadcasts); every chain is at
+    //      most 31 steps long.
     {
-        // Rows 32..63 take about four times the work of rows 0..31; warp w runs on scheduler w % 4,
-        // so the second head takes its row halves the other way round and every scheduler gets
-        // one long and one short warp of each CTA.
-        const int hh = tid >> 7, l = tid & 127, rr = (l & 63) ^ (32 * hh);
-        const bool trow = l < 64;
-        const float* A = AT + hh * kMat;
-        float2 x[kChunk / 2];  // x_{2m}, x_{2m+1}
-        if (trow) {
+        if (tid < 128) {
+            const int hh = warp >> 1, c0 = 32 * (warp & 1);  // head, first row / column of the block
+            const int rr = c0 + lane;
+            const float* A = AT + hh * kMat + c0;
+            float2 x[16];  // x_{c0 + 2m}, x_{c0 + 2m + 1}
 #pragma unroll
-            for (int m = 0; m < kChunk / 2; ++m) x[m] = make_float2(2 * m == rr ? 1.f : 0.f, 2 * m + 1 == rr ? 1.f : 0.f);
-        } else {
-            const float4* pr = reinterpret_cast<const float4*>(PP + hh * kMat + rr * kLdA);
+            for (int m = 0; m < 16; ++m) x[m] = make_float2(2 * m == lane ? 1.f : 0.f, 2 * m + 1 == lane ? 1.f : 0.f);
 #pragma unroll
-            for (int m = 0; m < kChunk / 4; ++m) {
-                const float4 v = pr[m];
-                x[2 * m] = make_float2(v.x, v.y);
-                x[2 * m + 1] = make_float2(v.z, v.w);
-            }
-        }
-        const int imax = (rr | 31);  // the warp's last row (warp-uniform)
-#pragma unroll
-        for (int i = kChunk - 1; i >= 1; --i) {
-            if (i <= imax) {
+            for (int i = 31; i >= 1; --i) {  // block-local row i
                 const float xi = (i & 1) ? x[i >> 1].y : x[i >> 1].x;
                 const float2 nx = make_float2(-xi, -xi);
-                const float4* ar = reinterpret_cast<const float4*>(A + i * kLdA);
-                // highest columns first: x_{i-1} is final soonest, so the next step can start while
-                // this one's other terms are still in flight
+                const float4* ar = reinterpret_cast<const float4*>(A + (c0 + i) * kLdA);
+                // highest columns first: x_{i-1} is final soonest, so the next step can start
+                // while this one's other terms are still in flight
 #pragma unroll
                 for (int m = (i - 1) / 4; m >= 0; --m) {
-                    const float4 a = ar[m];
+                    const float4 av = ar[m];
                     // pairs (4m, 4m+1) and (4m+2, 4m+3); only columns below i take the term
-                    if (4 * m + 3 < i) x[2 * m + 1] = __ffma2_rn(nx, make_float2(a.z, a.w), x[2 * m + 1]);
-                    else if (4 * m + 2 < i) x[2 * m + 1].x = fmaf(-xi, a.z, x[2 * m + 1].x);
-                    if (4 * m + 1 < i) x[2 * m] = __ffma2_rn(nx, make_float2(a.x, a.y), x[2 * m]);
-                    else x[2 * m].x = fmaf(-xi, a.x, x[2 * m].x);
+                    if (4 * m + 3 < i) x[2 * m + 1] = __ffma2_rn(nx, make_float2(av.z, av.w), x[2 * m + 1]);
+                    else if (4 * m + 2 < i) x[2 * m + 1].x = fmaf(-xi, av.z, x[2 * m + 1].x);
+                    if (4 * m + 1 < i) x[2 * m] = __ffma2_rn(nx, make_float2(av.x, av.y), x[2 * m]);
+                    else x[2 * m].x = fmaf(-xi, av.x, x[2 * m].x);
+                }
+            }
+            hbar(bid, 256);  // every thread is done reading A11 and A22
+            // the block's row, columns c0 .. c0 + 31; A21 (rows 32.., columns 0..31) stays
+            float4* dst = reinterpret_cast<float4*>(AT + hh * kMat + rr * kLdA + c0);
+#pragma unroll
+            for (int m = 0; m < 8; ++m) dst[m] = make_float4(x[2 * m].x, x[2 * m].y, x[2 * m + 1].x, x[2 * m + 1].y);
+        } else {
+            hbar(bid, 256);
+        }
+    }
+    hbar(bid, 256);  // T11 and T22 are complete
+
+    // The products below run on the warp tensor cores (m16n8k8, tf32).  Each fp32 factor goes in
+    // as a tf32 high part and its remainder, and hi hi + hi lo + lo hi keep about 21 bits, more
+    // than the bf16 splits downstream take.  Matrices are the row-major fp32 blocks above (row
+    // stride kLdA); lane (gq, tq) = (lane / 4, lane % 4).
+    const int gq = lane >> 2, tq = lane & 3;
+    auto frag_a = [&](const float* M, int r0, int k0, uint32_t* hi, uint32_t* lo) {
+        const float* pr = M + (r0 + gq) * kLdA + k0 + tq;
+        const float v4[4] = {pr[0], pr[8 * kLdA], pr[4], pr[8 * kLdA + 4]};
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+            hi[e] = tf32_hi(v4[e]);
+            lo[e] = __float_as_uint(v4[e] - __uint_as_float(hi[e]));
+        }
+    };
+    auto mma3 = [&](float* d, const uint32_t* ah, const uint32_t* al, const float* M, int k0, int n0) {
+        const float* pr = M + (k0 + tq) * kLdA + n0 + gq;
+        const float b0 = pr[0], b1 = pr[4 * kLdA];
+        const uint32_t bh0 = tf32_hi(b0), bh1 = tf32_hi(b1);
+        const uint32_t bl0 = __float_as_uint(b0 - __uint_as_float(bh0));
+        const uint32_t bl1 = __float_as_uint(b1 - __uint_as_float(bh1));
+        mma_tf32(d, ah[0], ah[1], ah[2], ah[3], bl0, bl1);
+        mma_tf32(d, al[0], al[1], al[2], al[3], bh0, bh1);
+        mma_tf32(d, ah[0], ah[1], ah[2], ah[3], bh0, bh1);
+    };
+    //  (b) Y = T22 A21 (rows 32..63, columns 0..31; T22 is lower triangular, so row block rb sums
+    //      k over 32 .. 32 + 16 rb + 15) and then T21 = -Y T11 (T11 lower triangular: column tile
+    //      nt sums k over 8 nt .. 31).  Warp w: head w / 4, row block (w / 2) % 2, and column
+    //      tiles {0, 3} or {1, 2} of the four, which gives every warp the same number of steps
+    //      of the second product.
+    {
+        const int hh = warp >> 2, rb = (warp >> 1) & 1, nh = warp & 1;
+        const int ntA = nh ? 1 : 0, ntB = nh ? 2 : 3;
+        float* M = AT + hh * kMat;
+        float y[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
+#pragma unroll
+        for (int s = 0; s < 4; ++s) {
+            if (s <= 2 * rb + 1) {
+                uint32_t ah[4], al[4];
+                frag_a(M, 32 + 16 * rb, 32 + 8 * s, ah, al);
+                mma3(y[0], ah, al, M, 32 + 8 * s, 8 * ntA);
+                mma3(y[1], ah, al, M, 32 + 8 * s, 8 * ntB);
+            }
+        }
+        hbar(bid, 256);  // every warp is done reading A21
+        float* yr = M + (32 + 16 * rb + gq) * kLdA + 2 * tq;
+#pragma unroll
+        for (int j = 0; j < 2; ++j) {
+            const int nt = j ? ntB : ntA;
+            *reinterpret_cast<float2*>(yr + 8 * nt) = make_float2(y[j][0], y[j][1]);
+            *reinterpret_cast<float2*>(yr + 8 * kLdA + 8 * nt) = make_float2(y[j][2], y[j][3]);
+        }
+        hbar(bid, 256);  // Y is complete (in A21's place)
+        float t21[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
+#pragma unroll
+        for (int s = 0; s < 4; ++s) {
+            if (s >= ntA) {  // ntA <= ntB
+                uint32_t ah[4], al[4];
+                frag_a(M, 32 + 16 * rb, 8 * s, ah, al);
+                mma3(t21[0], ah, al, M, 8 * s, 8 * ntA);
+                if (s >= ntB) mma3(t21[1], ah, al, M, 8 * s, 8 * ntB);
+            }
+        }
+        hbar(bid, 256);  // every warp is done reading Y
+#pragma unroll
+        for (int j = 0; j < 2; ++j) {
+            const int nt = j ? ntB : ntA;
+            *reinterpret_cast<float2*>(yr + 8 * nt) = make_float2(-t21[j][0], -t21[j][1]);
+            *reinterpret_cast<float2*>(yr + 8 * kLdA + 8 * nt) = make_float2(-t21[j][2], -t21[j][3]);
+        }
+    }
+    hbar(bid, 256);  // T is complete
+
+    // ---- 5. P T = P (I + A)^-1 per head.  Both factors are lower triangular, so tile (row block
+    //         ab of 16, column tile nt of 8) sums k over 8 nt .. 16 ab + 15 only (2 ab + 2 - nt
+    //         steps of 8), and the tiles past the block diagonal stay as P left them (zero).  The
+    //         70 tile-steps of a head go to its 4 warps as runs of column tiles of one row block,
+    //         17 or 18 steps each (one A fragment serves all tiles of a run):
+    //           warp 0: (3, tiles 0-1), (0, 0-1)      warp 1: (3, 2-3), (1, 0-1)
+    //           warp 2: (3, 4-7), (1, 2-3), (2, 4-5)  warp 3: (2, 0-3)
+    {
+        const int hh = warp >> 2, q = warp & 3;
+        const float* Pm = PP + hh * kMat;
+        const float* Tm = AT + hh * kMat;
+        // runs (row block, first tile, last tile); a row block of -1 marks no run
+        int run[3][3];
+        switch (q) {
+            case 0: run[0][0] = 3; run[0][1] = 0; run[0][2] = 1; run[1][0] = 0; run[1][1] = 0; run[1][2] = 1; run[2][0] = -1; break;
+            case 1: run[0][0] = 3; run[0][1] = 2; run[0][2] = 3; run[1][0] = 1; run[1][1] = 0; run[1][2] = 1; run[2][0] = -1; break;
+            case 2: run[0][0] = 3; run[0][1] = 4; run[0][2] = 7; run[1][0] = 1; run[1][1] = 2; run[1][2] = 3; run[2][0] = 2; break;
+            default: run[0][0] = 2; run[0][1] = 0; run[0][2] = 3; run[1][0] = -1; run[2][0] = -1; break;
+        }
+        if (q == 2) { run[2][1] = 4; run[2][2] = 5; }
+        float d[8][4];
+#pragma unroll
+        for (int t = 0; t < 8; ++t) d[t][0] = d[t][1] = d[t][2] = d[t][3] = 0.f;
+#pragma unroll
+        for (int u = 0; u < 3; ++u) {
+            const int ab = run[u][0], n0 = run[u][1], n1 = run[u][2];
+            if (ab < 0) continue;  // warp-uniform
+#pragma unroll
+            for (int s = 0; s < 8; ++s) {
+                if (s >= n0 && s <= 2 * ab + 1) {
+                    uint32_t ah[4], al[4];
+                    frag_a(Pm, 16 * ab, 8 * s, ah, al);
+#pragma unroll
+                    for (int j = 0; j < (u == 0 ? 4 : 2); ++j)  // accumulator slots: run 0 -> 0..3, 1 -> 4..5, 2 -> 6..7
+                        if (n0 + j <= n1 && n0 + j <= s) mma3(d[2 * u + (u > 0 ? 2 : 0) + j], ah, al, Tm, 8 * s, 8 * (n0 + j));
                 }
             }
         }
-        hbar(bid, 256);  // every thread is done reading A and P
-        float4* dst = reinterpret_cast<float4*>((trow ? AT : PP) + hh * kMat + rr * kLdA);
+        hbar(bid, 256);  // every warp is done reading P
 #pragma unroll
-        for (int m = 0; m < kChunk / 4; ++m) dst[m] = make_float4(x[2 * m].x, x[2 * m].y, x[2 * m + 1].x, x[2 * m + 1].y);
+        for (int u = 0; u < 3; ++u) {
+            const int ab = run[u][0], n0 = run[u][1], n1 = run[u][2];
+            if (ab < 0) continue;
+            float* dst = PP + hh * kMat + (16 * ab + gq) * kLdA + 2 * tq;
+#pragma unroll
+            for (int j = 0; j < (u == 0 ? 4 : 2); ++j) {
+                if (n0 + j <= n1) {
+                    const float* dj = d[2 * u + (u > 0 ? 2 : 0) + j];
+                    *reinterpret_cast<float2*>(dst + 8 * (n0 + j)) = make_float2(dj[0], dj[1]);
+                    *reinterpret_cast<float2*>(dst + 8 * kLdA + 8 * (n0 + j)) = make_float2(dj[2], dj[3]);
+                }
+            }
+        }
     }
     if (tid < 128) {  // per-column factors of step 6, once
         const int hh = tid >> 6, i = tid & 63;
