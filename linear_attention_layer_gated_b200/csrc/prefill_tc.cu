@@ -482,15 +482,16 @@ __device__ bool prep_item(const PrepArgs& a, int cid, int pair, unsigned char* s
             lo[e] = __float_as_uint(v4[e] - __uint_as_float(hi[e]));
         }
     };
-    auto mma3 = [&](float* d, const uint32_t* ah, const uint32_t* al, const float* M, int k0, int n0) {
+    // d += hi hi, e += hi lo + lo hi: two accumulators halve the chain of dependent MMAs
+    auto mma3 = [&](float* d, float* e, const uint32_t* ah, const uint32_t* al, const float* M, int k0, int n0) {
         const float* pr = M + (k0 + tq) * kLdA + n0 + gq;
         const float b0 = pr[0], b1 = pr[4 * kLdA];
         const uint32_t bh0 = tf32_hi(b0), bh1 = tf32_hi(b1);
         const uint32_t bl0 = __float_as_uint(b0 - __uint_as_float(bh0));
         const uint32_t bl1 = __float_as_uint(b1 - __uint_as_float(bh1));
-        mma_tf32(d, ah[0], ah[1], ah[2], ah[3], bl0, bl1);
-        mma_tf32(d, al[0], al[1], al[2], al[3], bh0, bh1);
+        mma_tf32(e, ah[0], ah[1], ah[2], ah[3], bl0, bl1);
         mma_tf32(d, ah[0], ah[1], ah[2], ah[3], bh0, bh1);
+        mma_tf32(e, al[0], al[1], al[2], al[3], bh0, bh1);
     };
     //  (b) Y = T22 A21 (rows 32..63, columns 0..31; T22 is lower triangular, so row block rb sums
     //      k over 32 .. 32 + 16 rb + 15) and then T21 = -Y T11 (T11 lower triangular: column tile
@@ -502,13 +503,14 @@ __device__ bool prep_item(const PrepArgs& a, int cid, int pair, unsigned char* s
         const int ntA = nh ? 1 : 0, ntB = nh ? 2 : 3;
         float* M = AT + hh * kMat;
         float y[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
+        float ye[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
 #pragma unroll
         for (int s = 0; s < 4; ++s) {
             if (s <= 2 * rb + 1) {
                 uint32_t ah[4], al[4];
                 frag_a(M, 32 + 16 * rb, 32 + 8 * s, ah, al);
-                mma3(y[0], ah, al, M, 32 + 8 * s, 8 * ntA);
-                mma3(y[1], ah, al, M, 32 + 8 * s, 8 * ntB);
+                mma3(y[0], ye[0], ah, al, M, 32 + 8 * s, 8 * ntA);
+                mma3(y[1], ye[1], ah, al, M, 32 + 8 * s, 8 * ntB);
             }
         }
         hbar(bid, 256);  // every warp is done reading A21
@@ -516,26 +518,28 @@ __device__ bool prep_item(const PrepArgs& a, int cid, int pair, unsigned char* s
 #pragma unroll
         for (int j = 0; j < 2; ++j) {
             const int nt = j ? ntB : ntA;
-            *reinterpret_cast<float2*>(yr + 8 * nt) = make_float2(y[j][0], y[j][1]);
-            *reinterpret_cast<float2*>(yr + 8 * kLdA + 8 * nt) = make_float2(y[j][2], y[j][3]);
+            *reinterpret_cast<float2*>(yr + 8 * nt) = make_float2(y[j][0] + ye[j][0], y[j][1] + ye[j][1]);
+            *reinterpret_cast<float2*>(yr + 8 * kLdA + 8 * nt) = make_float2(y[j][2] + ye[j][2], y[j][3] + ye[j][3]);
         }
         hbar(bid, 256);  // Y is complete (in A21's place)
         float t21[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
+        float te[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
 #pragma unroll
         for (int s = 0; s < 4; ++s) {
             if (s >= ntA) {  // ntA <= ntB
                 uint32_t ah[4], al[4];
                 frag_a(M, 32 + 16 * rb, 8 * s, ah, al);
-                mma3(t21[0], ah, al, M, 8 * s, 8 * ntA);
-                if (s >= ntB) mma3(t21[1], ah, al, M, 8 * s, 8 * ntB);
+                mma3(t21[0], te[0], ah, al, M, 8 * s, 8 * ntA);
+                if (s >= ntB) mma3(t21[1], te[1], ah, al, M, 8 * s, 8 * ntB);
             }
         }
         hbar(bid, 256);  // every warp is done reading Y
 #pragma unroll
         for (int j = 0; j < 2; ++j) {
             const int nt = j ? ntB : ntA;
-            *reinterpret_cast<float2*>(yr + 8 * nt) = make_float2(-t21[j][0], -t21[j][1]);
-            *reinterpret_cast<float2*>(yr + 8 * kLdA + 8 * nt) = make_float2(-t21[j][2], -t21[j][3]);
+            *reinterpret_cast<float2*>(yr + 8 * nt) = make_float2(-(t21[j][0] + te[j][0]), -(t21[j][1] + te[j][1]));
+            *reinterpret_cast<float2*>(yr + 8 * kLdA + 8 * nt) =
+                make_float2(-(t21[j][2] + te[j][2]), -(t21[j][3] + te[j][3]));
         }
     }
     hbar(bid, 256);  // T is complete
@@ -560,9 +564,9 @@ __device__ bool prep_item(const PrepArgs& a, int cid, int pair, unsigned char* s
             default: run[0][0] = 2; run[0][1] = 0; run[0][2] = 3; run[1][0] = -1; run[2][0] = -1; break;
         }
         if (q == 2) { run[2][1] = 4; run[2][2] = 5; }
-        float d[8][4];
+        float d[8][4], e[8][4];
 #pragma unroll
-        for (int t = 0; t < 8; ++t) d[t][0] = d[t][1] = d[t][2] = d[t][3] = 0.f;
+        for (int t = 0; t < 8; ++t) d[t][0] = d[t][1] = d[t][2] = d[t][3] = e[t][0] = e[t][1] = e[t][2] = e[t][3] = 0.f;
 #pragma unroll
         for (int u = 0; u < 3; ++u) {
             const int ab = run[u][0], n0 = run[u][1], n1 = run[u][2];
@@ -574,7 +578,7 @@ __device__ bool prep_item(const PrepArgs& a, int cid, int pair, unsigned char* s
                     frag_a(Pm, 16 * ab, 8 * s, ah, al);
 #pragma unroll
                     for (int j = 0; j < (u == 0 ? 4 : 2); ++j)  // accumulator slots: run 0 -> 0..3, 1 -> 4..5, 2 -> 6..7
-                        if (n0 + j <= n1 && n0 + j <= s) mma3(d[2 * u + (u > 0 ? 2 : 0) + j], ah, al, Tm, 8 * s, 8 * (n0 + j));
+                        if (n0 + j <= n1 && n0 + j <= s) mma3(d[2 * u + (u > 0 ? 2 : 0) + j], e[2 * u + (u > 0 ? 2 : 0) + j], ah, al, Tm, 8 * s, 8 * (n0 + j));
                 }
             }
         }
@@ -588,8 +592,9 @@ __device__ bool prep_item(const PrepArgs& a, int cid, int pair, unsigned char* s
             for (int j = 0; j < (u == 0 ? 4 : 2); ++j) {
                 if (n0 + j <= n1) {
                     const float* dj = d[2 * u + (u > 0 ? 2 : 0) + j];
-                    *reinterpret_cast<float2*>(dst + 8 * (n0 + j)) = make_float2(dj[0], dj[1]);
-                    *reinterpret_cast<float2*>(dst + 8 * kLdA + 8 * (n0 + j)) = make_float2(dj[2], dj[3]);
+                    const float* ej = e[2 * u + (u > 0 ? 2 : 0) + j];
+                    *reinterpret_cast<float2*>(dst + 8 * (n0 + j)) = make_float2(dj[0] + ej[0], dj[1] + ej[1]);
+                    *reinterpret_cast<float2*>(dst + 8 * kLdA + 8 * (n0 + j)) = make_float2(dj[2] + ej[2], dj[3] + ej[3]);
                 }
             }
         }
