@@ -29,9 +29,10 @@
 //                         first chunk id and a (seq, start, length) entry per chunk.
 //  K1 chunk_prep_kernel   one CTA (256 threads) per (chunk, pair of V heads sharing a QK head),
 //                         all chunks in parallel: q and k tiles by TMA; the Gram [Q;K][Q;K]^T
-//                         (tcgen05), whose diagonal gives the norms; decay masks A and P; the
-//                         rows of T by substitution in fp32 and P T from warp tf32 MMAs with
-//                         both factors split high / low; then per V head the
+//                         (tcgen05), whose diagonal gives the norms; decay masks A and P;
+//                         T = (I + A)^-1 in 32 x 32 blocks (the diagonal blocks by row
+//                         substitution in fp32, T21 = -T22 A21 T11) and P T, the products on
+//                         warp tf32 MMAs with both factors split high / low; then per V head the
 //                         coefficient rows are written to Tensor Memory and W and
 //                         diag(gam r_q) Q - (P T diag(b gam r_k)) K come out of one tcgen05
 //                         product with K; -W, Qt, the split [T diag(b); At] images, Kt in fp32
